@@ -1,0 +1,165 @@
+"""Float64 CPU oracle for grouped-query attention (GQA) decode.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package.  The product
+path (the CUDA library and its Python binding) never imports it, and this
+package never imports the product: the two share nothing but the seeded input
+generators, which hold none of the method's arithmetic.
+
+The oracle itself is plain C (``gqa_oracle.c``): it expands the bf16 bit
+patterns of q, K and V exactly to double, gathers K/V through the page table
+by plain indexing and evaluates softmax(scale * q K^T) V row by row in double.
+This module compiles it with gcc (``build()``) and marshals numpy arrays into
+it (``gqa_decode()``).
+
+What it computes follows "Grouped-Query Attention" (aiwiki; the PyTorch
+module's repeat_interleave broadcast and scaled_dot_product_attention call) and
+"GQA and MQA: Mathematical Foundations, KV-Cache Bandwidth Reduction ..."
+(llms.blog; "Multi-Query Attention / Mathematical Formulation" and
+"Grouped-Query Attention / Mathematical Formulation").  The header of
+``gqa_oracle.c`` lists the readings taken where those pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+__all__ = ["build", "load_library", "gqa_decode", "max_threads", "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE"]
+
+STATUS_BAD_SEQLEN = 1
+STATUS_BAD_PAGE = 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gqa_oracle.c")
+_OUT_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_OUT_DIR, "libgqa_oracle.so")
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile ``gqa_oracle.c`` into a shared library with gcc (OpenMP on).
+
+    Strict IEEE arithmetic: no -ffast-math, no FMA contraction.  Returns the
+    path of the library.
+    """
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    tmp = out + ".tmp.%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fopenmp", "-fPIC",
+           "-shared", "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def load_library(path: str):
+    """Open a compiled oracle library and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    lib.oracle_gqa_decode.restype = ctypes.c_int
+    lib.oracle_gqa_decode.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+        ctypes.c_double, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+        ctypes.c_void_p, ctypes.c_int32,
+    ]
+    lib.oracle_max_threads.restype = ctypes.c_int
+    lib.oracle_max_threads.argtypes = []
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = load_library(build())
+    return _lib
+
+
+def max_threads() -> int:
+    """Threads an OpenMP region of the oracle uses by default."""
+    return int(_load().oracle_max_threads())
+
+
+def _as_bits(a) -> np.ndarray:
+    """bf16 data as a C-contiguous uint16 array of bit patterns.
+
+    Accepts a numpy uint16/int16 array or a torch bfloat16 tensor (CPU)."""
+    if hasattr(a, "dtype") and str(getattr(a, "dtype")) == "torch.bfloat16":
+        import torch  # local: only needed when torch tensors are passed
+
+        a = a.detach().to("cpu").contiguous().view(torch.int16).numpy()
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.int16:
+        a = a.view(np.uint16)
+    if a.dtype != np.uint16:
+        raise TypeError("expected bf16 bit patterns (uint16) or a bfloat16 tensor, got %s" % a.dtype)
+    return a
+
+
+def _as_i32(a) -> Optional[np.ndarray]:
+    if a is None:
+        return None
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").numpy()
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def gqa_decode(q, k_cache, v_cache, seqlens, page_table=None, *, num_kv_heads: int,
+               scale: Optional[float] = None, rows=None,
+               threads: int = 0, lib=None) -> Tuple[np.ndarray, int]:
+    """Reference GQA decode in float64.
+
+    q         bf16 [b, H, d]
+    k_cache   bf16 [num_pages, G, P, d] (paged) or [b, G, m, d] (contiguous)
+    v_cache   same shape as k_cache
+    seqlens   int32 [b]
+    page_table int32 [b, max_pages_per_seq], or None for the contiguous cache
+    scale     softmax scale; default 1/sqrt(d), the scaled_dot_product_attention default
+    rows      optional flat row ids s*H + i to compute (default: all b*H rows)
+    lib       a library from ``load_library`` (default: the built oracle)
+
+    Returns (out, status): out float64 [b, H, d] (or [len(rows), d]) and the OR of
+    the status bits (1: a length outside [1, capacity]; 2: a page id outside the pool).
+    """
+    qb = _as_bits(q)
+    kb = _as_bits(k_cache)
+    vb = _as_bits(v_cache)
+    if qb.ndim != 3 or kb.ndim != 4 or kb.shape != vb.shape:
+        raise ValueError("q must be [b,H,d] and k/v caches [pages,G,P,d] of equal shape")
+    b, H, d = qb.shape
+    num_pages, G, P, dk = kb.shape
+    if dk != d or G != num_kv_heads:
+        raise ValueError("cache shape %s does not match q %s / G=%d" % (kb.shape, qb.shape, num_kv_heads))
+    sl = _as_i32(seqlens)
+    pt = _as_i32(page_table)
+    if sl.shape != (b,):
+        raise ValueError("seqlens must have shape [b]")
+    max_pages = 0
+    if pt is not None:
+        if pt.ndim != 2 or pt.shape[0] != b:
+            raise ValueError("page_table must be [b, max_pages_per_seq]")
+        max_pages = pt.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    rows_arr = None
+    nrows = b * H
+    if rows is not None:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        nrows = rows_arr.shape[0]
+    out = np.zeros((nrows, d), dtype=np.float64)
+    status = np.zeros(1, dtype=np.int32)
+    rc = (lib or _load()).oracle_gqa_decode(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, sl.ctypes.data,
+        None if pt is None else pt.ctypes.data, b, H, G, d, P, num_pages, max_pages,
+        float(scale), None if rows_arr is None else rows_arr.ctypes.data, nrows,
+        out.ctypes.data, status.ctypes.data, int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    if rows is None:
+        out = out.reshape(b, H, d)
+    return out, int(status[0])
