@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark: GQA decode over a KV cache on B200.
+
+One step = one decode step of the whole path for one batch of sequences: the
+split-KV decode kernel (group mapping, page-table translation, K/V tile loads,
+q.k scores, online softmax, p.V) and the combine kernel that merges the splits
+and normalises.  The inputs are resident in HBM when the timed region starts.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama70b]
+    python bench.py --impl reference ...        # the float64 CPU oracle instead
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own shard
+of sequences of the same shape (weak scaling, no collective on the data path);
+the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_bandwidth_b200 import accounting  # noqa: E402
+from kv_cache_bandwidth_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "GQA decode µs/step and KV-cache HBM GB/s as % of B200 peak (1 GPU)"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+# --------------------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kv_cache_bandwidth_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the decode kernel from a committed ncu capture,
+    if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("kernel_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clocks and clock-event reasons during the timed region (NVML)."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, interval_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.interval = interval_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- oracle leg
+
+def oracle_time(inp, target_s: float = 15.0, max_seq=None):
+    """Time the float64 oracle (as it stands, all host cores) on a bounded
+    sample of whole sequences of the workload.  Returns (GB/s, seconds,
+    threads, description)."""
+    import numpy as np
+
+    import oracle
+
+    w = inp.workload
+    q = inp.q.cpu()
+    kc, vc = inp.k_cache.cpu(), inp.v_cache.cpu()
+    sl = inp.seqlens.cpu()
+    pt = None if inp.page_table is None else inp.page_table.cpu()
+    threads = oracle.max_threads()
+    lens = sl.tolist()
+
+    def run(n_seq):
+        rows = np.arange(n_seq * w.H, dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.gqa_decode(q, kc, vc, sl, pt, num_kv_heads=w.G, scale=w.scale, rows=rows)
+        return time.perf_counter() - t0
+
+    probe = run(1)
+    per_seq = max(probe, 1e-6)
+    n = max(1, min(w.b if max_seq is None else max_seq, int(target_s / per_seq)))
+    dt = run(n) if n > 1 else probe
+    kv = accounting.kv_bytes_per_step(w.G, w.d, lens[:n])
+    desc = "%d of %d sequences (all %d heads each) of the workload, %.3g GB of KV" % (n, w.b, w.H, kv / 1e9)
+    return kv / dt / 1e9, dt, threads, desc
+
+
+def reference_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, device="cpu")
+    kv_step = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
+    # every step a bounded sample: a whole-sequence slice sized so the run ends in minutes
+    budget = max(5.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_time(inp, target_s=min(budget, 5.0))
+    vals, times, desc, threads = [], [], "", 0
+    for _ in range(args.steps):
+        gbs, dt, threads, desc = oracle_time(inp, target_s=budget)
+        vals.append(gbs)
+        times.append(dt)
+    value = statistics.median(vals)
+    ms = kv_step / (value * 1e9) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, inp, None),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": "each step: " + desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU leg
+
+def config_dict(w, inp, split_tokens):
+    kv = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
+    return {
+        "workload": w.name, "b": w.b, "H": w.H, "G": w.G, "d": w.d, "m": w.m,
+        "layout": "paged P=%d" % w.page_size if w.paged else "contiguous [b,G,m,d]",
+        "split_tokens": split_tokens, "kv_bytes_per_step": kv, "seed": w.seed,
+        "l2": ("inputs %.0f MiB > 126 MB L2 (no flush)" % (kv / 2 ** 20)) if kv > 2 * L2_BYTES
+        else "L2 flushed between steps",
+    }
+
+
+def main_gpu(args):
+    from kv_cache_bandwidth_b200 import gqa
+
+    world, rank, local = dist_setup()
+    w = WORKLOADS[args.workload]
+    w = w.with_(seed=w.seed + 1000 * rank)  # each rank: its own shard of sequences
+    inp = make_inputs(w, device="cuda")
+    kv_step = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
+    max_seqlen = int(inp.seqlens.max())
+    dims = gqa.dims_for(inp.q, inp.k_cache, inp.page_table)
+    split = args.split_tokens if args.split_tokens >= 0 else (w.split_tokens or 0)
+    if split == 0:
+        split = gqa.gqa_plan_split_tokens(dims, max_seqlen)
+    ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, max_seqlen, split)
+    out = torch.empty(inp.q.shape, dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    flush = None
+    if kv_step <= 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def step():
+        if args.entry == "cluster":
+            gqa.gqa_decode(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, out=out,
+                           status=status)
+        else:
+            gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                                 split_tokens=split, max_seqlen=max_seqlen, workspace=ws, out=out,
+                                 status=status)
+
+    launches_per_step = 1 if args.entry == "cluster" else 2
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError("decode reported status %d" % int(status.item()))
+
+    # ---- timed region: K steps, inputs resident in HBM
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ms = []
+    with ClockSampler(local) as clocks:
+        if flush is None:
+            barrier(world)
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            for _ in range(args.steps):
+                step()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            total_ms = ev0.elapsed_time(ev1)
+        else:
+            # small workload: flush L2 before every step, time each step alone
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            barrier(world)
+            torch.cuda.synchronize()
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                step()
+                b.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            step_ms = [a.elapsed_time(b) for a, b in evs]
+            total_ms = sum(step_ms)
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    value = world * kv_step / (ms_per_step * 1e-3) / 1e9
+    hbm, hbm_kind = peaks()
+
+    # ---- dominant kernel alone (decode kernel), CUDA events on its stream
+    kern_ms = None
+    if args.entry == "split":
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(max(args.steps, 10))]
+        for a, b in evs:
+            if flush is not None:
+                flush.zero_()
+            a.record(stream)
+            gqa.gqa_split_partials(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                                   split_tokens=split, max_seqlen=max_seqlen, workspace=ws, status=status)
+            b.record(stream)
+        torch.cuda.synchronize()
+        kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    else:
+        kern_ms = ms_per_step
+    kern_ms = max_over_ranks(kern_ms, world)
+    achieved = kv_step / (kern_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": recorded_traffic(args.workload),
+                "kernel": "gqa_decode_kernel (split-KV partials)" if args.entry == "split"
+                else "gqa_decode_kernel (cluster)", "peak_kind": hbm_kind,
+                "kernel_us": kern_ms * 1e3, "algorithmic_bytes_per_launch": kv_step}
+
+    # ---- end to end through the public API with host buffers
+    e2e = e2e_leg(args, inp, split, max_seqlen, ws, kv_step, world)
+
+    # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, dt, threads, desc = oracle_time(inp)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": desc + "; %.1f s of CPU time" % dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_dict(w, inp, split if args.entry == "split" else None),
+            "frac_of_peak_hbm": value / world / hbm, "peak_hbm_gbs": hbm, "peak_kind": hbm_kind,
+            "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
+            "entry": "gqa_decode_split" if args.entry == "split" else "gqa_decode",
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_leg(args, inp, split, max_seqlen, ws, kv_step, world):
+    """Same metric through the public call with host buffers: each step copies the
+    step's inputs (q, lengths, page table) from pinned host memory, runs the
+    decode and reads the result back.  The KV cache is the decode state and
+    stays resident in HBM."""
+    from kv_cache_bandwidth_b200 import gqa
+
+    h_q = inp.q.cpu().pin_memory()
+    h_sl = inp.seqlens.cpu().pin_memory()
+    h_pt = None if inp.page_table is None else inp.page_table.cpu().pin_memory()
+    h_out = torch.empty(inp.q.shape, dtype=torch.float32).pin_memory()
+    d_q = torch.empty_like(inp.q)
+    d_sl = torch.empty_like(inp.seqlens)
+    d_pt = None if h_pt is None else torch.empty_like(inp.page_table)
+    d_out = torch.empty(inp.q.shape, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    h2d = h_q.numel() * h_q.element_size() + h_sl.numel() * 4 + (0 if h_pt is None else h_pt.numel() * 4)
+    d2h = h_out.numel() * 4
+
+    def step():
+        d_q.copy_(h_q, non_blocking=True)
+        d_sl.copy_(h_sl, non_blocking=True)
+        if d_pt is not None:
+            d_pt.copy_(h_pt, non_blocking=True)
+        if args.entry == "cluster":
+            gqa.gqa_decode(d_q, inp.k_cache, inp.v_cache, d_sl, d_pt, out=d_out)
+        else:
+            gqa.gqa_decode_split(d_q, inp.k_cache, inp.v_cache, d_sl, d_pt, split_tokens=split,
+                                 max_seqlen=max_seqlen, workspace=ws, out=d_out)
+        h_out.copy_(d_out, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = max(10, min(args.steps, 200))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(n):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / n, world)
+    return {"value": world * kv_step / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "note": "q, lengths and page table H2D from pinned memory, output D2H; KV cache resident"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description="GQA decode benchmark (B200)")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama70b")
+    ap.add_argument("--entry", choices=["split", "cluster"], default="split")
+    ap.add_argument("--split-tokens", type=int, default=-1,
+                    help="-1: the workload's own split (or the library's plan); 0: the library's plan")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return reference_arm(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (use --impl reference for the CPU oracle)")
+    return main_gpu(args)
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())

@@ -1,0 +1,193 @@
+/*
+ * gqa.h -- C ABI of libgqa: grouped-query attention (GQA) decode over a
+ * contiguous or paged bf16 KV cache, written for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For every sequence s (one new query token each) and every
+ * query head i of H, with r = H / G query heads per KV group and
+ * g(i) = i / r:
+ *
+ *     out[s, i, :] = softmax_j( scale * q[s, i, :] . K[s, g(i), j, :] ) V[s, g(i), j, :]
+ *
+ * over the cached positions j < seqlens[s].  This is the attention of the
+ * PyTorch module in "Grouped-Query Attention" (aiwiki), where keys and values
+ * are broadcast to the query heads of their group with repeat_interleave(h // g,
+ * dim=1) and fed to scaled_dot_product_attention; the same page's closing note
+ * says the version that matters computes the KV-head index from the query-head
+ * index inside the kernel and reads the cache once.  For G = 1 it is the
+ * incremental multi-query attention of "GQA and MQA: Mathematical Foundations,
+ * KV-Cache Bandwidth Reduction ..." (llms.blog, "Multi-Query Attention /
+ * Mathematical Formulation": logits, softmax(logits + mask), weights . V); its
+ * "Grouped-Query Attention / Mathematical Formulation" gives the [b, G, m, d_k]
+ * cache.  The kernels read each KV group's keys and values from HBM once per
+ * decode step and share them among the group's r query heads on chip; nothing
+ * is expanded with repeat_interleave.
+ *
+ * Readings where the pages are silent: decode attends every cached position
+ * j < seqlens[s] (the new token's K/V is already in the cache); there is no
+ * causal mask beyond the length.  Paged pools follow the block-managed cache of
+ * the llms.blog page's "PagedAttention" section with the layout below.
+ *
+ * Layouts (all row-major, all device memory owned by the caller):
+ *   q          bf16  [b, H, d]
+ *   k_cache    bf16  paged: [num_pages, G, page_size, d]   (pool of pages)
+ *                    contiguous (page_table == NULL): [b, G, m, d] with
+ *                    m = dims->page_size (the capacity of every sequence)
+ *   v_cache    bf16  same layout as k_cache
+ *   seqlens    int32 [b]  cached tokens of each sequence, 1 <= len <= capacity
+ *   page_table int32 [b, max_pages_per_seq]: logical page t / page_size of
+ *              sequence s is pool page page_table[s * max_pages_per_seq + t / page_size];
+ *              entries past a sequence's length are never read (may be -1)
+ *   out        fp32  [b, H, d]  fully overwritten
+ *   status     uint32 (device), optional (may be NULL): the kernels OR
+ *              GQA_STATUS_* bits into it; the caller zeroes it
+ *
+ * Capacity: contiguous m = page_size; paged max_pages_per_seq * page_size.
+ *
+ * Errors.  Every argument check happens on the host before anything is
+ * launched; a failing call returns a negative GQA_ERR_* code and launches
+ * nothing.  Data-dependent problems found on the device (a length outside
+ * [1, capacity], a page id outside [0, num_pages)) never fault: the affected
+ * output rows are written as zeros and the matching GQA_STATUS_* bit is ORed
+ * into *status.  Page ids of the table are only turned into TMA coordinates,
+ * which the copy engine bounds-checks (an id outside the pool reads zeros and
+ * is flagged), so a corrupt table cannot make the kernel read outside the pool.
+ *
+ * Concurrency.  Calls are asynchronous on `stream` (a cudaStream_t passed as
+ * void*; NULL = the legacy default stream).  The library allocates no device
+ * memory and keeps no state between calls apart from per-device attribute
+ * caches; calls on different streams are independent if their output and
+ * workspace buffers are.
+ */
+#ifndef GQA_H
+#define GQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes of the host entry points. */
+#define GQA_OK 0
+#define GQA_ERR_NULL_POINTER (-1)  /* a required pointer is NULL */
+#define GQA_ERR_MISALIGNED (-2)    /* q/k/v/out/workspace not 16-byte aligned */
+#define GQA_ERR_HEADS (-3)         /* H % G != 0, or H/G above GQA_MAX_GROUP_RATIO */
+#define GQA_ERR_HEAD_DIM (-4)      /* head_dim not in {64, 128} */
+#define GQA_ERR_PAGE_SIZE (-5)     /* paged: page_size not a power of two in [8, 2^20] */
+#define GQA_ERR_DIMS (-6)          /* a size is < 1 or too large */
+#define GQA_ERR_SPLIT (-7)         /* split_tokens not a positive multiple of 128 */
+#define GQA_ERR_WORKSPACE (-8)     /* workspace NULL or smaller than required */
+#define GQA_ERR_CUDA (-9)          /* a CUDA runtime/driver call failed */
+#define GQA_ERR_DEVICE (-10)       /* current device is not sm_100 (B200) */
+
+/* Bits the kernels OR into *status. */
+#define GQA_STATUS_BAD_SEQLEN 1u   /* a length outside [1, capacity]: row zeroed */
+#define GQA_STATUS_BAD_PAGE 2u     /* a page id outside [0, num_pages): row zeroed */
+#define GQA_STATUS_TIMEOUT 4u      /* an on-chip pipeline wait gave up: output undefined */
+
+/* Largest supported group ratio r = H / G. */
+#define GQA_MAX_GROUP_RATIO 64
+
+/* gqa_dims.flags: choice of the q.k / p.v contraction (default: automatic). */
+#define GQA_FLAG_CONTRACT_MMA 1u   /* tensor cores (mma.sync m16n8k16 bf16) */
+#define GQA_FLAG_CONTRACT_FMA 2u   /* fp32 FMA on CUDA cores */
+
+typedef struct gqa_dims {
+    int32_t batch;             /* b: sequences, one query token each */
+    int32_t num_heads;         /* H: query heads */
+    int32_t num_kv_heads;      /* G: KV groups (heads of the cache) */
+    int32_t head_dim;          /* d = d_k = d_v: 64 or 128 */
+    int32_t page_size;         /* paged: tokens per page; contiguous: capacity m */
+    int32_t num_pages;         /* paged: pages in each pool; contiguous: ignored (= b) */
+    int32_t max_pages_per_seq; /* paged: row stride of page_table; contiguous: ignored */
+    uint32_t flags;            /* GQA_FLAG_*; 0 = automatic */
+} gqa_dims;
+
+/*
+ * gqa_decode -- one decode step without a workspace.
+ *
+ * Computes `out` as described above.  Each (sequence, KV group) is handled by
+ * one thread-block cluster whose blocks split the group's tokens and merge
+ * their partial softmax states through distributed shared memory, so no
+ * global scratch is needed.
+ *
+ * scale: the softmax scale (1/sqrt(d) is scaled_dot_product_attention's default).
+ * Returns GQA_OK or a GQA_ERR_* code (nothing launched on error).
+ */
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *seqlens, const int32_t *page_table, float *out,
+               const gqa_dims *dims, float scale, uint32_t *status, void *stream);
+
+/*
+ * Split-KV decode.  The tokens of every sequence are cut into consecutive
+ * splits of `split_tokens`; one thread block per (split, group, sequence)
+ * writes an unnormalised partial softmax state, and a second kernel merges the
+ * splits of each (sequence, head) exactly: with m_k the split's running
+ * maximum and l_k its sum of exponentials,
+ *     M = max_k m_k,  L = sum_k l_k 2^(m_k - M),  out = sum_k o_k 2^(m_k - M) / L.
+ * The merge is an exact re-association of the softmax of the pages' formula
+ * (the pages do not describe split-KV; it is how a long cache fills the GPU).
+ *
+ * split_tokens: a positive multiple of 128, or 0 to let the library choose
+ *               (gqa_plan_split_tokens).
+ * max_seqlen:   an upper bound of every seqlens[s] (sizes the grid and the
+ *               workspace); a length above it is treated as invalid
+ *               (GQA_STATUS_BAD_SEQLEN, row zeroed).
+ * workspace:    device memory of at least gqa_decode_split_workspace_size()
+ *               bytes, 16-byte aligned; its contents need no initialisation
+ *               and are scratch after the call.
+ */
+size_t gqa_decode_split_workspace_size(const gqa_dims *dims, int32_t max_seqlen,
+                                       int32_t split_tokens);
+
+int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *seqlens, const int32_t *page_table, float *out,
+                     const gqa_dims *dims, float scale, uint32_t *status,
+                     int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
+/*
+ * The two kernels of gqa_decode_split as separate calls (same arguments and
+ * workspace): gqa_split_partials writes the per-split partial states into the
+ * workspace; gqa_split_combine merges them into `out`.  Running the first and
+ * then the second on one stream is exactly gqa_decode_split.  The combine is
+ * also the merge step for partial states produced elsewhere (e.g. gathered
+ * from other GPUs into this workspace).
+ *
+ * Workspace layout (fp32, each array 256-byte aligned, S = ceil(max_seqlen /
+ * split_tokens)): o [b, H, S, d] unnormalised sum_j 2^(x_j - m) v_j;
+ * m [b, H, S] running maximum of x_j = scale * log2(e) * q.k_j;
+ * l [b, H, S] sum_j 2^(x_j - m), or -1 when the split met an invalid page id.
+ * Split k of sequence s covers tokens [k * split_tokens, min(len, (k+1) * split_tokens));
+ * the combine reads the splits k < ceil(len / split_tokens).
+ */
+int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *seqlens, const int32_t *page_table,
+                       const gqa_dims *dims, float scale, uint32_t *status,
+                       int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims,
+                      uint32_t *status, int32_t split_tokens, int32_t max_seqlen,
+                      const void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The split length gqa_decode_split uses when split_tokens == 0: enough
+ * (split, group, sequence) blocks to keep every SM busy, in multiples of 128
+ * tokens.  num_sms <= 0 queries the current device.  Returns a positive
+ * multiple of 128, or a GQA_ERR_* code.
+ */
+int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms);
+
+/* A static, human-readable name for a GQA_OK / GQA_ERR_* code. */
+const char *gqa_status_string(int code);
+
+/* ABI version of this header: (major << 16) | minor. */
+int32_t gqa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_H */

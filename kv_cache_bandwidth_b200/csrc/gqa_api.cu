@@ -1,0 +1,492 @@
+// gqa_api.cu -- the C ABI of libgqa (declared in include/gqa.h).
+//
+// Host side only: argument validation (before anything touches the GPU),
+// TMA descriptor encoding for the K and V pools, the split / cluster plan and
+// the kernel launches on the caller's stream.  No device memory is allocated
+// here; the only state kept between calls is per-device attribute caches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gqa.h"
+#include "gqa_kernels.cuh"
+
+namespace {
+
+using gqa::DecodeParams;
+using gqa::CombineParams;
+using gqa::Mode;
+
+constexpr int kMaxDevices = 64;
+constexpr int kSplitQuantum = 128;  // split_tokens granularity (a multiple of every tile)
+constexpr int kStages = 3;
+
+// ------------------------------------------------------------------ device info
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+  bool ok = false;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device_info(DeviceInfo *out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.ok) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    d.ok = true;
+  }
+  *out = d;
+  return d.major == 10 ? GQA_OK : GQA_ERR_DEVICE;
+}
+
+// ------------------------------------------------------------------ TMA encode
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *ptr = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// A 4-D view [pages][G][rows_per_page][D] of a bf16 pool, boxes of 64 x box_rows.
+int encode_pool(CUtensorMap *map, const void *base, int D, int rows_per_page, int G,
+                long long pages, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return GQA_ERR_CUDA;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows_per_page),
+                        static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(pages)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(rows_per_page) * D * 2,
+                           static_cast<cuuint64_t>(G) * rows_per_page * D * 2};
+  cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(box_rows), 1u, 1u};
+  cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ validation
+struct Shape {
+  int b, H, G, r, D, P, num_pages, max_pages;
+  bool paged;
+  long long capacity;
+  int nt, nhb;  // kernel variant: n8 tiles per consumer warp, head blocks
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const gqa_dims *dims, bool paged, Shape *sh) {
+  if (!dims) return GQA_ERR_NULL_POINTER;
+  const gqa_dims &d = *dims;
+  if (d.batch < 1 || d.num_heads < 1 || d.num_kv_heads < 1 || d.page_size < 1) return GQA_ERR_DIMS;
+  if (d.batch > 65535 || d.num_kv_heads > 65535) return GQA_ERR_DIMS;  // grid y/z limits
+  if (d.num_heads % d.num_kv_heads != 0) return GQA_ERR_HEADS;
+  const int r = d.num_heads / d.num_kv_heads;
+  if (r > GQA_MAX_GROUP_RATIO) return GQA_ERR_HEADS;
+  if (d.head_dim != 64 && d.head_dim != 128) return GQA_ERR_HEAD_DIM;
+  if (d.flags & ~(GQA_FLAG_CONTRACT_MMA | GQA_FLAG_CONTRACT_FMA)) return GQA_ERR_DIMS;
+  if ((d.flags & GQA_FLAG_CONTRACT_MMA) && (d.flags & GQA_FLAG_CONTRACT_FMA)) return GQA_ERR_DIMS;
+  Shape s{};
+  s.b = d.batch;
+  s.H = d.num_heads;
+  s.G = d.num_kv_heads;
+  s.r = r;
+  s.D = d.head_dim;
+  s.P = d.page_size;
+  s.paged = paged;
+  if (paged) {
+    if (d.page_size < 8 || d.page_size > (1 << 20) || (d.page_size & (d.page_size - 1)))
+      return GQA_ERR_PAGE_SIZE;
+    if (d.num_pages < 1 || d.max_pages_per_seq < 1) return GQA_ERR_DIMS;
+    s.num_pages = d.num_pages;
+    s.max_pages = d.max_pages_per_seq;
+    s.capacity = static_cast<long long>(d.max_pages_per_seq) * d.page_size;
+  } else {
+    s.num_pages = d.batch;
+    s.max_pages = 1;
+    s.capacity = d.page_size;
+  }
+  if (s.capacity > (1ll << 30)) return GQA_ERR_DIMS;
+  if (r <= 8) {
+    s.nt = 1;
+    s.nhb = 1;
+  } else if (r <= 16) {
+    s.nt = 2;
+    s.nhb = 1;
+  } else if (r <= 32) {
+    s.nt = 2;
+    s.nhb = 2;
+  } else {
+    s.nt = 2;
+    s.nhb = 4;
+  }
+  *sh = s;
+  return GQA_OK;
+}
+
+int check_inputs(const void *q, const void *k, const void *v, const int32_t *seqlens,
+                 const uint32_t *status) {
+  if (!q || !k || !v || !seqlens) return GQA_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return GQA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(status) & 3u))
+    return GQA_ERR_MISALIGNED;
+  return GQA_OK;
+}
+
+// ------------------------------------------------------------------ workspace
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct Workspace {
+  size_t o_bytes, m_bytes, total;
+};
+
+Workspace workspace_layout(const Shape &sh, int num_splits) {
+  Workspace w;
+  const size_t rows = static_cast<size_t>(sh.b) * sh.H * num_splits;
+  w.o_bytes = round256(rows * sh.D * sizeof(float));
+  w.m_bytes = round256(rows * sizeof(float));
+  w.total = w.o_bytes + 2 * w.m_bytes;
+  return w;
+}
+
+int split_plan(const Shape &sh, int sms, int max_seqlen) {
+  // Enough (split, group, sequence) blocks for several waves of two blocks per SM.
+  const long long units = static_cast<long long>(sh.b) * sh.G;
+  const long long want = 4ll * 2 * sms;
+  long long splits = (want + units - 1) / units;
+  splits = std::max<long long>(1, std::min<long long>(splits, (max_seqlen + kSplitQuantum - 1) / kSplitQuantum));
+  long long tokens = (max_seqlen + splits - 1) / splits;
+  tokens = (tokens + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
+  return static_cast<int>(std::max<long long>(kSplitQuantum, tokens));
+}
+
+int cluster_plan(const Shape &sh, int sms) {
+  // Blocks per (sequence, group): a power of two <= 8 that gives at least two
+  // blocks per SM, never more blocks than 128-token tiles of the capacity.
+  const long long units = static_cast<long long>(sh.b) * sh.G;
+  const long long max_by_len = std::max<long long>(1, sh.capacity / 128);
+  int c = 1;
+  while (c < 8 && units * c < 2ll * sms && 2 * c <= max_by_len) c *= 2;
+  return c;
+}
+
+// ------------------------------------------------------------------ launches
+template <int D, int NT, int NHB, bool PAGED, Mode MODE>
+int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p, dim3 grid,
+                    int cluster, cudaStream_t stream) {
+  constexpr int CH = (D == 64) ? 2 : 1;
+  using TL = gqa::Tile<D, NT, NHB, CH, kStages>;
+  auto kernel = gqa::gqa_decode_kernel<D, NT, NHB, CH, kStages, PAGED, MODE>;
+  const int smem = TL::kSmemBytes;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return GQA_ERR_CUDA;
+  if (MODE == Mode::kCluster && cluster > 1) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+      return GQA_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(TL::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  cfg.numAttrs = 0;
+  if (MODE == Mode::kCluster) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+template <int D, bool PAGED, Mode MODE>
+int launch_decode_d(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv,
+                    const DecodeParams &p, dim3 grid, int cluster, cudaStream_t stream) {
+  if (sh.nt == 1) return launch_decode_t<D, 1, 1, PAGED, MODE>(tk, tv, p, grid, cluster, stream);
+  switch (sh.nhb) {
+    case 1: return launch_decode_t<D, 2, 1, PAGED, MODE>(tk, tv, p, grid, cluster, stream);
+    case 2: return launch_decode_t<D, 2, 2, PAGED, MODE>(tk, tv, p, grid, cluster, stream);
+    default: return launch_decode_t<D, 2, 4, PAGED, MODE>(tk, tv, p, grid, cluster, stream);
+  }
+}
+
+template <bool PAGED, Mode MODE>
+int launch_decode(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p,
+                  dim3 grid, int cluster, cudaStream_t stream) {
+  return sh.D == 128 ? launch_decode_d<128, PAGED, MODE>(sh, tk, tv, p, grid, cluster, stream)
+                     : launch_decode_d<64, PAGED, MODE>(sh, tk, tv, p, grid, cluster, stream);
+}
+
+int tile_tokens(const Shape &sh) { return sh.D == 64 ? 128 : 64; }
+
+int encode_maps(const Shape &sh, const void *k, const void *v, CUtensorMap *tk, CUtensorMap *tv) {
+  const int T = tile_tokens(sh);
+  const int rows = sh.P;  // paged: page size; contiguous: capacity m
+  const long long pages = sh.paged ? sh.num_pages : sh.b;
+  const int box = sh.paged ? std::min(sh.P, T) : T;
+  int rc = encode_pool(tk, k, sh.D, rows, sh.G, pages, box);
+  if (rc == GQA_OK) rc = encode_pool(tv, v, sh.D, rows, sh.G, pages, box);
+  return rc;
+}
+
+DecodeParams base_params(const Shape &sh, const void *q, const int32_t *seqlens, const int32_t *pt,
+                         uint32_t *status, float scale) {
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.seqlens = seqlens;
+  p.page_table = pt;
+  p.status = status;
+  p.H = sh.H;
+  p.G = sh.G;
+  p.r = sh.r;
+  p.page_size = sh.P;
+  p.num_pages = sh.num_pages;
+  p.max_pages = sh.max_pages;
+  p.capacity = static_cast<int>(sh.capacity);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  return p;
+}
+
+struct SplitArgs {
+  Shape sh;
+  int split_tokens, num_splits;
+  Workspace ws;
+};
+
+int prepare_split(const gqa_dims *dims, bool paged, int32_t split_tokens, int32_t max_seqlen,
+                  const void *workspace, size_t workspace_bytes, int sms, SplitArgs *out) {
+  int rc = check_dims(dims, paged, &out->sh);
+  if (rc != GQA_OK) return rc;
+  if (max_seqlen < 1) return GQA_ERR_DIMS;
+  if (split_tokens < 0 || split_tokens % kSplitQuantum != 0) return GQA_ERR_SPLIT;
+  if (split_tokens == 0) {
+    if (sms <= 0) return GQA_ERR_SPLIT;
+    split_tokens = split_plan(out->sh, sms, max_seqlen);
+  }
+  out->split_tokens = split_tokens;
+  out->num_splits = (max_seqlen + split_tokens - 1) / split_tokens;
+  if (out->num_splits > 65535) return GQA_ERR_SPLIT;
+  out->ws = workspace_layout(out->sh, out->num_splits);
+  if (!workspace) return GQA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
+  if (workspace_bytes < out->ws.total) return GQA_ERR_WORKSPACE;
+  return GQA_OK;
+}
+
+int run_partials(const SplitArgs &a, const void *q, const void *k, const void *v,
+                 const int32_t *seqlens, const int32_t *pt, float scale, uint32_t *status,
+                 int32_t max_seqlen, void *workspace, cudaStream_t stream) {
+  CUtensorMap tk, tv;
+  int rc = encode_maps(a.sh, k, v, &tk, &tv);
+  if (rc != GQA_OK) return rc;
+  DecodeParams p = base_params(a.sh, q, seqlens, pt, status, scale);
+  p.capacity = static_cast<int>(std::min<long long>(a.sh.capacity, max_seqlen));
+  p.split_tokens = a.split_tokens;
+  p.num_splits = a.num_splits;
+  uint8_t *w = static_cast<uint8_t *>(workspace);
+  p.part_o = reinterpret_cast<float *>(w);
+  p.part_m = reinterpret_cast<float *>(w + a.ws.o_bytes);
+  p.part_l = reinterpret_cast<float *>(w + a.ws.o_bytes + a.ws.m_bytes);
+  dim3 grid(a.num_splits, a.sh.G, a.sh.b);
+  return a.sh.paged ? launch_decode<true, Mode::kSplit>(a.sh, tk, tv, p, grid, 1, stream)
+                    : launch_decode<false, Mode::kSplit>(a.sh, tk, tv, p, grid, 1, stream);
+}
+
+int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t *status,
+                int32_t max_seqlen, const void *workspace, cudaStream_t stream) {
+  CombineParams c{};
+  const uint8_t *w = static_cast<const uint8_t *>(workspace);
+  c.seqlens = seqlens;
+  c.out = out;
+  c.part_o = reinterpret_cast<const float *>(w);
+  c.part_m = reinterpret_cast<const float *>(w + a.ws.o_bytes);
+  c.part_l = reinterpret_cast<const float *>(w + a.ws.o_bytes + a.ws.m_bytes);
+  c.status = status;
+  c.b = a.sh.b;
+  c.H = a.sh.H;
+  c.max_len = max_seqlen;
+  c.split_tokens = a.split_tokens;
+  c.num_splits = a.num_splits;
+  const int rows = a.sh.b * a.sh.H;
+  const int rpb = 128 / (a.sh.D / 4);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((rows + rpb - 1) / rpb, 1, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = a.sh.D == 128 ? cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<128>, c)
+                                : cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<64>, c);
+  return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+int32_t gqa_abi_version(void) { return (1 << 16) | 0; }
+
+const char *gqa_status_string(int code) {
+  switch (code) {
+    case GQA_OK: return "ok";
+    case GQA_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case GQA_ERR_MISALIGNED: return "a buffer is not 16-byte aligned";
+    case GQA_ERR_HEADS: return "num_heads is not a multiple of num_kv_heads, or the group ratio exceeds 64";
+    case GQA_ERR_HEAD_DIM: return "head_dim must be 64 or 128";
+    case GQA_ERR_PAGE_SIZE: return "page_size must be a power of two in [8, 2^20]";
+    case GQA_ERR_DIMS: return "a size or flag is out of range";
+    case GQA_ERR_SPLIT: return "split_tokens must be 0 or a positive multiple of 128";
+    case GQA_ERR_WORKSPACE: return "workspace missing or too small";
+    case GQA_ERR_CUDA: return "a CUDA call failed";
+    case GQA_ERR_DEVICE: return "the current device is not an sm_100 (B200) GPU";
+    default: return "unknown status";
+  }
+}
+
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+               const int32_t *page_table, float *out, const gqa_dims *dims, float scale,
+               uint32_t *status, void *stream) {
+  Shape sh;
+  int rc = check_dims(dims, page_table != nullptr, &sh);
+  if (rc != GQA_OK) return rc;
+  rc = check_inputs(q, k_cache, v_cache, seqlens, status);
+  if (rc != GQA_OK) return rc;
+  if (!out) return GQA_ERR_NULL_POINTER;
+  if (!aligned16(out)) return GQA_ERR_MISALIGNED;
+  if (!std::isfinite(scale)) return GQA_ERR_DIMS;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+  CUtensorMap tk, tv;
+  if ((rc = encode_maps(sh, k_cache, v_cache, &tk, &tv)) != GQA_OK) return rc;
+  DecodeParams p = base_params(sh, q, seqlens, page_table, status, scale);
+  p.out = out;
+  const int c = cluster_plan(sh, dev.sms);
+  dim3 grid(c, sh.G, sh.b);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return sh.paged ? launch_decode<true, Mode::kCluster>(sh, tk, tv, p, grid, c, st)
+                  : launch_decode<false, Mode::kCluster>(sh, tk, tv, p, grid, c, st);
+}
+
+size_t gqa_decode_split_workspace_size(const gqa_dims *dims, int32_t max_seqlen, int32_t split_tokens) {
+  Shape sh;  // only b, H and d matter here
+  if (!dims || check_dims(dims, false, &sh) != GQA_OK) return 0;
+  if (max_seqlen < 1 || split_tokens < 0 || split_tokens % kSplitQuantum != 0) return 0;
+  if (split_tokens == 0) split_tokens = kSplitQuantum;  // the smallest split bounds every plan
+  const int splits = (max_seqlen + split_tokens - 1) / split_tokens;
+  return workspace_layout(sh, splits).total;
+}
+
+int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms) {
+  Shape sh;
+  if (!dims) return GQA_ERR_NULL_POINTER;
+  int rc = check_dims(dims, false, &sh);
+  if (rc != GQA_OK) return rc;
+  if (max_seqlen < 1) return GQA_ERR_DIMS;
+  if (num_sms <= 0) {
+    DeviceInfo dev;
+    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+    num_sms = dev.sms;
+  }
+  return split_plan(sh, num_sms, max_seqlen);
+}
+
+int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *seqlens, const int32_t *page_table, const gqa_dims *dims,
+                       float scale, uint32_t *status, int32_t split_tokens, int32_t max_seqlen,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+  int rc = check_inputs(q, k_cache, v_cache, seqlens, status);
+  if (rc != GQA_OK) return rc;
+  if (!std::isfinite(scale)) return GQA_ERR_DIMS;
+  SplitArgs a;
+  int sms = 0;
+  if (split_tokens == 0) {
+    Shape tmp;
+    if ((rc = check_dims(dims, page_table != nullptr, &tmp)) != GQA_OK) return rc;
+    DeviceInfo dev;
+    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+    sms = dev.sms;
+  }
+  rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace,
+                     workspace_bytes, sms, &a);
+  if (rc != GQA_OK) return rc;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+  return run_partials(a, q, k_cache, v_cache, seqlens, page_table, scale, status, max_seqlen,
+                      workspace, static_cast<cudaStream_t>(stream));
+}
+
+int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims, uint32_t *status,
+                      int32_t split_tokens, int32_t max_seqlen, const void *workspace,
+                      size_t workspace_bytes, void *stream) {
+  if (!seqlens || !out) return GQA_ERR_NULL_POINTER;
+  if (!aligned16(out)) return GQA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(status) & 3u))
+    return GQA_ERR_MISALIGNED;
+  if (split_tokens == 0) return GQA_ERR_SPLIT;  // the combine must know the split actually used
+  SplitArgs a;  // the merge needs b, H, d and the split geometry only
+  int rc = prepare_split(dims, false, split_tokens, max_seqlen, workspace, workspace_bytes, 0, &a);
+  if (rc != GQA_OK) return rc;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+  return run_combine(a, seqlens, out, status, max_seqlen, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                     const int32_t *page_table, float *out, const gqa_dims *dims, float scale,
+                     uint32_t *status, int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                     size_t workspace_bytes, void *stream) {
+  int rc = check_inputs(q, k_cache, v_cache, seqlens, status);
+  if (rc != GQA_OK) return rc;
+  if (!out) return GQA_ERR_NULL_POINTER;
+  if (!aligned16(out)) return GQA_ERR_MISALIGNED;
+  if (!std::isfinite(scale)) return GQA_ERR_DIMS;
+  int sms = 0;
+  if (split_tokens == 0) {
+    Shape tmp;
+    if ((rc = check_dims(dims, page_table != nullptr, &tmp)) != GQA_OK) return rc;
+    DeviceInfo dev;
+    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+    sms = dev.sms;
+  }
+  SplitArgs a;
+  rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace,
+                     workspace_bytes, sms, &a);
+  if (rc != GQA_OK) return rc;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = run_partials(a, q, k_cache, v_cache, seqlens, page_table, scale, status, max_seqlen, workspace, st);
+  if (rc != GQA_OK) return rc;
+  return run_combine(a, seqlens, out, status, max_seqlen, workspace, st);
+}
+
+}  // extern "C"

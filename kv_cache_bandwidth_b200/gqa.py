@@ -1,0 +1,212 @@
+"""Python binding of libgqa (include/gqa.h): argument marshalling only.
+
+Every entry point of the C ABI has a function of the same name here.  They take
+torch tensors that already live on the current CUDA device, pass their device
+pointers and the current stream to the library, and return what it returns.
+No step of the computation runs in Python, and there is no fallback: if
+``libgqa.so`` is missing, importing the library raises.
+
+    out = gqa_decode(q, k_cache, v_cache, seqlens, page_table)          # no workspace
+    out = gqa_decode_split(q, k_cache, v_cache, seqlens, page_table,
+                           split_tokens=4096, max_seqlen=131072)          # split-KV + combine
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "GqaError", "Dims", "load", "lib_path", "gqa_decode", "gqa_decode_split",
+    "gqa_split_partials", "gqa_split_combine", "gqa_decode_split_workspace_size",
+    "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version", "dims_for",
+    "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
+    "FLAG_CONTRACT_FMA", "ERRORS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libgqa.so")
+
+STATUS_BAD_SEQLEN = 1
+STATUS_BAD_PAGE = 2
+STATUS_TIMEOUT = 4
+FLAG_CONTRACT_MMA = 1
+FLAG_CONTRACT_FMA = 2
+
+ERRORS = {
+    0: "GQA_OK", -1: "GQA_ERR_NULL_POINTER", -2: "GQA_ERR_MISALIGNED", -3: "GQA_ERR_HEADS",
+    -4: "GQA_ERR_HEAD_DIM", -5: "GQA_ERR_PAGE_SIZE", -6: "GQA_ERR_DIMS", -7: "GQA_ERR_SPLIT",
+    -8: "GQA_ERR_WORKSPACE", -9: "GQA_ERR_CUDA", -10: "GQA_ERR_DEVICE",
+}
+
+
+class GqaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s (%s)" % (what, gqa_status_string(code), ERRORS.get(code, code)))
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    """Mirror of ``gqa_dims``."""
+
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+        ("max_pages_per_seq", ctypes.c_int32), ("flags", ctypes.c_uint32),
+    ]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_DECODE_ARGS = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), ctypes.c_float, _vp]
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Open libgqa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError("libgqa.so is missing at %s: build it with "
+                           "`python -m kv_cache_bandwidth_b200.build`" % _LIB_PATH)
+    lib = ctypes.CDLL(_LIB_PATH)
+    lib.gqa_decode.restype = ctypes.c_int
+    lib.gqa_decode.argtypes = _DECODE_ARGS + [_vp]
+    lib.gqa_decode_split.restype = ctypes.c_int
+    lib.gqa_decode_split.argtypes = _DECODE_ARGS + [ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
+    lib.gqa_split_partials.restype = ctypes.c_int
+    lib.gqa_split_partials.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), ctypes.c_float, _vp,
+                                       ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
+    lib.gqa_split_combine.restype = ctypes.c_int
+    lib.gqa_split_combine.argtypes = [_vp, _vp, ctypes.POINTER(Dims), _vp, ctypes.c_int32, ctypes.c_int32,
+                                      _vp, ctypes.c_size_t, _vp]
+    lib.gqa_decode_split_workspace_size.restype = ctypes.c_size_t
+    lib.gqa_decode_split_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32]
+    lib.gqa_plan_split_tokens.restype = ctypes.c_int32
+    lib.gqa_plan_split_tokens.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32]
+    lib.gqa_status_string.restype = ctypes.c_char_p
+    lib.gqa_status_string.argtypes = [ctypes.c_int]
+    lib.gqa_abi_version.restype = ctypes.c_int32
+    lib.gqa_abi_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def gqa_status_string(code: int) -> str:
+    return load().gqa_status_string(int(code)).decode()
+
+
+def gqa_abi_version() -> int:
+    return int(load().gqa_abi_version())
+
+
+def dims_for(q: torch.Tensor, k_cache: torch.Tensor, page_table: Optional[torch.Tensor],
+             flags: int = 0) -> Dims:
+    """``gqa_dims`` from tensor shapes: q [b,H,d]; cache [pages,G,P,d] or [b,G,m,d]."""
+    b, H, d = q.shape
+    pages, G, P, _ = k_cache.shape
+    max_pages = 0 if page_table is None else page_table.shape[1]
+    return Dims(b, H, G, d, P, pages, max_pages, flags)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise GqaError(rc, what)
+
+
+def _out_for(q: torch.Tensor, out: Optional[torch.Tensor]) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    return out
+
+
+def _scale(q: torch.Tensor, scale: Optional[float]) -> float:
+    return 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
+
+
+def gqa_decode(q, k_cache, v_cache, seqlens, page_table=None, *, out=None, scale=None,
+               status=None, stream=None, flags: int = 0) -> torch.Tensor:
+    """One decode step without a workspace (cluster kernel).  Returns ``out``."""
+    out = _out_for(q, out)
+    dims = dims_for(q, k_cache, page_table, flags)
+    rc = load().gqa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
+                           _ptr(out), ctypes.byref(dims), _scale(q, scale), _ptr(status), _stream(stream))
+    _check(rc, "gqa_decode")
+    return out
+
+
+def gqa_decode_split_workspace_size(dims: Dims, max_seqlen: int, split_tokens: int) -> int:
+    return int(load().gqa_decode_split_workspace_size(ctypes.byref(dims), int(max_seqlen), int(split_tokens)))
+
+
+def gqa_plan_split_tokens(dims: Dims, max_seqlen: int, num_sms: int = 0) -> int:
+    rc = int(load().gqa_plan_split_tokens(ctypes.byref(dims), int(max_seqlen), int(num_sms)))
+    if rc < 0:
+        raise GqaError(rc, "gqa_plan_split_tokens")
+    return rc
+
+
+def workspace_for(q, k_cache, page_table, max_seqlen: int, split_tokens: int) -> torch.Tensor:
+    """Allocate a workspace (torch, on q's device) big enough for the call."""
+    n = gqa_decode_split_workspace_size(dims_for(q, k_cache, page_table), max_seqlen, split_tokens)
+    if n == 0:
+        raise GqaError(-6, "gqa_decode_split_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def gqa_decode_split(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int = 0,
+                     max_seqlen: Optional[int] = None, workspace=None, out=None, scale=None,
+                     status=None, stream=None, flags: int = 0) -> torch.Tensor:
+    """Split-KV decode (partials kernel + combine kernel).  Returns ``out``.
+
+    max_seqlen defaults to the cache capacity (contiguous m, or
+    max_pages_per_seq * page_size)."""
+    out = _out_for(q, out)
+    if max_seqlen is None:
+        max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
+    if workspace is None:
+        workspace = workspace_for(q, k_cache, page_table, max_seqlen, split_tokens)
+    dims = dims_for(q, k_cache, page_table, flags)
+    rc = load().gqa_decode_split(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
+                                 _ptr(out), ctypes.byref(dims), _scale(q, scale), _ptr(status),
+                                 int(split_tokens), int(max_seqlen), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "gqa_decode_split")
+    return out
+
+
+def gqa_split_partials(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int,
+                       max_seqlen: int, workspace, scale=None, status=None, stream=None,
+                       flags: int = 0) -> None:
+    dims = dims_for(q, k_cache, page_table, flags)
+    rc = load().gqa_split_partials(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
+                                   ctypes.byref(dims), _scale(q, scale), _ptr(status), int(split_tokens),
+                                   int(max_seqlen), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "gqa_split_partials")
+
+
+def gqa_split_combine(seqlens, out, dims: Dims, *, split_tokens: int, max_seqlen: int, workspace,
+                      status=None, stream=None) -> torch.Tensor:
+    rc = load().gqa_split_combine(_ptr(seqlens), _ptr(out), ctypes.byref(dims), _ptr(status),
+                                  int(split_tokens), int(max_seqlen), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "gqa_split_combine")
+    return out

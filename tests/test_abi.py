@@ -1,0 +1,141 @@
+"""The C ABI without a GPU: every declared symbol is exported, host-side
+argument checks return their codes before anything touches a device, and the
+pure host arithmetic (workspace size, split plan) is right."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kv_cache_bandwidth_b200 import build as gqa_build
+from kv_cache_bandwidth_b200 import gqa
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "gqa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gqa_build.build()
+    return gqa.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(gqa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("gqa_decode", "gqa_decode_split", "gqa_decode_split_workspace_size", "gqa_split_partials",
+              "gqa_split_combine", "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_abi_version_and_strings(lib):
+    assert gqa.gqa_abi_version() >> 16 == 1
+    for code in gqa.ERRORS:
+        assert gqa.gqa_status_string(code)
+    assert gqa.gqa_status_string(0) == "ok"
+    assert gqa.gqa_status_string(12345) == "unknown status"
+
+
+def _dims(**kw):
+    base = dict(batch=2, num_heads=8, num_kv_heads=2, head_dim=64, page_size=256, num_pages=2,
+                max_pages_per_seq=0, flags=0)
+    base.update(kw)
+    return gqa.Dims(*[base[f] for f, _ in gqa.Dims._fields_])
+
+
+FAKE = 0x10000  # never dereferenced: every case below fails validation first
+
+
+def _decode(lib, dims, q=FAKE, k=FAKE, v=FAKE, seq=FAKE, pt=None, out=FAKE, scale=0.125, status=None):
+    return lib.gqa_decode(q, k, v, seq, pt, out, ctypes.byref(dims), scale, status, None)
+
+
+@pytest.mark.parametrize("case,kw,code", [
+    ("null q", dict(q=None), -1),
+    ("null out", dict(out=None), -1),
+    ("misaligned k", dict(k=FAKE + 8), -2),
+    ("misaligned out", dict(out=FAKE + 4), -2),
+    ("misaligned seqlens", dict(seq=FAKE + 2), -2),
+    ("nan scale", dict(scale=float("nan")), -6),
+])
+def test_decode_pointer_checks(lib, case, kw, code):
+    assert _decode(lib, _dims(), **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_heads=9), -3),
+    (dict(num_heads=130, num_kv_heads=2), -3),      # r = 65 > 64
+    (dict(head_dim=96), -4),
+    (dict(batch=0), -6),
+    (dict(num_kv_heads=0), -6),
+    (dict(flags=3), -6),
+    (dict(flags=8), -6),
+])
+def test_decode_dim_checks(lib, kw, code):
+    assert _decode(lib, _dims(**kw)) == code
+
+
+@pytest.mark.parametrize("P,code", [(12, -5), (4, -5), (0, -6)])
+def test_paged_page_size_checks(lib, P, code):
+    d = _dims(page_size=P, num_pages=8, max_pages_per_seq=4)
+    assert _decode(lib, d, pt=FAKE) == code
+
+
+def test_paged_needs_pool_sizes(lib):
+    assert _decode(lib, _dims(page_size=16, num_pages=0, max_pages_per_seq=4), pt=FAKE) == -6
+    assert _decode(lib, _dims(page_size=16, num_pages=8, max_pages_per_seq=0), pt=FAKE) == -6
+
+
+def test_workspace_size(lib):
+    d = _dims(batch=4, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072)
+    S = 131072 // 4096
+    rows = 4 * 32 * S
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert gqa.gqa_decode_split_workspace_size(d, 131072, 4096) == r256(rows * 128 * 4) + 2 * r256(rows * 4)
+    assert gqa.gqa_decode_split_workspace_size(d, 131072, 100) == 0       # not a multiple of 128
+    assert gqa.gqa_decode_split_workspace_size(d, 0, 4096) == 0
+    # split_tokens = 0 sizes for the finest split, which bounds every plan
+    assert gqa.gqa_decode_split_workspace_size(d, 4096, 0) == gqa.gqa_decode_split_workspace_size(d, 4096, 128)
+
+
+def test_split_checks(lib):
+    d = _dims()
+    ws = FAKE
+    call = lambda split, maxlen, nbytes, w=ws: lib.gqa_decode_split(
+        FAKE, FAKE, FAKE, FAKE, None, FAKE, ctypes.byref(d), 0.125, None, split, maxlen, w, nbytes, None)
+    need = gqa.gqa_decode_split_workspace_size(d, 256, 128)
+    assert call(100, 256, need) == -7
+    assert call(-128, 256, need) == -7
+    assert call(128, 0, need) == -6
+    assert call(128, 256, need - 1) == -8
+    assert call(128, 256, need, w=None) == -8
+    assert call(128, 256, need, w=FAKE + 8) == -2
+    assert lib.gqa_split_combine(FAKE, FAKE, ctypes.byref(d), None, 0, 256, ws, need, None) == -7
+
+
+def test_plan_split_tokens(lib):
+    # Llama-2-70B layer: 32 sequences x 8 groups on 148 SMs
+    d = _dims(batch=32, num_heads=64, num_kv_heads=8, head_dim=128, page_size=4096)
+    t = gqa.gqa_plan_split_tokens(d, 4096, 148)
+    assert t % 128 == 0 and 128 <= t <= 4096
+    blocks = 32 * 8 * -(-4096 // t)
+    assert blocks >= 2 * 148
+    # a single long sequence is cut finely enough to fill the GPU
+    d1 = _dims(batch=1, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072)
+    t1 = gqa.gqa_plan_split_tokens(d1, 131072, 148)
+    assert 4 * -(-131072 // t1) >= 2 * 148
+    # never below one quantum, never above the length rounded up
+    assert gqa.gqa_plan_split_tokens(d1, 1, 148) == 128
+    with pytest.raises(gqa.GqaError) as e:
+        gqa.gqa_plan_split_tokens(_dims(batch=0), 128, 148)
+    assert e.value.code == -6

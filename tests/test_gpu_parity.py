@@ -1,0 +1,268 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Tolerances: max-abs error <= 2e-3 and relative L2 error <= 1e-3 on the fp32
+output (bf16 inputs, fp32 accumulation); the integer path (page-table
+translation, length handling, status bits, zero rows) is compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_bandwidth_b200 import gqa
+from kv_cache_bandwidth_b200.workloads import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-3
+REL_L2 = 1e-3
+
+
+def assert_parity(got, ref, what=""):
+    g = got.detach().double().cpu().numpy().reshape(ref.shape)
+    diff = g - ref
+    max_abs = float(np.abs(diff).max(initial=0.0))
+    rel = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+    assert np.isfinite(g).all(), "%s: non-finite output" % what
+    assert max_abs <= MAX_ABS and rel <= REL_L2, "%s: max_abs %.3e rel_l2 %.3e" % (what, max_abs, rel)
+    return max_abs, rel
+
+
+def run_oracle(inp, rows=None, scale=None):
+    out, st = oracle.gqa_decode(inp.q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu(), inp.seqlens.cpu(),
+                                None if inp.page_table is None else inp.page_table.cpu(),
+                                num_kv_heads=inp.workload.G, scale=scale, rows=rows)
+    return out, st
+
+
+def status_word():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+def run_gpu(inp, entry, split_tokens=0, max_seqlen=None, scale=None, flags=0):
+    st = status_word()
+    if entry == "cluster":
+        out = gqa.gqa_decode(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, scale=scale,
+                             status=st, flags=flags)
+    else:
+        out = gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                                   split_tokens=split_tokens, max_seqlen=max_seqlen, scale=scale,
+                                   status=st, flags=flags)
+    torch.cuda.synchronize()
+    return out, int(st.item())
+
+
+def w_small(b, r, G, d, m, P=None, seed=5):
+    return Workload(name="grid", b=b, H=r * G, G=G, d=d, m=m, page_size=P,
+                    len_lo=1 if P else None, len_hi=m if P else None, seed=seed)
+
+
+# ---------------------------------------------------------------- small grid, full oracle
+
+LENS = [1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 255, 256, 257, 383, 384, 385, 500]
+GRID = []
+for d in (64, 128):
+    for r in (1, 2, 4, 7, 8, 16, 32, 64):
+        GRID.append((d, r))
+
+
+@pytest.mark.parametrize("d,r", GRID, ids=["d%d_r%d" % c for c in GRID])
+@pytest.mark.parametrize("layout", ["contig", "P8", "P16", "P64", "P256"])
+def test_grid_split_and_cluster(d, r, layout):
+    P = None if layout == "contig" else int(layout[1:])
+    G = 2 if r <= 16 else 1
+    lens = LENS if r <= 8 else LENS[::3]
+    w = w_small(b=len(lens), r=r, G=G, d=d, m=512, P=P, seed=d + r)
+    inp = make_inputs(w, device="cuda", lens=lens)
+    ref, st_ref = run_oracle(inp)
+    assert st_ref == 0
+    for entry, split in (("cluster", 0), ("split", 128), ("split", 384), ("split", 0), ("split", 1024)):
+        got, st = run_gpu(inp, entry, split_tokens=split)
+        assert st == 0
+        assert_parity(got, ref, "%s split=%d d=%d r=%d %s" % (entry, split, d, r, layout))
+
+
+def test_tiny_config_both_entry_points():
+    inp = make_inputs(WORKLOADS["tiny"], device="cuda")
+    ref, _ = run_oracle(inp)
+    for entry in ("cluster", "split"):
+        got, st = run_gpu(inp, entry)
+        assert st == 0
+        assert_parity(got, ref, "tiny " + entry)
+
+
+def test_scale_is_applied_in_fp32():
+    """A scale that is not a power of two must not be rounded to bf16."""
+    w = w_small(b=2, r=8, G=2, d=128, m=300)
+    inp = make_inputs(w, device="cuda", lens=[300, 77])
+    inp.q.mul_(4)  # larger logits make a rounded scale visible
+    for scale in (1 / 128 ** 0.5, 0.0, 0.3, -0.2):
+        ref, _ = run_oracle(inp, scale=scale)
+        for entry in ("cluster", "split"):
+            got, _ = run_gpu(inp, entry, scale=scale)
+            assert_parity(got, ref, "scale %g %s" % (scale, entry))
+
+
+def test_single_token_returns_v():
+    w = w_small(b=3, r=4, G=2, d=128, m=64)
+    inp = make_inputs(w, device="cuda", lens=[1, 1, 1])
+    for entry in ("cluster", "split"):
+        got, _ = run_gpu(inp, entry)
+        v0 = inp.v_cache[:, :, 0, :].float().repeat_interleave(4, dim=1)
+        assert torch.equal(got, v0), entry
+
+
+# ---------------------------------------------------------------- bit-exact integer path
+
+
+def _permute_pool(inp, seed):
+    """Same logical cache, pages moved to other physical ids."""
+    n = inp.k_cache.shape[0]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(seed)).to(inp.k_cache.device)
+    k = torch.empty_like(inp.k_cache)
+    v = torch.empty_like(inp.v_cache)
+    k[perm] = inp.k_cache
+    v[perm] = inp.v_cache
+    pt = inp.page_table.clone()
+    valid = pt >= 0
+    pt[valid] = perm.to(torch.int32)[pt[valid].long()]
+    return type(inp)(inp.q, k, v, inp.seqlens, pt, inp.workload)
+
+
+@pytest.mark.parametrize("entry", ["cluster", "split"])
+@pytest.mark.parametrize("P", [8, 16, 128])
+def test_page_permutation_bit_exact(entry, P):
+    w = w_small(b=5, r=8, G=2, d=128, m=1000, P=P)
+    inp = make_inputs(w, device="cuda", lens=[1000, 17, 640, 129, 999], spare_pages=3)
+    a, _ = run_gpu(inp, entry, split_tokens=256)
+    b, _ = run_gpu(_permute_pool(inp, 1), entry, split_tokens=256)
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("entry", ["cluster", "split"])
+def test_contiguous_equals_paged_single_page(entry):
+    w = Workload(name="c", b=3, H=16, G=2, d=128, m=512, seed=9)
+    inp = make_inputs(w, device="cuda", lens=[512, 300, 65])
+    a, _ = run_gpu(inp, entry, split_tokens=256)
+    pt = torch.arange(3, dtype=torch.int32, device="cuda").view(3, 1)
+    paged = type(inp)(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, pt, inp.workload)
+    b, _ = run_gpu(paged, entry, split_tokens=256)
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("entry", ["cluster", "split"])
+@pytest.mark.parametrize("P", [None, 16, 64])
+def test_nan_poison_past_lengths(entry, P):
+    w = w_small(b=4, r=8, G=2, d=128, m=700, P=P)
+    lens = [700, 33, 257, 1]
+    clean = make_inputs(w, device="cuda", lens=lens, spare_pages=2 if P else 0)
+    dirty = make_inputs(w, device="cuda", lens=lens, spare_pages=2 if P else 0, poison=True)
+    a, _ = run_gpu(clean, entry, split_tokens=256)
+    b, _ = run_gpu(dirty, entry, split_tokens=256)
+    assert torch.isfinite(b).all() and torch.equal(a, b)
+
+
+def test_partials_then_combine_equals_decode_split():
+    w = w_small(b=3, r=8, G=4, d=128, m=2048, P=16)
+    inp = make_inputs(w, device="cuda", lens=[2048, 1000, 5])
+    full, _ = run_gpu(inp, "split", split_tokens=512, max_seqlen=2048)
+    ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, 2048, 512)
+    gqa.gqa_split_partials(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, split_tokens=512,
+                           max_seqlen=2048, workspace=ws)
+    out = torch.empty_like(full)
+    gqa.gqa_split_combine(inp.seqlens, out, gqa.dims_for(inp.q, inp.k_cache, inp.page_table),
+                          split_tokens=512, max_seqlen=2048, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, full)
+
+
+def test_repeat_runs_bit_identical():
+    inp = make_inputs(w_small(b=4, r=8, G=2, d=128, m=3000, P=32), device="cuda", lens=[3000, 2000, 10, 1500])
+    for entry in ("cluster", "split"):
+        a, _ = run_gpu(inp, entry)
+        b, _ = run_gpu(inp, entry)
+        assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- data errors on the device
+
+
+@pytest.mark.parametrize("entry", ["cluster", "split"])
+def test_bad_page_id_sets_status_and_zeroes_row(entry):
+    w = w_small(b=3, r=8, G=2, d=128, m=512, P=16)
+    inp = make_inputs(w, device="cuda", lens=[512, 300, 40])
+    clean, st = run_gpu(inp, entry, split_tokens=128)
+    assert st == 0
+    n = inp.k_cache.shape[0]
+    for bad in (-1, n, 10 ** 7):
+        pt = inp.page_table.clone()
+        pt[1, 7] = bad
+        bad_inp = type(inp)(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, pt, inp.workload)
+        got, st = run_gpu(bad_inp, entry, split_tokens=128)
+        assert st == gqa.STATUS_BAD_PAGE
+        assert torch.count_nonzero(got[1]) == 0
+        assert torch.equal(got[0], clean[0]) and torch.equal(got[2], clean[2])
+    # entries past the length are never read
+    pt = inp.page_table.clone()
+    pt[2, 3:] = 10 ** 7
+    got, st = run_gpu(type(inp)(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, pt, inp.workload), entry,
+                      split_tokens=128)
+    assert st == 0 and torch.equal(got, clean)
+
+
+@pytest.mark.parametrize("entry", ["cluster", "split"])
+@pytest.mark.parametrize("paged", [False, True])
+def test_bad_length_sets_status_and_zeroes_row(entry, paged):
+    w = w_small(b=3, r=4, G=2, d=64, m=256, P=16 if paged else None)
+    inp = make_inputs(w, device="cuda", lens=[256, 100, 7])
+    clean, _ = run_gpu(inp, entry, split_tokens=128)
+    for bad in (0, -3, 257, 2 ** 30):
+        sl = inp.seqlens.clone()
+        sl[1] = bad
+        got, st = run_gpu(type(inp)(inp.q, inp.k_cache, inp.v_cache, sl, inp.page_table, inp.workload), entry,
+                          split_tokens=128)
+        assert st == gqa.STATUS_BAD_SEQLEN, (bad, st)
+        assert torch.count_nonzero(got[1]) == 0
+        assert torch.equal(got[0], clean[0]) and torch.equal(got[2], clean[2])
+
+
+def test_split_rejects_length_above_max_seqlen():
+    w = w_small(b=2, r=8, G=2, d=128, m=1024)
+    inp = make_inputs(w, device="cuda", lens=[1024, 200])
+    got, st = run_gpu(inp, "split", split_tokens=256, max_seqlen=512)
+    assert st == gqa.STATUS_BAD_SEQLEN
+    assert torch.count_nonzero(got[0]) == 0
+    ref, _ = run_oracle(inp)
+    assert_parity(got[1], ref[1], "row under max_seqlen")
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled rows
+
+
+def sampled_rows(w, n_seq=3, n_rand=48, seed=0):
+    g = np.random.default_rng(seed)
+    rows = set()
+    for s in g.choice(w.b, size=min(n_seq, w.b), replace=False):
+        rows.update(range(s * w.H, (s + 1) * w.H))
+    rows.update(g.choice(w.b * w.H, size=min(n_rand, w.b * w.H), replace=False).tolist())
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+FULL = ["llama70b", "ragged", "long1", "long4", "sweep_g1", "sweep_g2", "sweep_g4", "sweep_g8", "sweep_g32"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload_sampled(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w, device="cuda")
+    rows = sampled_rows(w)
+    ref, st_ref = run_oracle(inp, rows=rows)
+    assert st_ref == 0
+    cases = [("split", w.split_tokens)]
+    if w.split_tokens:
+        cases.append(("split", 0))
+    cases.append(("cluster", 0))
+    for entry, split in cases:
+        got, st = run_gpu(inp, entry, split_tokens=split)
+        assert st == 0
+        assert_parity(got.view(-1, w.d)[torch.from_numpy(rows).cuda()], ref, "%s %s split=%d" % (name, entry, split))
