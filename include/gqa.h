@@ -107,10 +107,12 @@ typedef struct gqa_dims {
 /*
  * gqa_decode -- one decode step without a workspace.
  *
- * Computes `out` as described above.  Each (sequence, KV group) is handled by
- * one thread-block cluster whose blocks split the group's tokens and merge
- * their partial softmax states through distributed shared memory, so no
- * global scratch is needed.
+ * Computes `out` as described above.  When the (sequence, group) units are
+ * enough to occupy every SM, a persistent grid streams one unit after another
+ * through a single TMA pipeline per block; otherwise each unit is handled by a
+ * thread-block cluster (up to 16 blocks) whose blocks split the unit's tokens
+ * and merge their partial softmax states through distributed shared memory.
+ * Either way no global scratch memory is used.
  *
  * scale: the softmax scale (1/sqrt(d) is scaled_dot_product_attention's default).
  * Returns GQA_OK or a GQA_ERR_* code (nothing launched on error).
@@ -121,16 +123,18 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
 
 /*
  * Split-KV decode.  The tokens of every sequence are cut into consecutive
- * splits of `split_tokens`; one thread block per (split, group, sequence)
- * writes an unnormalised partial softmax state, and a second kernel merges the
- * splits of each (sequence, head) exactly: with m_k the split's running
+ * splits of `split_tokens`; a persistent grid walks the (sequence, group,
+ * split) items, each yielding an unnormalised partial softmax state, and a
+ * second kernel merges the splits of each (sequence, head) exactly (it is not
+ * launched when every sequence fits in one split): with m_k the split's running
  * maximum and l_k its sum of exponentials,
  *     M = max_k m_k,  L = sum_k l_k 2^(m_k - M),  out = sum_k o_k 2^(m_k - M) / L.
  * The merge is an exact re-association of the softmax of the pages' formula
  * (the pages do not describe split-KV; it is how a long cache fills the GPU).
  *
  * split_tokens: a positive multiple of 128, or 0 to let the library choose
- *               (gqa_plan_split_tokens).
+ *               (gqa_plan_split_tokens: no split when the (sequence, group)
+ *               units already cover every SM, else about one item per SM).
  * max_seqlen:   an upper bound of every seqlens[s] (sizes the grid and the
  *               workspace); a length above it is treated as invalid
  *               (GQA_STATUS_BAD_SEQLEN, row zeroed).
@@ -153,17 +157,24 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache,
  * workspace; gqa_split_combine merges them into `out`.  Running the first and
  * then the second on one stream is exactly gqa_decode_split.  The combine is
  * also the merge step for partial states produced elsewhere (e.g. gathered
- * from other GPUs into this workspace).
+ * from other GPUs into this workspace).  split_tokens must be given (not 0).
+ *
+ * out (gqa_split_partials, may be NULL): a sequence that fits in one split is
+ * finished by the partials kernel itself, which writes its rows to `out` and
+ * marks split 0 so that the combine leaves them alone.  With out == NULL every
+ * row goes through the workspace and the combine.
  *
  * Workspace layout (fp32, each array 256-byte aligned, S = ceil(max_seqlen /
  * split_tokens)): o [b, H, S, d] unnormalised sum_j 2^(x_j - m) v_j;
  * m [b, H, S] running maximum of x_j = scale * log2(e) * q.k_j;
- * l [b, H, S] sum_j 2^(x_j - m), or -1 when the split met an invalid page id.
+ * l [b, H, S] sum_j 2^(x_j - m), or a marker: -1 the split met an invalid page
+ * id; -2 (split 0) the length is outside [1, capacity]; -3 (split 0) the row
+ * is already final in `out`.
  * Split k of sequence s covers tokens [k * split_tokens, min(len, (k+1) * split_tokens));
  * the combine reads the splits k < ceil(len / split_tokens).
  */
 int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
-                       const int32_t *seqlens, const int32_t *page_table,
+                       const int32_t *seqlens, const int32_t *page_table, float *out,
                        const gqa_dims *dims, float scale, uint32_t *status,
                        int32_t split_tokens, int32_t max_seqlen, void *workspace,
                        size_t workspace_bytes, void *stream);

@@ -25,7 +25,6 @@ using gqa::Mode;
 
 constexpr int kMaxDevices = 64;
 constexpr int kSplitQuantum = 128;  // split_tokens granularity (a multiple of every tile)
-constexpr int kStages = 3;
 
 // ------------------------------------------------------------------ device info
 struct DeviceInfo {
@@ -91,7 +90,7 @@ struct Shape {
   int b, H, G, r, D, P, num_pages, max_pages;
   bool paged;
   long long capacity;
-  int nt, nhb;  // kernel variant: n8 tiles per consumer warp, head blocks
+  int nt, nhb;  // kernel variant: n8 head tiles per consumer warp, head blocks
 };
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -128,19 +127,9 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh) {
     s.capacity = d.page_size;
   }
   if (s.capacity > (1ll << 30)) return GQA_ERR_DIMS;
-  if (r <= 8) {
-    s.nt = 1;
-    s.nhb = 1;
-  } else if (r <= 16) {
-    s.nt = 2;
-    s.nhb = 1;
-  } else if (r <= 32) {
-    s.nt = 2;
-    s.nhb = 2;
-  } else {
-    s.nt = 2;
-    s.nhb = 4;
-  }
+  if (static_cast<long long>(s.b) * s.H * s.D > (1ll << 31) - 1) return GQA_ERR_DIMS;
+  s.nt = r <= 8 ? 1 : 2;
+  s.nhb = r <= 16 ? 1 : (r <= 32 ? 2 : 4);
   *sh = s;
   return GQA_OK;
 }
@@ -170,51 +159,71 @@ Workspace workspace_layout(const Shape &sh, int num_splits) {
   return w;
 }
 
+// Split length when the caller leaves it to the library.  Blocks of a few
+// thousand tokens stream at the best per-block rate; the split is the longest
+// one (at most 4096 tokens) that still gives about 1.5 items per SM, in
+// multiples of 128 tokens.
 int split_plan(const Shape &sh, int sms, int max_seqlen) {
-  // Enough (split, group, sequence) blocks for several waves of two blocks per SM.
   const long long units = static_cast<long long>(sh.b) * sh.G;
-  const long long want = 4ll * 2 * sms;
-  long long splits = (want + units - 1) / units;
+  const long long want_items = (3ll * sms + 1) / 2;
+  long long splits = std::max<long long>((want_items + units - 1) / units, (max_seqlen + 4095) / 4096);
   splits = std::max<long long>(1, std::min<long long>(splits, (max_seqlen + kSplitQuantum - 1) / kSplitQuantum));
   long long tokens = (max_seqlen + splits - 1) / splits;
   tokens = (tokens + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
   return static_cast<int>(std::max<long long>(kSplitQuantum, tokens));
 }
 
+// Blocks per cluster for gqa_decode: 1 (one block per (sequence, group)
+// unit) when the units give about 1.5 blocks per SM; otherwise the smallest
+// power of two (at most 16) that does, never more blocks than 128-token tiles.
 int cluster_plan(const Shape &sh, int sms) {
-  // Blocks per (sequence, group): a power of two <= 8 that gives at least two
-  // blocks per SM, never more blocks than 128-token tiles of the capacity.
   const long long units = static_cast<long long>(sh.b) * sh.G;
+  const long long want = (3ll * sms + 1) / 2;
   const long long max_by_len = std::max<long long>(1, sh.capacity / 128);
   int c = 1;
-  while (c < 8 && units * c < 2ll * sms && 2 * c <= max_by_len) c *= 2;
+  while (c < 16 && units * c < want && 2 * c <= max_by_len) c *= 2;
   return c;
 }
 
 // ------------------------------------------------------------------ launches
-template <int D, int NT, int NHB, bool PAGED, Mode MODE>
-int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p, dim3 grid,
-                    int cluster, cudaStream_t stream) {
+// Pipeline shape per variant.  For r <= 8 (the common GQA ratios) the block
+// is small enough for several blocks per SM: "dual" runs two blocks of 3
+// stages, "trio" three blocks of 2 stages, "solo" one block of 6 stages.
+// Larger ratios run one block per SM with a 3- or 4-stage ring.
+#ifndef GQA_PIPE_POLICY
+#define GQA_PIPE_POLICY 0  // 0: automatic, 1: solo, 2: dual, 3: trio
+#endif
+
+enum class Pipe { kSolo, kDual, kTrio };
+
+struct Launch {
+  dim3 grid;
+  int cluster;
+  cudaStream_t stream;
+};
+
+template <int D, int NT, int NHB, int STAGES, bool PAGED, Mode MODE>
+int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p, const Launch &l) {
   constexpr int CH = (D == 64) ? 2 : 1;
-  using TL = gqa::Tile<D, NT, NHB, CH, kStages>;
-  auto kernel = gqa::gqa_decode_kernel<D, NT, NHB, CH, kStages, PAGED, MODE>;
+  using TL = gqa::Tile<D, NT, NHB, CH, STAGES>;
+  auto kernel = gqa::gqa_decode_kernel<D, NT, NHB, CH, STAGES, PAGED, MODE>;
   const int smem = TL::kSmemBytes;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return GQA_ERR_CUDA;
-  if (MODE == Mode::kCluster && cluster > 1) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+  if (MODE == Mode::kCluster && l.cluster > 8) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       return GQA_ERR_CUDA;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
+  cfg.gridDim = l.grid;
   cfg.blockDim = dim3(TL::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
+  cfg.stream = l.stream;
   cudaLaunchAttribute attr[1];
   cfg.numAttrs = 0;
   if (MODE == Mode::kCluster) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.x = l.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -223,22 +232,40 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
   return cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
-template <int D, bool PAGED, Mode MODE>
-int launch_decode_d(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv,
-                    const DecodeParams &p, dim3 grid, int cluster, cudaStream_t stream) {
-  if (sh.nt == 1) return launch_decode_t<D, 1, 1, PAGED, MODE>(tk, tv, p, grid, cluster, stream);
-  switch (sh.nhb) {
-    case 1: return launch_decode_t<D, 2, 1, PAGED, MODE>(tk, tv, p, grid, cluster, stream);
-    case 2: return launch_decode_t<D, 2, 2, PAGED, MODE>(tk, tv, p, grid, cluster, stream);
-    default: return launch_decode_t<D, 2, 4, PAGED, MODE>(tk, tv, p, grid, cluster, stream);
+Pipe pick_pipe(const Shape &sh) {
+  if (sh.nt != 1) return Pipe::kSolo;
+  switch (GQA_PIPE_POLICY) {
+    case 1: return Pipe::kSolo;
+    case 3: return Pipe::kTrio;
+    default: return Pipe::kDual;
   }
 }
 
-template <bool PAGED, Mode MODE>
+template <int D, bool PAGED, Mode MODE>
+int launch_decode_d(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv,
+                    const DecodeParams &p, const Launch &l) {
+  if (sh.nt == 1) {
+    switch (pick_pipe(sh)) {
+      case Pipe::kTrio: return launch_decode_t<D, 1, 1, 2, PAGED, MODE>(tk, tv, p, l);
+      case Pipe::kSolo: return launch_decode_t<D, 1, 1, 6, PAGED, MODE>(tk, tv, p, l);
+      default: return launch_decode_t<D, 1, 1, 3, PAGED, MODE>(tk, tv, p, l);
+    }
+  }
+  switch (sh.nhb) {
+    case 1: return launch_decode_t<D, 2, 1, 3, PAGED, MODE>(tk, tv, p, l);
+    case 2: return launch_decode_t<D, 2, 2, 4, PAGED, MODE>(tk, tv, p, l);
+    default: return launch_decode_t<D, 2, 4, 4, PAGED, MODE>(tk, tv, p, l);
+  }
+}
+
+template <Mode MODE>
 int launch_decode(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p,
-                  dim3 grid, int cluster, cudaStream_t stream) {
-  return sh.D == 128 ? launch_decode_d<128, PAGED, MODE>(sh, tk, tv, p, grid, cluster, stream)
-                     : launch_decode_d<64, PAGED, MODE>(sh, tk, tv, p, grid, cluster, stream);
+                  const Launch &l) {
+  if (sh.D == 128)
+    return sh.paged ? launch_decode_d<128, true, MODE>(sh, tk, tv, p, l)
+                    : launch_decode_d<128, false, MODE>(sh, tk, tv, p, l);
+  return sh.paged ? launch_decode_d<64, true, MODE>(sh, tk, tv, p, l)
+                  : launch_decode_d<64, false, MODE>(sh, tk, tv, p, l);
 }
 
 int tile_tokens(const Shape &sh) { return sh.D == 64 ? 128 : 64; }
@@ -271,6 +298,28 @@ DecodeParams base_params(const Shape &sh, const void *q, const int32_t *seqlens,
   return p;
 }
 
+// The items kernel: one block per (sequence, group, split) item.
+int run_items(const Shape &sh, const void *q, const void *k, const void *v, const int32_t *seqlens,
+              const int32_t *pt, float *out, float scale, uint32_t *status, int split_tokens,
+              int num_splits, int capacity, float *part_o, float *part_m, float *part_l,
+              cudaStream_t stream) {
+  CUtensorMap tk, tv;
+  int rc = encode_maps(sh, k, v, &tk, &tv);
+  if (rc != GQA_OK) return rc;
+  DecodeParams p = base_params(sh, q, seqlens, pt, status, scale);
+  p.out = out;
+  p.part_o = part_o;
+  p.part_m = part_m;
+  p.part_l = part_l;
+  p.capacity = capacity;
+  p.split_tokens = split_tokens;
+  p.num_splits = num_splits;
+  const long long items = static_cast<long long>(sh.b) * sh.G * num_splits;
+  if (items > (1ll << 31) - 1) return GQA_ERR_DIMS;
+  Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream};
+  return launch_decode<Mode::kItems>(sh, tk, tv, p, l);
+}
+
 struct SplitArgs {
   Shape sh;
   int split_tokens, num_splits;
@@ -298,22 +347,13 @@ int prepare_split(const gqa_dims *dims, bool paged, int32_t split_tokens, int32_
 }
 
 int run_partials(const SplitArgs &a, const void *q, const void *k, const void *v,
-                 const int32_t *seqlens, const int32_t *pt, float scale, uint32_t *status,
+                 const int32_t *seqlens, const int32_t *pt, float *out, float scale, uint32_t *status,
                  int32_t max_seqlen, void *workspace, cudaStream_t stream) {
-  CUtensorMap tk, tv;
-  int rc = encode_maps(a.sh, k, v, &tk, &tv);
-  if (rc != GQA_OK) return rc;
-  DecodeParams p = base_params(a.sh, q, seqlens, pt, status, scale);
-  p.capacity = static_cast<int>(std::min<long long>(a.sh.capacity, max_seqlen));
-  p.split_tokens = a.split_tokens;
-  p.num_splits = a.num_splits;
   uint8_t *w = static_cast<uint8_t *>(workspace);
-  p.part_o = reinterpret_cast<float *>(w);
-  p.part_m = reinterpret_cast<float *>(w + a.ws.o_bytes);
-  p.part_l = reinterpret_cast<float *>(w + a.ws.o_bytes + a.ws.m_bytes);
-  dim3 grid(a.num_splits, a.sh.G, a.sh.b);
-  return a.sh.paged ? launch_decode<true, Mode::kSplit>(a.sh, tk, tv, p, grid, 1, stream)
-                    : launch_decode<false, Mode::kSplit>(a.sh, tk, tv, p, grid, 1, stream);
+  const int capacity = static_cast<int>(std::min<long long>(a.sh.capacity, max_seqlen));
+  return run_items(a.sh, q, k, v, seqlens, pt, out, scale, status, a.split_tokens, a.num_splits,
+                   capacity, reinterpret_cast<float *>(w), reinterpret_cast<float *>(w + a.ws.o_bytes),
+                   reinterpret_cast<float *>(w + a.ws.o_bytes + a.ws.m_bytes), stream);
 }
 
 int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t *status,
@@ -385,15 +425,20 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
   if (!std::isfinite(scale)) return GQA_ERR_DIMS;
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int c = cluster_plan(sh, dev.sms);
+  if (c == 1) {
+    // enough (sequence, group) units: one item each, final rows, no scratch
+    const int split = static_cast<int>((sh.capacity + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum);
+    return run_items(sh, q, k_cache, v_cache, seqlens, page_table, out, scale, status, split, 1,
+                     static_cast<int>(sh.capacity), nullptr, nullptr, nullptr, st);
+  }
   CUtensorMap tk, tv;
   if ((rc = encode_maps(sh, k_cache, v_cache, &tk, &tv)) != GQA_OK) return rc;
   DecodeParams p = base_params(sh, q, seqlens, page_table, status, scale);
   p.out = out;
-  const int c = cluster_plan(sh, dev.sms);
-  dim3 grid(c, sh.G, sh.b);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return sh.paged ? launch_decode<true, Mode::kCluster>(sh, tk, tv, p, grid, c, st)
-                  : launch_decode<false, Mode::kCluster>(sh, tk, tv, p, grid, c, st);
+  Launch l{dim3(c, sh.G, sh.b), c, st};
+  return launch_decode<Mode::kCluster>(sh, tk, tv, p, l);
 }
 
 size_t gqa_decode_split_workspace_size(const gqa_dims *dims, int32_t max_seqlen, int32_t split_tokens) {
@@ -420,27 +465,21 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
 }
 
 int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
-                       const int32_t *seqlens, const int32_t *page_table, const gqa_dims *dims,
-                       float scale, uint32_t *status, int32_t split_tokens, int32_t max_seqlen,
-                       void *workspace, size_t workspace_bytes, void *stream) {
+                       const int32_t *seqlens, const int32_t *page_table, float *out,
+                       const gqa_dims *dims, float scale, uint32_t *status, int32_t split_tokens,
+                       int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream) {
   int rc = check_inputs(q, k_cache, v_cache, seqlens, status);
   if (rc != GQA_OK) return rc;
+  if (out && !aligned16(out)) return GQA_ERR_MISALIGNED;
   if (!std::isfinite(scale)) return GQA_ERR_DIMS;
+  if (split_tokens == 0) return GQA_ERR_SPLIT;  // the combine must be given the same split
   SplitArgs a;
-  int sms = 0;
-  if (split_tokens == 0) {
-    Shape tmp;
-    if ((rc = check_dims(dims, page_table != nullptr, &tmp)) != GQA_OK) return rc;
-    DeviceInfo dev;
-    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    sms = dev.sms;
-  }
-  rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace,
-                     workspace_bytes, sms, &a);
+  rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace, workspace_bytes,
+                     0, &a);
   if (rc != GQA_OK) return rc;
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-  return run_partials(a, q, k_cache, v_cache, seqlens, page_table, scale, status, max_seqlen,
+  return run_partials(a, q, k_cache, v_cache, seqlens, page_table, out, scale, status, max_seqlen,
                       workspace, static_cast<cudaStream_t>(stream));
 }
 
@@ -484,8 +523,9 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, co
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  rc = run_partials(a, q, k_cache, v_cache, seqlens, page_table, scale, status, max_seqlen, workspace, st);
-  if (rc != GQA_OK) return rc;
+  rc = run_partials(a, q, k_cache, v_cache, seqlens, page_table, out, scale, status, max_seqlen,
+                    workspace, st);
+  if (rc != GQA_OK || a.num_splits == 1) return rc;  // one split: rows are final already
   return run_combine(a, seqlens, out, status, max_seqlen, workspace, st);
 }
 

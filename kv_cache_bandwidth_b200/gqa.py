@@ -82,7 +82,7 @@ def load():
     lib.gqa_decode_split.restype = ctypes.c_int
     lib.gqa_decode_split.argtypes = _DECODE_ARGS + [ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
     lib.gqa_split_partials.restype = ctypes.c_int
-    lib.gqa_split_partials.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), ctypes.c_float, _vp,
+    lib.gqa_split_partials.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), ctypes.c_float, _vp,
                                        ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
     lib.gqa_split_combine.restype = ctypes.c_int
     lib.gqa_split_combine.argtypes = [_vp, _vp, ctypes.POINTER(Dims), _vp, ctypes.c_int32, ctypes.c_int32,
@@ -193,11 +193,13 @@ def gqa_decode_split(q, k_cache, v_cache, seqlens, page_table=None, *, split_tok
 
 
 def gqa_split_partials(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int,
-                       max_seqlen: int, workspace, scale=None, status=None, stream=None,
+                       max_seqlen: int, workspace, out=None, scale=None, status=None, stream=None,
                        flags: int = 0) -> None:
+    """Partials kernel only.  With ``out`` given, sequences that fit in one
+    split are finished here and left alone by the combine."""
     dims = dims_for(q, k_cache, page_table, flags)
     rc = load().gqa_split_partials(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
-                                   ctypes.byref(dims), _scale(q, scale), _ptr(status), int(split_tokens),
+                                   _ptr(out), ctypes.byref(dims), _scale(q, scale), _ptr(status), int(split_tokens),
                                    int(max_seqlen), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "gqa_split_partials")

@@ -124,17 +124,24 @@ def test_split_checks(lib):
 
 
 def test_plan_split_tokens(lib):
-    # Llama-2-70B layer: 32 sequences x 8 groups on 148 SMs
+    # Llama-2-70B layer: 32 sequences x 8 groups = 256 units already give
+    # ~1.5 blocks per SM on 148 SMs, and 4096 tokens is not above the cap: no split
     d = _dims(batch=32, num_heads=64, num_kv_heads=8, head_dim=128, page_size=4096)
-    t = gqa.gqa_plan_split_tokens(d, 4096, 148)
-    assert t % 128 == 0 and 128 <= t <= 4096
-    blocks = 32 * 8 * -(-4096 // t)
-    assert blocks >= 2 * 148
-    # a single long sequence is cut finely enough to fill the GPU
+    assert gqa.gqa_plan_split_tokens(d, 4096, 148) == 4096
+    # a single long sequence (4 groups): about 1.5 items per SM
     d1 = _dims(batch=1, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072)
     t1 = gqa.gqa_plan_split_tokens(d1, 131072, 148)
-    assert 4 * -(-131072 // t1) >= 2 * 148
-    # never below one quantum, never above the length rounded up
+    assert t1 % 128 == 0
+    items = 4 * -(-131072 // t1)
+    assert 1.4 * 148 <= items <= 1.6 * 148
+    # long sequences are cut to at most 4096 tokens even when units are plenty
+    d3 = _dims(batch=64, num_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=70000,
+               max_pages_per_seq=2048)
+    assert gqa.gqa_plan_split_tokens(d3, 32768, 148) == 4096
+    # 16 sequences x 1 group (MQA sweep): 14 splits of 8192 tokens -> 640 (rounded to 128)
+    d2 = _dims(batch=16, num_heads=32, num_kv_heads=1, head_dim=128, page_size=8192)
+    assert gqa.gqa_plan_split_tokens(d2, 8192, 148) == 640
+    # never below one quantum
     assert gqa.gqa_plan_split_tokens(d1, 1, 148) == 128
     with pytest.raises(gqa.GqaError) as e:
         gqa.gqa_plan_split_tokens(_dims(batch=0), 128, 148)

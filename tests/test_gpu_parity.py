@@ -162,18 +162,32 @@ def test_nan_poison_past_lengths(entry, P):
     assert torch.isfinite(b).all() and torch.equal(a, b)
 
 
-def test_partials_then_combine_equals_decode_split():
+@pytest.mark.parametrize("with_out", [True, False])
+def test_partials_then_combine_equals_decode_split(with_out):
     w = w_small(b=3, r=8, G=4, d=128, m=2048, P=16)
-    inp = make_inputs(w, device="cuda", lens=[2048, 1000, 5])
+    inp = make_inputs(w, device="cuda", lens=[2048, 1000, 5])   # 4, 2 and 1 splits
     full, _ = run_gpu(inp, "split", split_tokens=512, max_seqlen=2048)
     ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, 2048, 512)
+    out = torch.full_like(full, float("nan"))
     gqa.gqa_split_partials(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, split_tokens=512,
-                           max_seqlen=2048, workspace=ws)
-    out = torch.empty_like(full)
+                           max_seqlen=2048, workspace=ws, out=out if with_out else None)
     gqa.gqa_split_combine(inp.seqlens, out, gqa.dims_for(inp.q, inp.k_cache, inp.page_table),
                           split_tokens=512, max_seqlen=2048, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(out, full)
+
+
+def test_decode_items_path_many_units():
+    """gqa_decode with enough (sequence, group) units for every SM runs the
+    persistent items kernel (one unit per item, final rows, no scratch)."""
+    lens = [(37 * i) % 300 + 1 for i in range(80)]
+    for P in (None, 16):
+        w = w_small(b=80, r=8, G=2, d=128, m=300, P=P, seed=77)
+        inp = make_inputs(w, device="cuda", lens=lens)
+        ref, _ = run_oracle(inp)
+        got, st = run_gpu(inp, "cluster")
+        assert st == 0
+        assert_parity(got, ref, "items path P=%s" % P)
 
 
 def test_repeat_runs_bit_identical():
@@ -187,18 +201,18 @@ def test_repeat_runs_bit_identical():
 # ---------------------------------------------------------------- data errors on the device
 
 
-@pytest.mark.parametrize("entry", ["cluster", "split"])
-def test_bad_page_id_sets_status_and_zeroes_row(entry):
+@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 128), ("split", 512)])
+def test_bad_page_id_sets_status_and_zeroes_row(entry, split):
     w = w_small(b=3, r=8, G=2, d=128, m=512, P=16)
     inp = make_inputs(w, device="cuda", lens=[512, 300, 40])
-    clean, st = run_gpu(inp, entry, split_tokens=128)
+    clean, st = run_gpu(inp, entry, split_tokens=split)
     assert st == 0
     n = inp.k_cache.shape[0]
     for bad in (-1, n, 10 ** 7):
         pt = inp.page_table.clone()
         pt[1, 7] = bad
         bad_inp = type(inp)(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, pt, inp.workload)
-        got, st = run_gpu(bad_inp, entry, split_tokens=128)
+        got, st = run_gpu(bad_inp, entry, split_tokens=split)
         assert st == gqa.STATUS_BAD_PAGE
         assert torch.count_nonzero(got[1]) == 0
         assert torch.equal(got[0], clean[0]) and torch.equal(got[2], clean[2])
@@ -206,21 +220,21 @@ def test_bad_page_id_sets_status_and_zeroes_row(entry):
     pt = inp.page_table.clone()
     pt[2, 3:] = 10 ** 7
     got, st = run_gpu(type(inp)(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, pt, inp.workload), entry,
-                      split_tokens=128)
+                      split_tokens=split)
     assert st == 0 and torch.equal(got, clean)
 
 
-@pytest.mark.parametrize("entry", ["cluster", "split"])
+@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 128), ("split", 256)])
 @pytest.mark.parametrize("paged", [False, True])
-def test_bad_length_sets_status_and_zeroes_row(entry, paged):
+def test_bad_length_sets_status_and_zeroes_row(entry, split, paged):
     w = w_small(b=3, r=4, G=2, d=64, m=256, P=16 if paged else None)
     inp = make_inputs(w, device="cuda", lens=[256, 100, 7])
-    clean, _ = run_gpu(inp, entry, split_tokens=128)
+    clean, _ = run_gpu(inp, entry, split_tokens=split)
     for bad in (0, -3, 257, 2 ** 30):
         sl = inp.seqlens.clone()
         sl[1] = bad
         got, st = run_gpu(type(inp)(inp.q, inp.k_cache, inp.v_cache, sl, inp.page_table, inp.workload), entry,
-                          split_tokens=128)
+                          split_tokens=split)
         assert st == gqa.STATUS_BAD_SEQLEN, (bad, st)
         assert torch.count_nonzero(got[1]) == 0
         assert torch.equal(got[0], clean[0]) and torch.equal(got[2], clean[2])
