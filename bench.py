@@ -230,10 +230,16 @@ def reference_arm(args):
 
 def config_dict(w, inp, split_tokens):
     kv = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
+    if split_tokens is None:
+        decomp = "one block or cluster per (sequence, group)"
+    elif split_tokens == 0:
+        decomp = "equal-work ranges over all (sequence, group) tiles (stream-K) + combine"
+    else:
+        decomp = "fixed splits of %d tokens + combine" % split_tokens
     return {
         "workload": w.name, "b": w.b, "H": w.H, "G": w.G, "d": w.d, "m": w.m,
         "layout": "paged P=%d" % w.page_size if w.paged else "contiguous [b,G,m,d]",
-        "split_tokens": split_tokens, "kv_bytes_per_step": kv, "seed": w.seed,
+        "split_tokens": split_tokens, "decomposition": decomp, "kv_bytes_per_step": kv, "seed": w.seed,
         "l2": ("inputs %.0f MiB > 126 MB L2 (no flush)" % (kv / 2 ** 20)) if kv > 2 * L2_BYTES
         else "L2 flushed between steps",
     }
@@ -249,9 +255,8 @@ def main_gpu(args):
     kv_step = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
     max_seqlen = int(inp.seqlens.max())
     dims = gqa.dims_for(inp.q, inp.k_cache, inp.page_table)
-    split = args.split_tokens if args.split_tokens >= 0 else (w.split_tokens or 0)
-    if split == 0:
-        split = gqa.gqa_plan_split_tokens(dims, max_seqlen)
+    # 0: the library's choice (equal-work ranges); > 0: fixed splits of that many tokens
+    split = args.split_tokens if args.split_tokens >= 0 else w.split_tokens
     ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, max_seqlen, split)
     out = torch.empty(inp.q.shape, dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -269,8 +274,15 @@ def main_gpu(args):
                                  split_tokens=split, max_seqlen=max_seqlen, workspace=ws, out=out,
                                  status=status)
 
-    # the combine kernel runs only when some sequence spans more than one split
-    launches_per_step = 1 if (args.entry == "cluster" or -(-max_seqlen // split) == 1) else 2
+    # decode kernel + combine kernel; the fixed-split combine is skipped when
+    # every sequence fits in one split
+    eff_split = split if split > 0 else gqa.gqa_plan_split_tokens(dims, max_seqlen)
+    if args.entry == "cluster":
+        launches_per_step = 1
+    elif eff_split > 0 and -(-max_seqlen // eff_split) == 1:
+        launches_per_step = 1
+    else:
+        launches_per_step = 2
 
     # ---- warm-up
     for _ in range(args.warmup):
@@ -334,7 +346,8 @@ def main_gpu(args):
     achieved = kv_step / (kern_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": recorded_traffic(args.workload),
-                "kernel": "gqa_decode_kernel (persistent split-KV items)" if args.entry == "split"
+                "kernel": ("gqa_decode_kernel (equal-work ranges)" if eff_split == 0 else
+                           "gqa_decode_kernel (fixed splits)") if args.entry == "split"
                 else "gqa_decode_kernel (gqa_decode)", "peak_kind": hbm_kind,
                 "kernel_us": kern_ms * 1e3, "algorithmic_bytes_per_launch": kv_step}
 
@@ -353,7 +366,7 @@ def main_gpu(args):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": config_dict(w, inp, split if args.entry == "split" else None),
+            "data": "synthetic", "config": config_dict(w, inp, eff_split if args.entry == "split" else None),
             "frac_of_peak_hbm": value / world / hbm, "peak_hbm_gbs": hbm, "peak_kind": hbm_kind,
             "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
             "entry": "gqa_decode_split" if args.entry == "split" else "gqa_decode",
@@ -426,7 +439,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama70b")
     ap.add_argument("--entry", choices=["split", "cluster"], default="split")
     ap.add_argument("--split-tokens", type=int, default=-1,
-                    help="-1: the workload's own split (or the library's plan); 0: the library's plan")
+                    help="-1: the workload's own split (0 when it has none); 0: the library's "
+                         "equal-work ranges; > 0: fixed splits of that many tokens")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

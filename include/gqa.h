@@ -132,15 +132,24 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
  * The merge is an exact re-association of the softmax of the pages' formula
  * (the pages do not describe split-KV; it is how a long cache fills the GPU).
  *
- * split_tokens: a positive multiple of 128, or 0 to let the library choose
- *               (gqa_plan_split_tokens: no split when the (sequence, group)
- *               units already cover every SM, else about one item per SM).
+ * split_tokens: a positive multiple of 128 (fixed splits as above), or 0 to
+ *               let the library cut the work from the dims, max_seqlen and
+ *               the SM count: when max_seqlen <= 4096 and the (sequence,
+ *               group) units number at least 1.5 per SM, one split (no
+ *               combine); otherwise, for up to 1024 sequences, equal-work
+ *               ranges (stream-K): the tiles of all units, in order, are cut
+ *               into one contiguous range per resident thread block; a block
+ *               finishes the units that lie wholly in its range and leaves
+ *               partial states for the (at most two) units it shares with its
+ *               neighbours, which the second kernel merges.  Longer batches
+ *               use splits of 4096.
  * max_seqlen:   an upper bound of every seqlens[s] (sizes the grid and the
  *               workspace); a length above it is treated as invalid
  *               (GQA_STATUS_BAD_SEQLEN, row zeroed).
  * workspace:    device memory of at least gqa_decode_split_workspace_size()
- *               bytes, 16-byte aligned; its contents need no initialisation
- *               and are scratch after the call.
+ *               bytes for the same dims, max_seqlen and split_tokens, 16-byte
+ *               aligned; its contents need no initialisation and are scratch
+ *               after the call.
  */
 size_t gqa_decode_split_workspace_size(const gqa_dims *dims, int32_t max_seqlen,
                                        int32_t split_tokens);
@@ -157,15 +166,20 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache,
  * workspace; gqa_split_combine merges them into `out`.  Running the first and
  * then the second on one stream is exactly gqa_decode_split.  The combine is
  * also the merge step for partial states produced elsewhere (e.g. gathered
- * from other GPUs into this workspace).  split_tokens must be given (not 0).
+ * from other GPUs into this workspace).  Both calls must get the same dims,
+ * split_tokens and max_seqlen, on the same device.  When split_tokens == 0
+ * selects equal-work ranges, the workspace starts with a 256-byte header and
+ * one record per (sequence, group) unit, written by gqa_split_partials and
+ * read by gqa_split_combine, and `out` must be given to gqa_split_partials
+ * (units that one block covers whole are written there directly).
  *
  * out (gqa_split_partials, may be NULL): a sequence that fits in one split is
  * finished by the partials kernel itself, which writes its rows to `out` and
  * marks split 0 so that the combine leaves them alone.  With out == NULL every
  * row goes through the workspace and the combine.
  *
- * Workspace layout (fp32, each array 256-byte aligned, S = ceil(max_seqlen /
- * split_tokens)): o [b, H, S, d] unnormalised sum_j 2^(x_j - m) v_j;
+ * Workspace layout for fixed splits (fp32, each array 256-byte aligned,
+ * S = ceil(max_seqlen / split_tokens)): o [b, H, S, d] unnormalised sum_j 2^(x_j - m) v_j;
  * m [b, H, S] running maximum of x_j = scale * log2(e) * q.k_j;
  * l [b, H, S] sum_j 2^(x_j - m), or a marker: -1 the split met an invalid page
  * id; -2 (split 0) the length is outside [1, capacity]; -3 (split 0) the row
@@ -184,10 +198,10 @@ int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims,
                       const void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * The split length gqa_decode_split uses when split_tokens == 0: enough
- * (split, group, sequence) blocks to keep every SM busy, in multiples of 128
- * tokens.  num_sms <= 0 queries the current device.  Returns a positive
- * multiple of 128, or a GQA_ERR_* code.
+ * The decomposition gqa_decode_split (and the pair gqa_split_partials /
+ * gqa_split_combine) uses when split_tokens == 0: 0 for equal-work ranges, or
+ * the fixed split length (a positive multiple of 128) it falls back to.
+ * num_sms <= 0 queries the current device.  A negative value is a GQA_ERR_* code.
  */
 int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms);
 

@@ -25,6 +25,9 @@ using gqa::Mode;
 
 constexpr int kMaxDevices = 64;
 constexpr int kSplitQuantum = 128;  // split_tokens granularity (a multiple of every tile)
+constexpr int kMaxBalancedBlocks = 512;   // decode blocks of the balanced mode (workspace bound)
+constexpr int kMaxBalancedBatch = 1024;   // longer batches use fixed splits
+constexpr int kFallbackSplit = 4096;      // the fixed split used then
 
 // ------------------------------------------------------------------ device info
 struct DeviceInfo {
@@ -159,20 +162,6 @@ Workspace workspace_layout(const Shape &sh, int num_splits) {
   return w;
 }
 
-// Split length when the caller leaves it to the library.  Blocks of a few
-// thousand tokens stream at the best per-block rate; the split is the longest
-// one (at most 4096 tokens) that still gives about 1.5 items per SM, in
-// multiples of 128 tokens.
-int split_plan(const Shape &sh, int sms, int max_seqlen) {
-  const long long units = static_cast<long long>(sh.b) * sh.G;
-  const long long want_items = (3ll * sms + 1) / 2;
-  long long splits = std::max<long long>((want_items + units - 1) / units, (max_seqlen + 4095) / 4096);
-  splits = std::max<long long>(1, std::min<long long>(splits, (max_seqlen + kSplitQuantum - 1) / kSplitQuantum));
-  long long tokens = (max_seqlen + splits - 1) / splits;
-  tokens = (tokens + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
-  return static_cast<int>(std::max<long long>(kSplitQuantum, tokens));
-}
-
 // Blocks per cluster for gqa_decode: 1 (one block per (sequence, group)
 // unit) when the units give about 1.5 blocks per SM; otherwise the smallest
 // power of two (at most 16) that does, never more blocks than 128-token tiles.
@@ -203,13 +192,30 @@ struct Launch {
 };
 
 template <int D, int NT, int NHB, int STAGES, bool PAGED, Mode MODE>
-int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p, const Launch &l) {
+int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p, Launch l) {
   constexpr int CH = (D == 64) ? 2 : 1;
-  using TL = gqa::Tile<D, NT, NHB, CH, STAGES>;
+  using TL = gqa::Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBalanced>;
   auto kernel = gqa::gqa_decode_kernel<D, NT, NHB, CH, STAGES, PAGED, MODE>;
   const int smem = TL::kSmemBytes;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return GQA_ERR_CUDA;
+  if (MODE == Mode::kBalanced) {
+    // one block per resident slot of the GPU: grid.x holds the SM count on
+    // entry and becomes SMs x blocks per SM (capped by the workspace)
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, TL::kThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+      return GQA_ERR_CUDA;
+    l.grid.x = std::min<unsigned>(l.grid.x * per_sm, kMaxBalancedBlocks);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = l.grid;
+    cfg.blockDim = dim3(TL::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = l.stream;
+    cfg.numAttrs = 0;
+    if (cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) != cudaSuccess) return GQA_ERR_CUDA;
+    return static_cast<int>(l.grid.x);  // > 0: the number of decode blocks
+  }
   if (MODE == Mode::kCluster && l.cluster > 8) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       return GQA_ERR_CUDA;
@@ -320,6 +326,115 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   return launch_decode<Mode::kItems>(sh, tk, tv, p, l);
 }
 
+// ------------------------------------------------------------------ balanced mode
+// Workspace: a 256-byte header {decode blocks, capacity, total tiles} and one
+// record per (sequence, group) unit {first block, last block, slot}, both
+// written by the decode kernel for the combine, then the partial states
+// o [blocks][2][r][d], m and l [blocks][2][r].
+struct BalancedWorkspace {
+  size_t meta_off, o_off, m_off, l_off, total;
+};
+
+BalancedWorkspace balanced_layout(const Shape &sh) {
+  BalancedWorkspace w;
+  const size_t rows = static_cast<size_t>(kMaxBalancedBlocks) * 2 * sh.r;
+  w.meta_off = 256;
+  w.o_off = w.meta_off + round256(static_cast<size_t>(sh.b) * sh.G * 16);
+  w.m_off = w.o_off + round256(rows * sh.D * sizeof(float));
+  w.l_off = w.m_off + round256(rows * sizeof(float));
+  w.total = w.l_off + round256(rows * sizeof(float));
+  return w;
+}
+
+size_t auto_workspace_bytes(const Shape &sh, int max_seqlen) {
+  const int splits = (max_seqlen + kFallbackSplit - 1) / kFallbackSplit;
+  return std::max(balanced_layout(sh).total, workspace_layout(sh, splits).total);
+}
+
+int run_balanced_decode(const Shape &sh, int sms, const void *q, const void *k, const void *v,
+                        const int32_t *seqlens, const int32_t *pt, float *out, float scale,
+                        uint32_t *status, int32_t max_seqlen, void *workspace, cudaStream_t stream) {
+  CUtensorMap tk, tv;
+  int rc = encode_maps(sh, k, v, &tk, &tv);
+  if (rc != GQA_OK) return rc;
+  const BalancedWorkspace ws = balanced_layout(sh);
+  uint8_t *w = static_cast<uint8_t *>(workspace);
+  DecodeParams p = base_params(sh, q, seqlens, pt, status, scale);
+  p.out = out;
+  p.ws_header = reinterpret_cast<int *>(w);
+  p.ws_meta = reinterpret_cast<int4 *>(w + ws.meta_off);
+  p.part_o = reinterpret_cast<float *>(w + ws.o_off);
+  p.part_m = reinterpret_cast<float *>(w + ws.m_off);
+  p.part_l = reinterpret_cast<float *>(w + ws.l_off);
+  p.capacity = static_cast<int>(std::min<long long>(sh.capacity, max_seqlen));
+  p.b = sh.b;
+  Launch l{dim3(static_cast<unsigned>(sms), 1, 1), 1, stream};
+  rc = launch_decode<Mode::kBalanced>(sh, tk, tv, p, l);
+  return rc < 0 ? rc : GQA_OK;
+}
+
+int run_balanced_combine(const Shape &sh, const int32_t *seqlens, float *out, uint32_t *status,
+                         const void *workspace, cudaStream_t stream) {
+  const BalancedWorkspace ws = balanced_layout(sh);
+  const uint8_t *w = static_cast<const uint8_t *>(workspace);
+  CombineParams c{};
+  c.seqlens = seqlens;
+  c.out = out;
+  c.ws_header = reinterpret_cast<const int *>(w);
+  c.ws_meta = reinterpret_cast<const int4 *>(w + ws.meta_off);
+  c.part_o = reinterpret_cast<const float *>(w + ws.o_off);
+  c.part_m = reinterpret_cast<const float *>(w + ws.m_off);
+  c.part_l = reinterpret_cast<const float *>(w + ws.l_off);
+  c.status = status;
+  c.b = sh.b;
+  c.H = sh.H;
+  c.G = sh.G;
+  c.r = sh.r;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sh.b * sh.H), 1, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = sh.D == 128 ? cudaLaunchKernelEx(&cfg, gqa::gqa_combine_balanced_kernel<128, 64>, c)
+                              : cudaLaunchKernelEx(&cfg, gqa::gqa_combine_balanced_kernel<64, 128>, c);
+  return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+// split_tokens == 0 in the split API: the library's choice, made from the
+// dims, max_seqlen and the SM count only, so that gqa_split_partials and
+// gqa_split_combine make the same one.  Uniform work that already gives every
+// SM 1.5 blocks of at most 4096 tokens runs one block per (sequence, group) with
+// no combine; everything else runs equal-work ranges (fixed 4096-token splits
+// for batches too long to scan in every block).
+struct AutoChoice {
+  bool balanced;
+  int split_tokens;
+};
+
+AutoChoice choose_auto(const Shape &sh, int max_seqlen, int sms) {
+  const long long units = static_cast<long long>(sh.b) * sh.G;
+  if (max_seqlen <= kFallbackSplit && 2 * units >= 3ll * sms)
+    return {false, (max_seqlen + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum};
+  if (sh.b <= kMaxBalancedBatch) return {true, 0};
+  return {false, kFallbackSplit};
+}
+
+// split_tokens == 0 in the split API: checks shared by its entry points.
+int prepare_auto(const gqa_dims *dims, bool paged, int32_t max_seqlen, const void *workspace,
+                 size_t workspace_bytes, Shape *sh) {
+  int rc = check_dims(dims, paged, sh);
+  if (rc != GQA_OK) return rc;
+  if (max_seqlen < 1) return GQA_ERR_DIMS;
+  if (!workspace) return GQA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
+  if (workspace_bytes < auto_workspace_bytes(*sh, max_seqlen)) return GQA_ERR_WORKSPACE;
+  return GQA_OK;
+}
+
 struct SplitArgs {
   Shape sh;
   int split_tokens, num_splits;
@@ -331,11 +446,8 @@ int prepare_split(const gqa_dims *dims, bool paged, int32_t split_tokens, int32_
   int rc = check_dims(dims, paged, &out->sh);
   if (rc != GQA_OK) return rc;
   if (max_seqlen < 1) return GQA_ERR_DIMS;
-  if (split_tokens < 0 || split_tokens % kSplitQuantum != 0) return GQA_ERR_SPLIT;
-  if (split_tokens == 0) {
-    if (sms <= 0) return GQA_ERR_SPLIT;
-    split_tokens = split_plan(out->sh, sms, max_seqlen);
-  }
+  if (split_tokens <= 0 || split_tokens % kSplitQuantum != 0) return GQA_ERR_SPLIT;
+  (void)sms;
   out->split_tokens = split_tokens;
   out->num_splits = (max_seqlen + split_tokens - 1) / split_tokens;
   if (out->num_splits > 65535) return GQA_ERR_SPLIT;
@@ -372,9 +484,8 @@ int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t
   c.split_tokens = a.split_tokens;
   c.num_splits = a.num_splits;
   const int rows = a.sh.b * a.sh.H;
-  const int rpb = 128 / (a.sh.D / 4);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((rows + rpb - 1) / rpb, 1, 1);
+  cfg.gridDim = dim3(rows, 1, 1);
   cfg.blockDim = dim3(128, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -445,7 +556,7 @@ size_t gqa_decode_split_workspace_size(const gqa_dims *dims, int32_t max_seqlen,
   Shape sh;  // only b, H and d matter here
   if (!dims || check_dims(dims, false, &sh) != GQA_OK) return 0;
   if (max_seqlen < 1 || split_tokens < 0 || split_tokens % kSplitQuantum != 0) return 0;
-  if (split_tokens == 0) split_tokens = kSplitQuantum;  // the smallest split bounds every plan
+  if (split_tokens == 0) return auto_workspace_bytes(sh, max_seqlen);
   const int splits = (max_seqlen + split_tokens - 1) / split_tokens;
   return workspace_layout(sh, splits).total;
 }
@@ -461,7 +572,8 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
     num_sms = dev.sms;
   }
-  return split_plan(sh, num_sms, max_seqlen);
+  const AutoChoice ch = choose_auto(sh, max_seqlen, num_sms);
+  return ch.balanced ? 0 : ch.split_tokens;
 }
 
 int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
@@ -472,7 +584,21 @@ int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
   if (rc != GQA_OK) return rc;
   if (out && !aligned16(out)) return GQA_ERR_MISALIGNED;
   if (!std::isfinite(scale)) return GQA_ERR_DIMS;
-  if (split_tokens == 0) return GQA_ERR_SPLIT;  // the combine must be given the same split
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (split_tokens == 0) {
+    Shape sh;
+    if ((rc = prepare_auto(dims, page_table != nullptr, max_seqlen, workspace, workspace_bytes, &sh)) != GQA_OK)
+      return rc;
+    DeviceInfo dev;
+    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+    const AutoChoice ch = choose_auto(sh, max_seqlen, dev.sms);
+    if (ch.balanced) {
+      if (!out) return GQA_ERR_NULL_POINTER;  // whole units are finished straight into out
+      return run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale,
+                                 status, max_seqlen, workspace, st);
+    }
+    split_tokens = ch.split_tokens;
+  }
   SplitArgs a;
   rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace, workspace_bytes,
                      0, &a);
@@ -480,7 +606,7 @@ int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
   return run_partials(a, q, k_cache, v_cache, seqlens, page_table, out, scale, status, max_seqlen,
-                      workspace, static_cast<cudaStream_t>(stream));
+                      workspace, st);
 }
 
 int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims, uint32_t *status,
@@ -490,13 +616,23 @@ int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims, 
   if (!aligned16(out)) return GQA_ERR_MISALIGNED;
   if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(status) & 3u))
     return GQA_ERR_MISALIGNED;
-  if (split_tokens == 0) return GQA_ERR_SPLIT;  // the combine must know the split actually used
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc;
+  if (split_tokens == 0) {
+    Shape sh;  // the merge needs b, H, G and d only
+    if ((rc = prepare_auto(dims, false, max_seqlen, workspace, workspace_bytes, &sh)) != GQA_OK) return rc;
+    DeviceInfo dev;
+    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+    const AutoChoice ch = choose_auto(sh, max_seqlen, dev.sms);
+    if (ch.balanced) return run_balanced_combine(sh, seqlens, out, status, workspace, st);
+    split_tokens = ch.split_tokens;
+  }
   SplitArgs a;  // the merge needs b, H, d and the split geometry only
-  int rc = prepare_split(dims, false, split_tokens, max_seqlen, workspace, workspace_bytes, 0, &a);
+  rc = prepare_split(dims, false, split_tokens, max_seqlen, workspace, workspace_bytes, 0, &a);
   if (rc != GQA_OK) return rc;
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-  return run_combine(a, seqlens, out, status, max_seqlen, workspace, static_cast<cudaStream_t>(stream));
+  return run_combine(a, seqlens, out, status, max_seqlen, workspace, st);
 }
 
 int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
@@ -508,21 +644,28 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, co
   if (!out) return GQA_ERR_NULL_POINTER;
   if (!aligned16(out)) return GQA_ERR_MISALIGNED;
   if (!std::isfinite(scale)) return GQA_ERR_DIMS;
-  int sms = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (split_tokens == 0) {
-    Shape tmp;
-    if ((rc = check_dims(dims, page_table != nullptr, &tmp)) != GQA_OK) return rc;
+    Shape sh;
+    if ((rc = prepare_auto(dims, page_table != nullptr, max_seqlen, workspace, workspace_bytes, &sh)) != GQA_OK)
+      return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    sms = dev.sms;
+    const AutoChoice ch = choose_auto(sh, max_seqlen, dev.sms);
+    if (ch.balanced) {
+      rc = run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale, status,
+                               max_seqlen, workspace, st);
+      if (rc != GQA_OK) return rc;
+      return run_balanced_combine(sh, seqlens, out, status, workspace, st);
+    }
+    split_tokens = ch.split_tokens;
   }
   SplitArgs a;
   rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace,
-                     workspace_bytes, sms, &a);
+                     workspace_bytes, 0, &a);
   if (rc != GQA_OK) return rc;
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   rc = run_partials(a, q, k_cache, v_cache, seqlens, page_table, out, scale, status, max_seqlen,
                     workspace, st);
   if (rc != GQA_OK || a.num_splits == 1) return rc;  // one split: rows are final already

@@ -55,7 +55,12 @@ constexpr float kLFinal = -3.f;      // split 0: the only split already wrote th
 // kItems: one block per (sequence, group, split) item, blockIdx.x = item.
 // kCluster: one block per cluster rank; the blocks of a cluster share one
 // (sequence, group) and merge through distributed shared memory.
-enum class Mode { kItems, kCluster };
+// kBalanced: stream-K.  The tiles of all (sequence, group) units, in that
+// order, form one sequence that is cut into gridDim.x equal contiguous ranges;
+// a block streams its range through one pipeline, finishing the units that lie
+// wholly inside it and leaving partial states for the (at most two) units it
+// shares with its neighbours.
+enum class Mode { kItems, kCluster, kBalanced };
 
 struct DecodeParams {
   const __nv_bfloat16 *q;     // [b, H, D]
@@ -66,6 +71,8 @@ struct DecodeParams {
   float *part_m;              // [b, H, S]
   float *part_l;              // [b, H, S]
   uint32_t *status;           // optional
+  int *ws_header;             // balanced mode: {decode blocks, capacity, W lo, W hi} for the combine
+  int4 *ws_meta;              // balanced mode: per unit {first block, last block, slot in first block}
   int H, G, r;                // query heads, KV groups, heads per group
   int page_size;              // paged: tokens per page; contiguous: capacity m
   int num_pages;              // paged: pages in the pool
@@ -73,6 +80,7 @@ struct DecodeParams {
   int capacity;               // largest valid length
   int split_tokens;           // items mode: tokens per split
   int num_splits;             // items mode: S
+  int b;                      // sequences
   float scale_log2;           // scale * log2(e)
 };
 
@@ -84,9 +92,12 @@ struct CombineParams {
   const float *part_l;
   uint32_t *status;
   int b, H, max_len, split_tokens, num_splits;
+  int G, r;                   // balanced mode
+  const int *ws_header;       // balanced mode: {decode blocks, capacity, W lo, W hi}
+  const int4 *ws_meta;        // balanced mode: per unit {first block, last block, slot in first block}
 };
 
-template <int D, int NT, int NHB, int CH, int STAGES>
+template <int D, int NT, int NHB, int CH, int STAGES, bool BAL = false>
 struct Tile {
   static constexpr int kNWT = 4;                   // consumer warps along the token axis
   static constexpr int kHB = 8 * NT;               // query heads per consumer warp
@@ -100,20 +111,24 @@ struct Tile {
   static constexpr int kSteps = D / 16;            // k-steps of q.k, m-tiles of p.v
   static constexpr int kRPad = NHB * kHB;          // heads per block, padded
   static constexpr int kOStride = D + 4;           // padded merge row (floats)
-  static constexpr int kQBytes = kRPad * D * 2;    // the group's q block
-  // Shared memory (after 1 KiB alignment): ring | q block | per-warp m, l and
-  // per-head M, L | mbarriers | flags.  The merge of the output accumulators
-  // reuses the ring once every tile has been consumed.
-  static constexpr int kQOff = kRingBytes;
-  static constexpr int kMLOff = kQOff + kQBytes;
+  static constexpr int kQBytes = kRPad * D * 2;    // one q block
+  static constexpr int kQSlots = BAL ? 2 : 1;      // double-buffered when pieces follow each other
+  // Shared memory (after 1 KiB alignment): ring | [merge rows, balanced mode] |
+  // q slots | per-warp m, l and per-head M, L | mbarriers | flags.  With one
+  // piece per block the merge of the output accumulators reuses the ring once
+  // every tile has been consumed; in balanced mode the ring is already taking
+  // the next piece, so the merge rows have their own space.
+  static constexpr int kOSumOff = BAL ? kRingBytes : 0;
+  static constexpr int kQOff = kRingBytes + (BAL ? kRPad * kOStride * 4 : 0);
+  static constexpr int kMLOff = kQOff + kQSlots * kQBytes;
   static constexpr int kMLFloats = 2 * kNC * kHB + 2 * kRPad;
   static constexpr int kBarOff = (kMLOff + 4 * kMLFloats + 7) & ~7;
-  static constexpr int kNumBars = 2 * STAGES + 1;  // full, empty, q
+  static constexpr int kNumBars = 2 * STAGES + 2 * kQSlots;  // full, empty, q full, q empty
   static constexpr int kFlagOff = kBarOff + 8 * kNumBars;
   static constexpr int kNumFlags = STAGES + 2;     // bad tile per stage, abort, item bad
   static constexpr int kSmemBytes = 1024 + kFlagOff + 4 * kNumFlags;
   static constexpr int kMinBlocks = STAGES <= 2 ? 3 : (STAGES == 3 ? 2 : 1);
-  static_assert(kRPad * kOStride * 4 <= kRingBytes, "merge rows must fit in the ring");
+  static_assert(BAL || kRPad * kOStride * 4 <= kRingBytes, "merge rows must fit in the ring");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -130,15 +145,20 @@ __device__ __forceinline__ uint32_t keep_halves(uint32_t v, bool keep_lo, bool k
   return (keep_lo ? (v & 0x0000ffffu) : 0u) | (keep_hi ? (v & 0xffff0000u) : 0u);
 }
 
-// One unit of work: the token range [t_begin, t_end) of KV group g of sequence s.
-struct Item {
-  int s, g, k, len, t_begin, t_end;
+// One piece of work: the token range [t_begin, t_end) of KV group g of
+// sequence s, and where its result goes.
+struct Piece {
+  int s, g, len, k, t_begin, t_end;
   bool len_ok;
+  bool final_row;      // balanced mode: the piece is the whole unit
+  int slot;            // balanced mode: partial-state slot (2 per block)
+  bool first_of_unit;  // balanced mode: the piece starts at the unit's first tile
+  int last_block;      // balanced mode (first_of_unit): last block holding a tile of the unit
 };
 
 template <int T, Mode MODE>
-__device__ __forceinline__ Item make_item(const DecodeParams &p) {
-  Item it;
+__device__ __forceinline__ Piece make_item(const DecodeParams &p) {
+  Piece it;
   if (MODE == Mode::kItems) {
     const int i = blockIdx.x;
     it.k = i % p.num_splits;
@@ -154,6 +174,10 @@ __device__ __forceinline__ Item make_item(const DecodeParams &p) {
   it.len_ok = it.len >= 1 && it.len <= p.capacity;
   it.t_begin = 0;
   it.t_end = 0;
+  it.final_row = false;
+  it.slot = 0;
+  it.first_of_unit = false;
+  it.last_block = 0;
   if (it.len_ok) {
     if (MODE == Mode::kItems) {
       it.t_begin = it.k * p.split_tokens;
@@ -168,46 +192,164 @@ __device__ __forceinline__ Item make_item(const DecodeParams &p) {
   return it;
 }
 
+// Tiles of each (sequence, group) unit of sequence s; 0 for an invalid length.
+template <int T>
+__device__ __forceinline__ int unit_tiles(const int32_t *seqlens, int capacity, int s, int *len_out) {
+  const int len = __ldg(seqlens + s);
+  *len_out = len;
+  return (len >= 1 && len <= capacity) ? (len + T - 1) / T : 0;
+}
+
+__device__ __forceinline__ long long warp_sum64(long long v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// Total tiles of all units, and the position of global tile `start` in the
+// unit order (sequence-major, group-minor).  Every lane of the warp calls it
+// and gets the same answer.
+template <int T>
+__device__ __forceinline__ long long total_tiles(const int32_t *seqlens, int b, int G, int capacity,
+                                                 int lane) {
+  long long tot = 0;
+  for (int base = 0; base < b; base += 32) {
+    const int s = base + lane;
+    int len;
+    tot += (s < b) ? unit_tiles<T>(seqlens, capacity, s, &len) : 0;
+  }
+  return warp_sum64(tot) * G;
+}
+
+// Walks the pieces of this block's range in balanced mode.
+struct Walker {
+  long long remaining;  // tiles of the range not handed out yet
+  long long pos;        // global index of the next tile handed out
+  long long W;          // tiles of all units
+  int s, g, tile_in, tiles_s, len_s, count;
+};
+
+template <int T>
+__device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, int lane) {
+  const long long W = total_tiles<T>(p.seqlens, p.b, p.G, p.capacity, lane);
+  const long long N = gridDim.x, c = blockIdx.x;
+  const long long start = c * W / N;
+  wk.remaining = (c + 1) * W / N - start;
+  wk.pos = start;
+  wk.W = W;
+  wk.s = wk.g = wk.tile_in = wk.tiles_s = wk.len_s = wk.count = 0;
+  if (wk.remaining <= 0) {
+    wk.remaining = 0;
+    return;
+  }
+  long long acc = 0;
+  for (int base = 0; base < p.b; base += 32) {
+    const int s = base + lane;
+    int len = 0;
+    const long long t = (s < p.b) ? static_cast<long long>(unit_tiles<T>(p.seqlens, p.capacity, s, &len)) * p.G : 0;
+    long long inc = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long v = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += v;
+    }
+    const long long chunk = __shfl_sync(0xffffffffu, inc, 31);
+    if (start < acc + chunk) {
+      const unsigned hit = __ballot_sync(0xffffffffu, start < acc + inc);
+      const int L = __ffs(hit) - 1;
+      const long long before = acc + __shfl_sync(0xffffffffu, inc - t, L);
+      wk.s = base + L;
+      wk.len_s = __shfl_sync(0xffffffffu, len, L);
+      wk.tiles_s = (wk.len_s + T - 1) / T;
+      const long long in_seq = start - before;
+      wk.g = static_cast<int>(in_seq / wk.tiles_s);
+      wk.tile_in = static_cast<int>(in_seq % wk.tiles_s);
+      return;
+    }
+    acc += chunk;
+  }
+  wk.remaining = 0;  // not reached: start < W
+}
+
+template <int T>
+__device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, Piece &pc) {
+  if (wk.remaining <= 0) return false;
+  const int take = static_cast<int>(min(static_cast<long long>(wk.tiles_s - wk.tile_in), wk.remaining));
+  pc.s = wk.s;
+  pc.g = wk.g;
+  pc.k = 0;
+  pc.len = wk.len_s;
+  pc.len_ok = true;
+  pc.t_begin = wk.tile_in * T;
+  pc.t_end = min(wk.len_s, (wk.tile_in + take) * T);
+  pc.final_row = (wk.tile_in == 0 && take == wk.tiles_s);
+  pc.slot = 2 * static_cast<int>(blockIdx.x) + (wk.count == 0 ? 0 : 1);
+  // the block that holds a unit's first tile records which blocks share it
+  pc.first_of_unit = (wk.tile_in == 0);
+  if (pc.first_of_unit) {
+    const long long N = gridDim.x;
+    pc.last_block = static_cast<int>(((wk.pos + wk.tiles_s) * N - 1) / wk.W);
+  }
+  ++wk.count;
+  wk.pos += take;
+  wk.remaining -= take;
+  wk.tile_in = 0;
+  if (wk.remaining > 0) {
+    do {
+      if (++wk.g == p.G) {
+        wk.g = 0;
+        ++wk.s;
+        wk.tiles_s = unit_tiles<T>(p.seqlens, p.capacity, wk.s, &wk.len_s);
+      }
+    } while (wk.tiles_s == 0);
+  }
+  return true;
+}
+
 template <int D, int NT, int NHB, int CH, int STAGES, bool PAGED, Mode MODE>
-__global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES>::kThreads,
-                                  Tile<D, NT, NHB, CH, STAGES>::kMinBlocks)
+__global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBalanced>::kThreads,
+                                  Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBalanced>::kMinBlocks)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  using TL = Tile<D, NT, NHB, CH, STAGES>;
+  constexpr bool BAL = MODE == Mode::kBalanced;
+  using TL = Tile<D, NT, NHB, CH, STAGES, BAL>;
   constexpr int T = TL::kT;
   constexpr int nc = TL::kNC;  // consumer warps
   constexpr int r_pad = TL::kRPad;
+  constexpr int QS = TL::kQSlots;
   const float kNegInf = -__int_as_float(0x7f800000);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float *osum = reinterpret_cast<float *>(smem);                  // [r_pad][kOStride], after the loop
-  const uint32_t q_sm = smem_addr(smem + TL::kQOff);              // [r][D] bf16
+  float *osum = reinterpret_cast<float *>(smem + TL::kOSumOff);   // [r_pad][kOStride]
+  const uint32_t q_sm = smem_addr(smem + TL::kQOff);              // QS x [r_pad][D] bf16
   float *m_sm = reinterpret_cast<float *>(smem + TL::kMLOff);     // [nc][kHB]
   float *l_sm = m_sm + nc * TL::kHB;                              // [nc][kHB]
   float *M_blk = l_sm + nc * TL::kHB;                             // [r_pad]
   float *L_blk = M_blk + r_pad;                                   // [r_pad]
   const uint32_t bar_full = smem_addr(smem + TL::kBarOff);
   const uint32_t bar_empty = bar_full + 8 * STAGES;
-  const uint32_t bar_q = bar_empty + 8 * STAGES;
+  const uint32_t bar_qfull = bar_empty + 8 * STAGES;
+  const uint32_t bar_qempty = bar_qfull + 8 * QS;
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TL::kFlagOff);  // [STAGES]
   volatile int *abort_flag = tile_bad + STAGES;
   volatile int *item_bad = tile_bad + STAGES + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const Item w = make_item<T, MODE>(p);
 
+  Piece pc;
+  if (!BAL) pc = make_item<T, MODE>(p);
   if (MODE == Mode::kItems) {
     if (threadIdx.x == 0) pdl_launch_dependents();
-    if (w.t_begin >= w.t_end) {
+    if (pc.t_begin >= pc.t_end) {
       // Nothing to read.  An invalid length is handled once, by split 0: zero
       // rows in `out` and a marker in split 0 for the combine.
-      if (!w.len_ok && w.k == 0) {
+      if (!pc.len_ok && pc.k == 0) {
         for (int idx = threadIdx.x; idx < p.r * (D / 4); idx += blockDim.x) {
           const int h = idx / (D / 4), c4 = idx % (D / 4);
-          const size_t row = static_cast<size_t>(w.s) * p.H + static_cast<size_t>(w.g) * p.r + h;
+          const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + h;
           if (p.out) reinterpret_cast<float4 *>(p.out + row * D)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLBadLength;
         }
@@ -216,6 +358,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES>::kThreads,
       return;
     }
   }
+  if (BAL && threadIdx.x == 0) pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -223,36 +366,67 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES>::kThreads,
       mbar_init(bar_empty + 8 * i, nc);
       tile_bad[i] = 0;
     }
-    mbar_init(bar_q, 1);
+    for (int i = 0; i < QS; ++i) {
+      mbar_init(bar_qfull + 8 * i, 1);
+      mbar_init(bar_qempty + 8 * i, nc);
+    }
     *abort_flag = 0;
     *item_bad = 0;
     fence_mbarrier_init();
   }
   __syncthreads();
-  const int ntiles = w.t_end > w.t_begin ? (w.t_end - w.t_begin + T - 1) / T : 0;
+
+  // Every warp walks the same sequence of pieces.
+  Walker wk;
+  bool have;
+  if (BAL) {
+    walker_init<T>(wk, p, lane);
+    have = walker_next<T>(wk, p, pc);
+  } else {
+    have = pc.t_begin < pc.t_end;
+  }
 
   if (warp == nc) {
     // =================================================================== producer
-    if (ntiles > 0) {
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-        const uint32_t q_bytes = static_cast<uint32_t>(p.r * D * 2);
-        mbar_arrive_expect_tx(bar_q, q_bytes);
-        bulk_load(q_sm, p.q + (static_cast<size_t>(w.s) * p.H + static_cast<size_t>(w.g) * p.r) * D,
-                  q_bytes, bar_q);
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    const uint64_t policy = l2_policy_evict_first();
+    const int P = p.page_size;
+    const int ppt = PAGED ? max(1, T / P) : 1;  // pages per tile
+    const int br = PAGED ? min(P, T) : T;        // rows per TMA box
+    const uint32_t box_bytes = static_cast<uint32_t>(TL::kHalves * br * 128);
+    const uint32_t q_bytes = static_cast<uint32_t>(p.r * D * 2);
+    int tile = 0;  // tiles issued (ring position)
+    int n = 0;     // pieces started (q slot position)
+    while (have) {
+      // ---- q block of the piece's group
+      const int qs = n % QS;
+      if (n >= QS) {
+        bool ok = mbar_wait(bar_qempty + 8 * qs, ((n / QS) - 1) & 1);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok || *abort_flag) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            if (p.status) atomicOr(p.status, kStatusTimeout);
+          }
+          break;
+        }
       }
-      const uint64_t policy = l2_policy_evict_first();
-      const int P = p.page_size;
-      const int ppt = PAGED ? max(1, T / P) : 1;  // pages per tile
-      const int br = PAGED ? min(P, T) : T;        // rows per TMA box
-      const uint32_t box_bytes = static_cast<uint32_t>(TL::kHalves * br * 128);
-      const int32_t *pt_row = PAGED ? p.page_table + static_cast<size_t>(w.s) * p.max_pages : nullptr;
-      const int lp_end = PAGED ? (w.t_end + P - 1) / P : 0;  // logical pages holding tokens < t_end
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_qfull + 8 * qs, q_bytes);
+        bulk_load(q_sm + qs * TL::kQBytes,
+                  p.q + (static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r) * D, q_bytes,
+                  bar_qfull + 8 * qs);
+      }
+      ++n;
+      // ---- K/V tiles
+      const int32_t *pt_row = PAGED ? p.page_table + static_cast<size_t>(pc.s) * p.max_pages : nullptr;
+      const int lp_end = PAGED ? (pc.t_end + P - 1) / P : 0;  // logical pages holding tokens < t_end
       int cur_w = -1, nxt_w = -1, win = -1, nxt = -1;
-      int tile = 0;
-      for (; tile < ntiles; ++tile) {
-        const int t0 = w.t_begin + tile * T;
+      bool stop = false;
+      for (int t0 = pc.t_begin; t0 < pc.t_end; t0 += T, ++tile) {
         const int stage = tile % STAGES;
         const uint32_t full = bar_full + 8 * stage;
         if (tile >= STAGES) {
@@ -263,6 +437,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES>::kThreads,
               *abort_flag = 1;
               if (p.status) atomicOr(p.status, kStatusTimeout);
             }
+            stop = true;
             break;
           }
         }
@@ -296,28 +471,30 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES>::kThreads,
             const uint32_t off = static_cast<uint32_t>(lane * br * 128);
 #pragma unroll
             for (int h = 0; h < TL::kHalves; ++h) {
-              tma_load_4d(dst_k + h * T * 128 + off, &tm_k, full, h * 64, row, w.g, id, policy);
-              tma_load_4d(dst_v + h * T * 128 + off, &tm_v, full, h * 64, row, w.g, id, policy);
+              tma_load_4d(dst_k + h * T * 128 + off, &tm_k, full, h * 64, row, pc.g, id, policy);
+              tma_load_4d(dst_v + h * T * 128 + off, &tm_v, full, h * 64, row, pc.g, id, policy);
             }
           }
         } else if (lane == 0) {
           mbar_arrive_expect_tx(full, 2u * box_bytes);
 #pragma unroll
           for (int h = 0; h < TL::kHalves; ++h) {
-            tma_load_4d(dst_k + h * T * 128, &tm_k, full, h * 64, t0, w.g, w.s, policy);
-            tma_load_4d(dst_v + h * T * 128, &tm_v, full, h * 64, t0, w.g, w.s, policy);
+            tma_load_4d(dst_k + h * T * 128, &tm_k, full, h * 64, t0, pc.g, pc.s, policy);
+            tma_load_4d(dst_v + h * T * 128, &tm_v, full, h * 64, t0, pc.g, pc.s, policy);
           }
         }
       }
-      // Never leave with copies in flight: wait (bounded) for the last tiles
-      // and the q block; on the normal path these phases completed long ago.
-      if (lane == 0) {
-        for (int t = max(0, tile - STAGES); t < tile; ++t)
-          (void)mbar_wait(bar_full + 8 * (t % STAGES), (t / STAGES) & 1);
-        (void)mbar_wait(bar_q, 0);
-      }
+      if (stop || !BAL) break;
+      have = walker_next<T>(wk, p, pc);
     }
-  } else if (ntiles > 0) {
+    // Never leave with copies in flight: wait (bounded) for the last tiles and
+    // q blocks issued; on the normal path these phases completed long ago.
+    if (lane == 0) {
+      for (int t = max(0, tile - STAGES); t < tile; ++t)
+        (void)mbar_wait(bar_full + 8 * (t % STAGES), (t / STAGES) & 1);
+      for (int m = max(0, n - QS); m < n; ++m) (void)mbar_wait(bar_qfull + 8 * (m % QS), (m / QS) & 1);
+    }
+  } else {
     // =================================================================== consumers
     const int hb = warp / TL::kNWT;  // head block
     const int ws = warp % TL::kNWT;  // token slice within a tile
@@ -325,277 +502,306 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES>::kThreads,
     const int t4 = lane & 3;
     const int ctid = threadIdx.x;    // 0 .. nc*32-1
     const float sl = p.scale_log2;
-
-    // ---- q^T fragments (B operand of S^T = K q^T): head hb*kHB + j*8 + g8,
-    // dims ks*16 + 2*t4 (+1) and ks*16 + 8 + 2*t4 (+1); padding heads are 0.
-    if (!__shfl_sync(0xffffffffu, mbar_wait(bar_q, 0), 0)) {
-      if (lane == 0) {
-        *abort_flag = 1;
-        if (p.status) atomicOr(p.status, kStatusTimeout);
+    int tile = 0;
+    int n = 0;
+    if (BAL && blockIdx.x == 0 && ctid == 0) {
+      p.ws_header[0] = static_cast<int>(gridDim.x);
+      p.ws_header[1] = p.capacity;
+      p.ws_header[2] = static_cast<int>(wk.W & 0xffffffff);
+      p.ws_header[3] = static_cast<int>(wk.W >> 32);
+    }
+    if (MODE == Mode::kCluster && !have) {  // a block without tokens contributes nothing
+      for (int h = ctid; h < r_pad; h += nc * 32) {
+        M_blk[h] = kNegInf;
+        L_blk[h] = 0.f;
       }
     }
-    uint32_t bq[TL::kSteps][NT][2];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int hl = hb * TL::kHB + j * 8 + g8;
-      const bool valid = hl < p.r;
-      const uint32_t qrow = q_sm + (valid ? hl : 0) * D * 2;
-#pragma unroll
-      for (int ks = 0; ks < TL::kSteps; ++ks) {
-        bq[ks][j][0] = valid ? ld_shared_u32(qrow + (ks * 16 + 2 * t4) * 2) : 0u;
-        bq[ks][j][1] = valid ? ld_shared_u32(qrow + (ks * 16 + 8 + 2 * t4) * 2) : 0u;
-      }
-    }
-
-    float m_run[NT][2], l_run[NT][2];
-    float o[TL::kSteps][NT][4];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      m_run[j][0] = m_run[j][1] = kNegInf;
-      l_run[j][0] = l_run[j][1] = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < TL::kSteps; ++mt) o[mt][j][0] = o[mt][j][1] = o[mt][j][2] = o[mt][j][3] = 0.f;
-    }
-    int bad = 0;
-
-    for (int tile = 0; tile < ntiles && !*abort_flag; ++tile) {
-      const int t0 = w.t_begin + tile * T;
-      const int stage = tile % STAGES;
-      bool ok = mbar_wait(bar_full + 8 * stage, (tile / STAGES) & 1);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
+    while (have) {
+      // ---- q^T fragments (B operand of S^T = K q^T): head hb*kHB + j*8 + g8,
+      // dims ks*16 + 2*t4 (+1) and ks*16 + 8 + 2*t4 (+1); padding heads are 0.
+      const int qs = n % QS;
+      if (!__shfl_sync(0xffffffffu, mbar_wait(bar_qfull + 8 * qs, (n / QS) & 1), 0)) {
         if (lane == 0) {
           *abort_flag = 1;
           if (p.status) atomicOr(p.status, kStatusTimeout);
         }
-        break;
       }
-      if (PAGED) bad |= tile_bad[stage];
-      const uint32_t kbase = smem_addr(smem + stage * TL::kStageBytes);
-      const uint32_t vbase = kbase + TL::kTileBytes;
-
+      uint32_t bq[TL::kSteps][NT][2];
 #pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        const int row0 = (ws * CH + c) * 16;
-        // ---- S^T = K q^T for 16 tokens x kHB heads (two accumulator chains)
-        float sacc[NT][4], sacc2[NT][4];
+      for (int j = 0; j < NT; ++j) {
+        const int hl = hb * TL::kHB + j * 8 + g8;
+        const bool valid = hl < p.r;
+        const uint32_t qrow = q_sm + qs * TL::kQBytes + (valid ? hl : 0) * D * 2;
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
-          sacc2[j][0] = sacc2[j][1] = sacc2[j][2] = sacc2[j][3] = 0.f;
-        }
-        {
-          const int mi = lane >> 3;
-          const int row = row0 + (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-          for (int ks = 0; ks < TL::kSteps; ++ks) {
-            uint32_t a[4];
-            ldsm_x4(kbase + swz_offset<T>(row, ks * 16 + (mi >> 1) * 8), a);
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-              if (ks & 1)
-                mma_bf16_16816(sacc2[j], a, bq[ks][j][0], bq[ks][j][1]);
-              else
-                mma_bf16_16816(sacc[j], a, bq[ks][j][0], bq[ks][j][1]);
-            }
-          }
-        }
-        // ---- mask, scale, online softmax, P^T fragments
-        const int tok_a = t0 + row0 + g8;
-        const bool ok_a = tok_a < w.t_end;
-        const bool ok_b = tok_a + 8 < w.t_end;
-        uint32_t bh[NT][2], bl[NT][2];
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          const float x0 = ok_a ? (sacc[j][0] + sacc2[j][0]) * sl : kNegInf;  // token g8,   head 2*t4
-          const float x1 = ok_a ? (sacc[j][1] + sacc2[j][1]) * sl : kNegInf;  // token g8,   head 2*t4+1
-          const float x2 = ok_b ? (sacc[j][2] + sacc2[j][2]) * sl : kNegInf;  // token g8+8, head 2*t4
-          const float x3 = ok_b ? (sacc[j][3] + sacc2[j][3]) * sl : kNegInf;  // token g8+8, head 2*t4+1
-          float mx_a = fmaxf(x0, x2), mx_b = fmaxf(x1, x3);
-#pragma unroll
-          for (int off = 4; off < 32; off <<= 1) {
-            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
-            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
-          }
-          const float mn_a = fmaxf(m_run[j][0], mx_a);
-          const float mn_b = fmaxf(m_run[j][1], mx_b);
-          const float base_a = (mn_a == kNegInf) ? 0.f : mn_a;
-          const float base_b = (mn_b == kNegInf) ? 0.f : mn_b;
-          const float p0 = ex2(x0 - base_a), p1 = ex2(x1 - base_b);
-          const float p2 = ex2(x2 - base_a), p3 = ex2(x3 - base_b);
-          // rescale only when a running maximum moved (rare after the first tiles)
-          if (__any_sync(0xffffffffu, mn_a != m_run[j][0] || mn_b != m_run[j][1])) {
-            const float alpha_a = ex2(m_run[j][0] - base_a);
-            const float alpha_b = ex2(m_run[j][1] - base_b);
-            l_run[j][0] *= alpha_a;
-            l_run[j][1] *= alpha_b;
-#pragma unroll
-            for (int mt = 0; mt < TL::kSteps; ++mt) {
-              o[mt][j][0] *= alpha_a;
-              o[mt][j][1] *= alpha_b;
-              o[mt][j][2] *= alpha_a;
-              o[mt][j][3] *= alpha_b;
-            }
-          }
-          l_run[j][0] += p0 + p2;
-          l_run[j][1] += p1 + p3;
-          m_run[j][0] = mn_a;
-          m_run[j][1] = mn_b;
-          // high and residual bf16 parts, transposed into the B layout
-          bh[j][0] = movmatrix_trans(pack_bf16(p0, p1));
-          bh[j][1] = movmatrix_trans(pack_bf16(p2, p3));
-          bl[j][0] = movmatrix_trans(pack_bf16(p0 - bf16_round(p0), p1 - bf16_round(p1)));
-          bl[j][1] = movmatrix_trans(pack_bf16(p2 - bf16_round(p2), p3 - bf16_round(p3)));
-        }
-        // ---- O^T += V^T P^T
-        const bool tail = t0 + row0 + 16 > w.t_end;
-        const int tok_lo = t0 + row0 + 2 * t4;
-        const bool k0 = tok_lo < w.t_end, k1 = tok_lo + 1 < w.t_end;
-        const bool k8 = tok_lo + 8 < w.t_end, k9 = tok_lo + 9 < w.t_end;
-        {
-          const int mi = lane >> 3;
-          const int row = row0 + (mi >> 1) * 8 + (lane & 7);
-#pragma unroll
-          for (int mt = 0; mt < TL::kSteps; ++mt) {
-            uint32_t a[4];
-            ldsm_x4_trans(vbase + swz_offset<T>(row, mt * 16 + (mi & 1) * 8), a);
-            if (tail) {  // rows past the range may hold anything (even NaN): zero them
-              a[0] = keep_halves(a[0], k0, k1);
-              a[1] = keep_halves(a[1], k0, k1);
-              a[2] = keep_halves(a[2], k8, k9);
-              a[3] = keep_halves(a[3], k8, k9);
-            }
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-              mma_bf16_16816(o[mt][j], a, bh[j][0], bh[j][1]);
-              mma_bf16_16816(o[mt][j], a, bl[j][0], bl[j][1]);
-            }
-          }
+        for (int ks = 0; ks < TL::kSteps; ++ks) {
+          bq[ks][j][0] = valid ? ld_shared_u32(qrow + (ks * 16 + 2 * t4) * 2) : 0u;
+          bq[ks][j][1] = valid ? ld_shared_u32(qrow + (ks * 16 + 8 + 2 * t4) * 2) : 0u;
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_empty + 8 * stage);
-    }
+      if (lane == 0) mbar_arrive(bar_qempty + 8 * qs);
+      ++n;
 
-    // ---- merge the consumer warps of each head block (the ring is free now)
+      float m_run[NT][2], l_run[NT][2];
+      float o[TL::kSteps][NT][4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
+      for (int j = 0; j < NT; ++j) {
+        m_run[j][0] = m_run[j][1] = kNegInf;
+        l_run[j][0] = l_run[j][1] = 0.f;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1)
-          l_run[j][e] += __shfl_xor_sync(0xffffffffu, l_run[j][e], off);
+        for (int mt = 0; mt < TL::kSteps; ++mt) o[mt][j][0] = o[mt][j][1] = o[mt][j][2] = o[mt][j][3] = 0.f;
       }
-    }
-    if (g8 == 0) {
+      int bad = 0;
+
+      for (int t0 = pc.t_begin; t0 < pc.t_end && !*abort_flag; t0 += T, ++tile) {
+        const int stage = tile % STAGES;
+        bool ok = mbar_wait(bar_full + 8 * stage, (tile / STAGES) & 1);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            if (p.status) atomicOr(p.status, kStatusTimeout);
+          }
+          break;
+        }
+        if (PAGED) bad |= tile_bad[stage];
+        const uint32_t kbase = smem_addr(smem + stage * TL::kStageBytes);
+        const uint32_t vbase = kbase + TL::kTileBytes;
+
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int row0 = (ws * CH + c) * 16;
+          // ---- S^T = K q^T for 16 tokens x kHB heads (two accumulator chains)
+          float sacc[NT][4], sacc2[NT][4];
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+            sacc2[j][0] = sacc2[j][1] = sacc2[j][2] = sacc2[j][3] = 0.f;
+          }
+          {
+            const int mi = lane >> 3;
+            const int row = row0 + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int ks = 0; ks < TL::kSteps; ++ks) {
+              uint32_t a[4];
+              ldsm_x4(kbase + swz_offset<T>(row, ks * 16 + (mi >> 1) * 8), a);
+#pragma unroll
+              for (int j = 0; j < NT; ++j) {
+                if (ks & 1)
+                  mma_bf16_16816(sacc2[j], a, bq[ks][j][0], bq[ks][j][1]);
+                else
+                  mma_bf16_16816(sacc[j], a, bq[ks][j][0], bq[ks][j][1]);
+              }
+            }
+          }
+          // ---- mask, scale, online softmax, P^T fragments
+          const int tok_a = t0 + row0 + g8;
+          const bool ok_a = tok_a < pc.t_end;
+          const bool ok_b = tok_a + 8 < pc.t_end;
+          uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            const float x0 = ok_a ? (sacc[j][0] + sacc2[j][0]) * sl : kNegInf;  // token g8,   head 2*t4
+            const float x1 = ok_a ? (sacc[j][1] + sacc2[j][1]) * sl : kNegInf;  // token g8,   head 2*t4+1
+            const float x2 = ok_b ? (sacc[j][2] + sacc2[j][2]) * sl : kNegInf;  // token g8+8, head 2*t4
+            const float x3 = ok_b ? (sacc[j][3] + sacc2[j][3]) * sl : kNegInf;  // token g8+8, head 2*t4+1
+            float mx_a = fmaxf(x0, x2), mx_b = fmaxf(x1, x3);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+              mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+              mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+            }
+            const float mn_a = fmaxf(m_run[j][0], mx_a);
+            const float mn_b = fmaxf(m_run[j][1], mx_b);
+            const float base_a = (mn_a == kNegInf) ? 0.f : mn_a;
+            const float base_b = (mn_b == kNegInf) ? 0.f : mn_b;
+            const float p0 = ex2(x0 - base_a), p1 = ex2(x1 - base_b);
+            const float p2 = ex2(x2 - base_a), p3 = ex2(x3 - base_b);
+            // rescale only when a running maximum moved (rare after the first tiles)
+            if (__any_sync(0xffffffffu, mn_a != m_run[j][0] || mn_b != m_run[j][1])) {
+              const float alpha_a = ex2(m_run[j][0] - base_a);
+              const float alpha_b = ex2(m_run[j][1] - base_b);
+              l_run[j][0] *= alpha_a;
+              l_run[j][1] *= alpha_b;
+#pragma unroll
+              for (int mt = 0; mt < TL::kSteps; ++mt) {
+                o[mt][j][0] *= alpha_a;
+                o[mt][j][1] *= alpha_b;
+                o[mt][j][2] *= alpha_a;
+                o[mt][j][3] *= alpha_b;
+              }
+            }
+            l_run[j][0] += p0 + p2;
+            l_run[j][1] += p1 + p3;
+            m_run[j][0] = mn_a;
+            m_run[j][1] = mn_b;
+            // high and residual bf16 parts, transposed into the B layout
+            bh[j][0] = movmatrix_trans(pack_bf16(p0, p1));
+            bh[j][1] = movmatrix_trans(pack_bf16(p2, p3));
+            bl[j][0] = movmatrix_trans(pack_bf16(p0 - bf16_round(p0), p1 - bf16_round(p1)));
+            bl[j][1] = movmatrix_trans(pack_bf16(p2 - bf16_round(p2), p3 - bf16_round(p3)));
+          }
+          // ---- O^T += V^T P^T
+          const bool tail = t0 + row0 + 16 > pc.t_end;
+          const int tok_lo = t0 + row0 + 2 * t4;
+          const bool k0 = tok_lo < pc.t_end, k1 = tok_lo + 1 < pc.t_end;
+          const bool k8 = tok_lo + 8 < pc.t_end, k9 = tok_lo + 9 < pc.t_end;
+          {
+            const int mi = lane >> 3;
+            const int row = row0 + (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int mt = 0; mt < TL::kSteps; ++mt) {
+              uint32_t a[4];
+              ldsm_x4_trans(vbase + swz_offset<T>(row, mt * 16 + (mi & 1) * 8), a);
+              if (tail) {  // rows past the range may hold anything (even NaN): zero them
+                a[0] = keep_halves(a[0], k0, k1);
+                a[1] = keep_halves(a[1], k0, k1);
+                a[2] = keep_halves(a[2], k8, k9);
+                a[3] = keep_halves(a[3], k8, k9);
+              }
+#pragma unroll
+              for (int j = 0; j < NT; ++j) {
+                mma_bf16_16816(o[mt][j], a, bh[j][0], bh[j][1]);
+                mma_bf16_16816(o[mt][j], a, bl[j][0], bl[j][1]);
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty + 8 * stage);
+      }
+
+      // ---- merge the consumer warps of each head block
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1)
+            l_run[j][e] += __shfl_xor_sync(0xffffffffu, l_run[j][e], off);
+        }
+      }
+      if (g8 == 0) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int hl = j * 8 + 2 * t4 + e;
+            m_sm[warp * TL::kHB + hl] = m_run[j][e];
+            l_sm[warp * TL::kHB + hl] = l_run[j][e];
+          }
+        }
+      }
+      named_barrier(1, nc * 32);
+      float f[NT][2];
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int hl = j * 8 + 2 * t4 + e;
-          m_sm[warp * TL::kHB + hl] = m_run[j][e];
-          l_sm[warp * TL::kHB + hl] = l_run[j][e];
+          float M = kNegInf;
+#pragma unroll
+          for (int w2 = 0; w2 < TL::kNWT; ++w2) M = fmaxf(M, m_sm[(hb * TL::kNWT + w2) * TL::kHB + hl]);
+          f[j][e] = (M == kNegInf) ? 0.f : ex2(m_run[j][e] - M);
         }
       }
-    }
-    named_barrier(1, nc * 32);
-    float f[NT][2];
+      // deterministic accumulation: token slice 0 stores, slices 1..3 add in order
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
+      for (int step = 0; step < TL::kNWT; ++step) {
+        if (ws == step) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int hl = j * 8 + 2 * t4 + e;
-        float M = kNegInf;
+          for (int mt = 0; mt < TL::kSteps; ++mt) {
 #pragma unroll
-        for (int w2 = 0; w2 < TL::kNWT; ++w2) M = fmaxf(M, m_sm[(hb * TL::kNWT + w2) * TL::kHB + hl]);
-        f[j][e] = (M == kNegInf) ? 0.f : ex2(m_run[j][e] - M);
+            for (int j = 0; j < NT; ++j) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int dim = mt * 16 + g8 + (e >> 1) * 8;
+                const int h = hb * TL::kHB + j * 8 + 2 * t4 + (e & 1);
+                float *dst = osum + h * TL::kOStride + dim;
+                const float v = o[mt][j][e] * f[j][e & 1];
+                *dst = (step == 0) ? v : (*dst + v);
+              }
+            }
+          }
+        }
+        named_barrier(1, nc * 32);
       }
-    }
-    // deterministic accumulation: token slice 0 stores, slices 1..3 add in order
-#pragma unroll
-    for (int step = 0; step < TL::kNWT; ++step) {
-      if (ws == step) {
-#pragma unroll
-        for (int mt = 0; mt < TL::kSteps; ++mt) {
-#pragma unroll
-          for (int j = 0; j < NT; ++j) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int dim = mt * 16 + g8 + (e >> 1) * 8;
-              const int h = hb * TL::kHB + j * 8 + 2 * t4 + (e & 1);
-              float *dst = osum + h * TL::kOStride + dim;
-              const float v = o[mt][j][e] * f[j][e & 1];
-              *dst = (step == 0) ? v : (*dst + v);
+      for (int h = ctid; h < r_pad; h += nc * 32) {
+        const int hb2 = h / TL::kHB, hl = h % TL::kHB;
+        float M = kNegInf;
+        for (int w2 = 0; w2 < TL::kNWT; ++w2) M = fmaxf(M, m_sm[(hb2 * TL::kNWT + w2) * TL::kHB + hl]);
+        float L = 0.f;
+        if (M != kNegInf) {
+          for (int w2 = 0; w2 < TL::kNWT; ++w2) {
+            const int idx = (hb2 * TL::kNWT + w2) * TL::kHB + hl;
+            L += l_sm[idx] * ex2(m_sm[idx] - M);
+          }
+        }
+        M_blk[h] = M;
+        L_blk[h] = L;
+      }
+      if (MODE == Mode::kCluster && ctid == 0) *item_bad = bad;
+      named_barrier(1, nc * 32);
+
+      // ---- results of the piece
+      if (BAL && ctid == 0) {
+        if (pc.first_of_unit)
+          p.ws_meta[static_cast<size_t>(pc.s) * p.G + pc.g] =
+              make_int4(static_cast<int>(blockIdx.x), pc.last_block, pc.slot & 1, 0);
+      }
+      if (MODE != Mode::kCluster) {
+        const int n4 = D / 4;
+        bool final_row;
+        size_t pslot_base = 0;  // partial slot: index of head 0 in the m/l arrays
+        size_t pslot_stride = 1;
+        if (BAL) {
+          final_row = pc.final_row;
+          pslot_base = static_cast<size_t>(pc.slot) * p.r;
+        } else {
+          final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
+          pslot_base = (static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r) * p.num_splits + pc.k;
+          pslot_stride = p.num_splits;
+        }
+        for (int idx = ctid; idx < p.r * n4; idx += nc * 32) {
+          const int h = idx / n4, c4 = idx % n4;
+          const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + h;
+          const float4 src = *reinterpret_cast<const float4 *>(osum + h * TL::kOStride + 4 * c4);
+          if (final_row) {
+            const float L = L_blk[h];
+            float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!bad && L > 0.f) res = make_float4(src.x / L, src.y / L, src.z / L, src.w / L);
+            reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
+            if (!BAL && c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLFinal;
+          } else {
+            const size_t ps = pslot_base + static_cast<size_t>(h) * pslot_stride;
+            reinterpret_cast<float4 *>(p.part_o + ps * D)[c4] = src;
+            if (c4 == 0) {
+              p.part_m[ps] = M_blk[h];
+              p.part_l[ps] = bad ? kLBadPage : L_blk[h];
             }
           }
         }
       }
-      named_barrier(1, nc * 32);
-    }
-    for (int h = ctid; h < r_pad; h += nc * 32) {
-      const int hb2 = h / TL::kHB, hl = h % TL::kHB;
-      float M = kNegInf;
-      for (int w2 = 0; w2 < TL::kNWT; ++w2) M = fmaxf(M, m_sm[(hb2 * TL::kNWT + w2) * TL::kHB + hl]);
-      float L = 0.f;
-      if (M != kNegInf) {
-        for (int w2 = 0; w2 < TL::kNWT; ++w2) {
-          const int idx = (hb2 * TL::kNWT + w2) * TL::kHB + hl;
-          L += l_sm[idx] * ex2(m_sm[idx] - M);
-        }
-      }
-      M_blk[h] = M;
-      L_blk[h] = L;
-    }
-    if (ctid == 0) *item_bad = bad;
-    named_barrier(1, nc * 32);
-
-    if (MODE == Mode::kItems) {
-      const int n4 = D / 4;
-      const int ns = (w.len + p.split_tokens - 1) / p.split_tokens;
-      const bool final_row = (ns == 1) && p.out != nullptr;
-      for (int idx = ctid; idx < p.r * n4; idx += nc * 32) {
-        const int h = idx / n4, c4 = idx % n4;
-        const size_t row = static_cast<size_t>(w.s) * p.H + static_cast<size_t>(w.g) * p.r + h;
-        const float *src = osum + h * TL::kOStride + 4 * c4;
-        if (final_row) {
-          const float L = L_blk[h];
-          float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (!bad && L > 0.f) res = make_float4(src[0] / L, src[1] / L, src[2] / L, src[3] / L);
-          reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
-          if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLFinal;
-        } else {
-          const size_t ps = row * p.num_splits + w.k;
-          reinterpret_cast<float4 *>(p.part_o + ps * D)[c4] = make_float4(src[0], src[1], src[2], src[3]);
-          if (c4 == 0) {
-            p.part_m[ps] = M_blk[h];
-            p.part_l[ps] = bad ? kLBadPage : L_blk[h];
-          }
-        }
-      }
+      if (*abort_flag || !BAL) break;
+      have = walker_next<T>(wk, p, pc);
     }
   }
 
   if (MODE == Mode::kCluster) {
     // ---- merge the blocks of the cluster through distributed shared memory
-    if (ntiles == 0 && warp < nc) {  // a block without tokens contributes nothing
-      for (int h = threadIdx.x; h < r_pad; h += nc * 32) {
-        M_blk[h] = kNegInf;
-        L_blk[h] = 0.f;
-      }
-    }
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     if (cluster.block_rank() == 0) {
       const int nb = static_cast<int>(cluster.num_blocks());
       int bad = 0;
-      if (w.len_ok)
+      if (pc.len_ok)
         for (int c = 0; c < nb; ++c) bad |= *cluster.map_shared_rank(const_cast<int *>(item_bad), c);
       const int n4 = D / 4;
       for (int idx = threadIdx.x; idx < p.r * n4; idx += blockDim.x) {
         const int h = idx / n4, c4 = idx % n4;
         float L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (w.len_ok && !bad) {
+        if (pc.len_ok && !bad) {
           float M = kNegInf;
           for (int c = 0; c < nb; ++c) M = fmaxf(M, *cluster.map_shared_rank(M_blk + h, c));
           for (int c = 0; c < nb; ++c) {
@@ -612,72 +818,174 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES>::kThreads,
         }
         float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
         if (L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
-        const size_t row = static_cast<size_t>(w.s) * p.H + static_cast<size_t>(w.g) * p.r + h;
+        const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + h;
         reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
       }
-      if (threadIdx.x == 0 && !w.len_ok && p.status) atomicOr(p.status, kStatusBadSeqlen);
+      if (threadIdx.x == 0 && !pc.len_ok && p.status) atomicOr(p.status, kStatusBadSeqlen);
     }
     cluster.sync();
   }
 }
 
-// Merge the per-split partial states of every (sequence, head) row.  The
-// D/4 threads of a row load the split maxima and sums cooperatively (one
-// coalesced pass), reduce the maximum with warp shuffles, then accumulate the
-// rescaled partial outputs with the loads of consecutive splits in flight
-// together.
+// Merge the partial states (m_k, l_k, o_k) of one output row:
+//   M = max_k m_k,  L = sum_k l_k 2^(m_k - M),  out = sum_k o_k 2^(m_k - M) / L.
+// Built for latency: the contributions are taken in chunks of 512; for each
+// chunk every thread resolves one contribution's slot and loads its m and l
+// (all in flight together), the block reduces the maximum, each thread turns
+// its m into a weight, and then kNG groups of D/4 threads (one float4 of the
+// row each) add up the weighted o rows with precomputed addresses, several
+// loads in flight per thread.  Chunks are merged online (rescaled by
+// 2^(M_old - M_new)); the groups are summed in a fixed order, so the result is
+// deterministic.  `slot(k)` is the index of contribution k in the m/l arrays
+// (< 0: no contribution).  Any l < 0 (an invalid page) makes the row zero.
+template <int D, typename SlotFn>
+__device__ __forceinline__ void merge_row(const float *part_o, const float *part_m, const float *part_l,
+                                          int n_contrib, SlotFn slot, float4 *dst) {
+  constexpr int kTPR = D / 4;
+  constexpr int kNG = 128 / kTPR;
+  constexpr int kChunk = 512;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  __shared__ long long s_ps[kChunk];
+  __shared__ float s_w[kChunk], s_l[kChunk];
+  __shared__ float s_wmax[4];
+  __shared__ int s_wbad[4];
+  __shared__ float4 s_acc[kNG][kTPR];
+  __shared__ float s_L[kNG];
+  const int tid = threadIdx.x, grp = tid / kTPR, c4 = tid % kTPR;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  float M = kNegInf;  // running maximum (the same in every thread)
+  float L = 0.f;      // this group's running sum of l weights
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int bad = 0;
+  for (int base = 0; base < n_contrib && !bad; base += kChunk) {
+    const int cnt = min(kChunk, n_contrib - base);
+    float mx = kNegInf;
+    int bd = 0;
+    for (int i = tid; i < cnt; i += 128) {
+      const long long ps = slot(base + i);
+      s_ps[i] = ps;
+      float m = kNegInf, l = 0.f;
+      if (ps >= 0) {
+        m = part_m[ps];
+        l = part_l[ps];
+      }
+      s_w[i] = m;
+      s_l[i] = l;
+      mx = fmaxf(mx, m);
+      bd |= l < 0.f;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    bd = __any_sync(0xffffffffu, bd);
+    if (lane == 0) {
+      s_wmax[warp] = mx;
+      s_wbad[warp] = bd;
+    }
+    __syncthreads();
+    mx = fmaxf(fmaxf(s_wmax[0], s_wmax[1]), fmaxf(s_wmax[2], s_wmax[3]));
+    bad = s_wbad[0] | s_wbad[1] | s_wbad[2] | s_wbad[3];
+    if (!bad && mx != kNegInf) {
+      const float Mn = fmaxf(M, mx);
+      const float rescale = (M == kNegInf) ? 0.f : ex2(M - Mn);
+      L *= rescale;
+      acc.x *= rescale;
+      acc.y *= rescale;
+      acc.z *= rescale;
+      acc.w *= rescale;
+      M = Mn;
+      for (int i = tid; i < cnt; i += 128) s_w[i] = (s_ps[i] >= 0) ? ex2(s_w[i] - Mn) : 0.f;
+      __syncthreads();
+#pragma unroll 8
+      for (int i = grp; i < cnt; i += kNG) {
+        const long long ps = s_ps[i];
+        const float w = s_w[i];
+        if (ps >= 0) {
+          const float4 v = reinterpret_cast<const float4 *>(part_o + ps * D)[c4];
+          acc.x += v.x * w;
+          acc.y += v.y * w;
+          acc.z += v.z * w;
+          acc.w += v.w * w;
+          L += s_l[i] * w;
+        }
+      }
+    }
+    __syncthreads();  // the chunk's shared arrays are reused
+  }
+  s_acc[grp][c4] = acc;
+  if (c4 == 0) s_L[grp] = L;
+  __syncthreads();
+  if (grp == 0) {
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Lt = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNG; ++i) {
+      t.x += s_acc[i][c4].x;
+      t.y += s_acc[i][c4].y;
+      t.z += s_acc[i][c4].z;
+      t.w += s_acc[i][c4].w;
+      Lt += s_L[i];
+    }
+    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!bad && Lt > 0.f) res = make_float4(t.x / Lt, t.y / Lt, t.z / Lt, t.w / Lt);
+    *dst = res;
+  }
+}
+
+// Fixed splits: one block per (sequence, head) row merges the splits
+// k < ceil(len / split_tokens) of that row.
 template <int D>
 __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p) {
-  constexpr int kTPR = D / 4;         // threads per row (one float4 each)
-  constexpr int kRPB = 128 / kTPR;    // rows per block
-  const float kNegInf = -__int_as_float(0x7f800000);
-  const int row = blockIdx.x * kRPB + threadIdx.x / kTPR;
-  const int c4 = threadIdx.x % kTPR;
-  const unsigned mask = (kTPR == 32) ? 0xffffffffu : (0xffffu << (threadIdx.x & 16));
-  if (row >= p.b * p.H) return;  // whole row groups leave together
+  const int row = blockIdx.x;
   const int s = row / p.H;
   const int len = __ldg(p.seqlens + s);
+  float4 *dst = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D) + threadIdx.x % (D / 4);
   pdl_wait_primary();  // the partial states below come from the preceding kernel
-  float4 *dst = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D) + c4;
   if (len < 1 || len > p.max_len) {
-    *dst = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (c4 == 0 && p.status) atomicOr(p.status, kStatusBadSeqlen);
+    if (threadIdx.x < D / 4) *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusBadSeqlen);
     return;
   }
   const int ns = (len + p.split_tokens - 1) / p.split_tokens;
-  const float *mrow = p.part_m + static_cast<size_t>(row) * p.num_splits;
-  const float *lrow = p.part_l + static_cast<size_t>(row) * p.num_splits;
-  const float4 *orow = reinterpret_cast<const float4 *>(p.part_o + static_cast<size_t>(row) * p.num_splits * D);
-  // Markers in l: the decode kernel already wrote this row (a single split),
-  // or a split met an invalid page id / the length exceeds the capacity (the
-  // row is zero).
-  if (ns == 1 && lrow[0] == kLFinal) return;
-  float M = kNegInf;
-  bool bad = false;
-  for (int k = c4; k < ns; k += kTPR) {
-    M = fmaxf(M, mrow[k]);
-    bad |= lrow[k] < 0.f;
+  const long long base = static_cast<long long>(row) * p.num_splits;
+  // the decode kernel already wrote this row (a single split)
+  if (ns == 1 && p.part_l[base] == kLFinal) return;
+  merge_row<D>(p.part_o, p.part_m, p.part_l, ns, [&](int k) -> long long { return base + k; }, dst);
+}
+
+// Balanced mode: one block per (unit, head).  The decode kernel recorded, for
+// every unit, the first and last decode blocks holding its tiles and the slot
+// the first one used; every later block holds the unit's first piece of its
+// own range (slot 0), unless its range is empty.  Units one block covered whole
+// are final already; units with an invalid length get zero rows here.
+template <int D, int T>
+__global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const CombineParams p) {
+  const int u = blockIdx.x / p.r;
+  const int h = blockIdx.x % p.r;
+  const int s = u / p.G, g = u % p.G;
+  const size_t row = static_cast<size_t>(s) * p.H + static_cast<size_t>(g) * p.r + h;
+  float4 *dst = reinterpret_cast<float4 *>(p.out + row * D) + threadIdx.x % (D / 4);
+  const int len = __ldg(p.seqlens + s);
+  pdl_wait_primary();  // the header, unit records and partial states come from the decode kernel
+  const int N = p.ws_header[0];
+  const int capacity = p.ws_header[1];
+  if (len < 1 || len > capacity) {
+    if (threadIdx.x < D / 4) *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (threadIdx.x == 0 && h == 0 && p.status) atomicOr(p.status, kStatusBadSeqlen);
+    return;
   }
-#pragma unroll
-  for (int off = kTPR / 2; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(mask, M, off));
-  bad = __any_sync(mask, bad);
-  float L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (!bad && M != kNegInf) {
-#pragma unroll 4
-    for (int k = 0; k < ns; ++k) {
-      const float w = ex2(mrow[k] - M);
-      L += lrow[k] * w;
-      const float4 v = orow[static_cast<size_t>(k) * kTPR + c4];
-      acc.x += v.x * w;
-      acc.y += v.y * w;
-      acc.z += v.z * w;
-      acc.w += v.w * w;
-    }
-  }
-  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (!bad && L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
-  *dst = res;
+  const long long W = static_cast<long long>(static_cast<unsigned>(p.ws_header[2])) |
+                      (static_cast<long long>(p.ws_header[3]) << 32);
+  const int4 meta = p.ws_meta[u];
+  const int c_lo = meta.x, c_hi = meta.y, slot_lo = meta.z;
+  if (c_lo == c_hi) return;  // one decode block covered the unit: its rows are final
+  merge_row<D>(p.part_o, p.part_m, p.part_l, c_hi - c_lo + 1,
+               [&](int k) -> long long {
+                 const long long c = c_lo + k;
+                 if (k > 0 && (c * W / N) == ((c + 1) * W / N)) return -1;  // empty range
+                 return (2 * c + (k == 0 ? slot_lo : 0)) * p.r + h;
+               },
+               dst);
 }
 
 }  // namespace gqa

@@ -196,7 +196,8 @@ def gqa_split_partials(q, k_cache, v_cache, seqlens, page_table=None, *, split_t
                        max_seqlen: int, workspace, out=None, scale=None, status=None, stream=None,
                        flags: int = 0) -> None:
     """Partials kernel only.  With ``out`` given, sequences that fit in one
-    split are finished here and left alone by the combine."""
+    split (or, with split_tokens=0, units one block covers whole) are finished
+    here and left alone by the combine; split_tokens=0 requires ``out``."""
     dims = dims_for(q, k_cache, page_table, flags)
     rc = load().gqa_split_partials(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
                                    _ptr(out), ctypes.byref(dims), _scale(q, scale), _ptr(status), int(split_tokens),

@@ -104,8 +104,13 @@ def test_workspace_size(lib):
     assert gqa.gqa_decode_split_workspace_size(d, 131072, 4096) == r256(rows * 128 * 4) + 2 * r256(rows * 4)
     assert gqa.gqa_decode_split_workspace_size(d, 131072, 100) == 0       # not a multiple of 128
     assert gqa.gqa_decode_split_workspace_size(d, 0, 4096) == 0
-    # split_tokens = 0 sizes for the finest split, which bounds every plan
-    assert gqa.gqa_decode_split_workspace_size(d, 4096, 0) == gqa.gqa_decode_split_workspace_size(d, 4096, 128)
+    # split_tokens = 0: equal-work ranges (header + 2 slots of r heads for up to
+    # 512 blocks), or fixed splits of 4096 for batches above 1024 sequences
+    r = 32 // 4
+    bal = 256 + r256(4 * 4 * 16) + r256(512 * 2 * r * 128 * 4) + 2 * r256(512 * 2 * r * 4)
+    fixed = gqa.gqa_decode_split_workspace_size(d, 131072, 4096)
+    assert gqa.gqa_decode_split_workspace_size(d, 131072, 0) == max(bal, fixed)
+    assert gqa.gqa_decode_split_workspace_size(d, 4096, 0) == max(bal, gqa.gqa_decode_split_workspace_size(d, 4096, 4096))
 
 
 def test_split_checks(lib):
@@ -120,29 +125,29 @@ def test_split_checks(lib):
     assert call(128, 256, need - 1) == -8
     assert call(128, 256, need, w=None) == -8
     assert call(128, 256, need, w=FAKE + 8) == -2
-    assert lib.gqa_split_combine(FAKE, FAKE, ctypes.byref(d), None, 0, 256, ws, need, None) == -7
+    need0 = gqa.gqa_decode_split_workspace_size(d, 256, 0)
+    assert lib.gqa_split_combine(FAKE, FAKE, ctypes.byref(d), None, 0, 256, ws, need0 - 1, None) == -8
+    assert lib.gqa_split_combine(FAKE, FAKE, ctypes.byref(d), None, 100, 256, ws, need, None) == -7
+    assert lib.gqa_decode_split(FAKE, FAKE, FAKE, FAKE, None, FAKE, ctypes.byref(d), 0.125, None, 0, 256, ws,
+                                need0 - 1, None) == -8
 
 
 def test_plan_split_tokens(lib):
-    # Llama-2-70B layer: 32 sequences x 8 groups = 256 units already give
-    # ~1.5 blocks per SM on 148 SMs, and 4096 tokens is not above the cap: no split
+    # Llama-2-70B layer: 32 x 8 = 256 units >= 1.5 per SM on 148 SMs, 4096 tokens: one split
     d = _dims(batch=32, num_heads=64, num_kv_heads=8, head_dim=128, page_size=4096)
     assert gqa.gqa_plan_split_tokens(d, 4096, 148) == 4096
-    # a single long sequence (4 groups): about 1.5 items per SM
+    assert gqa.gqa_plan_split_tokens(d, 4000, 148) == 4096      # rounded up to 128
+    # too few units for the SMs: equal-work ranges
+    assert gqa.gqa_plan_split_tokens(d, 4096, 200) == 0
+    # long sequences: equal-work ranges
     d1 = _dims(batch=1, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072)
-    t1 = gqa.gqa_plan_split_tokens(d1, 131072, 148)
-    assert t1 % 128 == 0
-    items = 4 * -(-131072 // t1)
-    assert 1.4 * 148 <= items <= 1.6 * 148
-    # long sequences are cut to at most 4096 tokens even when units are plenty
+    assert gqa.gqa_plan_split_tokens(d1, 131072, 148) == 0
     d3 = _dims(batch=64, num_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=70000,
                max_pages_per_seq=2048)
-    assert gqa.gqa_plan_split_tokens(d3, 32768, 148) == 4096
-    # 16 sequences x 1 group (MQA sweep): 14 splits of 8192 tokens -> 640 (rounded to 128)
-    d2 = _dims(batch=16, num_heads=32, num_kv_heads=1, head_dim=128, page_size=8192)
-    assert gqa.gqa_plan_split_tokens(d2, 8192, 148) == 640
-    # never below one quantum
-    assert gqa.gqa_plan_split_tokens(d1, 1, 148) == 128
+    assert gqa.gqa_plan_split_tokens(d3, 32768, 148) == 0
+    # batches above 1024 sequences with long caches: fixed splits of 4096
+    d4 = _dims(batch=2000, num_heads=8, num_kv_heads=1, head_dim=64, page_size=8192)
+    assert gqa.gqa_plan_split_tokens(d4, 8192, 148) == 4096
     with pytest.raises(gqa.GqaError) as e:
         gqa.gqa_plan_split_tokens(_dims(batch=0), 128, 148)
     assert e.value.code == -6

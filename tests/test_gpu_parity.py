@@ -45,9 +45,14 @@ def run_gpu(inp, entry, split_tokens=0, max_seqlen=None, scale=None, flags=0):
         out = gqa.gqa_decode(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, scale=scale,
                              status=st, flags=flags)
     else:
-        out = gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
-                                   split_tokens=split_tokens, max_seqlen=max_seqlen, scale=scale,
-                                   status=st, flags=flags)
+        # the workspace is filled with NaN bytes: a read of any slot the call
+        # did not write shows up in the output
+        mx = max_seqlen or inp.k_cache.shape[2] * (1 if inp.page_table is None else inp.page_table.shape[1])
+        ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, mx, split_tokens).fill_(0xFF)
+        out = torch.full(inp.q.shape, float("nan"), dtype=torch.float32, device=inp.q.device)
+        gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                             split_tokens=split_tokens, max_seqlen=mx, scale=scale, workspace=ws,
+                             out=out, status=st, flags=flags)
     torch.cuda.synchronize()
     return out, int(st.item())
 
@@ -129,13 +134,13 @@ def _permute_pool(inp, seed):
     return type(inp)(inp.q, k, v, inp.seqlens, pt, inp.workload)
 
 
-@pytest.mark.parametrize("entry", ["cluster", "split"])
+@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 256), ("split", 0)])
 @pytest.mark.parametrize("P", [8, 16, 128])
-def test_page_permutation_bit_exact(entry, P):
+def test_page_permutation_bit_exact(entry, split, P):
     w = w_small(b=5, r=8, G=2, d=128, m=1000, P=P)
     inp = make_inputs(w, device="cuda", lens=[1000, 17, 640, 129, 999], spare_pages=3)
-    a, _ = run_gpu(inp, entry, split_tokens=256)
-    b, _ = run_gpu(_permute_pool(inp, 1), entry, split_tokens=256)
+    a, _ = run_gpu(inp, entry, split_tokens=split)
+    b, _ = run_gpu(_permute_pool(inp, 1), entry, split_tokens=split)
     assert torch.equal(a, b)
 
 
@@ -150,15 +155,15 @@ def test_contiguous_equals_paged_single_page(entry):
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("entry", ["cluster", "split"])
+@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 256), ("split", 0)])
 @pytest.mark.parametrize("P", [None, 16, 64])
-def test_nan_poison_past_lengths(entry, P):
+def test_nan_poison_past_lengths(entry, split, P):
     w = w_small(b=4, r=8, G=2, d=128, m=700, P=P)
     lens = [700, 33, 257, 1]
     clean = make_inputs(w, device="cuda", lens=lens, spare_pages=2 if P else 0)
     dirty = make_inputs(w, device="cuda", lens=lens, spare_pages=2 if P else 0, poison=True)
-    a, _ = run_gpu(clean, entry, split_tokens=256)
-    b, _ = run_gpu(dirty, entry, split_tokens=256)
+    a, _ = run_gpu(clean, entry, split_tokens=split)
+    b, _ = run_gpu(dirty, entry, split_tokens=split)
     assert torch.isfinite(b).all() and torch.equal(a, b)
 
 
@@ -175,6 +180,47 @@ def test_partials_then_combine_equals_decode_split(with_out):
                           split_tokens=512, max_seqlen=2048, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(out, full)
+
+
+@pytest.mark.parametrize("P", [None, 16])
+def test_balanced_partials_then_combine_equals_decode_split(P):
+    w = w_small(b=5, r=8, G=2, d=128, m=3000, P=P)
+    inp = make_inputs(w, device="cuda", lens=[3000, 7, 1500, 2999, 64])
+    full, _ = run_gpu(inp, "split", split_tokens=0, max_seqlen=3000)
+    ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, 3000, 0)
+    out = torch.full_like(full, float("nan"))
+    gqa.gqa_split_partials(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, split_tokens=0,
+                           max_seqlen=3000, workspace=ws, out=out)
+    gqa.gqa_split_combine(inp.seqlens, out, gqa.dims_for(inp.q, inp.k_cache, inp.page_table),
+                          split_tokens=0, max_seqlen=3000, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, full)
+
+
+@pytest.mark.parametrize("P", [None, 8, 32])
+@pytest.mark.parametrize("d,r,G", [(128, 8, 3), (64, 4, 2), (128, 1, 5), (128, 16, 2), (64, 32, 1)])
+def test_balanced_mixed_lengths(P, d, r, G):
+    """Equal-work ranges over units of very different lengths, with invalid
+    lengths interleaved: every unit boundary, block boundary and empty unit."""
+    lens = [1, 2000, 0, 63, 64, 65, 1999, -4, 700, 129, 1, 2048, 5000, 333]
+    w = w_small(b=len(lens), r=r, G=G, d=d, m=2048, P=P, seed=d + r + G)
+    inp = make_inputs(w, device="cuda", lens=[max(1, min(x, 2048)) for x in lens])
+    inp.seqlens.copy_(torch.tensor(lens, dtype=torch.int32))
+    ref, st_ref = run_oracle(inp)
+    assert st_ref == 1
+    got, st = run_gpu(inp, "split", split_tokens=0)
+    assert st == gqa.STATUS_BAD_SEQLEN
+    assert_parity(got, ref, "balanced P=%s d=%d r=%d G=%d" % (P, d, r, G))
+
+
+def test_balanced_falls_back_to_fixed_splits_for_long_batches():
+    lens = [(13 * i) % 200 + 1 for i in range(1030)]
+    w = w_small(b=1030, r=4, G=1, d=64, m=200, seed=3)
+    inp = make_inputs(w, device="cuda", lens=lens)
+    ref, _ = run_oracle(inp)
+    got, st = run_gpu(inp, "split", split_tokens=0)
+    assert st == 0
+    assert_parity(got, ref, "b=1030 fallback")
 
 
 def test_decode_items_path_many_units():
@@ -201,7 +247,7 @@ def test_repeat_runs_bit_identical():
 # ---------------------------------------------------------------- data errors on the device
 
 
-@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 128), ("split", 512)])
+@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 128), ("split", 512), ("split", 0)])
 def test_bad_page_id_sets_status_and_zeroes_row(entry, split):
     w = w_small(b=3, r=8, G=2, d=128, m=512, P=16)
     inp = make_inputs(w, device="cuda", lens=[512, 300, 40])
@@ -224,7 +270,7 @@ def test_bad_page_id_sets_status_and_zeroes_row(entry, split):
     assert st == 0 and torch.equal(got, clean)
 
 
-@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 128), ("split", 256)])
+@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 128), ("split", 256), ("split", 0)])
 @pytest.mark.parametrize("paged", [False, True])
 def test_bad_length_sets_status_and_zeroes_row(entry, split, paged):
     w = w_small(b=3, r=4, G=2, d=64, m=256, P=16 if paged else None)
