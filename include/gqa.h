@@ -205,6 +205,32 @@ int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims,
  */
 int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms);
 
+/*
+ * gqa_decode_split_static -- gqa_decode_split without a caller-provided
+ * workspace, for callers that may not allocate device memory while they
+ * decode (a process whose HBM is handed out by another memory manager, or a
+ * latency-critical loop that must stay out of the CUDA allocator).  The pages
+ * this library follows have no counterpart of it: it only moves the scratch.
+ *
+ * Same arguments and results as gqa_decode_split, minus workspace and
+ * workspace_bytes.  The scratch is a fixed array of GQA_STATIC_WORKSPACE_BYTES
+ * in the library's device module; each GPU that loads the library holds it
+ * until the process exits.  Problems whose gqa_decode_split_workspace_size()
+ * exceeds that size are rejected with GQA_ERR_WORKSPACE before anything runs.
+ * The first call on a device looks up the array's device address (a CUDA
+ * runtime call, no allocation) and caches it; make that first call before any
+ * stream capture.  All calls share the array: calls whose kernels overlap on
+ * the GPU (different streams or host threads) race on it.  Nothing in it needs
+ * to start at zero.  No cudaMalloc, cudaFree or other allocating routine is
+ * called.
+ */
+#define GQA_STATIC_WORKSPACE_BYTES (8u << 20)
+
+int gqa_decode_split_static(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens, const int32_t *page_table, float *out,
+                            const gqa_dims *dims, float scale, uint32_t *status,
+                            int32_t split_tokens, int32_t max_seqlen, void *stream);
+
 /* A static, human-readable name for a GQA_OK / GQA_ERR_* code. */
 const char *gqa_status_string(int code);
 

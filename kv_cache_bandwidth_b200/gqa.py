@@ -24,7 +24,7 @@ __all__ = [
     "gqa_split_partials", "gqa_split_combine", "gqa_decode_split_workspace_size",
     "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version", "dims_for",
     "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
-    "FLAG_CONTRACT_FMA", "ERRORS",
+    "FLAG_CONTRACT_FMA", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +91,8 @@ def load():
     lib.gqa_decode_split_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32]
     lib.gqa_plan_split_tokens.restype = ctypes.c_int32
     lib.gqa_plan_split_tokens.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32]
+    lib.gqa_decode_split_static.restype = ctypes.c_int
+    lib.gqa_decode_split_static.argtypes = _DECODE_ARGS + [ctypes.c_int32, ctypes.c_int32, _vp]
     lib.gqa_status_string.restype = ctypes.c_char_p
     lib.gqa_status_string.argtypes = [ctypes.c_int]
     lib.gqa_abi_version.restype = ctypes.c_int32
@@ -212,4 +214,26 @@ def gqa_split_combine(seqlens, out, dims: Dims, *, split_tokens: int, max_seqlen
                                   int(split_tokens), int(max_seqlen), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "gqa_split_combine")
+    return out
+
+
+STATIC_WORKSPACE_BYTES = 8 << 20  # GQA_STATIC_WORKSPACE_BYTES
+
+
+def gqa_decode_split_static(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int = 0,
+                            max_seqlen: Optional[int] = None, out=None, scale=None, status=None,
+                            stream=None, flags: int = 0) -> torch.Tensor:
+    """gqa_decode_split with the library's fixed device scratch instead of a
+    workspace: for callers that may not allocate device memory while they
+    decode.  ``out`` must be given by such callers (allocating it here is a
+    convenience for tests).  Concurrent calls on different streams race on the
+    shared scratch."""
+    out = _out_for(q, out)
+    if max_seqlen is None:
+        max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
+    dims = dims_for(q, k_cache, page_table, flags)
+    rc = load().gqa_decode_split_static(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+                                        _ptr(page_table), _ptr(out), ctypes.byref(dims), _scale(q, scale),
+                                        _ptr(status), int(split_tokens), int(max_seqlen), _stream(stream))
+    _check(rc, "gqa_decode_split_static")
     return out
