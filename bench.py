@@ -152,12 +152,9 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from kv_cache_bandwidth_b200 import dist as gdist
+
+    return x if world == 1 else gdist.max_over_ranks(x)
 
 
 # --------------------------------------------------------------------------- oracle leg

@@ -91,7 +91,7 @@ extern "C" {
 
 /* gqa_dims.flags: choice of the q.k / p.v contraction (default: automatic). */
 #define GQA_FLAG_CONTRACT_MMA 1u   /* tensor cores (mma.sync m16n8k16 bf16) */
-#define GQA_FLAG_CONTRACT_FMA 2u   /* fp32 FMA on CUDA cores */
+#define GQA_FLAG_CONTRACT_FMA 2u   /* fp32 FMA on CUDA cores; r = H/G <= 2 only (else GQA_ERR_HEADS) */
 
 typedef struct gqa_dims {
     int32_t batch;             /* b: sequences, one query token each */
@@ -99,8 +99,8 @@ typedef struct gqa_dims {
     int32_t num_kv_heads;      /* G: KV groups (heads of the cache) */
     int32_t head_dim;          /* d = d_k = d_v: 64 or 128 */
     int32_t page_size;         /* paged: tokens per page; contiguous: capacity m */
-    int32_t num_pages;         /* paged: pages in each pool; contiguous: ignored (= b) */
-    int32_t max_pages_per_seq; /* paged: row stride of page_table; contiguous: ignored */
+    int32_t num_pages;         /* paged: pages in each pool; contiguous: ignored (the pool is b sequences) */
+    int32_t max_pages_per_seq; /* paged: row stride of page_table; contiguous: 0 */
     uint32_t flags;            /* GQA_FLAG_*; 0 = automatic */
 } gqa_dims;
 
@@ -134,15 +134,17 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
  *
  * split_tokens: a positive multiple of 128 (fixed splits as above), or 0 to
  *               let the library cut the work from the dims, max_seqlen and
- *               the SM count: when max_seqlen <= 4096 and the (sequence,
- *               group) units number at least 1.5 per SM, one split (no
- *               combine); otherwise, for up to 1024 sequences, equal-work
- *               ranges (stream-K): the tiles of all units, in order, are cut
- *               into one contiguous range per resident thread block; a block
- *               finishes the units that lie wholly in its range and leaves
- *               partial states for the (at most two) units it shares with its
- *               neighbours, which the second kernel merges.  Longer batches
- *               use splits of 4096.
+ *               the SM count.  Paged dims (max_pages_per_seq > 0), the layout
+ *               of choice for unequal lengths, get equal-work ranges
+ *               (stream-K) for up to 1024 sequences: the tiles of all
+ *               (sequence, group) units, in order, are cut into one contiguous
+ *               range per resident thread block; a block finishes the units
+ *               that lie wholly in its range and leaves partial states for the
+ *               (at most two) units it shares with its neighbours, which the
+ *               second kernel merges (longer paged batches: splits of 4096).
+ *               Contiguous dims (max_pages_per_seq == 0) get fixed splits:
+ *               one per unit when the units number 1.5 per SM or more (no
+ *               combine), else just enough splits for that many items.
  * max_seqlen:   an upper bound of every seqlens[s] (sizes the grid and the
  *               workspace); a length above it is treated as invalid
  *               (GQA_STATUS_BAD_SEQLEN, row zeroed).

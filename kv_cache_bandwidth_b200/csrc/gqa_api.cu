@@ -94,6 +94,7 @@ struct Shape {
   bool paged;
   long long capacity;
   int nt, nhb;  // kernel variant: n8 head tiles per consumer warp, head blocks
+  bool fma;     // q.k and p.v on CUDA cores instead of tensor cores
 };
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -133,6 +134,8 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh) {
   if (static_cast<long long>(s.b) * s.H * s.D > (1ll << 31) - 1) return GQA_ERR_DIMS;
   s.nt = r <= 8 ? 1 : 2;
   s.nhb = r <= 16 ? 1 : (r <= 32 ? 2 : 4);
+  s.fma = (d.flags & GQA_FLAG_CONTRACT_FMA) != 0;
+  if (s.fma && r > 2) return GQA_ERR_HEADS;  // the CUDA-core contraction covers r <= 2
   *sh = s;
   return GQA_OK;
 }
@@ -191,11 +194,11 @@ struct Launch {
   cudaStream_t stream;
 };
 
-template <int D, int NT, int NHB, int STAGES, bool PAGED, Mode MODE>
+template <int D, int NT, int NHB, int STAGES, bool PAGED, Mode MODE, int FMA = 0>
 int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p, Launch l) {
   constexpr int CH = (D == 64) ? 2 : 1;
   using TL = gqa::Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBalanced>;
-  auto kernel = gqa::gqa_decode_kernel<D, NT, NHB, CH, STAGES, PAGED, MODE>;
+  auto kernel = gqa::gqa_decode_kernel<D, NT, NHB, CH, STAGES, PAGED, MODE, FMA>;
   const int smem = TL::kSmemBytes;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return GQA_ERR_CUDA;
@@ -250,6 +253,9 @@ Pipe pick_pipe(const Shape &sh) {
 template <int D, bool PAGED, Mode MODE>
 int launch_decode_d(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv,
                     const DecodeParams &p, const Launch &l) {
+  if (sh.fma)
+    return sh.r == 1 ? launch_decode_t<D, 1, 1, 3, PAGED, MODE, 1>(tk, tv, p, l)
+                     : launch_decode_t<D, 1, 1, 3, PAGED, MODE, 2>(tk, tv, p, l);
   if (sh.nt == 1) {
     switch (pick_pipe(sh)) {
       case Pipe::kTrio: return launch_decode_t<D, 1, 1, 2, PAGED, MODE>(tk, tv, p, l);
@@ -347,8 +353,12 @@ BalancedWorkspace balanced_layout(const Shape &sh) {
 }
 
 size_t auto_workspace_bytes(const Shape &sh, int max_seqlen) {
-  const int splits = (max_seqlen + kFallbackSplit - 1) / kFallbackSplit;
-  return std::max(balanced_layout(sh).total, workspace_layout(sh, splits).total);
+  const long long units = static_cast<long long>(sh.b) * sh.G;
+  const long long by_sms = (3ll * 256 + 1) / 2;  // 1.5 items per SM on the largest GPU covered
+  long long splits = std::max<long long>((max_seqlen + kFallbackSplit - 1) / kFallbackSplit,
+                                         (by_sms + units - 1) / units);
+  splits = std::min<long long>(splits, (max_seqlen + kSplitQuantum - 1) / kSplitQuantum);
+  return std::max(balanced_layout(sh).total, workspace_layout(sh, static_cast<int>(splits)).total);
 }
 
 int run_balanced_decode(const Shape &sh, int sms, const void *q, const void *k, const void *v,
@@ -406,21 +416,33 @@ int run_balanced_combine(const Shape &sh, const int32_t *seqlens, float *out, ui
 
 // split_tokens == 0 in the split API: the library's choice, made from the
 // dims, max_seqlen and the SM count only, so that gqa_split_partials and
-// gqa_split_combine make the same one.  Uniform work that already gives every
-// SM 1.5 blocks of at most 4096 tokens runs one block per (sequence, group) with
-// no combine; everything else runs equal-work ranges (fixed 4096-token splits
-// for batches too long to scan in every block).
+// gqa_split_combine make the same one.  A paged pool (dims->max_pages_per_seq
+// > 0) is the layout of choice for sequences of unequal lengths, so it gets
+// equal-work ranges (for up to kMaxBalancedBatch sequences; fixed 4096-token
+// splits beyond).  A contiguous cache gets fixed splits: one per (sequence,
+// group) when the units already give 1.5 blocks per SM, else just enough
+// splits for that.
 struct AutoChoice {
   bool balanced;
   int split_tokens;
 };
 
-AutoChoice choose_auto(const Shape &sh, int max_seqlen, int sms) {
+bool dims_paged(const gqa_dims *dims) { return dims->max_pages_per_seq > 0; }
+
+int round_split(long long tokens) {
+  tokens = (tokens + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
+  return static_cast<int>(std::max<long long>(kSplitQuantum, tokens));
+}
+
+AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
+  if (paged) {
+    if (sh.b <= kMaxBalancedBatch) return {true, 0};
+    return {false, kFallbackSplit};
+  }
   const long long units = static_cast<long long>(sh.b) * sh.G;
-  if (max_seqlen <= kFallbackSplit && 2 * units >= 3ll * sms)
-    return {false, (max_seqlen + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum};
-  if (sh.b <= kMaxBalancedBatch) return {true, 0};
-  return {false, kFallbackSplit};
+  const long long want = (3ll * sms + 1) / 2;
+  const long long splits = units >= want ? 1 : (want + units - 1) / units;
+  return {false, round_split((max_seqlen + splits - 1) / splits)};
 }
 
 // split_tokens == 0 in the split API: checks shared by its entry points.
@@ -572,7 +594,7 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
     num_sms = dev.sms;
   }
-  const AutoChoice ch = choose_auto(sh, max_seqlen, num_sms);
+  const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(num_sms, 256));
   return ch.balanced ? 0 : ch.split_tokens;
 }
 
@@ -591,7 +613,7 @@ int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
       return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    const AutoChoice ch = choose_auto(sh, max_seqlen, dev.sms);
+    const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) {
       if (!out) return GQA_ERR_NULL_POINTER;  // whole units are finished straight into out
       return run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale,
@@ -623,7 +645,7 @@ int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims, 
     if ((rc = prepare_auto(dims, false, max_seqlen, workspace, workspace_bytes, &sh)) != GQA_OK) return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    const AutoChoice ch = choose_auto(sh, max_seqlen, dev.sms);
+    const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) return run_balanced_combine(sh, seqlens, out, status, workspace, st);
     split_tokens = ch.split_tokens;
   }
@@ -651,7 +673,7 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, co
       return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    const AutoChoice ch = choose_auto(sh, max_seqlen, dev.sms);
+    const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) {
       rc = run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale, status,
                                max_seqlen, workspace, st);

@@ -306,7 +306,196 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
   return true;
 }
 
-template <int D, int NT, int NHB, int CH, int STAGES, bool PAGED, Mode MODE>
+// The q.k and p.v contractions on CUDA cores (fp32 FMA) for group ratios
+// r <= RMAX <= 2, as the alternative to the tensor-core path.  Same pipeline, same
+// piece, same merge: this consumes the piece's tiles and leaves the warp's
+// running maximum / sum in m_sm / l_sm (heads r..7 as -inf / 0) and its share
+// of the output rows accumulated in osum, exactly as the tensor-core path does.
+//
+// Lane layout per 16-token chunk: for q.k two lanes per token (lane = 2 t +
+// half), each covering half of d with the bf16 pairs of q held in registers;
+// for p.v each lane owns d/32 consecutive dims and takes token t's
+// probability from lane 2 t by shuffle.  Rows past the range are skipped, so
+// whatever they hold (even NaN) never enters the sums.
+template <int D, int T, int CH, int STAGES, bool PAGED, int NWT, int HB, int OSTRIDE, int RMAX>
+__device__ __forceinline__ int consume_fma(const DecodeParams &p, const Piece &pc, uint32_t q_slot,
+                                           uint8_t *smem, uint32_t bar_full, uint32_t bar_empty,
+                                           uint32_t bar_qempty_slot, volatile int *tile_bad,
+                                           volatile int *abort_flag, float *m_sm, float *l_sm, float *osum,
+                                           int &tile, int warp, int lane, int nc) {
+  constexpr int kRMax = RMAX;      // heads held by each lane (r <= RMAX)
+  constexpr int kPairs = D / 4;   // bf16 pairs of q per lane (half of d)
+  constexpr int kDpl = D / 32;    // output dims per lane
+  const float kNegInf = -__int_as_float(0x7f800000);
+  constexpr int kTileBytes = T * D * 2;
+  const int ws = warp % NWT;
+  const int tk = lane >> 1, half = lane & 1;
+  const int r = p.r;
+  const float sl = p.scale_log2;
+
+  uint32_t qf[kRMax][kPairs];
+#pragma unroll
+  for (int h = 0; h < kRMax; ++h) {
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i)
+      qf[h][i] = (h < r) ? ld_shared_u32(q_slot + h * D * 2 + (half * (D / 2) + 2 * i) * 2) : 0u;
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar_qempty_slot);
+
+  float m_run[kRMax], l_run[kRMax], o[kRMax][kDpl];
+#pragma unroll
+  for (int h = 0; h < kRMax; ++h) {
+    m_run[h] = kNegInf;
+    l_run[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kDpl; ++i) o[h][i] = 0.f;
+  }
+  int bad = 0;
+  for (int t0 = pc.t_begin; t0 < pc.t_end && !*abort_flag; t0 += T, ++tile) {
+    const int stage = tile % STAGES;
+    bool ok = mbar_wait(bar_full + 8 * stage, (tile / STAGES) & 1);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+      if (lane == 0) {
+        *abort_flag = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+      }
+      break;
+    }
+    if (PAGED) bad |= tile_bad[stage];
+    const uint32_t kbase = smem_addr(smem + stage * 2 * kTileBytes);
+    const uint32_t vbase = kbase + kTileBytes;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int row0 = (ws * CH + c) * 16;
+      // ---- q.k: this lane's half of d for token row0 + tk
+      float acc[kRMax];
+#pragma unroll
+      for (int h = 0; h < kRMax; ++h) acc[h] = 0.f;
+#pragma unroll
+      for (int ch8 = 0; ch8 < D / 16; ++ch8) {
+        uint32_t kw[4];
+        const uint32_t addr = kbase + swz_offset<T>(row0 + tk, half * (D / 2) + 8 * ch8);
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(kw[0]), "=r"(kw[1]), "=r"(kw[2]), "=r"(kw[3])
+                     : "r"(addr)
+                     : "memory");
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float k0 = __uint_as_float(kw[e] << 16), k1 = __uint_as_float(kw[e] & 0xffff0000u);
+#pragma unroll
+          for (int h = 0; h < kRMax; ++h) {
+            const uint32_t qw = qf[h][ch8 * 4 + e];
+            acc[h] = fmaf(__uint_as_float(qw << 16), k0, acc[h]);
+            acc[h] = fmaf(__uint_as_float(qw & 0xffff0000u), k1, acc[h]);
+          }
+        }
+      }
+      const bool live = t0 + row0 + tk < pc.t_end;
+      float pr[kRMax];
+#pragma unroll
+      for (int h = 0; h < kRMax; ++h) {
+        const float sdot = acc[h] + __shfl_xor_sync(0xffffffffu, acc[h], 1);
+        const float x = live ? sdot * sl : kNegInf;
+        float mx = x;
+#pragma unroll
+        for (int off = 2; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float mn = fmaxf(m_run[h], mx);
+        const float base = (mn == kNegInf) ? 0.f : mn;
+        pr[h] = ex2(x - base);
+        if (mn != m_run[h]) {  // uniform across the warp
+          const float alpha = ex2(m_run[h] - base);
+          l_run[h] *= alpha;
+#pragma unroll
+          for (int i = 0; i < kDpl; ++i) o[h][i] *= alpha;
+        }
+        l_run[h] += half == 0 ? pr[h] : 0.f;
+        m_run[h] = mn;
+      }
+      // ---- p.v: this lane's dims, token by token (rows past the range skipped)
+      const int n_live = min(16, pc.t_end - (t0 + row0));
+      for (int tt = 0; tt < n_live; ++tt) {
+        float pt[kRMax];
+#pragma unroll
+        for (int h = 0; h < kRMax; ++h) pt[h] = __shfl_sync(0xffffffffu, pr[h], 2 * tt);
+        const int col = lane * kDpl;
+        const uint32_t addr = vbase + swz_offset<T>(row0 + tt, col & ~7) + (col & 7) * 2;
+        float v[kDpl];
+        if (kDpl == 4) {
+          uint32_t w0, w1;
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(addr) : "memory");
+          v[0] = __uint_as_float(w0 << 16);
+          v[1] = __uint_as_float(w0 & 0xffff0000u);
+          v[2] = __uint_as_float(w1 << 16);
+          v[3] = __uint_as_float(w1 & 0xffff0000u);
+        } else {
+          const uint32_t w0 = ld_shared_u32(addr);
+          v[0] = __uint_as_float(w0 << 16);
+          v[1] = __uint_as_float(w0 & 0xffff0000u);
+        }
+#pragma unroll
+        for (int h = 0; h < kRMax; ++h) {
+#pragma unroll
+          for (int i = 0; i < kDpl; ++i) o[h][i] = fmaf(pt[h], v[i], o[h][i]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * stage);
+  }
+
+  // ---- this warp's state into the merge arrays
+#pragma unroll
+  for (int h = 0; h < kRMax; ++h) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], off);
+  }
+  if (lane < HB) {
+    float mv = kNegInf, lv = 0.f;
+#pragma unroll
+    for (int h = 0; h < kRMax; ++h) {
+      if (lane == h && h < r) {
+        mv = m_run[h];
+        lv = l_run[h];
+      }
+    }
+    m_sm[warp * HB + lane] = mv;
+    l_sm[warp * HB + lane] = lv;
+  }
+  named_barrier(1, nc * 32);
+  float f[kRMax];
+#pragma unroll
+  for (int h = 0; h < kRMax; ++h) {
+    float M = kNegInf;
+#pragma unroll
+    for (int w2 = 0; w2 < NWT; ++w2) M = fmaxf(M, m_sm[w2 * HB + h]);
+    f[h] = (M == kNegInf) ? 0.f : ex2(m_run[h] - M);
+  }
+  // deterministic accumulation: token slice 0 stores, slices 1..3 add in order
+#pragma unroll
+  for (int step = 0; step < NWT; ++step) {
+    if (ws == step) {
+#pragma unroll
+      for (int h = 0; h < kRMax; ++h) {
+        if (h < r) {
+#pragma unroll
+          for (int i = 0; i < kDpl; ++i) {
+            float *dst = osum + h * OSTRIDE + lane * kDpl + i;
+            const float v = o[h][i] * f[h];
+            *dst = (step == 0) ? v : (*dst + v);
+          }
+        }
+      }
+    }
+    named_barrier(1, nc * 32);
+  }
+  return bad;
+}
+
+// FMA: 0 runs the contractions on tensor cores; 1 or 2 runs them on CUDA
+// cores for group ratios up to that value.
+template <int D, int NT, int NHB, int CH, int STAGES, bool PAGED, Mode MODE, int FMA = 0>
 __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBalanced>::kThreads,
                                   Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBalanced>::kMinBlocks)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -526,6 +715,13 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
           if (p.status) atomicOr(p.status, kStatusTimeout);
         }
       }
+      ++n;
+      int bad = 0;
+      if constexpr (FMA > 0) {
+        bad = consume_fma<D, T, CH, STAGES, PAGED, TL::kNWT, TL::kHB, TL::kOStride, FMA>(
+            p, pc, q_sm + qs * TL::kQBytes, smem, bar_full, bar_empty, bar_qempty + 8 * qs, tile_bad,
+            abort_flag, m_sm, l_sm, osum, tile, warp, lane, nc);
+      } else {
       uint32_t bq[TL::kSteps][NT][2];
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
@@ -540,7 +736,6 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_qempty + 8 * qs);
-      ++n;
 
       float m_run[NT][2], l_run[NT][2];
       float o[TL::kSteps][NT][4];
@@ -551,7 +746,6 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
 #pragma unroll
         for (int mt = 0; mt < TL::kSteps; ++mt) o[mt][j][0] = o[mt][j][1] = o[mt][j][2] = o[mt][j][3] = 0.f;
       }
-      int bad = 0;
 
       for (int t0 = pc.t_begin; t0 < pc.t_end && !*abort_flag; t0 += T, ++tile) {
         const int stage = tile % STAGES;
@@ -726,6 +920,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         }
         named_barrier(1, nc * 32);
       }
+      }  // mma contraction
       for (int h = ctid; h < r_pad; h += nc * 32) {
         const int hb2 = h / TL::kHB, hl = h % TL::kHB;
         float M = kNegInf;

@@ -80,6 +80,7 @@ def test_decode_pointer_checks(lib, case, kw, code):
     (dict(num_kv_heads=0), -6),
     (dict(flags=3), -6),
     (dict(flags=8), -6),
+    (dict(flags=2), -3),                            # CUDA-core contraction: r = 4 > 2
 ])
 def test_decode_dim_checks(lib, kw, code):
     assert _decode(lib, _dims(**kw)) == code
@@ -108,9 +109,10 @@ def test_workspace_size(lib):
     # 512 blocks), or fixed splits of 4096 for batches above 1024 sequences
     r = 32 // 4
     bal = 256 + r256(4 * 4 * 16) + r256(512 * 2 * r * 128 * 4) + 2 * r256(512 * 2 * r * 4)
-    fixed = gqa.gqa_decode_split_workspace_size(d, 131072, 4096)
-    assert gqa.gqa_decode_split_workspace_size(d, 131072, 0) == max(bal, fixed)
-    assert gqa.gqa_decode_split_workspace_size(d, 4096, 0) == max(bal, gqa.gqa_decode_split_workspace_size(d, 4096, 4096))
+    # fixed splits for 1.5 items per SM on a GPU of up to 256 SMs: 384 / 16 units = 24 splits
+    fixed = gqa.gqa_decode_split_workspace_size(d, 131072, 131072 // 24 // 128 * 128)
+    assert gqa.gqa_decode_split_workspace_size(d, 131072, 0) >= max(bal, fixed)
+    assert gqa.gqa_decode_split_workspace_size(d, 4096, 0) >= max(bal, gqa.gqa_decode_split_workspace_size(d, 4096, 4096))
 
 
 def test_split_checks(lib):
@@ -133,20 +135,21 @@ def test_split_checks(lib):
 
 
 def test_plan_split_tokens(lib):
-    # Llama-2-70B layer: 32 x 8 = 256 units >= 1.5 per SM on 148 SMs, 4096 tokens: one split
+    # contiguous, Llama-2-70B layer: 32 x 8 = 256 units >= 1.5 per SM on 148 SMs: one split
     d = _dims(batch=32, num_heads=64, num_kv_heads=8, head_dim=128, page_size=4096)
     assert gqa.gqa_plan_split_tokens(d, 4096, 148) == 4096
     assert gqa.gqa_plan_split_tokens(d, 4000, 148) == 4096      # rounded up to 128
-    # too few units for the SMs: equal-work ranges
-    assert gqa.gqa_plan_split_tokens(d, 4096, 200) == 0
-    # long sequences: equal-work ranges
+    # contiguous, too few units: just enough splits for 1.5 items per SM
+    assert gqa.gqa_plan_split_tokens(d, 4096, 200) == 2048      # 300 items wanted / 256 units -> 2
     d1 = _dims(batch=1, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072)
-    assert gqa.gqa_plan_split_tokens(d1, 131072, 148) == 0
+    t1 = gqa.gqa_plan_split_tokens(d1, 131072, 148)             # 56 splits -> 2432 tokens
+    assert t1 == 2432 and 4 * -(-131072 // t1) >= 1.4 * 148   # rounding to 128 tokens trims a few
+    # paged: equal-work ranges, or splits of 4096 above 1024 sequences
     d3 = _dims(batch=64, num_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=70000,
                max_pages_per_seq=2048)
     assert gqa.gqa_plan_split_tokens(d3, 32768, 148) == 0
-    # batches above 1024 sequences with long caches: fixed splits of 4096
-    d4 = _dims(batch=2000, num_heads=8, num_kv_heads=1, head_dim=64, page_size=8192)
+    d4 = _dims(batch=2000, num_heads=8, num_kv_heads=1, head_dim=64, page_size=16, num_pages=10 ** 6,
+               max_pages_per_seq=512)
     assert gqa.gqa_plan_split_tokens(d4, 8192, 148) == 4096
     with pytest.raises(gqa.GqaError) as e:
         gqa.gqa_plan_split_tokens(_dims(batch=0), 128, 148)

@@ -87,6 +87,42 @@ def test_grid_split_and_cluster(d, r, layout):
         assert_parity(got, ref, "%s split=%d d=%d r=%d %s" % (entry, split, d, r, layout))
 
 
+@pytest.mark.parametrize("d,r", [(64, 1), (64, 2), (128, 1), (128, 2)])
+@pytest.mark.parametrize("layout", ["contig", "P16", "P256"])
+def test_fma_contraction(d, r, layout):
+    """The CUDA-core contraction (GQA_FLAG_CONTRACT_FMA) against the oracle on
+    every decomposition, with tile/page tails and NaN past the lengths."""
+    P = None if layout == "contig" else int(layout[1:])
+    lens = LENS
+    w = w_small(b=len(lens), r=r, G=3, d=d, m=512, P=P, seed=7 * d + r)
+    inp = make_inputs(w, device="cuda", lens=lens, poison=True, spare_pages=2 if P else 0)
+    ref, _ = run_oracle(inp)
+    for entry, split in (("cluster", 0), ("split", 128), ("split", 0), ("split", 1024)):
+        got, st = run_gpu(inp, entry, split_tokens=split, flags=gqa.FLAG_CONTRACT_FMA)
+        assert st == 0
+        assert_parity(got, ref, "fma %s split=%d d=%d r=%d %s" % (entry, split, d, r, layout))
+    # many units: gqa_decode's one-block-per-unit path
+    w2 = w_small(b=80, r=r, G=2, d=d, m=300, P=P, seed=3)
+    inp2 = make_inputs(w2, device="cuda", lens=[(37 * i) % 300 + 1 for i in range(80)])
+    ref2, _ = run_oracle(inp2)
+    got2, st2 = run_gpu(inp2, "cluster", flags=gqa.FLAG_CONTRACT_FMA)
+    assert st2 == 0
+    assert_parity(got2, ref2, "fma items d=%d r=%d" % (d, r))
+
+
+def test_fma_bad_page():
+    w = w_small(b=3, r=1, G=2, d=128, m=512, P=16)
+    inp = make_inputs(w, device="cuda", lens=[512, 300, 40])
+    clean, st = run_gpu(inp, "split", flags=gqa.FLAG_CONTRACT_FMA)
+    assert st == 0
+    pt = inp.page_table.clone()
+    pt[1, 3] = -1
+    bad = type(inp)(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, pt, inp.workload)
+    got, st = run_gpu(bad, "split", flags=gqa.FLAG_CONTRACT_FMA)
+    assert st == gqa.STATUS_BAD_PAGE and torch.count_nonzero(got[1]) == 0
+    assert torch.equal(got[0], clean[0]) and torch.equal(got[2], clean[2])
+
+
 def test_tiny_config_both_entry_points():
     inp = make_inputs(WORKLOADS["tiny"], device="cuda")
     ref, _ = run_oracle(inp)
