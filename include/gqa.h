@@ -143,8 +143,9 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
  *               (at most two) units it shares with its neighbours, which the
  *               second kernel merges (longer paged batches: splits of 4096).
  *               Contiguous dims (max_pages_per_seq == 0) get fixed splits:
- *               one per unit when the units number 1.5 per SM or more (no
- *               combine), else just enough splits for that many items.
+ *               one per unit when the units fill at least three quarters of
+ *               the GPU's resident blocks (no combine), else as many splits
+ *               per unit as still fit one wave of resident blocks.
  * max_seqlen:   an upper bound of every seqlens[s] (sizes the grid and the
  *               workspace); a length above it is treated as invalid
  *               (GQA_STATUS_BAD_SEQLEN, row zeroed).
@@ -182,7 +183,8 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache,
  *
  * Workspace layout for fixed splits (fp32, each array 256-byte aligned,
  * S = ceil(max_seqlen / split_tokens)): o [b, H, S, d] unnormalised sum_j 2^(x_j - m) v_j;
- * m [b, H, S] running maximum of x_j = scale * log2(e) * q.k_j;
+ * m [b, H, S] the base of the split's exponentials (at most 8 below the
+ * maximum of x_j = scale * log2(e) * q.k_j, never above it);
  * l [b, H, S] sum_j 2^(x_j - m), or a marker: -1 the split met an invalid page
  * id; -2 (split 0) the length is outside [1, capacity]; -3 (split 0) the row
  * is already final in `out`.

@@ -354,7 +354,7 @@ BalancedWorkspace balanced_layout(const Shape &sh) {
 
 size_t auto_workspace_bytes(const Shape &sh, int max_seqlen) {
   const long long units = static_cast<long long>(sh.b) * sh.G;
-  const long long by_sms = (3ll * 256 + 1) / 2;  // 1.5 items per SM on the largest GPU covered
+  const long long by_sms = 3ll * 256;  // one wave of up to three blocks per SM on GPUs of up to 256 SMs
   long long splits = std::max<long long>((max_seqlen + kFallbackSplit - 1) / kFallbackSplit,
                                          (by_sms + units - 1) / units);
   splits = std::min<long long>(splits, (max_seqlen + kSplitQuantum - 1) / kSplitQuantum);
@@ -434,14 +434,31 @@ int round_split(long long tokens) {
   return static_cast<int>(std::max<long long>(kSplitQuantum, tokens));
 }
 
+// Resident blocks per SM of the items kernel variant the shape runs (B200:
+// shared memory allows two blocks of the 3-stage ring; the 288- and 544-thread
+// variants for r > 16 fit once by registers).
+int blocks_per_sm(const Shape &sh) {
+  if (sh.fma) return 2;
+  if (sh.nt == 1) {
+    switch (pick_pipe(sh)) {
+      case Pipe::kTrio: return 3;
+      case Pipe::kSolo: return 1;
+      default: return 2;
+    }
+  }
+  return sh.nhb == 1 ? 2 : 1;
+}
+
 AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
   if (paged) {
     if (sh.b <= kMaxBalancedBatch) return {true, 0};
     return {false, kFallbackSplit};
   }
+  // One block per unit when the units fill three quarters of the resident
+  // slots; otherwise as many splits as still fit one wave.
   const long long units = static_cast<long long>(sh.b) * sh.G;
-  const long long want = (3ll * sms + 1) / 2;
-  const long long splits = units >= want ? 1 : (want + units - 1) / units;
+  const long long slots = static_cast<long long>(sms) * blocks_per_sm(sh);
+  const long long splits = 4 * units >= 3 * slots ? 1 : std::max<long long>(1, slots / units);
   return {false, round_split((max_seqlen + splits - 1) / splits)};
 }
 

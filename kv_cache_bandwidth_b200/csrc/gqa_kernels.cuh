@@ -24,8 +24,10 @@
 //     movmatrix; it is split into a bf16 high part and a bf16 residual so that
 //     the product keeps ~16 bits of the probabilities (a single bf16 rounding
 //     would leave ~1e-3 relative error);
-//   * online softmax in base 2: running maximum and sum per head, warp-shuffle
-//     reductions over the token rows, accumulator rescaling by 2^(m_old - m_new);
+//   * online softmax in base 2: a running base (within 2^8 of the maximum) and
+//     sum per head; the maximum is reduced across token rows with warp
+//     shuffles and the accumulators rescaled by 2^(m_old - m_new) only when a
+//     score passes the base by more than 8;
 //   * at the end the consumer warps merge their states in shared memory and
 //     either write a split's partial state (split-KV mode) or merge the blocks
 //     of a thread-block cluster through distributed shared memory and write the
@@ -765,13 +767,13 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
           const int row0 = (ws * CH + c) * 16;
-          // ---- S^T = K q^T for 16 tokens x kHB heads (two accumulator chains)
-          float sacc[NT][4], sacc2[NT][4];
+          // ---- S^T = K q^T for 16 tokens x kHB heads (four accumulator chains)
+          constexpr int kChains = TL::kSteps >= 4 ? 4 : TL::kSteps;
+          float sacc[kChains][NT][4];
 #pragma unroll
-          for (int j = 0; j < NT; ++j) {
-            sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
-            sacc2[j][0] = sacc2[j][1] = sacc2[j][2] = sacc2[j][3] = 0.f;
-          }
+          for (int c2 = 0; c2 < kChains; ++c2)
+#pragma unroll
+            for (int j = 0; j < NT; ++j) sacc[c2][j][0] = sacc[c2][j][1] = sacc[c2][j][2] = sacc[c2][j][3] = 0.f;
           {
             const int mi = lane >> 3;
             const int row = row0 + (mi & 1) * 8 + (lane & 7);
@@ -780,12 +782,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
               uint32_t a[4];
               ldsm_x4(kbase + swz_offset<T>(row, ks * 16 + (mi >> 1) * 8), a);
 #pragma unroll
-              for (int j = 0; j < NT; ++j) {
-                if (ks & 1)
-                  mma_bf16_16816(sacc2[j], a, bq[ks][j][0], bq[ks][j][1]);
-                else
-                  mma_bf16_16816(sacc[j], a, bq[ks][j][0], bq[ks][j][1]);
-              }
+              for (int j = 0; j < NT; ++j) mma_bf16_16816(sacc[ks % kChains][j], a, bq[ks][j][0], bq[ks][j][1]);
             }
           }
           // ---- mask, scale, online softmax, P^T fragments
@@ -795,26 +792,35 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
           uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
-            const float x0 = ok_a ? (sacc[j][0] + sacc2[j][0]) * sl : kNegInf;  // token g8,   head 2*t4
-            const float x1 = ok_a ? (sacc[j][1] + sacc2[j][1]) * sl : kNegInf;  // token g8,   head 2*t4+1
-            const float x2 = ok_b ? (sacc[j][2] + sacc2[j][2]) * sl : kNegInf;  // token g8+8, head 2*t4
-            const float x3 = ok_b ? (sacc[j][3] + sacc2[j][3]) * sl : kNegInf;  // token g8+8, head 2*t4+1
-            float mx_a = fmaxf(x0, x2), mx_b = fmaxf(x1, x3);
+            float sum[4];
 #pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-              mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
-              mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+            for (int e = 0; e < 4; ++e) {
+              sum[e] = sacc[0][j][e];
+#pragma unroll
+              for (int c2 = 1; c2 < kChains; ++c2) sum[e] += sacc[c2][j][e];
             }
-            const float mn_a = fmaxf(m_run[j][0], mx_a);
-            const float mn_b = fmaxf(m_run[j][1], mx_b);
-            const float base_a = (mn_a == kNegInf) ? 0.f : mn_a;
-            const float base_b = (mn_b == kNegInf) ? 0.f : mn_b;
-            const float p0 = ex2(x0 - base_a), p1 = ex2(x1 - base_b);
-            const float p2 = ex2(x2 - base_a), p3 = ex2(x3 - base_b);
-            // rescale only when a running maximum moved (rare after the first tiles)
-            if (__any_sync(0xffffffffu, mn_a != m_run[j][0] || mn_b != m_run[j][1])) {
-              const float alpha_a = ex2(m_run[j][0] - base_a);
-              const float alpha_b = ex2(m_run[j][1] - base_b);
+            const float x0 = ok_a ? sum[0] * sl : kNegInf;  // token g8,   head 2*t4
+            const float x1 = ok_a ? sum[1] * sl : kNegInf;  // token g8,   head 2*t4+1
+            const float x2 = ok_b ? sum[2] * sl : kNegInf;  // token g8+8, head 2*t4
+            const float x3 = ok_b ? sum[3] * sl : kNegInf;  // token g8+8, head 2*t4+1
+            // The exponentials use a base m_run that may trail the true running
+            // maximum by up to kSlack (p <= 2^kSlack): any base gives the same
+            // normalised result as long as l and o share it.  Only when a score
+            // passes the base by more than that is the maximum reduced across the
+            // token rows and the accumulators rescaled to the new base.
+            constexpr float kSlack = 8.f;
+            const bool over = fmaxf(x0, x2) > m_run[j][0] + kSlack || fmaxf(x1, x3) > m_run[j][1] + kSlack;
+            if (__any_sync(0xffffffffu, over)) {
+              float mx_a = fmaxf(x0, x2), mx_b = fmaxf(x1, x3);
+#pragma unroll
+              for (int off = 4; off < 32; off <<= 1) {
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+              }
+              const float mn_a = fmaxf(m_run[j][0], mx_a);
+              const float mn_b = fmaxf(m_run[j][1], mx_b);
+              const float alpha_a = (m_run[j][0] == kNegInf) ? 0.f : ex2(m_run[j][0] - mn_a);
+              const float alpha_b = (m_run[j][1] == kNegInf) ? 0.f : ex2(m_run[j][1] - mn_b);
               l_run[j][0] *= alpha_a;
               l_run[j][1] *= alpha_b;
 #pragma unroll
@@ -824,11 +830,15 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
                 o[mt][j][2] *= alpha_a;
                 o[mt][j][3] *= alpha_b;
               }
+              m_run[j][0] = mn_a;
+              m_run[j][1] = mn_b;
             }
+            const float base_a = (m_run[j][0] == kNegInf) ? 0.f : m_run[j][0];
+            const float base_b = (m_run[j][1] == kNegInf) ? 0.f : m_run[j][1];
+            const float p0 = ex2(x0 - base_a), p1 = ex2(x1 - base_b);
+            const float p2 = ex2(x2 - base_a), p3 = ex2(x3 - base_b);
             l_run[j][0] += p0 + p2;
             l_run[j][1] += p1 + p3;
-            m_run[j][0] = mn_a;
-            m_run[j][1] = mn_b;
             // high and residual bf16 parts, transposed into the B layout
             bh[j][0] = movmatrix_trans(pack_bf16(p0, p1));
             bh[j][1] = movmatrix_trans(pack_bf16(p2, p3));

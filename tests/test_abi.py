@@ -135,15 +135,22 @@ def test_split_checks(lib):
 
 
 def test_plan_split_tokens(lib):
-    # contiguous, Llama-2-70B layer: 32 x 8 = 256 units >= 1.5 per SM on 148 SMs: one split
+    # contiguous, Llama-2-70B layer: 32 x 8 = 256 units fill >= 3/4 of the
+    # 2 x 148 resident blocks: one split per unit
     d = _dims(batch=32, num_heads=64, num_kv_heads=8, head_dim=128, page_size=4096)
     assert gqa.gqa_plan_split_tokens(d, 4096, 148) == 4096
     assert gqa.gqa_plan_split_tokens(d, 4000, 148) == 4096      # rounded up to 128
-    # contiguous, too few units: just enough splits for 1.5 items per SM
-    assert gqa.gqa_plan_split_tokens(d, 4096, 200) == 2048      # 300 items wanted / 256 units -> 2
+    # 400 slots: 256 units are too few, but only one split per unit fits a wave
+    assert gqa.gqa_plan_split_tokens(d, 4096, 200) == 4096
+    assert gqa.gqa_plan_split_tokens(d, 4096, 400) == 2048      # SM counts are capped at 256: 512 slots, 2 splits
+    # one long sequence, 4 groups (r = 8, two blocks per SM): 74 splits, one wave of 296
     d1 = _dims(batch=1, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072)
-    t1 = gqa.gqa_plan_split_tokens(d1, 131072, 148)             # 56 splits -> 2432 tokens
-    assert t1 == 2432 and 4 * -(-131072 // t1) >= 1.4 * 148   # rounding to 128 tokens trims a few
+    t1 = gqa.gqa_plan_split_tokens(d1, 131072, 148)
+    assert t1 == 1792 and 4 * -(-131072 // t1) == 296
+    # MQA sweep (r = 32 runs one block per SM): 16 units -> 9 splits -> 144 items
+    d2 = _dims(batch=16, num_heads=32, num_kv_heads=1, head_dim=128, page_size=8192)
+    t2 = gqa.gqa_plan_split_tokens(d2, 8192, 148)
+    assert 16 * -(-8192 // t2) <= 148 and t2 == 1024
     # paged: equal-work ranges, or splits of 4096 above 1024 sequences
     d3 = _dims(batch=64, num_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=70000,
                max_pages_per_seq=2048)
