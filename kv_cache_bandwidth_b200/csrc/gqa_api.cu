@@ -93,7 +93,8 @@ struct Shape {
   int b, H, G, r, D, P, num_pages, max_pages;
   bool paged;
   long long capacity;
-  int nt, nhb;  // kernel variant: n8 head tiles per consumer warp, head blocks
+  int nt, nhb;  // kernel variant: n8 head tiles per consumer warp, head blocks of 8
+  int rc, hs;   // heads per block (min(r, 16)) and 16-head slices per group
   bool fma;     // q.k and p.v on CUDA cores instead of tensor cores
 };
 
@@ -103,7 +104,7 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh) {
   if (!dims) return GQA_ERR_NULL_POINTER;
   const gqa_dims &d = *dims;
   if (d.batch < 1 || d.num_heads < 1 || d.num_kv_heads < 1 || d.page_size < 1) return GQA_ERR_DIMS;
-  if (d.batch > 65535 || d.num_kv_heads > 65535) return GQA_ERR_DIMS;  // grid y/z limits
+  if (d.batch > 65535 || d.num_kv_heads > 16383) return GQA_ERR_DIMS;  // grid y/z limits (G x 4 slices)
   if (d.num_heads % d.num_kv_heads != 0) return GQA_ERR_HEADS;
   const int r = d.num_heads / d.num_kv_heads;
   if (r > GQA_MAX_GROUP_RATIO) return GQA_ERR_HEADS;
@@ -132,8 +133,13 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh) {
   }
   if (s.capacity > (1ll << 30)) return GQA_ERR_DIMS;
   if (static_cast<long long>(s.b) * s.H * s.D > (1ll << 31) - 1) return GQA_ERR_DIMS;
-  s.nt = r <= 8 ? 1 : 2;
-  s.nhb = r <= 16 ? 1 : (r <= 32 ? 2 : 4);
+  // A block serves at most 16 heads (two head blocks of 8); larger groups are
+  // cut into 16-head slices handled by separate blocks that stream the same
+  // KV range (the repeats of a tile are L2 hits).
+  s.rc = std::min(r, 16);
+  s.hs = (r + s.rc - 1) / s.rc;
+  s.nt = 1;
+  s.nhb = (s.rc + 7) / 8;
   s.fma = (d.flags & GQA_FLAG_CONTRACT_FMA) != 0;
   if (s.fma && r > 2) return GQA_ERR_HEADS;  // the CUDA-core contraction covers r <= 2
   *sh = s;
@@ -156,6 +162,8 @@ struct Workspace {
   size_t o_bytes, m_bytes, total;
 };
 
+long long units_of(const Shape &sh) { return static_cast<long long>(sh.b) * sh.G * sh.hs; }
+
 Workspace workspace_layout(const Shape &sh, int num_splits) {
   Workspace w;
   const size_t rows = static_cast<size_t>(sh.b) * sh.H * num_splits;
@@ -169,7 +177,7 @@ Workspace workspace_layout(const Shape &sh, int num_splits) {
 // unit) when the units give about 1.5 blocks per SM; otherwise the smallest
 // power of two (at most 16) that does, never more blocks than 128-token tiles.
 int cluster_plan(const Shape &sh, int sms) {
-  const long long units = static_cast<long long>(sh.b) * sh.G;
+  const long long units = units_of(sh);
   const long long want = (3ll * sms + 1) / 2;
   const long long max_by_len = std::max<long long>(1, sh.capacity / 128);
   int c = 1;
@@ -242,7 +250,7 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
 }
 
 Pipe pick_pipe(const Shape &sh) {
-  if (sh.nt != 1) return Pipe::kSolo;
+  if (sh.nhb != 1) return Pipe::kDual;
   switch (GQA_PIPE_POLICY) {
     case 1: return Pipe::kSolo;
     case 3: return Pipe::kTrio;
@@ -256,17 +264,11 @@ int launch_decode_d(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &t
   if (sh.fma)
     return sh.r == 1 ? launch_decode_t<D, 1, 1, 3, PAGED, MODE, 1>(tk, tv, p, l)
                      : launch_decode_t<D, 1, 1, 3, PAGED, MODE, 2>(tk, tv, p, l);
-  if (sh.nt == 1) {
-    switch (pick_pipe(sh)) {
-      case Pipe::kTrio: return launch_decode_t<D, 1, 1, 2, PAGED, MODE>(tk, tv, p, l);
-      case Pipe::kSolo: return launch_decode_t<D, 1, 1, 6, PAGED, MODE>(tk, tv, p, l);
-      default: return launch_decode_t<D, 1, 1, 3, PAGED, MODE>(tk, tv, p, l);
-    }
-  }
-  switch (sh.nhb) {
-    case 1: return launch_decode_t<D, 2, 1, 3, PAGED, MODE>(tk, tv, p, l);
-    case 2: return launch_decode_t<D, 2, 2, 4, PAGED, MODE>(tk, tv, p, l);
-    default: return launch_decode_t<D, 2, 4, 4, PAGED, MODE>(tk, tv, p, l);
+  if (sh.nhb == 2) return launch_decode_t<D, 1, 2, 3, PAGED, MODE>(tk, tv, p, l);
+  switch (pick_pipe(sh)) {
+    case Pipe::kTrio: return launch_decode_t<D, 1, 1, 2, PAGED, MODE>(tk, tv, p, l);
+    case Pipe::kSolo: return launch_decode_t<D, 1, 1, 6, PAGED, MODE>(tk, tv, p, l);
+    default: return launch_decode_t<D, 1, 1, 3, PAGED, MODE>(tk, tv, p, l);
   }
 }
 
@@ -302,6 +304,8 @@ DecodeParams base_params(const Shape &sh, const void *q, const int32_t *seqlens,
   p.H = sh.H;
   p.G = sh.G;
   p.r = sh.r;
+  p.rc = sh.rc;
+  p.hs = sh.hs;
   p.page_size = sh.P;
   p.num_pages = sh.num_pages;
   p.max_pages = sh.max_pages;
@@ -326,7 +330,7 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   p.capacity = capacity;
   p.split_tokens = split_tokens;
   p.num_splits = num_splits;
-  const long long items = static_cast<long long>(sh.b) * sh.G * num_splits;
+  const long long items = units_of(sh) * num_splits;
   if (items > (1ll << 31) - 1) return GQA_ERR_DIMS;
   Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream};
   return launch_decode<Mode::kItems>(sh, tk, tv, p, l);
@@ -343,9 +347,9 @@ struct BalancedWorkspace {
 
 BalancedWorkspace balanced_layout(const Shape &sh) {
   BalancedWorkspace w;
-  const size_t rows = static_cast<size_t>(kMaxBalancedBlocks) * 2 * sh.r;
+  const size_t rows = static_cast<size_t>(kMaxBalancedBlocks) * 2 * sh.rc;
   w.meta_off = 256;
-  w.o_off = w.meta_off + round256(static_cast<size_t>(sh.b) * sh.G * 16);
+  w.o_off = w.meta_off + round256(static_cast<size_t>(units_of(sh)) * 16);
   w.m_off = w.o_off + round256(rows * sh.D * sizeof(float));
   w.l_off = w.m_off + round256(rows * sizeof(float));
   w.total = w.l_off + round256(rows * sizeof(float));
@@ -353,7 +357,7 @@ BalancedWorkspace balanced_layout(const Shape &sh) {
 }
 
 size_t auto_workspace_bytes(const Shape &sh, int max_seqlen) {
-  const long long units = static_cast<long long>(sh.b) * sh.G;
+  const long long units = units_of(sh);
   const long long by_sms = 3ll * 256;  // one wave of up to three blocks per SM on GPUs of up to 256 SMs
   long long splits = std::max<long long>((max_seqlen + kFallbackSplit - 1) / kFallbackSplit,
                                          (by_sms + units - 1) / units);
@@ -400,8 +404,10 @@ int run_balanced_combine(const Shape &sh, const int32_t *seqlens, float *out, ui
   c.H = sh.H;
   c.G = sh.G;
   c.r = sh.r;
+  c.rc = sh.rc;
+  c.hs = sh.hs;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(sh.b * sh.H), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(units_of(sh) * sh.rc), 1, 1);
   cfg.blockDim = dim3(128, 1, 1);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -438,15 +444,12 @@ int round_split(long long tokens) {
 // shared memory allows two blocks of the 3-stage ring; the 288- and 544-thread
 // variants for r > 16 fit once by registers).
 int blocks_per_sm(const Shape &sh) {
-  if (sh.fma) return 2;
-  if (sh.nt == 1) {
-    switch (pick_pipe(sh)) {
-      case Pipe::kTrio: return 3;
-      case Pipe::kSolo: return 1;
-      default: return 2;
-    }
+  if (sh.fma || sh.nhb != 1) return 2;
+  switch (pick_pipe(sh)) {
+    case Pipe::kTrio: return 3;
+    case Pipe::kSolo: return 1;
+    default: return 2;
   }
-  return sh.nhb == 1 ? 2 : 1;
 }
 
 AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
@@ -456,7 +459,7 @@ AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
   }
   // One block per unit when the units fill three quarters of the resident
   // slots; otherwise as many splits as still fit one wave.
-  const long long units = static_cast<long long>(sh.b) * sh.G;
+  const long long units = units_of(sh);
   const long long slots = static_cast<long long>(sms) * blocks_per_sm(sh);
   const long long splits = 4 * units >= 3 * slots ? 1 : std::max<long long>(1, slots / units);
   return {false, round_split((max_seqlen + splits - 1) / splits)};
@@ -587,7 +590,7 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
   if ((rc = encode_maps(sh, k_cache, v_cache, &tk, &tv)) != GQA_OK) return rc;
   DecodeParams p = base_params(sh, q, seqlens, page_table, status, scale);
   p.out = out;
-  Launch l{dim3(c, sh.G, sh.b), c, st};
+  Launch l{dim3(c, sh.G * sh.hs, sh.b), c, st};
   return launch_decode<Mode::kCluster>(sh, tk, tv, p, l);
 }
 

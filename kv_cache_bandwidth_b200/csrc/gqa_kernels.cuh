@@ -76,6 +76,7 @@ struct DecodeParams {
   int *ws_header;             // balanced mode: {decode blocks, capacity, W lo, W hi} for the combine
   int4 *ws_meta;              // balanced mode: per unit {first block, last block, slot in first block}
   int H, G, r;                // query heads, KV groups, heads per group
+  int rc, hs;                 // heads per block (min(r, 16)) and head slices per group (ceil(r / rc))
   int page_size;              // paged: tokens per page; contiguous: capacity m
   int num_pages;              // paged: pages in the pool
   int max_pages;              // paged: page-table row stride
@@ -94,7 +95,7 @@ struct CombineParams {
   const float *part_l;
   uint32_t *status;
   int b, H, max_len, split_tokens, num_splits;
-  int G, r;                   // balanced mode
+  int G, r, rc, hs;           // balanced mode
   const int *ws_header;       // balanced mode: {decode blocks, capacity, W lo, W hi}
   const int4 *ws_meta;        // balanced mode: per unit {first block, last block, slot in first block}
 };
@@ -151,6 +152,7 @@ __device__ __forceinline__ uint32_t keep_halves(uint32_t v, bool keep_lo, bool k
 // sequence s, and where its result goes.
 struct Piece {
   int s, g, len, k, t_begin, t_end;
+  int j, h0, nh;       // head slice j of the group: heads h0 .. h0 + nh - 1
   bool len_ok;
   bool final_row;      // balanced mode: the piece is the whole unit
   int slot;            // balanced mode: partial-state slot (2 per block)
@@ -164,14 +166,19 @@ __device__ __forceinline__ Piece make_item(const DecodeParams &p) {
   if (MODE == Mode::kItems) {
     const int i = blockIdx.x;
     it.k = i % p.num_splits;
-    const int sg = i / p.num_splits;
+    const int t = i / p.num_splits;
+    it.j = t % p.hs;
+    const int sg = t / p.hs;
     it.g = sg % p.G;
     it.s = sg / p.G;
   } else {
     it.k = blockIdx.x;
-    it.g = blockIdx.y;
+    it.g = blockIdx.y / p.hs;
+    it.j = blockIdx.y % p.hs;
     it.s = blockIdx.z;
   }
+  it.h0 = it.j * p.rc;
+  it.nh = min(p.rc, p.r - it.h0);
   it.len = __ldg(p.seqlens + it.s);
   it.len_ok = it.len >= 1 && it.len <= p.capacity;
   it.t_begin = 0;
@@ -212,15 +219,15 @@ __device__ __forceinline__ long long warp_sum64(long long v) {
 // unit order (sequence-major, group-minor).  Every lane of the warp calls it
 // and gets the same answer.
 template <int T>
-__device__ __forceinline__ long long total_tiles(const int32_t *seqlens, int b, int G, int capacity,
-                                                 int lane) {
+__device__ __forceinline__ long long total_tiles(const int32_t *seqlens, int b, int units_per_seq,
+                                                 int capacity, int lane) {
   long long tot = 0;
   for (int base = 0; base < b; base += 32) {
     const int s = base + lane;
     int len;
     tot += (s < b) ? unit_tiles<T>(seqlens, capacity, s, &len) : 0;
   }
-  return warp_sum64(tot) * G;
+  return warp_sum64(tot) * units_per_seq;
 }
 
 // Walks the pieces of this block's range in balanced mode.
@@ -228,18 +235,18 @@ struct Walker {
   long long remaining;  // tiles of the range not handed out yet
   long long pos;        // global index of the next tile handed out
   long long W;          // tiles of all units
-  int s, g, tile_in, tiles_s, len_s, count;
+  int s, g, j, tile_in, tiles_s, len_s, count;
 };
 
 template <int T>
 __device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, int lane) {
-  const long long W = total_tiles<T>(p.seqlens, p.b, p.G, p.capacity, lane);
+  const long long W = total_tiles<T>(p.seqlens, p.b, p.G * p.hs, p.capacity, lane);
   const long long N = gridDim.x, c = blockIdx.x;
   const long long start = c * W / N;
   wk.remaining = (c + 1) * W / N - start;
   wk.pos = start;
   wk.W = W;
-  wk.s = wk.g = wk.tile_in = wk.tiles_s = wk.len_s = wk.count = 0;
+  wk.s = wk.g = wk.j = wk.tile_in = wk.tiles_s = wk.len_s = wk.count = 0;
   if (wk.remaining <= 0) {
     wk.remaining = 0;
     return;
@@ -248,7 +255,8 @@ __device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, i
   for (int base = 0; base < p.b; base += 32) {
     const int s = base + lane;
     int len = 0;
-    const long long t = (s < p.b) ? static_cast<long long>(unit_tiles<T>(p.seqlens, p.capacity, s, &len)) * p.G : 0;
+    const long long t =
+        (s < p.b) ? static_cast<long long>(unit_tiles<T>(p.seqlens, p.capacity, s, &len)) * p.G * p.hs : 0;
     long long inc = t;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -264,7 +272,9 @@ __device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, i
       wk.len_s = __shfl_sync(0xffffffffu, len, L);
       wk.tiles_s = (wk.len_s + T - 1) / T;
       const long long in_seq = start - before;
-      wk.g = static_cast<int>(in_seq / wk.tiles_s);
+      const int unit_in_seq = static_cast<int>(in_seq / wk.tiles_s);
+      wk.g = unit_in_seq / p.hs;
+      wk.j = unit_in_seq % p.hs;
       wk.tile_in = static_cast<int>(in_seq % wk.tiles_s);
       return;
     }
@@ -279,6 +289,9 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
   const int take = static_cast<int>(min(static_cast<long long>(wk.tiles_s - wk.tile_in), wk.remaining));
   pc.s = wk.s;
   pc.g = wk.g;
+  pc.j = wk.j;
+  pc.h0 = wk.j * p.rc;
+  pc.nh = min(p.rc, p.r - pc.h0);
   pc.k = 0;
   pc.len = wk.len_s;
   pc.len_ok = true;
@@ -298,10 +311,13 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
   wk.tile_in = 0;
   if (wk.remaining > 0) {
     do {
-      if (++wk.g == p.G) {
-        wk.g = 0;
-        ++wk.s;
-        wk.tiles_s = unit_tiles<T>(p.seqlens, p.capacity, wk.s, &wk.len_s);
+      if (++wk.j == p.hs) {
+        wk.j = 0;
+        if (++wk.g == p.G) {
+          wk.g = 0;
+          ++wk.s;
+          wk.tiles_s = unit_tiles<T>(p.seqlens, p.capacity, wk.s, &wk.len_s);
+        }
       }
     } while (wk.tiles_s == 0);
   }
@@ -332,7 +348,7 @@ __device__ __forceinline__ int consume_fma(const DecodeParams &p, const Piece &p
   constexpr int kTileBytes = T * D * 2;
   const int ws = warp % NWT;
   const int tk = lane >> 1, half = lane & 1;
-  const int r = p.r;
+  const int r = pc.nh;
   const float sl = p.scale_log2;
 
   uint32_t qf[kRMax][kPairs];
@@ -538,9 +554,9 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       // Nothing to read.  An invalid length is handled once, by split 0: zero
       // rows in `out` and a marker in split 0 for the combine.
       if (!pc.len_ok && pc.k == 0) {
-        for (int idx = threadIdx.x; idx < p.r * (D / 4); idx += blockDim.x) {
+        for (int idx = threadIdx.x; idx < pc.nh * (D / 4); idx += blockDim.x) {
           const int h = idx / (D / 4), c4 = idx % (D / 4);
-          const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + h;
+          const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
           if (p.out) reinterpret_cast<float4 *>(p.out + row * D)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLBadLength;
         }
@@ -588,7 +604,6 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
     const int ppt = PAGED ? max(1, T / P) : 1;  // pages per tile
     const int br = PAGED ? min(P, T) : T;        // rows per TMA box
     const uint32_t box_bytes = static_cast<uint32_t>(TL::kHalves * br * 128);
-    const uint32_t q_bytes = static_cast<uint32_t>(p.r * D * 2);
     int tile = 0;  // tiles issued (ring position)
     int n = 0;     // pieces started (q slot position)
     while (have) {
@@ -606,10 +621,11 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         }
       }
       if (lane == 0) {
+        const uint32_t q_bytes = static_cast<uint32_t>(pc.nh * D * 2);
         mbar_arrive_expect_tx(bar_qfull + 8 * qs, q_bytes);
         bulk_load(q_sm + qs * TL::kQBytes,
-                  p.q + (static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r) * D, q_bytes,
-                  bar_qfull + 8 * qs);
+                  p.q + (static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0) * D,
+                  q_bytes, bar_qfull + 8 * qs);
       }
       ++n;
       // ---- K/V tiles
@@ -728,7 +744,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         const int hl = hb * TL::kHB + j * 8 + g8;
-        const bool valid = hl < p.r;
+        const bool valid = hl < pc.nh;
         const uint32_t qrow = q_sm + qs * TL::kQBytes + (valid ? hl : 0) * D * 2;
 #pragma unroll
         for (int ks = 0; ks < TL::kSteps; ++ks) {
@@ -749,10 +765,11 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         for (int mt = 0; mt < TL::kSteps; ++mt) o[mt][j][0] = o[mt][j][1] = o[mt][j][2] = o[mt][j][3] = 0.f;
       }
 
-      for (int t0 = pc.t_begin; t0 < pc.t_end && !*abort_flag; t0 += T, ++tile) {
+      for (int t0 = pc.t_begin; t0 < pc.t_end; t0 += T, ++tile) {
         const int stage = tile % STAGES;
-        bool ok = mbar_wait(bar_full + 8 * stage, (tile / STAGES) & 1);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        // every lane polls the barrier; an abort elsewhere shows up here as a
+        // wait that runs out
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_full + 8 * stage, (tile / STAGES) & 1));
         if (!ok) {
           if (lane == 0) {
             *abort_flag = 1;
@@ -951,7 +968,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       // ---- results of the piece
       if (BAL && ctid == 0) {
         if (pc.first_of_unit)
-          p.ws_meta[static_cast<size_t>(pc.s) * p.G + pc.g] =
+          p.ws_meta[(static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j] =
               make_int4(static_cast<int>(blockIdx.x), pc.last_block, pc.slot & 1, 0);
       }
       if (MODE != Mode::kCluster) {
@@ -961,15 +978,16 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         size_t pslot_stride = 1;
         if (BAL) {
           final_row = pc.final_row;
-          pslot_base = static_cast<size_t>(pc.slot) * p.r;
+          pslot_base = static_cast<size_t>(pc.slot) * p.rc;
         } else {
           final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
-          pslot_base = (static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r) * p.num_splits + pc.k;
+          pslot_base =
+              (static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0) * p.num_splits + pc.k;
           pslot_stride = p.num_splits;
         }
-        for (int idx = ctid; idx < p.r * n4; idx += nc * 32) {
+        for (int idx = ctid; idx < pc.nh * n4; idx += nc * 32) {
           const int h = idx / n4, c4 = idx % n4;
-          const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + h;
+          const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
           const float4 src = *reinterpret_cast<const float4 *>(osum + h * TL::kOStride + 4 * c4);
           if (final_row) {
             const float L = L_blk[h];
@@ -1002,7 +1020,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       if (pc.len_ok)
         for (int c = 0; c < nb; ++c) bad |= *cluster.map_shared_rank(const_cast<int *>(item_bad), c);
       const int n4 = D / 4;
-      for (int idx = threadIdx.x; idx < p.r * n4; idx += blockDim.x) {
+      for (int idx = threadIdx.x; idx < pc.nh * n4; idx += blockDim.x) {
         const int h = idx / n4, c4 = idx % n4;
         float L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1023,7 +1041,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         }
         float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
         if (L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
-        const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + h;
+        const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
         reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
       }
       if (threadIdx.x == 0 && !pc.len_ok && p.status) atomicOr(p.status, kStatusBadSeqlen);
@@ -1165,10 +1183,12 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p)
 // are final already; units with an invalid length get zero rows here.
 template <int D, int T>
 __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const CombineParams p) {
-  const int u = blockIdx.x / p.r;
-  const int h = blockIdx.x % p.r;
-  const int s = u / p.G, g = u % p.G;
-  const size_t row = static_cast<size_t>(s) * p.H + static_cast<size_t>(g) * p.r + h;
+  const int u = blockIdx.x / p.rc;  // unit: (sequence, group, head slice)
+  const int h = blockIdx.x % p.rc;
+  const int j = u % p.hs;
+  const int s = u / (p.G * p.hs), g = (u / p.hs) % p.G;
+  if (j * p.rc + h >= p.r) return;  // the last slice of the group is narrower
+  const size_t row = static_cast<size_t>(s) * p.H + static_cast<size_t>(g) * p.r + j * p.rc + h;
   float4 *dst = reinterpret_cast<float4 *>(p.out + row * D) + threadIdx.x % (D / 4);
   const int len = __ldg(p.seqlens + s);
   pdl_wait_primary();  // the header, unit records and partial states come from the decode kernel
@@ -1188,7 +1208,7 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
                [&](int k) -> long long {
                  const long long c = c_lo + k;
                  if (k > 0 && (c * W / N) == ((c + 1) * W / N)) return -1;  // empty range
-                 return (2 * c + (k == 0 ? slot_lo : 0)) * p.r + h;
+                 return (2 * c + (k == 0 ? slot_lo : 0)) * p.rc + h;
                },
                dst);
 }
