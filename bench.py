@@ -225,6 +225,23 @@ def reference_arm(args):
 
 # --------------------------------------------------------------------------- GPU leg
 
+class L2Flush:
+    """Empties L2 of the step's inputs: writes a buffer of twice the L2 size,
+    then reads another of the same size, so that L2 holds only clean lines of
+    data the step never touches (a write alone would leave ~126 MB of dirty
+    lines for the timed step to write back)."""
+
+    def __init__(self):
+        n = 2 * L2_BYTES // 4
+        self.w = torch.empty(n, dtype=torch.float32, device="cuda")
+        self.r = torch.ones(n, dtype=torch.float32, device="cuda")
+        self.sink = None
+
+    def __call__(self):
+        self.w.zero_()
+        self.sink = self.r.sum()
+
+
 def config_dict(w, inp, split_tokens):
     kv = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
     if split_tokens is None:
@@ -238,7 +255,7 @@ def config_dict(w, inp, split_tokens):
         "layout": "paged P=%d" % w.page_size if w.paged else "contiguous [b,G,m,d]",
         "split_tokens": split_tokens, "decomposition": decomp, "kv_bytes_per_step": kv, "seed": w.seed,
         "l2": ("inputs %.0f MiB > 126 MB L2 (no flush)" % (kv / 2 ** 20)) if kv > 2 * L2_BYTES
-        else "L2 flushed between steps",
+        else "L2 flushed between steps (2x L2 written, then 2x L2 read)",
     }
 
 
@@ -258,9 +275,7 @@ def main_gpu(args):
     out = torch.empty(inp.q.shape, dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
-    flush = None
-    if kv_step <= 2 * L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush = L2Flush() if kv_step <= 2 * L2_BYTES else None
 
     def step():
         if args.entry == "cluster":
@@ -271,15 +286,12 @@ def main_gpu(args):
                                  split_tokens=split, max_seqlen=max_seqlen, workspace=ws, out=out,
                                  status=status)
 
-    # decode kernel + combine kernel; the fixed-split combine is skipped when
-    # every sequence fits in one split
+    # fixed splits, at most 16 of them: one launch (the decode kernel merges
+    # each unit's splits itself); more splits or equal-work ranges: decode
+    # kernel + combine kernel
     eff_split = split if split > 0 else gqa.gqa_plan_split_tokens(dims, max_seqlen)
-    if args.entry == "cluster":
-        launches_per_step = 1
-    elif eff_split > 0 and -(-max_seqlen // eff_split) == 1:
-        launches_per_step = 1
-    else:
-        launches_per_step = 2
+    n_splits = -(-max_seqlen // eff_split) if eff_split > 0 else 0
+    launches_per_step = 1 if (args.entry == "cluster" or 0 < n_splits <= gqa.SERIAL_MERGE_MAX_SPLITS) else 2
 
     # ---- warm-up
     for _ in range(args.warmup):
@@ -309,7 +321,7 @@ def main_gpu(args):
             barrier(world)
             torch.cuda.synchronize()
             for a, b in evs:
-                flush.zero_()
+                flush()
                 a.record(stream)
                 step()
                 b.record(stream)
@@ -323,28 +335,31 @@ def main_gpu(args):
     hbm, hbm_kind = peaks()
 
     # ---- dominant kernel alone (decode kernel), CUDA events on its stream
-    kern_ms = None
-    if args.entry == "split":
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(max(args.steps, 10))]
-        for a, b in evs:
-            if flush is not None:
-                flush.zero_()
-            a.record(stream)
-            gqa.gqa_split_partials(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
-                                   split_tokens=split, max_seqlen=max_seqlen, workspace=ws, out=out,
-                                   status=status)
-            b.record(stream)
-        torch.cuda.synchronize()
-        kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    else:
-        kern_ms = ms_per_step
+    # (one launch per step: the step's own launch, timed alone; two: the decode
+    # kernel without the combine)
+    def decode_only():
+        gqa.gqa_split_partials(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                               split_tokens=split, max_seqlen=max_seqlen, workspace=ws, out=out,
+                               status=status)
+
+    kern = step if launches_per_step == 1 else decode_only
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(max(args.steps, 10))]
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record(stream)
+        kern()
+        b.record(stream)
+    torch.cuda.synchronize()
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
     kern_ms = max_over_ranks(kern_ms, world)
     achieved = kv_step / (kern_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": recorded_traffic(args.workload),
                 "kernel": ("gqa_decode_kernel (equal-work ranges)" if eff_split == 0 else
-                           "gqa_decode_kernel (fixed splits)") if args.entry == "split"
+                           "gqa_decode_kernel (fixed splits%s)" % (", merged in-kernel" if launches_per_step == 1
+                                                                    else "")) if args.entry == "split"
                 else "gqa_decode_kernel (gqa_decode)", "peak_kind": hbm_kind,
                 "kernel_us": kern_ms * 1e3, "algorithmic_bytes_per_launch": kv_step}
 

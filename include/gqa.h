@@ -123,14 +123,18 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
 
 /*
  * Split-KV decode.  The tokens of every sequence are cut into consecutive
- * splits of `split_tokens`; a persistent grid walks the (sequence, group,
- * split) items, each yielding an unnormalised partial softmax state, and a
- * second kernel merges the splits of each (sequence, head) exactly (it is not
- * launched when every sequence fits in one split): with m_k the split's running
- * maximum and l_k its sum of exponentials,
+ * splits of `split_tokens`; one thread block per (sequence, group, split)
+ * item yields an unnormalised partial softmax state, and the splits of each
+ * (sequence, head) are merged exactly: with m_k the split's running maximum
+ * and l_k its sum of exponentials,
  *     M = max_k m_k,  L = sum_k l_k 2^(m_k - M),  out = sum_k o_k 2^(m_k - M) / L.
- * The merge is an exact re-association of the softmax of the pages' formula
- * (the pages do not describe split-KV; it is how a long cache fills the GPU).
+ * With at most GQA_MERGE_IN_KERNEL_MAX_SPLITS splits the decode kernel merges
+ * them itself (one launch): each block publishes its state and counts its
+ * arrival in a per-unit word of the workspace, and the block that completes a
+ * unit merges the unit's rows.  With more splits a second kernel merges them,
+ * one block per row.  The merge is an exact re-association of the softmax of
+ * the pages' formula (the pages do not describe split-KV; it is how a long
+ * cache fills the GPU).
  *
  * split_tokens: a positive multiple of 128 (fixed splits as above), or 0 to
  *               let the library cut the work from the dims, max_seqlen and
@@ -152,8 +156,14 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
  * workspace:    device memory of at least gqa_decode_split_workspace_size()
  *               bytes for the same dims, max_seqlen and split_tokens, 16-byte
  *               aligned; its contents need no initialisation and are scratch
- *               after the call.
+ *               after the call.  Each call tags the arrival words with its
+ *               own number, so a word left by another call, or any other
+ *               contents, counts as no arrival; a call captured in a CUDA
+ *               graph keeps its number and every replay leaves the words
+ *               ready for the next.  Calls that overlap on the GPU must use
+ *               different workspaces.
  */
+#define GQA_MERGE_IN_KERNEL_MAX_SPLITS 8
 size_t gqa_decode_split_workspace_size(const gqa_dims *dims, int32_t max_seqlen,
                                        int32_t split_tokens);
 
@@ -167,7 +177,8 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache,
  * The two kernels of gqa_decode_split as separate calls (same arguments and
  * workspace): gqa_split_partials writes the per-split partial states into the
  * workspace; gqa_split_combine merges them into `out`.  Running the first and
- * then the second on one stream is exactly gqa_decode_split.  The combine is
+ * then the second on one stream gives exactly (bit for bit) the result of
+ * gqa_decode_split, which merges in-kernel with the same arithmetic.  The combine is
  * also the merge step for partial states produced elsewhere (e.g. gathered
  * from other GPUs into this workspace).  Both calls must get the same dims,
  * split_tokens and max_seqlen, on the same device.  When split_tokens == 0
@@ -188,6 +199,9 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache,
  * l [b, H, S] sum_j 2^(x_j - m), or a marker: -1 the split met an invalid page
  * id; -2 (split 0) the length is outside [1, capacity]; -3 (split 0) the row
  * is already final in `out`.
+ * Then one 64-bit arrival word per (sequence, group, 16-head slice) unit,
+ * {call number: 40 bits, arrivals: 24 bits}, used by gqa_decode_split's
+ * in-kernel merge only (gqa_split_partials leaves it alone).
  * Split k of sequence s covers tokens [k * split_tokens, min(len, (k+1) * split_tokens));
  * the combine reads the splits k < ceil(len / split_tokens).
  */

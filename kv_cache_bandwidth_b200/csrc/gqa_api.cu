@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -16,6 +17,9 @@
 
 #include "gqa.h"
 #include "gqa_kernels.cuh"
+
+static_assert(GQA_MERGE_IN_KERNEL_MAX_SPLITS == gqa::kSerialMergeMax,
+              "the header's in-kernel merge limit is the kernels' serial-merge limit");
 
 namespace {
 
@@ -158,8 +162,10 @@ int check_inputs(const void *q, const void *k, const void *v, const int32_t *seq
 // ------------------------------------------------------------------ workspace
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Fixed splits: o [b, H, S, d], m and l [b, H, S], then one 64-bit arrival
+// word per (sequence, group, head slice) unit for the decode kernel's own merge.
 struct Workspace {
-  size_t o_bytes, m_bytes, total;
+  size_t o_bytes, m_bytes, ctr_off, total;
 };
 
 long long units_of(const Shape &sh) { return static_cast<long long>(sh.b) * sh.G * sh.hs; }
@@ -169,8 +175,16 @@ Workspace workspace_layout(const Shape &sh, int num_splits) {
   const size_t rows = static_cast<size_t>(sh.b) * sh.H * num_splits;
   w.o_bytes = round256(rows * sh.D * sizeof(float));
   w.m_bytes = round256(rows * sizeof(float));
-  w.total = w.o_bytes + 2 * w.m_bytes;
+  w.ctr_off = w.o_bytes + 2 * w.m_bytes;
+  w.total = w.ctr_off + round256(static_cast<size_t>(units_of(sh)) * sizeof(unsigned long long));
   return w;
+}
+
+// Tag of one call in the arrival words, in [1, 2^40 - 2]: never 0 or all ones,
+// the two patterns a cleared or poisoned workspace holds.
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> counter{0};
+  return counter.fetch_add(1, std::memory_order_relaxed) % ((1ull << 40) - 2) + 1;
 }
 
 // Blocks per cluster for gqa_decode: 1 (one block per (sequence, group)
@@ -208,8 +222,20 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
   using TL = gqa::Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBalanced>;
   auto kernel = gqa::gqa_decode_kernel<D, NT, NHB, CH, STAGES, PAGED, MODE, FMA>;
   const int smem = TL::kSmemBytes;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return GQA_ERR_CUDA;
+  // The shared-memory limit is a per-device attribute of the function: set it
+  // once per device (a repeat is harmless, so two threads racing here is too).
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    if (MODE == Mode::kCluster &&
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    attr_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
   if (MODE == Mode::kBalanced) {
     // one block per resident slot of the GPU: grid.x holds the SM count on
     // entry and becomes SMs x blocks per SM (capped by the workspace)
@@ -226,10 +252,6 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
     cfg.numAttrs = 0;
     if (cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) != cudaSuccess) return GQA_ERR_CUDA;
     return static_cast<int>(l.grid.x);  // > 0: the number of decode blocks
-  }
-  if (MODE == Mode::kCluster && l.cluster > 8) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-      return GQA_ERR_CUDA;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = l.grid;
@@ -318,7 +340,7 @@ DecodeParams base_params(const Shape &sh, const void *q, const int32_t *seqlens,
 int run_items(const Shape &sh, const void *q, const void *k, const void *v, const int32_t *seqlens,
               const int32_t *pt, float *out, float scale, uint32_t *status, int split_tokens,
               int num_splits, int capacity, float *part_o, float *part_m, float *part_l,
-              cudaStream_t stream) {
+              unsigned long long *unit_ctr, cudaStream_t stream) {
   CUtensorMap tk, tv;
   int rc = encode_maps(sh, k, v, &tk, &tv);
   if (rc != GQA_OK) return rc;
@@ -330,6 +352,8 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   p.capacity = capacity;
   p.split_tokens = split_tokens;
   p.num_splits = num_splits;
+  p.unit_ctr = unit_ctr;
+  p.epoch = unit_ctr ? next_epoch() : 0;
   const long long items = units_of(sh) * num_splits;
   if (items > (1ll << 31) - 1) return GQA_ERR_DIMS;
   Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream};
@@ -500,14 +524,18 @@ int prepare_split(const gqa_dims *dims, bool paged, int32_t split_tokens, int32_
   return GQA_OK;
 }
 
+// merge_here: the decode kernel merges each unit's splits itself (the block
+// that completes a unit does it); otherwise the partial states are left for
+// gqa_split_combine.
 int run_partials(const SplitArgs &a, const void *q, const void *k, const void *v,
                  const int32_t *seqlens, const int32_t *pt, float *out, float scale, uint32_t *status,
-                 int32_t max_seqlen, void *workspace, cudaStream_t stream) {
+                 int32_t max_seqlen, void *workspace, bool merge_here, cudaStream_t stream) {
   uint8_t *w = static_cast<uint8_t *>(workspace);
   const int capacity = static_cast<int>(std::min<long long>(a.sh.capacity, max_seqlen));
   return run_items(a.sh, q, k, v, seqlens, pt, out, scale, status, a.split_tokens, a.num_splits,
                    capacity, reinterpret_cast<float *>(w), reinterpret_cast<float *>(w + a.ws.o_bytes),
-                   reinterpret_cast<float *>(w + a.ws.o_bytes + a.ws.m_bytes), stream);
+                   reinterpret_cast<float *>(w + a.ws.o_bytes + a.ws.m_bytes),
+                   merge_here ? reinterpret_cast<unsigned long long *>(w + a.ws.ctr_off) : nullptr, stream);
 }
 
 int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t *status,
@@ -584,7 +612,7 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
     // enough (sequence, group) units: one item each, final rows, no scratch
     const int split = static_cast<int>((sh.capacity + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum);
     return run_items(sh, q, k_cache, v_cache, seqlens, page_table, out, scale, status, split, 1,
-                     static_cast<int>(sh.capacity), nullptr, nullptr, nullptr, st);
+                     static_cast<int>(sh.capacity), nullptr, nullptr, nullptr, nullptr, st);
   }
   CUtensorMap tk, tv;
   if ((rc = encode_maps(sh, k_cache, v_cache, &tk, &tv)) != GQA_OK) return rc;
@@ -648,7 +676,7 @@ int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
   return run_partials(a, q, k_cache, v_cache, seqlens, page_table, out, scale, status, max_seqlen,
-                      workspace, st);
+                      workspace, false, st);
 }
 
 int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims, uint32_t *status,
@@ -708,9 +736,14 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, co
   if (rc != GQA_OK) return rc;
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+  // Up to kSerialMergeMax splits: one launch, single-split rows final in their
+  // block and the others merged by the block that completes their unit.  More
+  // splits: their merge is too much work for one block, the combine kernel
+  // spreads it over one block per row.
+  const bool merge_here = a.num_splits <= gqa::kSerialMergeMax;
   rc = run_partials(a, q, k_cache, v_cache, seqlens, page_table, out, scale, status, max_seqlen,
-                    workspace, st);
-  if (rc != GQA_OK || a.num_splits == 1) return rc;  // one split: rows are final already
+                    workspace, merge_here, st);
+  if (rc != GQA_OK || merge_here) return rc;
   return run_combine(a, seqlens, out, status, max_seqlen, workspace, st);
 }
 

@@ -75,6 +75,8 @@ struct DecodeParams {
   uint32_t *status;           // optional
   int *ws_header;             // balanced mode: {decode blocks, capacity, W lo, W hi} for the combine
   int4 *ws_meta;              // balanced mode: per unit {first block, last block, slot in first block}
+  unsigned long long *unit_ctr;  // items mode: arrival word per unit, or null (the merge is left to the combine)
+  unsigned long long epoch;      // items mode: this call's tag in the arrival words, 1 .. 2^40 - 2
   int H, G, r;                // query heads, KV groups, heads per group
   int rc, hs;                 // heads per block (min(r, 16)) and head slices per group (ceil(r / rc))
   int page_size;              // paged: tokens per page; contiguous: capacity m
@@ -128,10 +130,11 @@ struct Tile {
   static constexpr int kBarOff = (kMLOff + 4 * kMLFloats + 7) & ~7;
   static constexpr int kNumBars = 2 * STAGES + 2 * kQSlots;  // full, empty, q full, q empty
   static constexpr int kFlagOff = kBarOff + 8 * kNumBars;
-  static constexpr int kNumFlags = STAGES + 2;     // bad tile per stage, abort, item bad
+  static constexpr int kNumFlags = STAGES + 3;     // bad tile per stage, abort, item bad, merge here
   static constexpr int kSmemBytes = 1024 + kFlagOff + 4 * kNumFlags;
   static constexpr int kMinBlocks = STAGES <= 2 ? 3 : (STAGES == 3 ? 2 : 1);
   static_assert(BAL || kRPad * kOStride * 4 <= kRingBytes, "merge rows must fit in the ring");
+
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -322,6 +325,209 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
     } while (wk.tiles_s == 0);
   }
   return true;
+}
+
+// Merge the partial states (m_k, l_k, o_k) of one output row:
+//   M = max_k m_k,  L = sum_k l_k 2^(m_k - M),  out = sum_k o_k 2^(m_k - M) / L.
+// Built for latency: the contributions are taken in chunks of 512; for each
+// chunk every thread resolves one contribution's slot and loads its m and l
+// (all in flight together), the 128 threads reduce the maximum, each thread
+// turns its m into a weight, and then kNG groups of D/4 threads (one float4 of
+// the row each) add up the weighted o rows with precomputed addresses, several
+// loads in flight per thread.  Chunks are merged online (rescaled by
+// 2^(M_old - M_new)); the groups are summed in a fixed order, so the result is
+// deterministic and the same wherever it runs (combine kernel or the decode
+// kernel's own merge).  `slot(k)` is the index of contribution k in the m/l
+// arrays (< 0: no contribution).  Any l < 0 (an invalid page) makes the row
+// zero.  The partial states are read through L2 (they may come from other
+// blocks of the same grid).  128 threads (tid 0..127) take part; `sync` is
+// their barrier and `sc` their shared scratch.
+template <int D>
+struct MergeScratch {
+  static constexpr int kTPR = D / 4;        // threads per row (one float4 each)
+  static constexpr int kNG = 128 / kTPR;    // row groups
+  static constexpr int kChunk = 512;        // contributions per round
+  float4 acc[kNG][kTPR];
+  long long ps[kChunk];
+  float w[kChunk], l[kChunk];
+  float wmax[4], L[kNG];
+  int wbad[4];
+};
+
+template <int D, typename SlotFn, typename SyncFn>
+__device__ __forceinline__ void merge_row(const float *part_o, const float *part_m, const float *part_l,
+                                          int n_contrib, SlotFn slot, float4 *dst, int tid,
+                                          MergeScratch<D> &sc, SyncFn sync) {
+  using SC = MergeScratch<D>;
+  constexpr int kTPR = SC::kTPR;
+  constexpr int kNG = SC::kNG;
+  constexpr int kChunk = SC::kChunk;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  const int grp = tid / kTPR, c4 = tid % kTPR;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  float M = kNegInf;  // running maximum (the same in every thread)
+  float L = 0.f;      // this group's running sum of l weights
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int bad = 0;
+  for (int base = 0; base < n_contrib && !bad; base += kChunk) {
+    const int cnt = min(kChunk, n_contrib - base);
+    float mx = kNegInf;
+    int bd = 0;
+    for (int i = tid; i < cnt; i += 128) {
+      const long long ps = slot(base + i);
+      sc.ps[i] = ps;
+      float m = kNegInf, l = 0.f;
+      if (ps >= 0) {
+        m = __ldcg(part_m + ps);
+        l = __ldcg(part_l + ps);
+      }
+      sc.w[i] = m;
+      sc.l[i] = l;
+      mx = fmaxf(mx, m);
+      bd |= l < 0.f;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    bd = __any_sync(0xffffffffu, bd);
+    if (lane == 0) {
+      sc.wmax[warp] = mx;
+      sc.wbad[warp] = bd;
+    }
+    sync();
+    mx = fmaxf(fmaxf(sc.wmax[0], sc.wmax[1]), fmaxf(sc.wmax[2], sc.wmax[3]));
+    bad = sc.wbad[0] | sc.wbad[1] | sc.wbad[2] | sc.wbad[3];
+    if (!bad && mx != kNegInf) {
+      const float Mn = fmaxf(M, mx);
+      const float rescale = (M == kNegInf) ? 0.f : ex2(M - Mn);
+      L *= rescale;
+      acc.x *= rescale;
+      acc.y *= rescale;
+      acc.z *= rescale;
+      acc.w *= rescale;
+      M = Mn;
+      for (int i = tid; i < cnt; i += 128) sc.w[i] = (sc.ps[i] >= 0) ? ex2(sc.w[i] - Mn) : 0.f;
+      sync();
+#pragma unroll 8
+      for (int i = grp; i < cnt; i += kNG) {
+        const long long ps = sc.ps[i];
+        const float w = sc.w[i];
+        if (ps >= 0) {
+          const float4 v = __ldcg(reinterpret_cast<const float4 *>(part_o + ps * D) + c4);
+          acc.x += v.x * w;
+          acc.y += v.y * w;
+          acc.z += v.z * w;
+          acc.w += v.w * w;
+          L += sc.l[i] * w;
+        }
+      }
+    }
+    sync();  // the chunk's shared arrays are reused
+  }
+  sc.acc[grp][c4] = acc;
+  if (c4 == 0) sc.L[grp] = L;
+  sync();
+  if (grp == 0) {
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Lt = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNG; ++i) {
+      t.x += sc.acc[i][c4].x;
+      t.y += sc.acc[i][c4].y;
+      t.z += sc.acc[i][c4].z;
+      t.w += sc.acc[i][c4].w;
+      Lt += sc.L[i];
+    }
+    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!bad && Lt > 0.f) res = make_float4(t.x / Lt, t.y / Lt, t.z / Lt, t.w / Lt);
+    *dst = res;
+  }
+  sync();  // the scratch is free for the next row
+}
+
+// Items mode: counts one split's arrival at its (sequence, group, head slice)
+// unit.  The unit's 64-bit word holds {epoch: 40 bits, count: 24 bits}; a word
+// with another epoch (an earlier call, or whatever the workspace held) counts
+// as zero arrivals, so the workspace needs no clearing.  Returns true for the
+// arrival that makes `need`, which also leaves the word at {epoch, 0}, ready
+// for a repeat of the same launch (a replayed CUDA graph keeps its epoch).
+// The compare-and-swap loop always progresses (a failed swap means another
+// arrival succeeded); the bound only guards against a word that keeps
+// changing for some other reason.
+__device__ __forceinline__ bool unit_arrive(unsigned long long *word, unsigned long long epoch, int need,
+                                            uint32_t *status) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(word);
+  for (int i = 0; i < (1 << 20); ++i) {
+    const unsigned long long cnt = ((cur >> 24) == epoch) ? (cur & 0xffffffull) : 0ull;
+    const bool last = cnt + 1 == static_cast<unsigned long long>(need);
+    const unsigned long long nxt = (epoch << 24) | (last ? 0ull : cnt + 1);
+    const unsigned long long prev = atomicCAS(word, cur, nxt);
+    if (prev == cur) return last;
+    cur = prev;
+  }
+  if (status) atomicOr(status, kStatusTimeout);
+  return false;
+}
+
+// NV float4 outputs (columns 4*c4 .. 4*c4+3 for c4 = c4_0 + i*c4_step, i < NV)
+// of one merged row from the row's ns <= kSerialMergeMax partial states at
+// slots base .. base + ns - 1, for rows with few splits.  Every thread works
+// alone (no barriers) and issues all its loads before it uses any, so the
+// merge costs about one trip to L2; each output takes the contributions in
+// ascending k with one accumulator, the same whatever NV is.  The decode
+// kernel's own merge and the combine kernel both use it for such rows, so the
+// two agree bit for bit.
+constexpr int kSerialMergeMax = 8;
+
+template <int D, int NV>
+__device__ __forceinline__ void merge_serial(const float *part_o, const float *part_m, const float *part_l,
+                                             long long base, int ns, int c4_0, int c4_step, float4 *dst_row) {
+  const float kNegInf = -__int_as_float(0x7f800000);
+  float m[kSerialMergeMax], l[kSerialMergeMax];
+  float4 v[NV][kSerialMergeMax];
+#pragma unroll
+  for (int k = 0; k < kSerialMergeMax; ++k) {
+    const long long kk = base + min(k, ns - 1);  // every load issued (slots past ns repeat the last)
+    m[k] = __ldcg(part_m + kk);
+    l[k] = __ldcg(part_l + kk);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) v[i][k] = __ldcg(reinterpret_cast<const float4 *>(part_o + kk * D) + c4_0 + i * c4_step);
+  }
+  float M = kNegInf;
+  bool bad = false;
+#pragma unroll
+  for (int k = 0; k < kSerialMergeMax; ++k) {
+    if (k < ns) {
+      M = fmaxf(M, m[k]);
+      bad |= l[k] < 0.f;
+    }
+  }
+  float4 acc[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f;
+  if (!bad && M != kNegInf) {
+#pragma unroll
+    for (int k = 0; k < kSerialMergeMax; ++k) {
+      if (k < ns) {
+        const float w = ex2(m[k] - M);
+        L += l[k] * w;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          acc[i].x += v[i][k].x * w;
+          acc[i].y += v[i][k].y * w;
+          acc[i].z += v[i][k].z * w;
+          acc[i].w += v[i][k].w * w;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!bad && L > 0.f) res = make_float4(acc[i].x / L, acc[i].y / L, acc[i].z / L, acc[i].w / L);
+    dst_row[c4_0 + i * c4_step] = res;
+  }
 }
 
 // The q.k and p.v contractions on CUDA cores (fp32 FMA) for group ratios
@@ -542,6 +748,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TL::kFlagOff);  // [STAGES]
   volatile int *abort_flag = tile_bad + STAGES;
   volatile int *item_bad = tile_bad + STAGES + 1;
+  volatile int *merge_here = tile_bad + STAGES + 2;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1004,6 +1211,37 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
             }
           }
         }
+        if (!BAL && p.unit_ctr != nullptr && !final_row) {
+          // ---- the block whose split completes the unit merges its splits
+          // (the combine kernel's arithmetic, in this grid): publish this
+          // block's partial states, count the arrival, and if it was the last
+          // one read everyone's states back through L2.
+          // (the barrier orders every consumer thread's stores before thread
+          // 0's fence, which makes them visible GPU-wide before its arrival;
+          // its second fence orders the other blocks' states, published the
+          // same way, before the merge's loads, which the barrier releases)
+          named_barrier(1, nc * 32);
+          const int ns = (pc.len + p.split_tokens - 1) / p.split_tokens;
+          if (ctid == 0) {
+            __threadfence();
+            const size_t u = (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j;
+            *merge_here = unit_arrive(p.unit_ctr + u, p.epoch, ns, p.status) ? 1 : 0;
+            __threadfence();
+          }
+          named_barrier(1, nc * 32);
+          if (*merge_here) {
+            // all rows at once: each thread takes two float4 columns of one
+            // row (half a row apart), so rows x D/8 threads cover the block
+            constexpr int kHalf = D / 8;
+            static_assert(TL::kRPad * kHalf <= nc * 32, "one pass of the consumer threads");
+            const int h = ctid / kHalf, c4 = ctid % kHalf;
+            if (h < pc.nh) {
+              const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
+              merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(row) * p.num_splits, ns,
+                                 c4, kHalf, reinterpret_cast<float4 *>(p.out + row * D));
+            }
+          }
+        }
       }
       if (*abort_flag || !BAL) break;
       have = walker_next<T>(wk, p, pc);
@@ -1050,111 +1288,6 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
   }
 }
 
-// Merge the partial states (m_k, l_k, o_k) of one output row:
-//   M = max_k m_k,  L = sum_k l_k 2^(m_k - M),  out = sum_k o_k 2^(m_k - M) / L.
-// Built for latency: the contributions are taken in chunks of 512; for each
-// chunk every thread resolves one contribution's slot and loads its m and l
-// (all in flight together), the block reduces the maximum, each thread turns
-// its m into a weight, and then kNG groups of D/4 threads (one float4 of the
-// row each) add up the weighted o rows with precomputed addresses, several
-// loads in flight per thread.  Chunks are merged online (rescaled by
-// 2^(M_old - M_new)); the groups are summed in a fixed order, so the result is
-// deterministic.  `slot(k)` is the index of contribution k in the m/l arrays
-// (< 0: no contribution).  Any l < 0 (an invalid page) makes the row zero.
-template <int D, typename SlotFn>
-__device__ __forceinline__ void merge_row(const float *part_o, const float *part_m, const float *part_l,
-                                          int n_contrib, SlotFn slot, float4 *dst) {
-  constexpr int kTPR = D / 4;
-  constexpr int kNG = 128 / kTPR;
-  constexpr int kChunk = 512;
-  const float kNegInf = -__int_as_float(0x7f800000);
-  __shared__ long long s_ps[kChunk];
-  __shared__ float s_w[kChunk], s_l[kChunk];
-  __shared__ float s_wmax[4];
-  __shared__ int s_wbad[4];
-  __shared__ float4 s_acc[kNG][kTPR];
-  __shared__ float s_L[kNG];
-  const int tid = threadIdx.x, grp = tid / kTPR, c4 = tid % kTPR;
-  const int warp = tid >> 5, lane = tid & 31;
-
-  float M = kNegInf;  // running maximum (the same in every thread)
-  float L = 0.f;      // this group's running sum of l weights
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int bad = 0;
-  for (int base = 0; base < n_contrib && !bad; base += kChunk) {
-    const int cnt = min(kChunk, n_contrib - base);
-    float mx = kNegInf;
-    int bd = 0;
-    for (int i = tid; i < cnt; i += 128) {
-      const long long ps = slot(base + i);
-      s_ps[i] = ps;
-      float m = kNegInf, l = 0.f;
-      if (ps >= 0) {
-        m = part_m[ps];
-        l = part_l[ps];
-      }
-      s_w[i] = m;
-      s_l[i] = l;
-      mx = fmaxf(mx, m);
-      bd |= l < 0.f;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    bd = __any_sync(0xffffffffu, bd);
-    if (lane == 0) {
-      s_wmax[warp] = mx;
-      s_wbad[warp] = bd;
-    }
-    __syncthreads();
-    mx = fmaxf(fmaxf(s_wmax[0], s_wmax[1]), fmaxf(s_wmax[2], s_wmax[3]));
-    bad = s_wbad[0] | s_wbad[1] | s_wbad[2] | s_wbad[3];
-    if (!bad && mx != kNegInf) {
-      const float Mn = fmaxf(M, mx);
-      const float rescale = (M == kNegInf) ? 0.f : ex2(M - Mn);
-      L *= rescale;
-      acc.x *= rescale;
-      acc.y *= rescale;
-      acc.z *= rescale;
-      acc.w *= rescale;
-      M = Mn;
-      for (int i = tid; i < cnt; i += 128) s_w[i] = (s_ps[i] >= 0) ? ex2(s_w[i] - Mn) : 0.f;
-      __syncthreads();
-#pragma unroll 8
-      for (int i = grp; i < cnt; i += kNG) {
-        const long long ps = s_ps[i];
-        const float w = s_w[i];
-        if (ps >= 0) {
-          const float4 v = reinterpret_cast<const float4 *>(part_o + ps * D)[c4];
-          acc.x += v.x * w;
-          acc.y += v.y * w;
-          acc.z += v.z * w;
-          acc.w += v.w * w;
-          L += s_l[i] * w;
-        }
-      }
-    }
-    __syncthreads();  // the chunk's shared arrays are reused
-  }
-  s_acc[grp][c4] = acc;
-  if (c4 == 0) s_L[grp] = L;
-  __syncthreads();
-  if (grp == 0) {
-    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Lt = 0.f;
-#pragma unroll
-    for (int i = 0; i < kNG; ++i) {
-      t.x += s_acc[i][c4].x;
-      t.y += s_acc[i][c4].y;
-      t.z += s_acc[i][c4].z;
-      t.w += s_acc[i][c4].w;
-      Lt += s_L[i];
-    }
-    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (!bad && Lt > 0.f) res = make_float4(t.x / Lt, t.y / Lt, t.z / Lt, t.w / Lt);
-    *dst = res;
-  }
-}
-
 // Fixed splits: one block per (sequence, head) row merges the splits
 // k < ceil(len / split_tokens) of that row.
 template <int D>
@@ -1173,7 +1306,15 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p)
   const long long base = static_cast<long long>(row) * p.num_splits;
   // the decode kernel already wrote this row (a single split)
   if (ns == 1 && p.part_l[base] == kLFinal) return;
-  merge_row<D>(p.part_o, p.part_m, p.part_l, ns, [&](int k) -> long long { return base + k; }, dst);
+  if (ns <= kSerialMergeMax) {
+    if (threadIdx.x < D / 4)
+      merge_serial<D, 1>(p.part_o, p.part_m, p.part_l, base, ns, threadIdx.x, 0,
+                         reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D));
+    return;
+  }
+  __shared__ MergeScratch<D> sc;
+  merge_row<D>(p.part_o, p.part_m, p.part_l, ns, [&](int k) -> long long { return base + k; }, dst,
+               threadIdx.x, sc, [] { __syncthreads(); });
 }
 
 // Balanced mode: one block per (unit, head).  The decode kernel recorded, for
@@ -1204,13 +1345,14 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
   const int4 meta = p.ws_meta[u];
   const int c_lo = meta.x, c_hi = meta.y, slot_lo = meta.z;
   if (c_lo == c_hi) return;  // one decode block covered the unit: its rows are final
+  __shared__ MergeScratch<D> sc;
   merge_row<D>(p.part_o, p.part_m, p.part_l, c_hi - c_lo + 1,
                [&](int k) -> long long {
                  const long long c = c_lo + k;
                  if (k > 0 && (c * W / N) == ((c + 1) * W / N)) return -1;  // empty range
                  return (2 * c + (k == 0 ? slot_lo : 0)) * p.rc + h;
                },
-               dst);
+               dst, threadIdx.x, sc, [] { __syncthreads(); });
 }
 
 }  // namespace gqa

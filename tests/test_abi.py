@@ -33,6 +33,13 @@ def test_header_declares_entry_points():
         assert n in names
 
 
+def test_binding_constants_match_header():
+    text = open(HEADER).read()
+    defs = dict(re.findall(r"^#define\s+(GQA_\w+)\s+(.+?)\s*$", text, flags=re.M))
+    assert int(defs["GQA_MERGE_IN_KERNEL_MAX_SPLITS"]) == gqa.SERIAL_MERGE_MAX_SPLITS
+    assert eval(defs["GQA_STATIC_WORKSPACE_BYTES"].replace("u", "")) == gqa.STATIC_WORKSPACE_BYTES
+
+
 def test_library_exports_every_declared_symbol(lib):
     missing = [n for n in declared_functions() if not hasattr(lib, n)]
     assert not missing, missing
@@ -102,7 +109,10 @@ def test_workspace_size(lib):
     S = 131072 // 4096
     rows = 4 * 32 * S
     r256 = lambda x: (x + 255) // 256 * 256
-    assert gqa.gqa_decode_split_workspace_size(d, 131072, 4096) == r256(rows * 128 * 4) + 2 * r256(rows * 4)
+    # o [b,H,S,d] + m, l [b,H,S] (fp32) + one 8-byte arrival word per (sequence, group) unit
+    units = 4 * 4
+    assert gqa.gqa_decode_split_workspace_size(d, 131072, 4096) == (
+        r256(rows * 128 * 4) + 2 * r256(rows * 4) + r256(units * 8))
     assert gqa.gqa_decode_split_workspace_size(d, 131072, 100) == 0       # not a multiple of 128
     assert gqa.gqa_decode_split_workspace_size(d, 0, 4096) == 0
     # split_tokens = 0: equal-work ranges (header + 2 slots of r heads for up to

@@ -272,6 +272,98 @@ def test_decode_items_path_many_units():
         assert_parity(got, ref, "items path P=%s" % P)
 
 
+def _split_call(inp, ws, out, split, mx, st=None):
+    gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, split_tokens=split,
+                         max_seqlen=mx, workspace=ws, out=out, status=st)
+
+
+def test_in_kernel_merge_under_graph_replay():
+    """Fixed splits merge inside the decode kernel, counted through per-unit
+    arrival words tagged with the call.  A captured graph replays the same tag:
+    every replay (and an eager call in between, with a new tag, on the same
+    workspace) must give the eager result bit for bit."""
+    w = w_small(b=3, r=8, G=2, d=128, m=2048, P=16, seed=9)
+    inp = make_inputs(w, device="cuda", lens=[2048, 1000, 5])   # 16, 8 and 1 splits of 128
+    ref, _ = run_oracle(inp)
+    eager, st = run_gpu(inp, "split", split_tokens=128, max_seqlen=2048)
+    assert st == 0
+    assert_parity(eager, ref, "eager")
+    ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, 2048, 128).fill_(0xFF)
+    out = torch.full_like(eager, float("nan"))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        _split_call(inp, ws, out, 128, 2048)   # warm-up outside capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            _split_call(inp, ws, out, 128, 2048)
+    torch.cuda.synchronize()
+    for i in range(4):
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager), "replay %d" % i
+        if i == 1:   # an eager call with its own tag on the same workspace
+            out.fill_(float("nan"))
+            _split_call(inp, ws, out, 128, 2048)
+            torch.cuda.synchronize()
+            assert torch.equal(out, eager)
+    del g
+
+
+def test_in_kernel_merge_workspace_shared_between_shapes():
+    """One workspace serves calls of different split geometry in turn: the
+    arrival words one call leaves behind must not confuse the next."""
+    w = w_small(b=2, r=4, G=3, d=64, m=4096, seed=21)
+    inp = make_inputs(w, device="cuda", lens=[4096, 3000])
+    ref, _ = run_oracle(inp)
+    ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, 4096, 128).fill_(0xFF)
+    for split in (128, 1024, 256, 128, 4096, 384):
+        out = torch.full(inp.q.shape, float("nan"), dtype=torch.float32, device="cuda")
+        st = status_word()
+        _split_call(inp, ws, out, split, 4096, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert_parity(out, ref, "split %d" % split)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_more_than_512_splits(d):
+    """More splits than the combine kernel takes per round (512): it rescales
+    across rounds."""
+    w = w_small(b=1, r=16, G=1, d=d, m=70000, seed=31)
+    inp = make_inputs(w, device="cuda", lens=[70000])
+    ref, _ = run_oracle(inp)
+    got, st = run_gpu(inp, "split", split_tokens=128, max_seqlen=70000)   # 547 splits
+    assert st == 0
+    assert_parity(got, ref, "547 splits d=%d" % d)
+
+
+@pytest.mark.parametrize("n_splits", [7, 8, 9, 17])
+def test_split_count_at_in_kernel_merge_limit(n_splits):
+    """Up to 8 splits merge inside the decode kernel, more in the combine
+    kernel; both sides of the limit, and sequences of 1 .. n splits in one
+    batch.  The pair partials + combine must agree with the one call bit for
+    bit."""
+    m = 128 * n_splits
+    lens = [m, m - 127, 129, 128, 1, 3 * 128 + 5]
+    w = w_small(b=len(lens), r=16, G=2, d=128, m=m, P=32, seed=n_splits)
+    inp = make_inputs(w, device="cuda", lens=lens)
+    ref, _ = run_oracle(inp)
+    got, st = run_gpu(inp, "split", split_tokens=128, max_seqlen=m)
+    assert st == 0
+    assert_parity(got, ref, "%d splits" % n_splits)
+    ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, m, 128)
+    out = torch.full_like(got, float("nan"))
+    gqa.gqa_split_partials(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, split_tokens=128,
+                           max_seqlen=m, workspace=ws, out=out)
+    gqa.gqa_split_combine(inp.seqlens, out, gqa.dims_for(inp.q, inp.k_cache, inp.page_table),
+                          split_tokens=128, max_seqlen=m, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, got)
+
+
 def test_repeat_runs_bit_identical():
     inp = make_inputs(w_small(b=4, r=8, G=2, d=128, m=3000, P=32), device="cuda", lens=[3000, 2000, 10, 1500])
     for entry in ("cluster", "split"):
