@@ -68,6 +68,10 @@ def load_library(path: str):
         ctypes.c_double, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
         ctypes.c_void_p, ctypes.c_int32,
     ]
+    if hasattr(lib, "oracle_gqa_decode_lse"):
+        lib.oracle_gqa_decode_lse.restype = ctypes.c_int
+        lib.oracle_gqa_decode_lse.argtypes = lib.oracle_gqa_decode.argtypes[:16] + [ctypes.c_void_p] + \
+            lib.oracle_gqa_decode.argtypes[16:]
     lib.oracle_max_threads.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     return lib
@@ -126,6 +130,23 @@ def gqa_decode(q, k_cache, v_cache, seqlens, page_table=None, *, num_kv_heads: i
     Returns (out, status): out float64 [b, H, d] (or [len(rows), d]) and the OR of
     the status bits (1: a length outside [1, capacity]; 2: a page id outside the pool).
     """
+    out, _, status = _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows, threads,
+                             lib, want_lse=False)
+    return out, status
+
+
+def gqa_decode_lse(q, k_cache, v_cache, seqlens, page_table=None, *, num_kv_heads: int,
+                   scale: Optional[float] = None, rows=None, threads: int = 0,
+                   lib=None) -> Tuple[np.ndarray, np.ndarray, int]:
+    """``gqa_decode`` plus lse float64 [b, H] (or [len(rows)]): the natural log
+    of the row's softmax normaliser, ln sum_j exp(scale * q . k_j); -inf for a
+    row with a status bit.  Returns (out, lse, status)."""
+    return _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows, threads, lib,
+                   want_lse=True)
+
+
+def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows, threads, lib, want_lse):
+    """Shared body of gqa_decode and gqa_decode_lse."""
     qb = _as_bits(q)
     kb = _as_bits(k_cache)
     vb = _as_bits(v_cache)
@@ -153,13 +174,20 @@ def gqa_decode(q, k_cache, v_cache, seqlens, page_table=None, *, num_kv_heads: i
         nrows = rows_arr.shape[0]
     out = np.zeros((nrows, d), dtype=np.float64)
     status = np.zeros(1, dtype=np.int32)
-    rc = (lib or _load()).oracle_gqa_decode(
-        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, sl.ctypes.data,
-        None if pt is None else pt.ctypes.data, b, H, G, d, P, num_pages, max_pages,
-        float(scale), None if rows_arr is None else rows_arr.ctypes.data, nrows,
-        out.ctypes.data, status.ctypes.data, int(threads))
+    args = [qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, sl.ctypes.data,
+            None if pt is None else pt.ctypes.data, b, H, G, d, P, num_pages, max_pages,
+            float(scale), None if rows_arr is None else rows_arr.ctypes.data, nrows, out.ctypes.data]
+    lse = None
+    lib = lib or _load()
+    if want_lse:
+        lse = np.zeros(nrows, dtype=np.float64)
+        rc = lib.oracle_gqa_decode_lse(*args, lse.ctypes.data, status.ctypes.data, int(threads))
+    else:
+        rc = lib.oracle_gqa_decode(*args, status.ctypes.data, int(threads))
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     if rows is None:
         out = out.reshape(b, H, d)
-    return out, int(status[0])
+        if lse is not None:
+            lse = lse.reshape(b, H)
+    return out, lse, int(status[0])

@@ -14,6 +14,7 @@
  *   l_j   = scale * sum_k q[s,i,k] * K[s,g(i),j,k]      for j < len_s
  *   w_j   = exp(l_j - max_j l_j) / sum_j exp(l_j - max_j l_j)
  *   out[s,i,:] = sum_j w_j * V[s,g(i),j,:]
+ *   lse[s,i]   = ln sum_j exp(l_j)            (oracle_gqa_decode_lse only)
  *
  * Sources, by page and section:
  *  - "Grouped-Query Attention" (aiwiki), the PyTorch module: keys and values are
@@ -39,7 +40,11 @@
  *    row t % P.  A NULL page table means the contiguous cache [b, G, m, d],
  *    i.e. page_size = m and sequence s is "page" s;
  *  - invalid data: len_s < 1 or len_s > capacity sets bit 1 of *status and a
- *    page id outside [0, num_pages) sets bit 2; such a row is written as zeros.
+ *    page id outside [0, num_pages) sets bit 2; such a row is written as zeros
+ *    (and its lse as -infinity).
+ *  - lse is the logarithm of the softmax's normaliser, sum_j exp(l_j), the
+ *    quantity that lets softmax results over disjoint parts of a sequence be
+ *    combined (a reading: the pages' softmax defines it but does not name it).
  *
  * Inputs are bf16 bit patterns (uint16), expanded exactly to double; every sum
  * is accumulated in double in the logical token order j = 0, 1, ..., len_s - 1.
@@ -87,7 +92,8 @@ static long long kv_row_offset(const int32_t *page_table, int32_t s, int32_t t,
 }
 
 /*
- * Decode attention for the listed rows.
+ * Decode attention for the listed rows; `lse` (may be NULL) receives
+ * ln sum_j exp(l_j) per row.
  *
  * q        [b, H, d] bf16 bits
  * k_cache  [num_pages, G, page_size, d] bf16 bits (contiguous: [b, G, m, d])
@@ -101,13 +107,13 @@ static long long kv_row_offset(const int32_t *page_table, int32_t s, int32_t t,
  *
  * Returns 0, or -1 on bad arguments (nothing is written then).
  */
-int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache,
-                      const uint16_t *v_cache, const int32_t *seqlens,
-                      const int32_t *page_table, int32_t b, int32_t H, int32_t G,
-                      int32_t d, int32_t page_size, int32_t num_pages,
-                      int32_t max_pages_per_seq, double scale,
-                      const int64_t *rows, int64_t nrows, double *out,
-                      int32_t *status, int32_t nthreads)
+static int decode_rows(const uint16_t *q, const uint16_t *k_cache,
+                       const uint16_t *v_cache, const int32_t *seqlens,
+                       const int32_t *page_table, int32_t b, int32_t H, int32_t G,
+                       int32_t d, int32_t page_size, int32_t num_pages,
+                       int32_t max_pages_per_seq, double scale,
+                       const int64_t *rows, int64_t nrows, double *out, double *lse,
+                       int32_t *status, int32_t nthreads)
 {
     if (!q || !k_cache || !v_cache || !seqlens || !out || !status)
         return -1;
@@ -133,6 +139,8 @@ int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache,
         double *o = out + n * (int64_t)d;
         for (int32_t k = 0; k < d; ++k)
             o[k] = 0.0;
+        if (lse)
+            lse[n] = -INFINITY;
         if (row < 0 || row >= (int64_t)b * H) {
             status_all |= ORACLE_STATUS_BAD_SEQLEN;
             continue;
@@ -188,6 +196,9 @@ int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache,
             logits[t] = exp(logits[t] - mx);
             denom += logits[t];
         }
+        /* ln sum_j exp(l_j) = mx + ln sum_j exp(l_j - mx) */
+        if (lse)
+            lse[n] = mx + log(denom);
 
         /* out = sum_j w_j v_j */
         for (int32_t t = 0; t < len; ++t) {
@@ -201,6 +212,49 @@ int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache,
     }
     *status = status_all;
     return 0;
+}
+
+/*
+ * Arguments:
+ * q        [b, H, d] bf16 bits
+ * k_cache  [num_pages, G, page_size, d] bf16 bits (contiguous: [b, G, m, d])
+ * v_cache  same layout as k_cache
+ * seqlens  [b] cached length of each sequence (the new token included)
+ * page_table [b, max_pages_per_seq] int32, or NULL for the contiguous cache
+ * rows     list of flat row ids s * H + i, or NULL for all b * H rows
+ * out      [nrows, d] float64 (row order of `rows`)
+ * status   receives the OR of the status bits of every computed row
+ * nthreads number of OpenMP threads (<= 0: library default)
+ * Returns 0, or -1 on bad arguments (nothing is written then).
+ */
+int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache,
+                      const uint16_t *v_cache, const int32_t *seqlens,
+                      const int32_t *page_table, int32_t b, int32_t H, int32_t G,
+                      int32_t d, int32_t page_size, int32_t num_pages,
+                      int32_t max_pages_per_seq, double scale,
+                      const int64_t *rows, int64_t nrows, double *out,
+                      int32_t *status, int32_t nthreads)
+{
+    return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, H, G, d,
+                       page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
+                       out, NULL, status, nthreads);
+}
+
+/* The same, plus lse [nrows] = ln sum_j exp(l_j) of each row (-inf for a row
+ * with a status bit). */
+int oracle_gqa_decode_lse(const uint16_t *q, const uint16_t *k_cache,
+                          const uint16_t *v_cache, const int32_t *seqlens,
+                          const int32_t *page_table, int32_t b, int32_t H, int32_t G,
+                          int32_t d, int32_t page_size, int32_t num_pages,
+                          int32_t max_pages_per_seq, double scale,
+                          const int64_t *rows, int64_t nrows, double *out, double *lse,
+                          int32_t *status, int32_t nthreads)
+{
+    if (!lse)
+        return -1;
+    return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, H, G, d,
+                       page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
+                       out, lse, status, nthreads);
 }
 
 /* Number of OpenMP threads a parallel region would use by default. */

@@ -23,6 +23,13 @@ What each pin compares against:
     logical cache in permuted pages; NaN in slots past each length.
   * error handling -- invalid lengths and page ids set status bits, zero rows.
   * brute force -- tiny cases summed in pure Python with math.fsum.
+
+``LSE_PINS`` take ``oracle.gqa_decode_lse`` instead and pin the log of each
+row's softmax normaliser, ln sum_j exp(scale q.k_j): one token gives its own
+logit; q = 0 gives ln len; torch.logsumexp in float64 on the broadcast keys;
+math.fsum brute force; and the identity that joins disjoint shards of a
+sequence (out = sum_p e^(lse_p - LSE) out_p, LSE = ln sum_p e^(lse_p)), which
+ties each output to its lse.
 """
 from __future__ import annotations
 
@@ -326,3 +333,102 @@ PINS = [
     pin_position_permutation, pin_paged_equals_contiguous, pin_tail_poison,
     pin_status_and_zero_rows, pin_rows_subset, pin_group_map,
 ]
+
+
+# ----------------------------------------------------------------------------
+# the log-sum-exp of each row (decode_lse: the signature of oracle.gqa_decode_lse)
+
+
+def run_lse(decode_lse, inp, scale=None, **kw):
+    return decode_lse(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                      num_kv_heads=inp.workload.G, scale=scale, **kw)
+
+
+def pin_lse_single_token(decode_lse):
+    w = small(seed=41)
+    inp = make_inputs(w, lens=[1, 1])
+    scale = 0.37
+    _, lse, st = run_lse(decode_lse, inp, scale=scale)
+    assert st == 0
+    q, k = bf16_f64(inp.q).tolist(), bf16_f64(inp.k_cache).tolist()
+    for s in range(w.b):
+        for i in range(w.H):
+            logit = scale * math.fsum(a * b for a, b in zip(q[s][i], k[s][i // w.r][0]))
+            assert abs(lse[s, i] - logit) <= 1e-13 * max(1.0, abs(logit)), "len 1: lse is the logit"
+
+
+def pin_lse_uniform(decode_lse):
+    w = small(seed=43)
+    inp = make_inputs(w, lens=[37, 5])
+    inp.q.zero_()
+    _, lse, _ = run_lse(decode_lse, inp)
+    for s in range(w.b):
+        assert np.allclose(lse[s], math.log(int(inp.seqlens[s])), rtol=0, atol=1e-14), "q = 0: lse = ln len"
+
+
+def pin_lse_torch_logsumexp(decode_lse):
+    w = small(b=3, H=8, G=2, d=16, m=40, seed=47)
+    inp = make_inputs(w, lens=[40, 17, 3])
+    scale = 0.21
+    _, lse, _ = run_lse(decode_lse, inp, scale=scale)
+    q = bf16_f64(inp.q)
+    k = bf16_f64(inp.k_cache).repeat_interleave(w.H // w.G, dim=1)
+    logits = torch.einsum("bhd,bhmd->bhm", q, k) * scale
+    pos = torch.arange(k.shape[2])
+    logits = logits.masked_fill(~(pos[None, None, :] < inp.seqlens[:, None, None].to(torch.int64)), -math.inf)
+    assert_close(lse, torch.logsumexp(logits, dim=-1).numpy(), rtol=1e-13, atol=1e-13, what="logsumexp")
+
+
+def pin_lse_brute_force(decode_lse):
+    w = small(b=2, H=4, G=2, d=3, m=6, seed=53)
+    inp = make_inputs(w, lens=[6, 2])
+    scale = 1.3
+    _, lse, _ = run_lse(decode_lse, inp, scale=scale)
+    q, k = bf16_f64(inp.q).tolist(), bf16_f64(inp.k_cache).tolist()
+    for s in range(w.b):
+        L = int(inp.seqlens[s])
+        for i in range(w.H):
+            g = i // (w.H // w.G)
+            z = [scale * math.fsum(q[s][i][c] * k[s][g][j][c] for c in range(w.d)) for j in range(L)]
+            ref = math.log(math.fsum(math.exp(x) for x in z))
+            assert abs(lse[s, i] - ref) <= 1e-13 * max(1.0, abs(ref)), "brute-force lse"
+
+
+def pin_lse_joins_shards(decode_lse):
+    """A sequence cut into three disjoint token ranges, each decoded as its own
+    cache: weighting each range's output by e^(lse_p - LSE) gives the output of
+    the whole sequence, and LSE its lse."""
+    w = small(b=1, H=8, G=4, d=16, m=50, seed=59)
+    inp = make_inputs(w, lens=[50])
+    full, lse_full, _ = run_lse(decode_lse, inp)
+    cuts = [0, 7, 31, 50]
+    outs, lses = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        part = make_inputs(w.with_(m=b - a), lens=[b - a])
+        part.q.copy_(inp.q)
+        part.k_cache.copy_(inp.k_cache[:, :, a:b])
+        part.v_cache.copy_(inp.v_cache[:, :, a:b])
+        o, l, st = run_lse(decode_lse, part)
+        assert st == 0
+        outs.append(o)
+        lses.append(l)
+    lses = np.stack(lses)                                   # [3, b, H]
+    top = lses.max(axis=0)
+    wts = np.exp(lses - top)
+    tot = wts.sum(axis=0)
+    joined = sum(wts[p][..., None] * outs[p] for p in range(3)) / tot[..., None]
+    assert_close(joined, full, rtol=1e-12, atol=1e-14, what="shards joined by lse")
+    assert_close(top + np.log(tot), lse_full, rtol=1e-13, atol=1e-13, what="joined lse")
+
+
+def pin_lse_invalid_rows(decode_lse):
+    w = small(seed=61)
+    inp = make_inputs(w, lens=[37, 5])
+    inp.seqlens[1] = 0
+    _, lse, st = run_lse(decode_lse, inp)
+    assert st & 1
+    assert np.all(np.isneginf(lse[1])) and np.all(np.isfinite(lse[0])), "invalid rows: lse -inf"
+
+
+LSE_PINS = [pin_lse_single_token, pin_lse_uniform, pin_lse_torch_logsumexp, pin_lse_brute_force,
+            pin_lse_joins_shards, pin_lse_invalid_rows]

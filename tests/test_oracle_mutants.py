@@ -10,7 +10,7 @@ import os
 import pytest
 
 import oracle
-from tests.oracle_pins import PINS
+from tests.oracle_pins import LSE_PINS, PINS
 
 MUTANTS = {
     "group map i % G": ("const int32_t g = i / r;", "const int32_t g = i % G;"),
@@ -31,6 +31,9 @@ MUTANTS = {
                            "for (int32_t t = 0; t < len - 1; ++t) {\n            const long long off"),
     "capacity check off by one": ("if (len < 1 || len > capacity)", "if (len < 1 || len > capacity + 1)"),
     "page bound off by one": ("if (page < 0 || page >= num_pages)", "if (page < 0 || page > num_pages)"),
+    "lse without the maximum": ("lse[n] = mx + log(denom);", "lse[n] = log(denom);"),
+    "lse not a logarithm": ("lse[n] = mx + log(denom);", "lse[n] = mx + denom;"),
+    "lse of the last logit": ("lse[n] = mx + log(denom);", "lse[n] = logits[len - 1];"),
 }
 
 
@@ -50,10 +53,12 @@ def test_pins_catch_mutant(name, tmp_path):
     path.write_text(mutated)
     lib = oracle.load_library(oracle.build(force=True, src=str(path), out=str(tmp_path / "libmutant.so")))
     decode = functools.partial(oracle.gqa_decode, lib=lib)
+    decode_lse = functools.partial(oracle.gqa_decode_lse, lib=lib)
     caught = []
-    for pin in PINS:
-        try:
-            pin(decode)
-        except (AssertionError, ValueError, IndexError):
-            caught.append(pin.__name__)
+    for pins, fn in ((PINS, decode), (LSE_PINS, decode_lse)):
+        for pin in pins:
+            try:
+                pin(fn)
+            except (AssertionError, ValueError, IndexError):
+                caught.append(pin.__name__)
     assert caught, "no pin caught the mutant %r" % name

@@ -2,9 +2,14 @@
 import pytest
 
 import oracle
-from tests.oracle_pins import PINS
+from tests.oracle_pins import LSE_PINS, PINS
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
 def test_oracle_pin(pin):
     pin(oracle.gqa_decode)
+
+
+@pytest.mark.parametrize("pin", LSE_PINS, ids=[p.__name__ for p in LSE_PINS])
+def test_oracle_lse_pin(pin):
+    pin(oracle.gqa_decode_lse)
