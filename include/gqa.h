@@ -216,6 +216,41 @@ int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims,
                       const void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gqa_decode_split_lse -- gqa_decode_split that also returns, for every output
+ * row (s, i), the natural-log sum of the row's exponentials,
+ *     lse[s*H + i] = ln sum_{j < len_s} exp(scale * q[s,i] . K[s,g(i),j]),
+ * and accepts seqlens[s] == 0 as an empty sequence (its rows are zero with
+ * lse = -inf, and no status bit is set).  This is the per-shard half of
+ * sequence-parallel decode: when the tokens of each sequence are spread over
+ * several GPUs (each holding its own pool, page table and lengths for its
+ * share), every GPU runs this call on its share, the (out, lse) pairs are
+ * gathered, and gqa_merge_lse combines them.  The result equals attention over
+ * the whole sequence (an exact re-association of the softmax of the pages'
+ * formula).  lse: fp32 [b, H] device memory, 4-byte aligned, not NULL.
+ * Everything else as gqa_decode_split.
+ */
+int gqa_decode_split_lse(const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *seqlens, const int32_t *page_table, float *out, float *lse,
+                         const gqa_dims *dims, float scale, uint32_t *status,
+                         int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
+ * gqa_merge_lse -- merges n_parts normalised partial results of the same rows,
+ * each weighted by its log-sum-exp:
+ *     LSE = ln sum_k exp(lse_k),   out = sum_k exp(lse_k - LSE) o_k.
+ * o_parts: fp32 [n_parts][rows][head_dim], 16-byte aligned (part-major, the
+ * layout an all-gather of [rows][head_dim] per part produces); lse_parts: fp32
+ * [n_parts][rows]; out: fp32 [rows][head_dim], 16-byte aligned; lse_out: fp32
+ * [rows] or NULL.  Parts with lse = -inf contribute nothing; a row with no
+ * non-empty part is zero with LSE -inf.  head_dim: 64 or 128.  The parts are
+ * taken in ascending order, so the result is deterministic.  Asynchronous on
+ * `stream`; GQA_OK or a GQA_ERR_* code (nothing launched on error).
+ */
+int gqa_merge_lse(const float *o_parts, const float *lse_parts, int32_t n_parts, int64_t rows,
+                  int32_t head_dim, float *out, float *lse_out, void *stream);
+
+/*
  * The decomposition gqa_decode_split (and the pair gqa_split_partials /
  * gqa_split_combine) uses when split_tokens == 0: 0 for equal-work ranges, or
  * the fixed split length (a positive multiple of 128) it falls back to.

@@ -336,11 +336,18 @@ DecodeParams base_params(const Shape &sh, const void *q, const int32_t *seqlens,
   return p;
 }
 
+// Optional per-row outputs of the split entry points: the log-sum-exp of
+// every final row, and whether a length of 0 is a valid (empty) sequence.
+struct RowExtras {
+  float *lse = nullptr;
+  bool empty_ok = false;
+};
+
 // The items kernel: one block per (sequence, group, split) item.
 int run_items(const Shape &sh, const void *q, const void *k, const void *v, const int32_t *seqlens,
               const int32_t *pt, float *out, float scale, uint32_t *status, int split_tokens,
               int num_splits, int capacity, float *part_o, float *part_m, float *part_l,
-              unsigned long long *unit_ctr, cudaStream_t stream) {
+              unsigned long long *unit_ctr, cudaStream_t stream, const RowExtras &ex = RowExtras()) {
   CUtensorMap tk, tv;
   int rc = encode_maps(sh, k, v, &tk, &tv);
   if (rc != GQA_OK) return rc;
@@ -354,6 +361,8 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   p.num_splits = num_splits;
   p.unit_ctr = unit_ctr;
   p.epoch = unit_ctr ? next_epoch() : 0;
+  p.lse = ex.lse;
+  p.empty_ok = ex.empty_ok ? 1 : 0;
   const long long items = units_of(sh) * num_splits;
   if (items > (1ll << 31) - 1) return GQA_ERR_DIMS;
   Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream};
@@ -391,7 +400,8 @@ size_t auto_workspace_bytes(const Shape &sh, int max_seqlen) {
 
 int run_balanced_decode(const Shape &sh, int sms, const void *q, const void *k, const void *v,
                         const int32_t *seqlens, const int32_t *pt, float *out, float scale,
-                        uint32_t *status, int32_t max_seqlen, void *workspace, cudaStream_t stream) {
+                        uint32_t *status, int32_t max_seqlen, void *workspace, cudaStream_t stream,
+                        const RowExtras &ex = RowExtras()) {
   CUtensorMap tk, tv;
   int rc = encode_maps(sh, k, v, &tk, &tv);
   if (rc != GQA_OK) return rc;
@@ -406,13 +416,15 @@ int run_balanced_decode(const Shape &sh, int sms, const void *q, const void *k, 
   p.part_l = reinterpret_cast<float *>(w + ws.l_off);
   p.capacity = static_cast<int>(std::min<long long>(sh.capacity, max_seqlen));
   p.b = sh.b;
+  p.lse = ex.lse;
+  p.empty_ok = ex.empty_ok ? 1 : 0;
   Launch l{dim3(static_cast<unsigned>(sms), 1, 1), 1, stream};
   rc = launch_decode<Mode::kBalanced>(sh, tk, tv, p, l);
   return rc < 0 ? rc : GQA_OK;
 }
 
 int run_balanced_combine(const Shape &sh, const int32_t *seqlens, float *out, uint32_t *status,
-                         const void *workspace, cudaStream_t stream) {
+                         const void *workspace, cudaStream_t stream, const RowExtras &ex = RowExtras()) {
   const BalancedWorkspace ws = balanced_layout(sh);
   const uint8_t *w = static_cast<const uint8_t *>(workspace);
   CombineParams c{};
@@ -430,6 +442,8 @@ int run_balanced_combine(const Shape &sh, const int32_t *seqlens, float *out, ui
   c.r = sh.r;
   c.rc = sh.rc;
   c.hs = sh.hs;
+  c.lse = ex.lse;
+  c.empty_ok = ex.empty_ok ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(units_of(sh) * sh.rc), 1, 1);
   cfg.blockDim = dim3(128, 1, 1);
@@ -529,17 +543,19 @@ int prepare_split(const gqa_dims *dims, bool paged, int32_t split_tokens, int32_
 // gqa_split_combine.
 int run_partials(const SplitArgs &a, const void *q, const void *k, const void *v,
                  const int32_t *seqlens, const int32_t *pt, float *out, float scale, uint32_t *status,
-                 int32_t max_seqlen, void *workspace, bool merge_here, cudaStream_t stream) {
+                 int32_t max_seqlen, void *workspace, bool merge_here, cudaStream_t stream,
+                 const RowExtras &ex = RowExtras()) {
   uint8_t *w = static_cast<uint8_t *>(workspace);
   const int capacity = static_cast<int>(std::min<long long>(a.sh.capacity, max_seqlen));
   return run_items(a.sh, q, k, v, seqlens, pt, out, scale, status, a.split_tokens, a.num_splits,
                    capacity, reinterpret_cast<float *>(w), reinterpret_cast<float *>(w + a.ws.o_bytes),
                    reinterpret_cast<float *>(w + a.ws.o_bytes + a.ws.m_bytes),
-                   merge_here ? reinterpret_cast<unsigned long long *>(w + a.ws.ctr_off) : nullptr, stream);
+                   merge_here ? reinterpret_cast<unsigned long long *>(w + a.ws.ctr_off) : nullptr, stream, ex);
 }
 
 int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t *status,
-                int32_t max_seqlen, const void *workspace, cudaStream_t stream) {
+                int32_t max_seqlen, const void *workspace, cudaStream_t stream,
+                const RowExtras &ex = RowExtras()) {
   CombineParams c{};
   const uint8_t *w = static_cast<const uint8_t *>(workspace);
   c.seqlens = seqlens;
@@ -553,6 +569,8 @@ int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t
   c.max_len = max_seqlen;
   c.split_tokens = a.split_tokens;
   c.num_splits = a.num_splits;
+  c.lse = ex.lse;
+  c.empty_ok = ex.empty_ok ? 1 : 0;
   const int rows = a.sh.b * a.sh.H;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows, 1, 1);
@@ -567,6 +585,52 @@ int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t
   cudaError_t e = a.sh.D == 128 ? cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<128>, c)
                                 : cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<64>, c);
   return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+}  // namespace
+
+namespace {
+
+int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                      const int32_t *page_table, float *out, const gqa_dims *dims, float scale,
+                      uint32_t *status, int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                      size_t workspace_bytes, void *stream, const RowExtras &ex) {
+  int rc = check_inputs(q, k_cache, v_cache, seqlens, status);
+  if (rc != GQA_OK) return rc;
+  if (!out) return GQA_ERR_NULL_POINTER;
+  if (!aligned16(out)) return GQA_ERR_MISALIGNED;
+  if (!std::isfinite(scale)) return GQA_ERR_DIMS;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (split_tokens == 0) {
+    Shape sh;
+    if ((rc = prepare_auto(dims, page_table != nullptr, max_seqlen, workspace, workspace_bytes, &sh)) != GQA_OK)
+      return rc;
+    DeviceInfo dev;
+    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+    const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(dev.sms, 256));
+    if (ch.balanced) {
+      rc = run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale, status,
+                               max_seqlen, workspace, st, ex);
+      if (rc != GQA_OK) return rc;
+      return run_balanced_combine(sh, seqlens, out, status, workspace, st, ex);
+    }
+    split_tokens = ch.split_tokens;
+  }
+  SplitArgs a;
+  rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace,
+                     workspace_bytes, 0, &a);
+  if (rc != GQA_OK) return rc;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+  // Up to kSerialMergeMax splits: one launch, single-split rows final in their
+  // block and the others merged by the block that completes their unit.  More
+  // splits: their merge is too much work for one block, the combine kernel
+  // spreads it over one block per row.
+  const bool merge_here = a.num_splits <= gqa::kSerialMergeMax;
+  rc = run_partials(a, q, k_cache, v_cache, seqlens, page_table, out, scale, status, max_seqlen,
+                    workspace, merge_here, st, ex);
+  if (rc != GQA_OK || merge_here) return rc;
+  return run_combine(a, seqlens, out, status, max_seqlen, workspace, st, ex);
 }
 
 }  // namespace
@@ -709,42 +773,45 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, co
                      const int32_t *page_table, float *out, const gqa_dims *dims, float scale,
                      uint32_t *status, int32_t split_tokens, int32_t max_seqlen, void *workspace,
                      size_t workspace_bytes, void *stream) {
-  int rc = check_inputs(q, k_cache, v_cache, seqlens, status);
-  if (rc != GQA_OK) return rc;
-  if (!out) return GQA_ERR_NULL_POINTER;
-  if (!aligned16(out)) return GQA_ERR_MISALIGNED;
-  if (!std::isfinite(scale)) return GQA_ERR_DIMS;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (split_tokens == 0) {
-    Shape sh;
-    if ((rc = prepare_auto(dims, page_table != nullptr, max_seqlen, workspace, workspace_bytes, &sh)) != GQA_OK)
-      return rc;
-    DeviceInfo dev;
-    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(dev.sms, 256));
-    if (ch.balanced) {
-      rc = run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale, status,
-                               max_seqlen, workspace, st);
-      if (rc != GQA_OK) return rc;
-      return run_balanced_combine(sh, seqlens, out, status, workspace, st);
-    }
-    split_tokens = ch.split_tokens;
-  }
-  SplitArgs a;
-  rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace,
-                     workspace_bytes, 0, &a);
-  if (rc != GQA_OK) return rc;
+  return decode_split_impl(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status, split_tokens,
+                           max_seqlen, workspace, workspace_bytes, stream, RowExtras());
+}
+
+int gqa_decode_split_lse(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                         const int32_t *page_table, float *out, float *lse, const gqa_dims *dims, float scale,
+                         uint32_t *status, int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+  if (!lse) return GQA_ERR_NULL_POINTER;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return GQA_ERR_MISALIGNED;
+  RowExtras ex;
+  ex.lse = lse;
+  ex.empty_ok = true;
+  return decode_split_impl(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status, split_tokens,
+                           max_seqlen, workspace, workspace_bytes, stream, ex);
+}
+
+int gqa_merge_lse(const float *o_parts, const float *lse_parts, int32_t n_parts, int64_t rows, int32_t head_dim,
+                  float *out, float *lse_out, void *stream) {
+  if (!o_parts || !lse_parts || !out) return GQA_ERR_NULL_POINTER;
+  if (!aligned16(o_parts) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse_out) & 3u))
+    return GQA_ERR_MISALIGNED;
+  if (head_dim != 64 && head_dim != 128) return GQA_ERR_HEAD_DIM;
+  if (n_parts < 1 || rows < 1) return GQA_ERR_DIMS;
+  const int rows_per_block = 128 / (head_dim / 4);
+  const long long blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > 0x7fffffffll) return GQA_ERR_DIMS;
   DeviceInfo dev;
-  if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-  // Up to kSerialMergeMax splits: one launch, single-split rows final in their
-  // block and the others merged by the block that completes their unit.  More
-  // splits: their merge is too much work for one block, the combine kernel
-  // spreads it over one block per row.
-  const bool merge_here = a.num_splits <= gqa::kSerialMergeMax;
-  rc = run_partials(a, q, k_cache, v_cache, seqlens, page_table, out, scale, status, max_seqlen,
-                    workspace, merge_here, st);
-  if (rc != GQA_OK || merge_here) return rc;
-  return run_combine(a, seqlens, out, status, max_seqlen, workspace, st);
+  int rc = current_device_info(&dev);
+  if (rc != GQA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (head_dim == 128)
+    gqa::gqa_merge_lse_kernel<128><<<static_cast<unsigned>(blocks), 128, 0, st>>>(o_parts, lse_parts, n_parts,
+                                                                                    rows, out, lse_out);
+  else
+    gqa::gqa_merge_lse_kernel<64><<<static_cast<unsigned>(blocks), 128, 0, st>>>(o_parts, lse_parts, n_parts,
+                                                                                   rows, out, lse_out);
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 }  // extern "C"

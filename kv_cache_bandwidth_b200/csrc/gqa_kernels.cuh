@@ -75,6 +75,8 @@ struct DecodeParams {
   uint32_t *status;           // optional
   int *ws_header;             // balanced mode: {decode blocks, capacity, W lo, W hi} for the combine
   int4 *ws_meta;              // balanced mode: per unit {first block, last block, slot in first block}
+  float *lse;                 // [b, H] natural-log sum of exp(scale q.k) of each final row, or null
+  int empty_ok;               // a length of 0 is valid: zero row, lse -inf, no status bit
   unsigned long long *unit_ctr;  // items mode: arrival word per unit, or null (the merge is left to the combine)
   unsigned long long epoch;      // items mode: this call's tag in the arrival words, 1 .. 2^40 - 2
   int H, G, r;                // query heads, KV groups, heads per group
@@ -100,7 +102,17 @@ struct CombineParams {
   int G, r, rc, hs;           // balanced mode
   const int *ws_header;       // balanced mode: {decode blocks, capacity, W lo, W hi}
   const int4 *ws_meta;        // balanced mode: per unit {first block, last block, slot in first block}
+  float *lse;                 // [b, H] or null, as in DecodeParams
+  int empty_ok;
 };
+
+// Natural-log sum of exp over a row from its base-2 state: the row's
+// exponentials sum to L * 2^M, so ln(sum) = (M + log2 L) ln 2; -inf for a
+// row without tokens.
+__device__ __forceinline__ float lse_from_state(float M, float L) {
+  const float kNegInf = -__int_as_float(0x7f800000);
+  return (L > 0.f && M != kNegInf) ? (M + log2f(L)) * 0.6931471805599453f : kNegInf;
+}
 
 template <int D, int NT, int NHB, int CH, int STAGES, bool BAL = false>
 struct Tile {
@@ -356,7 +368,7 @@ struct MergeScratch {
 
 template <int D, typename SlotFn, typename SyncFn>
 __device__ __forceinline__ void merge_row(const float *part_o, const float *part_m, const float *part_l,
-                                          int n_contrib, SlotFn slot, float4 *dst, int tid,
+                                          int n_contrib, SlotFn slot, float4 *dst, float *lse_dst, int tid,
                                           MergeScratch<D> &sc, SyncFn sync) {
   using SC = MergeScratch<D>;
   constexpr int kTPR = SC::kTPR;
@@ -441,6 +453,7 @@ __device__ __forceinline__ void merge_row(const float *part_o, const float *part
     float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
     if (!bad && Lt > 0.f) res = make_float4(t.x / Lt, t.y / Lt, t.z / Lt, t.w / Lt);
     *dst = res;
+    if (lse_dst && c4 == 0) *lse_dst = bad ? kNegInf : lse_from_state(M, Lt);
   }
   sync();  // the scratch is free for the next row
 }
@@ -481,7 +494,8 @@ constexpr int kSerialMergeMax = 8;
 
 template <int D, int NV>
 __device__ __forceinline__ void merge_serial(const float *part_o, const float *part_m, const float *part_l,
-                                             long long base, int ns, int c4_0, int c4_step, float4 *dst_row) {
+                                             long long base, int ns, int c4_0, int c4_step, float4 *dst_row,
+                                             float *lse_dst) {
   const float kNegInf = -__int_as_float(0x7f800000);
   float m[kSerialMergeMax], l[kSerialMergeMax];
   float4 v[NV][kSerialMergeMax];
@@ -528,6 +542,7 @@ __device__ __forceinline__ void merge_serial(const float *part_o, const float *p
     if (!bad && L > 0.f) res = make_float4(acc[i].x / L, acc[i].y / L, acc[i].z / L, acc[i].w / L);
     dst_row[c4_0 + i * c4_step] = res;
   }
+  if (lse_dst && c4_0 == 0) *lse_dst = bad ? kNegInf : lse_from_state(M, L);
 }
 
 // The q.k and p.v contractions on CUDA cores (fp32 FMA) for group ratios
@@ -761,13 +776,17 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       // Nothing to read.  An invalid length is handled once, by split 0: zero
       // rows in `out` and a marker in split 0 for the combine.
       if (!pc.len_ok && pc.k == 0) {
+        // (a length of 0 where empty sequences are allowed: the same zero row,
+        // with lse -inf and no status bit)
+        const bool empty = p.empty_ok && pc.len == 0;
         for (int idx = threadIdx.x; idx < pc.nh * (D / 4); idx += blockDim.x) {
           const int h = idx / (D / 4), c4 = idx % (D / 4);
           const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
           if (p.out) reinterpret_cast<float4 *>(p.out + row * D)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLBadLength;
+          if (c4 == 0 && p.lse) p.lse[row] = kNegInf;
         }
-        if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusBadSeqlen);
+        if (threadIdx.x == 0 && p.status && !empty) atomicOr(p.status, kStatusBadSeqlen);
       }
       return;
     }
@@ -1201,6 +1220,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
             float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
             if (!bad && L > 0.f) res = make_float4(src.x / L, src.y / L, src.z / L, src.w / L);
             reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
+            if (c4 == 0 && p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(M_blk[h], L);
             if (!BAL && c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLFinal;
           } else {
             const size_t ps = pslot_base + static_cast<size_t>(h) * pslot_stride;
@@ -1238,7 +1258,8 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
             if (h < pc.nh) {
               const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
               merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(row) * p.num_splits, ns,
-                                 c4, kHalf, reinterpret_cast<float4 *>(p.out + row * D));
+                                 c4, kHalf, reinterpret_cast<float4 *>(p.out + row * D),
+                                 p.lse ? p.lse + row : nullptr);
             }
           }
         }
@@ -1297,9 +1318,11 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p)
   const int len = __ldg(p.seqlens + s);
   float4 *dst = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D) + threadIdx.x % (D / 4);
   pdl_wait_primary();  // the partial states below come from the preceding kernel
+  float *lse_dst = p.lse ? p.lse + row : nullptr;
   if (len < 1 || len > p.max_len) {
     if (threadIdx.x < D / 4) *dst = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusBadSeqlen);
+    if (threadIdx.x == 0 && lse_dst) *lse_dst = -__int_as_float(0x7f800000);
+    if (threadIdx.x == 0 && p.status && !(p.empty_ok && len == 0)) atomicOr(p.status, kStatusBadSeqlen);
     return;
   }
   const int ns = (len + p.split_tokens - 1) / p.split_tokens;
@@ -1309,11 +1332,11 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p)
   if (ns <= kSerialMergeMax) {
     if (threadIdx.x < D / 4)
       merge_serial<D, 1>(p.part_o, p.part_m, p.part_l, base, ns, threadIdx.x, 0,
-                         reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D));
+                         reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D), lse_dst);
     return;
   }
   __shared__ MergeScratch<D> sc;
-  merge_row<D>(p.part_o, p.part_m, p.part_l, ns, [&](int k) -> long long { return base + k; }, dst,
+  merge_row<D>(p.part_o, p.part_m, p.part_l, ns, [&](int k) -> long long { return base + k; }, dst, lse_dst,
                threadIdx.x, sc, [] { __syncthreads(); });
 }
 
@@ -1335,9 +1358,11 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
   pdl_wait_primary();  // the header, unit records and partial states come from the decode kernel
   const int N = p.ws_header[0];
   const int capacity = p.ws_header[1];
+  float *lse_dst = p.lse ? p.lse + row : nullptr;
   if (len < 1 || len > capacity) {
     if (threadIdx.x < D / 4) *dst = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (threadIdx.x == 0 && h == 0 && p.status) atomicOr(p.status, kStatusBadSeqlen);
+    if (threadIdx.x == 0 && lse_dst) *lse_dst = -__int_as_float(0x7f800000);
+    if (threadIdx.x == 0 && h == 0 && p.status && !(p.empty_ok && len == 0)) atomicOr(p.status, kStatusBadSeqlen);
     return;
   }
   const long long W = static_cast<long long>(static_cast<unsigned>(p.ws_header[2])) |
@@ -1352,7 +1377,48 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
                  if (k > 0 && (c * W / N) == ((c + 1) * W / N)) return -1;  // empty range
                  return (2 * c + (k == 0 ? slot_lo : 0)) * p.rc + h;
                },
-               dst, threadIdx.x, sc, [] { __syncthreads(); });
+               dst, lse_dst, threadIdx.x, sc, [] { __syncthreads(); });
+}
+
+// Merge of normalised partial results weighted by their log-sum-exp, e.g. the
+// token shards of a sequence held by different GPUs, gathered into one buffer
+// part-major: o_parts [n_parts][rows][D], lse_parts [n_parts][rows].  Per row,
+//   LSE = ln sum_k e^(lse_k),  out = sum_k e^(lse_k - LSE) o_k,
+// the same re-association of the softmax as the split merge, written for
+// results that are already normalised.  Parts with lse = -inf (no tokens)
+// weigh nothing; a row whose parts are all empty is zero with LSE -inf.  One
+// thread per float4 of a row; the parts are taken in ascending order.
+template <int D>
+__global__ void __launch_bounds__(128)
+    gqa_merge_lse_kernel(const float *o_parts, const float *lse_parts, int n_parts, long long rows, float *out,
+                         float *lse_out) {
+  constexpr int kTPR = D / 4;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  const long long row = static_cast<long long>(blockIdx.x) * (128 / kTPR) + threadIdx.x / kTPR;
+  const int c4 = threadIdx.x % kTPR;
+  if (row >= rows) return;
+  float mx = kNegInf;
+  for (int k = 0; k < n_parts; ++k) mx = fmaxf(mx, __ldg(lse_parts + k * rows + row));
+  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lse = kNegInf;
+  if (mx != kNegInf) {
+    float S = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < n_parts; ++k) {
+      const float w = ex2((__ldg(lse_parts + k * rows + row) - mx) * 1.4426950408889634f);
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(o_parts + (k * rows + row) * D) + c4);
+      S += w;
+      acc.x += v.x * w;
+      acc.y += v.y * w;
+      acc.z += v.z * w;
+      acc.w += v.w * w;
+    }
+    res = make_float4(acc.x / S, acc.y / S, acc.z / S, acc.w / S);
+    lse = mx + logf(S);
+  }
+  reinterpret_cast<float4 *>(out + row * D)[c4] = res;
+  if (lse_out && c4 == 0) lse_out[row] = lse;
 }
 
 }  // namespace gqa

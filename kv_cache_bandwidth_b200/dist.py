@@ -10,14 +10,25 @@ when G < T, as "GQA and MQA: Mathematical Foundations, KV-Cache Bandwidth
 Reduction ..." describes under "Tensor Parallelism Implications") is the same
 independence along the other axis; `group_shard` gives that split.
 
-Nothing here moves tensors between ranks; torch.distributed is used only for
-the timing reduction and barriers.
+Sequence parallelism (long contexts) cuts along the third axis, the tokens of
+each sequence: rank t holds a contiguous run of each sequence's pages
+(`token_shard`) in its own pool, decodes its share with
+`gqa_decode_split_lse` (output rows normalised over its tokens, plus each
+row's log-sum-exp), and the ranks' results are joined by the one exchange on
+this path: an all-gather of (out, lse) -- b*H*(d+1) floats per rank -- into
+each rank's own memory, followed by `gqa_merge_lse` there
+(`merge_shards`).  Because the merge is an exact re-association of the
+softmax, the result is attention over the whole sequence.
+
+Apart from that all-gather, nothing here moves tensors between ranks;
+torch.distributed is otherwise used only for the timing reduction and barriers.
 """
 from __future__ import annotations
 
 from typing import List, Tuple
 
-__all__ = ["sequence_shard", "group_shard", "max_over_ranks", "weak_scaling_value"]
+__all__ = ["sequence_shard", "group_shard", "token_shard", "merge_shards", "sequence_parallel_decode",
+           "max_over_ranks", "weak_scaling_value"]
 
 
 def sequence_shard(num_sequences: int, world: int, rank: int) -> Tuple[int, int]:
@@ -52,6 +63,70 @@ def group_shard(num_heads: int, num_kv_heads: int, world: int, rank: int) -> Tup
         return heads, gs
     heads = list(range(rank * (H // T), (rank + 1) * (H // T)))
     return heads, list(range(G))
+
+
+def token_shard(length: int, world: int, rank: int, page_size: int = 1) -> Tuple[int, int]:
+    """Token range [begin, end) of one sequence that `rank` of `world` holds
+    under sequence parallelism.
+
+    The sequence's ceil(length / page_size) pages (the last one possibly
+    partial) are dealt out in contiguous runs that differ by at most one page,
+    so every rank's share is whole pages of its own pool.  A rank may hold
+    nothing of a short sequence (begin == end): it decodes that sequence as
+    empty (length 0), which the merge ignores."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank %d outside world of %d" % (rank, world))
+    if length < 0 or page_size < 1:
+        raise ValueError("negative length or page size < 1")
+    pages = -(-length // page_size)
+    p0, p1 = rank * pages // world, (rank + 1) * pages // world
+    return min(p0 * page_size, length), min(p1 * page_size, length)
+
+
+def _all_gather_stacked(t, group):
+    import torch
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    t = t.contiguous()
+    if dist.get_backend(group) == "nccl":
+        dst = torch.empty((world,) + tuple(t.shape), dtype=t.dtype, device=t.device)
+        dist.all_gather_into_tensor(dst, t, group=group)
+        return dst
+    parts = [torch.empty_like(t) for _ in range(world)]
+    dist.all_gather(parts, t, group=group)
+    return torch.stack(parts)
+
+
+def merge_shards(out_local, lse_local, group=None, merge=None):
+    """The exchange of sequence-parallel decode: all-gather every rank's
+    normalised rows `out_local` [*rows, d] and their log-sum-exp `lse_local`
+    [*rows] (part-major, rank order), then merge them on this rank.
+
+    `merge(o_parts, lse_parts) -> (out, lse)` defaults to the library's
+    gqa_merge_lse (the tensors must then be on this rank's GPU).  Every rank
+    takes the same collective steps in the same order.  Returns (out, lse)."""
+    import torch.distributed as dist
+
+    if merge is None:
+        from . import gqa
+        merge = gqa.gqa_merge_lse
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return merge(out_local.unsqueeze(0).contiguous(), lse_local.unsqueeze(0).contiguous())
+    o_parts = _all_gather_stacked(out_local, group)
+    lse_parts = _all_gather_stacked(lse_local, group)
+    return merge(o_parts, lse_parts)
+
+
+def sequence_parallel_decode(q, k_cache, v_cache, seqlens, page_table=None, *, group=None, **kw):
+    """Decode step of this rank's token share (its own pool, page table and
+    per-sequence lengths, 0 where it holds nothing) followed by the exchange:
+    returns (out, lse) of the whole sequences, the same on every rank.
+    Keyword arguments go to gqa_decode_split_lse."""
+    from . import gqa
+
+    out, lse = gqa.gqa_decode_split_lse(q, k_cache, v_cache, seqlens, page_table, **kw)
+    return merge_shards(out, lse, group=group)
 
 
 def max_over_ranks(value: float, group=None) -> float:

@@ -25,6 +25,7 @@ __all__ = [
     "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version", "dims_for",
     "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
     "FLAG_CONTRACT_FMA", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
+    "gqa_decode_split_lse", "gqa_merge_lse", "SERIAL_MERGE_MAX_SPLITS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -93,6 +94,11 @@ def load():
     lib.gqa_plan_split_tokens.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32]
     lib.gqa_decode_split_static.restype = ctypes.c_int
     lib.gqa_decode_split_static.argtypes = _DECODE_ARGS + [ctypes.c_int32, ctypes.c_int32, _vp]
+    lib.gqa_decode_split_lse.restype = ctypes.c_int
+    lib.gqa_decode_split_lse.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), ctypes.c_float,
+                                         _vp, ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
+    lib.gqa_merge_lse.restype = ctypes.c_int
+    lib.gqa_merge_lse.argtypes = [_vp, _vp, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp]
     lib.gqa_status_string.restype = ctypes.c_char_p
     lib.gqa_status_string.argtypes = [ctypes.c_int]
     lib.gqa_abi_version.restype = ctypes.c_int32
@@ -192,6 +198,51 @@ def gqa_decode_split(q, k_cache, v_cache, seqlens, page_table=None, *, split_tok
                                  workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "gqa_decode_split")
     return out
+
+
+def gqa_decode_split_lse(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int = 0,
+                         max_seqlen: Optional[int] = None, workspace=None, out=None, lse=None, scale=None,
+                         status=None, stream=None, flags: int = 0):
+    """``gqa_decode_split`` that also returns lse [b, H] (fp32): the natural
+    log of each row's softmax normaliser; a length of 0 is an empty sequence
+    (zero row, lse -inf).  Returns (out, lse)."""
+    out = _out_for(q, out)
+    if lse is None:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    if max_seqlen is None:
+        max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
+    if workspace is None:
+        workspace = workspace_for(q, k_cache, page_table, max_seqlen, split_tokens)
+    dims = dims_for(q, k_cache, page_table, flags)
+    rc = load().gqa_decode_split_lse(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
+                                     _ptr(out), _ptr(lse), ctypes.byref(dims), _scale(q, scale), _ptr(status),
+                                     int(split_tokens), int(max_seqlen), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "gqa_decode_split_lse")
+    return out, lse
+
+
+def gqa_merge_lse(o_parts, lse_parts, *, out=None, lse_out=None, stream=None):
+    """Merge normalised partial results by their log-sum-exp.
+
+    o_parts fp32 [n_parts, *rows, d] and lse_parts fp32 [n_parts, *rows], both
+    contiguous (part-major, as an all-gather stacks them).  Returns (out
+    [*rows, d], lse_out [*rows])."""
+    n_parts, d = o_parts.shape[0], o_parts.shape[-1]
+    rows_shape = tuple(o_parts.shape[1:-1])
+    if tuple(lse_parts.shape) != (n_parts,) + rows_shape:
+        raise ValueError("lse_parts must be [n_parts, *rows] matching o_parts [n_parts, *rows, d]")
+    if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
+        raise ValueError("o_parts and lse_parts must be contiguous")
+    if out is None:
+        out = torch.empty(rows_shape + (d,), dtype=torch.float32, device=o_parts.device)
+    if lse_out is None:
+        lse_out = torch.empty(rows_shape, dtype=torch.float32, device=o_parts.device)
+    rows = math.prod(rows_shape)
+    rc = load().gqa_merge_lse(_ptr(o_parts), _ptr(lse_parts), int(n_parts), int(rows), int(d), _ptr(out),
+                              _ptr(lse_out), _stream(stream))
+    _check(rc, "gqa_merge_lse")
+    return out, lse_out
 
 
 def gqa_split_partials(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int,

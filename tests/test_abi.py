@@ -171,3 +171,30 @@ def test_plan_split_tokens(lib):
     with pytest.raises(gqa.GqaError) as e:
         gqa.gqa_plan_split_tokens(_dims(batch=0), 128, 148)
     assert e.value.code == -6
+
+
+def test_merge_lse_argument_checks(lib):
+    vp = ctypes.c_void_p
+    f = lib.gqa_merge_lse
+    f.restype = ctypes.c_int
+    f.argtypes = [vp, vp, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, vp, vp, vp]
+    A = 1 << 20   # a 16-byte-aligned fake address (never dereferenced: the checks come first)
+    assert f(None, A, 2, 10, 128, A, None, None) == -1
+    assert f(A, A, 2, 10, 128, None, None, None) == -1
+    assert f(A + 4, A, 2, 10, 128, A, None, None) == -2
+    assert f(A, A + 2, 2, 10, 128, A, None, None) == -2
+    assert f(A, A, 2, 10, 96, A, None, None) == -4
+    assert f(A, A, 0, 10, 128, A, None, None) == -6
+    assert f(A, A, 2, 0, 128, A, None, None) == -6
+
+
+def test_decode_split_lse_needs_lse(lib):
+    d = _dims()
+    A = 1 << 20
+    vp = ctypes.c_void_p
+    f = lib.gqa_decode_split_lse
+    f.restype = ctypes.c_int
+    f.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(gqa.Dims), ctypes.c_float, vp, ctypes.c_int32,
+                  ctypes.c_int32, vp, ctypes.c_size_t, vp]
+    assert f(A, A, A, A, None, A, None, ctypes.byref(d), 0.1, None, 128, 256, A, 1 << 20, None) == -1
+    assert f(A, A, A, A, None, A, A + 2, ctypes.byref(d), 0.1, None, 128, 256, A, 1 << 20, None) == -2

@@ -1,6 +1,7 @@
 """Multi-rank host logic on CPU (gloo, world_size 2): sequence sharding,
 tensor-parallel group sharding, and the max-over-ranks timing reduction that
 bench.py uses for weakly scaled runs."""
+import math
 import os
 import socket
 
@@ -89,3 +90,84 @@ def test_two_rank_gloo_reduction():
     for rank, tmax, got in results:
         assert tmax == pytest.approx(1.25)
         assert got == [(0, 32), (32, 64)]
+
+
+def test_token_shard_covers_each_sequence_once():
+    for length in (0, 1, 5, 16, 17, 100, 4096, 4097):
+        for world in (1, 2, 3, 4, 8):
+            for P in (1, 16, 64):
+                spans = [gdist.token_shard(length, world, r, P) for r in range(world)]
+                assert spans[0][0] == 0 and spans[-1][1] == length
+                for (a, b), (c, d) in zip(spans, spans[1:]):
+                    assert b == c and a <= b
+                for a, b in spans:   # whole pages, except the sequence's own last one
+                    assert a % P == 0 and (b % P == 0 or b == length)
+                sizes = [-(-(b - a) // P) for a, b in spans]
+                assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        gdist.token_shard(10, 2, 2)
+
+
+def _lse_merge_reference(o_parts, lse_parts):
+    """The join of normalised shards, written out in float64 for the CPU test:
+    out = sum_p e^(lse_p - LSE) o_p, LSE = ln sum_p e^(lse_p)."""
+    top = lse_parts.max(dim=0).values
+    safe = torch.where(torch.isfinite(top), top, torch.zeros_like(top))
+    w = torch.exp(lse_parts - safe)
+    tot = w.sum(dim=0)
+    out = (w[..., None] * o_parts).sum(dim=0) / torch.where(tot > 0, tot, torch.ones_like(tot))[..., None]
+    return out, torch.where(tot > 0, safe + torch.log(tot), torch.full_like(tot, -math.inf))
+
+
+def _seq_parallel_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from kv_cache_bandwidth_b200.workloads import Workload, make_inputs
+
+        lens = [50, 3, 17, 1]
+        P = 8
+        w = Workload(name="sp", b=len(lens), H=8, G=2, d=16, m=50, seed=71)
+        inp = make_inputs(w, lens=lens)
+        spans = [gdist.token_shard(n, world, rank, P) for n in lens]
+        m_loc = max(1, max(b - a for a, b in spans))
+        loc = make_inputs(w.with_(m=m_loc), lens=[1] * w.b)
+        loc.q.copy_(inp.q)
+        for s, (a, b) in enumerate(spans):
+            loc.k_cache[s, :, : b - a] = inp.k_cache[s, :, a:b]
+            loc.v_cache[s, :, : b - a] = inp.v_cache[s, :, a:b]
+            loc.seqlens[s] = b - a
+        out_l, lse_l, _ = oracle.gqa_decode_lse(loc.q, loc.k_cache, loc.v_cache, loc.seqlens,
+                                                num_kv_heads=w.G)
+        out, lse = gdist.merge_shards(torch.from_numpy(out_l), torch.from_numpy(lse_l),
+                                      merge=_lse_merge_reference)
+        ref, ref_lse, st = oracle.gqa_decode_lse(inp.q, inp.k_cache, inp.v_cache, inp.seqlens,
+                                                 num_kv_heads=w.G)
+        assert st == 0
+        q.put((rank, float((out.numpy() - ref).__abs__().max()), float((lse.numpy() - ref_lse).__abs__().max()),
+               [b - a for a, b in spans]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_gloo_sequence_parallel_join():
+    """Two ranks each hold a contiguous page run of every sequence (one holds
+    nothing of the 1- and 3-token ones), decode their share with the oracle,
+    and join through merge_shards' all-gather: both get attention over the
+    whole sequences."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_seq_parallel_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[3] for r in results] == [[24, 0, 8, 0], [26, 3, 9, 1]]
+    for rank, err_out, err_lse, _ in results:
+        assert err_out < 1e-12 and err_lse < 1e-12, (rank, err_out, err_lse)
