@@ -80,6 +80,7 @@ extern "C" {
 #define GQA_ERR_WORKSPACE (-8)     /* workspace NULL or smaller than required */
 #define GQA_ERR_CUDA (-9)          /* a CUDA runtime/driver call failed */
 #define GQA_ERR_DEVICE (-10)       /* current device is not sm_100 (B200) */
+#define GQA_ERR_NO_PAGES (-11)     /* page pool (gqa_cache.h): not enough free pages */
 
 /* Bits the kernels OR into *status. */
 #define GQA_STATUS_BAD_SEQLEN 1u   /* a length outside [1, capacity]: row zeroed */

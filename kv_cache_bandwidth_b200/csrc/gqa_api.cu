@@ -653,6 +653,7 @@ const char *gqa_status_string(int code) {
     case GQA_ERR_WORKSPACE: return "workspace missing or too small";
     case GQA_ERR_CUDA: return "a CUDA call failed";
     case GQA_ERR_DEVICE: return "the current device is not an sm_100 (B200) GPU";
+    case GQA_ERR_NO_PAGES: return "the page pool has fewer free pages than requested";
     default: return "unknown status";
   }
 }

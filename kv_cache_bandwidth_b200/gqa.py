@@ -25,7 +25,7 @@ __all__ = [
     "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version", "dims_for",
     "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
     "FLAG_CONTRACT_FMA", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
-    "gqa_decode_split_lse", "gqa_merge_lse", "SERIAL_MERGE_MAX_SPLITS",
+    "gqa_decode_split_lse", "gqa_merge_lse", "SERIAL_MERGE_MAX_SPLITS", "gqa_kv_append", "PagePool",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +40,7 @@ FLAG_CONTRACT_FMA = 2
 ERRORS = {
     0: "GQA_OK", -1: "GQA_ERR_NULL_POINTER", -2: "GQA_ERR_MISALIGNED", -3: "GQA_ERR_HEADS",
     -4: "GQA_ERR_HEAD_DIM", -5: "GQA_ERR_PAGE_SIZE", -6: "GQA_ERR_DIMS", -7: "GQA_ERR_SPLIT",
-    -8: "GQA_ERR_WORKSPACE", -9: "GQA_ERR_CUDA", -10: "GQA_ERR_DEVICE",
+    -8: "GQA_ERR_WORKSPACE", -9: "GQA_ERR_CUDA", -10: "GQA_ERR_DEVICE", -11: "GQA_ERR_NO_PAGES",
 }
 
 
@@ -99,6 +99,18 @@ def load():
                                          _vp, ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
     lib.gqa_merge_lse.restype = ctypes.c_int
     lib.gqa_merge_lse.argtypes = [_vp, _vp, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp]
+    lib.gqa_kv_append.restype = ctypes.c_int
+    lib.gqa_kv_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), _vp, _vp]
+    lib.gqa_page_pool_create.restype = _vp
+    lib.gqa_page_pool_create.argtypes = [ctypes.c_int32]
+    lib.gqa_page_pool_destroy.restype = None
+    lib.gqa_page_pool_destroy.argtypes = [_vp]
+    lib.gqa_page_pool_available.restype = ctypes.c_int32
+    lib.gqa_page_pool_available.argtypes = [_vp]
+    lib.gqa_page_pool_alloc.restype = ctypes.c_int
+    lib.gqa_page_pool_alloc.argtypes = [_vp, ctypes.c_int32, _vp]
+    lib.gqa_page_pool_free.restype = ctypes.c_int
+    lib.gqa_page_pool_free.argtypes = [_vp, _vp, ctypes.c_int32]
     lib.gqa_status_string.restype = ctypes.c_char_p
     lib.gqa_status_string.argtypes = [ctypes.c_int]
     lib.gqa_abi_version.restype = ctypes.c_int32
@@ -243,6 +255,47 @@ def gqa_merge_lse(o_parts, lse_parts, *, out=None, lse_out=None, stream=None):
                               _ptr(lse_out), _stream(stream))
     _check(rc, "gqa_merge_lse")
     return out, lse_out
+
+
+def gqa_kv_append(k_new, v_new, k_cache, v_cache, seqlens, page_table=None, *, num_heads: Optional[int] = None,
+                  status=None, stream=None) -> None:
+    """Write k_new/v_new [b, G, d] at position seqlens[s] of every sequence's
+    cache and increment seqlens (include/gqa_cache.h)."""
+    b, G, d = k_new.shape
+    pages, G2, P, _ = k_cache.shape
+    max_pages = 0 if page_table is None else page_table.shape[1]
+    dims = Dims(b, num_heads or G2, G2, d, P, pages, max_pages, 0)
+    rc = load().gqa_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+                              _ptr(page_table), ctypes.byref(dims), _ptr(status), _stream(stream))
+    _check(rc, "gqa_kv_append")
+
+
+class PagePool:
+    """The library's host-side pool of page ids (gqa_page_pool_*)."""
+
+    def __init__(self, num_pages: int):
+        self._lib = load()
+        self._h = self._lib.gqa_page_pool_create(int(num_pages))
+        if not self._h:
+            raise ValueError("cannot create a pool of %d pages" % num_pages)
+
+    def __del__(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h:
+            self._lib.gqa_page_pool_destroy(h)
+
+    @property
+    def available(self) -> int:
+        return int(self._lib.gqa_page_pool_available(self._h))
+
+    def alloc(self, n: int):
+        ids = (ctypes.c_int32 * max(1, n))()
+        _check(self._lib.gqa_page_pool_alloc(self._h, int(n), ids), "gqa_page_pool_alloc")
+        return list(ids[:n])
+
+    def free(self, ids) -> None:
+        arr = (ctypes.c_int32 * max(1, len(ids)))(*ids)
+        _check(self._lib.gqa_page_pool_free(self._h, arr, len(ids)), "gqa_page_pool_free")
 
 
 def gqa_split_partials(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int,

@@ -10,7 +10,8 @@ import pytest
 from kv_cache_bandwidth_b200 import build as gqa_build
 from kv_cache_bandwidth_b200 import gqa
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "gqa.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+HEADER = os.path.join(INCLUDE, "gqa.h")
 
 
 @pytest.fixture(scope="module")
@@ -20,7 +21,7 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = "\n".join(open(os.path.join(INCLUDE, f)).read() for f in sorted(os.listdir(INCLUDE)) if f.endswith(".h"))
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(gqa_\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
@@ -29,7 +30,10 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("gqa_decode", "gqa_decode_split", "gqa_decode_split_workspace_size", "gqa_split_partials",
-              "gqa_split_combine", "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version"):
+              "gqa_split_combine", "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version",
+              "gqa_decode_split_lse", "gqa_merge_lse", "gqa_decode_split_static", "gqa_kv_append",
+              "gqa_page_pool_create", "gqa_page_pool_alloc", "gqa_page_pool_free", "gqa_page_pool_available",
+              "gqa_page_pool_destroy"):
         assert n in names
 
 
@@ -198,3 +202,44 @@ def test_decode_split_lse_needs_lse(lib):
                   ctypes.c_int32, vp, ctypes.c_size_t, vp]
     assert f(A, A, A, A, None, A, None, ctypes.byref(d), 0.1, None, 128, 256, A, 1 << 20, None) == -1
     assert f(A, A, A, A, None, A, A + 2, ctypes.byref(d), 0.1, None, 128, 256, A, 1 << 20, None) == -2
+
+
+def test_page_pool_hands_out_ids_deterministically(lib):
+    pool = gqa.PagePool(6)
+    assert pool.available == 6
+    assert pool.alloc(4) == [0, 1, 2, 3]
+    pool.free([2, 0])
+    assert pool.available == 4
+    assert pool.alloc(3) == [0, 2, 4]          # most recently freed first, then the untouched ones
+    assert pool.alloc(0) == []
+    with pytest.raises(gqa.GqaError) as e:
+        pool.alloc(2)                           # one left
+    assert e.value.code == -11 and pool.available == 1
+    for bad in ([6], [-1], [5], [1, 1]):        # outside, outside, never allocated, listed twice
+        with pytest.raises(gqa.GqaError) as e:
+            pool.free(bad)
+        assert e.value.code == -6
+    assert pool.available == 1                  # failed frees return nothing
+    pool.free([1, 3])
+    assert pool.alloc(3) == [3, 1, 5]
+    with pytest.raises(ValueError):
+        gqa.PagePool(0)
+
+
+def test_kv_append_argument_checks(lib):
+    vp = ctypes.c_void_p
+    f = lib.gqa_kv_append
+    f.restype = ctypes.c_int
+    f.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(gqa.Dims), vp, vp]
+    A = 1 << 20
+    d = _dims()
+    assert f(None, A, A, A, A, None, ctypes.byref(d), None, None) == -1
+    assert f(A, A, A, A, None, None, ctypes.byref(d), None, None) == -1
+    assert f(A + 8, A, A, A, A, None, ctypes.byref(d), None, None) == -2
+    assert f(A, A, A, A, A + 2, None, ctypes.byref(d), None, None) == -2
+    assert f(A, A, A, A, A, None, ctypes.byref(_dims(head_dim=96)), None, None) == -4
+    assert f(A, A, A, A, A, None, ctypes.byref(_dims(num_heads=7)), None, None) == -3
+    assert f(A, A, A, A, A, A, ctypes.byref(_dims(page_size=12, num_pages=4, max_pages_per_seq=2)),
+             None, None) == -5
+    assert f(A, A, A, A, A, A, ctypes.byref(_dims(page_size=16, num_pages=0, max_pages_per_seq=2)),
+             None, None) == -6
