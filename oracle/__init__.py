@@ -68,6 +68,10 @@ def load_library(path: str):
         ctypes.c_double, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
         ctypes.c_void_p, ctypes.c_int32,
     ]
+    if hasattr(lib, "oracle_gqa_decode_multi"):
+        a = lib.oracle_gqa_decode.argtypes
+        lib.oracle_gqa_decode_multi.restype = ctypes.c_int
+        lib.oracle_gqa_decode_multi.argtypes = a[:6] + [ctypes.c_int32] + a[6:16] + [ctypes.c_void_p] + a[16:]
     if hasattr(lib, "oracle_gqa_decode_lse"):
         lib.oracle_gqa_decode_lse.restype = ctypes.c_int
         lib.oracle_gqa_decode_lse.argtypes = lib.oracle_gqa_decode.argtypes[:16] + [ctypes.c_void_p] + \
@@ -145,14 +149,36 @@ def gqa_decode_lse(q, k_cache, v_cache, seqlens, page_table=None, *, num_kv_head
                    want_lse=True)
 
 
-def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows, threads, lib, want_lse):
-    """Shared body of gqa_decode and gqa_decode_lse."""
+def gqa_decode_verify(q, k_cache, v_cache, seqlens, page_table=None, *, num_kv_heads: int,
+                      scale: Optional[float] = None, rows=None, threads: int = 0,
+                      lib=None) -> Tuple[np.ndarray, np.ndarray, int]:
+    """Decode of nq query tokens per sequence (speculative verification).
+
+    q bf16 [b, nq, H, d]; query token t of sequence s attends the cached
+    positions j < seqlens[s] - (nq - 1 - t).  rows: flat ids (s*nq + t)*H + i.
+    Returns (out float64 [b, nq, H, d] (or [len(rows), d]), lse [b, nq, H]
+    (or [len(rows)]), status); a length below nq sets status bit 1."""
+    qb = _as_bits(q)
+    if qb.ndim != 4:
+        raise ValueError("q must be [b, nq, H, d]")
+    b, nq, H, d = qb.shape
+    flat = qb.reshape(b, nq * H, d)
+    out, lse, status = _decode(flat, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows, threads,
+                               lib, want_lse=True, nq=nq)
+    if rows is None:
+        out, lse = out.reshape(b, nq, H, d), lse.reshape(b, nq, H)
+    return out, lse, status
+
+
+def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows, threads, lib, want_lse, nq=1):
+    """Shared body of the decode functions (q given as [b, nq * H, d])."""
     qb = _as_bits(q)
     kb = _as_bits(k_cache)
     vb = _as_bits(v_cache)
     if qb.ndim != 3 or kb.ndim != 4 or kb.shape != vb.shape:
         raise ValueError("q must be [b,H,d] and k/v caches [pages,G,P,d] of equal shape")
     b, H, d = qb.shape
+    H //= nq
     num_pages, G, P, dk = kb.shape
     if dk != d or G != num_kv_heads:
         raise ValueError("cache shape %s does not match q %s / G=%d" % (kb.shape, qb.shape, num_kv_heads))
@@ -168,7 +194,7 @@ def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows,
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     rows_arr = None
-    nrows = b * H
+    nrows = b * nq * H
     if rows is not None:
         rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
         nrows = rows_arr.shape[0]
@@ -179,6 +205,13 @@ def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows,
             float(scale), None if rows_arr is None else rows_arr.ctypes.data, nrows, out.ctypes.data]
     lse = None
     lib = lib or _load()
+    if nq > 1:
+        lse = np.zeros(nrows, dtype=np.float64)
+        args.insert(6, nq)
+        rc = lib.oracle_gqa_decode_multi(*args, lse.ctypes.data, status.ctypes.data, int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments")
+        return out, lse, int(status[0])
     if want_lse:
         lse = np.zeros(nrows, dtype=np.float64)
         rc = lib.oracle_gqa_decode_lse(*args, lse.ctypes.data, status.ctypes.data, int(threads))

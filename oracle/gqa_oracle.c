@@ -16,6 +16,13 @@
  *   out[s,i,:] = sum_j w_j * V[s,g(i),j,:]
  *   lse[s,i]   = ln sum_j exp(l_j)            (oracle_gqa_decode_lse only)
  *
+ * oracle_gqa_decode_multi generalises this to nq query tokens per sequence
+ * (speculative-decoding verification): q and out are [b, nq, H, d], and query
+ * token t (0 .. nq-1) of sequence s attends the cached positions
+ * j < len_s - (nq - 1 - t), i.e. every cached token before it and itself,
+ * not the drafts after it (the mask of a causal decoder, aligned to the end
+ * of the cache).  nq = 1 is the decode above.
+ *
  * Sources, by page and section:
  *  - "Grouped-Query Attention" (aiwiki), the PyTorch module: keys and values are
  *    broadcast to the query heads of their group by repeat_interleave(h // g,
@@ -109,7 +116,7 @@ static long long kv_row_offset(const int32_t *page_table, int32_t s, int32_t t,
  */
 static int decode_rows(const uint16_t *q, const uint16_t *k_cache,
                        const uint16_t *v_cache, const int32_t *seqlens,
-                       const int32_t *page_table, int32_t b, int32_t H, int32_t G,
+                       const int32_t *page_table, int32_t b, int32_t nq, int32_t H, int32_t G,
                        int32_t d, int32_t page_size, int32_t num_pages,
                        int32_t max_pages_per_seq, double scale,
                        const int64_t *rows, int64_t nrows, double *out, double *lse,
@@ -117,14 +124,14 @@ static int decode_rows(const uint16_t *q, const uint16_t *k_cache,
 {
     if (!q || !k_cache || !v_cache || !seqlens || !out || !status)
         return -1;
-    if (b < 1 || H < 1 || G < 1 || d < 1 || page_size < 1 || num_pages < 1)
+    if (b < 1 || nq < 1 || H < 1 || G < 1 || d < 1 || page_size < 1 || num_pages < 1)
         return -1;
     if (H % G != 0)
         return -1;
     if (page_table != NULL && max_pages_per_seq < 1)
         return -1;
     if (rows == NULL)
-        nrows = (int64_t)b * H;
+        nrows = (int64_t)b * nq * H;
 
     const int32_t r = H / G;
     const long long capacity =
@@ -141,18 +148,21 @@ static int decode_rows(const uint16_t *q, const uint16_t *k_cache,
             o[k] = 0.0;
         if (lse)
             lse[n] = -INFINITY;
-        if (row < 0 || row >= (int64_t)b * H) {
+        if (row < 0 || row >= (int64_t)b * nq * H) {
             status_all |= ORACLE_STATUS_BAD_SEQLEN;
             continue;
         }
-        const int32_t s = (int32_t)(row / H);
+        const int32_t s = (int32_t)(row / ((int64_t)nq * H));   /* row = (s * nq + tq) * H + i */
+        const int32_t tq = (int32_t)((row / H) % nq);
         const int32_t i = (int32_t)(row % H);
         const int32_t g = i / r;
-        const int32_t len = seqlens[s];
-        if (len < 1 || len > capacity) {
+        const int32_t len_s = seqlens[s];
+        if (len_s < nq || len_s > capacity) {
             status_all |= ORACLE_STATUS_BAD_SEQLEN;
             continue;
         }
+        /* positions this query token sees: the cache up to and including itself */
+        const int32_t len = len_s - (nq - 1 - tq);
 
         /* Every page this row touches must lie in the pool. */
         int bad_page = 0;
@@ -235,7 +245,7 @@ int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache,
                       const int64_t *rows, int64_t nrows, double *out,
                       int32_t *status, int32_t nthreads)
 {
-    return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, H, G, d,
+    return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, 1, H, G, d,
                        page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
                        out, NULL, status, nthreads);
 }
@@ -252,7 +262,22 @@ int oracle_gqa_decode_lse(const uint16_t *q, const uint16_t *k_cache,
 {
     if (!lse)
         return -1;
-    return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, H, G, d,
+    return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, 1, H, G, d,
+                       page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
+                       out, lse, status, nthreads);
+}
+
+/* nq query tokens per sequence: q, out [b, nq, H, d] (rows (s * nq + t) * H + i),
+ * lse [nrows] or NULL; a length below nq is invalid (status bit 1). */
+int oracle_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache,
+                            const uint16_t *v_cache, const int32_t *seqlens,
+                            const int32_t *page_table, int32_t b, int32_t nq, int32_t H,
+                            int32_t G, int32_t d, int32_t page_size, int32_t num_pages,
+                            int32_t max_pages_per_seq, double scale,
+                            const int64_t *rows, int64_t nrows, double *out, double *lse,
+                            int32_t *status, int32_t nthreads)
+{
+    return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, nq, H, G, d,
                        page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
                        out, lse, status, nthreads);
 }

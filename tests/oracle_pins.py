@@ -24,6 +24,12 @@ What each pin compares against:
   * error handling -- invalid lengths and page ids set status bits, zero rows.
   * brute force -- tiny cases summed in pure Python with math.fsum.
 
+``VERIFY_PINS`` take ``oracle.gqa_decode_verify`` (nq query tokens per
+sequence, draft t seeing the cache up to and including itself): each draft
+against a one-token decode with the length it sees; torch's
+scaled_dot_product_attention in float64 with the end-aligned causal mask
+written out as a boolean matrix; math.fsum brute force; lengths below nq.
+
 ``LSE_PINS`` take ``oracle.gqa_decode_lse`` instead and pin the log of each
 row's softmax normaliser, ln sum_j exp(scale q.k_j): one token gives its own
 logit; q = 0 gives ln len; torch.logsumexp in float64 on the broadcast keys;
@@ -432,3 +438,80 @@ def pin_lse_invalid_rows(decode_lse):
 
 LSE_PINS = [pin_lse_single_token, pin_lse_uniform, pin_lse_torch_logsumexp, pin_lse_brute_force,
             pin_lse_joins_shards, pin_lse_invalid_rows]
+
+
+# ----------------------------------------------------------------------------
+# several query tokens per sequence (decode_verify: oracle.gqa_decode_verify)
+
+
+def _drafts(nq, b=3, H=8, G=2, d=16, m=40, seed=67, lens=(40, 9, 4)):
+    w = small(b=b, H=H, G=G, d=d, m=m, seed=seed)
+    inp = make_inputs(w, lens=list(lens))
+    gen = torch.Generator().manual_seed(seed + 1)
+    qv = torch.randn(b, nq, H, d, generator=gen).to(torch.bfloat16)
+    return w, inp, qv
+
+
+def pin_verify_each_draft_is_a_decode(decode_verify):
+    nq = 4
+    w, inp, qv = _drafts(nq)
+    out, lse, st = decode_verify(qv, inp.k_cache, inp.v_cache, inp.seqlens, num_kv_heads=w.G)
+    assert st == 0
+    for t in range(nq):
+        lens = inp.seqlens - (nq - 1 - t)
+        ref, ref_lse, _ = oracle_decode_lse(qv[:, t].contiguous(), inp.k_cache, inp.v_cache, lens, w.G)
+        assert_close(out[:, t], ref, rtol=1e-13, atol=1e-15, what="draft %d" % t)
+        assert_close(lse[:, t], ref_lse, rtol=1e-13, atol=1e-13, what="draft %d lse" % t)
+
+
+def pin_verify_sdpa_causal_mask(decode_verify):
+    nq = 3
+    w, inp, qv = _drafts(nq, seed=71, lens=(40, 3, 17))
+    scale = 0.3
+    out, _, _ = decode_verify(qv, inp.k_cache, inp.v_cache, inp.seqlens, num_kv_heads=w.G, scale=scale)
+    q = bf16_f64(qv).permute(0, 2, 1, 3)                                  # [b, H, nq, d]
+    k = bf16_f64(inp.k_cache).repeat_interleave(w.H // w.G, dim=1)
+    v = bf16_f64(inp.v_cache).repeat_interleave(w.H // w.G, dim=1)
+    m = k.shape[2]
+    mask = torch.zeros(w.b, 1, nq, m, dtype=torch.bool)
+    for s in range(w.b):
+        L = int(inp.seqlens[s])
+        for t in range(nq):
+            mask[s, 0, t, : L - (nq - 1 - t)] = True
+    ref = F.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=scale).permute(0, 2, 1, 3).numpy()
+    assert_close(out, ref, rtol=1e-12, atol=1e-14, what="sdpa, end-aligned causal mask")
+
+
+def pin_verify_brute_force(decode_verify):
+    nq = 2
+    w, inp, qv = _drafts(nq, b=2, H=4, G=2, d=3, m=5, seed=73, lens=(5, 2))
+    out, _, _ = decode_verify(qv, inp.k_cache, inp.v_cache, inp.seqlens, num_kv_heads=w.G, scale=0.9)
+    q, k, v = bf16_f64(qv).tolist(), bf16_f64(inp.k_cache).tolist(), bf16_f64(inp.v_cache).tolist()
+    for s in range(w.b):
+        for t in range(nq):
+            L = int(inp.seqlens[s]) - (nq - 1 - t)
+            for i in range(w.H):
+                g = i // (w.H // w.G)
+                z = [0.9 * math.fsum(q[s][t][i][c] * k[s][g][j][c] for c in range(w.d)) for j in range(L)]
+                e = [math.exp(x) for x in z]
+                tot = math.fsum(e)
+                ref = [math.fsum(e[j] / tot * v[s][g][j][c] for j in range(L)) for c in range(w.d)]
+                assert_close(out[s, t, i], ref, rtol=1e-13, atol=1e-15, what="brute force draft")
+
+
+def pin_verify_length_below_drafts(decode_verify):
+    nq = 3
+    w, inp, qv = _drafts(nq, lens=(40, 2, 3))
+    out, lse, st = decode_verify(qv, inp.k_cache, inp.v_cache, inp.seqlens, num_kv_heads=w.G)
+    assert st & 1
+    assert not out[1].any() and np.all(np.isneginf(lse[1]))
+    assert np.all(np.isfinite(lse[2])) and np.all(np.isfinite(lse[0]))
+
+
+def oracle_decode_lse(q, k, v, lens, G):
+    import oracle
+    return oracle.gqa_decode_lse(q, k, v, lens, num_kv_heads=G)
+
+
+VERIFY_PINS = [pin_verify_each_draft_is_a_decode, pin_verify_sdpa_causal_mask, pin_verify_brute_force,
+               pin_verify_length_below_drafts]

@@ -10,7 +10,7 @@ import os
 import pytest
 
 import oracle
-from tests.oracle_pins import LSE_PINS, PINS
+from tests.oracle_pins import LSE_PINS, PINS, VERIFY_PINS
 
 MUTANTS = {
     "group map i % G": ("const int32_t g = i / r;", "const int32_t g = i % G;"),
@@ -29,7 +29,10 @@ MUTANTS = {
     "group stride dropped": ("((page * G + g) * (long long)page_size", "((page + g) * (long long)page_size"),
     "last token dropped": ("for (int32_t t = 0; t < len; ++t) {\n            const long long off",
                            "for (int32_t t = 0; t < len - 1; ++t) {\n            const long long off"),
-    "capacity check off by one": ("if (len < 1 || len > capacity)", "if (len < 1 || len > capacity + 1)"),
+    "capacity check off by one": ("if (len_s < nq || len_s > capacity)", "if (len_s < nq || len_s > capacity + 1)"),
+    "draft mask reversed": ("const int32_t len = len_s - (nq - 1 - tq);", "const int32_t len = len_s - tq;"),
+    "draft mask off by one": ("const int32_t len = len_s - (nq - 1 - tq);", "const int32_t len = len_s - (nq - tq);"),
+    "draft index of the row": ("const int32_t tq = (int32_t)((row / H) % nq);", "const int32_t tq = (int32_t)(row % nq);"),
     "page bound off by one": ("if (page < 0 || page >= num_pages)", "if (page < 0 || page > num_pages)"),
     "lse without the maximum": ("lse[n] = mx + log(denom);", "lse[n] = log(denom);"),
     "lse not a logarithm": ("lse[n] = mx + log(denom);", "lse[n] = mx + denom;"),
@@ -54,8 +57,9 @@ def test_pins_catch_mutant(name, tmp_path):
     lib = oracle.load_library(oracle.build(force=True, src=str(path), out=str(tmp_path / "libmutant.so")))
     decode = functools.partial(oracle.gqa_decode, lib=lib)
     decode_lse = functools.partial(oracle.gqa_decode_lse, lib=lib)
+    decode_verify = functools.partial(oracle.gqa_decode_verify, lib=lib)
     caught = []
-    for pins, fn in ((PINS, decode), (LSE_PINS, decode_lse)):
+    for pins, fn in ((PINS, decode), (LSE_PINS, decode_lse), (VERIFY_PINS, decode_verify)):
         for pin in pins:
             try:
                 pin(fn)

@@ -2,7 +2,7 @@
 import pytest
 
 import oracle
-from tests.oracle_pins import LSE_PINS, PINS
+from tests.oracle_pins import LSE_PINS, PINS, VERIFY_PINS
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -13,3 +13,8 @@ def test_oracle_pin(pin):
 @pytest.mark.parametrize("pin", LSE_PINS, ids=[p.__name__ for p in LSE_PINS])
 def test_oracle_lse_pin(pin):
     pin(oracle.gqa_decode_lse)
+
+
+@pytest.mark.parametrize("pin", VERIFY_PINS, ids=[p.__name__ for p in VERIFY_PINS])
+def test_oracle_verify_pin(pin):
+    pin(oracle.gqa_decode_verify)
