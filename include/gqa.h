@@ -237,6 +237,33 @@ int gqa_decode_split_lse(const void *q, const void *k_cache, const void *v_cache
                          size_t workspace_bytes, void *stream);
 
 /*
+ * gqa_decode_verify -- decode of n_query new tokens per sequence at once, as
+ * when a target model verifies the draft tokens of speculative decoding.  The
+ * drafts are already in the cache (seqlens[s] counts them); query token t of
+ * sequence s attends the cached positions before it and itself,
+ *     j < seqlens[s] - (n_query - 1 - t),
+ * the end-aligned mask of a causal decoder.  For each KV group, the n_query * r
+ * (token, head) pairs form the group's rows and share each K/V tile read from
+ * HBM, so the cache is read once per step for all drafts.
+ *
+ * q: bf16 [b, n_query, H, d]; out: fp32 [b, n_query, H, d]; lse: fp32
+ * [b, n_query, H] or NULL (the natural-log normaliser of each row, as in
+ * gqa_decode_split_lse).  1 <= n_query <= 64.  A length below n_query is
+ * invalid (GQA_STATUS_BAD_SEQLEN, rows zeroed).  The workspace comes from
+ * gqa_decode_verify_workspace_size for the same dims, n_query, max_seqlen
+ * and split_tokens; everything else as gqa_decode_split (the CUDA-core
+ * contraction flag needs n_query == 1).  n_query == 1 is gqa_decode_split.
+ */
+size_t gqa_decode_verify_workspace_size(const gqa_dims *dims, int32_t n_query, int32_t max_seqlen,
+                                        int32_t split_tokens);
+
+int gqa_decode_verify(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *seqlens, const int32_t *page_table, float *out, float *lse,
+                      const gqa_dims *dims, int32_t n_query, float scale, uint32_t *status,
+                      int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                      size_t workspace_bytes, void *stream);
+
+/*
  * gqa_merge_lse -- merges n_parts normalised partial results of the same rows,
  * each weighted by its log-sum-exp:
  *     LSE = ln sum_k exp(lse_k),   out = sum_k exp(lse_k - LSE) o_k.

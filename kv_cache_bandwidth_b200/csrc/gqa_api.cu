@@ -97,14 +97,18 @@ struct Shape {
   int b, H, G, r, D, P, num_pages, max_pages;
   bool paged;
   long long capacity;
-  int nt, nhb;  // kernel variant: n8 head tiles per consumer warp, head blocks of 8
-  int rc, hs;   // heads per block (min(r, 16)) and 16-head slices per group
+  int nt, nhb;  // kernel variant: n8 row tiles per consumer warp, row blocks of 8
+  int nq, rq;   // query tokens per sequence and rows per group (nq * r, token-major)
+  int rc, hs;   // rows per block (min(rq, 16)) and 16-row slices per group
   bool fma;     // q.k and p.v on CUDA cores instead of tensor cores
 };
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_dims(const gqa_dims *dims, bool paged, Shape *sh) {
+// Largest number of query tokens per sequence (speculative verification).
+constexpr int kMaxQueryTokens = 64;
+
+int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1) {
   if (!dims) return GQA_ERR_NULL_POINTER;
   const gqa_dims &d = *dims;
   if (d.batch < 1 || d.num_heads < 1 || d.num_kv_heads < 1 || d.page_size < 1) return GQA_ERR_DIMS;
@@ -136,16 +140,20 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh) {
     s.capacity = d.page_size;
   }
   if (s.capacity > (1ll << 30)) return GQA_ERR_DIMS;
-  if (static_cast<long long>(s.b) * s.H * s.D > (1ll << 31) - 1) return GQA_ERR_DIMS;
-  // A block serves at most 16 heads (two head blocks of 8); larger groups are
-  // cut into 16-head slices handled by separate blocks that stream the same
-  // KV range (the repeats of a tile are L2 hits).
-  s.rc = std::min(r, 16);
-  s.hs = (r + s.rc - 1) / s.rc;
+  if (nq < 1 || nq > kMaxQueryTokens) return GQA_ERR_DIMS;
+  if (static_cast<long long>(s.b) * nq * s.H * s.D > (1ll << 31) - 1) return GQA_ERR_DIMS;
+  // The rows of a group are its (query token, head) pairs, token-major.  A
+  // block serves at most 16 rows (two row blocks of 8); larger groups are cut
+  // into 16-row slices handled by separate blocks that stream the same KV
+  // range (the repeats of a tile are L2 hits).
+  s.nq = nq;
+  s.rq = nq * r;
+  s.rc = std::min(s.rq, 16);
+  s.hs = (s.rq + s.rc - 1) / s.rc;
   s.nt = 1;
   s.nhb = (s.rc + 7) / 8;
   s.fma = (d.flags & GQA_FLAG_CONTRACT_FMA) != 0;
-  if (s.fma && r > 2) return GQA_ERR_HEADS;  // the CUDA-core contraction covers r <= 2
+  if (s.fma && (r > 2 || nq > 1)) return GQA_ERR_HEADS;  // the CUDA-core contraction covers r <= 2, one token
   *sh = s;
   return GQA_OK;
 }
@@ -172,7 +180,7 @@ long long units_of(const Shape &sh) { return static_cast<long long>(sh.b) * sh.G
 
 Workspace workspace_layout(const Shape &sh, int num_splits) {
   Workspace w;
-  const size_t rows = static_cast<size_t>(sh.b) * sh.H * num_splits;
+  const size_t rows = static_cast<size_t>(sh.b) * sh.nq * sh.H * num_splits;
   w.o_bytes = round256(rows * sh.D * sizeof(float));
   w.m_bytes = round256(rows * sizeof(float));
   w.ctr_off = w.o_bytes + 2 * w.m_bytes;
@@ -326,6 +334,8 @@ DecodeParams base_params(const Shape &sh, const void *q, const int32_t *seqlens,
   p.H = sh.H;
   p.G = sh.G;
   p.r = sh.r;
+  p.nq = sh.nq;
+  p.rq = sh.rq;
   p.rc = sh.rc;
   p.hs = sh.hs;
   p.page_size = sh.P;
@@ -341,6 +351,7 @@ DecodeParams base_params(const Shape &sh, const void *q, const int32_t *seqlens,
 struct RowExtras {
   float *lse = nullptr;
   bool empty_ok = false;
+  int nq = 1;  // query tokens per sequence
 };
 
 // The items kernel: one block per (sequence, group, split) item.
@@ -442,6 +453,8 @@ int run_balanced_combine(const Shape &sh, const int32_t *seqlens, float *out, ui
   c.r = sh.r;
   c.rc = sh.rc;
   c.hs = sh.hs;
+  c.nq = sh.nq;
+  c.rq = sh.rq;
   c.lse = ex.lse;
   c.empty_ok = ex.empty_ok ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
@@ -505,8 +518,8 @@ AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
 
 // split_tokens == 0 in the split API: checks shared by its entry points.
 int prepare_auto(const gqa_dims *dims, bool paged, int32_t max_seqlen, const void *workspace,
-                 size_t workspace_bytes, Shape *sh) {
-  int rc = check_dims(dims, paged, sh);
+                 size_t workspace_bytes, Shape *sh, int nq = 1) {
+  int rc = check_dims(dims, paged, sh, nq);
   if (rc != GQA_OK) return rc;
   if (max_seqlen < 1) return GQA_ERR_DIMS;
   if (!workspace) return GQA_ERR_WORKSPACE;
@@ -522,8 +535,8 @@ struct SplitArgs {
 };
 
 int prepare_split(const gqa_dims *dims, bool paged, int32_t split_tokens, int32_t max_seqlen,
-                  const void *workspace, size_t workspace_bytes, int sms, SplitArgs *out) {
-  int rc = check_dims(dims, paged, &out->sh);
+                  const void *workspace, size_t workspace_bytes, int sms, SplitArgs *out, int nq = 1) {
+  int rc = check_dims(dims, paged, &out->sh, nq);
   if (rc != GQA_OK) return rc;
   if (max_seqlen < 1) return GQA_ERR_DIMS;
   if (split_tokens <= 0 || split_tokens % kSplitQuantum != 0) return GQA_ERR_SPLIT;
@@ -571,7 +584,9 @@ int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t
   c.num_splits = a.num_splits;
   c.lse = ex.lse;
   c.empty_ok = ex.empty_ok ? 1 : 0;
-  const int rows = a.sh.b * a.sh.H;
+  c.nq = a.sh.nq;
+  c.rq = a.sh.rq;
+  const int rows = a.sh.b * a.sh.nq * a.sh.H;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows, 1, 1);
   cfg.blockDim = dim3(128, 1, 1);
@@ -603,7 +618,8 @@ int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, c
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (split_tokens == 0) {
     Shape sh;
-    if ((rc = prepare_auto(dims, page_table != nullptr, max_seqlen, workspace, workspace_bytes, &sh)) != GQA_OK)
+    if ((rc = prepare_auto(dims, page_table != nullptr, max_seqlen, workspace, workspace_bytes, &sh, ex.nq)) !=
+        GQA_OK)
       return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
@@ -618,7 +634,7 @@ int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, c
   }
   SplitArgs a;
   rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace,
-                     workspace_bytes, 0, &a);
+                     workspace_bytes, 0, &a, ex.nq);
   if (rc != GQA_OK) return rc;
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
@@ -787,6 +803,28 @@ int gqa_decode_split_lse(const void *q, const void *k_cache, const void *v_cache
   RowExtras ex;
   ex.lse = lse;
   ex.empty_ok = true;
+  return decode_split_impl(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status, split_tokens,
+                           max_seqlen, workspace, workspace_bytes, stream, ex);
+}
+
+size_t gqa_decode_verify_workspace_size(const gqa_dims *dims, int32_t n_query, int32_t max_seqlen,
+                                        int32_t split_tokens) {
+  Shape sh;
+  if (!dims || check_dims(dims, false, &sh, n_query) != GQA_OK) return 0;
+  if (max_seqlen < 1 || split_tokens < 0 || split_tokens % kSplitQuantum != 0) return 0;
+  if (split_tokens == 0) return auto_workspace_bytes(sh, max_seqlen);
+  return workspace_layout(sh, (max_seqlen + split_tokens - 1) / split_tokens).total;
+}
+
+int gqa_decode_verify(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                      const int32_t *page_table, float *out, float *lse, const gqa_dims *dims, int32_t n_query,
+                      float scale, uint32_t *status, int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                      size_t workspace_bytes, void *stream) {
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GQA_ERR_MISALIGNED;
+  if (n_query < 1 || n_query > kMaxQueryTokens) return GQA_ERR_DIMS;
+  RowExtras ex;
+  ex.lse = lse;
+  ex.nq = n_query;
   return decode_split_impl(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status, split_tokens,
                            max_seqlen, workspace, workspace_bytes, stream, ex);
 }

@@ -80,7 +80,8 @@ struct DecodeParams {
   unsigned long long *unit_ctr;  // items mode: arrival word per unit, or null (the merge is left to the combine)
   unsigned long long epoch;      // items mode: this call's tag in the arrival words, 1 .. 2^40 - 2
   int H, G, r;                // query heads, KV groups, heads per group
-  int rc, hs;                 // heads per block (min(r, 16)) and head slices per group (ceil(r / rc))
+  int nq, rq;                 // query tokens per sequence, rows per group (nq * r, token-major)
+  int rc, hs;                 // rows per block (min(rq, 16)) and row slices per group (ceil(rq / rc))
   int page_size;              // paged: tokens per page; contiguous: capacity m
   int num_pages;              // paged: pages in the pool
   int max_pages;              // paged: page-table row stride
@@ -100,11 +101,19 @@ struct CombineParams {
   uint32_t *status;
   int b, H, max_len, split_tokens, num_splits;
   int G, r, rc, hs;           // balanced mode
+  int nq, rq;                 // query tokens per sequence, rows per group
   const int *ws_header;       // balanced mode: {decode blocks, capacity, W lo, W hi}
   const int4 *ws_meta;        // balanced mode: per unit {first block, last block, slot in first block}
   float *lse;                 // [b, H] or null, as in DecodeParams
   int empty_ok;
 };
+
+// Row of q / out ([b, nq, H] flattened) for row rho = t * r + h (query token t,
+// head h of the group) of KV group g of sequence s.
+__device__ __forceinline__ size_t out_row(int s, int g, int rho, int nq, int r, int H) {
+  const int t = rho / r, h = rho - t * r;
+  return (static_cast<size_t>(s) * nq + t) * H + static_cast<size_t>(g) * r + h;
+}
 
 // Natural-log sum of exp over a row from its base-2 state: the row's
 // exponentials sum to L * 2^M, so ln(sum) = (M + log2 L) ln 2; -inf for a
@@ -193,9 +202,9 @@ __device__ __forceinline__ Piece make_item(const DecodeParams &p) {
     it.s = blockIdx.z;
   }
   it.h0 = it.j * p.rc;
-  it.nh = min(p.rc, p.r - it.h0);
+  it.nh = min(p.rc, p.rq - it.h0);
   it.len = __ldg(p.seqlens + it.s);
-  it.len_ok = it.len >= 1 && it.len <= p.capacity;
+  it.len_ok = it.len >= p.nq && it.len <= p.capacity;
   it.t_begin = 0;
   it.t_end = 0;
   it.final_row = false;
@@ -218,10 +227,10 @@ __device__ __forceinline__ Piece make_item(const DecodeParams &p) {
 
 // Tiles of each (sequence, group) unit of sequence s; 0 for an invalid length.
 template <int T>
-__device__ __forceinline__ int unit_tiles(const int32_t *seqlens, int capacity, int s, int *len_out) {
+__device__ __forceinline__ int unit_tiles(const int32_t *seqlens, int capacity, int nq, int s, int *len_out) {
   const int len = __ldg(seqlens + s);
   *len_out = len;
-  return (len >= 1 && len <= capacity) ? (len + T - 1) / T : 0;
+  return (len >= nq && len <= capacity) ? (len + T - 1) / T : 0;
 }
 
 __device__ __forceinline__ long long warp_sum64(long long v) {
@@ -235,12 +244,12 @@ __device__ __forceinline__ long long warp_sum64(long long v) {
 // and gets the same answer.
 template <int T>
 __device__ __forceinline__ long long total_tiles(const int32_t *seqlens, int b, int units_per_seq,
-                                                 int capacity, int lane) {
+                                                 int capacity, int nq, int lane) {
   long long tot = 0;
   for (int base = 0; base < b; base += 32) {
     const int s = base + lane;
     int len;
-    tot += (s < b) ? unit_tiles<T>(seqlens, capacity, s, &len) : 0;
+    tot += (s < b) ? unit_tiles<T>(seqlens, capacity, nq, s, &len) : 0;
   }
   return warp_sum64(tot) * units_per_seq;
 }
@@ -255,7 +264,7 @@ struct Walker {
 
 template <int T>
 __device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, int lane) {
-  const long long W = total_tiles<T>(p.seqlens, p.b, p.G * p.hs, p.capacity, lane);
+  const long long W = total_tiles<T>(p.seqlens, p.b, p.G * p.hs, p.capacity, p.nq, lane);
   const long long N = gridDim.x, c = blockIdx.x;
   const long long start = c * W / N;
   wk.remaining = (c + 1) * W / N - start;
@@ -271,7 +280,7 @@ __device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, i
     const int s = base + lane;
     int len = 0;
     const long long t =
-        (s < p.b) ? static_cast<long long>(unit_tiles<T>(p.seqlens, p.capacity, s, &len)) * p.G * p.hs : 0;
+        (s < p.b) ? static_cast<long long>(unit_tiles<T>(p.seqlens, p.capacity, p.nq, s, &len)) * p.G * p.hs : 0;
     long long inc = t;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -306,7 +315,7 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
   pc.g = wk.g;
   pc.j = wk.j;
   pc.h0 = wk.j * p.rc;
-  pc.nh = min(p.rc, p.r - pc.h0);
+  pc.nh = min(p.rc, p.rq - pc.h0);
   pc.k = 0;
   pc.len = wk.len_s;
   pc.len_ok = true;
@@ -331,7 +340,7 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
         if (++wk.g == p.G) {
           wk.g = 0;
           ++wk.s;
-          wk.tiles_s = unit_tiles<T>(p.seqlens, p.capacity, wk.s, &wk.len_s);
+          wk.tiles_s = unit_tiles<T>(p.seqlens, p.capacity, p.nq, wk.s, &wk.len_s);
         }
       }
     } while (wk.tiles_s == 0);
@@ -781,7 +790,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         const bool empty = p.empty_ok && pc.len == 0;
         for (int idx = threadIdx.x; idx < pc.nh * (D / 4); idx += blockDim.x) {
           const int h = idx / (D / 4), c4 = idx % (D / 4);
-          const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
+          const size_t row = out_row(pc.s, pc.g, pc.h0 + h, p.nq, p.r, p.H);
           if (p.out) reinterpret_cast<float4 *>(p.out + row * D)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLBadLength;
           if (c4 == 0 && p.lse) p.lse[row] = kNegInf;
@@ -849,9 +858,15 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       if (lane == 0) {
         const uint32_t q_bytes = static_cast<uint32_t>(pc.nh * D * 2);
         mbar_arrive_expect_tx(bar_qfull + 8 * qs, q_bytes);
-        bulk_load(q_sm + qs * TL::kQBytes,
-                  p.q + (static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0) * D,
-                  q_bytes, bar_qfull + 8 * qs);
+        // the slice's rows, in runs of consecutive heads of one query token
+        // (one run when there is one query token per sequence)
+        for (int rho = 0; rho < pc.nh;) {
+          const int a = pc.h0 + rho;
+          const int run = min(pc.nh - rho, p.r - a % p.r);
+          bulk_load(q_sm + qs * TL::kQBytes + rho * D * 2, p.q + out_row(pc.s, pc.g, a, p.nq, p.r, p.H) * D,
+                    static_cast<uint32_t>(run * D * 2), bar_qfull + 8 * qs);
+          rho += run;
+        }
       }
       ++n;
       // ---- K/V tiles
@@ -990,6 +1005,19 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
 #pragma unroll
         for (int mt = 0; mt < TL::kSteps; ++mt) o[mt][j][0] = o[mt][j][1] = o[mt][j][2] = o[mt][j][3] = 0.f;
       }
+      // End (exclusive) of the positions each of this lane's two rows sees in
+      // the piece: with several query tokens per sequence, query token t sees
+      // the cache up to and including itself, len - (nq - 1 - t); with one it
+      // is the piece's end.
+      int lim[NT][2];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int rho = pc.h0 + hb * TL::kHB + j * 8 + 2 * t4 + e;
+          lim[j][e] = min(pc.t_end, pc.len - (p.nq - 1 - rho / p.r));
+        }
+      }
 
       for (int t0 = pc.t_begin; t0 < pc.t_end; t0 += T, ++tile) {
         const int stage = tile % STAGES;
@@ -1030,8 +1058,6 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
           }
           // ---- mask, scale, online softmax, P^T fragments
           const int tok_a = t0 + row0 + g8;
-          const bool ok_a = tok_a < pc.t_end;
-          const bool ok_b = tok_a + 8 < pc.t_end;
           uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
@@ -1042,10 +1068,10 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
 #pragma unroll
               for (int c2 = 1; c2 < kChains; ++c2) sum[e] += sacc[c2][j][e];
             }
-            const float x0 = ok_a ? sum[0] * sl : kNegInf;  // token g8,   head 2*t4
-            const float x1 = ok_a ? sum[1] * sl : kNegInf;  // token g8,   head 2*t4+1
-            const float x2 = ok_b ? sum[2] * sl : kNegInf;  // token g8+8, head 2*t4
-            const float x3 = ok_b ? sum[3] * sl : kNegInf;  // token g8+8, head 2*t4+1
+            const float x0 = tok_a < lim[j][0] ? sum[0] * sl : kNegInf;      // token g8,   row 2*t4
+            const float x1 = tok_a < lim[j][1] ? sum[1] * sl : kNegInf;      // token g8,   row 2*t4+1
+            const float x2 = tok_a + 8 < lim[j][0] ? sum[2] * sl : kNegInf;  // token g8+8, row 2*t4
+            const float x3 = tok_a + 8 < lim[j][1] ? sum[3] * sl : kNegInf;  // token g8+8, row 2*t4+1
             // The exponentials use a base m_run that may trail the true running
             // maximum by up to kSlack (p <= 2^kSlack): any base gives the same
             // normalised result as long as l and o share it.  Only when a score
@@ -1199,21 +1225,13 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       }
       if (MODE != Mode::kCluster) {
         const int n4 = D / 4;
-        bool final_row;
-        size_t pslot_base = 0;  // partial slot: index of head 0 in the m/l arrays
-        size_t pslot_stride = 1;
-        if (BAL) {
-          final_row = pc.final_row;
-          pslot_base = static_cast<size_t>(pc.slot) * p.rc;
-        } else {
-          final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
-          pslot_base =
-              (static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0) * p.num_splits + pc.k;
-          pslot_stride = p.num_splits;
-        }
+        // partial slot of a row: balanced mode, the block's slot (rc rows
+        // each); fixed splits, split k of the output row ([b, nq, H, S])
+        const bool final_row =
+            BAL ? pc.final_row : (((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr);
         for (int idx = ctid; idx < pc.nh * n4; idx += nc * 32) {
           const int h = idx / n4, c4 = idx % n4;
-          const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
+          const size_t row = out_row(pc.s, pc.g, pc.h0 + h, p.nq, p.r, p.H);
           const float4 src = *reinterpret_cast<const float4 *>(osum + h * TL::kOStride + 4 * c4);
           if (final_row) {
             const float L = L_blk[h];
@@ -1223,7 +1241,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
             if (c4 == 0 && p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(M_blk[h], L);
             if (!BAL && c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLFinal;
           } else {
-            const size_t ps = pslot_base + static_cast<size_t>(h) * pslot_stride;
+            const size_t ps = BAL ? static_cast<size_t>(pc.slot) * p.rc + h : row * p.num_splits + pc.k;
             reinterpret_cast<float4 *>(p.part_o + ps * D)[c4] = src;
             if (c4 == 0) {
               p.part_m[ps] = M_blk[h];
@@ -1256,7 +1274,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
             static_assert(TL::kRPad * kHalf <= nc * 32, "one pass of the consumer threads");
             const int h = ctid / kHalf, c4 = ctid % kHalf;
             if (h < pc.nh) {
-              const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
+              const size_t row = out_row(pc.s, pc.g, pc.h0 + h, p.nq, p.r, p.H);
               merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(row) * p.num_splits, ns,
                                  c4, kHalf, reinterpret_cast<float4 *>(p.out + row * D),
                                  p.lse ? p.lse + row : nullptr);
@@ -1300,7 +1318,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         }
         float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
         if (L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
-        const size_t row = static_cast<size_t>(pc.s) * p.H + static_cast<size_t>(pc.g) * p.r + pc.h0 + h;
+        const size_t row = out_row(pc.s, pc.g, pc.h0 + h, p.nq, p.r, p.H);
         reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
       }
       if (threadIdx.x == 0 && !pc.len_ok && p.status) atomicOr(p.status, kStatusBadSeqlen);
@@ -1313,13 +1331,13 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
 // k < ceil(len / split_tokens) of that row.
 template <int D>
 __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p) {
-  const int row = blockIdx.x;
-  const int s = row / p.H;
+  const int row = blockIdx.x;       // [b, nq, H] flattened
+  const int s = row / (p.nq * p.H);
   const int len = __ldg(p.seqlens + s);
   float4 *dst = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D) + threadIdx.x % (D / 4);
   pdl_wait_primary();  // the partial states below come from the preceding kernel
   float *lse_dst = p.lse ? p.lse + row : nullptr;
-  if (len < 1 || len > p.max_len) {
+  if (len < p.nq || len > p.max_len) {
     if (threadIdx.x < D / 4) *dst = make_float4(0.f, 0.f, 0.f, 0.f);
     if (threadIdx.x == 0 && lse_dst) *lse_dst = -__int_as_float(0x7f800000);
     if (threadIdx.x == 0 && p.status && !(p.empty_ok && len == 0)) atomicOr(p.status, kStatusBadSeqlen);
@@ -1351,15 +1369,15 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
   const int h = blockIdx.x % p.rc;
   const int j = u % p.hs;
   const int s = u / (p.G * p.hs), g = (u / p.hs) % p.G;
-  if (j * p.rc + h >= p.r) return;  // the last slice of the group is narrower
-  const size_t row = static_cast<size_t>(s) * p.H + static_cast<size_t>(g) * p.r + j * p.rc + h;
+  if (j * p.rc + h >= p.rq) return;  // the last slice of the group is narrower
+  const size_t row = out_row(s, g, j * p.rc + h, p.nq, p.r, p.H);
   float4 *dst = reinterpret_cast<float4 *>(p.out + row * D) + threadIdx.x % (D / 4);
   const int len = __ldg(p.seqlens + s);
   pdl_wait_primary();  // the header, unit records and partial states come from the decode kernel
   const int N = p.ws_header[0];
   const int capacity = p.ws_header[1];
   float *lse_dst = p.lse ? p.lse + row : nullptr;
-  if (len < 1 || len > capacity) {
+  if (len < p.nq || len > capacity) {
     if (threadIdx.x < D / 4) *dst = make_float4(0.f, 0.f, 0.f, 0.f);
     if (threadIdx.x == 0 && lse_dst) *lse_dst = -__int_as_float(0x7f800000);
     if (threadIdx.x == 0 && h == 0 && p.status && !(p.empty_ok && len == 0)) atomicOr(p.status, kStatusBadSeqlen);

@@ -26,6 +26,7 @@ __all__ = [
     "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
     "FLAG_CONTRACT_FMA", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
     "gqa_decode_split_lse", "gqa_merge_lse", "SERIAL_MERGE_MAX_SPLITS", "gqa_kv_append", "PagePool",
+    "gqa_decode_verify", "gqa_decode_verify_workspace_size",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -99,6 +100,12 @@ def load():
                                          _vp, ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
     lib.gqa_merge_lse.restype = ctypes.c_int
     lib.gqa_merge_lse.argtypes = [_vp, _vp, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp]
+    lib.gqa_decode_verify.restype = ctypes.c_int
+    lib.gqa_decode_verify.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), ctypes.c_int32,
+                                      ctypes.c_float, _vp, ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
+    lib.gqa_decode_verify_workspace_size.restype = ctypes.c_size_t
+    lib.gqa_decode_verify_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32,
+                                                     ctypes.c_int32]
     lib.gqa_kv_append.restype = ctypes.c_int
     lib.gqa_kv_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), _vp, _vp]
     lib.gqa_page_pool_create.restype = _vp
@@ -255,6 +262,38 @@ def gqa_merge_lse(o_parts, lse_parts, *, out=None, lse_out=None, stream=None):
                               _ptr(lse_out), _stream(stream))
     _check(rc, "gqa_merge_lse")
     return out, lse_out
+
+
+def gqa_decode_verify_workspace_size(dims: Dims, n_query: int, max_seqlen: int, split_tokens: int) -> int:
+    return int(load().gqa_decode_verify_workspace_size(ctypes.byref(dims), int(n_query), int(max_seqlen),
+                                                       int(split_tokens)))
+
+
+def gqa_decode_verify(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int = 0,
+                      max_seqlen: Optional[int] = None, workspace=None, out=None, lse=None, want_lse: bool = False,
+                      scale=None, status=None, stream=None, flags: int = 0):
+    """Decode of n_query tokens per sequence (q [b, n_query, H, d]); token t
+    sees the cache up to seqlens[s] - (n_query - 1 - t).  Returns out
+    [b, n_query, H, d] (and lse [b, n_query, H] when want_lse or lse is given)."""
+    b, nq, H, d = q.shape
+    if out is None:
+        out = torch.empty((b, nq, H, d), dtype=torch.float32, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((b, nq, H), dtype=torch.float32, device=q.device)
+    if max_seqlen is None:
+        max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
+    pages, G, P, _ = k_cache.shape
+    dims = Dims(b, H, G, d, P, pages, 0 if page_table is None else page_table.shape[1], flags)
+    if workspace is None:
+        # (a size of 0 means invalid arguments: the call below names the error)
+        n = gqa_decode_verify_workspace_size(dims, nq, max_seqlen, split_tokens)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    rc = load().gqa_decode_verify(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table), _ptr(out),
+                                  _ptr(lse), ctypes.byref(dims), int(nq), _scale(q, scale), _ptr(status),
+                                  int(split_tokens), int(max_seqlen), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "gqa_decode_verify")
+    return (out, lse) if lse is not None else out
 
 
 def gqa_kv_append(k_new, v_new, k_cache, v_cache, seqlens, page_table=None, *, num_heads: Optional[int] = None,
