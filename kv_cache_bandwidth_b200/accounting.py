@@ -18,7 +18,7 @@ from typing import Iterable
 
 __all__ = [
     "kv_cache_elements", "kv_cache_bytes", "kv_bytes_per_step", "mha_to_gqa_reduction",
-    "decode_flops", "total_bytes_per_step", "page_block_bytes",
+    "decode_flops", "total_bytes_per_step", "page_block_bytes", "kv_bytes_unique_pages",
 ]
 
 
@@ -62,3 +62,23 @@ def total_bytes_per_step(b: int, num_heads: int, kv_heads: int, head_dim: int,
     seqlens = list(seqlens)
     return (kv_bytes_per_step(kv_heads, head_dim, seqlens) + b * num_heads * head_dim * 2
             + b * num_heads * head_dim * out_bytes + 4 * b + 4 * page_table_entries)
+
+
+def kv_bytes_unique_pages(kv_heads: int, head_dim: int, page_size: int, page_table, seqlens,
+                          elem_bytes: int = 2) -> int:
+    """KV bytes of a paged step counting every physical page once: the rows of
+    page p that any sequence reads (up to the largest offset any sequence uses
+    in it), K and V, all groups.  With pages shared between sequences (a
+    common prompt prefix stored once and referenced from several page-table
+    rows, as in the paged cache of the llms.blog page's "PagedAttention") this
+    is below kv_bytes_per_step, which counts what each sequence reads; the
+    decode kernels read per sequence, so the difference is what L2 can serve
+    when the sharing sequences run close together."""
+    rows_used = {}
+    for s, n in enumerate(seqlens):
+        n = int(n)
+        for lp in range(-(-n // page_size)):
+            pid = int(page_table[s][lp])
+            used = min(page_size, n - lp * page_size)
+            rows_used[pid] = max(rows_used.get(pid, 0), used)
+    return 2 * kv_heads * head_dim * elem_bytes * sum(rows_used.values())

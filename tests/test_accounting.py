@@ -80,3 +80,16 @@ def test_peaky_rows():
     assert (scaled | same).all()
     assert scaled.sum(dim=-1).tolist() == [[10, 10]], "1% of 1000 rows per group"
     assert torch.equal(peaky.v_cache, plain.v_cache)
+
+
+def test_unique_page_bytes_with_a_shared_prefix():
+    P, G, d = 16, 8, 128
+    per_token = 2 * G * d * 2
+    # three sequences share a 40-token prefix (pages 0, 1 and the first 8 rows of 2)
+    table = [[0, 1, 2, 3], [0, 1, 2, 4], [0, 1, 2, 5]]
+    lens = [50, 64, 40]
+    assert accounting.kv_bytes_per_step(G, d, lens) == sum(lens) * per_token
+    # page 2 is read up to row 16 (sequences 0 and 1 pass it); pages 3/4/5 hold 2, 16, 0 rows
+    assert accounting.kv_bytes_unique_pages(G, d, P, table, lens) == (16 + 16 + 16 + 2 + 16) * per_token
+    # no sharing: the two counts agree
+    assert accounting.kv_bytes_unique_pages(G, d, P, [[0, 1], [2, 3]], [20, 32]) == accounting.kv_bytes_per_step(G, d, [20, 32])

@@ -454,3 +454,43 @@ def test_full_size_workload_sampled(name):
         got, st = run_gpu(inp, entry, split_tokens=split)
         assert st == 0
         assert_parity(got.view(-1, w.d)[torch.from_numpy(rows).cuda()], ref, "%s %s split=%d" % (name, entry, split))
+
+
+@pytest.mark.parametrize("entry,split", [("cluster", 0), ("split", 0), ("split", 128)])
+def test_prefix_shared_pages(entry, split):
+    """Sequences that share a prompt prefix reference the same physical pages
+    from their page-table rows (aliasing).  The decode must equal the oracle
+    and, bit for bit, the same cache with every shared page duplicated."""
+    P, prefix_pages = 16, 5
+    lens = [prefix_pages * P + 37, prefix_pages * P, prefix_pages * P + 200, 3 * P + 5]
+    w = w_small(b=len(lens), r=8, G=2, d=128, m=512, P=P, seed=44)
+    base = make_inputs(w, device="cuda", lens=lens, spare_pages=prefix_pages * 3)
+    shared = base.page_table.clone()
+    dup = base.page_table.clone()
+    kd, vd = base.k_cache.clone(), base.v_cache.clone()
+    # sequences 1 and 2 take sequence 0's prefix pages (sequence 3 is shorter: its first 3 pages)
+    used = set(int(x) for x in base.page_table.flatten().tolist() if x >= 0)
+    spare = sorted(set(range(base.k_cache.shape[0])) - used)
+    for s in (1, 2, 3):
+        n = prefix_pages if s < 3 else 3
+        for lp in range(n):
+            src = int(base.page_table[0, lp])
+            shared[s, lp] = src
+            fresh = spare.pop()
+            kd[fresh] = base.k_cache[src]
+            vd[fresh] = base.v_cache[src]
+            dup[s, lp] = fresh
+    a_inp = base
+    a_inp.page_table.copy_(shared)
+    ref, st = run_oracle(a_inp)
+    assert st == 0
+    got, st = run_gpu(a_inp, entry, split_tokens=split)
+    assert st == 0
+    assert_parity(got, ref, "shared prefix %s %d" % (entry, split))
+    b_inp = make_inputs(w, device="cuda", lens=lens, spare_pages=prefix_pages * 3)
+    b_inp.q.copy_(base.q)
+    b_inp.k_cache.copy_(kd)
+    b_inp.v_cache.copy_(vd)
+    b_inp.page_table.copy_(dup)
+    got_dup, _ = run_gpu(b_inp, entry, split_tokens=split)
+    assert torch.equal(got, got_dup)
