@@ -257,7 +257,11 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
     cfg.blockDim = dim3(TL::kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = l.stream;
-    cfg.numAttrs = 0;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) != cudaSuccess) return GQA_ERR_CUDA;
     return static_cast<int>(l.grid.x);  // > 0: the number of decode blocks
   }
@@ -267,14 +271,18 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
   cfg.dynamicSmemBytes = smem;
   cfg.stream = l.stream;
   cudaLaunchAttribute attr[1];
-  cfg.numAttrs = 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (MODE == Mode::kCluster) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = l.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+  } else {
+    // items mode: may start while the previous kernel on the stream finishes
+    // (the kernel waits for it before touching memory)
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
   }
   return cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }

@@ -777,6 +777,12 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (items and balanced modes), the blocks may start while it finishes: wait
+  // for it to complete (and its memory to be visible) before reading anything
+  // it may have written (q, lengths, page table, cache, workspace).  A no-op
+  // when the launch is an ordinary one.
+  pdl_wait_primary();
   Piece pc;
   if (!BAL) pc = make_item<T, MODE>(p);
   if (MODE == Mode::kItems) {
