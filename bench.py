@@ -406,51 +406,74 @@ def main_gpu(args):
 def e2e_leg(args, inp, split, max_seqlen, ws, kv_step, world):
     """Same metric through the public call with host buffers: each step copies the
     step's inputs (q, lengths, page table) from pinned host memory, runs the
-    decode and reads the result back.  The KV cache is the decode state and
-    stays resident in HBM."""
+    decode and reads the result back into pinned host memory.  The KV cache is
+    the decode state and stays resident in HBM.
+
+    Steps are pipelined the way a serving loop would run them: two sets of
+    device input/output buffers, the copies on their own streams (the copy
+    engines) and the decode on a compute stream, so step i+1's inputs travel
+    and step i-1's result returns while step i decodes.  Events order every
+    buffer reuse."""
     from kv_cache_bandwidth_b200 import gqa
 
     h_q = inp.q.cpu().pin_memory()
     h_sl = inp.seqlens.cpu().pin_memory()
     h_pt = None if inp.page_table is None else inp.page_table.cpu().pin_memory()
-    h_out = torch.empty(inp.q.shape, dtype=torch.float32).pin_memory()
-    d_q = torch.empty_like(inp.q)
-    d_sl = torch.empty_like(inp.seqlens)
-    d_pt = None if h_pt is None else torch.empty_like(inp.page_table)
-    d_out = torch.empty(inp.q.shape, dtype=torch.float32, device="cuda")
-    stream = torch.cuda.current_stream()
+    h_out = [torch.empty(inp.q.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    d_q = [torch.empty_like(inp.q) for _ in range(2)]
+    d_sl = [torch.empty_like(inp.seqlens) for _ in range(2)]
+    d_pt = [None if h_pt is None else torch.empty_like(inp.page_table) for _ in range(2)]
+    d_out = [torch.empty(inp.q.shape, dtype=torch.float32, device="cuda") for _ in range(2)]
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in comp_done + out_done:
+        e.record(torch.cuda.current_stream())
     h2d = h_q.numel() * h_q.element_size() + h_sl.numel() * 4 + (0 if h_pt is None else h_pt.numel() * 4)
-    d2h = h_out.numel() * 4
+    d2h = h_out[0].numel() * 4
 
-    def step():
-        d_q.copy_(h_q, non_blocking=True)
-        d_sl.copy_(h_sl, non_blocking=True)
-        if d_pt is not None:
-            d_pt.copy_(h_pt, non_blocking=True)
-        if args.entry == "cluster":
-            gqa.gqa_decode(d_q, inp.k_cache, inp.v_cache, d_sl, d_pt, out=d_out)
-        else:
-            gqa.gqa_decode_split(d_q, inp.k_cache, inp.v_cache, d_sl, d_pt, split_tokens=split,
-                                 max_seqlen=max_seqlen, workspace=ws, out=d_out)
-        h_out.copy_(d_out, non_blocking=True)
+    def step(i):
+        k = i % 2
+        with torch.cuda.stream(s_in):      # inputs of step i (buffer k is free once step i-2 decoded)
+            s_in.wait_event(comp_done[k])
+            d_q[k].copy_(h_q, non_blocking=True)
+            d_sl[k].copy_(h_sl, non_blocking=True)
+            if h_pt is not None:
+                d_pt[k].copy_(h_pt, non_blocking=True)
+            in_done[k].record(s_in)
+        with torch.cuda.stream(s_comp):    # decode of step i (its output buffer is free once read back)
+            s_comp.wait_event(in_done[k])
+            s_comp.wait_event(out_done[k])
+            if args.entry == "cluster":
+                gqa.gqa_decode(d_q[k], inp.k_cache, inp.v_cache, d_sl[k], d_pt[k], out=d_out[k], stream=s_comp)
+            else:
+                gqa.gqa_decode_split(d_q[k], inp.k_cache, inp.v_cache, d_sl[k], d_pt[k], split_tokens=split,
+                                     max_seqlen=max_seqlen, workspace=ws, out=d_out[k], stream=s_comp)
+            comp_done[k].record(s_comp)
+        with torch.cuda.stream(s_out):     # result of step i back to the host
+            s_out.wait_event(comp_done[k])
+            h_out[k].copy_(d_out[k], non_blocking=True)
+            out_done[k].record(s_out)
 
-    for _ in range(3):
-        step()
+    for i in range(3):
+        step(i)
     torch.cuda.synchronize()
     n = max(10, min(args.steps, 200))
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    ev0.record(stream)
-    for _ in range(n):
-        step()
-    ev1.record(stream)
+    ev0.record(s_in)
+    for i in range(n):
+        step(i)
+    s_in.wait_stream(s_out)
+    ev1.record(s_in)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(ev0.elapsed_time(ev1) / n, world)
     return {"value": world * kv_step / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "note": "q, lengths and page table H2D from pinned memory, output D2H; KV cache resident"}
+            "note": "every step: q, lengths (and page table) H2D from pinned memory, decode, output D2H to "
+                    "pinned memory; steps pipelined over copy and compute streams; KV cache resident"}
 
 
 def main(argv=None):
