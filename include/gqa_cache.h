@@ -52,6 +52,21 @@ int gqa_kv_append(const void *k_new, const void *v_new, void *k_cache, void *v_c
                   uint32_t *status, void *stream);
 
 /*
+ * gqa_append_decode_split -- one decode step of a growing cache in one call:
+ * gqa_kv_append(k_new, v_new, ...) followed by gqa_decode_split over the
+ * cache with the new token (seqlens as incremented by the append; max_seqlen
+ * bounds the lengths after it).  The decode kernel is launched as a
+ * programmatic dependent of the append, so its blocks are dispatched while
+ * the append runs and wait for it on the GPU before reading the cache.  Every
+ * argument of both steps is checked before anything is launched; the results
+ * equal the two calls made one after the other, bit for bit.
+ */
+int gqa_append_decode_split(const void *k_new, const void *v_new, const void *q, void *k_cache,
+                            void *v_cache, int32_t *seqlens, const int32_t *page_table, float *out,
+                            const gqa_dims *dims, float scale, uint32_t *status, int32_t split_tokens,
+                            int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * A pool of page ids 0 .. num_pages-1 (host memory only; no GPU call).  Ids
  * are handed out lowest first from a fresh pool and most recently freed first
  * afterwards, so a sequence of calls always gives the same ids.  All calls on

@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "gqa.h"
+#include "gqa_cache.h"
 #include "gqa_kernels.cuh"
 
 static_assert(GQA_MERGE_IN_KERNEL_MAX_SPLITS == gqa::kSerialMergeMax,
@@ -363,6 +364,7 @@ struct RowExtras {
   float *lse = nullptr;
   bool empty_ok = false;
   int nq = 1;  // query tokens per sequence
+  bool force_pdl = false;  // dependent launch even for one item per unit (behind a short kernel)
 };
 
 // The items kernel: one block per (sequence, group, split) item.
@@ -391,7 +393,7 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   // partly idle kernel (a combine, a previous step's merge); with one item per
   // unit the grid follows a full decode grid, where measured it cost ~3 %
   // (its early blocks only wait, and the grid no longer starts as one wave).
-  Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream, num_splits > 1};
+  Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream, num_splits > 1 || ex.force_pdl};
   return launch_decode<Mode::kItems>(sh, tk, tv, p, l);
 }
 
@@ -818,6 +820,32 @@ int gqa_decode_split_lse(const void *q, const void *k_cache, const void *v_cache
   RowExtras ex;
   ex.lse = lse;
   ex.empty_ok = true;
+  return decode_split_impl(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status, split_tokens,
+                           max_seqlen, workspace, workspace_bytes, stream, ex);
+}
+
+int gqa_append_decode_split(const void *k_new, const void *v_new, const void *q, void *k_cache, void *v_cache,
+                            int32_t *seqlens, const int32_t *page_table, float *out, const gqa_dims *dims,
+                            float scale, uint32_t *status, int32_t split_tokens, int32_t max_seqlen,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+  // every argument of the decode is checked before the append is launched
+  Shape sh;
+  int rc = check_dims(dims, page_table != nullptr, &sh);
+  if (rc != GQA_OK) return rc;
+  if ((rc = check_inputs(q, k_cache, v_cache, seqlens, status)) != GQA_OK) return rc;
+  if (!out) return GQA_ERR_NULL_POINTER;
+  if (!aligned16(out)) return GQA_ERR_MISALIGNED;
+  if (!std::isfinite(scale) || max_seqlen < 1) return GQA_ERR_DIMS;
+  if (split_tokens < 0 || split_tokens % kSplitQuantum != 0) return GQA_ERR_SPLIT;
+  if (!workspace) return GQA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
+  const size_t need = split_tokens == 0 ? auto_workspace_bytes(sh, max_seqlen)
+                                        : workspace_layout(sh, (max_seqlen + split_tokens - 1) / split_tokens).total;
+  if (workspace_bytes < need) return GQA_ERR_WORKSPACE;
+  rc = gqa_kv_append(k_new, v_new, k_cache, v_cache, seqlens, page_table, dims, status, stream);
+  if (rc != GQA_OK) return rc;
+  RowExtras ex;
+  ex.force_pdl = true;  // the decode's blocks are dispatched while the append runs
   return decode_split_impl(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status, split_tokens,
                            max_seqlen, workspace, workspace_bytes, stream, ex);
 }

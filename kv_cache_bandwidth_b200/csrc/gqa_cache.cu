@@ -32,6 +32,9 @@ struct AppendParams {
 template <int D>
 __global__ void __launch_bounds__(128) gqa_kv_append_kernel(const AppendParams p) {
   constexpr int kW = D / 8;
+  // A decode launched right behind this kernel as its programmatic dependent
+  // may be dispatched now; it waits for this grid to finish before it reads.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int s = blockIdx.x;
   const int t = p.seqlens[s];
   if (t < 0 || static_cast<long long>(t) >= p.capacity) {

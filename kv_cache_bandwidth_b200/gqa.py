@@ -26,7 +26,7 @@ __all__ = [
     "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
     "FLAG_CONTRACT_FMA", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
     "gqa_decode_split_lse", "gqa_merge_lse", "SERIAL_MERGE_MAX_SPLITS", "gqa_kv_append", "PagePool",
-    "gqa_decode_verify", "gqa_decode_verify_workspace_size",
+    "gqa_decode_verify", "gqa_decode_verify_workspace_size", "gqa_append_decode_split",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -106,6 +106,10 @@ def load():
     lib.gqa_decode_verify_workspace_size.restype = ctypes.c_size_t
     lib.gqa_decode_verify_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32,
                                                      ctypes.c_int32]
+    lib.gqa_append_decode_split.restype = ctypes.c_int
+    lib.gqa_append_decode_split.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims),
+                                            ctypes.c_float, _vp, ctypes.c_int32, ctypes.c_int32, _vp,
+                                            ctypes.c_size_t, _vp]
     lib.gqa_kv_append.restype = ctypes.c_int
     lib.gqa_kv_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), _vp, _vp]
     lib.gqa_page_pool_create.restype = _vp
@@ -307,6 +311,26 @@ def gqa_kv_append(k_new, v_new, k_cache, v_cache, seqlens, page_table=None, *, n
     rc = load().gqa_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
                               _ptr(page_table), ctypes.byref(dims), _ptr(status), _stream(stream))
     _check(rc, "gqa_kv_append")
+
+
+def gqa_append_decode_split(k_new, v_new, q, k_cache, v_cache, seqlens, page_table=None, *,
+                            split_tokens: int = 0, max_seqlen: Optional[int] = None, workspace=None, out=None,
+                            scale=None, status=None, stream=None, flags: int = 0) -> torch.Tensor:
+    """gqa_kv_append then gqa_decode_split in one call (the decode launched as a
+    dependent of the append).  Returns ``out``."""
+    out = _out_for(q, out)
+    if max_seqlen is None:
+        max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
+    if workspace is None:
+        workspace = workspace_for(q, k_cache, page_table, max_seqlen, split_tokens)
+    dims = dims_for(q, k_cache, page_table, flags)
+    rc = load().gqa_append_decode_split(_ptr(k_new), _ptr(v_new), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(seqlens), _ptr(page_table), _ptr(out), ctypes.byref(dims),
+                                        _scale(q, scale), _ptr(status), int(split_tokens), int(max_seqlen),
+                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream(stream))
+    _check(rc, "gqa_append_decode_split")
+    return out
 
 
 class PagePool:

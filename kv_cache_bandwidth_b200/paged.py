@@ -42,6 +42,13 @@ class PagedKVCache:
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, status: Optional[torch.Tensor] = None,
                stream=None) -> None:
         """Append one token [b, G, d] to every sequence."""
+        self._open_pages()
+        gqa.gqa_kv_append(k_new, v_new, self.k, self.v, self.seqlens, self.table, status=status, stream=stream)
+        for s in range(self.b):
+            self.lengths[s] += 1
+
+    def _open_pages(self) -> None:
+        """Give a fresh page to every sequence whose next token starts one."""
         need = [s for s in range(self.b) if self.lengths[s] % self.P == 0]
         if any(self.lengths[s] // self.P >= self.max_pages for s in need):
             raise ValueError("a sequence is at its capacity")
@@ -51,9 +58,20 @@ class PagedKVCache:
                 self.table_host[s, self.lengths[s] // self.P] = pid
             rows = torch.tensor(need, dtype=torch.int64)
             self.table[rows.to(self.table.device)] = self.table_host[rows].to(self.table.device, non_blocking=True)
-        gqa.gqa_kv_append(k_new, v_new, self.k, self.v, self.seqlens, self.table, status=status, stream=stream)
+
+    def append_decode(self, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, *, split_tokens: int = 0,
+                      max_seqlen: Optional[int] = None, workspace=None, out=None, status=None, stream=None):
+        """Append one token [b, G, d] to every sequence and decode q [b, H, d]
+        over the grown cache in one library call.  Returns the output."""
+        self._open_pages()
+        if max_seqlen is None:
+            max_seqlen = self.max_pages * self.P
+        out = gqa.gqa_append_decode_split(k_new, v_new, q, self.k, self.v, self.seqlens, self.table,
+                                          split_tokens=split_tokens, max_seqlen=max_seqlen, workspace=workspace,
+                                          out=out, status=status, stream=stream)
         for s in range(self.b):
             self.lengths[s] += 1
+        return out
 
     def free_sequence(self, s: int) -> None:
         """Return sequence s's pages to the pool; it starts again empty."""

@@ -90,3 +90,29 @@ def test_growing_cache_decodes_like_the_whole_sequence(P, split):
     lens = torch.tensor([steps, 4, steps, steps], dtype=torch.int32)
     ref, _ = oracle.gqa_decode(src.q.cpu(), src.k_cache.cpu(), src.v_cache.cpu(), lens, num_kv_heads=G)
     assert_parity(out[1], ref[1], "recycled sequence")
+
+
+@pytest.mark.parametrize("P,split", [(16, 0), (32, 128)])
+def test_append_decode_in_one_call(P, split):
+    """gqa_append_decode_split (append, then the decode as its dependent launch)
+    equals gqa_kv_append followed by gqa_decode_split bit for bit, step after
+    step, and matches the oracle."""
+    b, H, G, d, steps = 3, 16, 2, 128, 70
+    w = Workload(name="ad", b=b, H=H, G=G, d=d, m=steps, seed=303)
+    src = make_inputs(w, device="cuda", lens=[steps] * b)
+    n_pages = -(-steps // P)
+    one = PagedKVCache(b, G, d, P, num_pages=b * n_pages, max_pages_per_seq=n_pages)
+    two = PagedKVCache(b, G, d, P, num_pages=b * n_pages, max_pages_per_seq=n_pages)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for t in range(steps):
+        kn, vn = src.k_cache[:, :, t].contiguous(), src.v_cache[:, :, t].contiguous()
+        a = one.append_decode(kn, vn, src.q, split_tokens=split, status=st)
+        two.append(kn, vn, status=st)
+        c = gqa.gqa_decode_split(src.q, two.k, two.v, two.seqlens, two.table, split_tokens=split,
+                                 max_seqlen=n_pages * P, status=st)
+        torch.cuda.synchronize()
+        assert torch.equal(a, c), "step %d" % t
+    assert int(st.item()) == 0
+    ref, _ = oracle.gqa_decode(src.q.cpu(), src.k_cache.cpu(), src.v_cache.cpu(),
+                               torch.full((b,), steps, dtype=torch.int32), num_kv_heads=G)
+    assert_parity(a, ref, "append+decode")
