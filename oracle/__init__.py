@@ -72,6 +72,10 @@ def load_library(path: str):
         a = lib.oracle_gqa_decode.argtypes
         lib.oracle_gqa_decode_multi.restype = ctypes.c_int
         lib.oracle_gqa_decode_multi.argtypes = a[:6] + [ctypes.c_int32] + a[6:16] + [ctypes.c_void_p] + a[16:]
+    if hasattr(lib, "oracle_gqa_decode_mapped"):
+        a = lib.oracle_gqa_decode.argtypes
+        lib.oracle_gqa_decode_mapped.restype = ctypes.c_int
+        lib.oracle_gqa_decode_mapped.argtypes = a[:16] + [ctypes.c_void_p] + a[16:] + [ctypes.c_void_p]
     if hasattr(lib, "oracle_gqa_decode_lse"):
         lib.oracle_gqa_decode_lse.restype = ctypes.c_int
         lib.oracle_gqa_decode_lse.argtypes = lib.oracle_gqa_decode.argtypes[:16] + [ctypes.c_void_p] + \
@@ -170,7 +174,18 @@ def gqa_decode_verify(q, k_cache, v_cache, seqlens, page_table=None, *, num_kv_h
     return out, lse, status
 
 
-def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows, threads, lib, want_lse, nq=1):
+def gqa_decode_mapped(q, k_cache, v_cache, seqlens, page_table=None, *, group_of_head, scale=None, rows=None,
+                      threads: int = 0, lib=None) -> Tuple[np.ndarray, np.ndarray, int]:
+    """Decode with any group map: query head i uses KV group group_of_head[i]
+    (values in [0, G); groups may be of unequal size or empty).  Returns
+    (out [b, H, d] (or [len(rows), d]), lse, status)."""
+    gmap = np.ascontiguousarray(np.asarray(group_of_head), dtype=np.int32)
+    return _decode(q, k_cache, v_cache, seqlens, page_table, None, scale, rows, threads, lib, want_lse=True,
+                   group_map=gmap)
+
+
+def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows, threads, lib, want_lse, nq=1,
+            group_map=None):
     """Shared body of the decode functions (q given as [b, nq * H, d])."""
     qb = _as_bits(q)
     kb = _as_bits(k_cache)
@@ -180,6 +195,10 @@ def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows,
     b, H, d = qb.shape
     H //= nq
     num_pages, G, P, dk = kb.shape
+    if num_kv_heads is None:
+        num_kv_heads = G
+        if group_map is None or group_map.shape != (H,):
+            raise ValueError("group_of_head must have one entry per query head")
     if dk != d or G != num_kv_heads:
         raise ValueError("cache shape %s does not match q %s / G=%d" % (kb.shape, qb.shape, num_kv_heads))
     sl = _as_i32(seqlens)
@@ -205,6 +224,15 @@ def _decode(q, k_cache, v_cache, seqlens, page_table, num_kv_heads, scale, rows,
             float(scale), None if rows_arr is None else rows_arr.ctypes.data, nrows, out.ctypes.data]
     lse = None
     lib = lib or _load()
+    if group_map is not None:
+        lse = np.zeros(nrows, dtype=np.float64)
+        rc = lib.oracle_gqa_decode_mapped(*args, lse.ctypes.data, status.ctypes.data, int(threads),
+                                          group_map.ctypes.data)
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments")
+        if rows is None:
+            out, lse = out.reshape(b, H, d), lse.reshape(b, H)
+        return out, lse, int(status[0])
     if nq > 1:
         lse = np.zeros(nrows, dtype=np.float64)
         args.insert(6, nq)

@@ -23,6 +23,11 @@
  * not the drafts after it (the mask of a causal decoder, aligned to the end
  * of the cache).  nq = 1 is the decode above.
  *
+ * oracle_gqa_decode_mapped takes the KV group of every query head from a table,
+ * g(i) = group_of_head[i] (any values in [0, G), groups of unequal size or
+ * with no head allowed), instead of g(i) = i / (H/G); H need not be a multiple
+ * of G.  The table i -> i / (H/G) is the decode above.
+ *
  * Sources, by page and section:
  *  - "Grouped-Query Attention" (aiwiki), the PyTorch module: keys and values are
  *    broadcast to the query heads of their group by repeat_interleave(h // g,
@@ -120,14 +125,18 @@ static int decode_rows(const uint16_t *q, const uint16_t *k_cache,
                        int32_t d, int32_t page_size, int32_t num_pages,
                        int32_t max_pages_per_seq, double scale,
                        const int64_t *rows, int64_t nrows, double *out, double *lse,
-                       int32_t *status, int32_t nthreads)
+                       int32_t *status, int32_t nthreads, const int32_t *group_of_head)
 {
     if (!q || !k_cache || !v_cache || !seqlens || !out || !status)
         return -1;
     if (b < 1 || nq < 1 || H < 1 || G < 1 || d < 1 || page_size < 1 || num_pages < 1)
         return -1;
-    if (H % G != 0)
+    if (group_of_head == NULL && H % G != 0)
         return -1;
+    if (group_of_head != NULL)
+        for (int32_t i = 0; i < H; ++i)
+            if (group_of_head[i] < 0 || group_of_head[i] >= G)
+                return -1;
     if (page_table != NULL && max_pages_per_seq < 1)
         return -1;
     if (rows == NULL)
@@ -155,7 +164,7 @@ static int decode_rows(const uint16_t *q, const uint16_t *k_cache,
         const int32_t s = (int32_t)(row / ((int64_t)nq * H));   /* row = (s * nq + tq) * H + i */
         const int32_t tq = (int32_t)((row / H) % nq);
         const int32_t i = (int32_t)(row % H);
-        const int32_t g = i / r;
+        const int32_t g = group_of_head ? group_of_head[i] : i / r;
         const int32_t len_s = seqlens[s];
         if (len_s < nq || len_s > capacity) {
             status_all |= ORACLE_STATUS_BAD_SEQLEN;
@@ -247,7 +256,7 @@ int oracle_gqa_decode(const uint16_t *q, const uint16_t *k_cache,
 {
     return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, 1, H, G, d,
                        page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
-                       out, NULL, status, nthreads);
+                       out, NULL, status, nthreads, NULL);
 }
 
 /* The same, plus lse [nrows] = ln sum_j exp(l_j) of each row (-inf for a row
@@ -264,7 +273,7 @@ int oracle_gqa_decode_lse(const uint16_t *q, const uint16_t *k_cache,
         return -1;
     return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, 1, H, G, d,
                        page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
-                       out, lse, status, nthreads);
+                       out, lse, status, nthreads, NULL);
 }
 
 /* nq query tokens per sequence: q, out [b, nq, H, d] (rows (s * nq + t) * H + i),
@@ -279,7 +288,23 @@ int oracle_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache,
 {
     return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, nq, H, G, d,
                        page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
-                       out, lse, status, nthreads);
+                       out, lse, status, nthreads, NULL);
+}
+
+/* Any group map: group_of_head[H] with values in [0, G); lse [nrows] or NULL. */
+int oracle_gqa_decode_mapped(const uint16_t *q, const uint16_t *k_cache,
+                             const uint16_t *v_cache, const int32_t *seqlens,
+                             const int32_t *page_table, int32_t b, int32_t H, int32_t G,
+                             int32_t d, int32_t page_size, int32_t num_pages,
+                             int32_t max_pages_per_seq, double scale,
+                             const int64_t *rows, int64_t nrows, double *out, double *lse,
+                             int32_t *status, int32_t nthreads, const int32_t *group_of_head)
+{
+    if (!group_of_head)
+        return -1;
+    return decode_rows(q, k_cache, v_cache, seqlens, page_table, b, 1, H, G, d,
+                       page_size, num_pages, max_pages_per_seq, scale, rows, nrows,
+                       out, lse, status, nthreads, group_of_head);
 }
 
 /* Number of OpenMP threads a parallel region would use by default. */

@@ -30,6 +30,12 @@ against a one-token decode with the length it sees; torch's
 scaled_dot_product_attention in float64 with the end-aligned causal mask
 written out as a boolean matrix; math.fsum brute force; lengths below nq.
 
+``MAPPED_PINS`` take ``oracle.gqa_decode_mapped`` (any table g(i)): torch's
+scaled_dot_product_attention in float64 on keys/values gathered with
+index_select by the table, permuting the query heads together with the
+table, and math.fsum brute force, on maps with groups of unequal size, empty
+groups and H not a multiple of G.
+
 ``LSE_PINS`` take ``oracle.gqa_decode_lse`` instead and pin the log of each
 row's softmax normaliser, ln sum_j exp(scale q.k_j): one token gives its own
 logit; q = 0 gives ln len; torch.logsumexp in float64 on the broadcast keys;
@@ -515,3 +521,69 @@ def oracle_decode_lse(q, k, v, lens, G):
 
 VERIFY_PINS = [pin_verify_each_draft_is_a_decode, pin_verify_sdpa_causal_mask, pin_verify_brute_force,
                pin_verify_length_below_drafts]
+
+
+# ----------------------------------------------------------------------------
+# any group map (decode_mapped: oracle.gqa_decode_mapped)
+
+
+def pin_mapped_sdpa_gather(decode_mapped):
+    """Groups of sizes 4, 0, 3 in shuffled order, H = 7 with G = 3."""
+    gmap = [2, 0, 0, 2, 0, 2, 0]
+    w = Workload(name="map", b=2, H=7, G=3, d=16, m=30, seed=83)
+    inp = make_inputs(w, lens=[30, 11])
+    out, _, st = decode_mapped(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, group_of_head=gmap, scale=0.4)
+    assert st == 0
+    idx = torch.tensor(gmap)
+    q = bf16_f64(inp.q).unsqueeze(2)
+    k = bf16_f64(inp.k_cache).index_select(1, idx)
+    v = bf16_f64(inp.v_cache).index_select(1, idx)
+    pos = torch.arange(k.shape[2])
+    mask = (pos[None, :] < inp.seqlens[:, None].to(torch.int64))[:, None, None, :]
+    ref = F.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=0.4).squeeze(2).numpy()
+    assert_close(out, ref, rtol=1e-12, atol=1e-14, what="mapped sdpa")
+
+
+def pin_mapped_head_permutation(decode_mapped):
+    """Permuting the query heads together with their map entries permutes the
+    output rows and nothing else."""
+    gmap = [1, 1, 0, 3, 3, 3, 0, 1]
+    w = Workload(name="map", b=2, H=8, G=4, d=8, m=25, seed=89)
+    inp = make_inputs(w, lens=[25, 6])
+    out, lse, _ = decode_mapped(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, group_of_head=gmap)
+    perm = [5, 2, 7, 0, 1, 6, 4, 3]
+    q2 = inp.q[:, perm].contiguous()
+    out2, lse2, _ = decode_mapped(q2, inp.k_cache, inp.v_cache, inp.seqlens, group_of_head=[gmap[i] for i in perm])
+    assert np.array_equal(out2, out[:, perm]) and np.array_equal(lse2, lse[:, perm])
+
+
+def pin_mapped_brute_force(decode_mapped):
+    gmap = [1, 0, 1]
+    w = Workload(name="map", b=2, H=3, G=2, d=3, m=4, seed=97)
+    inp = make_inputs(w, lens=[4, 2])
+    out, _, _ = decode_mapped(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, group_of_head=gmap, scale=1.1)
+    q, k, v = bf16_f64(inp.q).tolist(), bf16_f64(inp.k_cache).tolist(), bf16_f64(inp.v_cache).tolist()
+    for s in range(w.b):
+        L = int(inp.seqlens[s])
+        for i in range(w.H):
+            g = gmap[i]
+            z = [1.1 * math.fsum(q[s][i][c] * k[s][g][j][c] for c in range(w.d)) for j in range(L)]
+            e = [math.exp(x) for x in z]
+            tot = math.fsum(e)
+            ref = [math.fsum(e[j] / tot * v[s][g][j][c] for j in range(L)) for c in range(w.d)]
+            assert_close(out[s, i], ref, rtol=1e-13, atol=1e-15, what="brute force mapped")
+
+
+def pin_mapped_rejects_bad_entries(decode_mapped):
+    w = Workload(name="map", b=1, H=4, G=2, d=8, m=5, seed=101)
+    inp = make_inputs(w, lens=[5])
+    for bad in ([0, 1, 2, 0], [0, -1, 1, 1]):
+        try:
+            decode_mapped(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, group_of_head=bad)
+        except ValueError:
+            continue
+        raise AssertionError("a map entry outside [0, G) must be rejected")
+
+
+MAPPED_PINS = [pin_mapped_sdpa_gather, pin_mapped_head_permutation, pin_mapped_brute_force,
+               pin_mapped_rejects_bad_entries]

@@ -10,10 +10,11 @@ import os
 import pytest
 
 import oracle
-from tests.oracle_pins import LSE_PINS, PINS, VERIFY_PINS
+from tests.oracle_pins import LSE_PINS, MAPPED_PINS, PINS, VERIFY_PINS
 
 MUTANTS = {
-    "group map i % G": ("const int32_t g = i / r;", "const int32_t g = i % G;"),
+    "group map i % G": ("const int32_t g = group_of_head ? group_of_head[i] : i / r;",
+                        "const int32_t g = group_of_head ? group_of_head[i] : i % G;"),
     "scale dropped": ("logits[t] = scale * dot;", "logits[t] = dot;"),
     "page row index transposed": ("row_in_page = t % page_size;", "row_in_page = t / page_size;"),
     "page table stride": ("page_table[(long long)s * max_pages_per_seq + t / page_size]",
@@ -32,6 +33,10 @@ MUTANTS = {
     "capacity check off by one": ("if (len_s < nq || len_s > capacity)", "if (len_s < nq || len_s > capacity + 1)"),
     "draft mask reversed": ("const int32_t len = len_s - (nq - 1 - tq);", "const int32_t len = len_s - tq;"),
     "draft mask off by one": ("const int32_t len = len_s - (nq - 1 - tq);", "const int32_t len = len_s - (nq - tq);"),
+    "map read at the next head": ("const int32_t g = group_of_head ? group_of_head[i] : i / r;",
+                                  "const int32_t g = group_of_head ? group_of_head[(i + 1) % H] : i / r;"),
+    "map of head 0 for every head": ("const int32_t g = group_of_head ? group_of_head[i] : i / r;",
+                                     "const int32_t g = group_of_head ? group_of_head[0] : i / r;"),
     "draft index of the row": ("const int32_t tq = (int32_t)((row / H) % nq);", "const int32_t tq = (int32_t)(row % nq);"),
     "page bound off by one": ("if (page < 0 || page >= num_pages)", "if (page < 0 || page > num_pages)"),
     "lse without the maximum": ("lse[n] = mx + log(denom);", "lse[n] = log(denom);"),
@@ -58,8 +63,10 @@ def test_pins_catch_mutant(name, tmp_path):
     decode = functools.partial(oracle.gqa_decode, lib=lib)
     decode_lse = functools.partial(oracle.gqa_decode_lse, lib=lib)
     decode_verify = functools.partial(oracle.gqa_decode_verify, lib=lib)
+    decode_mapped = functools.partial(oracle.gqa_decode_mapped, lib=lib)
     caught = []
-    for pins, fn in ((PINS, decode), (LSE_PINS, decode_lse), (VERIFY_PINS, decode_verify)):
+    for pins, fn in ((PINS, decode), (LSE_PINS, decode_lse), (VERIFY_PINS, decode_verify),
+                     (MAPPED_PINS, decode_mapped)):
         for pin in pins:
             try:
                 pin(fn)

@@ -2,7 +2,7 @@
 import pytest
 
 import oracle
-from tests.oracle_pins import LSE_PINS, PINS, VERIFY_PINS
+from tests.oracle_pins import LSE_PINS, MAPPED_PINS, PINS, VERIFY_PINS
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -18,3 +18,8 @@ def test_oracle_lse_pin(pin):
 @pytest.mark.parametrize("pin", VERIFY_PINS, ids=[p.__name__ for p in VERIFY_PINS])
 def test_oracle_verify_pin(pin):
     pin(oracle.gqa_decode_verify)
+
+
+@pytest.mark.parametrize("pin", MAPPED_PINS, ids=[p.__name__ for p in MAPPED_PINS])
+def test_oracle_mapped_pin(pin):
+    pin(oracle.gqa_decode_mapped)
