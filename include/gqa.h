@@ -264,6 +264,33 @@ int gqa_decode_verify(const void *q, const void *k_cache, const void *v_cache,
                       size_t workspace_bytes, void *stream);
 
 /*
+ * gqa_decode_split_mapped -- gqa_decode_split with the KV group of every query
+ * head taken from a table, g(i) = group_of_head[i], instead of i / (H/G):
+ * groups may have unequal sizes or no head at all, and num_heads need not be
+ * a multiple of num_kv_heads (the non-uniform grouping of "Beyond Uniform
+ * Query Distribution: Key-Driven Grouped Query Attention", Figure 1, with the
+ * map given at inference).  Each group's K/V is still read once and shared by
+ * its heads on chip.
+ *
+ * group_of_head: HOST memory, num_heads int32 entries in [0, num_kv_heads)
+ * (else GQA_ERR_HEADS); num_heads <= 256, num_kv_heads <= 256.  The map is
+ * read during the call only.  lse: fp32 [b, H] or NULL, as in
+ * gqa_decode_split_lse.  Runs on fixed splits (split_tokens = 0: the library
+ * picks them, for paged caches too); the workspace comes from
+ * gqa_decode_split_mapped_workspace_size with the same arguments.  The
+ * CUDA-core contraction flag is not available with a map.  A map
+ * g(i) = i / (H/G) gives exactly gqa_decode_split's result.
+ */
+size_t gqa_decode_split_mapped_workspace_size(const gqa_dims *dims, const int32_t *group_of_head,
+                                              int32_t max_seqlen, int32_t split_tokens);
+
+int gqa_decode_split_mapped(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens, const int32_t *page_table, float *out, float *lse,
+                            const gqa_dims *dims, const int32_t *group_of_head, float scale,
+                            uint32_t *status, int32_t split_tokens, int32_t max_seqlen, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
  * gqa_merge_lse -- merges n_parts normalised partial results of the same rows,
  * each weighted by its log-sum-exp:
  *     LSE = ln sum_k exp(lse_k),   out = sum_k exp(lse_k - LSE) o_k.

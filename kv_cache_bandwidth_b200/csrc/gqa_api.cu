@@ -96,6 +96,7 @@ int encode_pool(CUtensorMap *map, const void *base, int D, int rows_per_page, in
 // ------------------------------------------------------------------ validation
 struct Shape {
   int b, H, G, r, D, P, num_pages, max_pages;
+  bool mapped;  // group of each head from a table (r = the largest group)
   bool paged;
   long long capacity;
   int nt, nhb;  // kernel variant: n8 row tiles per consumer warp, row blocks of 8
@@ -109,13 +110,27 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Largest number of query tokens per sequence (speculative verification).
 constexpr int kMaxQueryTokens = 64;
 
-int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1) {
+// group_of_head (host memory, num_heads entries) or null: with a table, H need
+// not be a multiple of G and r becomes the largest group's size.
+int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1, const int32_t *group_of_head = nullptr) {
   if (!dims) return GQA_ERR_NULL_POINTER;
   const gqa_dims &d = *dims;
   if (d.batch < 1 || d.num_heads < 1 || d.num_kv_heads < 1 || d.page_size < 1) return GQA_ERR_DIMS;
   if (d.batch > 65535 || d.num_kv_heads > 16383) return GQA_ERR_DIMS;  // grid y/z limits (G x 4 slices)
-  if (d.num_heads % d.num_kv_heads != 0) return GQA_ERR_HEADS;
-  const int r = d.num_heads / d.num_kv_heads;
+  int r;
+  if (group_of_head) {
+    if (d.num_heads > gqa::kMaxMapHeads || d.num_kv_heads > gqa::kMaxMapGroups || nq != 1) return GQA_ERR_HEADS;
+    int count[gqa::kMaxMapGroups] = {};
+    for (int i = 0; i < d.num_heads; ++i) {
+      if (group_of_head[i] < 0 || group_of_head[i] >= d.num_kv_heads) return GQA_ERR_HEADS;
+      ++count[group_of_head[i]];
+    }
+    r = 1;
+    for (int g = 0; g < d.num_kv_heads; ++g) r = std::max(r, count[g]);
+  } else {
+    if (d.num_heads % d.num_kv_heads != 0) return GQA_ERR_HEADS;
+    r = d.num_heads / d.num_kv_heads;
+  }
   if (r > GQA_MAX_GROUP_RATIO) return GQA_ERR_HEADS;
   if (d.head_dim != 64 && d.head_dim != 128) return GQA_ERR_HEAD_DIM;
   if (d.flags & ~(GQA_FLAG_CONTRACT_MMA | GQA_FLAG_CONTRACT_FMA)) return GQA_ERR_DIMS;
@@ -125,6 +140,7 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1) {
   s.H = d.num_heads;
   s.G = d.num_kv_heads;
   s.r = r;
+  s.mapped = group_of_head != nullptr;
   s.D = d.head_dim;
   s.P = d.page_size;
   s.paged = paged;
@@ -154,7 +170,7 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1) {
   s.nt = 1;
   s.nhb = (s.rc + 7) / 8;
   s.fma = (d.flags & GQA_FLAG_CONTRACT_FMA) != 0;
-  if (s.fma && (r > 2 || nq > 1)) return GQA_ERR_HEADS;  // the CUDA-core contraction covers r <= 2, one token
+  if (s.fma && (r > 2 || nq > 1 || s.mapped)) return GQA_ERR_HEADS;  // CUDA-core path: r <= 2, one token, no map
   *sh = s;
   return GQA_OK;
 }
@@ -365,7 +381,21 @@ struct RowExtras {
   bool empty_ok = false;
   int nq = 1;  // query tokens per sequence
   bool force_pdl = false;  // dependent launch even for one item per unit (behind a short kernel)
+  const int32_t *group_of_head = nullptr;  // host table of each head's KV group, or null
 };
+
+// The device form of a group table: heads sorted by group (stable), offsets.
+void fill_group_map(const int32_t *group_of_head, int H, int G, gqa::GroupMap *m) {
+  int count[gqa::kMaxMapGroups + 1] = {};
+  for (int i = 0; i < H; ++i) ++count[group_of_head[i] + 1];
+  m->off[0] = 0;
+  for (int g = 0; g < G; ++g) m->off[g + 1] = static_cast<uint16_t>(m->off[g] + count[g + 1]);
+  int fill[gqa::kMaxMapGroups] = {};
+  for (int i = 0; i < H; ++i) {
+    const int g = group_of_head[i];
+    m->heads[m->off[g] + fill[g]++] = static_cast<uint8_t>(i);
+  }
+}
 
 // The items kernel: one block per (sequence, group, split) item.
 int run_items(const Shape &sh, const void *q, const void *k, const void *v, const int32_t *seqlens,
@@ -387,6 +417,10 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   p.epoch = unit_ctr ? next_epoch() : 0;
   p.lse = ex.lse;
   p.empty_ok = ex.empty_ok ? 1 : 0;
+  if (ex.group_of_head) {
+    p.mapped = 1;
+    fill_group_map(ex.group_of_head, sh.H, sh.G, &p.map);
+  }
   const long long items = units_of(sh) * num_splits;
   if (items > (1ll << 31) - 1) return GQA_ERR_DIMS;
   // Programmatic dependent launch pays off when the grid follows a short or
@@ -535,8 +569,8 @@ AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
 
 // split_tokens == 0 in the split API: checks shared by its entry points.
 int prepare_auto(const gqa_dims *dims, bool paged, int32_t max_seqlen, const void *workspace,
-                 size_t workspace_bytes, Shape *sh, int nq = 1) {
-  int rc = check_dims(dims, paged, sh, nq);
+                 size_t workspace_bytes, Shape *sh, int nq = 1, const int32_t *group_of_head = nullptr) {
+  int rc = check_dims(dims, paged, sh, nq, group_of_head);
   if (rc != GQA_OK) return rc;
   if (max_seqlen < 1) return GQA_ERR_DIMS;
   if (!workspace) return GQA_ERR_WORKSPACE;
@@ -552,8 +586,9 @@ struct SplitArgs {
 };
 
 int prepare_split(const gqa_dims *dims, bool paged, int32_t split_tokens, int32_t max_seqlen,
-                  const void *workspace, size_t workspace_bytes, int sms, SplitArgs *out, int nq = 1) {
-  int rc = check_dims(dims, paged, &out->sh, nq);
+                  const void *workspace, size_t workspace_bytes, int sms, SplitArgs *out, int nq = 1,
+                  const int32_t *group_of_head = nullptr) {
+  int rc = check_dims(dims, paged, &out->sh, nq, group_of_head);
   if (rc != GQA_OK) return rc;
   if (max_seqlen < 1) return GQA_ERR_DIMS;
   if (split_tokens <= 0 || split_tokens % kSplitQuantum != 0) return GQA_ERR_SPLIT;
@@ -635,12 +670,13 @@ int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, c
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (split_tokens == 0) {
     Shape sh;
-    if ((rc = prepare_auto(dims, page_table != nullptr, max_seqlen, workspace, workspace_bytes, &sh, ex.nq)) !=
-        GQA_OK)
+    if ((rc = prepare_auto(dims, page_table != nullptr, max_seqlen, workspace, workspace_bytes, &sh, ex.nq,
+                           ex.group_of_head)) != GQA_OK)
       return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(dev.sms, 256));
+    // (a group map runs on fixed splits only: the library picks them as for a contiguous cache)
+    const AutoChoice ch = choose_auto(sh, dims_paged(dims) && !sh.mapped, max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) {
       rc = run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale, status,
                                max_seqlen, workspace, st, ex);
@@ -651,7 +687,7 @@ int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, c
   }
   SplitArgs a;
   rc = prepare_split(dims, page_table != nullptr, split_tokens, max_seqlen, workspace,
-                     workspace_bytes, 0, &a, ex.nq);
+                     workspace_bytes, 0, &a, ex.nq, ex.group_of_head);
   if (rc != GQA_OK) return rc;
   DeviceInfo dev;
   if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
@@ -846,6 +882,28 @@ int gqa_append_decode_split(const void *k_new, const void *v_new, const void *q,
   if (rc != GQA_OK) return rc;
   RowExtras ex;
   ex.force_pdl = true;  // the decode's blocks are dispatched while the append runs
+  return decode_split_impl(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status, split_tokens,
+                           max_seqlen, workspace, workspace_bytes, stream, ex);
+}
+
+size_t gqa_decode_split_mapped_workspace_size(const gqa_dims *dims, const int32_t *group_of_head,
+                                              int32_t max_seqlen, int32_t split_tokens) {
+  Shape sh;
+  if (!dims || !group_of_head || check_dims(dims, false, &sh, 1, group_of_head) != GQA_OK) return 0;
+  if (max_seqlen < 1 || split_tokens < 0 || split_tokens % kSplitQuantum != 0) return 0;
+  if (split_tokens == 0) return auto_workspace_bytes(sh, max_seqlen);
+  return workspace_layout(sh, (max_seqlen + split_tokens - 1) / split_tokens).total;
+}
+
+int gqa_decode_split_mapped(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                            const int32_t *page_table, float *out, float *lse, const gqa_dims *dims,
+                            const int32_t *group_of_head, float scale, uint32_t *status, int32_t split_tokens,
+                            int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!group_of_head) return GQA_ERR_NULL_POINTER;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GQA_ERR_MISALIGNED;
+  RowExtras ex;
+  ex.lse = lse;
+  ex.group_of_head = group_of_head;
   return decode_split_impl(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status, split_tokens,
                            max_seqlen, workspace, workspace_bytes, stream, ex);
 }

@@ -64,6 +64,16 @@ constexpr float kLFinal = -3.f;      // split 0: the only split already wrote th
 // shares with its neighbours.
 enum class Mode { kItems, kCluster, kBalanced };
 
+// Any query-head to KV-group table (items mode): the heads sorted by group
+// (stable) and each group's first position in that order, so that group g
+// serves heads map_heads[map_off[g] .. map_off[g + 1]).
+constexpr int kMaxMapHeads = 256;
+constexpr int kMaxMapGroups = 256;
+struct GroupMap {
+  uint8_t heads[kMaxMapHeads];
+  uint16_t off[kMaxMapGroups + 1];
+};
+
 struct DecodeParams {
   const __nv_bfloat16 *q;     // [b, H, D]
   const int32_t *seqlens;     // [b]
@@ -90,6 +100,8 @@ struct DecodeParams {
   int num_splits;             // items mode: S
   int b;                      // sequences
   float scale_log2;           // scale * log2(e)
+  int mapped;                 // the group of each head comes from `map` (items mode, one query token)
+  GroupMap map;
 };
 
 struct CombineParams {
@@ -113,6 +125,18 @@ struct CombineParams {
 __device__ __forceinline__ size_t out_row(int s, int g, int rho, int nq, int r, int H) {
   const int t = rho / r, h = rho - t * r;
   return (static_cast<size_t>(s) * nq + t) * H + static_cast<size_t>(g) * r + h;
+}
+
+// Row of q / out of row rho of KV group g of sequence s, with or without a
+// group map.
+__device__ __forceinline__ size_t row_of(const DecodeParams &p, int s, int g, int rho) {
+  if (p.mapped) return static_cast<size_t>(s) * p.H + p.map.heads[p.map.off[g] + rho];
+  return out_row(s, g, rho, p.nq, p.r, p.H);
+}
+
+// Rows of KV group g: nq * r, or the group's own size under a map.
+__device__ __forceinline__ int group_rows(const DecodeParams &p, int g) {
+  return p.mapped ? static_cast<int>(p.map.off[g + 1]) - static_cast<int>(p.map.off[g]) : p.rq;
 }
 
 // Natural-log sum of exp over a row from its base-2 state: the row's
@@ -202,7 +226,7 @@ __device__ __forceinline__ Piece make_item(const DecodeParams &p) {
     it.s = blockIdx.z;
   }
   it.h0 = it.j * p.rc;
-  it.nh = min(p.rc, p.rq - it.h0);
+  it.nh = min(p.rc, group_rows(p, it.g) - it.h0);  // <= 0: a slice past a small group (mapped)
   it.len = __ldg(p.seqlens + it.s);
   it.len_ok = it.len >= p.nq && it.len <= p.capacity;
   it.t_begin = 0;
@@ -787,6 +811,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
   if (!BAL) pc = make_item<T, MODE>(p);
   if (MODE == Mode::kItems) {
     if (threadIdx.x == 0) pdl_launch_dependents();
+    if (pc.nh <= 0) return;  // a slice past the rows of a small group (group map): no rows, nothing to do
     if (pc.t_begin >= pc.t_end) {
       // Nothing to read.  An invalid length is handled once, by split 0: zero
       // rows in `out` and a marker in split 0 for the combine.
@@ -796,7 +821,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         const bool empty = p.empty_ok && pc.len == 0;
         for (int idx = threadIdx.x; idx < pc.nh * (D / 4); idx += blockDim.x) {
           const int h = idx / (D / 4), c4 = idx % (D / 4);
-          const size_t row = out_row(pc.s, pc.g, pc.h0 + h, p.nq, p.r, p.H);
+          const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
           if (p.out) reinterpret_cast<float4 *>(p.out + row * D)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLBadLength;
           if (c4 == 0 && p.lse) p.lse[row] = kNegInf;
@@ -868,8 +893,8 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         // (one run when there is one query token per sequence)
         for (int rho = 0; rho < pc.nh;) {
           const int a = pc.h0 + rho;
-          const int run = min(pc.nh - rho, p.r - a % p.r);
-          bulk_load(q_sm + qs * TL::kQBytes + rho * D * 2, p.q + out_row(pc.s, pc.g, a, p.nq, p.r, p.H) * D,
+          const int run = p.mapped ? 1 : min(pc.nh - rho, p.r - a % p.r);  // mapped: one row per copy
+          bulk_load(q_sm + qs * TL::kQBytes + rho * D * 2, p.q + row_of(p, pc.s, pc.g, a) * D,
                     static_cast<uint32_t>(run * D * 2), bar_qfull + 8 * qs);
           rho += run;
         }
@@ -1237,7 +1262,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
             BAL ? pc.final_row : (((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr);
         for (int idx = ctid; idx < pc.nh * n4; idx += nc * 32) {
           const int h = idx / n4, c4 = idx % n4;
-          const size_t row = out_row(pc.s, pc.g, pc.h0 + h, p.nq, p.r, p.H);
+          const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
           const float4 src = *reinterpret_cast<const float4 *>(osum + h * TL::kOStride + 4 * c4);
           if (final_row) {
             const float L = L_blk[h];
@@ -1280,7 +1305,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
             static_assert(TL::kRPad * kHalf <= nc * 32, "one pass of the consumer threads");
             const int h = ctid / kHalf, c4 = ctid % kHalf;
             if (h < pc.nh) {
-              const size_t row = out_row(pc.s, pc.g, pc.h0 + h, p.nq, p.r, p.H);
+              const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
               merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(row) * p.num_splits, ns,
                                  c4, kHalf, reinterpret_cast<float4 *>(p.out + row * D),
                                  p.lse ? p.lse + row : nullptr);
@@ -1324,7 +1349,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         }
         float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
         if (L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
-        const size_t row = out_row(pc.s, pc.g, pc.h0 + h, p.nq, p.r, p.H);
+        const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
         reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
       }
       if (threadIdx.x == 0 && !pc.len_ok && p.status) atomicOr(p.status, kStatusBadSeqlen);

@@ -27,6 +27,7 @@ __all__ = [
     "FLAG_CONTRACT_FMA", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
     "gqa_decode_split_lse", "gqa_merge_lse", "SERIAL_MERGE_MAX_SPLITS", "gqa_kv_append", "PagePool",
     "gqa_decode_verify", "gqa_decode_verify_workspace_size", "gqa_append_decode_split",
+    "gqa_decode_split_mapped", "gqa_decode_split_mapped_workspace_size",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -106,6 +107,13 @@ def load():
     lib.gqa_decode_verify_workspace_size.restype = ctypes.c_size_t
     lib.gqa_decode_verify_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32,
                                                      ctypes.c_int32]
+    lib.gqa_decode_split_mapped.restype = ctypes.c_int
+    lib.gqa_decode_split_mapped.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims), _vp,
+                                            ctypes.c_float, _vp, ctypes.c_int32, ctypes.c_int32, _vp,
+                                            ctypes.c_size_t, _vp]
+    lib.gqa_decode_split_mapped_workspace_size.restype = ctypes.c_size_t
+    lib.gqa_decode_split_mapped_workspace_size.argtypes = [ctypes.POINTER(Dims), _vp, ctypes.c_int32,
+                                                           ctypes.c_int32]
     lib.gqa_append_decode_split.restype = ctypes.c_int
     lib.gqa_append_decode_split.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Dims),
                                             ctypes.c_float, _vp, ctypes.c_int32, ctypes.c_int32, _vp,
@@ -311,6 +319,43 @@ def gqa_kv_append(k_new, v_new, k_cache, v_cache, seqlens, page_table=None, *, n
     rc = load().gqa_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
                               _ptr(page_table), ctypes.byref(dims), _ptr(status), _stream(stream))
     _check(rc, "gqa_kv_append")
+
+
+def _host_map(group_of_head):
+    arr = (ctypes.c_int32 * len(group_of_head))(*[int(x) for x in group_of_head])
+    return arr
+
+
+def gqa_decode_split_mapped_workspace_size(dims: Dims, group_of_head, max_seqlen: int, split_tokens: int) -> int:
+    return int(load().gqa_decode_split_mapped_workspace_size(ctypes.byref(dims), _host_map(group_of_head),
+                                                             int(max_seqlen), int(split_tokens)))
+
+
+def gqa_decode_split_mapped(q, k_cache, v_cache, seqlens, page_table=None, *, group_of_head, split_tokens: int = 0,
+                            max_seqlen: Optional[int] = None, workspace=None, out=None, lse=None,
+                            want_lse: bool = False, scale=None, status=None, stream=None, flags: int = 0):
+    """Split decode with query head i using KV group group_of_head[i] (a host
+    list of H ints).  Returns out (and lse when want_lse or lse is given)."""
+    out = _out_for(q, out)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    if max_seqlen is None:
+        max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
+    dims = dims_for(q, k_cache, page_table, flags)
+    gmap = _host_map(group_of_head)
+    if len(group_of_head) != dims.num_heads:
+        raise ValueError("group_of_head needs one entry per query head")
+    if workspace is None:
+        # (a size of 0 means invalid arguments: the call below names the error)
+        n = int(load().gqa_decode_split_mapped_workspace_size(ctypes.byref(dims), gmap, int(max_seqlen),
+                                                              int(split_tokens)))
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    rc = load().gqa_decode_split_mapped(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
+                                        _ptr(out), _ptr(lse), ctypes.byref(dims), gmap, _scale(q, scale),
+                                        _ptr(status), int(split_tokens), int(max_seqlen), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "gqa_decode_split_mapped")
+    return (out, lse) if lse is not None else out
 
 
 def gqa_append_decode_split(k_new, v_new, q, k_cache, v_cache, seqlens, page_table=None, *,
