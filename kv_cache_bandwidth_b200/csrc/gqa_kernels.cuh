@@ -6,18 +6,20 @@
 // "Grouped-Query Attention" (aiwiki) done inside the kernel instead of with
 // repeat_interleave, as that page's closing note asks.
 //
-// One thread block owns one (sequence, KV group, token range) item.  Its keys
-// and values cross HBM once and are shared on chip by the group's r = H/G
-// query heads:
+// One thread block owns one (sequence, KV group, row slice, token range)
+// item.  The rows of a group are its r = H/G query heads (times the query
+// tokens of a verification step, or the heads a group table assigns), cut
+// into slices of at most 16.  The group's keys and values cross HBM once per
+// slice and are shared on chip by the slice's rows:
 //
-//   * a producer warp bulk-copies the group's q block into shared memory and
+//   * a producer warp bulk-copies the slice's q rows into shared memory and
 //     streams K and V tiles of T tokens into a STAGES-deep shared-memory ring
 //     with TMA (128-byte swizzle), translating logical pages through the page
 //     table (a window of 32 page ids per warp, the next window prefetched);
-//   * consumer warps (4 along the token axis x head blocks of 8 or 16 heads)
-//     run the two small contractions on tensor cores with the roles of the
+//   * consumer warps (4 along the token axis x 1 or 2 row blocks of 8) run
+//     the two small contractions on tensor cores with the roles of the
 //     operands swapped so that the tile's tokens fill the M = 16 rows of
-//     mma.m16n8k16 and the group's heads the N = 8 columns:
+//     mma.m16n8k16 and the slice's rows the N = 8 columns:
 //         S^T[tokens, heads] = K_tile q^T            (A = K from smem, B = q in registers)
 //         O^T[d, heads]     += V_tile^T P^T           (A = V^T via ldmatrix.trans)
 //     P^T goes from the accumulator layout of S^T to the B-operand layout with
@@ -29,9 +31,10 @@
 //     shuffles and the accumulators rescaled by 2^(m_old - m_new) only when a
 //     score passes the base by more than 8;
 //   * at the end the consumer warps merge their states in shared memory and
-//     either write a split's partial state (split-KV mode) or merge the blocks
-//     of a thread-block cluster through distributed shared memory and write the
-//     normalised output (cluster mode).
+//     write the normalised rows (a whole unit), or a split's partial state --
+//     which the block completing the unit merges in place for up to 8 splits,
+//     and a combine kernel otherwise -- or merge the blocks of a thread-block
+//     cluster through distributed shared memory (cluster mode).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -151,7 +154,7 @@ template <int D, int NT, int NHB, int CH, int STAGES, bool BAL = false>
 struct Tile {
   static constexpr int kNWT = 4;                   // consumer warps along the token axis
   static constexpr int kHB = 8 * NT;               // query heads per consumer warp
-  static constexpr int kNC = kNWT * NHB;           // consumer warps (NHB head blocks)
+  static constexpr int kNC = kNWT * NHB;           // consumer warps (NHB row blocks)
   static constexpr int kThreads = 32 * (kNC + 1);  // + one producer warp
   static constexpr int kT = kNWT * 16 * CH;        // tokens per pipeline stage
   static constexpr int kHalves = D / 64;           // 128-byte swizzle atoms per row
@@ -159,7 +162,7 @@ struct Tile {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = STAGES * kStageBytes;
   static constexpr int kSteps = D / 16;            // k-steps of q.k, m-tiles of p.v
-  static constexpr int kRPad = NHB * kHB;          // heads per block, padded
+  static constexpr int kRPad = NHB * kHB;          // rows per block, padded
   static constexpr int kOStride = D + 4;           // padded merge row (floats)
   static constexpr int kQBytes = kRPad * D * 2;    // one q block
   static constexpr int kQSlots = BAL ? 2 : 1;      // double-buffered when pieces follow each other
@@ -975,7 +978,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
     }
   } else {
     // =================================================================== consumers
-    const int hb = warp / TL::kNWT;  // head block
+    const int hb = warp / TL::kNWT;  // row block
     const int ws = warp % TL::kNWT;  // token slice within a tile
     const int g8 = lane >> 2;
     const int t4 = lane & 3;
@@ -1175,7 +1178,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         if (lane == 0) mbar_arrive(bar_empty + 8 * stage);
       }
 
-      // ---- merge the consumer warps of each head block
+      // ---- merge the consumer warps of each row block
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
 #pragma unroll

@@ -8,7 +8,7 @@ No step of the computation runs in Python, and there is no fallback: if
 
     out = gqa_decode(q, k_cache, v_cache, seqlens, page_table)          # no workspace
     out = gqa_decode_split(q, k_cache, v_cache, seqlens, page_table,
-                           split_tokens=4096, max_seqlen=131072)          # split-KV + combine
+                           split_tokens=4096, max_seqlen=131072)          # split-KV, merged
 """
 from __future__ import annotations
 
@@ -213,7 +213,8 @@ def workspace_for(q, k_cache, page_table, max_seqlen: int, split_tokens: int) ->
 def gqa_decode_split(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int = 0,
                      max_seqlen: Optional[int] = None, workspace=None, out=None, scale=None,
                      status=None, stream=None, flags: int = 0) -> torch.Tensor:
-    """Split-KV decode (partials kernel + combine kernel).  Returns ``out``.
+    """Split-KV decode (the decode kernel, merging up to 8 splits itself, plus
+    the combine kernel for more splits or equal-work ranges).  Returns ``out``.
 
     max_seqlen defaults to the cache capacity (contiguous m, or
     max_pages_per_seq * page_size)."""
