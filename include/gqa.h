@@ -93,6 +93,10 @@ extern "C" {
 /* gqa_dims.flags: choice of the q.k / p.v contraction (default: automatic). */
 #define GQA_FLAG_CONTRACT_MMA 1u   /* tensor cores (mma.sync m16n8k16 bf16) */
 #define GQA_FLAG_CONTRACT_FMA 2u   /* fp32 FMA on CUDA cores; r = H/G <= 2 only (else GQA_ERR_HEADS) */
+#define GQA_FLAG_CONTRACT_TCGEN05 4u /* 5th-gen tensor cores (tcgen05, accumulators in tensor memory): one block
+                                        takes all rows of a group (r times the query tokens, <= 128), d = 128
+                                        only; split entry points (fixed splits) only.  flags == 0 picks it by
+                                        itself for more than 32 rows per group at d = 128 */
 
 typedef struct gqa_dims {
     int32_t batch;             /* b: sequences, one query token each */

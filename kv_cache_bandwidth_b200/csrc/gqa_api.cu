@@ -18,6 +18,7 @@
 #include "gqa.h"
 #include "gqa_cache.h"
 #include "gqa_kernels.cuh"
+#include "gqa_verify_tc.cuh"
 
 static_assert(GQA_MERGE_IN_KERNEL_MAX_SPLITS == gqa::kSerialMergeMax,
               "the header's in-kernel merge limit is the kernels' serial-merge limit");
@@ -97,6 +98,7 @@ int encode_pool(CUtensorMap *map, const void *base, int D, int rows_per_page, in
 struct Shape {
   int b, H, G, r, D, P, num_pages, max_pages;
   bool mapped;  // group of each head from a table (r = the largest group)
+  bool tc;      // the tcgen05 kernel: all rows of a group in one block (d = 128, <= 128 rows)
   bool paged;
   long long capacity;
   int nt, nhb;  // kernel variant: n8 row tiles per consumer warp, row blocks of 8
@@ -112,7 +114,13 @@ constexpr int kMaxQueryTokens = 64;
 
 // group_of_head (host memory, num_heads entries) or null: with a table, H need
 // not be a multiple of G and r becomes the largest group's size.
-int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1, const int32_t *group_of_head = nullptr) {
+// Rows per group above which the automatic choice is the tcgen05 kernel
+// (measured: with 64 and 128 rows it beats the 16-row mma.sync slices by 1.3x
+// and 2.4x; with 32 or fewer its one-thread-per-row softmax leaves lanes idle).
+constexpr int kTcAutoRows = 32;
+
+int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1, const int32_t *group_of_head = nullptr,
+               bool auto_tc = true) {
   if (!dims) return GQA_ERR_NULL_POINTER;
   const gqa_dims &d = *dims;
   if (d.batch < 1 || d.num_heads < 1 || d.num_kv_heads < 1 || d.page_size < 1) return GQA_ERR_DIMS;
@@ -133,8 +141,8 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1, const in
   }
   if (r > GQA_MAX_GROUP_RATIO) return GQA_ERR_HEADS;
   if (d.head_dim != 64 && d.head_dim != 128) return GQA_ERR_HEAD_DIM;
-  if (d.flags & ~(GQA_FLAG_CONTRACT_MMA | GQA_FLAG_CONTRACT_FMA)) return GQA_ERR_DIMS;
-  if ((d.flags & GQA_FLAG_CONTRACT_MMA) && (d.flags & GQA_FLAG_CONTRACT_FMA)) return GQA_ERR_DIMS;
+  if (d.flags & ~(GQA_FLAG_CONTRACT_MMA | GQA_FLAG_CONTRACT_FMA | GQA_FLAG_CONTRACT_TCGEN05)) return GQA_ERR_DIMS;
+  if (__builtin_popcount(d.flags) > 1) return GQA_ERR_DIMS;  // one contraction choice at most
   Shape s{};
   s.b = d.batch;
   s.H = d.num_heads;
@@ -170,6 +178,15 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1, const in
   s.nt = 1;
   s.nhb = (s.rc + 7) / 8;
   s.fma = (d.flags & GQA_FLAG_CONTRACT_FMA) != 0;
+  s.tc = (d.flags & GQA_FLAG_CONTRACT_TCGEN05) != 0 ||
+         (auto_tc && d.flags == 0 && s.D == 128 && s.rq > kTcAutoRows && s.rq <= gqa::TcTile::kM);
+  if (s.tc) {
+    // one block takes all rows of a group: up to 128 rows, d = 128
+    if (s.D != 128) return GQA_ERR_HEAD_DIM;
+    if (s.rq > gqa::TcTile::kM) return GQA_ERR_HEADS;
+    s.rc = s.rq;
+    s.hs = 1;
+  }
   if (s.fma && (r > 2 || nq > 1 || s.mapped)) return GQA_ERR_HEADS;  // CUDA-core path: r <= 2, one token, no map
   *sh = s;
   return GQA_OK;
@@ -342,6 +359,36 @@ int launch_decode(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv,
 
 int tile_tokens(const Shape &sh) { return sh.D == 64 ? 128 : 64; }
 
+// The tcgen05 kernel (items mode; d = 128, 64-token tiles like the mma.sync kernel).
+int launch_verify_tc(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p,
+                     const Launch &l) {
+  auto kernel = sh.paged ? gqa::gqa_verify_tc_kernel<true> : gqa::gqa_verify_tc_kernel<false>;
+  constexpr int smem = gqa::TcTile::kSmemBytes;
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(gqa::gqa_verify_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess ||
+        cudaFuncSetAttribute(gqa::gqa_verify_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    attr_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = l.grid;
+  cfg.blockDim = dim3(gqa::TcTile::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = l.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
 int encode_maps(const Shape &sh, const void *k, const void *v, CUtensorMap *tk, CUtensorMap *tv) {
   const int T = tile_tokens(sh);
   const int rows = sh.P;  // paged: page size; contiguous: capacity m
@@ -428,6 +475,7 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   // unit the grid follows a full decode grid, where measured it cost ~3 %
   // (its early blocks only wait, and the grid no longer starts as one wave).
   Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream, num_splits > 1 || ex.force_pdl};
+  if (sh.tc) return launch_verify_tc(sh, tk, tv, p, l);
   return launch_decode<Mode::kItems>(sh, tk, tv, p, l);
 }
 
@@ -537,6 +585,10 @@ struct AutoChoice {
 
 bool dims_paged(const gqa_dims *dims) { return dims->max_pages_per_seq > 0; }
 
+// Equal-work ranges serve paged dims, with neither a group table nor the
+// tcgen05 kernel (both run on fixed splits only).
+bool balanced_ok(const gqa_dims *dims, const Shape &sh) { return dims_paged(dims) && !sh.mapped && !sh.tc; }
+
 int round_split(long long tokens) {
   tokens = (tokens + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
   return static_cast<int>(std::max<long long>(kSplitQuantum, tokens));
@@ -546,6 +598,7 @@ int round_split(long long tokens) {
 // shared memory allows two blocks of the 3-stage ring; the 288- and 544-thread
 // variants for r > 16 fit once by registers).
 int blocks_per_sm(const Shape &sh) {
+  if (sh.tc) return 1;
   if (sh.fma || sh.nhb != 1) return 2;
   switch (pick_pipe(sh)) {
     case Pipe::kTrio: return 3;
@@ -676,7 +729,7 @@ int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, c
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
     // (a group map runs on fixed splits only: the library picks them as for a contiguous cache)
-    const AutoChoice ch = choose_auto(sh, dims_paged(dims) && !sh.mapped, max_seqlen, std::min(dev.sms, 256));
+    const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) {
       rc = run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale, status,
                                max_seqlen, workspace, st, ex);
@@ -731,8 +784,9 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
                const int32_t *page_table, float *out, const gqa_dims *dims, float scale,
                uint32_t *status, void *stream) {
   Shape sh;
-  int rc = check_dims(dims, page_table != nullptr, &sh);
+  int rc = check_dims(dims, page_table != nullptr, &sh, 1, nullptr, /*auto_tc=*/false);
   if (rc != GQA_OK) return rc;
+  if (sh.tc) return GQA_ERR_DIMS;  // the tcgen05 kernel runs behind the split entry points only
   rc = check_inputs(q, k_cache, v_cache, seqlens, status);
   if (rc != GQA_OK) return rc;
   if (!out) return GQA_ERR_NULL_POINTER;
@@ -776,7 +830,7 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
     num_sms = dev.sms;
   }
-  const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(num_sms, 256));
+  const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, std::min(num_sms, 256));
   return ch.balanced ? 0 : ch.split_tokens;
 }
 
@@ -795,7 +849,7 @@ int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,
       return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(dev.sms, 256));
+    const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) {
       if (!out) return GQA_ERR_NULL_POINTER;  // whole units are finished straight into out
       return run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale,
@@ -827,7 +881,7 @@ int gqa_split_combine(const int32_t *seqlens, float *out, const gqa_dims *dims, 
     if ((rc = prepare_auto(dims, false, max_seqlen, workspace, workspace_bytes, &sh)) != GQA_OK) return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    const AutoChoice ch = choose_auto(sh, dims_paged(dims), max_seqlen, std::min(dev.sms, 256));
+    const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) return run_balanced_combine(sh, seqlens, out, status, workspace, st);
     split_tokens = ch.split_tokens;
   }

@@ -1,0 +1,460 @@
+// gqa_verify_tc.cuh -- decode of many rows per KV group on the 5th-generation
+// tensor cores (tcgen05): the rows of a verification step (n query tokens x r
+// heads) or of a large group ratio, up to 128 per block, against d = 128.
+//
+// With more than 16 rows per group the mma.sync kernel has to cut the rows
+// into 16-row slices, each with its own pass over the group's keys and values
+// and its own share of the legacy tensor pipe's throughput.  Here one block
+// takes all rows of its (sequence, group, split) item and the contractions
+// become real matrix products on the tensor cores, with the accumulators in
+// tensor memory:
+//
+//   S[rows, 64 tokens]  = Q[rows, 128] . K_tile[64, 128]^T        (M = 128, N = 64)
+//   O[rows, 128]       += P[rows, 64] . V_tile[64, 128]            (M = 128, N = 128)
+//
+// Rows are padded to M = 128; P enters as a bf16 high part and a bf16
+// residual (two MMAs), as in the mma.sync kernel.  Warp roles:
+//   * warps 0-3: one row per thread (the thread's tensor-memory lane).  Each
+//     tile: read the row's 64 scores from tensor memory, mask (the row's own
+//     causal limit among the drafts), online softmax in base 2 with the lazy
+//     rescale (a row whose maximum moves by more than 2^8 rescales its O row in
+//     tensor memory), write P to shared memory in the 128-byte swizzle;
+//   * warp 4: the TMA producer of the K/V ring (as in the mma.sync kernel);
+//   * warp 5: tensor-memory allocation; one thread issues the MMAs and signals
+//     their completion on mbarriers with tcgen05.commit.
+// S (in tensor memory) and P (in shared memory) are double-buffered: the
+// scores of tile t+1 are computed and its softmax runs while the P.V of tile t
+// is on the tensor cores.  The epilogue writes final rows
+// or partial states in the layout of the mma.sync kernel, so the same merges
+// (in this kernel for up to 8 splits, the combine kernel otherwise) apply.
+#pragma once
+
+#include "gqa_kernels.cuh"
+#include "tc05.cuh"
+
+namespace gqa {
+
+struct TcTile {
+  static constexpr int kD = 128;
+  static constexpr int kT = 64;                        // tokens per tile
+  static constexpr int kM = 128;                       // rows of every MMA (padded)
+  static constexpr int kStages = 3;
+  static constexpr int kHalf = kT * 128;               // one 64-column half of a K or V tile
+  static constexpr int kTileBytes = 2 * kHalf;         // 16 KB
+  static constexpr int kStageBytes = 2 * kTileBytes;   // K + V
+  static constexpr int kQOff = kStages * kStageBytes;  // Q: two halves of kM rows x 128 B
+  static constexpr int kQHalf = kM * 128;
+  static constexpr int kPOff = kQOff + 2 * kQHalf;     // P: 2 buffers x (high part, residual) x kM rows x 64 tokens
+  static constexpr int kPPart = kM * 128;
+  static constexpr int kBarOff = kPOff + 4 * kPPart;
+  // full[3], empty[3], s_full[2], s_free[2], p_full[2], pv_done[2]
+  static constexpr int kNumBars = 2 * kStages + 8;
+  static constexpr int kMiscOff = kBarOff + 8 * kNumBars;  // tmem base, tile_bad[3], abort, merge here
+  static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * 8;
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kTmemCols = 256;           // S (2 x 64 columns) + O (128)
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+// TMA producer for one piece (items mode): K and V tiles of 64 tokens into the
+// 3-stage ring, pages translated through the table as in the mma.sync kernel.
+template <bool PAGED>
+__device__ __forceinline__ void tc_produce(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeParams &p,
+                                           const Piece &pc, uint32_t sbase, uint32_t full0, uint32_t empty0,
+                                           volatile int *tile_bad, volatile int *abort_flag, int lane) {
+  using TT = TcTile;
+  constexpr int T = TT::kT;
+  constexpr int ST = TT::kStages;
+  if (lane == 0) {
+    tma_prefetch_desc(tm_k);
+    tma_prefetch_desc(tm_v);
+  }
+  const uint64_t policy = l2_policy_evict_first();
+  const int P = p.page_size;
+  const int ppt = PAGED ? max(1, T / P) : 1;  // pages per tile
+  const int br = PAGED ? min(P, T) : T;        // rows per TMA box
+  const uint32_t box_bytes = static_cast<uint32_t>(2 * br * 128);
+  const int32_t *pt_row = PAGED ? p.page_table + static_cast<size_t>(pc.s) * p.max_pages : nullptr;
+  const int lp_end = PAGED ? (pc.t_end + P - 1) / P : 0;
+  int cur_w = -1, nxt_w = -1, win = -1, nxt = -1;
+  int tile = 0;
+  for (int t0 = pc.t_begin; t0 < pc.t_end; t0 += T, ++tile) {
+    const int stage = tile % ST;
+    const uint32_t full = full0 + 8 * stage;
+    if (tile >= ST) {
+      bool ok = mbar_wait(empty0 + 8 * stage, ((tile / ST) - 1) & 1);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok || *abort_flag) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          if (p.status) atomicOr(p.status, kStatusTimeout);
+        }
+        break;
+      }
+    }
+    const uint32_t dst_k = sbase + stage * TT::kStageBytes;
+    const uint32_t dst_v = dst_k + TT::kTileBytes;
+    if (PAGED) {
+      const int lp0 = t0 / P;
+      const int wnd = lp0 >> 5;
+      if (wnd != cur_w) {
+        const int idx = wnd * 32 + lane;
+        win = (wnd == nxt_w) ? nxt : (idx < lp_end ? __ldg(pt_row + idx) : -1);
+        cur_w = wnd;
+        nxt_w = wnd + 1;
+        const int nidx = nxt_w * 32 + lane;
+        nxt = nidx < lp_end ? __ldg(pt_row + nidx) : -1;
+      }
+      const int n_here = min(ppt, lp_end - lp0);
+      const int id = __shfl_sync(0xffffffffu, win, (lp0 & 31) + min(lane, ppt - 1));
+      const bool mine = lane < n_here;
+      const bool bad = mine && (id < 0 || id >= p.num_pages);
+      const unsigned bad_mask = __ballot_sync(0xffffffffu, bad);
+      const unsigned good_mask = __ballot_sync(0xffffffffu, mine && !bad);
+      if (lane == 0) {
+        tile_bad[stage] = bad_mask ? 1 : 0;
+        if (bad_mask && p.status) atomicOr(p.status, kStatusBadPage);
+        mbar_arrive_expect_tx(full, 2u * box_bytes * __popc(good_mask));
+      }
+      __syncwarp();
+      if (mine && !bad) {
+        const int row = (P >= T) ? (t0 % P) : 0;
+        const uint32_t off = static_cast<uint32_t>(lane * br * 128);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          tma_load_4d(dst_k + h * TT::kHalf + off, tm_k, full, h * 64, row, pc.g, id, policy);
+          tma_load_4d(dst_v + h * TT::kHalf + off, tm_v, full, h * 64, row, pc.g, id, policy);
+        }
+      }
+    } else if (lane == 0) {
+      mbar_arrive_expect_tx(full, 2u * box_bytes);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tma_load_4d(dst_k + h * TT::kHalf, tm_k, full, h * 64, t0, pc.g, pc.s, policy);
+        tma_load_4d(dst_v + h * TT::kHalf, tm_v, full, h * 64, t0, pc.g, pc.s, policy);
+      }
+    }
+  }
+  // never leave with copies in flight (bounded waits)
+  if (lane == 0) {
+    for (int t = max(0, tile - ST); t < tile; ++t) (void)mbar_wait(full0 + 8 * (t % ST), (t / ST) & 1);
+  }
+}
+
+template <bool PAGED>
+__global__ void __launch_bounds__(TcTile::kThreads, 1)
+    gqa_verify_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                         const DecodeParams p) {
+  using TT = TcTile;
+  constexpr int D = TT::kD;
+  constexpr int T = TT::kT;
+  constexpr int ST = TT::kStages;
+  const float kNegInf = -__int_as_float(0x7f800000);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bars = sbase + TT::kBarOff;
+  const uint32_t full0 = bars, empty0 = bars + 8 * ST;
+  const uint32_t s_full0 = bars + 16 * ST, s_free0 = s_full0 + 16;
+  const uint32_t p_full0 = s_free0 + 16, pv_done0 = p_full0 + 16;
+  volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
+  volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
+  volatile int *abort_flag = tile_bad + ST;
+  volatile int *merge_here = tile_bad + ST + 1;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  pdl_wait_primary();
+  const Piece pc = make_item<T, Mode::kItems>(p);
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  if (pc.nh <= 0) return;
+  if (pc.t_begin >= pc.t_end) {
+    // nothing to read; an invalid length is handled once, by split 0
+    if (!pc.len_ok && pc.k == 0) {
+      const bool empty = p.empty_ok && pc.len == 0;
+      for (int idx = threadIdx.x; idx < pc.nh * (D / 4); idx += blockDim.x) {
+        const int h = idx / (D / 4), c4 = idx % (D / 4);
+        const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
+        if (p.out) reinterpret_cast<float4 *>(p.out + row * D)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLBadLength;
+        if (c4 == 0 && p.lse) p.lse[row] = kNegInf;
+      }
+      if (threadIdx.x == 0 && p.status && !empty) atomicOr(p.status, kStatusBadSeqlen);
+    }
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(full0 + 8 * i, 1);
+      mbar_init(empty0 + 8 * i, 1);  // one tcgen05.commit per use
+      tile_bad[i] = 0;
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full0 + 8 * i, 1);
+      mbar_init(s_free0 + 8 * i, 4);  // one arrival per softmax warp
+      mbar_init(p_full0 + 8 * i, 4);
+      mbar_init(pv_done0 + 8 * i, 1);
+    }
+    *abort_flag = 0;
+    *merge_here = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 5) {
+    tc_alloc(smem_addr(const_cast<uint32_t *>(tmem_slot)), TT::kTmemCols);
+    tc_relinquish();
+  }
+  if (threadIdx.x < 128) {
+    // this thread's q row into Q (128-byte swizzle, two 64-column halves); padding rows are zero
+    const int r = threadIdx.x;
+    const bool valid = r < pc.nh;
+    const uint4 *src = valid ? reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + r) * D) : nullptr;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+      const int h = c >> 3, c8 = c & 7;
+      *reinterpret_cast<uint4 *>(smem + TT::kQOff + h * TT::kQHalf + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
+
+  if (warp == 4) {
+    // ============================================================ producer
+    tc_produce<PAGED>(&tm_k, &tm_v, p, pc, sbase, full0, empty0, tile_bad, abort_flag, lane);
+  } else if (warp == 5) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = tc_idesc_bf16(128, 64, false);
+      constexpr uint32_t kIdescPV = tc_idesc_bf16(128, 128, true);
+      const uint32_t q_sm = sbase + TT::kQOff;
+      bool ok = true;
+      for (int t = 0; t <= n_tiles && ok; ++t) {
+        if (t < n_tiles) {
+          // ---- S[t % 2] = Q K_t^T
+          const int st = t % ST;
+          ok = mbar_wait(full0 + 8 * st, (t / ST) & 1);
+          if (ok && t >= 2) ok = mbar_wait(s_free0 + 8 * (t & 1), ((t >> 1) - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kt = sbase + st * TT::kStageBytes;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t koff = (ks >> 2) * TT::kHalf + (ks & 3) * 32;
+            const uint32_t qoff = (ks >> 2) * TT::kQHalf + (ks & 3) * 32;
+            tc_mma(tmem + (t & 1) * 64, tc_smem_desc(q_sm + qoff, 16, 1024), tc_smem_desc(kt + koff, 16, 1024),
+                   kIdescQK, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full0 + 8 * (t & 1));
+        }
+        if (t >= 1) {
+          // ---- O += P_{t-1} V_{t-1} (high part and residual of P)
+          const int u = t - 1, st = u % ST;
+          ok = mbar_wait(p_full0 + 8 * (u & 1), (u >> 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t vt = sbase + st * TT::kStageBytes + TT::kTileBytes;
+          const uint32_t phi = sbase + TT::kPOff + (u & 1) * 2 * TT::kPPart, plo = phi + TT::kPPart;
+#pragma unroll
+          for (int ks = 0; ks < T / 16; ++ks) {
+            const uint64_t vdesc = tc_smem_desc(vt + ks * 16 * 128, TT::kHalf, 1024);
+            tc_mma(tmem + 128, tc_smem_desc(phi + ks * 32, 16, 1024), vdesc, kIdescPV, (u > 0 || ks > 0) ? 1u : 0u);
+            tc_mma(tmem + 128, tc_smem_desc(plo + ks * 32, 16, 1024), vdesc, kIdescPV, 1u);
+          }
+          tc_commit(empty0 + 8 * st);  // the stage's K and V are no longer read
+          tc_commit(pv_done0 + 8 * (u & 1));
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+      }
+    }
+  } else {
+    // ============================================================ softmax rows
+    const int r = threadIdx.x;  // row of the slice = tensor-memory lane
+    const bool valid = r < pc.nh;
+    const bool warp_active = warp * 32 < pc.nh;
+    // the positions this row sees: with several query tokens per sequence,
+    // query token t sees the cache up to and including itself
+    const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + r) / p.r)) : 0;
+    const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sl = p.scale_log2;
+    float m_run = kNegInf, l_run = 0.f;
+    int bad = 0;
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int t0 = pc.t_begin + t * T;
+      const int st = t % ST;
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * (t & 1), (t >> 1) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[2][32];
+      tc_ld32(lane_tmem + (t & 1) * 64, sv[0]);
+      tc_ld32(lane_tmem + (t & 1) * 64 + 32, sv[1]);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free0 + 8 * (t & 1));
+      if (PAGED) bad |= tile_bad[st];
+      // V rows past the piece's end may hold anything (even NaN): zero them so
+      // that P = 0 there meets zeros
+      const int valid_rows = min(T, pc.t_end - t0);
+      if (valid_rows < T) {
+        uint8_t *vt = smem + st * TT::kStageBytes + TT::kTileBytes;
+        for (int idx = r; idx < (T - valid_rows) * 16; idx += 128) {
+          const int row = valid_rows + idx / 16, c = idx % 16;
+          *reinterpret_cast<uint4 *>(vt + (c >> 3) * TT::kHalf + row * 128 + ((c & 7) << 4)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      if (warp_active) {
+        float x[64];
+        float mx = kNegInf;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          x[j] = (t0 + j < lim) ? __uint_as_float(sv[j >> 5][j & 31]) * sl : kNegInf;
+          mx = fmaxf(mx, x[j]);
+        }
+        // lazy rescale: only when a score passes the base by more than 2^8
+        const bool need = mx > m_run + 8.f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float mn = need ? fmaxf(m_run, mx) : m_run;
+          const float alpha = need ? ((m_run == kNegInf) ? 0.f : ex2(m_run - mn)) : 1.f;
+          l_run *= alpha;
+          if (t > 0) {
+            // O holds tiles 0 .. t-1: rescale this row once their MMAs are done
+            ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t ov[32];
+              tc_ld32(lane_tmem + 128 + c * 32, ov);
+              tc_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+              tc_st32(lane_tmem + 128 + c * 32, ov);
+            }
+            tc_wait_st();
+            tc_fence_before();
+          }
+          m_run = mn;
+        }
+        const float base = (m_run == kNegInf) ? 0.f : m_run;
+        // P buffer t % 2 is free once the MMAs of tile t-2 are done
+        if (t > 1) {
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * (t & 1), ((t >> 1) - 1) & 1));
+          if (!ok) break;
+        }
+        uint8_t *ph = smem + TT::kPOff + (t & 1) * 2 * TT::kPPart + r * 128;
+        uint8_t *pl = ph + TT::kPPart;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = ex2(x[c * 8 + 2 * e] - base), p1 = ex2(x[c * 8 + 2 * e + 1] - base);
+            l_run += p0 + p1;
+            hi[e] = pack_bf16(p0, p1);
+            lo[e] = pack_bf16(p0 - bf16_round(p0), p1 - bf16_round(p1));
+          }
+          const int sw = (c ^ (r & 7)) << 4;
+          *reinterpret_cast<uint4 *>(ph + sw) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4 *>(pl + sw) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+      // (p_full is one barrier per P buffer: a warp reaches tile t+2 only
+      // after s_full of t+2, i.e. after the MMA thread issued the P.V of tile
+      // t, so its next arrival on the same barrier cannot fall into tile t's
+      // phase)
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full0 + 8 * (t & 1));
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      if (p.status) atomicOr(p.status, kStatusTimeout);
+    }
+    // ---- the row's result: O from tensor memory once the last MMAs are done
+    const bool done =
+        ok && __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1));
+    tc_fence_after();
+    const bool final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
+    const size_t row = valid ? row_of(p, pc.s, pc.g, pc.h0 + r) : 0;
+    const size_t ps = row * p.num_splits + pc.k;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t ov[32];
+      tc_ld32(lane_tmem + 128 + c * 32, ov);
+      tc_wait_ld();
+      if (valid) {
+        if (final_row) {
+          const float inv = (!bad && done && l_run > 0.f) ? 1.f / l_run : 0.f;
+          float4 *dst = reinterpret_cast<float4 *>(p.out + row * D) + c * 8;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(ov[4 * j]) * inv, __uint_as_float(ov[4 * j + 1]) * inv,
+                                 __uint_as_float(ov[4 * j + 2]) * inv, __uint_as_float(ov[4 * j + 3]) * inv);
+        } else {
+          float4 *dst = reinterpret_cast<float4 *>(p.part_o + ps * D) + c * 8;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(ov[4 * j]), __uint_as_float(ov[4 * j + 1]),
+                                 __uint_as_float(ov[4 * j + 2]), __uint_as_float(ov[4 * j + 3]));
+        }
+      }
+    }
+    if (valid) {
+      if (final_row) {
+        if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_run, l_run);
+        if (p.part_l) p.part_l[row * p.num_splits] = kLFinal;
+      } else {
+        p.part_m[ps] = m_run;
+        p.part_l[ps] = bad ? kLBadPage : l_run;
+      }
+    }
+    tc_fence_before();
+    if (p.unit_ctr != nullptr && !final_row) {
+      // ---- the block whose split completes the unit merges its splits (as
+      // in the mma.sync kernel)
+      named_barrier(1, 128);
+      const int ns = (pc.len + p.split_tokens - 1) / p.split_tokens;
+      if (r == 0) {
+        __threadfence();
+        const size_t u = (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j;
+        *merge_here = unit_arrive(p.unit_ctr + u, p.epoch, ns, p.status) ? 1 : 0;
+        __threadfence();
+      }
+      named_barrier(1, 128);
+      if (*merge_here) {
+        constexpr int kHalfRow = D / 8;  // two float4 columns per thread, half a row apart
+        for (int rb = 0; rb < pc.nh; rb += 128 / kHalfRow) {
+          const int h = rb + r / kHalfRow, c4 = r % kHalfRow;
+          if (h < pc.nh) {
+            const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
+            merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns,
+                               c4, kHalfRow, reinterpret_cast<float4 *>(p.out + mrow * D),
+                               p.lse ? p.lse + mrow : nullptr);
+          }
+        }
+      }
+    }
+  }
+
+  // ---- teardown: every tensor-memory access is done before the columns go back
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tc_dealloc(tmem, TT::kTmemCols);
+  }
+}
+
+}  // namespace gqa

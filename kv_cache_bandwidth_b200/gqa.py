@@ -24,7 +24,7 @@ __all__ = [
     "gqa_split_partials", "gqa_split_combine", "gqa_decode_split_workspace_size",
     "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version", "dims_for",
     "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
-    "FLAG_CONTRACT_FMA", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
+    "FLAG_CONTRACT_FMA", "FLAG_CONTRACT_TCGEN05", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
     "gqa_decode_split_lse", "gqa_merge_lse", "SERIAL_MERGE_MAX_SPLITS", "gqa_kv_append", "PagePool",
     "gqa_decode_verify", "gqa_decode_verify_workspace_size", "gqa_append_decode_split",
     "gqa_decode_split_mapped", "gqa_decode_split_mapped_workspace_size",
@@ -38,6 +38,7 @@ STATUS_BAD_PAGE = 2
 STATUS_TIMEOUT = 4
 FLAG_CONTRACT_MMA = 1
 FLAG_CONTRACT_FMA = 2
+FLAG_CONTRACT_TCGEN05 = 4
 
 ERRORS = {
     0: "GQA_OK", -1: "GQA_ERR_NULL_POINTER", -2: "GQA_ERR_MISALIGNED", -3: "GQA_ERR_HEADS",
@@ -202,12 +203,19 @@ def gqa_plan_split_tokens(dims: Dims, max_seqlen: int, num_sms: int = 0) -> int:
     return rc
 
 
-def workspace_for(q, k_cache, page_table, max_seqlen: int, split_tokens: int) -> torch.Tensor:
+def workspace_for(q, k_cache, page_table, max_seqlen: int, split_tokens: int, flags: int = 0) -> torch.Tensor:
     """Allocate a workspace (torch, on q's device) big enough for the call."""
-    n = gqa_decode_split_workspace_size(dims_for(q, k_cache, page_table), max_seqlen, split_tokens)
+    n = gqa_decode_split_workspace_size(dims_for(q, k_cache, page_table, flags), max_seqlen, split_tokens)
     if n == 0:
         raise GqaError(-6, "gqa_decode_split_workspace_size")
     return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def _workspace_or_stub(q, k_cache, page_table, max_seqlen, split_tokens, flags):
+    """workspace_for, or a stub when the arguments are invalid, so that the
+    entry point itself names the error."""
+    n = gqa_decode_split_workspace_size(dims_for(q, k_cache, page_table, flags), max_seqlen, split_tokens)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
 
 
 def gqa_decode_split(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int = 0,
@@ -222,7 +230,7 @@ def gqa_decode_split(q, k_cache, v_cache, seqlens, page_table=None, *, split_tok
     if max_seqlen is None:
         max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
     if workspace is None:
-        workspace = workspace_for(q, k_cache, page_table, max_seqlen, split_tokens)
+        workspace = _workspace_or_stub(q, k_cache, page_table, max_seqlen, split_tokens, flags)
     dims = dims_for(q, k_cache, page_table, flags)
     rc = load().gqa_decode_split(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
                                  _ptr(out), ctypes.byref(dims), _scale(q, scale), _ptr(status),
@@ -244,7 +252,7 @@ def gqa_decode_split_lse(q, k_cache, v_cache, seqlens, page_table=None, *, split
     if max_seqlen is None:
         max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
     if workspace is None:
-        workspace = workspace_for(q, k_cache, page_table, max_seqlen, split_tokens)
+        workspace = _workspace_or_stub(q, k_cache, page_table, max_seqlen, split_tokens, flags)
     dims = dims_for(q, k_cache, page_table, flags)
     rc = load().gqa_decode_split_lse(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(page_table),
                                      _ptr(out), _ptr(lse), ctypes.byref(dims), _scale(q, scale), _ptr(status),
@@ -368,7 +376,7 @@ def gqa_append_decode_split(k_new, v_new, q, k_cache, v_cache, seqlens, page_tab
     if max_seqlen is None:
         max_seqlen = k_cache.shape[2] * (1 if page_table is None else page_table.shape[1])
     if workspace is None:
-        workspace = workspace_for(q, k_cache, page_table, max_seqlen, split_tokens)
+        workspace = _workspace_or_stub(q, k_cache, page_table, max_seqlen, split_tokens, flags)
     dims = dims_for(q, k_cache, page_table, flags)
     rc = load().gqa_append_decode_split(_ptr(k_new), _ptr(v_new), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                         _ptr(seqlens), _ptr(page_table), _ptr(out), ctypes.byref(dims),
