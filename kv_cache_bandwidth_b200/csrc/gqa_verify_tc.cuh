@@ -14,13 +14,16 @@
 //
 // Rows are padded to M = 128; P enters as a bf16 high part and a bf16
 // residual (two MMAs), as in the mma.sync kernel.  Warp roles:
-//   * warps 0-3: one row per thread (the thread's tensor-memory lane).  Each
-//     tile: read the row's 64 scores from tensor memory, mask (the row's own
-//     causal limit among the drafts), online softmax in base 2 with the lazy
-//     rescale (a row whose maximum moves by more than 2^8 rescales its O row in
-//     tensor memory), write P to shared memory in the 128-byte swizzle;
-//   * warp 4: the TMA producer of the K/V ring (as in the mma.sync kernel);
-//   * warp 5: tensor-memory allocation; one thread issues the MMAs and signals
+//   * warps 0-7: two threads per row (warps w and w+4 share the tensor-memory
+//     lanes of rows 32(w%4) ..), each taking 32 of a tile's 64 tokens.  Each
+//     tile: read the half-row of scores from tensor memory, mask (the row's
+//     own causal limit among the drafts), agree with the partner thread on the
+//     row's maximum through shared memory, online softmax in base 2 with the
+//     lazy rescale (a row whose maximum moves by more than 2^8 rescales its O
+//     row in tensor memory, each thread half of the columns), write P to
+//     shared memory in the 128-byte swizzle;
+//   * warp 8: the TMA producer of the K/V ring (as in the mma.sync kernel);
+//   * warp 9: tensor-memory allocation; one thread issues the MMAs and signals
 //     their completion on mbarriers with tcgen05.commit.
 // S (in tensor memory) and P (in shared memory) are double-buffered: the
 // scores of tile t+1 are computed and its softmax runs while the P.V of tile t
@@ -47,11 +50,14 @@ struct TcTile {
   static constexpr int kPOff = kQOff + 2 * kQHalf;     // P: 2 buffers x (high part, residual) x kM rows x 64 tokens
   static constexpr int kPPart = kM * 128;
   static constexpr int kBarOff = kPOff + 4 * kPPart;
-  // full[3], empty[3], s_full[2], s_free[2], p_full[2], pv_done[2]
-  static constexpr int kNumBars = 2 * kStages + 8;
-  static constexpr int kMiscOff = kBarOff + 8 * kNumBars;  // tmem base, tile_bad[3], abort, merge here
+  // full[3], empty[3], s_full[2], s_free[2], p_full[2], pv_done[2], x_full[2]
+  static constexpr int kNumBars = 2 * kStages + 10;
+  static constexpr int kXOff = kBarOff + 8 * kNumBars;  // row maxima of each half row: [2 tiles][2][kM] floats
+  static constexpr int kLOff = kXOff + 4 * 2 * 2 * kM;  // the halves' sums at the end: [2][kM] floats
+  static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[3], abort, merge here
   static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * 8;
-  static constexpr int kThreads = 192;
+  static constexpr int kSoftmaxWarps = 8;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
   static constexpr uint32_t kTmemCols = 256;           // S (2 x 64 columns) + O (128)
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   const uint32_t bars = sbase + TT::kBarOff;
   const uint32_t full0 = bars, empty0 = bars + 8 * ST;
   const uint32_t s_full0 = bars + 16 * ST, s_free0 = s_full0 + 16;
-  const uint32_t p_full0 = s_free0 + 16, pv_done0 = p_full0 + 16;
+  const uint32_t p_full0 = s_free0 + 16, pv_done0 = p_full0 + 16, x_full0 = pv_done0 + 16;
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
   volatile int *abort_flag = tile_bad + ST;
@@ -194,15 +200,17 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full0 + 8 * i, 1);
-      mbar_init(s_free0 + 8 * i, 4);  // one arrival per softmax warp
-      mbar_init(p_full0 + 8 * i, 4);
+      mbar_init(s_free0 + 8 * i, TT::kSoftmaxWarps);  // one arrival per softmax warp
+      mbar_init(p_full0 + 8 * i, TT::kSoftmaxWarps);
       mbar_init(pv_done0 + 8 * i, 1);
+      mbar_init(x_full0 + 8 * i, TT::kSoftmaxWarps);
     }
     *abort_flag = 0;
     *merge_here = 0;
     fence_mbarrier_init();
   }
-  if (warp == 5) {
+  constexpr int kProducerWarp = TT::kSoftmaxWarps, kMmaWarp = TT::kSoftmaxWarps + 1;
+  if (warp == kMmaWarp) {
     tc_alloc(smem_addr(const_cast<uint32_t *>(tmem_slot)), TT::kTmemCols);
     tc_relinquish();
   }
@@ -225,10 +233,10 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ============================================================ producer
     tc_produce<PAGED>(&tm_k, &tm_v, p, pc, sbase, full0, empty0, tile_bad, abort_flag, lane);
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ============================================================ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescQK = tc_idesc_bf16(128, 64, false);
@@ -278,15 +286,20 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     }
   } else {
     // ============================================================ softmax rows
-    const int r = threadIdx.x;  // row of the slice = tensor-memory lane
+    constexpr int kSM = 32 * TT::kSoftmaxWarps;  // softmax threads
+    const int sm = threadIdx.x;                  // 0 .. kSM-1
+    const int half = sm / 128;                   // tokens [32 half, 32 half + 32) of every tile
+    const int r = sm % 128;                      // row of the slice = tensor-memory lane
     const bool valid = r < pc.nh;
-    const bool warp_active = warp * 32 < pc.nh;
+    const bool warp_active = (warp % 4) * 32 < pc.nh;
     // the positions this row sees: with several query tokens per sequence,
     // query token t sees the cache up to and including itself
     const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + r) / p.r)) : 0;
-    const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_tmem = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    float *xmax = reinterpret_cast<float *>(smem + TT::kXOff);  // [tile % 2][half][row]
+    float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);  // [half][row]
     const float sl = p.scale_log2;
-    float m_run = kNegInf, l_run = 0.f;
+    float m_run = kNegInf, l_run = 0.f;  // the row's base (shared by the pair) and this half's sum
     int bad = 0;
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
@@ -295,9 +308,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * (t & 1), (t >> 1) & 1));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[2][32];
-      tc_ld32(lane_tmem + (t & 1) * 64, sv[0]);
-      tc_ld32(lane_tmem + (t & 1) * 64 + 32, sv[1]);
+      uint32_t sv[32];
+      tc_ld32(lane_tmem + (t & 1) * 64 + half * 32, sv);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -308,20 +320,30 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       const int valid_rows = min(T, pc.t_end - t0);
       if (valid_rows < T) {
         uint8_t *vt = smem + st * TT::kStageBytes + TT::kTileBytes;
-        for (int idx = r; idx < (T - valid_rows) * 16; idx += 128) {
+        for (int idx = sm; idx < (T - valid_rows) * 16; idx += kSM) {
           const int row = valid_rows + idx / 16, c = idx % 16;
           *reinterpret_cast<uint4 *>(vt + (c >> 3) * TT::kHalf + row * 128 + ((c & 7) << 4)) =
               make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      if (warp_active) {
-        float x[64];
-        float mx = kNegInf;
+      float x[32];
+      float mx = kNegInf;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          x[j] = (t0 + j < lim) ? __uint_as_float(sv[j >> 5][j & 31]) * sl : kNegInf;
-          mx = fmaxf(mx, x[j]);
-        }
+      for (int j = 0; j < 32; ++j) {
+        x[j] = (t0 + half * 32 + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
+        mx = fmaxf(mx, x[j]);
+      }
+      // the row's maximum over both halves, exchanged through shared memory
+      // (every softmax warp takes part; the buffer of tile t is written again
+      // at tile t+2, which no warp reaches before all have passed the P
+      // hand-over of tile t)
+      xmax[((t & 1) * 2 + half) * 128 + r] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(x_full0 + 8 * (t & 1));
+      ok = __all_sync(0xffffffffu, mbar_wait(x_full0 + 8 * (t & 1), (t >> 1) & 1));
+      if (!ok) break;
+      mx = fmaxf(mx, xmax[((t & 1) * 2 + (half ^ 1)) * 128 + r]);
+      if (warp_active) {
         // lazy rescale: only when a score passes the base by more than 2^8
         const bool need = mx > m_run + 8.f;
         if (__any_sync(0xffffffffu, need)) {
@@ -329,18 +351,18 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
           const float alpha = need ? ((m_run == kNegInf) ? 0.f : ex2(m_run - mn)) : 1.f;
           l_run *= alpha;
           if (t > 0) {
-            // O holds tiles 0 .. t-1: rescale this row once their MMAs are done
+            // O holds tiles 0 .. t-1: rescale this half of the row once their MMAs are done
             ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
               uint32_t ov[32];
-              tc_ld32(lane_tmem + 128 + c * 32, ov);
+              tc_ld32(lane_tmem + 128 + half * 64 + c * 32, ov);
               tc_wait_ld();
 #pragma unroll
               for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-              tc_st32(lane_tmem + 128 + c * 32, ov);
+              tc_st32(lane_tmem + 128 + half * 64 + c * 32, ov);
             }
             tc_wait_st();
             tc_fence_before();
@@ -356,7 +378,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         uint8_t *ph = smem + TT::kPOff + (t & 1) * 2 * TT::kPPart + r * 128;
         uint8_t *pl = ph + TT::kPPart;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -365,7 +387,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
             hi[e] = pack_bf16(p0, p1);
             lo[e] = pack_bf16(p0 - bf16_round(p0), p1 - bf16_round(p1));
           }
-          const int sw = (c ^ (r & 7)) << 4;
+          const int sw = ((half * 4 + c) ^ (r & 7)) << 4;
           *reinterpret_cast<uint4 *>(ph + sw) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4 *>(pl + sw) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
@@ -386,24 +408,28 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     const bool done =
         ok && __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1));
     tc_fence_after();
+    lsum[half * 128 + r] = l_run;
+    named_barrier(1, kSM);
+    const float l_row = lsum[r] + lsum[128 + r];
     const bool final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
     const size_t row = valid ? row_of(p, pc.s, pc.g, pc.h0 + r) : 0;
     const size_t ps = row * p.num_splits + pc.k;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       uint32_t ov[32];
-      tc_ld32(lane_tmem + 128 + c * 32, ov);
+      const int col = half * 64 + c * 32;
+      tc_ld32(lane_tmem + 128 + col, ov);
       tc_wait_ld();
       if (valid) {
         if (final_row) {
-          const float inv = (!bad && done && l_run > 0.f) ? 1.f / l_run : 0.f;
-          float4 *dst = reinterpret_cast<float4 *>(p.out + row * D) + c * 8;
+          const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
+          float4 *dst = reinterpret_cast<float4 *>(p.out + row * D + col);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             dst[j] = make_float4(__uint_as_float(ov[4 * j]) * inv, __uint_as_float(ov[4 * j + 1]) * inv,
                                  __uint_as_float(ov[4 * j + 2]) * inv, __uint_as_float(ov[4 * j + 3]) * inv);
         } else {
-          float4 *dst = reinterpret_cast<float4 *>(p.part_o + ps * D) + c * 8;
+          float4 *dst = reinterpret_cast<float4 *>(p.part_o + ps * D + col);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             dst[j] = make_float4(__uint_as_float(ov[4 * j]), __uint_as_float(ov[4 * j + 1]),
@@ -411,32 +437,32 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         }
       }
     }
-    if (valid) {
+    if (valid && half == 0) {
       if (final_row) {
-        if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_run, l_run);
+        if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_run, l_row);
         if (p.part_l) p.part_l[row * p.num_splits] = kLFinal;
       } else {
         p.part_m[ps] = m_run;
-        p.part_l[ps] = bad ? kLBadPage : l_run;
+        p.part_l[ps] = bad ? kLBadPage : l_row;
       }
     }
     tc_fence_before();
     if (p.unit_ctr != nullptr && !final_row) {
       // ---- the block whose split completes the unit merges its splits (as
       // in the mma.sync kernel)
-      named_barrier(1, 128);
+      named_barrier(1, kSM);
       const int ns = (pc.len + p.split_tokens - 1) / p.split_tokens;
-      if (r == 0) {
+      if (sm == 0) {
         __threadfence();
         const size_t u = (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j;
         *merge_here = unit_arrive(p.unit_ctr + u, p.epoch, ns, p.status) ? 1 : 0;
         __threadfence();
       }
-      named_barrier(1, 128);
+      named_barrier(1, kSM);
       if (*merge_here) {
         constexpr int kHalfRow = D / 8;  // two float4 columns per thread, half a row apart
-        for (int rb = 0; rb < pc.nh; rb += 128 / kHalfRow) {
-          const int h = rb + r / kHalfRow, c4 = r % kHalfRow;
+        for (int rb = 0; rb < pc.nh; rb += kSM / kHalfRow) {
+          const int h = rb + sm / kHalfRow, c4 = sm % kHalfRow;
           if (h < pc.nh) {
             const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
             merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns,
@@ -451,7 +477,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   // ---- teardown: every tensor-memory access is done before the columns go back
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tc_dealloc(tmem, TT::kTmemCols);
   }
