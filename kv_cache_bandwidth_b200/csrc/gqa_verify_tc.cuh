@@ -13,7 +13,10 @@
 //   O[rows, 128]       += P[rows, 64] . V_tile[64, 128]            (M = 128, N = 128)
 //
 // Rows are padded to M = 128; P enters as a bf16 high part and a bf16
-// residual (two MMAs), as in the mma.sync kernel.  Warp roles:
+// residual (two MMAs), as in the mma.sync kernel.  P is written to tensor
+// memory over its own scores (each thread over the columns it has read) and
+// the P.V product takes its A operand from there, which leaves shared memory
+// to a 5-stage K/V ring.  Warp roles:
 //   * warps 0-7: two threads per row (warps w and w+4 share the tensor-memory
 //     lanes of rows 32(w%4) ..), each taking 32 of a tile's 64 tokens.  Each
 //     tile: read the half-row of scores from tensor memory, mask (the row's
@@ -21,13 +24,13 @@
 //     row's maximum through shared memory, online softmax in base 2 with the
 //     lazy rescale (a row whose maximum moves by more than 2^8 rescales its O
 //     row in tensor memory, each thread half of the columns), write P to
-//     shared memory in the 128-byte swizzle;
+//     tensor memory;
 //   * warp 8: the TMA producer of the K/V ring (as in the mma.sync kernel);
 //   * warp 9: tensor-memory allocation; one thread issues the MMAs and signals
 //     their completion on mbarriers with tcgen05.commit.
-// S (in tensor memory) and P (in shared memory) are double-buffered: the
-// scores of tile t+1 are computed and its softmax runs while the P.V of tile t
-// is on the tensor cores.  The epilogue writes final rows
+// S and P share two tensor-memory buffers: the scores of tile t+1 are
+// computed and its softmax runs while the P.V of tile t is on the tensor
+// cores; a buffer takes new scores once the P.V that read it is done.  The epilogue writes final rows
 // or partial states in the layout of the mma.sync kernel, so the same merges
 // (in this kernel for up to 8 splits, the combine kernel otherwise) apply.
 #pragma once
@@ -41,29 +44,27 @@ struct TcTile {
   static constexpr int kD = 128;
   static constexpr int kT = 64;                        // tokens per tile
   static constexpr int kM = 128;                       // rows of every MMA (padded)
-  static constexpr int kStages = 3;
+  static constexpr int kStages = 5;
   static constexpr int kHalf = kT * 128;               // one 64-column half of a K or V tile
   static constexpr int kTileBytes = 2 * kHalf;         // 16 KB
   static constexpr int kStageBytes = 2 * kTileBytes;   // K + V
   static constexpr int kQOff = kStages * kStageBytes;  // Q: two halves of kM rows x 128 B
   static constexpr int kQHalf = kM * 128;
-  static constexpr int kPOff = kQOff + 2 * kQHalf;     // P: 2 buffers x (high part, residual) x kM rows x 64 tokens
-  static constexpr int kPPart = kM * 128;
-  static constexpr int kBarOff = kPOff + 4 * kPPart;
-  // full[3], empty[3], s_full[2], s_free[2], p_full[2], pv_done[2], x_full[2]
-  static constexpr int kNumBars = 2 * kStages + 10;
+  static constexpr int kBarOff = kQOff + 2 * kQHalf;
+  // full[kStages], empty[kStages], s_full[2], p_full[2], pv_done[2], x_full[2]
+  static constexpr int kNumBars = 2 * kStages + 8;
   static constexpr int kXOff = kBarOff + 8 * kNumBars;  // row maxima of each half row: [2 tiles][2][kM] floats
   static constexpr int kLOff = kXOff + 4 * 2 * 2 * kM;  // the halves' sums at the end: [2][kM] floats
-  static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[3], abort, merge here
-  static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * 8;
+  static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[kStages], abort, merge here
+  static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * (kStages + 3);
   static constexpr int kSoftmaxWarps = 8;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
-  static constexpr uint32_t kTmemCols = 256;           // S (2 x 64 columns) + O (128)
+  static constexpr uint32_t kTmemCols = 256;           // S, then P over it (2 x 64 columns) + O (128)
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 // TMA producer for one piece (items mode): K and V tiles of 64 tokens into the
-// 3-stage ring, pages translated through the table as in the mma.sync kernel.
+// stage ring, pages translated through the table as in the mma.sync kernel.
 template <bool PAGED>
 __device__ __forceinline__ void tc_produce(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeParams &p,
                                            const Piece &pc, uint32_t sbase, uint32_t full0, uint32_t empty0,
@@ -163,8 +164,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bars = sbase + TT::kBarOff;
   const uint32_t full0 = bars, empty0 = bars + 8 * ST;
-  const uint32_t s_full0 = bars + 16 * ST, s_free0 = s_full0 + 16;
-  const uint32_t p_full0 = s_free0 + 16, pv_done0 = p_full0 + 16, x_full0 = pv_done0 + 16;
+  const uint32_t s_full0 = bars + 16 * ST;
+  const uint32_t p_full0 = s_full0 + 16, pv_done0 = p_full0 + 16, x_full0 = pv_done0 + 16;
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
   volatile int *abort_flag = tile_bad + ST;
@@ -200,8 +201,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full0 + 8 * i, 1);
-      mbar_init(s_free0 + 8 * i, TT::kSoftmaxWarps);  // one arrival per softmax warp
-      mbar_init(p_full0 + 8 * i, TT::kSoftmaxWarps);
+      mbar_init(p_full0 + 8 * i, TT::kSoftmaxWarps);  // one arrival per softmax warp
       mbar_init(pv_done0 + 8 * i, 1);
       mbar_init(x_full0 + 8 * i, TT::kSoftmaxWarps);
     }
@@ -248,7 +248,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
           // ---- S[t % 2] = Q K_t^T
           const int st = t % ST;
           ok = mbar_wait(full0 + 8 * st, (t / ST) & 1);
-          if (ok && t >= 2) ok = mbar_wait(s_free0 + 8 * (t & 1), ((t >> 1) - 1) & 1);
+          // buffer t % 2 holds P of tile t-2 until its P.V is done
+          if (ok && t >= 2) ok = mbar_wait(pv_done0 + 8 * (t & 1), ((t >> 1) - 1) & 1);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kt = sbase + st * TT::kStageBytes;
@@ -268,12 +269,14 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t vt = sbase + st * TT::kStageBytes + TT::kTileBytes;
-          const uint32_t phi = sbase + TT::kPOff + (u & 1) * 2 * TT::kPPart, plo = phi + TT::kPPart;
 #pragma unroll
           for (int ks = 0; ks < T / 16; ++ks) {
+            // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of
+            // the buffer, the residual 16 columns further
             const uint64_t vdesc = tc_smem_desc(vt + ks * 16 * 128, TT::kHalf, 1024);
-            tc_mma(tmem + 128, tc_smem_desc(phi + ks * 32, 16, 1024), vdesc, kIdescPV, (u > 0 || ks > 0) ? 1u : 0u);
-            tc_mma(tmem + 128, tc_smem_desc(plo + ks * 32, 16, 1024), vdesc, kIdescPV, 1u);
+            const uint32_t pa = tmem + (u & 1) * 64 + 32 * (ks >> 1) + 8 * (ks & 1);
+            tc_mma_ts(tmem + 128, pa, vdesc, kIdescPV, (u > 0 || ks > 0) ? 1u : 0u);
+            tc_mma_ts(tmem + 128, pa + 16, vdesc, kIdescPV, 1u);
           }
           tc_commit(empty0 + 8 * st);  // the stage's K and V are no longer read
           tc_commit(pv_done0 + 8 * (u & 1));
@@ -311,9 +314,6 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       uint32_t sv[32];
       tc_ld32(lane_tmem + (t & 1) * 64 + half * 32, sv);
       tc_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free0 + 8 * (t & 1));
       if (PAGED) bad |= tile_bad[st];
       // V rows past the piece's end may hold anything (even NaN): zero them so
       // that P = 0 there meets zeros
@@ -370,33 +370,28 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
           m_run = mn;
         }
         const float base = (m_run == kNegInf) ? 0.f : m_run;
-        // P buffer t % 2 is free once the MMAs of tile t-2 are done
-        if (t > 1) {
-          ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * (t & 1), ((t >> 1) - 1) & 1));
-          if (!ok) break;
-        }
-        uint8_t *ph = smem + TT::kPOff + (t & 1) * 2 * TT::kPPart + r * 128;
-        uint8_t *pl = ph + TT::kPPart;
+        // P over this thread's own 32 score columns: high part in the first
+        // 16, residual in the next 16 (the buffer's scores of tile t are no
+        // longer needed, and the MMAs of tile t-2 that read it are done, since
+        // the scores of tile t came after them)
+        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2(x[c * 8 + 2 * e] - base), p1 = ex2(x[c * 8 + 2 * e + 1] - base);
-            l_run += p0 + p1;
-            hi[e] = pack_bf16(p0, p1);
-            lo[e] = pack_bf16(p0 - bf16_round(p0), p1 - bf16_round(p1));
-          }
-          const int sw = ((half * 4 + c) ^ (r & 7)) << 4;
-          *reinterpret_cast<uint4 *>(ph + sw) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4 *>(pl + sw) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
+          l_run += p0 + p1;
+          hi[e] = pack_bf16(p0, p1);
+          lo[e] = pack_bf16(p0 - bf16_round(p0), p1 - bf16_round(p1));
         }
+        tc_st16(lane_tmem + (t & 1) * 64 + half * 32, hi);
+        tc_st16(lane_tmem + (t & 1) * 64 + half * 32 + 16, lo);
+        tc_wait_st();
       }
       // (p_full is one barrier per P buffer: a warp reaches tile t+2 only
       // after s_full of t+2, i.e. after the MMA thread issued the P.V of tile
       // t, so its next arrival on the same barrier cannot fall into tile t's
       // phase)
-      fence_proxy_async_smem();
+      tc_fence_before();
+      if (valid_rows < T) fence_proxy_async_smem();  // the zeroed V rows, for the tensor core
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full0 + 8 * (t & 1));
     }
