@@ -1143,10 +1143,13 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
             l_run[j][0] += p0 + p2;
             l_run[j][1] += p1 + p3;
             // high and residual bf16 parts, transposed into the B layout
-            bh[j][0] = movmatrix_trans(pack_bf16(p0, p1));
-            bh[j][1] = movmatrix_trans(pack_bf16(p2, p3));
-            bl[j][0] = movmatrix_trans(pack_bf16(p0 - bf16_round(p0), p1 - bf16_round(p1)));
-            bl[j][1] = movmatrix_trans(pack_bf16(p2 - bf16_round(p2), p3 - bf16_round(p3)));
+            uint32_t h01, l01, h23, l23;
+            split_bf16x2(p0, p1, h01, l01);
+            split_bf16x2(p2, p3, h23, l23);
+            bh[j][0] = movmatrix_trans(h01);
+            bh[j][1] = movmatrix_trans(h23);
+            bl[j][0] = movmatrix_trans(l01);
+            bl[j][1] = movmatrix_trans(l23);
           }
           // ---- O^T += V^T P^T
           const bool tail = t0 + row0 + 16 > pc.t_end;

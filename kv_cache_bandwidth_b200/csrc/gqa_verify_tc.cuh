@@ -28,11 +28,12 @@
 //   * warp 8: the TMA producer of the K/V ring (as in the mma.sync kernel);
 //   * warp 9: tensor-memory allocation; one thread issues the MMAs and signals
 //     their completion on mbarriers with tcgen05.commit.
-// S and P share two tensor-memory buffers: the scores of tile t+1 are
-// computed and its softmax runs while the P.V of tile t is on the tensor
-// cores; a buffer takes new scores once the P.V that read it is done.  The epilogue writes final rows
-// or partial states in the layout of the mma.sync kernel, so the same merges
-// (in this kernel for up to 8 splits, the combine kernel otherwise) apply.
+// S and P share three tensor-memory buffers: the scores of tiles t+1 and t+2
+// are computed and the softmax of t+1 runs while the P.V of tile t is on the
+// tensor cores; a buffer takes new scores once the P.V that read it is done.
+// The epilogue writes final rows or partial states in the layout of the
+// mma.sync kernel, so the same merges (in this kernel for up to 8 splits, the
+// combine kernel otherwise) apply.
 #pragma once
 
 #include "gqa_kernels.cuh"
@@ -51,15 +52,18 @@ struct TcTile {
   static constexpr int kQOff = kStages * kStageBytes;  // Q: two halves of kM rows x 128 B
   static constexpr int kQHalf = kM * 128;
   static constexpr int kBarOff = kQOff + 2 * kQHalf;
-  // full[kStages], empty[kStages], s_full[2], p_full[2], pv_done[2], x_full[2]
-  static constexpr int kNumBars = 2 * kStages + 8;
-  static constexpr int kXOff = kBarOff + 8 * kNumBars;  // row maxima of each half row: [2 tiles][2][kM] floats
-  static constexpr int kLOff = kXOff + 4 * 2 * 2 * kM;  // the halves' sums at the end: [2][kM] floats
+  static constexpr int kSP = 3;                        // S/P buffers in tensor memory
+  // full[kStages], empty[kStages], s_full[kSP], p_full[kSP], pv_done[kSP], x_full[kSP]
+  static constexpr int kNumBars = 2 * kStages + 4 * kSP;
+  static constexpr int kXOff = kBarOff + 8 * kNumBars;  // row maxima of each half row: [kSP tiles][2][kM] floats
+  static constexpr int kLOff = kXOff + 4 * kSP * 2 * kM;  // the halves' sums at the end: [2][kM] floats
   static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[kStages], abort, merge here
   static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * (kStages + 3);
   static constexpr int kSoftmaxWarps = 8;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
-  static constexpr uint32_t kTmemCols = 256;           // S, then P over it (2 x 64 columns) + O (128)
+  static constexpr uint32_t kOCol = 256;               // O: columns 256 .. 383
+  static constexpr uint32_t kTmemCols = 512;           // S, then P over it (kSP x 64 columns) + O
+  static_assert(kSP * kT <= static_cast<int>(kOCol), "S/P buffers below O");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -164,8 +168,9 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bars = sbase + TT::kBarOff;
   const uint32_t full0 = bars, empty0 = bars + 8 * ST;
+  constexpr int SP = TT::kSP;
   const uint32_t s_full0 = bars + 16 * ST;
-  const uint32_t p_full0 = s_full0 + 16, pv_done0 = p_full0 + 16, x_full0 = pv_done0 + 16;
+  const uint32_t p_full0 = s_full0 + 8 * SP, pv_done0 = p_full0 + 8 * SP, x_full0 = pv_done0 + 8 * SP;
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
   volatile int *abort_flag = tile_bad + ST;
@@ -199,7 +204,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       mbar_init(empty0 + 8 * i, 1);  // one tcgen05.commit per use
       tile_bad[i] = 0;
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < SP; ++i) {
       mbar_init(s_full0 + 8 * i, 1);
       mbar_init(p_full0 + 8 * i, TT::kSoftmaxWarps);  // one arrival per softmax warp
       mbar_init(pv_done0 + 8 * i, 1);
@@ -238,6 +243,9 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     tc_produce<PAGED>(&tm_k, &tm_v, p, pc, sbase, full0, empty0, tile_bad, abort_flag, lane);
   } else if (warp == kMmaWarp) {
     // ============================================================ MMA issuer
+    // (the tensor pipe runs the products in issue order: the scores of tile
+    // t go ahead of the P.V of tile t-1, so that the softmax of t can start
+    // while that P.V runs)
     if (lane == 0) {
       constexpr uint32_t kIdescQK = tc_idesc_bf16(128, 64, false);
       constexpr uint32_t kIdescPV = tc_idesc_bf16(128, 128, true);
@@ -245,11 +253,11 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       bool ok = true;
       for (int t = 0; t <= n_tiles && ok; ++t) {
         if (t < n_tiles) {
-          // ---- S[t % 2] = Q K_t^T
+          // ---- S[t % SP] = Q K_t^T
           const int st = t % ST;
           ok = mbar_wait(full0 + 8 * st, (t / ST) & 1);
-          // buffer t % 2 holds P of tile t-2 until its P.V is done
-          if (ok && t >= 2) ok = mbar_wait(pv_done0 + 8 * (t & 1), ((t >> 1) - 1) & 1);
+          // buffer t % SP holds P of tile t-SP until its P.V is done
+          if (ok && t >= SP) ok = mbar_wait(pv_done0 + 8 * (t % SP), ((t / SP) - 1) & 1);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kt = sbase + st * TT::kStageBytes;
@@ -257,15 +265,15 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
           for (int ks = 0; ks < D / 16; ++ks) {
             const uint32_t koff = (ks >> 2) * TT::kHalf + (ks & 3) * 32;
             const uint32_t qoff = (ks >> 2) * TT::kQHalf + (ks & 3) * 32;
-            tc_mma(tmem + (t & 1) * 64, tc_smem_desc(q_sm + qoff, 16, 1024), tc_smem_desc(kt + koff, 16, 1024),
+            tc_mma(tmem + (t % SP) * 64, tc_smem_desc(q_sm + qoff, 16, 1024), tc_smem_desc(kt + koff, 16, 1024),
                    kIdescQK, ks > 0 ? 1u : 0u);
           }
-          tc_commit(s_full0 + 8 * (t & 1));
+          tc_commit(s_full0 + 8 * (t % SP));
         }
         if (t >= 1) {
-          // ---- O += P_{t-1} V_{t-1} (high part and residual of P)
+          // ---- O += P_{t-1} V_{t-1} (high part and residual of P, from tensor memory)
           const int u = t - 1, st = u % ST;
-          ok = mbar_wait(p_full0 + 8 * (u & 1), (u >> 1) & 1);
+          ok = mbar_wait(p_full0 + 8 * (u % SP), (u / SP) & 1);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vt = sbase + st * TT::kStageBytes + TT::kTileBytes;
@@ -274,12 +282,12 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
             // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of
             // the buffer, the residual 16 columns further
             const uint64_t vdesc = tc_smem_desc(vt + ks * 16 * 128, TT::kHalf, 1024);
-            const uint32_t pa = tmem + (u & 1) * 64 + 32 * (ks >> 1) + 8 * (ks & 1);
-            tc_mma_ts(tmem + 128, pa, vdesc, kIdescPV, (u > 0 || ks > 0) ? 1u : 0u);
-            tc_mma_ts(tmem + 128, pa + 16, vdesc, kIdescPV, 1u);
+            const uint32_t pa = tmem + (u % SP) * 64 + 32 * (ks >> 1) + 8 * (ks & 1);
+            tc_mma_ts(tmem + TT::kOCol, pa, vdesc, kIdescPV, (u > 0 || ks > 0) ? 1u : 0u);
+            tc_mma_ts(tmem + TT::kOCol, pa + 16, vdesc, kIdescPV, 1u);
           }
           tc_commit(empty0 + 8 * st);  // the stage's K and V are no longer read
-          tc_commit(pv_done0 + 8 * (u & 1));
+          tc_commit(pv_done0 + 8 * (u % SP));
         }
       }
       if (!ok) {
@@ -299,7 +307,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     // query token t sees the cache up to and including itself
     const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + r) / p.r)) : 0;
     const uint32_t lane_tmem = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-    float *xmax = reinterpret_cast<float *>(smem + TT::kXOff);  // [tile % 2][half][row]
+    float *xmax = reinterpret_cast<float *>(smem + TT::kXOff);  // [tile % SP][half][row]
     float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);  // [half][row]
     const float sl = p.scale_log2;
     float m_run = kNegInf, l_run = 0.f;  // the row's base (shared by the pair) and this half's sum
@@ -308,11 +316,12 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     for (int t = 0; t < n_tiles; ++t) {
       const int t0 = pc.t_begin + t * T;
       const int st = t % ST;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * (t & 1), (t >> 1) & 1));
+      const int b = t % SP;
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (t / SP) & 1));
       if (!ok) break;
       tc_fence_after();
       uint32_t sv[32];
-      tc_ld32(lane_tmem + (t & 1) * 64 + half * 32, sv);
+      tc_ld32(lane_tmem + b * 64 + half * 32, sv);
       tc_wait_ld();
       if (PAGED) bad |= tile_bad[st];
       // V rows past the piece's end may hold anything (even NaN): zero them so
@@ -327,22 +336,26 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         }
       }
       float x[32];
-      float mx = kNegInf;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x[j] = (t0 + half * 32 + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
-        mx = fmaxf(mx, x[j]);
+      for (int j = 0; j < 32; ++j) x[j] = (t0 + half * 32 + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
+      float mx;
+      {
+        float m8[8];  // a tree, not a chain of 32 dependent steps
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(fmaxf(x[4 * k], x[4 * k + 1]), fmaxf(x[4 * k + 2], x[4 * k + 3]));
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       }
       // the row's maximum over both halves, exchanged through shared memory
       // (every softmax warp takes part; the buffer of tile t is written again
-      // at tile t+2, which no warp reaches before all have passed the P
-      // hand-over of tile t)
-      xmax[((t & 1) * 2 + half) * 128 + r] = mx;
+      // at tile t+SP, which no warp reaches before all have passed the P
+      // hand-over of tile t: the scores of t+SP come after the P.V of t+1
+      // is issued)
+      xmax[(b * 2 + half) * 128 + r] = mx;
       __syncwarp();
-      if (lane == 0) mbar_arrive(x_full0 + 8 * (t & 1));
-      ok = __all_sync(0xffffffffu, mbar_wait(x_full0 + 8 * (t & 1), (t >> 1) & 1));
+      if (lane == 0) mbar_arrive(x_full0 + 8 * b);
+      ok = __all_sync(0xffffffffu, mbar_wait(x_full0 + 8 * b, (t / SP) & 1));
       if (!ok) break;
-      mx = fmaxf(mx, xmax[((t & 1) * 2 + (half ^ 1)) * 128 + r]);
+      mx = fmaxf(mx, xmax[(b * 2 + (half ^ 1)) * 128 + r]);
       if (warp_active) {
         // lazy rescale: only when a score passes the base by more than 2^8
         const bool need = mx > m_run + 8.f;
@@ -352,17 +365,17 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
           l_run *= alpha;
           if (t > 0) {
             // O holds tiles 0 .. t-1: rescale this half of the row once their MMAs are done
-            ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1));
+            ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((t - 1) % SP), ((t - 1) / SP) & 1));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               uint32_t ov[32];
-              tc_ld32(lane_tmem + 128 + half * 64 + c * 32, ov);
+              tc_ld32(lane_tmem + TT::kOCol + half * 64 + c * 32, ov);
               tc_wait_ld();
 #pragma unroll
               for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-              tc_st32(lane_tmem + 128 + half * 64 + c * 32, ov);
+              tc_st32(lane_tmem + TT::kOCol + half * 64 + c * 32, ov);
             }
             tc_wait_st();
             tc_fence_before();
@@ -372,28 +385,27 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         const float base = (m_run == kNegInf) ? 0.f : m_run;
         // P over this thread's own 32 score columns: high part in the first
         // 16, residual in the next 16 (the buffer's scores of tile t are no
-        // longer needed, and the MMAs of tile t-2 that read it are done, since
+        // longer needed, and the MMAs of tile t-SP that read it are done, since
         // the scores of tile t came after them)
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
           l_run += p0 + p1;
-          hi[e] = pack_bf16(p0, p1);
-          lo[e] = pack_bf16(p0 - bf16_round(p0), p1 - bf16_round(p1));
+          split_bf16x2(p0, p1, hi[e], lo[e]);
         }
-        tc_st16(lane_tmem + (t & 1) * 64 + half * 32, hi);
-        tc_st16(lane_tmem + (t & 1) * 64 + half * 32 + 16, lo);
+        tc_st16(lane_tmem + b * 64 + half * 32, hi);
+        tc_st16(lane_tmem + b * 64 + half * 32 + 16, lo);
         tc_wait_st();
       }
-      // (p_full is one barrier per P buffer: a warp reaches tile t+2 only
-      // after s_full of t+2, i.e. after the MMA thread issued the P.V of tile
-      // t, so its next arrival on the same barrier cannot fall into tile t's
-      // phase)
+      // (p_full is one barrier per P buffer: a warp reaches tile t+SP only
+      // after s_full of t+SP, i.e. after the MMA thread issued the P.V of
+      // tile t, so its next arrival on the same barrier cannot fall into tile
+      // t's phase)
       tc_fence_before();
       if (valid_rows < T) fence_proxy_async_smem();  // the zeroed V rows, for the tensor core
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full0 + 8 * (t & 1));
+      if (lane == 0) mbar_arrive(p_full0 + 8 * b);
     }
     if (!ok && lane == 0) {
       *abort_flag = 1;
@@ -401,7 +413,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     }
     // ---- the row's result: O from tensor memory once the last MMAs are done
     const bool done =
-        ok && __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1));
+        ok && __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((n_tiles - 1) % SP), ((n_tiles - 1) / SP) & 1));
     tc_fence_after();
     lsum[half * 128 + r] = l_run;
     named_barrier(1, kSM);
@@ -413,7 +425,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     for (int c = 0; c < 2; ++c) {
       uint32_t ov[32];
       const int col = half * 64 + c * 32;
-      tc_ld32(lane_tmem + 128 + col, ov);
+      tc_ld32(lane_tmem + TT::kOCol + col, ov);
       tc_wait_ld();
       if (valid) {
         if (final_row) {

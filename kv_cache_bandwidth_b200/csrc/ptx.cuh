@@ -145,8 +145,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ float bf16_round(float x) {
-  return __bfloat162float(__float2bfloat16_rn(x));
+// (a, b) as bf16 pairs: hi = the round-to-nearest values, lo = the rounded
+// residuals a - hi.a, b - hi.b (hi.a is the low half).  The residuals are
+// taken from hi's own bits, so one packed conversion serves both.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+  hi = pack_bf16(a, b);
+  lo = pack_bf16(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
 }
 
 // ---------------------------------------------------------------- PDL
