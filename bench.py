@@ -7,6 +7,7 @@ q.k scores, online softmax, p.V) and the combine kernel that merges the splits
 and normalises.  The inputs are resident in HBM when the timed region starts.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama70b]
+    python bench.py --query-tokens 8 ...        # a verification step: 8 query tokens per sequence
     python bench.py --impl reference ...        # the float64 CPU oracle instead
 
 Prints one JSON line (rank 0).  Under torchrun every rank runs its own shard
@@ -32,7 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from kv_cache_bandwidth_b200 import accounting  # noqa: E402
-from kv_cache_bandwidth_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+from kv_cache_bandwidth_b200.workloads import WORKLOADS, draw_verify_q, make_inputs  # noqa: E402
 
 METRIC = "GQA decode µs/step and KV-cache HBM GB/s as % of B200 peak (1 GPU)"
 FALLBACK_HBM_GBS = 6650.0
@@ -59,6 +60,10 @@ def kernel_source_hash() -> str:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
+
+
+def traffic_key(workload: str, n_query: int = 1) -> str:
+    return workload if n_query == 1 else "%s_verify%d" % (workload, n_query)
 
 
 def recorded_traffic(workload: str):
@@ -159,17 +164,20 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # --------------------------------------------------------------------------- oracle leg
 
-def oracle_time(inp, target_s: float = 15.0, max_seq=None):
+def oracle_time(inp, target_s: float = 15.0, max_seq=None, q_verify=None):
     """Time the float64 oracle (as it stands, all host cores) on a bounded
     sample of whole sequences of the workload, about target_s of CPU time: a
     prefix of the sequences when the workload is larger, or the whole workload
-    repeated when it is smaller.  Returns (GB/s, seconds, threads, description)."""
+    repeated when it is smaller.  q_verify (bf16 [b, n, H, d]): time the
+    oracle's verification decode of those query tokens instead.
+    Returns (GB/s, seconds, threads, description)."""
     import numpy as np
 
     import oracle
 
     w = inp.workload
-    q = inp.q.cpu()
+    q = inp.q.cpu() if q_verify is None else q_verify.cpu()
+    nq = 1 if q_verify is None else q.shape[1]
     kc, vc = inp.k_cache.cpu(), inp.v_cache.cpu()
     sl = inp.seqlens.cpu()
     pt = None if inp.page_table is None else inp.page_table.cpu()
@@ -177,9 +185,12 @@ def oracle_time(inp, target_s: float = 15.0, max_seq=None):
     lens = sl.tolist()
 
     def run(n_seq):
-        rows = np.arange(n_seq * w.H, dtype=np.int64)
+        rows = np.arange(n_seq * nq * w.H, dtype=np.int64)
         t0 = time.perf_counter()
-        oracle.gqa_decode(q, kc, vc, sl, pt, num_kv_heads=w.G, scale=w.scale, rows=rows)
+        if q_verify is None:
+            oracle.gqa_decode(q, kc, vc, sl, pt, num_kv_heads=w.G, scale=w.scale, rows=rows)
+        else:
+            oracle.gqa_decode_verify(q, kc, vc, sl, pt, num_kv_heads=w.G, scale=w.scale, rows=rows)
         return time.perf_counter() - t0
 
     probe = run(1)
@@ -193,8 +204,8 @@ def oracle_time(inp, target_s: float = 15.0, max_seq=None):
         for _ in range(reps - 1):
             dt += run(n)
     kv = accounting.kv_bytes_per_step(w.G, w.d, lens[:n])
-    desc = "%d of %d sequences (all %d heads each) of the workload, %.3g GB of KV, %d run(s)" % (
-        n, w.b, w.H, kv / 1e9, reps)
+    desc = "%d of %d sequences (all %d heads%s each) of the workload, %.3g GB of KV, %d run(s)" % (
+        n, w.b, w.H, "" if nq == 1 else " x %d query tokens" % nq, kv / 1e9, reps)
     return reps * kv / dt / 1e9, dt, threads, desc
 
 
@@ -205,14 +216,15 @@ def reference_arm(args):
         return 0
     w = WORKLOADS[args.workload]
     inp = make_inputs(w, device="cpu")
+    qv = draw_verify_q(w, args.query_tokens) if args.query_tokens > 1 else None
     kv_step = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
     # every step a bounded sample: a whole-sequence slice sized so the run ends in minutes
     budget = min(15.0, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        oracle_time(inp, target_s=budget)
+        oracle_time(inp, target_s=budget, q_verify=qv)
     vals, times, desc, threads = [], [], "", 0
     for _ in range(args.steps):
-        gbs, dt, threads, desc = oracle_time(inp, target_s=budget)
+        gbs, dt, threads, desc = oracle_time(inp, target_s=budget, q_verify=qv)
         vals.append(gbs)
         times.append(dt)
     value = statistics.median(vals)
@@ -221,7 +233,7 @@ def reference_arm(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_dict(w, inp, None),
+        "data": "synthetic", "config": config_dict(w, inp, None, args.query_tokens),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": "each step: " + desc},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -250,7 +262,7 @@ class L2Flush:
         self.sink = self.r.sum()
 
 
-def config_dict(w, inp, split_tokens):
+def config_dict(w, inp, split_tokens, n_query=1):
     kv = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
     if split_tokens is None:
         decomp = "one block or cluster per (sequence, group)"
@@ -261,13 +273,19 @@ def config_dict(w, inp, split_tokens):
         decomp = "fixed splits of %d tokens (%d per sequence), %s" % (
             split_tokens, n_splits, "one block per (sequence, group), final rows" if n_splits == 1 else
             "merged in the decode kernel" if n_splits <= 8 else "combine kernel")
-    return {
-        "workload": w.name, "b": w.b, "H": w.H, "G": w.G, "d": w.d, "m": w.m,
+    cfg = {
+        "workload": w.name if n_query == 1 else "verification step, %d query tokens per sequence, over %s" % (
+            n_query, w.name), "b": w.b, "H": w.H, "G": w.G, "d": w.d, "m": w.m,
         "layout": "paged P=%d" % w.page_size if w.paged else "contiguous [b,G,m,d]",
         "split_tokens": split_tokens, "decomposition": decomp, "kv_bytes_per_step": kv, "seed": w.seed,
         "l2": ("inputs %.0f MiB > 126 MB L2 (no flush)" % (kv / 2 ** 20)) if kv > 2 * L2_BYTES
         else "L2 flushed between steps (2x L2 written, then 2x L2 read)",
     }
+    if n_query > 1:
+        cfg["query_tokens"] = n_query
+        cfg["rows_per_kv_group"] = n_query * w.r
+        cfg["mask"] = "query token t of n sees cached positions < len - (n - 1 - t)"
+    return cfg
 
 
 def main_gpu(args):
@@ -277,27 +295,31 @@ def main_gpu(args):
     w = WORKLOADS[args.workload]
     w = w.with_(seed=w.seed + 1000 * rank)  # each rank: its own shard of sequences
     inp = make_inputs(w, device="cuda")
+    nq = args.query_tokens
+    q = inp.q if nq == 1 else draw_verify_q(w, nq, device="cuda")
     kv_step = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
     max_seqlen = int(inp.seqlens.max())
     dims = gqa.dims_for(inp.q, inp.k_cache, inp.page_table)
     # 0: the library's choice (equal-work ranges); > 0: fixed splits of that many tokens
     split = args.split_tokens if args.split_tokens >= 0 else w.split_tokens
-    ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, max_seqlen, split)
-    out = torch.empty(inp.q.shape, dtype=torch.float32, device="cuda")
+    if nq > 1 and split == 0:
+        # verification runs fixed splits: one split per sequence
+        split = -(-max_seqlen // 256) * 256
+    if nq == 1:
+        ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, max_seqlen, split)
+    else:
+        ws = torch.empty(max(256, gqa.gqa_decode_verify_workspace_size(dims, nq, max_seqlen, split)),
+                         dtype=torch.uint8, device="cuda")
+    call = decode_call(args, inp, nq, split, max_seqlen, ws)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
     flush = L2Flush() if kv_step <= 2 * L2_BYTES else None
 
     def step():
-        if args.entry == "cluster":
-            gqa.gqa_decode(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, out=out,
-                           status=status)
-        else:
-            gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
-                                 split_tokens=split, max_seqlen=max_seqlen, workspace=ws, out=out,
-                                 status=status)
+        call(q, inp.seqlens, inp.page_table, out, status=status)
 
-    # fixed splits, at most 16 of them: one launch (the decode kernel merges
+    # fixed splits, at most 8 of them: one launch (the decode kernel merges
     # each unit's splits itself); more splits or equal-work ranges: decode
     # kernel + combine kernel
     eff_split = split if split > 0 else gqa.gqa_plan_split_tokens(dims, max_seqlen)
@@ -353,7 +375,7 @@ def main_gpu(args):
                                split_tokens=split, max_seqlen=max_seqlen, workspace=ws, out=out,
                                status=status)
 
-    kern = step if launches_per_step == 1 else decode_only
+    kern = step if (launches_per_step == 1 or nq > 1) else decode_only
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(max(args.steps, 10))]
     for a, b in evs:
@@ -366,21 +388,28 @@ def main_gpu(args):
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
     kern_ms = max_over_ranks(kern_ms, world)
     achieved = kv_step / (kern_ms * 1e-3) / 1e9
+    if nq > 1:
+        tc = nq * w.r > gqa.TC_AUTO_ROWS and w.d == 128
+        kname = "%s (verification, %d rows per KV group%s)" % (
+            "gqa_verify_tc_kernel" if tc else "gqa_decode_kernel", nq * w.r,
+            "" if launches_per_step == 1 else "; decode + combine timed together")
+    elif args.entry == "split":
+        kname = ("gqa_decode_kernel (equal-work ranges)" if eff_split == 0 else
+                 "gqa_decode_kernel (fixed splits%s)" % (", merged in-kernel" if launches_per_step == 1 else ""))
+    else:
+        kname = "gqa_decode_kernel (gqa_decode)"
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": recorded_traffic(args.workload),
-                "kernel": ("gqa_decode_kernel (equal-work ranges)" if eff_split == 0 else
-                           "gqa_decode_kernel (fixed splits%s)" % (", merged in-kernel" if launches_per_step == 1
-                                                                    else "")) if args.entry == "split"
-                else "gqa_decode_kernel (gqa_decode)", "peak_kind": hbm_kind,
+                "frac": achieved / hbm, "traffic": recorded_traffic(traffic_key(args.workload, nq)),
+                "kernel": kname, "peak_kind": hbm_kind,
                 "kernel_us": kern_ms * 1e3, "algorithmic_bytes_per_launch": kv_step}
 
     # ---- end to end through the public API with host buffers
-    e2e = e2e_leg(args, inp, split, max_seqlen, ws, kv_step, world)
+    e2e = e2e_leg(args, inp, q, call, kv_step, world)
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        gbs, dt, threads, desc = oracle_time(inp)
+        gbs, dt, threads, desc = oracle_time(inp, q_verify=None if nq == 1 else q)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": desc + "; %.1f s of CPU time" % dt}
 
@@ -389,10 +418,11 @@ def main_gpu(args):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": config_dict(w, inp, eff_split if args.entry == "split" else None),
+            "data": "synthetic",
+            "config": config_dict(w, inp, eff_split if args.entry == "split" else None, nq),
             "frac_of_peak_hbm": value / world / hbm, "peak_hbm_gbs": hbm, "peak_kind": hbm_kind,
             "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
-            "entry": "gqa_decode_split" if args.entry == "split" else "gqa_decode",
+            "entry": "gqa_decode_verify" if nq > 1 else "gqa_decode_split" if args.entry == "split" else "gqa_decode",
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(),
         }
@@ -403,7 +433,24 @@ def main_gpu(args):
     return 0
 
 
-def e2e_leg(args, inp, split, max_seqlen, ws, kv_step, world):
+def decode_call(args, inp, nq, split, max_seqlen, ws):
+    """The public call one step makes: (q, seqlens, page_table, out, status=,
+    stream=) -> None, on the resident KV cache."""
+    from kv_cache_bandwidth_b200 import gqa
+
+    def call(q, sl, pt, out, status=None, stream=None):
+        if nq > 1:
+            gqa.gqa_decode_verify(q, inp.k_cache, inp.v_cache, sl, pt, split_tokens=split, max_seqlen=max_seqlen,
+                                  workspace=ws, out=out, status=status, stream=stream)
+        elif args.entry == "cluster":
+            gqa.gqa_decode(q, inp.k_cache, inp.v_cache, sl, pt, out=out, status=status, stream=stream)
+        else:
+            gqa.gqa_decode_split(q, inp.k_cache, inp.v_cache, sl, pt, split_tokens=split, max_seqlen=max_seqlen,
+                                 workspace=ws, out=out, status=status, stream=stream)
+    return call
+
+
+def e2e_leg(args, inp, q, call, kv_step, world):
     """Same metric through the public call with host buffers: each step copies the
     step's inputs (q, lengths, page table) from pinned host memory, runs the
     decode and reads the result back into pinned host memory.  The KV cache is
@@ -414,16 +461,14 @@ def e2e_leg(args, inp, split, max_seqlen, ws, kv_step, world):
     engines) and the decode on a compute stream, so step i+1's inputs travel
     and step i-1's result returns while step i decodes.  Events order every
     buffer reuse."""
-    from kv_cache_bandwidth_b200 import gqa
-
-    h_q = inp.q.cpu().pin_memory()
+    h_q = q.cpu().pin_memory()
     h_sl = inp.seqlens.cpu().pin_memory()
     h_pt = None if inp.page_table is None else inp.page_table.cpu().pin_memory()
-    h_out = [torch.empty(inp.q.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
-    d_q = [torch.empty_like(inp.q) for _ in range(2)]
+    h_out = [torch.empty(q.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    d_q = [torch.empty_like(q) for _ in range(2)]
     d_sl = [torch.empty_like(inp.seqlens) for _ in range(2)]
     d_pt = [None if h_pt is None else torch.empty_like(inp.page_table) for _ in range(2)]
-    d_out = [torch.empty(inp.q.shape, dtype=torch.float32, device="cuda") for _ in range(2)]
+    d_out = [torch.empty(q.shape, dtype=torch.float32, device="cuda") for _ in range(2)]
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()  # noqa: E731
     in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
@@ -444,11 +489,7 @@ def e2e_leg(args, inp, split, max_seqlen, ws, kv_step, world):
         with torch.cuda.stream(s_comp):    # decode of step i (its output buffer is free once read back)
             s_comp.wait_event(in_done[k])
             s_comp.wait_event(out_done[k])
-            if args.entry == "cluster":
-                gqa.gqa_decode(d_q[k], inp.k_cache, inp.v_cache, d_sl[k], d_pt[k], out=d_out[k], stream=s_comp)
-            else:
-                gqa.gqa_decode_split(d_q[k], inp.k_cache, inp.v_cache, d_sl[k], d_pt[k], split_tokens=split,
-                                     max_seqlen=max_seqlen, workspace=ws, out=d_out[k], stream=s_comp)
+            call(d_q[k], d_sl[k], d_pt[k], d_out[k], stream=s_comp)
             comp_done[k].record(s_comp)
         with torch.cuda.stream(s_out):     # result of step i back to the host
             s_out.wait_event(comp_done[k])
@@ -488,6 +529,8 @@ def main(argv=None):
                     help="-1: the workload's own split (0 when it has none); 0: the library's "
                          "equal-work ranges; > 0: fixed splits of that many tokens")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--query-tokens", type=int, default=1,
+                    help="query tokens per sequence (> 1: a verification step through gqa_decode_verify)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

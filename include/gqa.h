@@ -96,7 +96,8 @@ extern "C" {
 #define GQA_FLAG_CONTRACT_TCGEN05 4u /* 5th-gen tensor cores (tcgen05, accumulators in tensor memory): one block
                                         takes all rows of a group (r times the query tokens, <= 128), d = 128
                                         only; split entry points (fixed splits) only.  flags == 0 picks it by
-                                        itself for more than 32 rows per group at d = 128 */
+                                        itself for more than GQA_TC_AUTO_ROWS rows per group at d = 128 */
+#define GQA_TC_AUTO_ROWS 32
 
 typedef struct gqa_dims {
     int32_t batch;             /* b: sequences, one query token each */

@@ -117,7 +117,7 @@ constexpr int kMaxQueryTokens = 64;
 // Rows per group above which the automatic choice is the tcgen05 kernel
 // (measured: with 64 and 128 rows it beats the 16-row mma.sync slices by 1.3x
 // and 2.4x; with 32 or fewer its one-thread-per-row softmax leaves lanes idle).
-constexpr int kTcAutoRows = 32;
+constexpr int kTcAutoRows = GQA_TC_AUTO_ROWS;
 
 int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1, const int32_t *group_of_head = nullptr,
                bool auto_tc = true) {

@@ -22,6 +22,7 @@ do not depend on one another's sizes:
   stream 4: pages   a random permutation of the page pool (paged workloads)
   stream 5: peaky   per (sequence, group), floor(frac * m) distinct key rows
                     multiplied by 8 (exact in bf16)
+  stream 6: q of a verification step (n query tokens per sequence), as q
 """
 from __future__ import annotations
 
@@ -31,7 +32,7 @@ from typing import Dict, List, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "Inputs", "BF16_NAN_BITS"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "draw_verify_q", "Inputs", "BF16_NAN_BITS"]
 
 BF16_NAN_BITS = 0x7FC0  # a quiet NaN in bf16
 
@@ -172,6 +173,12 @@ def make_inputs(w: Workload, device="cpu", lens: Optional[List[int]] = None,
         _poison_unused(k, v, w, seqlens, page_table)
     pt = None if page_table is None else page_table.to(device)
     return Inputs(q, k, v, seqlens.to(device), pt, w)
+
+
+def draw_verify_q(w: Workload, n_query: int, device="cpu") -> torch.Tensor:
+    """The query tokens of a verification step over the same cache: bf16
+    [b, n_query, H, d] (the last n_query cached positions are the drafts)."""
+    return _randn_bf16((w.b, n_query, w.H, w.d), w.seed, 6, device)
 
 
 def _logical_rows(w: Workload, s: int, rows: torch.Tensor, page_table) -> tuple:

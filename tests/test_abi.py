@@ -41,6 +41,7 @@ def test_binding_constants_match_header():
     text = open(HEADER).read()
     defs = dict(re.findall(r"^#define\s+(GQA_\w+)\s+(.+?)\s*$", text, flags=re.M))
     assert int(defs["GQA_MERGE_IN_KERNEL_MAX_SPLITS"]) == gqa.SERIAL_MERGE_MAX_SPLITS
+    assert int(defs["GQA_TC_AUTO_ROWS"]) == gqa.TC_AUTO_ROWS
     assert eval(defs["GQA_STATIC_WORKSPACE_BYTES"].replace("u", "")) == gqa.STATIC_WORKSPACE_BYTES
 
 
