@@ -26,8 +26,10 @@
 //     row in tensor memory, each thread half of the columns), write P to
 //     tensor memory;
 //   * warp 8: the TMA producer of the K/V ring (as in the mma.sync kernel);
-//   * warp 9: tensor-memory allocation; one thread issues the MMAs and signals
-//     their completion on mbarriers with tcgen05.commit.
+//   * warp 9: tensor-memory allocation; one thread issues the Q K^T products;
+//   * warp 10: one thread issues the P.V products.  The two issuers run
+//     concurrently (the tensor pipe overlaps their products) and signal
+//     completion on mbarriers with tcgen05.commit.
 // S and P share three tensor-memory buffers: the scores of tiles t+1 and t+2
 // are computed and the softmax of t+1 runs while the P.V of tile t is on the
 // tensor cores; a buffer takes new scores once the P.V that read it is done.
@@ -60,7 +62,7 @@ struct TcTile {
   static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[kStages], abort, merge here
   static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * (kStages + 3);
   static constexpr int kSoftmaxWarps = 8;
-  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
   static constexpr uint32_t kOCol = 256;               // O: columns 256 .. 383
   static constexpr uint32_t kTmemCols = 512;           // S, then P over it (kSP x 64 columns) + O
   static_assert(kSP * kT <= static_cast<int>(kOCol), "S/P buffers below O");
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     *merge_here = 0;
     fence_mbarrier_init();
   }
-  constexpr int kProducerWarp = TT::kSoftmaxWarps, kMmaWarp = TT::kSoftmaxWarps + 1;
+  constexpr int kProducerWarp = TT::kSoftmaxWarps, kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
   if (warp == kMmaWarp) {
     tc_alloc(smem_addr(const_cast<uint32_t *>(tmem_slot)), TT::kTmemCols);
     tc_relinquish();
@@ -242,53 +244,62 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     // ============================================================ producer
     tc_produce<PAGED>(&tm_k, &tm_v, p, pc, sbase, full0, empty0, tile_bad, abort_flag, lane);
   } else if (warp == kMmaWarp) {
-    // ============================================================ MMA issuer
-    // (the tensor pipe runs the products in issue order: the scores of tile
-    // t go ahead of the P.V of tile t-1, so that the softmax of t can start
-    // while that P.V runs)
+    // ============================================================ Q K^T issuer
     if (lane == 0) {
       constexpr uint32_t kIdescQK = tc_idesc_bf16(128, 64, false);
-      constexpr uint32_t kIdescPV = tc_idesc_bf16(128, 128, true);
-      const uint32_t q_sm = sbase + TT::kQOff;
+      // Q's descriptors are the same for every tile; a K-step adds to the
+      // start-address field (addresses stay below 256 KB: no carry)
+      uint64_t qd[D / 16];
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        qd[ks] = tc_smem_desc(sbase + TT::kQOff + (ks >> 2) * TT::kQHalf + (ks & 3) * 32, 16, 1024);
       bool ok = true;
-      for (int t = 0; t <= n_tiles && ok; ++t) {
-        if (t < n_tiles) {
-          // ---- S[t % SP] = Q K_t^T
-          const int st = t % ST;
-          ok = mbar_wait(full0 + 8 * st, (t / ST) & 1);
-          // buffer t % SP holds P of tile t-SP until its P.V is done
-          if (ok && t >= SP) ok = mbar_wait(pv_done0 + 8 * (t % SP), ((t / SP) - 1) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kt = sbase + st * TT::kStageBytes;
+      for (int t = 0; t < n_tiles; ++t) {
+        // ---- S[t % SP] = Q K_t^T once K_t has landed and the buffer's last P.V is done
+        const int st = t % ST;
+        ok = mbar_wait(full0 + 8 * st, (t / ST) & 1);
+        if (ok && t >= SP) ok = mbar_wait(pv_done0 + 8 * (t % SP), ((t / SP) - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t kd = tc_smem_desc(sbase + st * TT::kStageBytes, 16, 1024);
+        const uint32_t d = tmem + (t % SP) * 64;
+        tc_mma(d, qd[0], kd, kIdescQK, 0u);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t koff = (ks >> 2) * TT::kHalf + (ks & 3) * 32;
-            const uint32_t qoff = (ks >> 2) * TT::kQHalf + (ks & 3) * 32;
-            tc_mma(tmem + (t % SP) * 64, tc_smem_desc(q_sm + qoff, 16, 1024), tc_smem_desc(kt + koff, 16, 1024),
-                   kIdescQK, ks > 0 ? 1u : 0u);
-          }
-          tc_commit(s_full0 + 8 * (t % SP));
-        }
-        if (t >= 1) {
-          // ---- O += P_{t-1} V_{t-1} (high part and residual of P, from tensor memory)
-          const int u = t - 1, st = u % ST;
-          ok = mbar_wait(p_full0 + 8 * (u % SP), (u / SP) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t vt = sbase + st * TT::kStageBytes + TT::kTileBytes;
+        for (int ks = 1; ks < D / 16; ++ks)
+          tc_mma(d, qd[ks], kd + ((static_cast<uint32_t>((ks >> 2) * TT::kHalf + (ks & 3) * 32)) >> 4), kIdescQK, 1u);
+        tc_commit(s_full0 + 8 * (t % SP));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (p.status) atomicOr(p.status, kStatusTimeout);
+      }
+    }
+  } else if (warp == kPvWarp) {
+    // ============================================================ P.V issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescPV = tc_idesc_bf16(128, 128, true);
+      bool ok = true;
+      for (int u = 0; u < n_tiles; ++u) {
+        // ---- O += P_u V_u (high part and residual of P, from tensor memory)
+        const int st = u % ST;
+        ok = mbar_wait(p_full0 + 8 * (u % SP), (u / SP) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t vd = tc_smem_desc(sbase + st * TT::kStageBytes + TT::kTileBytes, TT::kHalf, 1024);
+        const uint32_t pb = tmem + (u % SP) * 64;
 #pragma unroll
-          for (int ks = 0; ks < T / 16; ++ks) {
-            // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of
-            // the buffer, the residual 16 columns further
-            const uint64_t vdesc = tc_smem_desc(vt + ks * 16 * 128, TT::kHalf, 1024);
-            const uint32_t pa = tmem + (u % SP) * 64 + 32 * (ks >> 1) + 8 * (ks & 1);
-            tc_mma_ts(tmem + TT::kOCol, pa, vdesc, kIdescPV, (u > 0 || ks > 0) ? 1u : 0u);
-            tc_mma_ts(tmem + TT::kOCol, pa + 16, vdesc, kIdescPV, 1u);
-          }
-          tc_commit(empty0 + 8 * st);  // the stage's K and V are no longer read
-          tc_commit(pv_done0 + 8 * (u % SP));
+        for (int ks = 0; ks < T / 16; ++ks) {
+          // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of
+          // the buffer, the residual 16 columns further
+          const uint64_t vdk = vd + ((ks * 16 * 128) >> 4);
+          const uint32_t pa = pb + 32 * (ks >> 1) + 8 * (ks & 1);
+          tc_mma_ts(tmem + TT::kOCol, pa, vdk, kIdescPV, (u > 0 || ks > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + TT::kOCol, pa + 16, vdk, kIdescPV, 1u);
         }
+        // K_u was read by the scores of tile u, done before its P existed; V_u
+        // and P_u by these products
+        tc_commit(empty0 + 8 * st);
+        tc_commit(pv_done0 + 8 * (u % SP));
       }
       if (!ok) {
         *abort_flag = 1;
