@@ -13,7 +13,8 @@
 //   O[rows, 128]       += P[rows, 64] . V_tile[64, 128]            (M = 128, N = 128)
 //
 // Rows are padded to M = 128; P enters as a bf16 high part and a bf16
-// residual (two MMAs), as in the mma.sync kernel.  P is written to tensor
+// residual (two MMAs), as in the mma.sync kernel, here both truncated (byte
+// permutes, no conversions: P to within 2^-14 relative).  P is written to tensor
 // memory over its own scores (each thread over the columns it has read) and
 // the P.V product takes its A operand from there, which leaves shared memory
 // to a 5-stage K/V ring.  Warp roles:
@@ -315,8 +316,10 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     const bool valid = r < pc.nh;
     const bool warp_active = (warp % 4) * 32 < pc.nh;
     // the positions this row sees: with several query tokens per sequence,
-    // query token t sees the cache up to and including itself
-    const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + r) / p.r)) : 0;
+    // query token t sees the cache up to and including itself (a padding row,
+    // q = 0, sees the whole piece: its scores are 0, its result unused, and it
+    // keeps to the unmasked path of its warp)
+    const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + r) / p.r)) : pc.t_end;
     const uint32_t lane_tmem = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     float *xmax = reinterpret_cast<float *>(smem + TT::kXOff);  // [tile % SP][half][row]
     float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);  // [half][row]
@@ -347,8 +350,15 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         }
       }
       float x[32];
+      const int tb = t0 + half * 32;  // this thread's first token of the tile
+      if (tb + 32 <= lim) {
+        // all of them visible (every tile but the row's last)
 #pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] = (t0 + half * 32 + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
+        for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(sv[j]) * sl;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
+      }
       float mx;
       {
         float m8[8];  // a tree, not a chain of 32 dependent steps
@@ -403,7 +413,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
           l_run += p0 + p1;
-          split_bf16x2(p0, p1, hi[e], lo[e]);
+          split_bf16x2_rz(p0, p1, hi[e], lo[e]);
         }
         tc_st16(lane_tmem + b * 64 + half * 32, hi);
         tc_st16(lane_tmem + b * 64 + half * 32 + 16, lo);

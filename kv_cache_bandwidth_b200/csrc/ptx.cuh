@@ -153,6 +153,17 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uin
   lo = pack_bf16(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
 }
 
+// The same split with both parts truncated (the upper 16 bits of each float,
+// byte permutes instead of conversions): hi.a has 8 significant bits of a, so
+// |a - hi.a| < 2^-7 |a| is exact in fp32 and its truncation loses < 2^-7 of
+// it; the pair represents a to within 2^-14 relative.
+__device__ __forceinline__ void split_bf16x2_rz(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+  hi = __byte_perm(ua, ub, 0x7632);  // a's upper half low, b's upper half high
+  const float ra = a - __uint_as_float(ua & 0xffff0000u), rb = b - __uint_as_float(ub & 0xffff0000u);
+  lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
+}
+
 // ---------------------------------------------------------------- PDL
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
