@@ -97,7 +97,8 @@ extern "C" {
                                         takes all rows of a group (r times the query tokens, <= 128), d = 128
                                         only; split entry points (fixed splits) only.  flags == 0 picks it by
                                         itself for more than GQA_TC_AUTO_ROWS rows per group at d = 128 */
-#define GQA_TC_AUTO_ROWS 32
+/* Above this many rows per group the mma.sync kernel would need a second 16-row slice. */
+#define GQA_TC_AUTO_ROWS 16
 
 typedef struct gqa_dims {
     int32_t batch;             /* b: sequences, one query token each */

@@ -440,7 +440,7 @@ def gqa_split_combine(seqlens, out, dims: Dims, *, split_tokens: int, max_seqlen
 
 STATIC_WORKSPACE_BYTES = 8 << 20  # GQA_STATIC_WORKSPACE_BYTES
 SERIAL_MERGE_MAX_SPLITS = 8       # GQA_MERGE_IN_KERNEL_MAX_SPLITS
-TC_AUTO_ROWS = 32                 # GQA_TC_AUTO_ROWS: flags == 0 takes tcgen05 above this many rows per group
+TC_AUTO_ROWS = 16                 # GQA_TC_AUTO_ROWS: flags == 0 takes tcgen05 above this many rows per group
 
 
 def gqa_decode_split_static(q, k_cache, v_cache, seqlens, page_table=None, *, split_tokens: int = 0,
