@@ -219,7 +219,7 @@ def reference_arm(args):
     qv = draw_verify_q(w, args.query_tokens) if args.query_tokens > 1 else None
     kv_step = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
     # every step a bounded sample: a whole-sequence slice sized so the run ends in minutes
-    budget = min(15.0, 120.0 / max(1, args.steps + args.warmup))
+    budget = args.oracle_seconds if args.oracle_seconds > 0 else min(15.0, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_time(inp, target_s=budget, q_verify=qv)
     vals, times, desc, threads = [], [], "", 0
@@ -409,7 +409,8 @@ def main_gpu(args):
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        gbs, dt, threads, desc = oracle_time(inp, q_verify=None if nq == 1 else q)
+        gbs, dt, threads, desc = oracle_time(inp, target_s=args.oracle_seconds if args.oracle_seconds > 0 else 15.0,
+                                             q_verify=None if nq == 1 else q)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": desc + "; %.1f s of CPU time" % dt}
 
@@ -529,6 +530,9 @@ def main(argv=None):
                     help="-1: the workload's own split (0 when it has none); 0: the library's "
                          "equal-work ranges; > 0: fixed splits of that many tokens")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-seconds", type=float, default=0.0,
+                    help="CPU seconds of oracle work per timed sample (0: 15 s for cpu_baseline; the reference "
+                         "arm spreads about two minutes over its steps)")
     ap.add_argument("--query-tokens", type=int, default=1,
                     help="query tokens per sequence (> 1: a verification step through gqa_decode_verify)")
     args = ap.parse_args(argv)
