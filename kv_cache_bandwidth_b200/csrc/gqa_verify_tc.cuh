@@ -19,13 +19,14 @@
 // the P.V product takes its A operand from there, which leaves shared memory
 // to a 5-stage K/V ring.  Warp roles:
 //   * warps 0-7: two threads per row (warps w and w+4 share the tensor-memory
-//     lanes of rows 32(w%4) ..), each taking 32 of a tile's 64 tokens.  Each
-//     tile: read the half-row of scores from tensor memory, mask (the row's
-//     own causal limit among the drafts), agree with the partner thread on the
-//     row's maximum through shared memory, online softmax in base 2 with the
-//     lazy rescale (a row whose maximum moves by more than 2^8 rescales its O
-//     row in tensor memory, each thread half of the columns), write P to
-//     tensor memory;
+//     lanes of rows 32(w%4) ..), each taking 32 of a tile's 64 tokens with a
+//     softmax state of its own: its running base and sum, and its own O in
+//     tensor memory (the P.V of its tokens accumulates there).  Each tile:
+//     read the half-row of scores from tensor memory, mask (the row's own
+//     causal limit among the drafts), online softmax in base 2 with the lazy
+//     rescale (a half whose maximum moves by more than 2^8 rescales its O row
+//     in tensor memory), write P to tensor memory.  The two halves of a row
+//     meet once, at the end, as two partial states merged exactly;
 //   * warp 8: the TMA producer of the K/V ring (as in the mma.sync kernel);
 //   * warp 9: tensor-memory allocation; one thread issues the Q K^T products;
 //   * warp 10: one thread issues the P.V products.  The two issuers run
@@ -56,17 +57,17 @@ struct TcTile {
   static constexpr int kQHalf = kM * 128;
   static constexpr int kBarOff = kQOff + 2 * kQHalf;
   static constexpr int kSP = 3;                        // S/P buffers in tensor memory
-  // full[kStages], empty[kStages], s_full[kSP], p_full[kSP], pv_done[kSP], x_full[kSP]
-  static constexpr int kNumBars = 2 * kStages + 4 * kSP;
-  static constexpr int kXOff = kBarOff + 8 * kNumBars;  // row maxima of each half row: [kSP tiles][2][kM] floats
-  static constexpr int kLOff = kXOff + 4 * kSP * 2 * kM;  // the halves' sums at the end: [2][kM] floats
+  // full[kStages], empty[kStages], s_full[kSP], p_full[kSP], pv_done[kSP]
+  static constexpr int kNumBars = 2 * kStages + 3 * kSP;
+  static constexpr int kXOff = kBarOff + 8 * kNumBars;  // the halves' bases at the end: [2][kM] floats
+  static constexpr int kLOff = kXOff + 4 * 2 * kM;      // the halves' sums at the end: [2][kM] floats
   static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[kStages], abort, merge here
   static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * (kStages + 3);
   static constexpr int kSoftmaxWarps = 8;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
-  static constexpr uint32_t kOCol = 256;               // O: columns 256 .. 383
-  static constexpr uint32_t kTmemCols = 512;           // S, then P over it (kSP x 64 columns) + O
-  static_assert(kSP * kT <= static_cast<int>(kOCol), "S/P buffers below O");
+  static constexpr uint32_t kOCol = 256;               // O of the first halves: 256 .. 383, second: 384 .. 511
+  static constexpr uint32_t kTmemCols = 512;           // S, then P over it (kSP x 64 columns) + 2 O
+  static_assert(kSP * kT <= static_cast<int>(kOCol) && kOCol + 2 * kD <= kTmemCols, "tensor-memory columns");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -173,7 +174,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   const uint32_t full0 = bars, empty0 = bars + 8 * ST;
   constexpr int SP = TT::kSP;
   const uint32_t s_full0 = bars + 16 * ST;
-  const uint32_t p_full0 = s_full0 + 8 * SP, pv_done0 = p_full0 + 8 * SP, x_full0 = pv_done0 + 8 * SP;
+  const uint32_t p_full0 = s_full0 + 8 * SP, pv_done0 = p_full0 + 8 * SP;
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
   volatile int *abort_flag = tile_bad + ST;
@@ -211,7 +212,6 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       mbar_init(s_full0 + 8 * i, 1);
       mbar_init(p_full0 + 8 * i, TT::kSoftmaxWarps);  // one arrival per softmax warp
       mbar_init(pv_done0 + 8 * i, 1);
-      mbar_init(x_full0 + 8 * i, TT::kSoftmaxWarps);
     }
     *abort_flag = 0;
     *merge_here = 0;
@@ -291,11 +291,13 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < T / 16; ++ks) {
           // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of
-          // the buffer, the residual 16 columns further
+          // the buffer, the residual 16 columns further; into the O of the
+          // half of the row that owns them
           const uint64_t vdk = vd + ((ks * 16 * 128) >> 4);
           const uint32_t pa = pb + 32 * (ks >> 1) + 8 * (ks & 1);
-          tc_mma_ts(tmem + TT::kOCol, pa, vdk, kIdescPV, (u > 0 || ks > 0) ? 1u : 0u);
-          tc_mma_ts(tmem + TT::kOCol, pa + 16, vdk, kIdescPV, 1u);
+          const uint32_t od = tmem + TT::kOCol + D * (ks >> 1);
+          tc_mma_ts(od, pa, vdk, kIdescPV, (u > 0 || (ks & 1)) ? 1u : 0u);
+          tc_mma_ts(od, pa + 16, vdk, kIdescPV, 1u);
         }
         // K_u was read by the scores of tile u, done before its P existed; V_u
         // and P_u by these products
@@ -321,10 +323,10 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     // keeps to the unmasked path of its warp)
     const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + r) / p.r)) : pc.t_end;
     const uint32_t lane_tmem = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-    float *xmax = reinterpret_cast<float *>(smem + TT::kXOff);  // [tile % SP][half][row]
-    float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);  // [half][row]
+    float *mbase = reinterpret_cast<float *>(smem + TT::kXOff);  // [half][row]
+    float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);   // [half][row]
     const float sl = p.scale_log2;
-    float m_run = kNegInf, l_run = 0.f;  // the row's base (shared by the pair) and this half's sum
+    float m_run = kNegInf, l_run = 0.f;  // this half's base and sum
     int bad = 0;
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
@@ -366,17 +368,6 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         for (int k = 0; k < 8; ++k) m8[k] = fmaxf(fmaxf(x[4 * k], x[4 * k + 1]), fmaxf(x[4 * k + 2], x[4 * k + 3]));
         mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       }
-      // the row's maximum over both halves, exchanged through shared memory
-      // (every softmax warp takes part; the buffer of tile t is written again
-      // at tile t+SP, which no warp reaches before all have passed the P
-      // hand-over of tile t: the scores of t+SP come after the P.V of t+1
-      // is issued)
-      xmax[(b * 2 + half) * 128 + r] = mx;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(x_full0 + 8 * b);
-      ok = __all_sync(0xffffffffu, mbar_wait(x_full0 + 8 * b, (t / SP) & 1));
-      if (!ok) break;
-      mx = fmaxf(mx, xmax[(b * 2 + (half ^ 1)) * 128 + r]);
       if (warp_active) {
         // lazy rescale: only when a score passes the base by more than 2^8
         const bool need = mx > m_run + 8.f;
@@ -385,18 +376,18 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
           const float alpha = need ? ((m_run == kNegInf) ? 0.f : ex2(m_run - mn)) : 1.f;
           l_run *= alpha;
           if (t > 0) {
-            // O holds tiles 0 .. t-1: rescale this half of the row once their MMAs are done
+            // this half's O holds tiles 0 .. t-1: rescale it once their MMAs are done
             ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((t - 1) % SP), ((t - 1) / SP) & 1));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
               uint32_t ov[32];
-              tc_ld32(lane_tmem + TT::kOCol + half * 64 + c * 32, ov);
+              tc_ld32(lane_tmem + TT::kOCol + half * D + c * 32, ov);
               tc_wait_ld();
 #pragma unroll
               for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-              tc_st32(lane_tmem + TT::kOCol + half * 64 + c * 32, ov);
+              tc_st32(lane_tmem + TT::kOCol + half * D + c * 32, ov);
             }
             tc_wait_st();
             tc_fence_before();
@@ -436,41 +427,44 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     const bool done =
         ok && __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((n_tiles - 1) % SP), ((n_tiles - 1) / SP) & 1));
     tc_fence_after();
+    // the row's two partial states, merged exactly: M = max(m0, m1), weights
+    // 2^(m_h - M) (0 for a half that saw no position)
+    mbase[half * 128 + r] = m_run;
     lsum[half * 128 + r] = l_run;
     named_barrier(1, kSM);
-    const float l_row = lsum[r] + lsum[128 + r];
+    const float m0 = mbase[r], m1 = mbase[128 + r];
+    const float m_row = fmaxf(m0, m1);
+    const float w0 = (m0 == kNegInf) ? 0.f : ex2(m0 - m_row), w1 = (m1 == kNegInf) ? 0.f : ex2(m1 - m_row);
+    const float l_row = lsum[r] * w0 + lsum[128 + r] * w1;
     const bool final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
     const size_t row = valid ? row_of(p, pc.s, pc.g, pc.h0 + r) : 0;
     const size_t ps = row * p.num_splits + pc.k;
+    const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
+    const float s0 = final_row ? w0 * inv : w0, s1 = final_row ? w1 * inv : w1;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      uint32_t ov[32];
-      const int col = half * 64 + c * 32;
-      tc_ld32(lane_tmem + TT::kOCol + col, ov);
+      uint32_t oa[32], ob[32];
+      const int col = half * 64 + c * 32;  // this thread writes columns [64 half, 64 half + 64)
+      tc_ld32(lane_tmem + TT::kOCol + col, oa);
+      tc_ld32(lane_tmem + TT::kOCol + D + col, ob);
       tc_wait_ld();
       if (valid) {
-        if (final_row) {
-          const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
-          float4 *dst = reinterpret_cast<float4 *>(p.out + row * D + col);
+        float4 *dst = reinterpret_cast<float4 *>((final_row ? p.out + row * D : p.part_o + ps * D) + col);
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(__uint_as_float(ov[4 * j]) * inv, __uint_as_float(ov[4 * j + 1]) * inv,
-                                 __uint_as_float(ov[4 * j + 2]) * inv, __uint_as_float(ov[4 * j + 3]) * inv);
-        } else {
-          float4 *dst = reinterpret_cast<float4 *>(p.part_o + ps * D + col);
+        for (int j = 0; j < 8; ++j) {
+          float v[4];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(__uint_as_float(ov[4 * j]), __uint_as_float(ov[4 * j + 1]),
-                                 __uint_as_float(ov[4 * j + 2]), __uint_as_float(ov[4 * j + 3]));
+          for (int e = 0; e < 4; ++e) v[e] = __uint_as_float(oa[4 * j + e]) * s0 + __uint_as_float(ob[4 * j + e]) * s1;
+          dst[j] = make_float4(v[0], v[1], v[2], v[3]);
         }
       }
     }
     if (valid && half == 0) {
       if (final_row) {
-        if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_run, l_row);
+        if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_row, l_row);
         if (p.part_l) p.part_l[row * p.num_splits] = kLFinal;
       } else {
-        p.part_m[ps] = m_run;
+        p.part_m[ps] = m_row;
         p.part_l[ps] = bad ? kLBadPage : l_row;
       }
     }
