@@ -53,10 +53,20 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# The sources each profiled kernel is built from (its own header, the helpers
+# it includes and the launch code); a committed ncu record stays valid while
+# these hash the same.
+KERNEL_SOURCES = {
+    "gqa_decode_kernel": ("gqa_api.cu", "gqa_kernels.cuh", "ptx.cuh"),
+    "gqa_verify_tc_kernel": ("gqa_api.cu", "gqa_kernels.cuh", "gqa_verify_tc.cuh", "ptx.cuh", "tc05.cuh"),
+}
+
+
+def kernel_source_hash(files=None) -> str:
+    """sha256 (16 hex digits) over the named csrc files (default: all of them)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kv_cache_bandwidth_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -74,7 +84,7 @@ def recorded_traffic(workload: str):
         with open(path) as f:
             d = json.load(f)
         e = d.get(workload)
-        if e and e.get("kernel_hash") == kernel_source_hash():
+        if e and e.get("kernel_hash") == kernel_source_hash(KERNEL_SOURCES.get(e.get("kernel_name"))):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
