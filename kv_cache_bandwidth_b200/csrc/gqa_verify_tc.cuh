@@ -14,10 +14,10 @@
 //
 // Rows are padded to M = 128; P enters as a bf16 high part and a bf16
 // residual (two MMAs), as in the mma.sync kernel, here both truncated (byte
-// permutes, no conversions: P to within 2^-14 relative).  P is written to tensor
-// memory over its own scores (each thread over the columns it has read) and
-// the P.V product takes its A operand from there, which leaves shared memory
-// to a 5-stage K/V ring.  Warp roles:
+// permutes, no conversions: P to within 2^-14 relative).  P is written to
+// tensor memory over its own scores (each thread over the columns it has read)
+// and the P.V product takes its A operand from there, which leaves shared
+// memory to a 5-stage K/V ring.  Warp roles:
 //   * warps 0-7: two threads per row (warps w and w+4 share the tensor-memory
 //     lanes of rows 32(w%4) ..), each taking 32 of a tile's 64 tokens with a
 //     softmax state of its own: its running base and sum, and its own O in
@@ -217,7 +217,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     *merge_here = 0;
     fence_mbarrier_init();
   }
-  constexpr int kProducerWarp = TT::kSoftmaxWarps, kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
+  constexpr int kProducerWarp = TT::kSoftmaxWarps;  // then the Q K^T issuer (allocates), the P.V issuer
+  constexpr int kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
   if (warp == kMmaWarp) {
     tc_alloc(smem_addr(const_cast<uint32_t *>(tmem_slot)), TT::kTmemCols);
     tc_relinquish();
@@ -411,9 +412,9 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         tc_wait_st();
       }
       // (p_full is one barrier per P buffer: a warp reaches tile t+SP only
-      // after s_full of t+SP, i.e. after the MMA thread issued the P.V of
-      // tile t, so its next arrival on the same barrier cannot fall into tile
-      // t's phase)
+      // after s_full of t+SP, and the scores of t+SP are issued only once the
+      // P.V of tile t is done, so its next arrival on the same barrier cannot
+      // fall into tile t's phase)
       tc_fence_before();
       if (valid_rows < T) fence_proxy_async_smem();  // the zeroed V rows, for the tensor core
       __syncwarp();
