@@ -1,0 +1,57 @@
+"""bench.py host logic (CPU only): the sources each profiled kernel is built
+from, the rule that a committed ncu traffic record counts only while those
+sources hash the same, and the verification fields of the config."""
+import json
+import os
+
+import bench
+from kv_cache_bandwidth_b200.workloads import WORKLOADS, make_inputs
+
+CSRC = os.path.join(bench.ROOT, "kv_cache_bandwidth_b200", "csrc")
+
+
+def test_kernel_sources_exist():
+    for kernel, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            assert os.path.isfile(os.path.join(CSRC, f)), (kernel, f)
+
+
+def test_every_record_names_its_kernel_and_summary():
+    with open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")) as f:
+        records = json.load(f)
+    for key, e in records.items():
+        assert e["kernel_name"] in bench.KERNEL_SOURCES, key
+        assert list(e["sources"]) == list(bench.KERNEL_SOURCES[e["kernel_name"]]), key
+        assert os.path.isfile(os.path.join(bench.ROOT, e["summary"])), key
+        assert e["dram_bytes_per_launch"] > 0
+
+
+def test_traffic_record_follows_its_sources(tmp_path, monkeypatch):
+    pkg = tmp_path / "kv_cache_bandwidth_b200"
+    pkg.mkdir()
+    os.symlink(CSRC, pkg / "csrc")
+    (tmp_path / "profiles").mkdir()
+    files = bench.KERNEL_SOURCES["gqa_decode_kernel"]
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    good = bench.kernel_source_hash(files)
+    records = {"w_ok": {"kernel_name": "gqa_decode_kernel", "kernel_hash": good, "dram_bytes_per_launch": 123.0},
+               "w_stale": {"kernel_name": "gqa_decode_kernel", "kernel_hash": "0" * 16,
+                           "dram_bytes_per_launch": 456.0}}
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(records))
+    assert bench.recorded_traffic("w_ok") == 123.0
+    assert bench.recorded_traffic("w_stale") is None
+    assert bench.recorded_traffic("absent") is None
+    # the hash covers exactly the named files: another kernel's sources give another hash
+    assert bench.kernel_source_hash(bench.KERNEL_SOURCES["gqa_verify_tc_kernel"]) != good
+
+
+def test_traffic_keys_and_verification_config():
+    assert bench.traffic_key("llama70b") == "llama70b"
+    assert bench.traffic_key("llama70b", 8) == "llama70b_verify8"
+    w = WORKLOADS["tiny"]
+    inp = make_inputs(w)
+    c1 = bench.config_dict(w, inp, 128)
+    assert "query_tokens" not in c1 and c1["workload"] == w.name
+    c4 = bench.config_dict(w, inp, 128, 4)
+    assert c4["query_tokens"] == 4 and c4["rows_per_kv_group"] == 4 * w.r
+    assert c4["kv_bytes_per_step"] == c1["kv_bytes_per_step"]
