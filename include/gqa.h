@@ -250,7 +250,10 @@ int gqa_decode_split_lse(const void *q, const void *k_cache, const void *v_cache
  *     j < seqlens[s] - (n_query - 1 - t),
  * the end-aligned mask of a causal decoder.  For each KV group, the n_query * r
  * (token, head) pairs form the group's rows and share each K/V tile read from
- * HBM, so the cache is read once per step for all drafts.
+ * HBM: with up to 16 rows per group (the mma.sync kernel), or up to 128 at
+ * d = 128 (the tcgen05 kernel, taken by itself above GQA_TC_AUTO_ROWS rows),
+ * the cache is read once per step for all drafts; with more rows, the
+ * mma.sync kernel reads it once per 16-row slice.
  *
  * q: bf16 [b, n_query, H, d]; out: fp32 [b, n_query, H, d]; lse: fp32
  * [b, n_query, H] or NULL (the natural-log normaliser of each row, as in
