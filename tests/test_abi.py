@@ -244,3 +244,21 @@ def test_kv_append_argument_checks(lib):
              None, None) == -5
     assert f(A, A, A, A, A, A, ctypes.byref(_dims(page_size=16, num_pages=0, max_pages_per_seq=2)),
              None, None) == -6
+
+
+def test_tcgen05_flag_checks(lib):
+    """The tcgen05 contraction is rejected on the host where it does not
+    apply: d = 64, more than 128 rows per group, the cluster entry point, or
+    together with another contraction flag."""
+    tc = gqa.FLAG_CONTRACT_TCGEN05
+    d64 = _dims(head_dim=64, flags=tc)
+    assert lib.gqa_decode_split(FAKE, FAKE, FAKE, FAKE, None, FAKE, ctypes.byref(d64), 0.125, None, 128, 256,
+                                FAKE, 1 << 20, None) == -4
+    d128 = _dims(head_dim=128, num_heads=16, num_kv_heads=2, flags=tc)   # r = 8
+    # 17 query tokens x 8 heads = 136 rows per group > 128
+    assert lib.gqa_decode_verify(FAKE, FAKE, FAKE, FAKE, None, FAKE, None, ctypes.byref(d128), 17, 0.125, None,
+                                 128, 256, FAKE, 1 << 24, None) == -3
+    assert _decode(lib, _dims(head_dim=128, flags=tc)) == -6                # no cluster variant
+    assert _decode(lib, _dims(head_dim=128, flags=tc | gqa.FLAG_CONTRACT_MMA)) == -6
+    # 16 tokens x 8 heads = 128 rows fit: the workspace size is defined
+    assert lib.gqa_decode_verify_workspace_size(ctypes.byref(d128), 16, 256, 128) > 0
