@@ -3,14 +3,20 @@
 
 One step = one decode step of the whole path for one batch of sequences: the
 split-KV decode kernel (group mapping, page-table translation, K/V tile loads,
-q.k scores, online softmax, p.V) and the combine kernel that merges the splits
-and normalises.  The inputs are resident in HBM when the timed region starts.
+q.k scores, online softmax, p.V) and, where the decomposition needs one, the
+combine kernel that merges the splits and normalises.  The inputs are resident
+in HBM when the timed region starts.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama70b]
-    python bench.py --query-tokens 8 ...        # a verification step: 8 query tokens per sequence
-    python bench.py --impl reference ...        # the float64 CPU oracle instead
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ragged]
+    python bench.py --query-tokens 8 --workload llama70b   # a verification step: 8 query tokens per sequence
+    python bench.py --impl reference ...                    # the float64 CPU oracle instead
 
-Prints one JSON line (rank 0).  Under torchrun every rank runs its own shard
+Prints one JSON line (rank 0).  The headline is the workload named by
+--workload (default: the ragged paged batch, the largest single-GPU
+configuration); ``per_config`` holds the same measurement for every workload
+(tiny, Llama-2-70B layer, ragged, long-context b=1 and b=4, the group-ratio
+sweep G = 1, 2, 4, 8, 32) and two verification steps, taken in the same
+process at the same step count.  Under torchrun every rank runs its own shard
 of sequences of the same shape (weak scaling, no collective on the data path);
 the time is the maximum over ranks.
 """
@@ -20,7 +26,6 @@ import argparse
 import datetime
 import hashlib
 import json
-import math
 import os
 import statistics
 import sys
@@ -39,6 +44,13 @@ METRIC = "GQA decode µs/step and KV-cache HBM GB/s as % of B200 peak (1 GPU)"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
+# The workloads of per_config, and the verification steps measured beside them.
+PER_CONFIG = ["tiny", "llama70b", "ragged", "long1", "long4", "sweep_g1", "sweep_g2", "sweep_g4", "sweep_g8",
+              "sweep_g32"]
+PER_CONFIG_VERIFY = [("llama70b", 8), ("llama70b", 16)]
+# Copies of a cache that fits in L2 that the steps rotate over (at most): the
+# other copies' bytes between two reads of one copy must exceed twice the L2.
+MAX_ROTATE_COPIES = 16
 
 
 # --------------------------------------------------------------------------- helpers
@@ -91,6 +103,32 @@ def recorded_traffic(workload: str):
     return None
 
 
+def l2_plan(kv_bytes: int):
+    """How steps of a workload are kept from reading L2-resident data:
+    ("resident", 1) when the KV bytes exceed three times the L2 (each step
+    streams the cache through L2 and evicts its own start long before the
+    next step reads it again); ("rotate", n) when n <=
+    MAX_ROTATE_COPIES copies of the cache, read in turn, put more than twice
+    the L2 between two reads of one copy; else ("flush", 1): L2 is flushed
+    before every step and each step is timed alone."""
+    if kv_bytes > 3 * L2_BYTES:
+        return "resident", 1
+    n = 2 + (2 * L2_BYTES) // kv_bytes if kv_bytes else MAX_ROTATE_COPIES + 1
+    if n <= MAX_ROTATE_COPIES:
+        return "rotate", n
+    return "flush", 1
+
+
+def l2_desc(kv_bytes: int) -> str:
+    how, n = l2_plan(kv_bytes)
+    if how == "resident":
+        return "inputs %.0f MiB > 3x the 126 MB L2, steps back to back (no flush)" % (kv_bytes / 2 ** 20)
+    if how == "rotate":
+        return ("steps back to back over %d copies of the %.0f MiB cache in turn (%.0f MiB of other copies "
+                "between two reads of one copy > 2x L2)" % (n, kv_bytes / 2 ** 20, (n - 1) * kv_bytes / 2 ** 20))
+    return "L2 flushed before every step (2x L2 written, then 2x L2 read), each step timed alone"
+
+
 class ClockSampler:
     """Samples SM clocks and clock-event reasons during the timed region (NVML)."""
 
@@ -115,21 +153,25 @@ class ClockSampler:
         except Exception:
             self._nv = None
 
-    def _run(self):
+    def _sample(self):
         nv = self._nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for b, name in self.REASONS.items():
+                if bits & b and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for b, name in self.REASONS.items():
-                    if bits & b and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.interval)
 
     def __enter__(self):
         if self._nv is not None:
+            self._stop.clear()
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
         return self
@@ -138,6 +180,7 @@ class ClockSampler:
         self._stop.set()
         if self._thread is not None:
             self._thread.join()
+            self._thread = None
 
     def summary(self):
         if not self.samples:
@@ -170,6 +213,45 @@ def max_over_ranks(x: float, world: int) -> float:
     from kv_cache_bandwidth_b200 import dist as gdist
 
     return x if world == 1 else gdist.max_over_ranks(x)
+
+
+def config_dict(w, inp, n_query=1):
+    """The workload a line measures (the same dict in both arms): its shape,
+    layout, KV bytes, seed and how L2 is kept out of the timing.  How the
+    library decomposes the step is reported beside it, under "plan"."""
+    kv = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
+    cfg = {
+        "workload": w.name if n_query == 1 else "verification step, %d query tokens per sequence, over %s" % (
+            n_query, w.name), "b": w.b, "H": w.H, "G": w.G, "d": w.d, "m": w.m,
+        "layout": "paged P=%d" % w.page_size if w.paged else "contiguous [b,G,m,d]",
+        "kv_bytes_per_step": kv, "seed": w.seed, "l2": l2_desc(kv),
+    }
+    if w.len_lo is not None:
+        cfg["lengths"] = "uniform integers in [%d, %d] (seeded)" % (w.len_lo, w.len_hi)
+    if w.peaky_frac > 0:
+        cfg["peaky"] = "%.0f%% of key rows x8 per (sequence, group)" % (100 * w.peaky_frac)
+    if n_query > 1:
+        cfg["query_tokens"] = n_query
+        cfg["rows_per_kv_group"] = n_query * w.r
+        cfg["mask"] = "query token t of n sees cached positions < len - (n - 1 - t)"
+    return cfg
+
+
+def plan_dict(split_tokens, max_len, n_query=1, tc=False, entry="split"):
+    """The library's decomposition of a step (GPU arm only)."""
+    if entry == "cluster":
+        decomp = "gqa_decode: one block or cluster per (sequence, group)"
+    elif split_tokens == 0:
+        decomp = "equal-work ranges over all (sequence, group) tiles (stream-K) + combine"
+    else:
+        n_splits = -(-max_len // split_tokens)
+        decomp = "fixed splits of %d tokens (%d per sequence), %s" % (
+            split_tokens, n_splits, "one block per (sequence, group), final rows" if n_splits == 1 else
+            "merged in the decode kernel" if n_splits <= 8 else "combine kernel")
+    d = {"split_tokens": split_tokens, "decomposition": decomp}
+    if n_query > 1:
+        d["kernel"] = "gqa_verify_tc_kernel (tcgen05)" if tc else "gqa_decode_kernel (mma.sync)"
+    return d
 
 
 # --------------------------------------------------------------------------- oracle leg
@@ -243,7 +325,7 @@ def reference_arm(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_dict(w, inp, None, args.query_tokens),
+        "data": "synthetic", "config": config_dict(w, inp, args.query_tokens),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": "each step: " + desc},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -272,170 +354,262 @@ class L2Flush:
         self.sink = self.r.sum()
 
 
-def config_dict(w, inp, split_tokens, n_query=1):
-    kv = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
-    if split_tokens is None:
-        decomp = "one block or cluster per (sequence, group)"
-    elif split_tokens == 0:
-        decomp = "equal-work ranges over all (sequence, group) tiles (stream-K) + combine"
-    else:
-        n_splits = -(-max(int(x) for x in inp.seqlens.tolist()) // split_tokens)
-        decomp = "fixed splits of %d tokens (%d per sequence), %s" % (
-            split_tokens, n_splits, "one block per (sequence, group), final rows" if n_splits == 1 else
-            "merged in the decode kernel" if n_splits <= 8 else "combine kernel")
-    cfg = {
-        "workload": w.name if n_query == 1 else "verification step, %d query tokens per sequence, over %s" % (
-            n_query, w.name), "b": w.b, "H": w.H, "G": w.G, "d": w.d, "m": w.m,
-        "layout": "paged P=%d" % w.page_size if w.paged else "contiguous [b,G,m,d]",
-        "split_tokens": split_tokens, "decomposition": decomp, "kv_bytes_per_step": kv, "seed": w.seed,
-        "l2": ("inputs %.0f MiB > 126 MB L2 (no flush)" % (kv / 2 ** 20)) if kv > 2 * L2_BYTES
-        else "L2 flushed between steps (2x L2 written, then 2x L2 read)",
-    }
-    if n_query > 1:
-        cfg["query_tokens"] = n_query
-        cfg["rows_per_kv_group"] = n_query * w.r
-        cfg["mask"] = "query token t of n sees cached positions < len - (n - 1 - t)"
-    return cfg
+class Case:
+    """One workload instance on the GPU and the public call of one step.
 
+    The KV cache is the decode state and stays resident; a cache that fits in
+    L2 is held in several copies that successive steps read in turn (see
+    l2_plan), so that back-to-back steps still stream from HBM."""
 
-def main_gpu(args):
-    from kv_cache_bandwidth_b200 import gqa
+    def __init__(self, args, w, nq, rank, with_copies=True):
+        from kv_cache_bandwidth_b200 import gqa
 
-    world, rank, local = dist_setup()
-    w = WORKLOADS[args.workload]
-    w = w.with_(seed=w.seed + 1000 * rank)  # each rank: its own shard of sequences
-    inp = make_inputs(w, device="cuda")
-    nq = args.query_tokens
-    q = inp.q if nq == 1 else draw_verify_q(w, nq, device="cuda")
-    kv_step = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
-    max_seqlen = int(inp.seqlens.max())
-    dims = gqa.dims_for(inp.q, inp.k_cache, inp.page_table)
-    # 0: the library's choice (equal-work ranges); > 0: fixed splits of that many tokens
-    split = args.split_tokens if args.split_tokens >= 0 else w.split_tokens
-    if nq > 1 and split == 0:
-        # verification runs fixed splits: one split per sequence
-        split = -(-max_seqlen // 256) * 256
-    if nq == 1:
-        ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, max_seqlen, split)
-    else:
-        ws = torch.empty(max(256, gqa.gqa_decode_verify_workspace_size(dims, nq, max_seqlen, split)),
-                         dtype=torch.uint8, device="cuda")
-    call = decode_call(args, inp, nq, split, max_seqlen, ws)
-    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    stream = torch.cuda.current_stream()
-    flush = L2Flush() if kv_step <= 2 * L2_BYTES else None
+        self.gqa = gqa
+        self.w = w = w.with_(seed=w.seed + 1000 * rank)  # each rank: its own shard of sequences
+        self.nq = nq
+        self.entry = args.entry
+        self.inp = inp = make_inputs(w, device="cuda")
+        self.q = inp.q if nq == 1 else draw_verify_q(w, nq, device="cuda")
+        self.kv_step = accounting.kv_bytes_per_step(w.G, w.d, inp.seqlens.tolist())
+        self.max_seqlen = int(inp.seqlens.max())
+        self.dims = gqa.dims_for(inp.q, inp.k_cache, inp.page_table)
+        # 0: the library's choice (equal-work ranges for a paged cache); > 0:
+        # fixed splits of that many tokens; -1: the library's plan
+        split = args.split_tokens
+        if nq > 1 and split <= 0:
+            split = -(-self.max_seqlen // 256) * 256  # verification runs fixed splits: one per sequence
+        if split < 0:
+            split = 0
+        self.split = split
+        if nq == 1:
+            self.ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, self.max_seqlen, split)
+        else:
+            n = gqa.gqa_decode_verify_workspace_size(self.dims, nq, self.max_seqlen, split)
+            self.ws = torch.empty(max(256, n), dtype=torch.uint8, device="cuda")
+        self.eff_split = split if split > 0 else gqa.gqa_plan_split_tokens(self.dims, self.max_seqlen)
+        n_splits = -(-self.max_seqlen // self.eff_split) if self.eff_split > 0 else 0
+        self.launches_per_step = 1 if (self.entry == "cluster" or 0 < n_splits <= gqa.SERIAL_MERGE_MAX_SPLITS) else 2
+        self.tc = nq * w.r > gqa.TC_AUTO_ROWS and w.d == 128
+        self.out = torch.empty(self.q.shape, dtype=torch.float32, device="cuda")
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.how, n_copies = l2_plan(self.kv_step)
+        self.caches = [(inp.k_cache, inp.v_cache)]
+        if with_copies:
+            for _ in range(n_copies - 1):
+                self.caches.append((inp.k_cache.clone(), inp.v_cache.clone()))
+        self.flush = L2Flush() if self.how == "flush" else None
+        self.i = 0
 
-    def step():
-        call(q, inp.seqlens, inp.page_table, out, status=status)
+    def call(self, q, sl, pt, out, k, v, status=None, stream=None):
+        gqa = self.gqa
+        if self.nq > 1:
+            gqa.gqa_decode_verify(q, k, v, sl, pt, split_tokens=self.split, max_seqlen=self.max_seqlen,
+                                  workspace=self.ws, out=out, status=status, stream=stream)
+        elif self.entry == "cluster":
+            gqa.gqa_decode(q, k, v, sl, pt, out=out, status=status, stream=stream)
+        else:
+            gqa.gqa_decode_split(q, k, v, sl, pt, split_tokens=self.split, max_seqlen=self.max_seqlen,
+                                 workspace=self.ws, out=out, status=status, stream=stream)
 
-    # fixed splits, at most 8 of them: one launch (the decode kernel merges
-    # each unit's splits itself); more splits or equal-work ranges: decode
-    # kernel + combine kernel
-    eff_split = split if split > 0 else gqa.gqa_plan_split_tokens(dims, max_seqlen)
-    n_splits = -(-max_seqlen // eff_split) if eff_split > 0 else 0
-    launches_per_step = 1 if (args.entry == "cluster" or 0 < n_splits <= gqa.SERIAL_MERGE_MAX_SPLITS) else 2
+    def step(self):
+        k, v = self.caches[self.i % len(self.caches)]
+        self.i += 1
+        self.call(self.q, self.inp.seqlens, self.inp.page_table, self.out, k, v, status=self.status)
 
-    # ---- warm-up
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if int(status.item()) != 0:
-        raise RuntimeError("decode reported status %d" % int(status.item()))
+    def decode_only(self):
+        """The decode kernel alone (the step without its combine launch)."""
+        k, v = self.caches[self.i % len(self.caches)]
+        self.i += 1
+        self.gqa.gqa_split_partials(self.inp.q, k, v, self.inp.seqlens, self.inp.page_table,
+                                    split_tokens=self.split, max_seqlen=self.max_seqlen, workspace=self.ws,
+                                    out=self.out, status=self.status)
 
-    # ---- timed region: K steps, inputs resident in HBM
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ms = []
-    with ClockSampler(local) as clocks:
-        if flush is None:
+    def check_status(self):
+        torch.cuda.synchronize()
+        st = int(self.status.item())
+        if st != 0:
+            raise RuntimeError("%s: decode reported status %d" % (self.w.name, st))
+
+    def time_steps(self, steps, world):
+        """ms per step, max over ranks: back-to-back steps between two events
+        (resident or rotating caches), or flush + one event pair per step."""
+        stream = torch.cuda.current_stream()
+        if self.how != "flush":
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             barrier(world)
             torch.cuda.synchronize()
             ev0.record(stream)
-            for _ in range(args.steps):
-                step()
+            for _ in range(steps):
+                self.step()
             ev1.record(stream)
             torch.cuda.synchronize()
             barrier(world)
-            total_ms = ev0.elapsed_time(ev1)
+            total = ev0.elapsed_time(ev1)
         else:
-            # small workload: flush L2 before every step, time each step alone
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
+            total = sum(self.time_flushed(steps, world, sync=False))
+        return max_over_ranks(total, world) / steps
+
+    def time_flushed(self, steps, world, sync=True, fn=None):
+        """Per-step ms of `fn` (default: one step), each launch alone after an
+        L2 flush, between its own event pair."""
+        fn = fn or self.step
+        flush = self.flush or L2Flush()
+        stream = torch.cuda.current_stream()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        if sync:
             barrier(world)
-            torch.cuda.synchronize()
-            for a, b in evs:
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        if sync:
+            barrier(world)
+        return [a.elapsed_time(b) for a, b in evs]
+
+    def kernel_ms(self, steps, world):
+        """The dominant kernel (the decode kernel) alone: mean of isolated
+        launches between CUDA events on its stream, L2 flushed first when the
+        cache fits in it; for a one-launch step that is the step itself."""
+        kern = self.step if (self.launches_per_step == 1 or self.nq > 1) else self.decode_only
+        stream = torch.cuda.current_stream()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(max(steps, 10))]
+        flush = None if self.how == "resident" else (self.flush or L2Flush())
+        for a, b in evs:
+            if flush is not None:
                 flush()
-                a.record(stream)
-                step()
-                b.record(stream)
-            torch.cuda.synchronize()
-            barrier(world)
-            step_ms = [a.elapsed_time(b) for a, b in evs]
-            total_ms = sum(step_ms)
-    total_ms = max_over_ranks(total_ms, world)
-    ms_per_step = total_ms / args.steps
-    value = world * kv_step / (ms_per_step * 1e-3) / 1e9
+            a.record(stream)
+            kern()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
+
+    def kernel_name(self):
+        if self.nq > 1:
+            return "%s (verification, %d rows per KV group%s)" % (
+                "gqa_verify_tc_kernel" if self.tc else "gqa_decode_kernel", self.nq * self.w.r,
+                "" if self.launches_per_step == 1 else "; decode + combine timed together")
+        if self.entry == "split":
+            if self.eff_split == 0:
+                return "gqa_decode_kernel (equal-work ranges)"
+            return "gqa_decode_kernel (fixed splits%s)" % (", merged in-kernel" if self.launches_per_step == 1 else "")
+        return "gqa_decode_kernel (gqa_decode)"
+
+    def plan(self):
+        return plan_dict(self.eff_split, self.max_seqlen, self.nq, self.tc, self.entry)
+
+    def free(self):
+        self.caches = []
+        self.inp = None
+        self.ws = None
+        self.flush = None
+
+
+def measure_point(args, name, nq, world, rank, hbm):
+    """One per_config entry: the same step timing as the headline, the
+    kernel alone, and for caches that fit in L2 the flush-then-event time."""
+    case = Case(args, WORKLOADS[name], nq, rank)
+    for _ in range(args.warmup):
+        case.step()
+    case.check_status()
+    ms = case.time_steps(args.steps, world)
+    kern = case.kernel_ms(args.steps, world)
+    case.check_status()
+    kv = case.kv_step
+    d = {"us_per_step": ms * 1e3, "kv_bytes": kv, "gbs": world * kv / (ms * 1e-3) / 1e9,
+         "frac": kv / (ms * 1e-3) / 1e9 / hbm, "kernel_us": kern * 1e3,
+         "kernel_frac": kv / (kern * 1e-3) / 1e9 / hbm, "timing": case.how,
+         "traffic": recorded_traffic(traffic_key(name, nq)), "plan": case.plan()["decomposition"]}
+    if case.how == "rotate":
+        flushed = max_over_ranks(statistics.median(case.time_flushed(max(args.steps, 10), world)), world)
+        d["us_flushed"] = flushed * 1e3
+        d["frac_flushed"] = kv / (flushed * 1e-3) / 1e9 / hbm
+    case.free()
+    del case
+    torch.cuda.empty_cache()
+    return d
+
+
+def main_gpu(args):
+    world, rank, local = dist_setup()
     hbm, hbm_kind = peaks()
+    nq = args.query_tokens
+    case = Case(args, WORKLOADS[args.workload], nq, rank)
+    w, inp = case.w, case.inp
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        case.step()
+    case.check_status()
+
+    # ---- timed region: K steps, inputs resident in HBM
+    clocks = ClockSampler(local)
+    with clocks:
+        ms_per_step = case.time_steps(args.steps, world)
+    timed_samples = len(clocks.samples)
+    # ---- the same step repeated for >= 1 s, so that the clock record has
+    # samples even when the timed region is a few milliseconds
+    with clocks:
+        t_end = time.perf_counter() + max(1.0, args.clock_window)
+        n_win = 0
+        while time.perf_counter() < t_end:
+            for _ in range(32):
+                case.step()
+            n_win += 32
+            torch.cuda.synchronize()
+    case.check_status()
+    value = world * case.kv_step / (ms_per_step * 1e-3) / 1e9
 
     # ---- dominant kernel alone (decode kernel), CUDA events on its stream
-    # (one launch per step: the step's own launch, timed alone; two: the decode
-    # kernel without the combine)
-    def decode_only():
-        gqa.gqa_split_partials(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
-                               split_tokens=split, max_seqlen=max_seqlen, workspace=ws, out=out,
-                               status=status)
-
-    kern = step if (launches_per_step == 1 or nq > 1) else decode_only
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(max(args.steps, 10))]
-    for a, b in evs:
-        if flush is not None:
-            flush()
-        a.record(stream)
-        kern()
-        b.record(stream)
-    torch.cuda.synchronize()
-    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    kern_ms = max_over_ranks(kern_ms, world)
-    achieved = kv_step / (kern_ms * 1e-3) / 1e9
-    if nq > 1:
-        tc = nq * w.r > gqa.TC_AUTO_ROWS and w.d == 128
-        kname = "%s (verification, %d rows per KV group%s)" % (
-            "gqa_verify_tc_kernel" if tc else "gqa_decode_kernel", nq * w.r,
-            "" if launches_per_step == 1 else "; decode + combine timed together")
-    elif args.entry == "split":
-        kname = ("gqa_decode_kernel (equal-work ranges)" if eff_split == 0 else
-                 "gqa_decode_kernel (fixed splits%s)" % (", merged in-kernel" if launches_per_step == 1 else ""))
-    else:
-        kname = "gqa_decode_kernel (gqa_decode)"
+    kern_ms = case.kernel_ms(args.steps, world)
+    achieved = case.kv_step / (kern_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": recorded_traffic(traffic_key(args.workload, nq)),
-                "kernel": kname, "peak_kind": hbm_kind,
-                "kernel_us": kern_ms * 1e3, "algorithmic_bytes_per_launch": kv_step}
+                "kernel": case.kernel_name(), "peak_kind": hbm_kind,
+                "kernel_us": kern_ms * 1e3, "algorithmic_bytes_per_launch": case.kv_step}
 
     # ---- end to end through the public API with host buffers
-    e2e = e2e_leg(args, inp, q, call, kv_step, world)
+    e2e = e2e_leg(args, case, world)
+    plan = case.plan()
+    launches = case.launches_per_step * args.steps
+    cfg = config_dict(w, inp, nq)
 
     # ---- CPU baseline: the oracle on host cores (rank 0, N = 1 only)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         gbs, dt, threads, desc = oracle_time(inp, target_s=args.oracle_seconds if args.oracle_seconds > 0 else 15.0,
-                                             q_verify=None if nq == 1 else q)
+                                             q_verify=None if nq == 1 else case.q)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": desc + "; %.1f s of CPU time" % dt}
+    case.free()
+    del case
+    torch.cuda.empty_cache()
+
+    # ---- every workload, measured the same way in this process
+    per_config = {}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            per_config[name] = measure_point(args, name, 1, world, rank, hbm)
+        for name, n in PER_CONFIG_VERIFY:
+            per_config[traffic_key(name, n)] = measure_point(args, name, n, world, rank, hbm)
 
     if rank == 0:
+        clk = clocks.summary()
+        clk["timed_region_samples"] = timed_samples
+        clk["window"] = "timed region + %d more steps over >= %.1f s" % (n_win, max(1.0, args.clock_window))
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": config_dict(w, inp, eff_split if args.entry == "split" else None, nq),
+            "data": "synthetic", "config": cfg, "plan": plan,
             "frac_of_peak_hbm": value / world / hbm, "peak_hbm_gbs": hbm, "peak_kind": hbm_kind,
             "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
             "entry": "gqa_decode_verify" if nq > 1 else "gqa_decode_split" if args.entry == "split" else "gqa_decode",
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(),
+            "gpu_launches": launches, "clocks": clk, "per_config": per_config,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -444,34 +618,19 @@ def main_gpu(args):
     return 0
 
 
-def decode_call(args, inp, nq, split, max_seqlen, ws):
-    """The public call one step makes: (q, seqlens, page_table, out, status=,
-    stream=) -> None, on the resident KV cache."""
-    from kv_cache_bandwidth_b200 import gqa
-
-    def call(q, sl, pt, out, status=None, stream=None):
-        if nq > 1:
-            gqa.gqa_decode_verify(q, inp.k_cache, inp.v_cache, sl, pt, split_tokens=split, max_seqlen=max_seqlen,
-                                  workspace=ws, out=out, status=status, stream=stream)
-        elif args.entry == "cluster":
-            gqa.gqa_decode(q, inp.k_cache, inp.v_cache, sl, pt, out=out, status=status, stream=stream)
-        else:
-            gqa.gqa_decode_split(q, inp.k_cache, inp.v_cache, sl, pt, split_tokens=split, max_seqlen=max_seqlen,
-                                 workspace=ws, out=out, status=status, stream=stream)
-    return call
-
-
-def e2e_leg(args, inp, q, call, kv_step, world):
+def e2e_leg(args, case, world):
     """Same metric through the public call with host buffers: each step copies the
     step's inputs (q, lengths, page table) from pinned host memory, runs the
     decode and reads the result back into pinned host memory.  The KV cache is
-    the decode state and stays resident in HBM.
+    the decode state and stays resident in HBM (copies of it read in turn when
+    it fits in L2, as in the device-timed steps).
 
     Steps are pipelined the way a serving loop would run them: two sets of
     device input/output buffers, the copies on their own streams (the copy
     engines) and the decode on a compute stream, so step i+1's inputs travel
     and step i-1's result returns while step i decodes.  Events order every
     buffer reuse."""
+    inp, q = case.inp, case.q
     h_q = q.cpu().pin_memory()
     h_sl = inp.seqlens.cpu().pin_memory()
     h_pt = None if inp.page_table is None else inp.page_table.cpu().pin_memory()
@@ -490,6 +649,7 @@ def e2e_leg(args, inp, q, call, kv_step, world):
 
     def step(i):
         k = i % 2
+        kc, vc = case.caches[i % len(case.caches)]
         with torch.cuda.stream(s_in):      # inputs of step i (buffer k is free once step i-2 decoded)
             s_in.wait_event(comp_done[k])
             d_q[k].copy_(h_q, non_blocking=True)
@@ -500,7 +660,7 @@ def e2e_leg(args, inp, q, call, kv_step, world):
         with torch.cuda.stream(s_comp):    # decode of step i (its output buffer is free once read back)
             s_comp.wait_event(in_done[k])
             s_comp.wait_event(out_done[k])
-            call(d_q[k], d_sl[k], d_pt[k], d_out[k], stream=s_comp)
+            case.call(d_q[k], d_sl[k], d_pt[k], d_out[k], kc, vc, stream=s_comp)
             comp_done[k].record(s_comp)
         with torch.cuda.stream(s_out):     # result of step i back to the host
             s_out.wait_event(comp_done[k])
@@ -522,7 +682,7 @@ def e2e_leg(args, inp, q, call, kv_step, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(ev0.elapsed_time(ev1) / n, world)
-    return {"value": world * kv_step / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+    return {"value": world * case.kv_step / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "note": "every step: q, lengths (and page table) H2D from pinned memory, decode, output D2H to "
                     "pinned memory; steps pipelined over copy and compute streams; KV cache resident"}
@@ -531,15 +691,18 @@ def e2e_leg(args, inp, q, call, kv_step, world):
 def main(argv=None):
     ap = argparse.ArgumentParser(description="GQA decode benchmark (B200)")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama70b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ragged")
     ap.add_argument("--entry", choices=["split", "cluster"], default="split")
     ap.add_argument("--split-tokens", type=int, default=-1,
-                    help="-1: the workload's own split (0 when it has none); 0: the library's "
-                         "equal-work ranges; > 0: fixed splits of that many tokens")
+                    help="-1: the library's plan; 0: the library's automatic choice at run time (the same); "
+                         "> 0: fixed splits of that many tokens")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="measure the headline workload only")
+    ap.add_argument("--clock-window", type=float, default=1.0,
+                    help="seconds of repeated steps sampled for clocks after the timed region (>= 1)")
     ap.add_argument("--oracle-seconds", type=float, default=0.0,
                     help="CPU seconds of oracle work per timed sample (0: 15 s for cpu_baseline; the reference "
                          "arm spreads about two minutes over its steps)")

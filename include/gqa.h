@@ -85,7 +85,9 @@ extern "C" {
 /* Bits the kernels OR into *status. */
 #define GQA_STATUS_BAD_SEQLEN 1u   /* a length outside [1, capacity]: row zeroed */
 #define GQA_STATUS_BAD_PAGE 2u     /* a page id outside [0, num_pages): row zeroed */
-#define GQA_STATUS_TIMEOUT 4u      /* an on-chip pipeline wait gave up: output undefined */
+#define GQA_STATUS_TIMEOUT 4u      /* an on-chip pipeline wait gave up: output undefined; before replaying a
+                                      captured graph whose call reported it, zero its workspace (a unit's
+                                      arrival count may have been left part-way) */
 
 /* Largest supported group ratio r = H / G. */
 #define GQA_MAX_GROUP_RATIO 64
@@ -334,12 +336,15 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
  * in the library's device module; each GPU that loads the library holds it
  * until the process exits.  Problems whose gqa_decode_split_workspace_size()
  * exceeds that size are rejected with GQA_ERR_WORKSPACE before anything runs.
- * The first call on a device looks up the array's device address (a CUDA
- * runtime call, no allocation) and caches it; make that first call before any
- * stream capture.  All calls share the array: calls whose kernels overlap on
- * the GPU (different streams or host threads) race on it.  Nothing in it needs
- * to start at zero.  No cudaMalloc, cudaFree or other allocating routine is
- * called.
+ * Argument errors take precedence over GQA_ERR_WORKSPACE, in the order
+ * gqa_decode_split checks them.  The first call on a device looks up the
+ * array's device address (a CUDA runtime call, no allocation) and caches it
+ * for the life of the process; make that first call before any stream
+ * capture, and do not use the library across cudaDeviceReset (the cached
+ * address would be stale).  All calls share the array: calls whose kernels
+ * overlap on the GPU (different streams or host threads) race on it.  Nothing
+ * in it needs to start at zero.  No cudaMalloc, cudaFree or other allocating
+ * routine is called.
  */
 #define GQA_STATIC_WORKSPACE_BYTES (8u << 20)
 

@@ -6,6 +6,11 @@ The library is compiled in-tree for sm_100a only, with nvcc:
 
 The ptxas resource report (registers, spills, shared memory per kernel) is kept
 in ``kv_cache_bandwidth_b200/_build/ptxas.log``.
+
+A second library, ``libgqa_test_hooks.so``, is the same sources built for the
+bounded-wait tests: every wait gives up after ~10 ms instead of ~2 s, and an
+extra entry point (gqa_test_skip_tile) makes one block's producer leave one
+K/V tile out so that a wait runs out.  Nothing but those tests loads it.
 """
 from __future__ import annotations
 
@@ -21,7 +26,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgqa.so")
+TEST_LIB = os.path.join(PKG, "libgqa_test_hooks.so")
 BUILD_DIR = os.path.join(PKG, "_build")
+# the test library's wait limit: ~10 ms at the B200's clocks
+TEST_FLAGS = ["-DGQA_TEST_HOOKS", "-DGQA_WAIT_LIMIT_CYCLES=20000000ll"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH_FLAGS + [
@@ -45,28 +53,42 @@ def inputs():
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "gqa.h"), __file__]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in inputs())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+    """Build libgqa.so and libgqa_test_hooks.so (two nvcc runs in parallel);
+    returns the path of libgqa.so."""
+    jobs = [(lib, extra, log) for lib, extra, log in ((LIB, [], "ptxas.log"),
+                                                      (TEST_LIB, TEST_FLAGS, "ptxas_test_hooks.log"))
+            if force or not up_to_date(lib)]
+    if not jobs:
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
-    tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [nvcc()] + NVCC_FLAGS + ["-o", tmp] + sources()
-    proc = subprocess.run(cmd, capture_output=True, text=True)
-    with open(os.path.join(BUILD_DIR, "ptxas.log"), "w") as f:
-        f.write(" ".join(cmd) + "\n" + proc.stdout + proc.stderr)
-    if proc.returncode != 0:
-        sys.stderr.write(proc.stdout + proc.stderr)
-        raise RuntimeError("nvcc failed building libgqa.so (exit %d)" % proc.returncode)
-    if verbose:
-        sys.stderr.write(proc.stderr)
-    os.replace(tmp, LIB)
+    procs = []
+    for lib, extra, log in jobs:
+        tmp = lib + ".tmp.%d" % os.getpid()
+        cmd = [nvcc()] + NVCC_FLAGS + extra + ["-o", tmp] + sources()
+        procs.append((lib, tmp, log, cmd,
+                      subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)))
+    failed = None
+    for lib, tmp, log, cmd, proc in procs:
+        out, err = proc.communicate()
+        with open(os.path.join(BUILD_DIR, log), "w") as f:
+            f.write(" ".join(cmd) + "\n" + out + err)
+        if proc.returncode != 0:
+            sys.stderr.write(out + err)
+            failed = failed or "nvcc failed building %s (exit %d)" % (os.path.basename(lib), proc.returncode)
+            continue
+        if verbose:
+            sys.stderr.write(err)
+        os.replace(tmp, lib)
+    if failed:
+        raise RuntimeError(failed)
     return LIB
 
 

@@ -762,6 +762,16 @@ extern "C" {
 
 int32_t gqa_abi_version(void) { return (1 << 16) | 0; }
 
+#ifdef GQA_TEST_HOOKS
+// Test library only (not declared in gqa.h): the producer of decode block
+// `block` leaves out the K/V tile at ring position `ring_pos` of its pipeline
+// (-1, -1: none), so that a test can make a bounded wait run out.
+int gqa_test_skip_tile(int32_t block, int32_t ring_pos) {
+  const int v[2] = {block, ring_pos};
+  return cudaMemcpyToSymbol(gqa::g_test_skip_tile, v, sizeof(v)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+#endif
+
 const char *gqa_status_string(int code) {
   switch (code) {
     case GQA_OK: return "ok";

@@ -925,6 +925,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         }
         const uint32_t dst_k = smem_addr(smem + stage * TL::kStageBytes);
         const uint32_t dst_v = dst_k + TL::kTileBytes;
+        if (test_skip_tile(tile)) continue;  // test builds only
         if (PAGED) {
           const int lp0 = t0 / P;
           const int wnd = lp0 >> 5;

@@ -32,7 +32,11 @@ std::mutex g_scratch_mu;
 
 // Device address of the array for the current device.  In host code the
 // array's name is only a host-side handle, so the address is looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached.  The cache assumes the
+// device's context lives as long as the process: after cudaDeviceReset (or a
+// release and re-creation of the primary context) the module is loaded again
+// elsewhere and the cached address is stale, so the library must not be used
+// across a device reset.
 int scratch_address(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
@@ -54,10 +58,16 @@ extern "C" int gqa_decode_split_static(const void *q, const void *k_cache, const
                                        const gqa_dims *dims, float scale, uint32_t *status,
                                        int32_t split_tokens, int32_t max_seqlen, void *stream) {
   const size_t need = gqa_decode_split_workspace_size(dims, max_seqlen, split_tokens);
-  if (need == 0)  // invalid arguments: let the regular entry point name the error
-    return gqa_decode_split(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status,
-                            split_tokens, max_seqlen, nullptr, 0, stream);
-  if (need > GQA_STATIC_WORKSPACE_BYTES) return GQA_ERR_WORKSPACE;
+  if (need == 0 || need > GQA_STATIC_WORKSPACE_BYTES) {
+    // Invalid arguments, or a problem too large for the array: the regular
+    // entry point, given no workspace, runs all of its checks in its own order
+    // and stops at the workspace test at the latest (it launches nothing
+    // without one), so an argument error is reported ahead of
+    // GQA_ERR_WORKSPACE exactly as gqa_decode_split reports it.
+    const int rc = gqa_decode_split(q, k_cache, v_cache, seqlens, page_table, out, dims, scale, status,
+                                    split_tokens, max_seqlen, nullptr, 0, stream);
+    return rc == GQA_OK ? GQA_ERR_WORKSPACE : rc;
+  }
   void *scratch = nullptr;
   const int rc = scratch_address(&scratch);
   if (rc != GQA_OK) return rc;

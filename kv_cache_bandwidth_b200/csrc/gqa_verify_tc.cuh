@@ -57,8 +57,9 @@ struct TcTile {
   static constexpr int kQHalf = kM * 128;
   static constexpr int kBarOff = kQOff + 2 * kQHalf;
   static constexpr int kSP = 3;                        // S/P buffers in tensor memory
-  // full[kStages], empty[kStages], s_full[kSP], p_full[kSP], pv_done[kSP]
-  static constexpr int kNumBars = 2 * kStages + 3 * kSP;
+  // full[kStages], empty[kStages], s_full[kSP], p_full[kSP], pv_done[kSP],
+  // drain[2] (one per MMA issuer: all its products done before teardown)
+  static constexpr int kNumBars = 2 * kStages + 3 * kSP + 2;
   static constexpr int kXOff = kBarOff + 8 * kNumBars;  // the halves' bases at the end: [2][kM] floats
   static constexpr int kLOff = kXOff + 4 * 2 * kM;      // the halves' sums at the end: [2][kM] floats
   static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[kStages], abort, merge here
@@ -109,6 +110,7 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap *tm_k, const CUtens
     }
     const uint32_t dst_k = sbase + stage * TT::kStageBytes;
     const uint32_t dst_v = dst_k + TT::kTileBytes;
+    if (test_skip_tile(tile)) continue;  // test builds only
     if (PAGED) {
       const int lp0 = t0 / P;
       const int wnd = lp0 >> 5;
@@ -175,6 +177,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   constexpr int SP = TT::kSP;
   const uint32_t s_full0 = bars + 16 * ST;
   const uint32_t p_full0 = s_full0 + 8 * SP, pv_done0 = p_full0 + 8 * SP;
+  const uint32_t drain0 = pv_done0 + 8 * SP;  // [2]: the Q K^T issuer's, the P.V issuer's
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
   volatile int *abort_flag = tile_bad + ST;
@@ -213,6 +216,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       mbar_init(p_full0 + 8 * i, TT::kSoftmaxWarps);  // one arrival per softmax warp
       mbar_init(pv_done0 + 8 * i, 1);
     }
+    mbar_init(drain0, 1);
+    mbar_init(drain0 + 8, 1);
     *abort_flag = 0;
     *merge_here = 0;
     fence_mbarrier_init();
@@ -275,6 +280,10 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         *abort_flag = 1;
         if (p.status) atomicOr(p.status, kStatusTimeout);
       }
+      // every product this thread issued is done before the block tears down
+      // (on an early exit, products already issued may still be running)
+      tc_commit(drain0);
+      if (!mbar_wait(drain0, 0) && p.status) atomicOr(p.status, kStatusTimeout);
     }
   } else if (warp == kPvWarp) {
     // ============================================================ P.V issuer
@@ -309,6 +318,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
         *abort_flag = 1;
         if (p.status) atomicOr(p.status, kStatusTimeout);
       }
+      tc_commit(drain0 + 8);
+      if (!mbar_wait(drain0 + 8, 0) && p.status) atomicOr(p.status, kStatusTimeout);
     }
   } else {
     // ============================================================ softmax rows
@@ -497,7 +508,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     }
   }
 
-  // ---- teardown: every tensor-memory access is done before the columns go back
+  // ---- teardown: every tensor-memory access is done before the columns go
+  // back (the two issuers waited above for their last products to finish)
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

@@ -13,8 +13,24 @@
 namespace gqa {
 
 // About two seconds at the B200's top SM clock; any legitimate pipeline wait
-// is shorter by six orders of magnitude.
-constexpr long long kWaitLimitCycles = 4000000000ll;
+// is shorter by six orders of magnitude.  (The library built for the
+// bounded-wait tests sets a limit of a few milliseconds.)
+#ifndef GQA_WAIT_LIMIT_CYCLES
+#define GQA_WAIT_LIMIT_CYCLES 4000000000ll
+#endif
+constexpr long long kWaitLimitCycles = GQA_WAIT_LIMIT_CYCLES;
+
+#ifdef GQA_TEST_HOOKS
+// Test builds only: {block, ring position} of one K/V tile that the block's
+// TMA producer leaves out (nothing is copied and nothing arrives on its
+// barrier), so that the waits for it run out; {-1, -1} leaves nothing out.
+__device__ int g_test_skip_tile[2] = {-1, -1};
+__device__ __forceinline__ bool test_skip_tile(int ring_pos) {
+  return static_cast<int>(blockIdx.x) == g_test_skip_tile[0] && ring_pos == g_test_skip_tile[1];
+}
+#else
+__device__ __forceinline__ bool test_skip_tile(int) { return false; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

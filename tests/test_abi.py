@@ -262,3 +262,33 @@ def test_tcgen05_flag_checks(lib):
     assert _decode(lib, _dims(head_dim=128, flags=tc | gqa.FLAG_CONTRACT_MMA)) == -6
     # 16 tokens x 8 heads = 128 rows fit: the workspace size is defined
     assert lib.gqa_decode_verify_workspace_size(ctypes.byref(d128), 16, 256, 128) > 0
+
+
+def _static(lib, dims, q=FAKE, k=FAKE, v=FAKE, seq=FAKE, out=FAKE, scale=0.1, split=0, max_seqlen=4096):
+    return lib.gqa_decode_split_static(q, k, v, seq, None, out, ctypes.byref(dims), scale, None, split,
+                                       max_seqlen, None)
+
+
+@pytest.mark.parametrize("case,kw,code", [
+    ("null q", dict(q=None), -1),
+    ("misaligned k", dict(k=FAKE + 8), -2),
+    ("nan scale", dict(scale=float("nan")), -6),
+    ("bad split", dict(split=100), -7),
+    ("valid but too large for the array", dict(), -8),
+])
+def test_static_entry_point_reports_argument_errors_first(lib, case, kw, code):
+    """gqa_decode_split_static on a problem whose scratch exceeds the fixed
+    array (r = 64, equal-work ranges): an argument error is reported as
+    gqa_decode_split reports it, and only a valid call gets GQA_ERR_WORKSPACE."""
+    d = gqa.Dims(2, 128, 2, 128, 4096, 2, 0, 0)
+    assert gqa.gqa_decode_split_workspace_size(d, 4096, 0) > gqa.STATIC_WORKSPACE_BYTES
+    assert _static(lib, d, **kw) == code
+
+
+def test_test_hooks_only_in_the_test_library(lib):
+    """The entry point that leaves a tile out exists only in the library the
+    bounded-wait tests load, never in libgqa.so."""
+    assert not hasattr(lib, "gqa_test_skip_tile")
+    hooks = ctypes.CDLL(gqa_build.TEST_LIB)
+    assert hasattr(hooks, "gqa_test_skip_tile")
+    assert hasattr(hooks, "gqa_decode_split")

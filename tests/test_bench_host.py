@@ -50,8 +50,27 @@ def test_traffic_keys_and_verification_config():
     assert bench.traffic_key("llama70b", 8) == "llama70b_verify8"
     w = WORKLOADS["tiny"]
     inp = make_inputs(w)
-    c1 = bench.config_dict(w, inp, 128)
+    c1 = bench.config_dict(w, inp)
     assert "query_tokens" not in c1 and c1["workload"] == w.name
-    c4 = bench.config_dict(w, inp, 128, 4)
+    c4 = bench.config_dict(w, inp, 4)
     assert c4["query_tokens"] == 4 and c4["rows_per_kv_group"] == 4 * w.r
     assert c4["kv_bytes_per_step"] == c1["kv_bytes_per_step"]
+    # the config names the workload only: the library's split plan is reported apart
+    assert "split_tokens" not in c1 and "decomposition" not in c1
+    p = bench.plan_dict(4096, 131072)
+    assert p["split_tokens"] == 4096 and "32 per sequence" in p["decomposition"]
+    assert "equal-work" in bench.plan_dict(0, 32768)["decomposition"]
+
+
+def test_l2_plan_keeps_steps_out_of_l2():
+    L2 = bench.L2_BYTES
+    assert bench.l2_plan(4 * L2) == ("resident", 1)
+    for kv in (L2 // 4, L2 // 2, L2, 2 * L2, 3 * L2):
+        how, n = bench.l2_plan(kv)
+        assert how == "rotate" and 2 <= n <= bench.MAX_ROTATE_COPIES
+        # between two reads of one copy, the other copies' bytes exceed twice the L2
+        assert (n - 1) * kv > 2 * L2
+        assert (n - 2) * kv <= 2 * L2  # and no more copies than that needs
+    assert bench.l2_plan(256 * 1024) == ("flush", 1)
+    assert bench.l2_plan(0) == ("flush", 1)
+    assert "flushed" in bench.l2_desc(1000) and "copies" in bench.l2_desc(L2)

@@ -8,6 +8,9 @@ import sys
 
 import pytest
 
+import bench
+from kv_cache_bandwidth_b200.workloads import WORKLOADS, make_inputs
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -31,6 +34,9 @@ def test_reference_line(extra):
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    # the same workload description as the GPU arm's line (no plan in it)
+    assert d["config"] == bench.config_dict(WORKLOADS["tiny"], make_inputs(WORKLOADS["tiny"]),
+                                            int(extra[1]) if extra else 1)
     if extra:
         assert d["config"]["query_tokens"] == 3
         assert "3 query tokens" in d["cpu_baseline"]["sample"]

@@ -5,7 +5,8 @@ must stay out of the CUDA allocator).
 
 It must give what gqa_decode_split gives with a caller-allocated workspace,
 call after call: the scratch is shared and keeps the previous call's contents,
-so each case runs twice in a row, on the equal-work and the fixed-split paths.
+so each case runs twice in a row, on the equal-work and the fixed-split paths,
+and each call is also checked directly against the float64 oracle.
 This file is collected last on purpose; it also passes when run alone.
 """
 import ctypes
@@ -14,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from kv_cache_bandwidth_b200 import gqa
 from kv_cache_bandwidth_b200.workloads import Workload, make_inputs
 
@@ -43,6 +45,11 @@ def test_static_scratch_matches_workspace_entry_point(name, w, split):
     inp = make_inputs(w, device="cuda")
     ref = gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
                                split_tokens=split)
+    expect, st_ref = oracle.gqa_decode(inp.q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu(), inp.seqlens.cpu(),
+                                       None if inp.page_table is None else inp.page_table.cpu(),
+                                       num_kv_heads=w.G)
+    assert st_ref == 0
+    expect = torch.from_numpy(expect).reshape(inp.q.shape)
     for call in range(2):
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
         out = torch.full(inp.q.shape, float("nan"), dtype=torch.float32, device="cuda")
@@ -51,6 +58,7 @@ def test_static_scratch_matches_workspace_entry_point(name, w, split):
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         assert _close(out, ref), "%s, call %d" % (name, call)
+        assert _close(out, expect), "%s, call %d, against the oracle" % (name, call)
 
 
 def test_static_scratch_rejects_problems_that_do_not_fit():
