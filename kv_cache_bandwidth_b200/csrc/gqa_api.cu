@@ -231,13 +231,14 @@ unsigned long long next_epoch() {
 
 // Blocks per cluster for gqa_decode: 1 (one block per (sequence, group)
 // unit) when the units give about 1.5 blocks per SM; otherwise the smallest
-// power of two (at most 16) that does, never more blocks than 128-token tiles.
+// power of two (at most 16, gqa::kMaxClusterBlocks) that does, never more
+// blocks than 128-token tiles.
 int cluster_plan(const Shape &sh, int sms) {
   const long long units = units_of(sh);
   const long long want = (3ll * sms + 1) / 2;
   const long long max_by_len = std::max<long long>(1, sh.capacity / 128);
   int c = 1;
-  while (c < 16 && units * c < want && 2 * c <= max_by_len) c *= 2;
+  while (c < gqa::kMaxClusterBlocks && units * c < want && 2 * c <= max_by_len) c *= 2;
   return c;
 }
 
@@ -305,7 +306,7 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
   cfg.blockDim = dim3(TL::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = l.stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (MODE == Mode::kCluster) {
@@ -313,6 +314,11 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
     attr[0].val.clusterDim.x = l.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    if (l.pdl) {
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.numAttrs = 2;
+    }
   } else if (l.pdl) {
     // items mode: may start while the previous kernel on the stream finishes
     // (the kernel waits for it before touching memory)
@@ -362,18 +368,20 @@ int tile_tokens(const Shape &sh) { return sh.D == 64 ? 128 : 64; }
 // The tcgen05 kernel (items mode; d = 128, 64-token tiles like the mma.sync kernel).
 int launch_verify_tc(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p,
                      const Launch &l) {
-  auto kernel = sh.paged ? gqa::gqa_verify_tc_kernel<true> : gqa::gqa_verify_tc_kernel<false>;
+  // at most 64 rows: spread over the four lane quarters of tensor memory
+  const bool spread = sh.rc <= 64;
+  auto kernel = sh.paged ? (spread ? gqa::gqa_verify_tc_kernel<true, true> : gqa::gqa_verify_tc_kernel<true, false>)
+                         : (spread ? gqa::gqa_verify_tc_kernel<false, true> : gqa::gqa_verify_tc_kernel<false, false>);
   constexpr int smem = gqa::TcTile::kSmemBytes;
   static std::atomic<unsigned long long> attr_set{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load(std::memory_order_acquire) & bit)) {
-    if (cudaFuncSetAttribute(gqa::gqa_verify_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess ||
-        cudaFuncSetAttribute(gqa::gqa_verify_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return GQA_ERR_CUDA;
+    for (auto k : {gqa::gqa_verify_tc_kernel<true, true>, gqa::gqa_verify_tc_kernel<true, false>,
+                   gqa::gqa_verify_tc_kernel<false, true>, gqa::gqa_verify_tc_kernel<false, false>})
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return GQA_ERR_CUDA;
     attr_set.fetch_or(bit, std::memory_order_acq_rel);
   }
   cudaLaunchConfig_t cfg = {};
@@ -816,7 +824,9 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
   if ((rc = encode_maps(sh, k_cache, v_cache, &tk, &tv)) != GQA_OK) return rc;
   DecodeParams p = base_params(sh, q, seqlens, page_table, status, scale);
   p.out = out;
-  Launch l{dim3(c, sh.G * sh.hs, sh.b), c, st};
+  // launched as a programmatic dependent: the blocks set themselves up while
+  // the previous kernel on the stream finishes
+  Launch l{dim3(c, sh.G * sh.hs, sh.b), c, st, true};
   return launch_decode<Mode::kCluster>(sh, tk, tv, p, l);
 }
 

@@ -57,6 +57,9 @@ constexpr float kLBadPage = -1.f;    // the split met a page id outside the pool
 constexpr float kLBadLength = -2.f;  // split 0: the length is outside [1, capacity]
 constexpr float kLFinal = -3.f;      // split 0: the only split already wrote the final row
 
+// Largest thread-block cluster of the cluster mode (non-portable size).
+constexpr int kMaxClusterBlocks = 16;
+
 // kItems: one block per (sequence, group, split) item, blockIdx.x = item.
 // kCluster: one block per cluster rank; the blocks of a cluster share one
 // (sequence, group) and merge through distributed shared memory.
@@ -171,7 +174,19 @@ struct Tile {
   // piece per block the merge of the output accumulators reuses the ring once
   // every tile has been consumed; in balanced mode the ring is already taking
   // the next piece, so the merge rows have their own space.
-  static constexpr int kOSumOff = BAL ? kRingBytes : 0;
+  // One piece per block (items and cluster modes): once every tile has been
+  // consumed the ring holds each consumer warp's raw O rows ([kNC][kHB]
+  // [kOStride] floats from offset 0), then the block's merged rows (osum).
+  // The cluster mode's receive area ([blocks][rows per owner][D + 4] floats,
+  // blocks x rows <= kRPad + 16) reuses the warps' rows, which are dead by
+  // then.  In balanced mode the ring is already taking the next piece, so the
+  // merged rows have their own space after it.
+  static constexpr int kWarpOBytes = kNC * kHB * kOStride * 4;
+  static constexpr int kWarpOOff = 0;
+  static constexpr int kOSumOff = BAL ? kRingBytes : kWarpOBytes;
+  static constexpr int kRecvOff = 0;
+  static_assert(BAL || kOSumOff + kRPad * kOStride * 4 <= kRingBytes, "warp rows and merged rows must fit in the ring");
+  static_assert(BAL || (kRPad + 16) * (D + 4) * 4 <= kOSumOff, "cluster receive area must not reach the merged rows");
   static constexpr int kQOff = kRingBytes + (BAL ? kRPad * kOStride * 4 : 0);
   static constexpr int kMLOff = kQOff + kQSlots * kQBytes;
   static constexpr int kMLFloats = 2 * kNC * kHB + 2 * kRPad;
@@ -181,7 +196,6 @@ struct Tile {
   static constexpr int kNumFlags = STAGES + 3;     // bad tile per stage, abort, item bad, merge here
   static constexpr int kSmemBytes = 1024 + kFlagOff + 4 * kNumFlags;
   static constexpr int kMinBlocks = STAGES <= 2 ? 3 : (STAGES == 3 ? 2 : 1);
-  static_assert(BAL || kRPad * kOStride * 4 <= kRingBytes, "merge rows must fit in the ring");
 
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -494,28 +508,41 @@ __device__ __forceinline__ void merge_row(const float *part_o, const float *part
   sync();  // the scratch is free for the next row
 }
 
-// Items mode: counts one split's arrival at its (sequence, group, head slice)
-// unit.  The unit's 64-bit word holds {epoch: 40 bits, count: 24 bits}; a word
-// with another epoch (an earlier call, or whatever the workspace held) counts
-// as zero arrivals, so the workspace needs no clearing.  Returns true for the
-// arrival that makes `need`, which also leaves the word at {epoch, 0}, ready
-// for a repeat of the same launch (a replayed CUDA graph keeps its epoch).
-// The compare-and-swap loop always progresses (a failed swap means another
-// arrival succeeded); the bound only guards against a word that keeps
-// changing for some other reason.
+// Items mode: the arrival word of a (sequence, group, head slice) unit with
+// several splits holds {call tag: 40 bits, arrivals: 24 bits}.  Every block of
+// the unit claims the word for its call when it starts: a word with another
+// tag (an earlier call, or whatever the workspace held) is set to {tag, 0} by
+// one compare-and-swap, and a word that already carries the tag is left alone.
+// That happens microseconds before any block of the unit can finish, while the
+// block's first K/V loads are in flight.  At the end every block counts its
+// arrival with one atomic add, so arrivals that come together do not retry;
+// the arrival that makes `need` resets the word to {tag, 0}, ready for a repeat
+// of the same launch (a replayed CUDA graph keeps its tag).  The workspace
+// therefore needs no clearing, and a word poisoned with any other tag is
+// harmless.
+__device__ __forceinline__ void unit_claim(unsigned long long *word, unsigned long long epoch) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(word);
+  for (int i = 0; i < 64 && (cur >> 24) != epoch; ++i) {
+    const unsigned long long prev = atomicCAS(word, cur, epoch << 24);
+    if (prev == cur) return;
+    cur = prev;  // another block of the unit claimed it first (or it changed): look again
+  }
+}
+
+// Counts one split's arrival at its unit (after unit_claim by every block of
+// the unit).  Returns true for the arrival that completes the unit.  A word
+// that does not carry the call's tag (its claim gave up) sets the timeout bit
+// and completes nothing.
 __device__ __forceinline__ bool unit_arrive(unsigned long long *word, unsigned long long epoch, int need,
                                             uint32_t *status) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(word);
-  for (int i = 0; i < (1 << 20); ++i) {
-    const unsigned long long cnt = ((cur >> 24) == epoch) ? (cur & 0xffffffull) : 0ull;
-    const bool last = cnt + 1 == static_cast<unsigned long long>(need);
-    const unsigned long long nxt = (epoch << 24) | (last ? 0ull : cnt + 1);
-    const unsigned long long prev = atomicCAS(word, cur, nxt);
-    if (prev == cur) return last;
-    cur = prev;
+  const unsigned long long old = atomicAdd(word, 1ull);
+  if ((old >> 24) != epoch) {
+    if (status) atomicOr(status, kStatusTimeout);
+    return false;
   }
-  if (status) atomicOr(status, kStatusTimeout);
-  return false;
+  const bool last = (old & 0xffffffull) + 1 == static_cast<unsigned long long>(need);
+  if (last) atomicExch(word, epoch << 24);
+  return last;
 }
 
 // NV float4 outputs (columns 4*c4 .. 4*c4+3 for c4 = c4_0 + i*c4_step, i < NV)
@@ -804,6 +831,28 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // The block's own setup touches only shared memory and the kernel
+  // parameters: it runs before the wait below.
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, nc);
+      tile_bad[i] = 0;
+    }
+    for (int i = 0; i < QS; ++i) {
+      mbar_init(bar_qfull + 8 * i, 1);
+      mbar_init(bar_qempty + 8 * i, nc);
+    }
+    *abort_flag = 0;
+    *item_bad = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == nc && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  __syncthreads();
+
   // Launched as a programmatic dependent of the previous kernel on the stream
   // (items and balanced modes), the blocks may start while it finishes: wait
   // for it to complete (and its memory to be visible) before reading anything
@@ -834,23 +883,11 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       return;
     }
   }
-  if (BAL && threadIdx.x == 0) pdl_launch_dependents();
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(bar_full + 8 * i, 1);
-      mbar_init(bar_empty + 8 * i, nc);
-      tile_bad[i] = 0;
-    }
-    for (int i = 0; i < QS; ++i) {
-      mbar_init(bar_qfull + 8 * i, 1);
-      mbar_init(bar_qempty + 8 * i, nc);
-    }
-    *abort_flag = 0;
-    *item_bad = 0;
-    fence_mbarrier_init();
-  }
-  __syncthreads();
+  if (MODE != Mode::kItems && threadIdx.x == 0) pdl_launch_dependents();
+  // a unit with several splits: claim its arrival word for this call
+  if (MODE == Mode::kItems && threadIdx.x == 0 && p.unit_ctr != nullptr &&
+      (pc.len + p.split_tokens - 1) / p.split_tokens > 1)
+    unit_claim(p.unit_ctr + (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j, p.epoch);
 
   // Every warp walks the same sequence of pieces.
   Walker wk;
@@ -864,10 +901,6 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
 
   if (warp == nc) {
     // =================================================================== producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-    }
     const uint64_t policy = l2_policy_evict_first();
     const int P = p.page_size;
     const int ppt = PAGED ? max(1, T / P) : 1;  // pages per tile
@@ -1203,63 +1236,146 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
           }
         }
       }
-      named_barrier(1, nc * 32);
-      float f[NT][2];
+      if constexpr (BAL) {
+        named_barrier(1, nc * 32);
+        float f[NT][2];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) {
+        for (int j = 0; j < NT; ++j) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int hl = j * 8 + 2 * t4 + e;
-          float M = kNegInf;
+          for (int e = 0; e < 2; ++e) {
+            const int hl = j * 8 + 2 * t4 + e;
+            float M = kNegInf;
 #pragma unroll
-          for (int w2 = 0; w2 < TL::kNWT; ++w2) M = fmaxf(M, m_sm[(hb * TL::kNWT + w2) * TL::kHB + hl]);
-          f[j][e] = (M == kNegInf) ? 0.f : ex2(m_run[j][e] - M);
-        }
-      }
-      // deterministic accumulation: token slice 0 stores, slices 1..3 add in order
-#pragma unroll
-      for (int step = 0; step < TL::kNWT; ++step) {
-        if (ws == step) {
-#pragma unroll
-          for (int mt = 0; mt < TL::kSteps; ++mt) {
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int dim = mt * 16 + g8 + (e >> 1) * 8;
-                const int h = hb * TL::kHB + j * 8 + 2 * t4 + (e & 1);
-                float *dst = osum + h * TL::kOStride + dim;
-                const float v = o[mt][j][e] * f[j][e & 1];
-                *dst = (step == 0) ? v : (*dst + v);
-              }
-            }
+            for (int w2 = 0; w2 < TL::kNWT; ++w2) M = fmaxf(M, m_sm[(hb * TL::kNWT + w2) * TL::kHB + hl]);
+            f[j][e] = (M == kNegInf) ? 0.f : ex2(m_run[j][e] - M);
           }
         }
+        // deterministic accumulation: token slice 0 stores, slices 1..3 add in
+        // order (each adding slice reads all its values before it writes any,
+        // so that the loads are in flight together)
+#pragma unroll
+        for (int step = 0; step < TL::kNWT; ++step) {
+          if (ws == step) {
+            float prev[TL::kSteps][NT][4];
+#pragma unroll
+            for (int mt = 0; mt < TL::kSteps; ++mt)
+#pragma unroll
+              for (int j = 0; j < NT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int dim = mt * 16 + g8 + (e >> 1) * 8;
+                  const int h = hb * TL::kHB + j * 8 + 2 * t4 + (e & 1);
+                  prev[mt][j][e] = (step == 0) ? 0.f : osum[h * TL::kOStride + dim];
+                }
+#pragma unroll
+            for (int mt = 0; mt < TL::kSteps; ++mt)
+#pragma unroll
+              for (int j = 0; j < NT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int dim = mt * 16 + g8 + (e >> 1) * 8;
+                  const int h = hb * TL::kHB + j * 8 + 2 * t4 + (e & 1);
+                  osum[h * TL::kOStride + dim] = prev[mt][j][e] + o[mt][j][e] * f[j][e & 1];
+                }
+          }
+          named_barrier(1, nc * 32);
+        }
+      } else {
+        // each warp's raw O rows into its own region of the ring (once every
+        // warp is done with the last tile); the output pass below merges the
+        // four token slices of every row in one go
         named_barrier(1, nc * 32);
+        float *ow = reinterpret_cast<float *>(smem + TL::kWarpOOff) + warp * TL::kHB * TL::kOStride;
+#pragma unroll
+        for (int mt = 0; mt < TL::kSteps; ++mt)
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              ow[(j * 8 + 2 * t4 + (e & 1)) * TL::kOStride + mt * 16 + g8 + (e >> 1) * 8] = o[mt][j][e];
       }
       }  // mma contraction
-      for (int h = ctid; h < r_pad; h += nc * 32) {
-        const int hb2 = h / TL::kHB, hl = h % TL::kHB;
-        float M = kNegInf;
-        for (int w2 = 0; w2 < TL::kNWT; ++w2) M = fmaxf(M, m_sm[(hb2 * TL::kNWT + w2) * TL::kHB + hl]);
-        float L = 0.f;
-        if (M != kNegInf) {
-          for (int w2 = 0; w2 < TL::kNWT; ++w2) {
-            const int idx = (hb2 * TL::kNWT + w2) * TL::kHB + hl;
-            L += l_sm[idx] * ex2(m_sm[idx] - M);
+      if (FMA > 0 || BAL) {
+        for (int h = ctid; h < r_pad; h += nc * 32) {
+          const int hb2 = h / TL::kHB, hl = h % TL::kHB;
+          float M = kNegInf;
+          for (int w2 = 0; w2 < TL::kNWT; ++w2) M = fmaxf(M, m_sm[(hb2 * TL::kNWT + w2) * TL::kHB + hl]);
+          float L = 0.f;
+          if (M != kNegInf) {
+            for (int w2 = 0; w2 < TL::kNWT; ++w2) {
+              const int idx = (hb2 * TL::kNWT + w2) * TL::kHB + hl;
+              L += l_sm[idx] * ex2(m_sm[idx] - M);
+            }
           }
+          M_blk[h] = M;
+          L_blk[h] = L;
         }
-        M_blk[h] = M;
-        L_blk[h] = L;
       }
       if (MODE == Mode::kCluster && ctid == 0) *item_bad = bad;
       named_barrier(1, nc * 32);
-
       // ---- results of the piece
       if (BAL && ctid == 0) {
         if (pc.first_of_unit)
           p.ws_meta[(static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j] =
               make_int4(static_cast<int>(blockIdx.x), pc.last_block, pc.slot & 1, 0);
+      }
+      constexpr bool kWarpRows = FMA == 0 && !BAL;  // the rows are still per warp (ow)
+      if (kWarpRows) {
+        // ---- one pass over the rows: merge the row's four token slices
+        // (M = max m_w, weights 2^(m_w - M), in slice order: deterministic)
+        // and write the result: final rows, a split's partial state, or
+        // (cluster mode) the block's merged row for the cluster merge
+        const int n4 = D / 4;
+        const bool final_row = MODE == Mode::kItems &&
+                               ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
+        const float *ow = reinterpret_cast<const float *>(smem + TL::kWarpOOff);
+        for (int idx = ctid; idx < pc.nh * n4; idx += nc * 32) {
+          const int h = idx / n4, c4 = idx % n4;
+          const int hb2 = h / TL::kHB, hl = h % TL::kHB;
+          float mw[TL::kNWT];
+          float M = kNegInf;
+#pragma unroll
+          for (int w2 = 0; w2 < TL::kNWT; ++w2) {
+            mw[w2] = m_sm[(hb2 * TL::kNWT + w2) * TL::kHB + hl];
+            M = fmaxf(M, mw[w2]);
+          }
+          float L = 0.f;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int w2 = 0; w2 < TL::kNWT; ++w2) {
+            const int wi = hb2 * TL::kNWT + w2;
+            const float wt = (M == kNegInf) ? 0.f : ex2(mw[w2] - M);
+            const float4 v = *reinterpret_cast<const float4 *>(ow + (wi * TL::kHB + hl) * TL::kOStride + 4 * c4);
+            L += l_sm[wi * TL::kHB + hl] * wt;
+            acc.x += v.x * wt;
+            acc.y += v.y * wt;
+            acc.z += v.z * wt;
+            acc.w += v.w * wt;
+          }
+          if (MODE == Mode::kCluster) {
+            *reinterpret_cast<float4 *>(osum + h * TL::kOStride + 4 * c4) = acc;
+            if (c4 == 0) {
+              M_blk[h] = M;
+              L_blk[h] = L;
+            }
+            continue;
+          }
+          const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
+          if (final_row) {
+            float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!bad && L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
+            reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
+            if (c4 == 0 && p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(M, L);
+            if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLFinal;
+          } else {
+            const size_t ps = row * p.num_splits + pc.k;
+            reinterpret_cast<float4 *>(p.part_o + ps * D)[c4] = acc;
+            if (c4 == 0) {
+              p.part_m[ps] = M;
+              p.part_l[ps] = bad ? kLBadPage : L;
+            }
+          }
+        }
       }
       if (MODE != Mode::kCluster) {
         const int n4 = D / 4;
@@ -1267,7 +1383,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
         // each); fixed splits, split k of the output row ([b, nq, H, S])
         const bool final_row =
             BAL ? pc.final_row : (((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr);
-        for (int idx = ctid; idx < pc.nh * n4; idx += nc * 32) {
+        for (int idx = ctid; !kWarpRows && idx < pc.nh * n4; idx += nc * 32) {
           const int h = idx / n4, c4 = idx % n4;
           const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
           const float4 src = *reinterpret_cast<const float4 *>(osum + h * TL::kOStride + 4 * c4);
@@ -1326,42 +1442,67 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
   }
 
   if (MODE == Mode::kCluster) {
-    // ---- merge the blocks of the cluster through distributed shared memory
+    // ---- merge the blocks of the cluster through distributed shared memory.
+    // Block k of the nb blocks owns rows [k nh / nb, (k + 1) nh / nb).  Once
+    // every block has its merged rows (osum, M_blk, L_blk), each block pushes
+    // each of its rows into the owner's receive area with remote stores (no
+    // round trip waits on them), one cluster barrier makes them visible, and
+    // each owner merges its rows from its own shared memory, the blocks in
+    // rank order (deterministic).  The receive area lies in the ring, past the
+    // merged rows: at the first barrier every block is done with its ring.
+    constexpr int kRS = D + 4;  // receive row: o[D], then M, L, bad
     cg::cluster_group cluster = cg::this_cluster();
+    const int nb = static_cast<int>(cluster.num_blocks());
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int rows_max = (pc.nh + nb - 1) / nb;  // rows per owner, at most
+    float *recv = reinterpret_cast<float *>(smem + TL::kRecvOff);  // [nb][rows_max][kRS]
     cluster.sync();
-    if (cluster.block_rank() == 0) {
-      const int nb = static_cast<int>(cluster.num_blocks());
-      int bad = 0;
-      if (pc.len_ok)
-        for (int c = 0; c < nb; ++c) bad |= *cluster.map_shared_rank(const_cast<int *>(item_bad), c);
-      const int n4 = D / 4;
-      for (int idx = threadIdx.x; idx < pc.nh * n4; idx += blockDim.x) {
-        const int h = idx / n4, c4 = idx % n4;
-        float L = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (pc.len_ok && !bad) {
-          float M = kNegInf;
-          for (int c = 0; c < nb; ++c) M = fmaxf(M, *cluster.map_shared_rank(M_blk + h, c));
-          for (int c = 0; c < nb; ++c) {
-            const float Mc = *cluster.map_shared_rank(M_blk + h, c);
-            if (Mc == kNegInf) continue;  // a block without tokens
-            const float wgt = ex2(Mc - M);
-            L += *cluster.map_shared_rank(L_blk + h, c) * wgt;
-            const float *src = cluster.map_shared_rank(osum + h * TL::kOStride + 4 * c4, c);
-            acc.x += src[0] * wgt;
-            acc.y += src[1] * wgt;
-            acc.z += src[2] * wgt;
-            acc.w += src[3] * wgt;
-          }
-        }
-        float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
-        const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
-        reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
-      }
-      if (threadIdx.x == 0 && !pc.len_ok && p.status) atomicOr(p.status, kStatusBadSeqlen);
+    const int n4 = D / 4;
+    const float bad_mine = static_cast<float>(*item_bad);
+    for (int idx = threadIdx.x; idx < pc.nh * (n4 + 1); idx += blockDim.x) {
+      const int h = idx / (n4 + 1), part = idx % (n4 + 1);
+      const int k = (h * nb + nb - 1) / pc.nh;  // owner: the largest k with k nh / nb <= h
+      const int k_own = (k * pc.nh / nb > h) ? k - 1 : k;
+      const int r_lo_k = k_own * pc.nh / nb;
+      float *dst = cluster.map_shared_rank(recv, k_own) + (rank * rows_max + (h - r_lo_k)) * kRS;
+      if (part < n4)
+        reinterpret_cast<float4 *>(dst)[part] = *reinterpret_cast<const float4 *>(osum + h * TL::kOStride + 4 * part);
+      else
+        reinterpret_cast<float4 *>(dst)[n4] = make_float4(M_blk[h], L_blk[h], bad_mine, 0.f);
     }
     cluster.sync();
+    const int r_lo = rank * pc.nh / nb, r_hi = (rank + 1) * pc.nh / nb;
+    for (int idx = threadIdx.x; idx < (r_hi - r_lo) * n4; idx += blockDim.x) {
+      const int hr = idx / n4, c4 = idx % n4;
+      float M = kNegInf;
+      bool bad = false;
+      for (int c = 0; c < nb; ++c) {
+        const float4 meta = reinterpret_cast<const float4 *>(recv + (c * rows_max + hr) * kRS)[n4];
+        M = fmaxf(M, meta.x);
+        bad |= meta.z != 0.f;
+      }
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (pc.len_ok && !bad && M != kNegInf) {
+        for (int c = 0; c < nb; ++c) {
+          const float *src = recv + (c * rows_max + hr) * kRS;
+          const float4 meta = reinterpret_cast<const float4 *>(src)[n4];
+          if (meta.x == kNegInf) continue;  // a block without tokens contributes nothing
+          const float wgt = ex2(meta.x - M);
+          const float4 v = reinterpret_cast<const float4 *>(src)[c4];
+          L += meta.y * wgt;
+          acc.x += v.x * wgt;
+          acc.y += v.y * wgt;
+          acc.z += v.z * wgt;
+          acc.w += v.w * wgt;
+        }
+      }
+      float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
+      const size_t row = row_of(p, pc.s, pc.g, pc.h0 + r_lo + hr);
+      reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
+    }
+    if (rank == 0 && threadIdx.x == 0 && !pc.len_ok && p.status) atomicOr(p.status, kStatusBadSeqlen);
   }
 }
 

@@ -58,8 +58,9 @@ struct TcTile {
   static constexpr int kBarOff = kQOff + 2 * kQHalf;
   static constexpr int kSP = 3;                        // S/P buffers in tensor memory
   // full[kStages], empty[kStages], s_full[kSP], p_full[kSP], pv_done[kSP],
-  // drain[2] (one per MMA issuer: all its products done before teardown)
-  static constexpr int kNumBars = 2 * kStages + 3 * kSP + 2;
+  // drain[2] (one per MMA issuer: all its products done before teardown),
+  // q_full (Q written to shared memory)
+  static constexpr int kNumBars = 2 * kStages + 3 * kSP + 3;
   static constexpr int kXOff = kBarOff + 8 * kNumBars;  // the halves' bases at the end: [2][kM] floats
   static constexpr int kLOff = kXOff + 4 * 2 * kM;      // the halves' sums at the end: [2][kM] floats
   static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[kStages], abort, merge here
@@ -158,7 +159,222 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap *tm_k, const CUtens
   }
 }
 
+// The block whose split completes the unit merges the unit's splits (as in
+// the mma.sync kernel): the 256 softmax threads, two float4 columns of one row
+// each.  Called by all of them, after their partial states are written.
+__device__ __forceinline__ void tc_merge_unit(const DecodeParams &p, const Piece &pc, int sm,
+                                              volatile int *merge_here) {
+  constexpr int D = TcTile::kD;
+  constexpr int kSM = 32 * TcTile::kSoftmaxWarps;
+  named_barrier(1, kSM);
+  const int ns = (pc.len + p.split_tokens - 1) / p.split_tokens;
+  if (sm == 0) {
+    __threadfence();
+    const size_t u = (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j;
+    *merge_here = unit_arrive(p.unit_ctr + u, p.epoch, ns, p.status) ? 1 : 0;
+    __threadfence();
+  }
+  named_barrier(1, kSM);
+  if (*merge_here) {
+    constexpr int kHalfRow = D / 8;  // two float4 columns per thread, half a row apart
+    for (int rb = 0; rb < pc.nh; rb += kSM / kHalfRow) {
+      const int h = rb + sm / kHalfRow, c4 = sm % kHalfRow;
+      if (h < pc.nh) {
+        const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
+        merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns, c4,
+                           kHalfRow, reinterpret_cast<float4 *>(p.out + mrow * D), p.lse ? p.lse + mrow : nullptr);
+      }
+    }
+  }
+}
+
+// Softmax warps with at most 64 rows (SPREAD): quarter qd = warp % 4 of the
+// tensor-memory lanes holds rows qd * rpq .. in its first rpq <= 16 lanes
+// (rpq = ceil(rows / 4)).  Warp w takes tokens [32 h, 32 h + 32) of every
+// tile, h = w / 4, and within it thread t the 16 tokens [32 h + 16 (t / 16),
+// + 16) of lane t % 16 (the 16x32bx2 shape).  The two threads of a row in one
+// warp share its running base (their maximum meets through one shuffle) and
+// the row's O_h in tensor memory; the two warps of a quarter keep separate
+// states and O_h, merged once at the end.  P's high part goes over the
+// thread's first 8 score columns, its residual over the next 8.
 template <bool PAGED>
+__device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const Piece &pc, uint8_t *smem,
+                                                  uint32_t tmem, uint32_t s_full0, uint32_t p_full0,
+                                                  uint32_t pv_done0, volatile int *tile_bad,
+                                                  volatile int *abort_flag, volatile int *merge_here, int n_tiles,
+                                                  int warp, int lane) {
+  using TT = TcTile;
+  constexpr int D = TT::kD;
+  constexpr int T = TT::kT;
+  constexpr int ST = TT::kStages;
+  constexpr int SP = TT::kSP;
+  constexpr int kSM = 32 * TT::kSoftmaxWarps;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  const int sm = threadIdx.x;
+  const int qd = warp % 4;                 // lane quarter
+  const int half = warp / 4;               // tokens [32 half, 32 half + 32) of every tile
+  const int sub = lane >> 4;               // ... of which [16 sub, 16 sub + 16)
+  const int li = lane & 15;                // lane within the quarter
+  const int rpq = (pc.nh + 3) / 4;         // rows per quarter
+  const int rho = qd * rpq + li;           // row of the slice
+  const bool valid = li < rpq && rho < pc.nh;
+  const bool warp_active = qd * rpq < pc.nh;
+  const int slot = qd * 32 + li;           // tensor-memory lane of the row
+  // the positions this row sees (a padding slot sees the whole piece: its
+  // scores are 0 and its result unused)
+  const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + rho) / p.r)) : pc.t_end;
+  const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+  float *mbase = reinterpret_cast<float *>(smem + TT::kXOff);  // [half][slot]
+  float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);   // [half][slot]
+  const float sl = p.scale_log2;
+  float m_run = kNegInf, l_run = 0.f;  // this half's base (shared by the pair) and this thread's sum
+  int bad = 0;
+  bool ok = true;
+  for (int t = 0; t < n_tiles; ++t) {
+    const int t0 = pc.t_begin + t * T;
+    const int st = t % ST;
+    const int b = t % SP;
+    ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (t / SP) & 1));
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t sv[16];
+    tc_ld16x2_x16<16>(lane_tmem + b * 64 + half * 32, sv);
+    tc_wait_ld();
+    if (PAGED) bad |= tile_bad[st];
+    // V rows past the piece's end may hold anything (even NaN): zero them so
+    // that P = 0 there meets zeros
+    const int valid_rows = min(T, pc.t_end - t0);
+    if (valid_rows < T) {
+      uint8_t *vt = smem + st * TT::kStageBytes + TT::kTileBytes;
+      for (int idx = sm; idx < (T - valid_rows) * 16; idx += kSM) {
+        const int row = valid_rows + idx / 16, c = idx % 16;
+        *reinterpret_cast<uint4 *>(vt + (c >> 3) * TT::kHalf + row * 128 + ((c & 7) << 4)) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    float x[16];
+    const int tb = t0 + half * 32 + sub * 16;  // this thread's first token of the tile
+    if (tb + 16 <= lim) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[j] = __uint_as_float(sv[j]) * sl;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
+    }
+    float mx;
+    {
+      float m4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) m4[k] = fmaxf(fmaxf(x[4 * k], x[4 * k + 1]), fmaxf(x[4 * k + 2], x[4 * k + 3]));
+      mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the row's other 16 tokens of this half
+    if (warp_active) {
+      // lazy rescale: only when a score passes the base by more than 2^8 (the
+      // same decision in both threads of the row)
+      const bool need = mx > m_run + 8.f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float mn = need ? fmaxf(m_run, mx) : m_run;
+        const float alpha = need ? ((m_run == kNegInf) ? 0.f : ex2(m_run - mn)) : 1.f;
+        l_run *= alpha;
+        if (t > 0) {
+          // O_h holds tiles 0 .. t-1: rescale it once their MMAs are done;
+          // thread sub takes columns [64 sub, 64 sub + 64) of the row
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((t - 1) % SP), ((t - 1) / SP) & 1));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t ov[32];
+            tc_ld16x2_x32<64>(lane_tmem + TT::kOCol + half * D + c * 32, ov);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+            tc_st16x2_x32<64>(lane_tmem + TT::kOCol + half * D + c * 32, ov);
+          }
+          tc_wait_st();
+          tc_fence_before();
+        }
+        m_run = mn;
+      }
+      const float base = (m_run == kNegInf) ? 0.f : m_run;
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
+        l_run += p0 + p1;
+        split_bf16x2_rz(p0, p1, hi[e], lo[e]);
+      }
+      tc_st16x2_x8<16>(lane_tmem + b * 64 + half * 32, hi);
+      tc_st16x2_x8<16>(lane_tmem + b * 64 + half * 32 + 8, lo);
+      tc_wait_st();
+    }
+    tc_fence_before();
+    if (valid_rows < T) fence_proxy_async_smem();  // the zeroed V rows, for the tensor core
+    __syncwarp();
+    if (lane == 0) mbar_arrive(p_full0 + 8 * b);
+  }
+  if (!ok && lane == 0) {
+    *abort_flag = 1;
+    if (p.status) atomicOr(p.status, kStatusTimeout);
+  }
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);  // the half's sum of the row
+  // ---- the row's result: O from tensor memory once the last MMAs are done
+  const bool done =
+      ok && __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((n_tiles - 1) % SP), ((n_tiles - 1) / SP) & 1));
+  tc_fence_after();
+  if (sub == 0) {
+    mbase[half * 128 + slot] = m_run;
+    lsum[half * 128 + slot] = l_run;
+  }
+  named_barrier(1, kSM);
+  const float m0 = mbase[slot], m1 = mbase[128 + slot];
+  const float m_row = fmaxf(m0, m1);
+  const float w0 = (m0 == kNegInf) ? 0.f : ex2(m0 - m_row), w1 = (m1 == kNegInf) ? 0.f : ex2(m1 - m_row);
+  const float l_row = lsum[slot] * w0 + lsum[128 + slot] * w1;
+  const bool final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
+  const size_t row = valid ? row_of(p, pc.s, pc.g, pc.h0 + rho) : 0;
+  const size_t ps = row * p.num_splits + pc.k;
+  const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
+  const float s0 = final_row ? w0 * inv : w0, s1 = final_row ? w1 * inv : w1;
+  {
+    // this thread writes columns [64 half + 32 sub, + 32) of the row
+    uint32_t oa[32], ob[32];
+    tc_ld16x2_x32<32>(lane_tmem + TT::kOCol + half * 64, oa);
+    tc_ld16x2_x32<32>(lane_tmem + TT::kOCol + D + half * 64, ob);
+    tc_wait_ld();
+    if (valid) {
+      const int col = half * 64 + sub * 32;
+      float4 *dst = reinterpret_cast<float4 *>((final_row ? p.out + row * D : p.part_o + ps * D) + col);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = __uint_as_float(oa[4 * j + e]) * s0 + __uint_as_float(ob[4 * j + e]) * s1;
+        dst[j] = make_float4(v[0], v[1], v[2], v[3]);
+      }
+    }
+  }
+  if (valid && half == 0 && sub == 0) {
+    if (final_row) {
+      if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_row, l_row);
+      if (p.part_l) p.part_l[row * p.num_splits] = kLFinal;
+    } else {
+      p.part_m[ps] = m_row;
+      p.part_l[ps] = bad ? kLBadPage : l_row;
+    }
+  }
+  tc_fence_before();
+  if (p.unit_ctr != nullptr && !final_row) tc_merge_unit(p, pc, sm, merge_here);
+}
+
+// SPREAD (at most 64 rows): the rows sit in the first 16 lanes of each of the
+// four tensor-memory lane quarters, ceil(rows / 4) per quarter, so that the
+// softmax work is shared by all four SM sub-partitions; four threads take
+// each row (two warps, 16 tokens each of their 32), through the 16-lane
+// tensor-memory shapes.  Otherwise (up to 128 rows) row i is lane i and two
+// threads take each row.
+template <bool PAGED, bool SPREAD>
 __global__ void __launch_bounds__(TcTile::kThreads, 1)
     gqa_verify_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const DecodeParams p) {
@@ -178,6 +394,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   const uint32_t s_full0 = bars + 16 * ST;
   const uint32_t p_full0 = s_full0 + 8 * SP, pv_done0 = p_full0 + 8 * SP;
   const uint32_t drain0 = pv_done0 + 8 * SP;  // [2]: the Q K^T issuer's, the P.V issuer's
+  const uint32_t q_full = drain0 + 16;
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
   volatile int *abort_flag = tile_bad + ST;
@@ -185,26 +402,10 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  pdl_wait_primary();
-  const Piece pc = make_item<T, Mode::kItems>(p);
-  if (threadIdx.x == 0) pdl_launch_dependents();
-  if (pc.nh <= 0) return;
-  if (pc.t_begin >= pc.t_end) {
-    // nothing to read; an invalid length is handled once, by split 0
-    if (!pc.len_ok && pc.k == 0) {
-      const bool empty = p.empty_ok && pc.len == 0;
-      for (int idx = threadIdx.x; idx < pc.nh * (D / 4); idx += blockDim.x) {
-        const int h = idx / (D / 4), c4 = idx % (D / 4);
-        const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
-        if (p.out) reinterpret_cast<float4 *>(p.out + row * D)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLBadLength;
-        if (c4 == 0 && p.lse) p.lse[row] = kNegInf;
-      }
-      if (threadIdx.x == 0 && p.status && !empty) atomicOr(p.status, kStatusBadSeqlen);
-    }
-    return;
-  }
-
+  // The block's own setup (barriers, tensor memory) touches no global memory:
+  // it runs before the wait for the previous kernel on the stream.
+  constexpr int kProducerWarp = TT::kSoftmaxWarps;  // then the Q K^T issuer (allocates), the P.V issuer
+  constexpr int kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
       mbar_init(full0 + 8 * i, 1);
@@ -218,21 +419,60 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     }
     mbar_init(drain0, 1);
     mbar_init(drain0 + 8, 1);
+    mbar_init(q_full, 128);  // one arrival per Q row
     *abort_flag = 0;
     *merge_here = 0;
     fence_mbarrier_init();
   }
-  constexpr int kProducerWarp = TT::kSoftmaxWarps;  // then the Q K^T issuer (allocates), the P.V issuer
-  constexpr int kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
   if (warp == kMmaWarp) {
     tc_alloc(smem_addr(const_cast<uint32_t *>(tmem_slot)), TT::kTmemCols);
     tc_relinquish();
   }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  pdl_wait_primary();
+  const Piece pc = make_item<T, Mode::kItems>(p);
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  if (pc.nh <= 0 || pc.t_begin >= pc.t_end) {
+    // nothing to read; an invalid length is handled once, by split 0
+    if (pc.nh > 0 && !pc.len_ok && pc.k == 0) {
+      const bool empty = p.empty_ok && pc.len == 0;
+      for (int idx = threadIdx.x; idx < pc.nh * (D / 4); idx += blockDim.x) {
+        const int h = idx / (D / 4), c4 = idx % (D / 4);
+        const size_t row = row_of(p, pc.s, pc.g, pc.h0 + h);
+        if (p.out) reinterpret_cast<float4 *>(p.out + row * D)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c4 == 0 && p.part_l) p.part_l[row * p.num_splits] = kLBadLength;
+        if (c4 == 0 && p.lse) p.lse[row] = kNegInf;
+      }
+      if (threadIdx.x == 0 && p.status && !empty) atomicOr(p.status, kStatusBadSeqlen);
+    }
+    if (warp == kMmaWarp) tc_dealloc(tmem, TT::kTmemCols);
+    return;
+  }
+  // a unit with several splits: claim its arrival word for this call
+  if (threadIdx.x == 0 && p.unit_ctr != nullptr && (pc.len + p.split_tokens - 1) / p.split_tokens > 1)
+    unit_claim(p.unit_ctr + (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j, p.epoch);
   if (threadIdx.x < 128) {
-    // this thread's q row into Q (128-byte swizzle, two 64-column halves); padding rows are zero
+    // the q row of this thread's slot into Q (128-byte swizzle, two 64-column
+    // halves; padding slots are zero), while the producer already streams
+    // K and V; the Q K^T issuer waits for all 128 slots
     const int r = threadIdx.x;
-    const bool valid = r < pc.nh;
-    const uint4 *src = valid ? reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + r) * D) : nullptr;
+    int rho = r;  // the row of the slice held by slot r
+    bool valid = r < pc.nh;
+    if (SPREAD) {
+      const int rpq = (pc.nh + 3) / 4, li = r % 32;
+      rho = (r / 32) * rpq + li;
+      valid = li < rpq && rho < pc.nh;
+    }
+    const uint4 *src =
+        valid ? reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + rho) * D) : nullptr;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
@@ -240,11 +480,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       *reinterpret_cast<uint4 *>(smem + TT::kQOff + h * TT::kQHalf + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
     }
     fence_proxy_async_smem();
+    mbar_arrive(q_full);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
   const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
 
   if (warp == kProducerWarp) {
@@ -260,8 +497,8 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
         qd[ks] = tc_smem_desc(sbase + TT::kQOff + (ks >> 2) * TT::kQHalf + (ks & 3) * 32, 16, 1024);
-      bool ok = true;
-      for (int t = 0; t < n_tiles; ++t) {
+      bool ok = mbar_wait(q_full, 0);
+      for (int t = 0; ok && t < n_tiles; ++t) {
         // ---- S[t % SP] = Q K_t^T once K_t has landed and the buffer's last P.V is done
         const int st = t % ST;
         ok = mbar_wait(full0 + 8 * st, (t / ST) & 1);
@@ -303,11 +540,13 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
           // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of
           // the buffer, the residual 16 columns further; into the O of the
           // half of the row that owns them
+          // (SPREAD: the thread of tokens 16 ks .. wrote its high part at
+          // column 16 ks and its residual 8 columns further)
           const uint64_t vdk = vd + ((ks * 16 * 128) >> 4);
-          const uint32_t pa = pb + 32 * (ks >> 1) + 8 * (ks & 1);
+          const uint32_t pa = SPREAD ? pb + 16 * ks : pb + 32 * (ks >> 1) + 8 * (ks & 1);
           const uint32_t od = tmem + TT::kOCol + D * (ks >> 1);
           tc_mma_ts(od, pa, vdk, kIdescPV, (u > 0 || (ks & 1)) ? 1u : 0u);
-          tc_mma_ts(od, pa + 16, vdk, kIdescPV, 1u);
+          tc_mma_ts(od, pa + (SPREAD ? 8 : 16), vdk, kIdescPV, 1u);
         }
         // K_u was read by the scores of tile u, done before its P existed; V_u
         // and P_u by these products
@@ -321,6 +560,10 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       tc_commit(drain0 + 8);
       if (!mbar_wait(drain0 + 8, 0) && p.status) atomicOr(p.status, kStatusTimeout);
     }
+  } else if (SPREAD) {
+    // ============================================================ softmax rows, spread
+    tc_softmax_spread<PAGED>(p, pc, smem, tmem, s_full0, p_full0, pv_done0, tile_bad, abort_flag, merge_here,
+                             n_tiles, warp, lane);
   } else {
     // ============================================================ softmax rows
     constexpr int kSM = 32 * TT::kSoftmaxWarps;  // softmax threads
@@ -481,31 +724,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
       }
     }
     tc_fence_before();
-    if (p.unit_ctr != nullptr && !final_row) {
-      // ---- the block whose split completes the unit merges its splits (as
-      // in the mma.sync kernel)
-      named_barrier(1, kSM);
-      const int ns = (pc.len + p.split_tokens - 1) / p.split_tokens;
-      if (sm == 0) {
-        __threadfence();
-        const size_t u = (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j;
-        *merge_here = unit_arrive(p.unit_ctr + u, p.epoch, ns, p.status) ? 1 : 0;
-        __threadfence();
-      }
-      named_barrier(1, kSM);
-      if (*merge_here) {
-        constexpr int kHalfRow = D / 8;  // two float4 columns per thread, half a row apart
-        for (int rb = 0; rb < pc.nh; rb += kSM / kHalfRow) {
-          const int h = rb + sm / kHalfRow, c4 = sm % kHalfRow;
-          if (h < pc.nh) {
-            const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
-            merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns,
-                               c4, kHalfRow, reinterpret_cast<float4 *>(p.out + mrow * D),
-                               p.lse ? p.lse + mrow : nullptr);
-          }
-        }
-      }
-    }
+    if (p.unit_ctr != nullptr && !final_row) tc_merge_unit(p, pc, sm, merge_here);
   }
 
   // ---- teardown: every tensor-memory access is done before the columns go
