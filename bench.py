@@ -237,10 +237,13 @@ def config_dict(w, inp, n_query=1):
     return cfg
 
 
-def plan_dict(split_tokens, max_len, n_query=1, tc=False, entry="split"):
+def plan_dict(split_tokens, max_len, n_query=1, tc=False, entry="split", cluster=0):
     """The library's decomposition of a step (GPU arm only)."""
     if entry == "cluster":
         decomp = "gqa_decode: one block or cluster per (sequence, group)"
+    elif cluster > 1:
+        decomp = ("thread-block clusters of %d blocks per (sequence, group), merged through distributed shared "
+                  "memory (one kernel)" % cluster)
     elif split_tokens == 0:
         decomp = "equal-work ranges over all (sequence, group) tiles (stream-K) + combine"
     else:
@@ -249,6 +252,8 @@ def plan_dict(split_tokens, max_len, n_query=1, tc=False, entry="split"):
             split_tokens, n_splits, "one block per (sequence, group), final rows" if n_splits == 1 else
             "merged in the decode kernel" if n_splits <= 8 else "combine kernel")
     d = {"split_tokens": split_tokens, "decomposition": decomp}
+    if cluster > 1:
+        d["cluster_blocks"] = cluster
     if n_query > 1:
         d["kernel"] = "gqa_verify_tc_kernel (tcgen05)" if tc else "gqa_decode_kernel (mma.sync)"
     return d
@@ -375,21 +380,27 @@ class Case:
         self.dims = gqa.dims_for(inp.q, inp.k_cache, inp.page_table)
         # 0: the library's choice (equal-work ranges for a paged cache); > 0:
         # fixed splits of that many tokens; -1: the library's plan
-        split = args.split_tokens
-        if nq > 1 and split <= 0:
-            split = -(-self.max_seqlen // 256) * 256  # verification runs fixed splits: one per sequence
-        if split < 0:
-            split = 0
+        split = max(0, args.split_tokens)
         self.split = split
         if nq == 1:
             self.ws = gqa.workspace_for(inp.q, inp.k_cache, inp.page_table, self.max_seqlen, split)
         else:
             n = gqa.gqa_decode_verify_workspace_size(self.dims, nq, self.max_seqlen, split)
             self.ws = torch.empty(max(256, n), dtype=torch.uint8, device="cuda")
-        self.eff_split = split if split > 0 else gqa.gqa_plan_split_tokens(self.dims, self.max_seqlen)
-        n_splits = -(-self.max_seqlen // self.eff_split) if self.eff_split > 0 else 0
-        self.launches_per_step = 1 if (self.entry == "cluster" or 0 < n_splits <= gqa.SERIAL_MERGE_MAX_SPLITS) else 2
+        self.cluster = 0
         self.tc = nq * w.r > gqa.TC_AUTO_ROWS and w.d == 128
+        if split > 0:
+            self.eff_split = split
+        elif nq == 1 and self.entry == "split":
+            kind, self.eff_split, c = gqa.gqa_plan_decomposition(self.dims, self.max_seqlen)
+            self.cluster = c if kind == gqa.PLAN_CLUSTERS else 0
+        elif self.tc:
+            self.eff_split = 0  # the tcgen05 kernel: equal-work ranges
+        else:
+            self.eff_split = gqa.gqa_plan_split_tokens(self.dims, self.max_seqlen)
+        n_splits = -(-self.max_seqlen // self.eff_split) if self.eff_split > 0 else 0
+        self.launches_per_step = 1 if (self.entry == "cluster" or self.cluster > 1 or
+                                       0 < n_splits <= gqa.SERIAL_MERGE_MAX_SPLITS) else 2
         self.out = torch.empty(self.q.shape, dtype=torch.float32, device="cuda")
         self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.how, n_copies = l2_plan(self.kv_step)
@@ -420,6 +431,9 @@ class Case:
         """The decode kernel alone (the step without its combine launch)."""
         k, v = self.caches[self.i % len(self.caches)]
         self.i += 1
+        if self.nq > 1:  # no two-kernel entry point for verification: the whole step
+            self.step()
+            return
         self.gqa.gqa_split_partials(self.inp.q, k, v, self.inp.seqlens, self.inp.page_table,
                                     split_tokens=self.split, max_seqlen=self.max_seqlen, workspace=self.ws,
                                     out=self.out, status=self.status)
@@ -473,7 +487,7 @@ class Case:
         """The dominant kernel (the decode kernel) alone: mean of isolated
         launches between CUDA events on its stream, L2 flushed first when the
         cache fits in it; for a one-launch step that is the step itself."""
-        kern = self.step if (self.launches_per_step == 1 or self.nq > 1) else self.decode_only
+        kern = self.step if self.launches_per_step == 1 else self.decode_only
         stream = torch.cuda.current_stream()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(max(steps, 10))]
@@ -488,18 +502,24 @@ class Case:
         return max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
 
     def kernel_name(self):
+        tc_name = "gqa_verify_tc_balanced_kernel" if self.eff_split == 0 else "gqa_verify_tc_kernel"
         if self.nq > 1:
             return "%s (verification, %d rows per KV group%s)" % (
-                "gqa_verify_tc_kernel" if self.tc else "gqa_decode_kernel", self.nq * self.w.r,
+                tc_name if self.tc else "gqa_decode_kernel", self.nq * self.w.r,
                 "" if self.launches_per_step == 1 else "; decode + combine timed together")
+        if self.tc:
+            return "%s (%d rows per KV group)" % (tc_name, self.w.r)
         if self.entry == "split":
+            if self.cluster > 1:
+                return "gqa_decode_kernel (thread-block clusters of %d, merged in distributed shared memory)" % (
+                    self.cluster)
             if self.eff_split == 0:
                 return "gqa_decode_kernel (equal-work ranges)"
             return "gqa_decode_kernel (fixed splits%s)" % (", merged in-kernel" if self.launches_per_step == 1 else "")
         return "gqa_decode_kernel (gqa_decode)"
 
     def plan(self):
-        return plan_dict(self.eff_split, self.max_seqlen, self.nq, self.tc, self.entry)
+        return plan_dict(self.eff_split, self.max_seqlen, self.nq, self.tc, self.entry, self.cluster)
 
     def free(self):
         self.caches = []

@@ -157,7 +157,10 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
  *               second kernel merges (longer paged batches: splits of 4096).
  *               Contiguous dims (max_pages_per_seq == 0) get fixed splits:
  *               one per unit when the units fill at least three quarters of
- *               the GPU's resident blocks (no combine), else as many splits
+ *               the GPU's resident blocks (no combine); with too few units
+ *               for that, gqa_decode_split (one query token, no lse) runs
+ *               thread-block clusters when they fill the GPU (see
+ *               gqa_plan_decomposition); otherwise as many splits
  *               per unit as still fit one wave of resident blocks.
  * max_seqlen:   an upper bound of every seqlens[s] (sizes the grid and the
  *               workspace); a length above it is treated as invalid
@@ -317,12 +320,36 @@ int gqa_merge_lse(const float *o_parts, const float *lse_parts, int32_t n_parts,
                   int32_t head_dim, float *out, float *lse_out, void *stream);
 
 /*
- * The decomposition gqa_decode_split (and the pair gqa_split_partials /
- * gqa_split_combine) uses when split_tokens == 0: 0 for equal-work ranges, or
- * the fixed split length (a positive multiple of 128) it falls back to.
- * num_sms <= 0 queries the current device.  A negative value is a GQA_ERR_* code.
+ * The decomposition the pair gqa_split_partials / gqa_split_combine uses
+ * when split_tokens == 0 (and gqa_decode_split, unless gqa_plan_decomposition
+ * says GQA_PLAN_CLUSTERS): 0 for equal-work ranges, or the fixed split length
+ * (a positive multiple of 128) it falls back to.  num_sms <= 0 queries the
+ * current device.  A negative value is a GQA_ERR_* code.
  */
 int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms);
+
+/*
+ * The decomposition gqa_decode_split runs with split_tokens == 0 for one
+ * query token per sequence (gqa_decode_split_lse, gqa_decode_verify and
+ * gqa_decode_split_mapped never take the cluster one):
+ *   GQA_PLAN_EQUAL_WORK    equal-work ranges + combine kernel (paged dims);
+ *   GQA_PLAN_FIXED_SPLITS  fixed splits of *split_tokens_out tokens, merged in
+ *                          the decode kernel (<= 8 splits) or by the combine;
+ *   GQA_PLAN_CLUSTERS      a contiguous cache with too few (sequence, group)
+ *                          units to fill the GPU one block each: the cluster
+ *                          decomposition of gqa_decode, *cluster_out blocks per
+ *                          thread-block cluster (<= 8) sharing each unit's
+ *                          tokens and merging through distributed shared
+ *                          memory, one kernel and no workspace (the workspace
+ *                          passed is not touched).
+ * split_tokens_out / cluster_out may be NULL.  num_sms <= 0 queries the
+ * current device.  A negative value is a GQA_ERR_* code.
+ */
+#define GQA_PLAN_EQUAL_WORK 0
+#define GQA_PLAN_FIXED_SPLITS 1
+#define GQA_PLAN_CLUSTERS 2
+int32_t gqa_plan_decomposition(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms,
+                               int32_t *split_tokens_out, int32_t *cluster_out);
 
 /*
  * gqa_decode_split_static -- gqa_decode_split without a caller-provided

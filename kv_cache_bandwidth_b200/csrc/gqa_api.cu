@@ -397,6 +397,43 @@ int launch_verify_tc(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &
   return cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// The tcgen05 kernel on equal-work ranges: one persistent block per SM
+// (grid.x holds the SM count on entry); returns the number of blocks.
+constexpr int kMaxBalancedBlocksTc = 256;
+
+int launch_tc_balanced(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p,
+                       const Launch &l) {
+  const bool spread = sh.rc <= 64;
+  auto kernel = sh.paged ? (spread ? gqa::gqa_verify_tc_balanced_kernel<true, true>
+                                   : gqa::gqa_verify_tc_balanced_kernel<true, false>)
+                         : (spread ? gqa::gqa_verify_tc_balanced_kernel<false, true>
+                                   : gqa::gqa_verify_tc_balanced_kernel<false, false>);
+  constexpr int smem = gqa::TcBalTile::kSmemBytes;
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load(std::memory_order_acquire) & bit)) {
+    for (auto k : {gqa::gqa_verify_tc_balanced_kernel<true, true>, gqa::gqa_verify_tc_balanced_kernel<true, false>,
+                   gqa::gqa_verify_tc_balanced_kernel<false, true>, gqa::gqa_verify_tc_balanced_kernel<false, false>})
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    attr_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min<unsigned>(l.grid.x, kMaxBalancedBlocksTc), 1, 1);
+  cfg.blockDim = dim3(gqa::TcBalTile::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) != cudaSuccess) return GQA_ERR_CUDA;
+  return static_cast<int>(cfg.gridDim.x);
+}
+
 int encode_maps(const Shape &sh, const void *k, const void *v, CUtensorMap *tk, CUtensorMap *tv) {
   const int T = tile_tokens(sh);
   const int rows = sh.P;  // paged: page size; contiguous: capacity m
@@ -498,7 +535,7 @@ struct BalancedWorkspace {
 
 BalancedWorkspace balanced_layout(const Shape &sh) {
   BalancedWorkspace w;
-  const size_t rows = static_cast<size_t>(kMaxBalancedBlocks) * 2 * sh.rc;
+  const size_t rows = static_cast<size_t>(sh.tc ? kMaxBalancedBlocksTc : kMaxBalancedBlocks) * 2 * sh.rc;
   w.meta_off = 256;
   w.o_off = w.meta_off + round256(static_cast<size_t>(units_of(sh)) * 16);
   w.m_off = w.o_off + round256(rows * sh.D * sizeof(float));
@@ -537,7 +574,7 @@ int run_balanced_decode(const Shape &sh, int sms, const void *q, const void *k, 
   p.lse = ex.lse;
   p.empty_ok = ex.empty_ok ? 1 : 0;
   Launch l{dim3(static_cast<unsigned>(sms), 1, 1), 1, stream};
-  rc = launch_decode<Mode::kBalanced>(sh, tk, tv, p, l);
+  rc = sh.tc ? launch_tc_balanced(sh, tk, tv, p, l) : launch_decode<Mode::kBalanced>(sh, tk, tv, p, l);
   return rc < 0 ? rc : GQA_OK;
 }
 
@@ -593,9 +630,10 @@ struct AutoChoice {
 
 bool dims_paged(const gqa_dims *dims) { return dims->max_pages_per_seq > 0; }
 
-// Equal-work ranges serve paged dims, with neither a group table nor the
-// tcgen05 kernel (both run on fixed splits only).
-bool balanced_ok(const gqa_dims *dims, const Shape &sh) { return dims_paged(dims) && !sh.mapped && !sh.tc; }
+// Equal-work ranges serve paged dims, and the tcgen05 kernel in either
+// layout (its persistent blocks would otherwise run units in waves of one
+// block per SM); a group table runs on fixed splits only.
+bool balanced_ok(const gqa_dims *dims, const Shape &sh) { return (dims_paged(dims) || sh.tc) && !sh.mapped; }
 
 int round_split(long long tokens) {
   tokens = (tokens + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
@@ -626,6 +664,23 @@ AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
   const long long slots = static_cast<long long>(sms) * blocks_per_sm(sh);
   const long long splits = 4 * units >= 3 * slots ? 1 : std::max<long long>(1, slots / units);
   return {false, round_split((max_seqlen + splits - 1) / splits)};
+}
+
+// split_tokens == 0 in gqa_decode_split: a contiguous cache whose (sequence,
+// group) units are too few to fill the GPU one block each runs the cluster
+// decomposition of gqa_decode instead of fixed splits when that fills at least
+// three quarters of the resident blocks with portable clusters (<= 8 blocks):
+// one kernel, the splits of a unit merged through distributed shared memory,
+// no workspace.  Only for one query token without lse output or group table
+// (the cluster kernel writes final rows only), and not for the tcgen05 kernel.
+// Returns the blocks per cluster, or 0 for the fixed-split / equal-work plan.
+int auto_cluster(const Shape &sh, bool paged, bool lse, int sms) {
+  if (paged || lse || sh.mapped || sh.tc || sh.fma || sh.nq != 1) return 0;
+  const int c = cluster_plan(sh, sms);
+  if (c < 2 || c > 8) return 0;
+  const long long blocks = units_of(sh) * c;
+  const long long slots = static_cast<long long>(sms) * blocks_per_sm(sh);
+  return (4 * blocks >= 3 * slots && 10 * blocks <= 9 * slots) ? c : 0;
 }
 
 // split_tokens == 0 in the split API: checks shared by its entry points.
@@ -715,6 +770,21 @@ int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t
   return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// The cluster decomposition (gqa_decode, and gqa_decode_split's choice for
+// contiguous caches with few units): grid (c, G x slices, b), clusters of c.
+int run_cluster(const Shape &sh, int c, const void *q, const void *k, const void *v, const int32_t *seqlens,
+                const int32_t *pt, float *out, float scale, uint32_t *status, cudaStream_t st) {
+  CUtensorMap tk, tv;
+  int rc = encode_maps(sh, k, v, &tk, &tv);
+  if (rc != GQA_OK) return rc;
+  DecodeParams p = base_params(sh, q, seqlens, pt, status, scale);
+  p.out = out;
+  // launched as a programmatic dependent: the blocks set themselves up while
+  // the previous kernel on the stream finishes
+  Launch l{dim3(c, sh.G * sh.hs, sh.b), c, st, true};
+  return launch_decode<Mode::kCluster>(sh, tk, tv, p, l);
+}
+
 }  // namespace
 
 namespace {
@@ -736,6 +806,8 @@ int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, c
       return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+    const int c = auto_cluster(sh, dims_paged(dims), ex.lse != nullptr, std::min(dev.sms, 256));
+    if (c > 0) return run_cluster(sh, c, q, k_cache, v_cache, seqlens, page_table, out, scale, status, st);
     // (a group map runs on fixed splits only: the library picks them as for a contiguous cache)
     const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) {
@@ -820,14 +892,7 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
     return run_items(sh, q, k_cache, v_cache, seqlens, page_table, out, scale, status, split, 1,
                      static_cast<int>(sh.capacity), nullptr, nullptr, nullptr, nullptr, st);
   }
-  CUtensorMap tk, tv;
-  if ((rc = encode_maps(sh, k_cache, v_cache, &tk, &tv)) != GQA_OK) return rc;
-  DecodeParams p = base_params(sh, q, seqlens, page_table, status, scale);
-  p.out = out;
-  // launched as a programmatic dependent: the blocks set themselves up while
-  // the previous kernel on the stream finishes
-  Launch l{dim3(c, sh.G * sh.hs, sh.b), c, st, true};
-  return launch_decode<Mode::kCluster>(sh, tk, tv, p, l);
+  return run_cluster(sh, c, q, k_cache, v_cache, seqlens, page_table, out, scale, status, st);
 }
 
 size_t gqa_decode_split_workspace_size(const gqa_dims *dims, int32_t max_seqlen, int32_t split_tokens) {
@@ -852,6 +917,32 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
   }
   const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, std::min(num_sms, 256));
   return ch.balanced ? 0 : ch.split_tokens;
+}
+
+int32_t gqa_plan_decomposition(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms,
+                               int32_t *split_tokens_out, int32_t *cluster_out) {
+  Shape sh;
+  if (!dims) return GQA_ERR_NULL_POINTER;
+  int rc = check_dims(dims, dims_paged(dims), &sh);
+  if (rc != GQA_OK) return rc;
+  if (max_seqlen < 1) return GQA_ERR_DIMS;
+  if (num_sms <= 0) {
+    DeviceInfo dev;
+    if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
+    num_sms = dev.sms;
+  }
+  num_sms = std::min(num_sms, 256);
+  if (split_tokens_out) *split_tokens_out = 0;
+  if (cluster_out) *cluster_out = 1;
+  const int c = auto_cluster(sh, dims_paged(dims), false, num_sms);
+  if (c > 0) {
+    if (cluster_out) *cluster_out = c;
+    return GQA_PLAN_CLUSTERS;
+  }
+  const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, num_sms);
+  if (ch.balanced) return GQA_PLAN_EQUAL_WORK;
+  if (split_tokens_out) *split_tokens_out = ch.split_tokens;
+  return GQA_PLAN_FIXED_SPLITS;
 }
 
 int gqa_split_partials(const void *q, const void *k_cache, const void *v_cache,

@@ -38,6 +38,16 @@
 // The epilogue writes final rows or partial states in the layout of the
 // mma.sync kernel, so the same merges (in this kernel for up to 8 splits, the
 // combine kernel otherwise) apply.
+//
+// Two decompositions: one block per (sequence, group, split) item
+// (gqa_verify_tc_kernel), or equal-work ranges (gqa_verify_tc_balanced_kernel):
+// one persistent block per SM walks its contiguous range of the tiles of all
+// (sequence, group) units, the K/V ring streaming across unit boundaries; Q
+// is double-buffered (the producer warp fills the next unit's Q while the
+// current one runs), and the P.V products of a new unit wait only until the
+// softmax warps have read the previous unit's O out of tensor memory.  Units
+// shared with a neighbouring block leave partial states for the balanced
+// combine kernel, exactly as in the mma.sync kernel's equal-work mode.
 #pragma once
 
 #include "gqa_kernels.cuh"
@@ -45,26 +55,31 @@
 
 namespace gqa {
 
-struct TcTile {
+// Shared-memory layout of the tcgen05 kernels: a STAGES-deep ring of K/V tiles
+// of 64 tokens (32 KB per stage) and QBUFS buffers of Q (128 rows x d = 128).
+template <int STAGES, int QBUFS>
+struct TcLayout {
   static constexpr int kD = 128;
   static constexpr int kT = 64;                        // tokens per tile
   static constexpr int kM = 128;                       // rows of every MMA (padded)
-  static constexpr int kStages = 5;
+  static constexpr int kStages = STAGES;
+  static constexpr int kQBufs = QBUFS;
   static constexpr int kHalf = kT * 128;               // one 64-column half of a K or V tile
   static constexpr int kTileBytes = 2 * kHalf;         // 16 KB
   static constexpr int kStageBytes = 2 * kTileBytes;   // K + V
-  static constexpr int kQOff = kStages * kStageBytes;  // Q: two halves of kM rows x 128 B
+  static constexpr int kQOff = kStages * kStageBytes;  // Q: two halves of kM rows x 128 B per buffer
   static constexpr int kQHalf = kM * 128;
-  static constexpr int kBarOff = kQOff + 2 * kQHalf;
+  static constexpr int kQBytes = 2 * kQHalf;
+  static constexpr int kBarOff = kQOff + kQBufs * kQBytes;
   static constexpr int kSP = 3;                        // S/P buffers in tensor memory
   // full[kStages], empty[kStages], s_full[kSP], p_full[kSP], pv_done[kSP],
   // drain[2] (one per MMA issuer: all its products done before teardown),
-  // q_full (Q written to shared memory)
-  static constexpr int kNumBars = 2 * kStages + 3 * kSP + 3;
+  // q_full[kQBufs], q_empty[kQBufs], o_free (O read out: the next unit's P.V may start)
+  static constexpr int kNumBars = 2 * kStages + 3 * kSP + 2 + 2 * kQBufs + 1;
   static constexpr int kXOff = kBarOff + 8 * kNumBars;  // the halves' bases at the end: [2][kM] floats
   static constexpr int kLOff = kXOff + 4 * 2 * kM;      // the halves' sums at the end: [2][kM] floats
-  static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[kStages], abort, merge here
-  static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * (kStages + 3);
+  static constexpr int kMiscOff = kLOff + 4 * 2 * kM;  // tmem base, tile_bad[kStages], abort, merge here, stop
+  static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * (kStages + 4);
   static constexpr int kSoftmaxWarps = 8;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
   static constexpr uint32_t kOCol = 256;               // O of the first halves: 256 .. 383, second: 384 .. 511
@@ -72,20 +87,103 @@ struct TcTile {
   static_assert(kSP * kT <= static_cast<int>(kOCol) && kOCol + 2 * kD <= kTmemCols, "tensor-memory columns");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
+using TcTile = TcLayout<5, 1>;     // one piece per block
+using TcBalTile = TcLayout<4, 2>;  // equal-work ranges: pieces follow each other
 
-// TMA producer for one piece (items mode): K and V tiles of 64 tokens into the
-// stage ring, pages translated through the table as in the mma.sync kernel.
-template <bool PAGED>
-__device__ __forceinline__ void tc_produce(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeParams &p,
-                                           const Piece &pc, uint32_t sbase, uint32_t full0, uint32_t empty0,
-                                           volatile int *tile_bad, volatile int *abort_flag, int lane) {
-  using TT = TcTile;
+struct TcBars {
+  uint32_t full0, empty0, s_full0, p_full0, pv_done0, drain0, q_full0, q_empty0, o_free;
+};
+
+template <class TT>
+__device__ __forceinline__ TcBars tc_bars(uint32_t sbase) {
+  TcBars b;
+  b.full0 = sbase + TT::kBarOff;
+  b.empty0 = b.full0 + 8 * TT::kStages;
+  b.s_full0 = b.empty0 + 8 * TT::kStages;
+  b.p_full0 = b.s_full0 + 8 * TT::kSP;
+  b.pv_done0 = b.p_full0 + 8 * TT::kSP;
+  b.drain0 = b.pv_done0 + 8 * TT::kSP;
+  b.q_full0 = b.drain0 + 16;
+  b.q_empty0 = b.q_full0 + 8 * TT::kQBufs;
+  b.o_free = b.q_empty0 + 8 * TT::kQBufs;
+  return b;
+}
+
+// One thread initialises every barrier.  q_full_count: arrivals that make a Q
+// buffer full (128 Q rows, or the producer warp's one arrival).
+template <class TT>
+__device__ __forceinline__ void tc_init_bars(const TcBars &b, volatile int *tile_bad, uint32_t q_full_count) {
+  for (int i = 0; i < TT::kStages; ++i) {
+    mbar_init(b.full0 + 8 * i, 1);
+    mbar_init(b.empty0 + 8 * i, 1);  // one tcgen05.commit per use
+    tile_bad[i] = 0;
+  }
+  for (int i = 0; i < TT::kSP; ++i) {
+    mbar_init(b.s_full0 + 8 * i, 1);
+    mbar_init(b.p_full0 + 8 * i, TT::kSoftmaxWarps);  // one arrival per softmax warp
+    mbar_init(b.pv_done0 + 8 * i, 1);
+  }
+  mbar_init(b.drain0, 1);
+  mbar_init(b.drain0 + 8, 1);
+  for (int i = 0; i < TT::kQBufs; ++i) {
+    mbar_init(b.q_full0 + 8 * i, q_full_count);
+    mbar_init(b.q_empty0 + 8 * i, 1);
+  }
+  mbar_init(b.o_free, TT::kSoftmaxWarps);
+}
+
+// Row of the slice held by Q slot r, or -1 for a padding slot.  SPREAD: the
+// rows sit in the first ceil(nh / 4) lanes of each 32-lane quarter.
+template <bool SPREAD>
+__device__ __forceinline__ int tc_slot_row(int r, int nh) {
+  if (SPREAD) {
+    const int rpq = (nh + 3) / 4, li = r % 32, rho = (r / 32) * rpq + li;
+    return (li < rpq && rho < nh) ? rho : -1;
+  }
+  return r < nh ? r : -1;
+}
+
+// Byte offset of 16-byte chunk c (of 16) of Q slot r: two 64-column halves in
+// the 128-byte swizzle TMA would write.
+template <class TT>
+__device__ __forceinline__ int tc_q_offset(int r, int c) {
+  return (c >> 3) * TT::kQHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+// The producer warp fills one Q buffer with the piece's rows (padding slots
+// zero): 128 slots x 16 chunks, two slots per round of the 32 lanes, 16 loads
+// in flight per lane; then makes the writes visible to the tensor core.
+template <class TT, bool SPREAD>
+__device__ __forceinline__ void tc_fill_q_warp(const DecodeParams &p, const Piece &pc, uint8_t *qbuf, int lane) {
+  constexpr int D = TT::kD;
+  for (int base = 0; base < TT::kM * 16; base += 32 * 16) {
+    uint4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int idx = base + i * 32 + lane, r = idx >> 4, c = idx & 15;
+      const int rho = tc_slot_row<SPREAD>(r, pc.nh);
+      v[i] = rho >= 0 ? __ldg(reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + rho) * D) + c)
+                      : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int idx = base + i * 32 + lane, r = idx >> 4, c = idx & 15;
+      *reinterpret_cast<uint4 *>(qbuf + tc_q_offset<TT>(r, c)) = v[i];
+    }
+  }
+  fence_proxy_async_smem();
+}
+
+// TMA producer for one piece: K and V tiles of 64 tokens into the stage ring
+// from ring position `tile` on (advanced past the piece), pages translated
+// through the table as in the mma.sync kernel.  False if the block aborted.
+template <class TT, bool PAGED>
+__device__ __forceinline__ bool tc_produce_piece(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                                                 const DecodeParams &p, const Piece &pc, uint32_t sbase,
+                                                 const TcBars &bars, volatile int *tile_bad,
+                                                 volatile int *abort_flag, int lane, int &tile) {
   constexpr int T = TT::kT;
   constexpr int ST = TT::kStages;
-  if (lane == 0) {
-    tma_prefetch_desc(tm_k);
-    tma_prefetch_desc(tm_v);
-  }
   const uint64_t policy = l2_policy_evict_first();
   const int P = p.page_size;
   const int ppt = PAGED ? max(1, T / P) : 1;  // pages per tile
@@ -94,19 +192,18 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap *tm_k, const CUtens
   const int32_t *pt_row = PAGED ? p.page_table + static_cast<size_t>(pc.s) * p.max_pages : nullptr;
   const int lp_end = PAGED ? (pc.t_end + P - 1) / P : 0;
   int cur_w = -1, nxt_w = -1, win = -1, nxt = -1;
-  int tile = 0;
   for (int t0 = pc.t_begin; t0 < pc.t_end; t0 += T, ++tile) {
     const int stage = tile % ST;
-    const uint32_t full = full0 + 8 * stage;
+    const uint32_t full = bars.full0 + 8 * stage;
     if (tile >= ST) {
-      bool ok = mbar_wait(empty0 + 8 * stage, ((tile / ST) - 1) & 1);
+      bool ok = mbar_wait(bars.empty0 + 8 * stage, ((tile / ST) - 1) & 1);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok || *abort_flag) {
         if (lane == 0) {
           *abort_flag = 1;
           if (p.status) atomicOr(p.status, kStatusTimeout);
         }
-        break;
+        return false;
       }
     }
     const uint32_t dst_k = sbase + stage * TT::kStageBytes;
@@ -153,10 +250,15 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap *tm_k, const CUtens
       }
     }
   }
-  // never leave with copies in flight (bounded waits)
-  if (lane == 0) {
-    for (int t = max(0, tile - ST); t < tile; ++t) (void)mbar_wait(full0 + 8 * (t % ST), (t / ST) & 1);
-  }
+  return true;
+}
+
+// Never leave with copies in flight: wait (bounded) for the last tiles issued.
+template <class TT>
+__device__ __forceinline__ void tc_produce_drain(const TcBars &bars, int tile, int lane) {
+  constexpr int ST = TT::kStages;
+  if (lane == 0)
+    for (int t = max(0, tile - ST); t < tile; ++t) (void)mbar_wait(bars.full0 + 8 * (t % ST), (t / ST) & 1);
 }
 
 // The block whose split completes the unit merges the unit's splits (as in
@@ -164,7 +266,7 @@ __device__ __forceinline__ void tc_produce(const CUtensorMap *tm_k, const CUtens
 // each.  Called by all of them, after their partial states are written.
 __device__ __forceinline__ void tc_merge_unit(const DecodeParams &p, const Piece &pc, int sm,
                                               volatile int *merge_here) {
-  constexpr int D = TcTile::kD;
+  constexpr int D = 128;
   constexpr int kSM = 32 * TcTile::kSoftmaxWarps;
   named_barrier(1, kSM);
   const int ns = (pc.len + p.split_tokens - 1) / p.split_tokens;
@@ -188,22 +290,47 @@ __device__ __forceinline__ void tc_merge_unit(const DecodeParams &p, const Piece
   }
 }
 
-// Softmax warps with at most 64 rows (SPREAD): quarter qd = warp % 4 of the
-// tensor-memory lanes holds rows qd * rpq .. in its first rpq <= 16 lanes
+// Where the rows of a piece go.  final_row: normalised rows into out (and
+// lse).  Otherwise partial states: slot >= 0 is the block's partial slot of
+// the equal-work mode (row rho at slot * rc + rho); slot < 0 is split k of the
+// output row (items mode; the unit's last arrival merges it in this kernel
+// when the call has arrival words).
+struct TcDest {
+  bool final_row;
+  int slot;
+};
+
+__device__ __forceinline__ size_t tc_part_index(const DecodeParams &p, const Piece &pc, const TcDest &dst,
+                                                size_t row, int rho) {
+  return dst.slot >= 0 ? static_cast<size_t>(dst.slot) * p.rc + rho : row * p.num_splits + pc.k;
+}
+
+// After the rows of a piece are written: the softmax threads agree (through
+// one barrier) on whether the block stops, so that they all take the same
+// barriers in the next piece.
+__device__ __forceinline__ bool tc_piece_done(volatile int *stop, volatile int *abort_flag, int sm, int n_threads) {
+  if (sm == 0) *stop = *abort_flag;
+  named_barrier(1, n_threads);
+  return *stop == 0;
+}
+
+// Softmax warps with at most 64 rows (SPREAD), for one piece of n_tiles tiles
+// starting at global tile gt0 of the block's pipeline: quarter qd = warp % 4 of
+// the tensor-memory lanes holds rows qd * rpq .. in its first rpq <= 16 lanes
 // (rpq = ceil(rows / 4)).  Warp w takes tokens [32 h, 32 h + 32) of every
 // tile, h = w / 4, and within it thread t the 16 tokens [32 h + 16 (t / 16),
 // + 16) of lane t % 16 (the 16x32bx2 shape).  The two threads of a row in one
 // warp share its running base (their maximum meets through one shuffle) and
 // the row's O_h in tensor memory; the two warps of a quarter keep separate
 // states and O_h, merged once at the end.  P's high part goes over the
-// thread's first 8 score columns, its residual over the next 8.
-template <bool PAGED>
-__device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const Piece &pc, uint8_t *smem,
-                                                  uint32_t tmem, uint32_t s_full0, uint32_t p_full0,
-                                                  uint32_t pv_done0, volatile int *tile_bad,
-                                                  volatile int *abort_flag, volatile int *merge_here, int n_tiles,
-                                                  int warp, int lane) {
-  using TT = TcTile;
+// thread's first 8 score columns, its residual over the next 8.  Returns
+// false once the block stops (a timeout).
+template <class TT, bool PAGED>
+__device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const Piece &pc, uint8_t *smem,
+                                                  uint32_t tmem, const TcBars &bars, volatile int *tile_bad,
+                                                  volatile int *abort_flag, volatile int *merge_here,
+                                                  volatile int *stop, int gt0,
+                                                  int n_tiles, const TcDest &dest, int warp, int lane) {
   constexpr int D = TT::kD;
   constexpr int T = TT::kT;
   constexpr int ST = TT::kStages;
@@ -231,10 +358,11 @@ __device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const P
   int bad = 0;
   bool ok = true;
   for (int t = 0; t < n_tiles; ++t) {
+    const int gt = gt0 + t;
     const int t0 = pc.t_begin + t * T;
-    const int st = t % ST;
-    const int b = t % SP;
-    ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (t / SP) & 1));
+    const int st = gt % ST;
+    const int b = gt % SP;
+    ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full0 + 8 * b, (gt / SP) & 1));
     if (!ok) break;
     tc_fence_after();
     uint32_t sv[16];
@@ -278,9 +406,9 @@ __device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const P
         const float alpha = need ? ((m_run == kNegInf) ? 0.f : ex2(m_run - mn)) : 1.f;
         l_run *= alpha;
         if (t > 0) {
-          // O_h holds tiles 0 .. t-1: rescale it once their MMAs are done;
-          // thread sub takes columns [64 sub, 64 sub + 64) of the row
-          ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((t - 1) % SP), ((t - 1) / SP) & 1));
+          // O_h holds the piece's tiles 0 .. t-1: rescale it once their MMAs
+          // are done; thread sub takes columns [64 sub, 64 sub + 64) of the row
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done0 + 8 * ((gt - 1) % SP), ((gt - 1) / SP) & 1));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -312,7 +440,7 @@ __device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const P
     tc_fence_before();
     if (valid_rows < T) fence_proxy_async_smem();  // the zeroed V rows, for the tensor core
     __syncwarp();
-    if (lane == 0) mbar_arrive(p_full0 + 8 * b);
+    if (lane == 0) mbar_arrive(bars.p_full0 + 8 * b);
   }
   if (!ok && lane == 0) {
     *abort_flag = 1;
@@ -320,8 +448,8 @@ __device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const P
   }
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);  // the half's sum of the row
   // ---- the row's result: O from tensor memory once the last MMAs are done
-  const bool done =
-      ok && __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((n_tiles - 1) % SP), ((n_tiles - 1) / SP) & 1));
+  const int glast = gt0 + n_tiles - 1;
+  const bool done = ok && __all_sync(0xffffffffu, mbar_wait(bars.pv_done0 + 8 * (glast % SP), (glast / SP) & 1));
   tc_fence_after();
   if (sub == 0) {
     mbase[half * 128 + slot] = m_run;
@@ -332,11 +460,10 @@ __device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const P
   const float m_row = fmaxf(m0, m1);
   const float w0 = (m0 == kNegInf) ? 0.f : ex2(m0 - m_row), w1 = (m1 == kNegInf) ? 0.f : ex2(m1 - m_row);
   const float l_row = lsum[slot] * w0 + lsum[128 + slot] * w1;
-  const bool final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
   const size_t row = valid ? row_of(p, pc.s, pc.g, pc.h0 + rho) : 0;
-  const size_t ps = row * p.num_splits + pc.k;
+  const size_t ps = tc_part_index(p, pc, dest, row, rho);
   const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
-  const float s0 = final_row ? w0 * inv : w0, s1 = final_row ? w1 * inv : w1;
+  const float s0 = dest.final_row ? w0 * inv : w0, s1 = dest.final_row ? w1 * inv : w1;
   {
     // this thread writes columns [64 half + 32 sub, + 32) of the row
     uint32_t oa[32], ob[32];
@@ -345,7 +472,7 @@ __device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const P
     tc_wait_ld();
     if (valid) {
       const int col = half * 64 + sub * 32;
-      float4 *dst = reinterpret_cast<float4 *>((final_row ? p.out + row * D : p.part_o + ps * D) + col);
+      float4 *dst = reinterpret_cast<float4 *>((dest.final_row ? p.out + row * D : p.part_o + ps * D) + col);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float v[4];
@@ -356,16 +483,277 @@ __device__ __forceinline__ void tc_softmax_spread(const DecodeParams &p, const P
     }
   }
   if (valid && half == 0 && sub == 0) {
-    if (final_row) {
+    if (dest.final_row) {
       if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_row, l_row);
-      if (p.part_l) p.part_l[row * p.num_splits] = kLFinal;
+      if (dest.slot < 0 && p.part_l) p.part_l[row * p.num_splits] = kLFinal;
     } else {
       p.part_m[ps] = m_row;
       p.part_l[ps] = bad ? kLBadPage : l_row;
     }
   }
   tc_fence_before();
-  if (p.unit_ctr != nullptr && !final_row) tc_merge_unit(p, pc, sm, merge_here);
+  if (dest.slot < 0 && p.unit_ctr != nullptr && !dest.final_row) tc_merge_unit(p, pc, sm, merge_here);
+  return tc_piece_done(stop, abort_flag, sm, kSM) && ok;
+}
+
+// Softmax warps with up to 128 rows, for one piece (as tc_softmax_spread):
+// row i is lane i, two threads per row (warps w and w + 4 share the lanes of
+// quarter w % 4), each on 32 of a tile's 64 tokens with a softmax state and an
+// O of its own, merged once at the end.
+template <class TT, bool PAGED>
+__device__ __forceinline__ bool tc_softmax_wide(const DecodeParams &p, const Piece &pc, uint8_t *smem,
+                                                uint32_t tmem, const TcBars &bars, volatile int *tile_bad,
+                                                volatile int *abort_flag, volatile int *merge_here,
+                                                  volatile int *stop, int gt0,
+                                                int n_tiles, const TcDest &dest, int warp, int lane) {
+  constexpr int D = TT::kD;
+  constexpr int T = TT::kT;
+  constexpr int ST = TT::kStages;
+  constexpr int SP = TT::kSP;
+  constexpr int kSM = 32 * TT::kSoftmaxWarps;  // softmax threads
+  const float kNegInf = -__int_as_float(0x7f800000);
+  const int sm = threadIdx.x;                  // 0 .. kSM-1
+  const int half = sm / 128;                   // tokens [32 half, 32 half + 32) of every tile
+  const int r = sm % 128;                      // row of the slice = tensor-memory lane
+  const bool valid = r < pc.nh;
+  const bool warp_active = (warp % 4) * 32 < pc.nh;
+  // the positions this row sees: with several query tokens per sequence,
+  // query token t sees the cache up to and including itself (a padding row,
+  // q = 0, sees the whole piece: its scores are 0, its result unused, and it
+  // keeps to the unmasked path of its warp)
+  const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + r) / p.r)) : pc.t_end;
+  const uint32_t lane_tmem = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+  float *mbase = reinterpret_cast<float *>(smem + TT::kXOff);  // [half][row]
+  float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);   // [half][row]
+  const float sl = p.scale_log2;
+  float m_run = kNegInf, l_run = 0.f;  // this half's base and sum
+  int bad = 0;
+  bool ok = true;
+  for (int t = 0; t < n_tiles; ++t) {
+    const int gt = gt0 + t;
+    const int t0 = pc.t_begin + t * T;
+    const int st = gt % ST;
+    const int b = gt % SP;
+    ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full0 + 8 * b, (gt / SP) & 1));
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t sv[32];
+    tc_ld32(lane_tmem + b * 64 + half * 32, sv);
+    tc_wait_ld();
+    if (PAGED) bad |= tile_bad[st];
+    // V rows past the piece's end may hold anything (even NaN): zero them so
+    // that P = 0 there meets zeros
+    const int valid_rows = min(T, pc.t_end - t0);
+    if (valid_rows < T) {
+      uint8_t *vt = smem + st * TT::kStageBytes + TT::kTileBytes;
+      for (int idx = sm; idx < (T - valid_rows) * 16; idx += kSM) {
+        const int row = valid_rows + idx / 16, c = idx % 16;
+        *reinterpret_cast<uint4 *>(vt + (c >> 3) * TT::kHalf + row * 128 + ((c & 7) << 4)) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    float x[32];
+    const int tb = t0 + half * 32;  // this thread's first token of the tile
+    if (tb + 32 <= lim) {
+      // all of them visible (every tile but the row's last)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(sv[j]) * sl;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
+    }
+    float mx;
+    {
+      float m8[8];  // a tree, not a chain of 32 dependent steps
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m8[k] = fmaxf(fmaxf(x[4 * k], x[4 * k + 1]), fmaxf(x[4 * k + 2], x[4 * k + 3]));
+      mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+    }
+    if (warp_active) {
+      // lazy rescale: only when a score passes the base by more than 2^8
+      const bool need = mx > m_run + 8.f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float mn = need ? fmaxf(m_run, mx) : m_run;
+        const float alpha = need ? ((m_run == kNegInf) ? 0.f : ex2(m_run - mn)) : 1.f;
+        l_run *= alpha;
+        if (t > 0) {
+          // this half's O holds the piece's tiles 0 .. t-1: rescale it once their MMAs are done
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done0 + 8 * ((gt - 1) % SP), ((gt - 1) / SP) & 1));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tc_ld32(lane_tmem + TT::kOCol + half * D + c * 32, ov);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+            tc_st32(lane_tmem + TT::kOCol + half * D + c * 32, ov);
+          }
+          tc_wait_st();
+          tc_fence_before();
+        }
+        m_run = mn;
+      }
+      const float base = (m_run == kNegInf) ? 0.f : m_run;
+      // P over this thread's own 32 score columns: high part in the first
+      // 16, residual in the next 16 (the buffer's scores of tile t are no
+      // longer needed, and the MMAs of tile t-SP that read it are done, since
+      // the scores of tile t came after them)
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
+        l_run += p0 + p1;
+        split_bf16x2_rz(p0, p1, hi[e], lo[e]);
+      }
+      tc_st16(lane_tmem + b * 64 + half * 32, hi);
+      tc_st16(lane_tmem + b * 64 + half * 32 + 16, lo);
+      tc_wait_st();
+    }
+    // (p_full is one barrier per P buffer: a warp reaches tile t+SP only
+    // after s_full of t+SP, and the scores of t+SP are issued only once the
+    // P.V of tile t is done, so its next arrival on the same barrier cannot
+    // fall into tile t's phase)
+    tc_fence_before();
+    if (valid_rows < T) fence_proxy_async_smem();  // the zeroed V rows, for the tensor core
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars.p_full0 + 8 * b);
+  }
+  if (!ok && lane == 0) {
+    *abort_flag = 1;
+    if (p.status) atomicOr(p.status, kStatusTimeout);
+  }
+  // ---- the row's result: O from tensor memory once the last MMAs are done
+  const int glast = gt0 + n_tiles - 1;
+  const bool done = ok && __all_sync(0xffffffffu, mbar_wait(bars.pv_done0 + 8 * (glast % SP), (glast / SP) & 1));
+  tc_fence_after();
+  // the row's two partial states, merged exactly: M = max(m0, m1), weights
+  // 2^(m_h - M) (0 for a half that saw no position)
+  mbase[half * 128 + r] = m_run;
+  lsum[half * 128 + r] = l_run;
+  named_barrier(1, kSM);
+  const float m0 = mbase[r], m1 = mbase[128 + r];
+  const float m_row = fmaxf(m0, m1);
+  const float w0 = (m0 == kNegInf) ? 0.f : ex2(m0 - m_row), w1 = (m1 == kNegInf) ? 0.f : ex2(m1 - m_row);
+  const float l_row = lsum[r] * w0 + lsum[128 + r] * w1;
+  const size_t row = valid ? row_of(p, pc.s, pc.g, pc.h0 + r) : 0;
+  const size_t ps = tc_part_index(p, pc, dest, row, r);
+  const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
+  const float s0 = dest.final_row ? w0 * inv : w0, s1 = dest.final_row ? w1 * inv : w1;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t oa[32], ob[32];
+    const int col = half * 64 + c * 32;  // this thread writes columns [64 half, 64 half + 64)
+    tc_ld32(lane_tmem + TT::kOCol + col, oa);
+    tc_ld32(lane_tmem + TT::kOCol + D + col, ob);
+    tc_wait_ld();
+    if (valid) {
+      float4 *dst = reinterpret_cast<float4 *>((dest.final_row ? p.out + row * D : p.part_o + ps * D) + col);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = __uint_as_float(oa[4 * j + e]) * s0 + __uint_as_float(ob[4 * j + e]) * s1;
+        dst[j] = make_float4(v[0], v[1], v[2], v[3]);
+      }
+    }
+  }
+  if (valid && half == 0) {
+    if (dest.final_row) {
+      if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_row, l_row);
+      if (dest.slot < 0 && p.part_l) p.part_l[row * p.num_splits] = kLFinal;
+    } else {
+      p.part_m[ps] = m_row;
+      p.part_l[ps] = bad ? kLBadPage : l_row;
+    }
+  }
+  tc_fence_before();
+  if (dest.slot < 0 && p.unit_ctr != nullptr && !dest.final_row) tc_merge_unit(p, pc, sm, merge_here);
+  return tc_piece_done(stop, abort_flag, sm, kSM) && ok;
+}
+
+// The Q K^T products of one piece (one thread): S[gt % SP] = Q K_gt^T for
+// the piece's tiles, once K has landed and the buffer's last P.V is done.
+template <class TT>
+__device__ __forceinline__ bool tc_issue_qk(uint32_t sbase, uint32_t qbuf, uint32_t tmem, const TcBars &bars,
+                                            int gt0, int n_tiles) {
+  constexpr int D = TT::kD;
+  constexpr int ST = TT::kStages;
+  constexpr int SP = TT::kSP;
+  constexpr uint32_t kIdescQK = tc_idesc_bf16(128, 64, false);
+  // Q's descriptors are the same for every tile; a K-step adds to the
+  // start-address field (addresses stay below 256 KB: no carry)
+  uint64_t qd[D / 16];
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks)
+    qd[ks] = tc_smem_desc(qbuf + (ks >> 2) * TT::kQHalf + (ks & 3) * 32, 16, 1024);
+  for (int t = 0; t < n_tiles; ++t) {
+    const int gt = gt0 + t;
+    const int st = gt % ST;
+    bool ok = mbar_wait(bars.full0 + 8 * st, (gt / ST) & 1);
+    if (ok && gt >= SP) ok = mbar_wait(bars.pv_done0 + 8 * (gt % SP), ((gt / SP) - 1) & 1);
+    if (!ok) return false;
+    tc_fence_after();
+    const uint64_t kd = tc_smem_desc(sbase + st * TT::kStageBytes, 16, 1024);
+    const uint32_t d = tmem + (gt % SP) * 64;
+    tc_mma(d, qd[0], kd, kIdescQK, 0u);
+#pragma unroll
+    for (int ks = 1; ks < D / 16; ++ks)
+      tc_mma(d, qd[ks], kd + ((static_cast<uint32_t>((ks >> 2) * TT::kHalf + (ks & 3) * 32)) >> 4), kIdescQK, 1u);
+    tc_commit(bars.s_full0 + 8 * (gt % SP));
+  }
+  return true;
+}
+
+// The P.V products of one piece (one thread): O_h += P V for the piece's
+// tiles, the high part and the residual of P read from tensor memory; the
+// piece's first tile starts the accumulators afresh.
+template <class TT, bool SPREAD>
+__device__ __forceinline__ bool tc_issue_pv(uint32_t sbase, uint32_t tmem, const TcBars &bars, int gt0,
+                                            int n_tiles) {
+  constexpr int D = TT::kD;
+  constexpr int T = TT::kT;
+  constexpr int ST = TT::kStages;
+  constexpr int SP = TT::kSP;
+  constexpr uint32_t kIdescPV = tc_idesc_bf16(128, 128, true);
+  for (int u = 0; u < n_tiles; ++u) {
+    const int gt = gt0 + u;
+    const int st = gt % ST;
+    if (!mbar_wait(bars.p_full0 + 8 * (gt % SP), (gt / SP) & 1)) return false;
+    tc_fence_after();
+    const uint64_t vd = tc_smem_desc(sbase + st * TT::kStageBytes + TT::kTileBytes, TT::kHalf, 1024);
+    const uint32_t pb = tmem + (gt % SP) * 64;
+#pragma unroll
+    for (int ks = 0; ks < T / 16; ++ks) {
+      // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of the
+      // buffer, the residual 16 columns further (SPREAD: the thread of those
+      // tokens wrote its high part at column 16 ks, its residual 8 further);
+      // into the O of the half of the row that owns them
+      const uint64_t vdk = vd + ((ks * 16 * 128) >> 4);
+      const uint32_t pa = SPREAD ? pb + 16 * ks : pb + 32 * (ks >> 1) + 8 * (ks & 1);
+      const uint32_t od = tmem + TT::kOCol + D * (ks >> 1);
+      tc_mma_ts(od, pa, vdk, kIdescPV, (u > 0 || (ks & 1)) ? 1u : 0u);
+      tc_mma_ts(od, pa + (SPREAD ? 8 : 16), vdk, kIdescPV, 1u);
+    }
+    // K was read by the scores of this tile, done before its P existed; V and
+    // P by these products
+    tc_commit(bars.empty0 + 8 * st);
+    tc_commit(bars.pv_done0 + 8 * (gt % SP));
+  }
+  return true;
+}
+
+// An issuer's last step: every product it issued is done before the block
+// tears down (on an early exit, products already issued may still be running).
+__device__ __forceinline__ void tc_issuer_drain(uint32_t drain_bar, const DecodeParams &p) {
+  tc_commit(drain_bar);
+  if (!mbar_wait(drain_bar, 0) && p.status) atomicOr(p.status, kStatusTimeout);
+}
+
+__device__ __forceinline__ void tc_abort(const DecodeParams &p, volatile int *abort_flag) {
+  *abort_flag = 1;
+  if (p.status) atomicOr(p.status, kStatusTimeout);
 }
 
 // SPREAD (at most 64 rows): the rows sit in the first 16 lanes of each of the
@@ -381,24 +769,18 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   using TT = TcTile;
   constexpr int D = TT::kD;
   constexpr int T = TT::kT;
-  constexpr int ST = TT::kStages;
   const float kNegInf = -__int_as_float(0x7f800000);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_addr(smem);
-  const uint32_t bars = sbase + TT::kBarOff;
-  const uint32_t full0 = bars, empty0 = bars + 8 * ST;
-  constexpr int SP = TT::kSP;
-  const uint32_t s_full0 = bars + 16 * ST;
-  const uint32_t p_full0 = s_full0 + 8 * SP, pv_done0 = p_full0 + 8 * SP;
-  const uint32_t drain0 = pv_done0 + 8 * SP;  // [2]: the Q K^T issuer's, the P.V issuer's
-  const uint32_t q_full = drain0 + 16;
+  const TcBars bars = tc_bars<TT>(sbase);
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
   volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
-  volatile int *abort_flag = tile_bad + ST;
-  volatile int *merge_here = tile_bad + ST + 1;
+  volatile int *abort_flag = tile_bad + TT::kStages;
+  volatile int *merge_here = tile_bad + TT::kStages + 1;
+  volatile int *stop = tile_bad + TT::kStages + 2;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -407,21 +789,10 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   constexpr int kProducerWarp = TT::kSoftmaxWarps;  // then the Q K^T issuer (allocates), the P.V issuer
   constexpr int kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < ST; ++i) {
-      mbar_init(full0 + 8 * i, 1);
-      mbar_init(empty0 + 8 * i, 1);  // one tcgen05.commit per use
-      tile_bad[i] = 0;
-    }
-    for (int i = 0; i < SP; ++i) {
-      mbar_init(s_full0 + 8 * i, 1);
-      mbar_init(p_full0 + 8 * i, TT::kSoftmaxWarps);  // one arrival per softmax warp
-      mbar_init(pv_done0 + 8 * i, 1);
-    }
-    mbar_init(drain0, 1);
-    mbar_init(drain0 + 8, 1);
-    mbar_init(q_full, 128);  // one arrival per Q row
+    tc_init_bars<TT>(bars, tile_bad, 128);  // one arrival per Q row
     *abort_flag = 0;
     *merge_here = 0;
+    *stop = 0;
     fence_mbarrier_init();
   }
   if (warp == kMmaWarp) {
@@ -460,275 +831,210 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   if (threadIdx.x == 0 && p.unit_ctr != nullptr && (pc.len + p.split_tokens - 1) / p.split_tokens > 1)
     unit_claim(p.unit_ctr + (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j, p.epoch);
   if (threadIdx.x < 128) {
-    // the q row of this thread's slot into Q (128-byte swizzle, two 64-column
-    // halves; padding slots are zero), while the producer already streams
-    // K and V; the Q K^T issuer waits for all 128 slots
+    // the q row of this thread's slot into Q (padding slots are zero), while
+    // the producer already streams K and V; the Q K^T issuer waits for all
+    // 128 slots
     const int r = threadIdx.x;
-    int rho = r;  // the row of the slice held by slot r
-    bool valid = r < pc.nh;
-    if (SPREAD) {
-      const int rpq = (pc.nh + 3) / 4, li = r % 32;
-      rho = (r / 32) * rpq + li;
-      valid = li < rpq && rho < pc.nh;
-    }
-    const uint4 *src =
-        valid ? reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + rho) * D) : nullptr;
+    const int rho = tc_slot_row<SPREAD>(r, pc.nh);
+    const uint4 *src = rho >= 0 ? reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + rho) * D)
+                                : nullptr;
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-      const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-      const int h = c >> 3, c8 = c & 7;
-      *reinterpret_cast<uint4 *>(smem + TT::kQOff + h * TT::kQHalf + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
+      const uint4 v = rho >= 0 ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4 *>(smem + TT::kQOff + tc_q_offset<TT>(r, c)) = v;
     }
     fence_proxy_async_smem();
-    mbar_arrive(q_full);
+    mbar_arrive(bars.q_full0);
   }
   const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
 
   if (warp == kProducerWarp) {
     // ============================================================ producer
-    tc_produce<PAGED>(&tm_k, &tm_v, p, pc, sbase, full0, empty0, tile_bad, abort_flag, lane);
+    int tile = 0;
+    (void)tc_produce_piece<TT, PAGED>(&tm_k, &tm_v, p, pc, sbase, bars, tile_bad, abort_flag, lane, tile);
+    tc_produce_drain<TT>(bars, tile, lane);
   } else if (warp == kMmaWarp) {
     // ============================================================ Q K^T issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = tc_idesc_bf16(128, 64, false);
-      // Q's descriptors are the same for every tile; a K-step adds to the
-      // start-address field (addresses stay below 256 KB: no carry)
-      uint64_t qd[D / 16];
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-        qd[ks] = tc_smem_desc(sbase + TT::kQOff + (ks >> 2) * TT::kQHalf + (ks & 3) * 32, 16, 1024);
-      bool ok = mbar_wait(q_full, 0);
-      for (int t = 0; ok && t < n_tiles; ++t) {
-        // ---- S[t % SP] = Q K_t^T once K_t has landed and the buffer's last P.V is done
-        const int st = t % ST;
-        ok = mbar_wait(full0 + 8 * st, (t / ST) & 1);
-        if (ok && t >= SP) ok = mbar_wait(pv_done0 + 8 * (t % SP), ((t / SP) - 1) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t kd = tc_smem_desc(sbase + st * TT::kStageBytes, 16, 1024);
-        const uint32_t d = tmem + (t % SP) * 64;
-        tc_mma(d, qd[0], kd, kIdescQK, 0u);
-#pragma unroll
-        for (int ks = 1; ks < D / 16; ++ks)
-          tc_mma(d, qd[ks], kd + ((static_cast<uint32_t>((ks >> 2) * TT::kHalf + (ks & 3) * 32)) >> 4), kIdescQK, 1u);
-        tc_commit(s_full0 + 8 * (t % SP));
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        if (p.status) atomicOr(p.status, kStatusTimeout);
-      }
-      // every product this thread issued is done before the block tears down
-      // (on an early exit, products already issued may still be running)
-      tc_commit(drain0);
-      if (!mbar_wait(drain0, 0) && p.status) atomicOr(p.status, kStatusTimeout);
+      const bool ok = mbar_wait(bars.q_full0, 0) && tc_issue_qk<TT>(sbase, sbase + TT::kQOff, tmem, bars, 0, n_tiles);
+      if (!ok) tc_abort(p, abort_flag);
+      tc_issuer_drain(bars.drain0, p);
     }
   } else if (warp == kPvWarp) {
     // ============================================================ P.V issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescPV = tc_idesc_bf16(128, 128, true);
-      bool ok = true;
-      for (int u = 0; u < n_tiles; ++u) {
-        // ---- O += P_u V_u (high part and residual of P, from tensor memory)
-        const int st = u % ST;
-        ok = mbar_wait(p_full0 + 8 * (u % SP), (u / SP) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t vd = tc_smem_desc(sbase + st * TT::kStageBytes + TT::kTileBytes, TT::kHalf, 1024);
-        const uint32_t pb = tmem + (u % SP) * 64;
-#pragma unroll
-        for (int ks = 0; ks < T / 16; ++ks) {
-          // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of
-          // the buffer, the residual 16 columns further; into the O of the
-          // half of the row that owns them
-          // (SPREAD: the thread of tokens 16 ks .. wrote its high part at
-          // column 16 ks and its residual 8 columns further)
-          const uint64_t vdk = vd + ((ks * 16 * 128) >> 4);
-          const uint32_t pa = SPREAD ? pb + 16 * ks : pb + 32 * (ks >> 1) + 8 * (ks & 1);
-          const uint32_t od = tmem + TT::kOCol + D * (ks >> 1);
-          tc_mma_ts(od, pa, vdk, kIdescPV, (u > 0 || (ks & 1)) ? 1u : 0u);
-          tc_mma_ts(od, pa + (SPREAD ? 8 : 16), vdk, kIdescPV, 1u);
-        }
-        // K_u was read by the scores of tile u, done before its P existed; V_u
-        // and P_u by these products
-        tc_commit(empty0 + 8 * st);
-        tc_commit(pv_done0 + 8 * (u % SP));
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        if (p.status) atomicOr(p.status, kStatusTimeout);
-      }
-      tc_commit(drain0 + 8);
-      if (!mbar_wait(drain0 + 8, 0) && p.status) atomicOr(p.status, kStatusTimeout);
+      if (!tc_issue_pv<TT, SPREAD>(sbase, tmem, bars, 0, n_tiles)) tc_abort(p, abort_flag);
+      tc_issuer_drain(bars.drain0 + 8, p);
     }
-  } else if (SPREAD) {
-    // ============================================================ softmax rows, spread
-    tc_softmax_spread<PAGED>(p, pc, smem, tmem, s_full0, p_full0, pv_done0, tile_bad, abort_flag, merge_here,
-                             n_tiles, warp, lane);
   } else {
     // ============================================================ softmax rows
-    constexpr int kSM = 32 * TT::kSoftmaxWarps;  // softmax threads
-    const int sm = threadIdx.x;                  // 0 .. kSM-1
-    const int half = sm / 128;                   // tokens [32 half, 32 half + 32) of every tile
-    const int r = sm % 128;                      // row of the slice = tensor-memory lane
-    const bool valid = r < pc.nh;
-    const bool warp_active = (warp % 4) * 32 < pc.nh;
-    // the positions this row sees: with several query tokens per sequence,
-    // query token t sees the cache up to and including itself (a padding row,
-    // q = 0, sees the whole piece: its scores are 0, its result unused, and it
-    // keeps to the unmasked path of its warp)
-    const int lim = valid ? min(pc.t_end, pc.len - (p.nq - 1 - (pc.h0 + r) / p.r)) : pc.t_end;
-    const uint32_t lane_tmem = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-    float *mbase = reinterpret_cast<float *>(smem + TT::kXOff);  // [half][row]
-    float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);   // [half][row]
-    const float sl = p.scale_log2;
-    float m_run = kNegInf, l_run = 0.f;  // this half's base and sum
-    int bad = 0;
-    bool ok = true;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int t0 = pc.t_begin + t * T;
-      const int st = t % ST;
-      const int b = t % SP;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (t / SP) & 1));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sv[32];
-      tc_ld32(lane_tmem + b * 64 + half * 32, sv);
-      tc_wait_ld();
-      if (PAGED) bad |= tile_bad[st];
-      // V rows past the piece's end may hold anything (even NaN): zero them so
-      // that P = 0 there meets zeros
-      const int valid_rows = min(T, pc.t_end - t0);
-      if (valid_rows < T) {
-        uint8_t *vt = smem + st * TT::kStageBytes + TT::kTileBytes;
-        for (int idx = sm; idx < (T - valid_rows) * 16; idx += kSM) {
-          const int row = valid_rows + idx / 16, c = idx % 16;
-          *reinterpret_cast<uint4 *>(vt + (c >> 3) * TT::kHalf + row * 128 + ((c & 7) << 4)) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      float x[32];
-      const int tb = t0 + half * 32;  // this thread's first token of the tile
-      if (tb + 32 <= lim) {
-        // all of them visible (every tile but the row's last)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(sv[j]) * sl;
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
-      }
-      float mx;
-      {
-        float m8[8];  // a tree, not a chain of 32 dependent steps
-#pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(fmaxf(x[4 * k], x[4 * k + 1]), fmaxf(x[4 * k + 2], x[4 * k + 3]));
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      }
-      if (warp_active) {
-        // lazy rescale: only when a score passes the base by more than 2^8
-        const bool need = mx > m_run + 8.f;
-        if (__any_sync(0xffffffffu, need)) {
-          const float mn = need ? fmaxf(m_run, mx) : m_run;
-          const float alpha = need ? ((m_run == kNegInf) ? 0.f : ex2(m_run - mn)) : 1.f;
-          l_run *= alpha;
-          if (t > 0) {
-            // this half's O holds tiles 0 .. t-1: rescale it once their MMAs are done
-            ok = __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((t - 1) % SP), ((t - 1) / SP) & 1));
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tc_ld32(lane_tmem + TT::kOCol + half * D + c * 32, ov);
-              tc_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-              tc_st32(lane_tmem + TT::kOCol + half * D + c * 32, ov);
-            }
-            tc_wait_st();
-            tc_fence_before();
-          }
-          m_run = mn;
-        }
-        const float base = (m_run == kNegInf) ? 0.f : m_run;
-        // P over this thread's own 32 score columns: high part in the first
-        // 16, residual in the next 16 (the buffer's scores of tile t are no
-        // longer needed, and the MMAs of tile t-SP that read it are done, since
-        // the scores of tile t came after them)
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
-          l_run += p0 + p1;
-          split_bf16x2_rz(p0, p1, hi[e], lo[e]);
-        }
-        tc_st16(lane_tmem + b * 64 + half * 32, hi);
-        tc_st16(lane_tmem + b * 64 + half * 32 + 16, lo);
-        tc_wait_st();
-      }
-      // (p_full is one barrier per P buffer: a warp reaches tile t+SP only
-      // after s_full of t+SP, and the scores of t+SP are issued only once the
-      // P.V of tile t is done, so its next arrival on the same barrier cannot
-      // fall into tile t's phase)
-      tc_fence_before();
-      if (valid_rows < T) fence_proxy_async_smem();  // the zeroed V rows, for the tensor core
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full0 + 8 * b);
-    }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      if (p.status) atomicOr(p.status, kStatusTimeout);
-    }
-    // ---- the row's result: O from tensor memory once the last MMAs are done
-    const bool done =
-        ok && __all_sync(0xffffffffu, mbar_wait(pv_done0 + 8 * ((n_tiles - 1) % SP), ((n_tiles - 1) / SP) & 1));
-    tc_fence_after();
-    // the row's two partial states, merged exactly: M = max(m0, m1), weights
-    // 2^(m_h - M) (0 for a half that saw no position)
-    mbase[half * 128 + r] = m_run;
-    lsum[half * 128 + r] = l_run;
-    named_barrier(1, kSM);
-    const float m0 = mbase[r], m1 = mbase[128 + r];
-    const float m_row = fmaxf(m0, m1);
-    const float w0 = (m0 == kNegInf) ? 0.f : ex2(m0 - m_row), w1 = (m1 == kNegInf) ? 0.f : ex2(m1 - m_row);
-    const float l_row = lsum[r] * w0 + lsum[128 + r] * w1;
-    const bool final_row = ((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr;
-    const size_t row = valid ? row_of(p, pc.s, pc.g, pc.h0 + r) : 0;
-    const size_t ps = row * p.num_splits + pc.k;
-    const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
-    const float s0 = final_row ? w0 * inv : w0, s1 = final_row ? w1 * inv : w1;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t oa[32], ob[32];
-      const int col = half * 64 + c * 32;  // this thread writes columns [64 half, 64 half + 64)
-      tc_ld32(lane_tmem + TT::kOCol + col, oa);
-      tc_ld32(lane_tmem + TT::kOCol + D + col, ob);
-      tc_wait_ld();
-      if (valid) {
-        float4 *dst = reinterpret_cast<float4 *>((final_row ? p.out + row * D : p.part_o + ps * D) + col);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float v[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) v[e] = __uint_as_float(oa[4 * j + e]) * s0 + __uint_as_float(ob[4 * j + e]) * s1;
-          dst[j] = make_float4(v[0], v[1], v[2], v[3]);
-        }
-      }
-    }
-    if (valid && half == 0) {
-      if (final_row) {
-        if (p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(m_row, l_row);
-        if (p.part_l) p.part_l[row * p.num_splits] = kLFinal;
-      } else {
-        p.part_m[ps] = m_row;
-        p.part_l[ps] = bad ? kLBadPage : l_row;
-      }
-    }
-    tc_fence_before();
-    if (p.unit_ctr != nullptr && !final_row) tc_merge_unit(p, pc, sm, merge_here);
+    const TcDest dest{((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr, -1};
+    if (SPREAD)
+      (void)tc_softmax_spread<TT, PAGED>(p, pc, smem, tmem, bars, tile_bad, abort_flag, merge_here, stop, 0,
+                                         n_tiles, dest, warp, lane);
+    else
+      (void)tc_softmax_wide<TT, PAGED>(p, pc, smem, tmem, bars, tile_bad, abort_flag, merge_here, stop, 0,
+                                       n_tiles, dest, warp, lane);
   }
 
   // ---- teardown: every tensor-memory access is done before the columns go
   // back (the two issuers waited above for their last products to finish)
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tc_dealloc(tmem, TT::kTmemCols);
+  }
+}
+
+// Equal-work ranges on the tcgen05 tensor cores: one persistent block per SM
+// walks its range [c W / N, (c + 1) W / N) of the W tiles of all (sequence,
+// group) units (the Walker of the mma.sync kernel's balanced mode; every role
+// walks the same pieces).  Per piece n: the producer warp fills Q buffer n % 2
+// (once the Q K^T products of piece n - 2 are done with it) and streams the
+// piece's tiles into the ring, which runs on across pieces; the Q K^T issuer
+// takes Q buffer n % 2; the P.V issuer starts the piece's accumulators once
+// the softmax warps have read piece n - 1's O out (o_free); the softmax warps
+// write whole units' rows final and the (at most two) units shared with a
+// neighbouring block as partial states in the block's two slots, with the
+// records the balanced combine kernel merges them from.
+template <bool PAGED, bool SPREAD>
+__global__ void __launch_bounds__(TcBalTile::kThreads, 1)
+    gqa_verify_tc_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                  const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+  using TT = TcBalTile;
+  constexpr int T = TT::kT;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const TcBars bars = tc_bars<TT>(sbase);
+  volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
+  volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
+  volatile int *abort_flag = tile_bad + TT::kStages;
+  volatile int *merge_here = tile_bad + TT::kStages + 1;  // (no in-kernel merge in this mode)
+  volatile int *stop = tile_bad + TT::kStages + 2;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int kProducerWarp = TT::kSoftmaxWarps;
+  constexpr int kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
+
+  if (threadIdx.x == 0) {
+    tc_init_bars<TT>(bars, tile_bad, 1);  // the producer warp arrives once per Q buffer fill
+    *abort_flag = 0;
+    *merge_here = 0;
+    *stop = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tc_alloc(smem_addr(const_cast<uint32_t *>(tmem_slot)), TT::kTmemCols);
+    tc_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  pdl_wait_primary();
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  Walker wk;
+  Piece pc;
+  walker_init<T>(wk, p, lane);  // every lane of every warp: the same pieces
+  bool have = walker_next<T>(wk, p, pc);
+
+  if (warp == kProducerWarp) {
+    // ============================================================ producer
+    int tile = 0;
+    for (int n = 0; have; ++n) {
+      const int qb = n % 2;
+      if (n >= 2) {
+        bool ok = lane == 0 ? mbar_wait(bars.q_empty0 + 8 * qb, ((n / 2) - 1) & 1) : true;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok || *abort_flag) {
+          if (lane == 0) tc_abort(p, abort_flag);
+          break;
+        }
+      }
+      tc_fill_q_warp<TT, SPREAD>(p, pc, smem + TT::kQOff + qb * TT::kQBytes, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.q_full0 + 8 * qb);
+      if (!tc_produce_piece<TT, PAGED>(&tm_k, &tm_v, p, pc, sbase, bars, tile_bad, abort_flag, lane, tile)) break;
+      have = walker_next<T>(wk, p, pc);
+    }
+    tc_produce_drain<TT>(bars, tile, lane);
+  } else if (warp == kMmaWarp) {
+    // ============================================================ Q K^T issuer
+    if (lane == 0) {
+      int gt = 0;
+      for (int n = 0; have; ++n) {
+        const int qb = n % 2;
+        const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
+        bool ok = mbar_wait(bars.q_full0 + 8 * qb, (n / 2) & 1) && !*abort_flag;
+        ok = ok && tc_issue_qk<TT>(sbase, sbase + TT::kQOff + qb * TT::kQBytes, tmem, bars, gt, n_tiles);
+        if (!ok) {
+          tc_abort(p, abort_flag);
+          break;
+        }
+        tc_commit(bars.q_empty0 + 8 * qb);  // Q buffer qb is free once these products are done
+        gt += n_tiles;
+        have = walker_next<T>(wk, p, pc);
+      }
+      tc_issuer_drain(bars.drain0, p);
+    }
+  } else if (warp == kPvWarp) {
+    // ============================================================ P.V issuer
+    if (lane == 0) {
+      int gt = 0;
+      for (int n = 0; have; ++n) {
+        const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
+        // the piece's products start O afresh: the previous piece's O must be read out
+        bool ok = (n == 0 || mbar_wait(bars.o_free, (n - 1) & 1)) && !*abort_flag;
+        if (ok) tc_fence_after();
+        ok = ok && tc_issue_pv<TT, SPREAD>(sbase, tmem, bars, gt, n_tiles);
+        if (!ok) {
+          tc_abort(p, abort_flag);
+          break;
+        }
+        gt += n_tiles;
+        have = walker_next<T>(wk, p, pc);
+      }
+      tc_issuer_drain(bars.drain0 + 8, p);
+    }
+  } else {
+    // ============================================================ softmax rows
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      p.ws_header[0] = static_cast<int>(gridDim.x);
+      p.ws_header[1] = p.capacity;
+      p.ws_header[2] = static_cast<int>(wk.W & 0xffffffff);
+      p.ws_header[3] = static_cast<int>(wk.W >> 32);
+    }
+    int gt = 0;
+    while (have) {
+      const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
+      if (threadIdx.x == 0 && pc.first_of_unit)
+        p.ws_meta[(static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j] =
+            make_int4(static_cast<int>(blockIdx.x), pc.last_block, pc.slot & 1, 0);
+      const TcDest dest{pc.final_row, pc.slot};
+      const bool go = SPREAD ? tc_softmax_spread<TT, PAGED>(p, pc, smem, tmem, bars, tile_bad, abort_flag,
+                                                           merge_here, stop, gt, n_tiles, dest, warp, lane)
+                             : tc_softmax_wide<TT, PAGED>(p, pc, smem, tmem, bars, tile_bad, abort_flag, merge_here,
+                                                         stop, gt, n_tiles, dest, warp, lane);
+      // O has been read out: the next piece's P.V products may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.o_free);
+      if (!go) break;
+      gt += n_tiles;
+      have = walker_next<T>(wk, p, pc);
+    }
+  }
+
+  // ---- teardown: every tensor-memory access is done before the columns go back
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

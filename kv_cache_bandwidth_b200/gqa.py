@@ -22,7 +22,8 @@ import torch
 __all__ = [
     "GqaError", "Dims", "load", "lib_path", "gqa_decode", "gqa_decode_split",
     "gqa_split_partials", "gqa_split_combine", "gqa_decode_split_workspace_size",
-    "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version", "dims_for",
+    "gqa_plan_split_tokens", "gqa_plan_decomposition", "PLAN_EQUAL_WORK", "PLAN_FIXED_SPLITS", "PLAN_CLUSTERS",
+    "gqa_status_string", "gqa_abi_version", "dims_for",
     "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
     "FLAG_CONTRACT_FMA", "FLAG_CONTRACT_TCGEN05", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
     "gqa_decode_split_lse", "gqa_merge_lse", "SERIAL_MERGE_MAX_SPLITS", "gqa_kv_append", "PagePool",
@@ -95,6 +96,9 @@ def load():
     lib.gqa_decode_split_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32]
     lib.gqa_plan_split_tokens.restype = ctypes.c_int32
     lib.gqa_plan_split_tokens.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32]
+    lib.gqa_plan_decomposition.restype = ctypes.c_int32
+    lib.gqa_plan_decomposition.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     lib.gqa_decode_split_static.restype = ctypes.c_int
     lib.gqa_decode_split_static.argtypes = _DECODE_ARGS + [ctypes.c_int32, ctypes.c_int32, _vp]
     lib.gqa_decode_split_lse.restype = ctypes.c_int
@@ -201,6 +205,22 @@ def gqa_plan_split_tokens(dims: Dims, max_seqlen: int, num_sms: int = 0) -> int:
     if rc < 0:
         raise GqaError(rc, "gqa_plan_split_tokens")
     return rc
+
+
+PLAN_EQUAL_WORK = 0
+PLAN_FIXED_SPLITS = 1
+PLAN_CLUSTERS = 2
+
+
+def gqa_plan_decomposition(dims: Dims, max_seqlen: int, num_sms: int = 0):
+    """(plan, split_tokens, blocks per cluster) that gqa_decode_split runs with
+    split_tokens == 0 (plan: PLAN_EQUAL_WORK, PLAN_FIXED_SPLITS or PLAN_CLUSTERS)."""
+    split, cluster = ctypes.c_int32(0), ctypes.c_int32(0)
+    rc = int(load().gqa_plan_decomposition(ctypes.byref(dims), int(max_seqlen), int(num_sms),
+                                           ctypes.byref(split), ctypes.byref(cluster)))
+    if rc < 0:
+        raise GqaError(rc, "gqa_plan_decomposition")
+    return rc, int(split.value), int(cluster.value)
 
 
 def workspace_for(q, k_cache, page_table, max_seqlen: int, split_tokens: int, flags: int = 0) -> torch.Tensor:

@@ -30,7 +30,8 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("gqa_decode", "gqa_decode_split", "gqa_decode_split_workspace_size", "gqa_split_partials",
-              "gqa_split_combine", "gqa_plan_split_tokens", "gqa_status_string", "gqa_abi_version",
+              "gqa_split_combine", "gqa_plan_split_tokens", "gqa_plan_decomposition", "gqa_status_string",
+              "gqa_abi_version",
               "gqa_decode_split_lse", "gqa_merge_lse", "gqa_decode_split_static", "gqa_kv_append",
               "gqa_page_pool_create", "gqa_page_pool_alloc", "gqa_page_pool_free", "gqa_page_pool_available",
               "gqa_page_pool_destroy"):
@@ -162,10 +163,13 @@ def test_plan_split_tokens(lib):
     d1 = _dims(batch=1, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072)
     t1 = gqa.gqa_plan_split_tokens(d1, 131072, 148)
     assert t1 == 1792 and 4 * -(-131072 // t1) == 296
-    # MQA sweep (r = 32 runs one block per SM): 16 units -> 9 splits -> 144 items
+    # MQA sweep (r = 32: the tcgen05 kernel): equal-work ranges over persistent blocks
     d2 = _dims(batch=16, num_heads=32, num_kv_heads=1, head_dim=128, page_size=8192)
-    t2 = gqa.gqa_plan_split_tokens(d2, 8192, 148)
-    assert 16 * -(-8192 // t2) <= 148 and t2 == 1024
+    assert gqa.gqa_plan_split_tokens(d2, 8192, 148) == 0
+    # forced mma.sync contraction for the same shape: fixed splits, 16-row slices
+    d2m = _dims(batch=16, num_heads=32, num_kv_heads=1, head_dim=128, page_size=8192, flags=gqa.FLAG_CONTRACT_MMA)
+    t2 = gqa.gqa_plan_split_tokens(d2m, 8192, 148)
+    assert t2 > 0 and 32 * -(-8192 // t2) <= 296
     # paged: equal-work ranges, or splits of 4096 above 1024 sequences
     d3 = _dims(batch=64, num_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=70000,
                max_pages_per_seq=2048)
@@ -292,3 +296,32 @@ def test_test_hooks_only_in_the_test_library(lib):
     hooks = ctypes.CDLL(gqa_build.TEST_LIB)
     assert hasattr(hooks, "gqa_test_skip_tile")
     assert hasattr(hooks, "gqa_decode_split")
+
+
+def test_plan_decomposition(lib):
+    """The decomposition gqa_decode_split runs with split_tokens = 0: clusters
+    for contiguous caches whose units are too few for one block each but fill
+    the GPU as portable clusters; fixed splits or equal-work ranges otherwise."""
+    def plan(**kw):
+        return gqa.gqa_plan_decomposition(_dims(**kw), kw.pop("_len", kw["page_size"]), 148)
+    sweep = dict(batch=16, num_heads=32, head_dim=128, page_size=8192)
+    assert plan(num_kv_heads=2, **sweep) == (gqa.PLAN_CLUSTERS, 0, 8)     # 32 units x 8 = 256 blocks
+    assert plan(num_kv_heads=4, **sweep) == (gqa.PLAN_CLUSTERS, 0, 4)     # 64 units x 4
+    assert plan(num_kv_heads=8, **sweep) == (gqa.PLAN_CLUSTERS, 0, 2)     # 128 units x 2
+    # r = 32: the tcgen05 kernel, equal-work ranges
+    assert plan(num_kv_heads=1, **sweep) == (gqa.PLAN_EQUAL_WORK, 0, 1)
+    # MHA: 512 units fill the GPU one block each
+    assert plan(num_kv_heads=32, **sweep) == (gqa.PLAN_FIXED_SPLITS, 8192, 1)
+    # Llama-2-70B layer: one split per unit; long context, 4 units: clusters would be too few
+    assert plan(batch=32, num_heads=64, num_kv_heads=8, head_dim=128, page_size=4096) == (
+        gqa.PLAN_FIXED_SPLITS, 4096, 1)
+    assert plan(batch=1, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072) == (
+        gqa.PLAN_FIXED_SPLITS, 1792, 1)
+    # paged: equal-work ranges
+    d3 = _dims(batch=64, num_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=70000,
+               max_pages_per_seq=2048)
+    assert gqa.gqa_plan_decomposition(d3, 32768, 148) == (gqa.PLAN_EQUAL_WORK, 0, 1)
+    # the two-kernel plan is unchanged by the cluster choice
+    assert gqa.gqa_plan_split_tokens(_dims(num_kv_heads=2, **sweep), 8192, 148) == 1024
+    assert lib.gqa_plan_decomposition(None, 10, 148, None, None) == -1
+    assert lib.gqa_plan_decomposition(ctypes.byref(_dims(num_heads=9)), 10, 148, None, None) == -3

@@ -494,3 +494,30 @@ def test_prefix_shared_pages(entry, split):
     b_inp.page_table.copy_(dup)
     got_dup, _ = run_gpu(b_inp, entry, split_tokens=split)
     assert torch.equal(got, got_dup)
+
+
+def test_split_entry_runs_clusters_for_few_units():
+    """A contiguous cache with 32 (sequence, group) units: gqa_decode_split
+    with split_tokens = 0 runs thread-block clusters (merged through
+    distributed shared memory) and agrees with the oracle, lengths from 1 to
+    the capacity mixed; an invalid length sets its status bit and zeroes its
+    rows; the lse entry point keeps to fixed splits and agrees too."""
+    w = Workload(name="few units", b=16, H=8, G=2, d=64, m=2048, seed=41)
+    lens = [2048, 1, 5, 129, 2047, 300, 1024, 77, 2048, 640, 1500, 64, 65, 999, 2000, 3]
+    inp = make_inputs(w, device="cuda", lens=lens)
+    dims = gqa.dims_for(inp.q, inp.k_cache, None)
+    assert gqa.gqa_plan_decomposition(dims, 2048)[0] == gqa.PLAN_CLUSTERS
+    ref, st_ref = run_oracle(inp)
+    assert st_ref == 0
+    got, st = run_gpu(inp, "split", split_tokens=0, max_seqlen=2048)
+    assert st == 0
+    assert_parity(got, ref, "clusters through gqa_decode_split")
+    out, lse = gqa.gqa_decode_split_lse(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, None, max_seqlen=2048)
+    torch.cuda.synchronize()
+    assert_parity(out, ref, "lse entry point")
+    inp.seqlens[5] = 0
+    got, st = run_gpu(inp, "split", split_tokens=0, max_seqlen=2048)
+    assert st == gqa.STATUS_BAD_SEQLEN
+    assert torch.all(got[5] == 0)
+    keep = [s for s in range(w.b) if s != 5]
+    assert_parity(got[keep], ref[keep], "valid rows next to an invalid one")
