@@ -394,8 +394,6 @@ class Case:
         elif nq == 1 and self.entry == "split":
             kind, self.eff_split, c = gqa.gqa_plan_decomposition(self.dims, self.max_seqlen)
             self.cluster = c if kind == gqa.PLAN_CLUSTERS else 0
-        elif self.tc:
-            self.eff_split = 0  # the tcgen05 kernel: equal-work ranges
         else:
             self.eff_split = gqa.gqa_plan_split_tokens(self.dims, self.max_seqlen)
         n_splits = -(-self.max_seqlen // self.eff_split) if self.eff_split > 0 else 0
@@ -502,7 +500,7 @@ class Case:
         return max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
 
     def kernel_name(self):
-        tc_name = "gqa_verify_tc_balanced_kernel" if self.eff_split == 0 else "gqa_verify_tc_kernel"
+        tc_name = "gqa_verify_tc_kernel"
         if self.nq > 1:
             return "%s (verification, %d rows per KV group%s)" % (
                 tc_name if self.tc else "gqa_decode_kernel", self.nq * self.w.r,

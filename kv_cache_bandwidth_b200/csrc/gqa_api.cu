@@ -372,15 +372,19 @@ int launch_verify_tc(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &
   const bool spread = sh.rc <= 64;
   auto kernel = sh.paged ? (spread ? gqa::gqa_verify_tc_kernel<true, true> : gqa::gqa_verify_tc_kernel<true, false>)
                          : (spread ? gqa::gqa_verify_tc_kernel<false, true> : gqa::gqa_verify_tc_kernel<false, false>);
-  constexpr int smem = gqa::TcTile::kSmemBytes;
+  const int smem = spread ? gqa::TcTileSpread::kSmemBytes : gqa::TcTile::kSmemBytes;
   static std::atomic<unsigned long long> attr_set{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load(std::memory_order_acquire) & bit)) {
-    for (auto k : {gqa::gqa_verify_tc_kernel<true, true>, gqa::gqa_verify_tc_kernel<true, false>,
-                   gqa::gqa_verify_tc_kernel<false, true>, gqa::gqa_verify_tc_kernel<false, false>})
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    for (auto k : {gqa::gqa_verify_tc_kernel<true, true>, gqa::gqa_verify_tc_kernel<false, true>})
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gqa::TcTileSpread::kSmemBytes) !=
+          cudaSuccess)
+        return GQA_ERR_CUDA;
+    for (auto k : {gqa::gqa_verify_tc_kernel<true, false>, gqa::gqa_verify_tc_kernel<false, false>})
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gqa::TcTile::kSmemBytes) !=
+          cudaSuccess)
         return GQA_ERR_CUDA;
     attr_set.fetch_or(bit, std::memory_order_acq_rel);
   }
@@ -395,43 +399,6 @@ int launch_verify_tc(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &
   cfg.attrs = attr;
   cfg.numAttrs = l.pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
-}
-
-// The tcgen05 kernel on equal-work ranges: one persistent block per SM
-// (grid.x holds the SM count on entry); returns the number of blocks.
-constexpr int kMaxBalancedBlocksTc = 256;
-
-int launch_tc_balanced(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p,
-                       const Launch &l) {
-  const bool spread = sh.rc <= 64;
-  auto kernel = sh.paged ? (spread ? gqa::gqa_verify_tc_balanced_kernel<true, true>
-                                   : gqa::gqa_verify_tc_balanced_kernel<true, false>)
-                         : (spread ? gqa::gqa_verify_tc_balanced_kernel<false, true>
-                                   : gqa::gqa_verify_tc_balanced_kernel<false, false>);
-  constexpr int smem = gqa::TcBalTile::kSmemBytes;
-  static std::atomic<unsigned long long> attr_set{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_set.load(std::memory_order_acquire) & bit)) {
-    for (auto k : {gqa::gqa_verify_tc_balanced_kernel<true, true>, gqa::gqa_verify_tc_balanced_kernel<true, false>,
-                   gqa::gqa_verify_tc_balanced_kernel<false, true>, gqa::gqa_verify_tc_balanced_kernel<false, false>})
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return GQA_ERR_CUDA;
-    attr_set.fetch_or(bit, std::memory_order_acq_rel);
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(std::min<unsigned>(l.grid.x, kMaxBalancedBlocksTc), 1, 1);
-  cfg.blockDim = dim3(gqa::TcBalTile::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = l.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, tk, tv, p) != cudaSuccess) return GQA_ERR_CUDA;
-  return static_cast<int>(cfg.gridDim.x);
 }
 
 int encode_maps(const Shape &sh, const void *k, const void *v, CUtensorMap *tk, CUtensorMap *tv) {
@@ -535,7 +502,7 @@ struct BalancedWorkspace {
 
 BalancedWorkspace balanced_layout(const Shape &sh) {
   BalancedWorkspace w;
-  const size_t rows = static_cast<size_t>(sh.tc ? kMaxBalancedBlocksTc : kMaxBalancedBlocks) * 2 * sh.rc;
+  const size_t rows = static_cast<size_t>(kMaxBalancedBlocks) * 2 * sh.rc;
   w.meta_off = 256;
   w.o_off = w.meta_off + round256(static_cast<size_t>(units_of(sh)) * 16);
   w.m_off = w.o_off + round256(rows * sh.D * sizeof(float));
@@ -574,7 +541,7 @@ int run_balanced_decode(const Shape &sh, int sms, const void *q, const void *k, 
   p.lse = ex.lse;
   p.empty_ok = ex.empty_ok ? 1 : 0;
   Launch l{dim3(static_cast<unsigned>(sms), 1, 1), 1, stream};
-  rc = sh.tc ? launch_tc_balanced(sh, tk, tv, p, l) : launch_decode<Mode::kBalanced>(sh, tk, tv, p, l);
+  rc = launch_decode<Mode::kBalanced>(sh, tk, tv, p, l);
   return rc < 0 ? rc : GQA_OK;
 }
 
@@ -602,7 +569,8 @@ int run_balanced_combine(const Shape &sh, const int32_t *seqlens, float *out, ui
   c.lse = ex.lse;
   c.empty_ok = ex.empty_ok ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(units_of(sh) * sh.rc), 1, 1);
+  const int rows_per_block = 128 / (sh.D / 4);  // the combine's rows per block
+  cfg.gridDim = dim3(static_cast<unsigned>(units_of(sh) * ((sh.rc + rows_per_block - 1) / rows_per_block)), 1, 1);
   cfg.blockDim = dim3(128, 1, 1);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -630,10 +598,9 @@ struct AutoChoice {
 
 bool dims_paged(const gqa_dims *dims) { return dims->max_pages_per_seq > 0; }
 
-// Equal-work ranges serve paged dims, and the tcgen05 kernel in either
-// layout (its persistent blocks would otherwise run units in waves of one
-// block per SM); a group table runs on fixed splits only.
-bool balanced_ok(const gqa_dims *dims, const Shape &sh) { return (dims_paged(dims) || sh.tc) && !sh.mapped; }
+// Equal-work ranges serve paged dims, with neither a group table nor the
+// tcgen05 kernel (both run on fixed splits only).
+bool balanced_ok(const gqa_dims *dims, const Shape &sh) { return dims_paged(dims) && !sh.mapped && !sh.tc; }
 
 int round_split(long long tokens) {
   tokens = (tokens + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;

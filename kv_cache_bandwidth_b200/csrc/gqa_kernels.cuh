@@ -546,8 +546,9 @@ __device__ __forceinline__ bool unit_arrive(unsigned long long *word, unsigned l
 }
 
 // NV float4 outputs (columns 4*c4 .. 4*c4+3 for c4 = c4_0 + i*c4_step, i < NV)
-// of one merged row from the row's ns <= kSerialMergeMax partial states at
-// slots base .. base + ns - 1, for rows with few splits.  Every thread works
+// of one merged row from the row's ns partial states at slots slot(0) ..
+// slot(ns - 1) (a negative slot: no contribution; slot(0) is one), for rows
+// with few splits (one round trip to L2 per kSerialMergeMax of them).  Every thread works
 // alone (no barriers) and issues all its loads before it uses any, so the
 // merge costs about one trip to L2; each output takes the contributions in
 // ascending k with one accumulator, the same whatever NV is.  The decode
@@ -555,38 +556,61 @@ __device__ __forceinline__ bool unit_arrive(unsigned long long *word, unsigned l
 // two agree bit for bit.
 constexpr int kSerialMergeMax = 8;
 
-template <int D, int NV>
-__device__ __forceinline__ void merge_serial(const float *part_o, const float *part_m, const float *part_l,
-                                             long long base, int ns, int c4_0, int c4_step, float4 *dst_row,
-                                             float *lse_dst) {
+template <int D, int NV, bool CHUNKED = false, typename SlotFn>
+__device__ __forceinline__ void merge_serial_at(const float *part_o, const float *part_m, const float *part_l,
+                                                SlotFn slot, int ns, int c4_0, int c4_step, float4 *dst_row,
+                                                float *lse_dst) {
   const float kNegInf = -__int_as_float(0x7f800000);
-  float m[kSerialMergeMax], l[kSerialMergeMax];
-  float4 v[NV][kSerialMergeMax];
-#pragma unroll
-  for (int k = 0; k < kSerialMergeMax; ++k) {
-    const long long kk = base + min(k, ns - 1);  // every load issued (slots past ns repeat the last)
-    m[k] = __ldcg(part_m + kk);
-    l[k] = __ldcg(part_l + kk);
-#pragma unroll
-    for (int i = 0; i < NV; ++i) v[i][k] = __ldcg(reinterpret_cast<const float4 *>(part_o + kk * D) + c4_0 + i * c4_step);
-  }
-  float M = kNegInf;
-  bool bad = false;
-#pragma unroll
-  for (int k = 0; k < kSerialMergeMax; ++k) {
-    if (k < ns) {
-      M = fmaxf(M, m[k]);
-      bad |= l[k] < 0.f;
-    }
-  }
+  const long long first = slot(0);
+  float M = kNegInf;  // running maximum over the chunks so far
+  float L = 0.f;
   float4 acc[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float L = 0.f;
-  if (!bad && M != kNegInf) {
+  bool bad = false;
+  // chunks of kSerialMergeMax contributions (CHUNKED; otherwise ns <=
+  // kSerialMergeMax, one chunk), merged online: the sums so far are rescaled
+  // by 2^(M_old - M_new)
+  const int k_end = CHUNKED ? ns : 1;
+  for (int k0 = 0; k0 < k_end; k0 += kSerialMergeMax) {
+    float m[kSerialMergeMax], l[kSerialMergeMax];
+    float4 v[NV][kSerialMergeMax];
+    bool use[kSerialMergeMax];
 #pragma unroll
     for (int k = 0; k < kSerialMergeMax; ++k) {
-      if (k < ns) {
+      long long kk = k0 + k < ns ? slot(k0 + k) : -1;
+      use[k] = kk >= 0;
+      if (!use[k]) kk = first;  // every load issued (unused ones repeat the first)
+      m[k] = __ldcg(part_m + kk);
+      l[k] = __ldcg(part_l + kk);
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        v[i][k] = __ldcg(reinterpret_cast<const float4 *>(part_o + kk * D) + c4_0 + i * c4_step);
+    }
+    float Mc = M;
+#pragma unroll
+    for (int k = 0; k < kSerialMergeMax; ++k) {
+      if (use[k]) {
+        Mc = fmaxf(Mc, m[k]);
+        bad |= l[k] < 0.f;
+      }
+    }
+    if (bad || Mc == kNegInf) continue;
+    if (M != Mc) {
+      const float r = (M == kNegInf) ? 0.f : ex2(M - Mc);
+      L *= r;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        acc[i].x *= r;
+        acc[i].y *= r;
+        acc[i].z *= r;
+        acc[i].w *= r;
+      }
+      M = Mc;
+    }
+#pragma unroll
+    for (int k = 0; k < kSerialMergeMax; ++k) {
+      if (use[k]) {
         const float w = ex2(m[k] - M);
         L += l[k] * w;
 #pragma unroll
@@ -606,6 +630,15 @@ __device__ __forceinline__ void merge_serial(const float *part_o, const float *p
     dst_row[c4_0 + i * c4_step] = res;
   }
   if (lse_dst && c4_0 == 0) *lse_dst = bad ? kNegInf : lse_from_state(M, L);
+}
+
+// merge_serial_at over the ns consecutive slots base .. base + ns - 1.
+template <int D, int NV>
+__device__ __forceinline__ void merge_serial(const float *part_o, const float *part_m, const float *part_l,
+                                             long long base, int ns, int c4_0, int c4_step, float4 *dst_row,
+                                             float *lse_dst) {
+  merge_serial_at<D, NV>(part_o, part_m, part_l, [base](int k) -> long long { return base + k; }, ns, c4_0, c4_step,
+                         dst_row, lse_dst);
 }
 
 // The q.k and p.v contractions on CUDA cores (fp32 FMA) for group ratios
@@ -1537,29 +1570,38 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p)
                threadIdx.x, sc, [] { __syncthreads(); });
 }
 
-// Balanced mode: one block per (unit, head).  The decode kernel recorded, for
-// every unit, the first and last decode blocks holding its tiles and the slot
-// the first one used; every later block holds the unit's first piece of its
-// own range (slot 0), unless its range is empty.  Units one block covered whole
-// are final already; units with an invalid length get zero rows here.
+// Balanced mode: one block per (unit, group of 128 / (D / 4) rows), one
+// float4 column of one row per thread.  The decode kernel recorded, for every
+// unit, the first and last decode blocks holding its tiles and the slot the
+// first one used; every later block holds the unit's first piece of its own
+// range (slot 0), unless its range is empty.  Units one block covered whole
+// are final already; units with an invalid length get zero rows here.  Up to
+// 4 kSerialMergeMax contributions each thread merges its column alone
+// (merge_serial_at: no barriers, kSerialMergeMax loads in flight at once);
+// more, and the block merges its rows one after another with merge_row.
 template <int D, int T>
 __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const CombineParams p) {
-  const int u = blockIdx.x / p.rc;  // unit: (sequence, group, head slice)
-  const int h = blockIdx.x % p.rc;
+  constexpr int kTPR = D / 4;         // threads per row
+  constexpr int kRPB = 128 / kTPR;    // rows per block
+  const int rblocks = (p.rc + kRPB - 1) / kRPB;
+  const int u = blockIdx.x / rblocks;  // unit: (sequence, group, head slice)
+  const int h0 = (blockIdx.x % rblocks) * kRPB;
   const int j = u % p.hs;
   const int s = u / (p.G * p.hs), g = (u / p.hs) % p.G;
-  if (j * p.rc + h >= p.rq) return;  // the last slice of the group is narrower
-  const size_t row = out_row(s, g, j * p.rc + h, p.nq, p.r, p.H);
-  float4 *dst = reinterpret_cast<float4 *>(p.out + row * D) + threadIdx.x % (D / 4);
+  const int c4 = threadIdx.x % kTPR;
+  const int h = h0 + threadIdx.x / kTPR;
+  const bool row_ok = h < p.rc && j * p.rc + h < p.rq;  // (the last slice of a group is narrower)
+  const size_t row = row_ok ? out_row(s, g, j * p.rc + h, p.nq, p.r, p.H) : 0;
+  float4 *dst = reinterpret_cast<float4 *>(p.out + row * D);
   const int len = __ldg(p.seqlens + s);
   pdl_wait_primary();  // the header, unit records and partial states come from the decode kernel
   const int N = p.ws_header[0];
   const int capacity = p.ws_header[1];
-  float *lse_dst = p.lse ? p.lse + row : nullptr;
+  float *lse_dst = (p.lse && row_ok) ? p.lse + row : nullptr;
   if (len < p.nq || len > capacity) {
-    if (threadIdx.x < D / 4) *dst = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (threadIdx.x == 0 && lse_dst) *lse_dst = -__int_as_float(0x7f800000);
-    if (threadIdx.x == 0 && h == 0 && p.status && !(p.empty_ok && len == 0)) atomicOr(p.status, kStatusBadSeqlen);
+    if (row_ok) dst[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c4 == 0 && lse_dst) *lse_dst = -__int_as_float(0x7f800000);
+    if (threadIdx.x == 0 && h0 == 0 && p.status && !(p.empty_ok && len == 0)) atomicOr(p.status, kStatusBadSeqlen);
     return;
   }
   const long long W = static_cast<long long>(static_cast<unsigned>(p.ws_header[2])) |
@@ -1567,14 +1609,30 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
   const int4 meta = p.ws_meta[u];
   const int c_lo = meta.x, c_hi = meta.y, slot_lo = meta.z;
   if (c_lo == c_hi) return;  // one decode block covered the unit: its rows are final
+  const int nc = c_hi - c_lo + 1;
+  if (nc <= 4 * kSerialMergeMax) {
+    if (row_ok)
+      merge_serial_at<D, 1, true>(p.part_o, p.part_m, p.part_l,
+                                  [&](int k) -> long long {
+                              const long long c = c_lo + k;
+                              if (k > 0 && (c * W / N) == ((c + 1) * W / N)) return -1;  // empty range
+                              return (2 * c + (k == 0 ? slot_lo : 0)) * p.rc + h;
+                            },
+                            nc, c4, 0, dst, lse_dst);
+    return;
+  }
   __shared__ MergeScratch<D> sc;
-  merge_row<D>(p.part_o, p.part_m, p.part_l, c_hi - c_lo + 1,
-               [&](int k) -> long long {
-                 const long long c = c_lo + k;
-                 if (k > 0 && (c * W / N) == ((c + 1) * W / N)) return -1;  // empty range
-                 return (2 * c + (k == 0 ? slot_lo : 0)) * p.rc + h;
-               },
-               dst, lse_dst, threadIdx.x, sc, [] { __syncthreads(); });
+  for (int hh = h0; hh < h0 + kRPB && hh < p.rc && j * p.rc + hh < p.rq; ++hh) {  // (uniform in the block)
+    const size_t row2 = out_row(s, g, j * p.rc + hh, p.nq, p.r, p.H);
+    merge_row<D>(p.part_o, p.part_m, p.part_l, nc,
+                 [&](int k) -> long long {
+                   const long long c = c_lo + k;
+                   if (k > 0 && (c * W / N) == ((c + 1) * W / N)) return -1;  // empty range
+                   return (2 * c + (k == 0 ? slot_lo : 0)) * p.rc + hh;
+                 },
+                 reinterpret_cast<float4 *>(p.out + row2 * D) + threadIdx.x % kTPR,
+                 p.lse ? p.lse + row2 : nullptr, threadIdx.x, sc, [] { __syncthreads(); });
+  }
 }
 
 // Merge of normalised partial results weighted by their log-sum-exp, e.g. the

@@ -38,17 +38,10 @@
 // The epilogue writes final rows or partial states in the layout of the
 // mma.sync kernel, so the same merges (in this kernel for up to 8 splits, the
 // combine kernel otherwise) apply.
-//
-// Two decompositions: one block per (sequence, group, split) item
-// (gqa_verify_tc_kernel), or equal-work ranges (gqa_verify_tc_balanced_kernel):
-// one persistent block per SM walks its contiguous range of the tiles of all
-// (sequence, group) units, the K/V ring streaming across unit boundaries; Q
-// is double-buffered (the producer warp fills the next unit's Q while the
-// current one runs), and the P.V products of a new unit wait only until the
-// softmax warps have read the previous unit's O out of tensor memory.  Units
-// shared with a neighbouring block leave partial states for the balanced
-// combine kernel, exactly as in the mma.sync kernel's equal-work mode.
+
 #pragma once
+
+#include <type_traits>
 
 #include "gqa_kernels.cuh"
 #include "tc05.cuh"
@@ -56,19 +49,27 @@
 namespace gqa {
 
 // Shared-memory layout of the tcgen05 kernels: a STAGES-deep ring of K/V tiles
-// of 64 tokens (32 KB per stage) and QBUFS buffers of Q (128 rows x d = 128).
-template <int STAGES, int QBUFS>
+// of 64 tokens (32 KB per stage) and QBUFS buffers of Q (QROWS rows x d = 128).
+// QROWS = 128: the Q K^T product has M = 128, row i in tensor-memory lane i.
+// QROWS = 64 (at most 64 rows, SPREAD): M = 64, whose accumulator rows sit in
+// the first 16 lanes of each 32-lane quarter (row m in lane m % 16 + 32 (m /
+// 16)), exactly where the spread softmax reads them; Q then takes half the
+// shared memory.  The P.V product always has M = 128 (P from tensor memory,
+// lane = row): the lanes no row uses hold leftovers whose products land in O
+// rows that are never read.
+template <int STAGES, int QBUFS, int QROWS>
 struct TcLayout {
   static constexpr int kD = 128;
   static constexpr int kT = 64;                        // tokens per tile
-  static constexpr int kM = 128;                       // rows of every MMA (padded)
+  static constexpr int kM = 128;                       // rows of the P.V product (padded)
+  static constexpr int kQRows = QROWS;                 // rows of the Q K^T product (padded)
   static constexpr int kStages = STAGES;
   static constexpr int kQBufs = QBUFS;
   static constexpr int kHalf = kT * 128;               // one 64-column half of a K or V tile
   static constexpr int kTileBytes = 2 * kHalf;         // 16 KB
   static constexpr int kStageBytes = 2 * kTileBytes;   // K + V
-  static constexpr int kQOff = kStages * kStageBytes;  // Q: two halves of kM rows x 128 B per buffer
-  static constexpr int kQHalf = kM * 128;
+  static constexpr int kQOff = kStages * kStageBytes;  // Q: two halves of QROWS rows x 128 B per buffer
+  static constexpr int kQHalf = kQRows * 128;
   static constexpr int kQBytes = 2 * kQHalf;
   static constexpr int kBarOff = kQOff + kQBufs * kQBytes;
   static constexpr int kSP = 3;                        // S/P buffers in tensor memory
@@ -87,8 +88,12 @@ struct TcLayout {
   static_assert(kSP * kT <= static_cast<int>(kOCol) && kOCol + 2 * kD <= kTmemCols, "tensor-memory columns");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
-using TcTile = TcLayout<5, 1>;     // one piece per block
-using TcBalTile = TcLayout<4, 2>;  // equal-work ranges: pieces follow each other
+// One piece per block (up to 128 rows), and its SPREAD form (up to 64 rows,
+// whose smaller Q leaves room for a sixth ring stage).
+using TcTile = TcLayout<5, 1, 128>;
+using TcTileSpread = TcLayout<6, 1, 64>;
+template <bool SPREAD>
+using TcItemTile = typename std::conditional<SPREAD, TcTileSpread, TcTile>::type;
 
 struct TcBars {
   uint32_t full0, empty0, s_full0, p_full0, pv_done0, drain0, q_full0, q_empty0, o_free;
@@ -132,12 +137,14 @@ __device__ __forceinline__ void tc_init_bars(const TcBars &b, volatile int *tile
   mbar_init(b.o_free, TT::kSoftmaxWarps);
 }
 
-// Row of the slice held by Q slot r, or -1 for a padding slot.  SPREAD: the
-// rows sit in the first ceil(nh / 4) lanes of each 32-lane quarter.
+// Row of the slice held by Q slot (row of the Q K^T product) r, or -1 for a
+// padding slot.  SPREAD (64 slots, M = 64): slot r lands in lane r % 16 of
+// quarter r / 16, which holds rows qd * rpq .. in its first rpq = ceil(nh / 4)
+// lanes.
 template <bool SPREAD>
 __device__ __forceinline__ int tc_slot_row(int r, int nh) {
   if (SPREAD) {
-    const int rpq = (nh + 3) / 4, li = r % 32, rho = (r / 32) * rpq + li;
+    const int rpq = (nh + 3) / 4, li = r % 16, rho = (r / 16) * rpq + li;
     return (li < rpq && rho < nh) ? rho : -1;
   }
   return r < nh ? r : -1;
@@ -148,30 +155,6 @@ __device__ __forceinline__ int tc_slot_row(int r, int nh) {
 template <class TT>
 __device__ __forceinline__ int tc_q_offset(int r, int c) {
   return (c >> 3) * TT::kQHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-}
-
-// The producer warp fills one Q buffer with the piece's rows (padding slots
-// zero): 128 slots x 16 chunks, two slots per round of the 32 lanes, 16 loads
-// in flight per lane; then makes the writes visible to the tensor core.
-template <class TT, bool SPREAD>
-__device__ __forceinline__ void tc_fill_q_warp(const DecodeParams &p, const Piece &pc, uint8_t *qbuf, int lane) {
-  constexpr int D = TT::kD;
-  for (int base = 0; base < TT::kM * 16; base += 32 * 16) {
-    uint4 v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int idx = base + i * 32 + lane, r = idx >> 4, c = idx & 15;
-      const int rho = tc_slot_row<SPREAD>(r, pc.nh);
-      v[i] = rho >= 0 ? __ldg(reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + rho) * D) + c)
-                      : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int idx = base + i * 32 + lane, r = idx >> 4, c = idx & 15;
-      *reinterpret_cast<uint4 *>(qbuf + tc_q_offset<TT>(r, c)) = v[i];
-    }
-  }
-  fence_proxy_async_smem();
 }
 
 // TMA producer for one piece: K and V tiles of 64 tokens into the stage ring
@@ -681,7 +664,7 @@ __device__ __forceinline__ bool tc_issue_qk(uint32_t sbase, uint32_t qbuf, uint3
   constexpr int D = TT::kD;
   constexpr int ST = TT::kStages;
   constexpr int SP = TT::kSP;
-  constexpr uint32_t kIdescQK = tc_idesc_bf16(128, 64, false);
+  constexpr uint32_t kIdescQK = tc_idesc_bf16(TT::kQRows, 64, false);
   // Q's descriptors are the same for every tile; a K-step adds to the
   // start-address field (addresses stay below 256 KB: no carry)
   uint64_t qd[D / 16];
@@ -766,7 +749,7 @@ template <bool PAGED, bool SPREAD>
 __global__ void __launch_bounds__(TcTile::kThreads, 1)
     gqa_verify_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const DecodeParams p) {
-  using TT = TcTile;
+  using TT = TcItemTile<SPREAD>;
   constexpr int D = TT::kD;
   constexpr int T = TT::kT;
   const float kNegInf = -__int_as_float(0x7f800000);
@@ -789,7 +772,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   constexpr int kProducerWarp = TT::kSoftmaxWarps;  // then the Q K^T issuer (allocates), the P.V issuer
   constexpr int kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
   if (threadIdx.x == 0) {
-    tc_init_bars<TT>(bars, tile_bad, 128);  // one arrival per Q row
+    tc_init_bars<TT>(bars, tile_bad, TT::kQRows);  // one arrival per Q slot
     *abort_flag = 0;
     *merge_here = 0;
     *stop = 0;
@@ -830,10 +813,10 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   // a unit with several splits: claim its arrival word for this call
   if (threadIdx.x == 0 && p.unit_ctr != nullptr && (pc.len + p.split_tokens - 1) / p.split_tokens > 1)
     unit_claim(p.unit_ctr + (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j, p.epoch);
-  if (threadIdx.x < 128) {
+  if (threadIdx.x < TT::kQRows) {
     // the q row of this thread's slot into Q (padding slots are zero), while
     // the producer already streams K and V; the Q K^T issuer waits for all
-    // 128 slots
+    // the slots
     const int r = threadIdx.x;
     const int rho = tc_slot_row<SPREAD>(r, pc.nh);
     const uint4 *src = rho >= 0 ? reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + rho) * D)
@@ -879,162 +862,6 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
 
   // ---- teardown: every tensor-memory access is done before the columns go
   // back (the two issuers waited above for their last products to finish)
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tc_dealloc(tmem, TT::kTmemCols);
-  }
-}
-
-// Equal-work ranges on the tcgen05 tensor cores: one persistent block per SM
-// walks its range [c W / N, (c + 1) W / N) of the W tiles of all (sequence,
-// group) units (the Walker of the mma.sync kernel's balanced mode; every role
-// walks the same pieces).  Per piece n: the producer warp fills Q buffer n % 2
-// (once the Q K^T products of piece n - 2 are done with it) and streams the
-// piece's tiles into the ring, which runs on across pieces; the Q K^T issuer
-// takes Q buffer n % 2; the P.V issuer starts the piece's accumulators once
-// the softmax warps have read piece n - 1's O out (o_free); the softmax warps
-// write whole units' rows final and the (at most two) units shared with a
-// neighbouring block as partial states in the block's two slots, with the
-// records the balanced combine kernel merges them from.
-template <bool PAGED, bool SPREAD>
-__global__ void __launch_bounds__(TcBalTile::kThreads, 1)
-    gqa_verify_tc_balanced_kernel(const __grid_constant__ CUtensorMap tm_k,
-                                  const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  using TT = TcBalTile;
-  constexpr int T = TT::kT;
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t sbase = smem_addr(smem);
-  const TcBars bars = tc_bars<TT>(sbase);
-  volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + TT::kMiscOff);
-  volatile int *tile_bad = reinterpret_cast<volatile int *>(smem + TT::kMiscOff + 4);  // [ST]
-  volatile int *abort_flag = tile_bad + TT::kStages;
-  volatile int *merge_here = tile_bad + TT::kStages + 1;  // (no in-kernel merge in this mode)
-  volatile int *stop = tile_bad + TT::kStages + 2;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  constexpr int kProducerWarp = TT::kSoftmaxWarps;
-  constexpr int kMmaWarp = TT::kSoftmaxWarps + 1, kPvWarp = TT::kSoftmaxWarps + 2;
-
-  if (threadIdx.x == 0) {
-    tc_init_bars<TT>(bars, tile_bad, 1);  // the producer warp arrives once per Q buffer fill
-    *abort_flag = 0;
-    *merge_here = 0;
-    *stop = 0;
-    fence_mbarrier_init();
-  }
-  if (warp == kMmaWarp) {
-    tc_alloc(smem_addr(const_cast<uint32_t *>(tmem_slot)), TT::kTmemCols);
-    tc_relinquish();
-  }
-  if (warp == kProducerWarp && lane == 0) {
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  pdl_wait_primary();
-  if (threadIdx.x == 0) pdl_launch_dependents();
-  Walker wk;
-  Piece pc;
-  walker_init<T>(wk, p, lane);  // every lane of every warp: the same pieces
-  bool have = walker_next<T>(wk, p, pc);
-
-  if (warp == kProducerWarp) {
-    // ============================================================ producer
-    int tile = 0;
-    for (int n = 0; have; ++n) {
-      const int qb = n % 2;
-      if (n >= 2) {
-        bool ok = lane == 0 ? mbar_wait(bars.q_empty0 + 8 * qb, ((n / 2) - 1) & 1) : true;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok || *abort_flag) {
-          if (lane == 0) tc_abort(p, abort_flag);
-          break;
-        }
-      }
-      tc_fill_q_warp<TT, SPREAD>(p, pc, smem + TT::kQOff + qb * TT::kQBytes, lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars.q_full0 + 8 * qb);
-      if (!tc_produce_piece<TT, PAGED>(&tm_k, &tm_v, p, pc, sbase, bars, tile_bad, abort_flag, lane, tile)) break;
-      have = walker_next<T>(wk, p, pc);
-    }
-    tc_produce_drain<TT>(bars, tile, lane);
-  } else if (warp == kMmaWarp) {
-    // ============================================================ Q K^T issuer
-    if (lane == 0) {
-      int gt = 0;
-      for (int n = 0; have; ++n) {
-        const int qb = n % 2;
-        const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
-        bool ok = mbar_wait(bars.q_full0 + 8 * qb, (n / 2) & 1) && !*abort_flag;
-        ok = ok && tc_issue_qk<TT>(sbase, sbase + TT::kQOff + qb * TT::kQBytes, tmem, bars, gt, n_tiles);
-        if (!ok) {
-          tc_abort(p, abort_flag);
-          break;
-        }
-        tc_commit(bars.q_empty0 + 8 * qb);  // Q buffer qb is free once these products are done
-        gt += n_tiles;
-        have = walker_next<T>(wk, p, pc);
-      }
-      tc_issuer_drain(bars.drain0, p);
-    }
-  } else if (warp == kPvWarp) {
-    // ============================================================ P.V issuer
-    if (lane == 0) {
-      int gt = 0;
-      for (int n = 0; have; ++n) {
-        const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
-        // the piece's products start O afresh: the previous piece's O must be read out
-        bool ok = (n == 0 || mbar_wait(bars.o_free, (n - 1) & 1)) && !*abort_flag;
-        if (ok) tc_fence_after();
-        ok = ok && tc_issue_pv<TT, SPREAD>(sbase, tmem, bars, gt, n_tiles);
-        if (!ok) {
-          tc_abort(p, abort_flag);
-          break;
-        }
-        gt += n_tiles;
-        have = walker_next<T>(wk, p, pc);
-      }
-      tc_issuer_drain(bars.drain0 + 8, p);
-    }
-  } else {
-    // ============================================================ softmax rows
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-      p.ws_header[0] = static_cast<int>(gridDim.x);
-      p.ws_header[1] = p.capacity;
-      p.ws_header[2] = static_cast<int>(wk.W & 0xffffffff);
-      p.ws_header[3] = static_cast<int>(wk.W >> 32);
-    }
-    int gt = 0;
-    while (have) {
-      const int n_tiles = (pc.t_end - pc.t_begin + T - 1) / T;
-      if (threadIdx.x == 0 && pc.first_of_unit)
-        p.ws_meta[(static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j] =
-            make_int4(static_cast<int>(blockIdx.x), pc.last_block, pc.slot & 1, 0);
-      const TcDest dest{pc.final_row, pc.slot};
-      const bool go = SPREAD ? tc_softmax_spread<TT, PAGED>(p, pc, smem, tmem, bars, tile_bad, abort_flag,
-                                                           merge_here, stop, gt, n_tiles, dest, warp, lane)
-                             : tc_softmax_wide<TT, PAGED>(p, pc, smem, tmem, bars, tile_bad, abort_flag, merge_here,
-                                                         stop, gt, n_tiles, dest, warp, lane);
-      // O has been read out: the next piece's P.V products may overwrite it
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars.o_free);
-      if (!go) break;
-      gt += n_tiles;
-      have = walker_next<T>(wk, p, pc);
-    }
-  }
-
-  // ---- teardown: every tensor-memory access is done before the columns go back
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

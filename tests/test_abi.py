@@ -163,13 +163,10 @@ def test_plan_split_tokens(lib):
     d1 = _dims(batch=1, num_heads=32, num_kv_heads=4, head_dim=128, page_size=131072)
     t1 = gqa.gqa_plan_split_tokens(d1, 131072, 148)
     assert t1 == 1792 and 4 * -(-131072 // t1) == 296
-    # MQA sweep (r = 32: the tcgen05 kernel): equal-work ranges over persistent blocks
+    # MQA sweep (r = 32 runs the tcgen05 kernel, one block per SM): 16 units -> 9 splits -> 144 items
     d2 = _dims(batch=16, num_heads=32, num_kv_heads=1, head_dim=128, page_size=8192)
-    assert gqa.gqa_plan_split_tokens(d2, 8192, 148) == 0
-    # forced mma.sync contraction for the same shape: fixed splits, 16-row slices
-    d2m = _dims(batch=16, num_heads=32, num_kv_heads=1, head_dim=128, page_size=8192, flags=gqa.FLAG_CONTRACT_MMA)
-    t2 = gqa.gqa_plan_split_tokens(d2m, 8192, 148)
-    assert t2 > 0 and 32 * -(-8192 // t2) <= 296
+    t2 = gqa.gqa_plan_split_tokens(d2, 8192, 148)
+    assert 16 * -(-8192 // t2) <= 148 and t2 == 1024
     # paged: equal-work ranges, or splits of 4096 above 1024 sequences
     d3 = _dims(batch=64, num_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=70000,
                max_pages_per_seq=2048)
@@ -308,8 +305,8 @@ def test_plan_decomposition(lib):
     assert plan(num_kv_heads=2, **sweep) == (gqa.PLAN_CLUSTERS, 0, 8)     # 32 units x 8 = 256 blocks
     assert plan(num_kv_heads=4, **sweep) == (gqa.PLAN_CLUSTERS, 0, 4)     # 64 units x 4
     assert plan(num_kv_heads=8, **sweep) == (gqa.PLAN_CLUSTERS, 0, 2)     # 128 units x 2
-    # r = 32: the tcgen05 kernel, equal-work ranges
-    assert plan(num_kv_heads=1, **sweep) == (gqa.PLAN_EQUAL_WORK, 0, 1)
+    # r = 32: the tcgen05 kernel, fixed splits
+    assert plan(num_kv_heads=1, **sweep) == (gqa.PLAN_FIXED_SPLITS, 1024, 1)
     # MHA: 512 units fill the GPU one block each
     assert plan(num_kv_heads=32, **sweep) == (gqa.PLAN_FIXED_SPLITS, 8192, 1)
     # Llama-2-70B layer: one split per unit; long context, 4 units: clusters would be too few
