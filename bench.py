@@ -563,6 +563,16 @@ def main_gpu(args):
         case.step()
     case.check_status()
 
+    if args.profile_only:
+        # for a profiler: the warm-up above and K plain steps, nothing else
+        for _ in range(args.steps):
+            case.step()
+        case.check_status()
+        if rank == 0:
+            print(json.dumps({"profile_only": True, "workload": w.name, "steps": args.steps,
+                              "warmup": args.warmup, "plan": case.plan()}), flush=True)
+        return 0
+
     # ---- timed region: K steps, inputs resident in HBM
     clocks = ClockSampler(local)
     with clocks:
@@ -719,6 +729,8 @@ def main(argv=None):
                          "> 0: fixed splits of that many tokens")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="measure the headline workload only")
+    ap.add_argument("--profile-only", action="store_true",
+                    help="run the warm-up and --steps plain steps of the workload and exit (for ncu); no timing")
     ap.add_argument("--clock-window", type=float, default=1.0,
                     help="seconds of repeated steps sampled for clocks after the timed region (>= 1)")
     ap.add_argument("--oracle-seconds", type=float, default=0.0,

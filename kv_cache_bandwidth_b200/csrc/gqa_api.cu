@@ -430,6 +430,7 @@ DecodeParams base_params(const Shape &sh, const void *q, const int32_t *seqlens,
   p.max_pages = sh.max_pages;
   p.capacity = static_cast<int>(sh.capacity);
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.ups = sh.G * sh.hs;
   return p;
 }
 
@@ -443,8 +444,9 @@ struct RowExtras {
   const int32_t *group_of_head = nullptr;  // host table of each head's KV group, or null
 };
 
-// The device form of a group table: heads sorted by group (stable), offsets.
-void fill_group_map(const int32_t *group_of_head, int H, int G, gqa::GroupMap *m) {
+// The device form of a group table: heads sorted by group (stable), offsets,
+// and the (group, slice of rc rows) units that hold rows.
+void fill_group_map(const int32_t *group_of_head, int H, int G, int rc, gqa::GroupMap *m) {
   int count[gqa::kMaxMapGroups + 1] = {};
   for (int i = 0; i < H; ++i) ++count[group_of_head[i] + 1];
   m->off[0] = 0;
@@ -454,6 +456,14 @@ void fill_group_map(const int32_t *group_of_head, int H, int G, gqa::GroupMap *m
     const int g = group_of_head[i];
     m->heads[m->off[g] + fill[g]++] = static_cast<uint8_t>(i);
   }
+  int n = 0;
+  for (int g = 0; g < G; ++g)
+    for (int j = 0; j * rc < count[g + 1]; ++j) {  // at most H slices in all: each holds a row
+      m->slice_g[n] = static_cast<uint8_t>(g);
+      m->slice_j[n] = static_cast<uint8_t>(j);
+      ++n;
+    }
+  m->n_slices = static_cast<uint16_t>(n);
 }
 
 // The items kernel: one block per (sequence, group, split) item.
@@ -478,7 +488,7 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   p.empty_ok = ex.empty_ok ? 1 : 0;
   if (ex.group_of_head) {
     p.mapped = 1;
-    fill_group_map(ex.group_of_head, sh.H, sh.G, &p.map);
+    fill_group_map(ex.group_of_head, sh.H, sh.G, sh.rc, &p.map);
   }
   const long long items = units_of(sh) * num_splits;
   if (items > (1ll << 31) - 1) return GQA_ERR_DIMS;
@@ -540,6 +550,11 @@ int run_balanced_decode(const Shape &sh, int sms, const void *q, const void *k, 
   p.b = sh.b;
   p.lse = ex.lse;
   p.empty_ok = ex.empty_ok ? 1 : 0;
+  if (ex.group_of_head) {
+    p.mapped = 1;
+    fill_group_map(ex.group_of_head, sh.H, sh.G, sh.rc, &p.map);
+    p.ups = p.map.n_slices;
+  }
   Launch l{dim3(static_cast<unsigned>(sms), 1, 1), 1, stream};
   rc = launch_decode<Mode::kBalanced>(sh, tk, tv, p, l);
   return rc < 0 ? rc : GQA_OK;
@@ -568,9 +583,16 @@ int run_balanced_combine(const Shape &sh, const int32_t *seqlens, float *out, ui
   c.rq = sh.rq;
   c.lse = ex.lse;
   c.empty_ok = ex.empty_ok ? 1 : 0;
+  c.ups = sh.G * sh.hs;
+  if (ex.group_of_head) {
+    c.mapped = 1;
+    fill_group_map(ex.group_of_head, sh.H, sh.G, sh.rc, &c.map);
+    c.ups = c.map.n_slices;
+  }
   cudaLaunchConfig_t cfg = {};
   const int rows_per_block = 128 / (sh.D / 4);  // the combine's rows per block
-  cfg.gridDim = dim3(static_cast<unsigned>(units_of(sh) * ((sh.rc + rows_per_block - 1) / rows_per_block)), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(static_cast<long long>(sh.b) * c.ups *
+                                           ((sh.rc + rows_per_block - 1) / rows_per_block)), 1, 1);
   cfg.blockDim = dim3(128, 1, 1);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -598,9 +620,9 @@ struct AutoChoice {
 
 bool dims_paged(const gqa_dims *dims) { return dims->max_pages_per_seq > 0; }
 
-// Equal-work ranges serve paged dims, with neither a group table nor the
-// tcgen05 kernel (both run on fixed splits only).
-bool balanced_ok(const gqa_dims *dims, const Shape &sh) { return dims_paged(dims) && !sh.mapped && !sh.tc; }
+// Equal-work ranges serve paged dims (with or without a group table), not the
+// tcgen05 kernel (fixed splits only).
+bool balanced_ok(const gqa_dims *dims, const Shape &sh) { return dims_paged(dims) && !sh.tc; }
 
 int round_split(long long tokens) {
   tokens = (tokens + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;

@@ -78,6 +78,11 @@ constexpr int kMaxMapGroups = 256;
 struct GroupMap {
   uint8_t heads[kMaxMapHeads];
   uint16_t off[kMaxMapGroups + 1];
+  // the (group, row slice) units that hold rows, in (group, slice) order:
+  // equal-work ranges walk only these (a slice past a small group has none)
+  uint8_t slice_g[kMaxMapHeads];
+  uint8_t slice_j[kMaxMapHeads];
+  uint16_t n_slices;
 };
 
 struct DecodeParams {
@@ -106,7 +111,8 @@ struct DecodeParams {
   int num_splits;             // items mode: S
   int b;                      // sequences
   float scale_log2;           // scale * log2(e)
-  int mapped;                 // the group of each head comes from `map` (items mode, one query token)
+  int mapped;                 // the group of each head comes from `map` (one query token)
+  int ups;                    // balanced mode: units per sequence (G x hs, or the map's slices)
   GroupMap map;
 };
 
@@ -124,6 +130,9 @@ struct CombineParams {
   const int4 *ws_meta;        // balanced mode: per unit {first block, last block, slot in first block}
   float *lse;                 // [b, H] or null, as in DecodeParams
   int empty_ok;
+  int ups;                    // balanced mode: units per sequence
+  int mapped;                 // balanced mode: rows resolve through `map`
+  GroupMap map;
 };
 
 // Row of q / out ([b, nq, H] flattened) for row rho = t * r + h (query token t,
@@ -143,6 +152,18 @@ __device__ __forceinline__ size_t row_of(const DecodeParams &p, int s, int g, in
 // Rows of KV group g: nq * r, or the group's own size under a map.
 __device__ __forceinline__ int group_rows(const DecodeParams &p, int g) {
   return p.mapped ? static_cast<int>(p.map.off[g + 1]) - static_cast<int>(p.map.off[g]) : p.rq;
+}
+
+// Group and row slice of unit u of a sequence (balanced mode): u = g hs + j,
+// or the map's u-th slice that holds rows.
+__device__ __forceinline__ void unit_gj(bool mapped, const GroupMap &map, int hs, int u, int *g, int *j) {
+  if (mapped) {
+    *g = map.slice_g[u];
+    *j = map.slice_j[u];
+  } else {
+    *g = u / hs;
+    *j = u % hs;
+  }
 }
 
 // Natural-log sum of exp over a row from its base-2 state: the row's
@@ -216,7 +237,7 @@ __device__ __forceinline__ uint32_t keep_halves(uint32_t v, bool keep_lo, bool k
 // One piece of work: the token range [t_begin, t_end) of KV group g of
 // sequence s, and where its result goes.
 struct Piece {
-  int s, g, len, k, t_begin, t_end;
+  int s, g, u, len, k, t_begin, t_end;  // u: balanced mode, the unit's index within its sequence
   int j, h0, nh;       // head slice j of the group: heads h0 .. h0 + nh - 1
   bool len_ok;
   bool final_row;      // balanced mode: the piece is the whole unit
@@ -300,18 +321,18 @@ struct Walker {
   long long remaining;  // tiles of the range not handed out yet
   long long pos;        // global index of the next tile handed out
   long long W;          // tiles of all units
-  int s, g, j, tile_in, tiles_s, len_s, count;
+  int s, u, g, j, tile_in, tiles_s, len_s, count;  // u: unit within the sequence, (g, j) its group and slice
 };
 
 template <int T>
 __device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, int lane) {
-  const long long W = total_tiles<T>(p.seqlens, p.b, p.G * p.hs, p.capacity, p.nq, lane);
+  const long long W = total_tiles<T>(p.seqlens, p.b, p.ups, p.capacity, p.nq, lane);
   const long long N = gridDim.x, c = blockIdx.x;
   const long long start = c * W / N;
   wk.remaining = (c + 1) * W / N - start;
   wk.pos = start;
   wk.W = W;
-  wk.s = wk.g = wk.j = wk.tile_in = wk.tiles_s = wk.len_s = wk.count = 0;
+  wk.s = wk.u = wk.g = wk.j = wk.tile_in = wk.tiles_s = wk.len_s = wk.count = 0;
   if (wk.remaining <= 0) {
     wk.remaining = 0;
     return;
@@ -321,7 +342,7 @@ __device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, i
     const int s = base + lane;
     int len = 0;
     const long long t =
-        (s < p.b) ? static_cast<long long>(unit_tiles<T>(p.seqlens, p.capacity, p.nq, s, &len)) * p.G * p.hs : 0;
+        (s < p.b) ? static_cast<long long>(unit_tiles<T>(p.seqlens, p.capacity, p.nq, s, &len)) * p.ups : 0;
     long long inc = t;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -337,9 +358,8 @@ __device__ __forceinline__ void walker_init(Walker &wk, const DecodeParams &p, i
       wk.len_s = __shfl_sync(0xffffffffu, len, L);
       wk.tiles_s = (wk.len_s + T - 1) / T;
       const long long in_seq = start - before;
-      const int unit_in_seq = static_cast<int>(in_seq / wk.tiles_s);
-      wk.g = unit_in_seq / p.hs;
-      wk.j = unit_in_seq % p.hs;
+      wk.u = static_cast<int>(in_seq / wk.tiles_s);
+      unit_gj(p.mapped, p.map, p.hs, wk.u, &wk.g, &wk.j);
       wk.tile_in = static_cast<int>(in_seq % wk.tiles_s);
       return;
     }
@@ -353,10 +373,11 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
   if (wk.remaining <= 0) return false;
   const int take = static_cast<int>(min(static_cast<long long>(wk.tiles_s - wk.tile_in), wk.remaining));
   pc.s = wk.s;
+  pc.u = wk.u;
   pc.g = wk.g;
   pc.j = wk.j;
   pc.h0 = wk.j * p.rc;
-  pc.nh = min(p.rc, p.rq - pc.h0);
+  pc.nh = min(p.rc, group_rows(p, wk.g) - pc.h0);
   pc.k = 0;
   pc.len = wk.len_s;
   pc.len_ok = true;
@@ -376,15 +397,13 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
   wk.tile_in = 0;
   if (wk.remaining > 0) {
     do {
-      if (++wk.j == p.hs) {
-        wk.j = 0;
-        if (++wk.g == p.G) {
-          wk.g = 0;
-          ++wk.s;
-          wk.tiles_s = unit_tiles<T>(p.seqlens, p.capacity, p.nq, wk.s, &wk.len_s);
-        }
+      if (++wk.u == p.ups) {
+        wk.u = 0;
+        ++wk.s;
+        wk.tiles_s = unit_tiles<T>(p.seqlens, p.capacity, p.nq, wk.s, &wk.len_s);
       }
     } while (wk.tiles_s == 0);
+    unit_gj(p.mapped, p.map, p.hs, wk.u, &wk.g, &wk.j);
   }
   return true;
 }
@@ -1349,7 +1368,7 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       // ---- results of the piece
       if (BAL && ctid == 0) {
         if (pc.first_of_unit)
-          p.ws_meta[(static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j] =
+          p.ws_meta[static_cast<size_t>(pc.s) * p.ups + pc.u] =
               make_int4(static_cast<int>(blockIdx.x), pc.last_block, pc.slot & 1, 0);
       }
       constexpr bool kWarpRows = FMA == 0 && !BAL;  // the rows are still per warp (ow)
@@ -1586,12 +1605,21 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
   const int rblocks = (p.rc + kRPB - 1) / kRPB;
   const int u = blockIdx.x / rblocks;  // unit: (sequence, group, head slice)
   const int h0 = (blockIdx.x % rblocks) * kRPB;
-  const int j = u % p.hs;
-  const int s = u / (p.G * p.hs), g = (u / p.hs) % p.G;
+  const int s = u / p.ups;
+  int g, j;
+  unit_gj(p.mapped, p.map, p.hs, u % p.ups, &g, &j);
+  // rows of the slice (the last slice of a group is narrower; a group table
+  // gives each group its own size)
+  const int slice_rows =
+      min(p.rc, (p.mapped ? static_cast<int>(p.map.off[g + 1]) - static_cast<int>(p.map.off[g]) : p.rq) - j * p.rc);
+  auto row_at = [&](int hh) -> size_t {
+    return p.mapped ? static_cast<size_t>(s) * p.H + p.map.heads[p.map.off[g] + j * p.rc + hh]
+                    : out_row(s, g, j * p.rc + hh, p.nq, p.r, p.H);
+  };
   const int c4 = threadIdx.x % kTPR;
   const int h = h0 + threadIdx.x / kTPR;
-  const bool row_ok = h < p.rc && j * p.rc + h < p.rq;  // (the last slice of a group is narrower)
-  const size_t row = row_ok ? out_row(s, g, j * p.rc + h, p.nq, p.r, p.H) : 0;
+  const bool row_ok = h < slice_rows;
+  const size_t row = row_ok ? row_at(h) : 0;
   float4 *dst = reinterpret_cast<float4 *>(p.out + row * D);
   const int len = __ldg(p.seqlens + s);
   pdl_wait_primary();  // the header, unit records and partial states come from the decode kernel
@@ -1622,8 +1650,8 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
     return;
   }
   __shared__ MergeScratch<D> sc;
-  for (int hh = h0; hh < h0 + kRPB && hh < p.rc && j * p.rc + hh < p.rq; ++hh) {  // (uniform in the block)
-    const size_t row2 = out_row(s, g, j * p.rc + hh, p.nq, p.r, p.H);
+  for (int hh = h0; hh < h0 + kRPB && hh < slice_rows; ++hh) {  // (uniform in the block)
+    const size_t row2 = row_at(hh);
     merge_row<D>(p.part_o, p.part_m, p.part_l, nc,
                  [&](int k) -> long long {
                    const long long c = c_lo + k;

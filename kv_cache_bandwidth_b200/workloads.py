@@ -83,6 +83,10 @@ WORKLOADS: Dict[str, Workload] = {
     "ragged": Workload(name="ragged paged decode b64 H32 G8 d128 len U[128,32768] P16",
                        b=64, H=32, G=8, d=128, m=32768, page_size=16, len_lo=128,
                        len_hi=32768, seed=1236),
+    # the ragged recipe on 8 sequences: the ragged decode kernel at a size a
+    # full profiler capture (tens of replays) handles
+    "ragged_b8": Workload(name="ragged paged decode b8 H32 G8 d128 len U[128,32768] P16 (profiling size)",
+                          b=8, H=32, G=8, d=128, m=32768, page_size=16, len_lo=128, len_hi=32768, seed=1236),
     "long1": Workload(name="long-context split-KV decode b1 H32 G4 d128 m131072 peaky",
                       b=1, H=32, G=4, d=128, m=131072, peaky_frac=0.01, split_tokens=4096,
                       seed=1237),

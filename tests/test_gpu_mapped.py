@@ -55,16 +55,45 @@ def test_mapped_against_oracle(H, G, big, d, layout, split):
     assert_lse(lse, ref_lse, "map H=%d G=%d" % (H, G))
 
 
-def test_uniform_map_equals_decode_split():
-    w = Workload(name="u", b=4, H=32, G=4, d=128, m=2000, seed=5)
+@pytest.mark.parametrize("P", [None, 16])
+def test_uniform_map_equals_decode_split(P):
+    """The table i -> i / r gives the same pieces and arithmetic as no table:
+    equal bit for bit on fixed splits and (paged, split_tokens = 0) on
+    equal-work ranges."""
+    w = Workload(name="u", b=4, H=32, G=4, d=128, m=2000, page_size=P, len_lo=1 if P else None,
+                 len_hi=2000 if P else None, seed=5)
     inp = make_inputs(w, device="cuda", lens=[2000, 1000, 17, 1500])
     gmap = [i // 8 for i in range(32)]
     for split in (0, 128, 512):
-        a = gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, None, split_tokens=split)
-        b = gqa.gqa_decode_split_mapped(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, None, group_of_head=gmap,
-                                        split_tokens=split)
+        a = gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, split_tokens=split)
+        b = gqa.gqa_decode_split_mapped(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                                        group_of_head=gmap, split_tokens=split)
         torch.cuda.synchronize()
         assert torch.equal(a, b), "split %d" % split
+
+
+def test_mapped_equal_work_ranges_many_slices():
+    """A paged batch with a table whose groups need 1, 2 and 3 slices of 16
+    rows and one empty group, on equal-work ranges (split_tokens = 0, the
+    mma.sync contraction: 16-row slices): every slice that holds rows is
+    walked once, none that holds none."""
+    H, G = 48, 4
+    gmap = [0] * 40 + [1] * 1 + [3] * 7  # group 2 empty; group 0 needs three slices, group 3 one
+    random.Random(9).shuffle(gmap)
+    lens = [5000, 64, 1, 2047, 4096, 333, 16, 3000]
+    w = Workload(name="slices", b=len(lens), H=H, G=G, d=128, m=5000, page_size=16, len_lo=1, len_hi=5000, seed=11)
+    inp = make_inputs(w, device="cuda", lens=lens)
+    ref, ref_lse, st_ref = oracle.gqa_decode_mapped(inp.q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu(),
+                                                    inp.seqlens.cpu(), inp.page_table.cpu(), group_of_head=gmap)
+    assert st_ref == 0
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = gqa.gqa_decode_split_mapped(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                                           group_of_head=gmap, split_tokens=0, want_lse=True, status=st,
+                                           flags=gqa.FLAG_CONTRACT_MMA)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_parity(out, ref, "equal-work ranges with a group table")
+    assert_lse(lse, ref_lse, "equal-work ranges with a group table")
 
 
 def test_mapped_argument_checks():
