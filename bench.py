@@ -578,16 +578,6 @@ def main_gpu(args):
     with clocks:
         ms_per_step = case.time_steps(args.steps, world)
     timed_samples = len(clocks.samples)
-    # ---- the same step repeated for >= 1 s, so that the clock record has
-    # samples even when the timed region is a few milliseconds
-    with clocks:
-        t_end = time.perf_counter() + max(1.0, args.clock_window)
-        n_win = 0
-        while time.perf_counter() < t_end:
-            for _ in range(32):
-                case.step()
-            n_win += 32
-            torch.cuda.synchronize()
     case.check_status()
     value = world * case.kv_step / (ms_per_step * 1e-3) / 1e9
 
@@ -612,10 +602,6 @@ def main_gpu(args):
                                              q_verify=None if nq == 1 else case.q)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": desc + "; %.1f s of CPU time" % dt}
-    case.free()
-    del case
-    torch.cuda.empty_cache()
-
     # ---- every workload, measured the same way in this process
     per_config = {}
     if not args.no_per_config:
@@ -623,6 +609,22 @@ def main_gpu(args):
             per_config[name] = measure_point(args, name, 1, world, rank, hbm)
         for name, n in PER_CONFIG_VERIFY:
             per_config[traffic_key(name, n)] = measure_point(args, name, n, world, rank, hbm)
+
+    # ---- last: the headline step repeated for >= 1 s, so that the clock
+    # record has samples even when the timed region is a few milliseconds (at
+    # the end, so that the heat it leaves behind touches no other measurement)
+    with clocks:
+        t_end = time.perf_counter() + max(1.0, args.clock_window)
+        n_win = 0
+        while time.perf_counter() < t_end:
+            for _ in range(32):
+                case.step()
+            n_win += 32
+            torch.cuda.synchronize()
+    case.check_status()
+    case.free()
+    del case
+    torch.cuda.empty_cache()
 
     if rank == 0:
         clk = clocks.summary()
