@@ -466,6 +466,19 @@ void fill_group_map(const int32_t *group_of_head, int H, int G, int rc, gqa::Gro
   m->n_slices = static_cast<uint16_t>(n);
 }
 
+// L2 a dependent launch may fill ahead of its wait: the first tiles of every
+// block's piece, GQA_PREFETCH_L2_BYTES over the grid (about half of the L2),
+// at most the piece.
+#ifndef GQA_PREFETCH_L2_BYTES
+#define GQA_PREFETCH_L2_BYTES (64ll << 20)
+#endif
+int prefetch_tiles(const Shape &sh, long long blocks, int piece_tokens) {
+  const int T = tile_tokens(sh);
+  const long long tile_bytes = 4ll * T * sh.D;  // K and V, bf16
+  const long long per_block = GQA_PREFETCH_L2_BYTES / std::max<long long>(1, blocks / sh.hs) / tile_bytes;
+  return static_cast<int>(std::min<long long>(per_block, (piece_tokens + T - 1) / T));
+}
+
 // The items kernel: one block per (sequence, group, split) item.
 int run_items(const Shape &sh, const void *q, const void *k, const void *v, const int32_t *seqlens,
               const int32_t *pt, float *out, float scale, uint32_t *status, int split_tokens,
@@ -497,6 +510,7 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   // unit the grid follows a full decode grid, where measured it cost ~3 %
   // (its early blocks only wait, and the grid no longer starts as one wave).
   Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream, num_splits > 1 || ex.force_pdl};
+  if (l.pdl) p.prefetch_tiles = prefetch_tiles(sh, items, split_tokens);
   if (sh.tc) return launch_verify_tc(sh, tk, tv, p, l);
   return launch_decode<Mode::kItems>(sh, tk, tv, p, l);
 }
@@ -771,6 +785,7 @@ int run_cluster(const Shape &sh, int c, const void *q, const void *k, const void
   // launched as a programmatic dependent: the blocks set themselves up while
   // the previous kernel on the stream finishes
   Launch l{dim3(c, sh.G * sh.hs, sh.b), c, st, true};
+  p.prefetch_tiles = prefetch_tiles(sh, units_of(sh) * c, static_cast<int>((sh.capacity + c - 1) / c));
   return launch_decode<Mode::kCluster>(sh, tk, tv, p, l);
 }
 

@@ -113,6 +113,8 @@ struct DecodeParams {
   float scale_log2;           // scale * log2(e)
   int mapped;                 // the group of each head comes from `map` (one query token)
   int ups;                    // balanced mode: units per sequence (G x hs, or the map's slices)
+  int prefetch_tiles;         // items and cluster modes: tiles of the block's piece brought into L2
+                              // before the wait for the previous kernel on the stream (0: none)
   GroupMap map;
 };
 
@@ -285,6 +287,74 @@ __device__ __forceinline__ Piece make_item(const DecodeParams &p) {
     }
   }
   return it;
+}
+
+// Before the wait for the previous kernel on the stream (a programmatic
+// dependent launch lets the block start while that kernel still runs): bring
+// the first p.prefetch_tiles tiles of the block's piece into L2, so that the
+// HBM reads of this step overlap the tail of the previous one (its last
+// blocks' merges).  The length and page ids read here may still be written by
+// that kernel, so they are only a hint: they pick the addresses to prefetch
+// (page ids outside the pool are skipped, coordinates outside the cache are
+// skipped by the tensor map) and nothing else; the piece itself is computed
+// from the values read after the wait.  One slice per unit prefetches (the
+// slices of a unit read the same tiles).  Called by one warp.
+template <int D, int T, Mode MODE, bool PAGED>
+__device__ __forceinline__ void prefetch_piece_l2(const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                                                  const DecodeParams &p, int lane) {
+  if (MODE == Mode::kBalanced || p.prefetch_tiles <= 0) return;
+  int k, g, j, s;
+  if (MODE == Mode::kItems) {
+    const int i = blockIdx.x;
+    k = i % p.num_splits;
+    const int t = i / p.num_splits;
+    j = t % p.hs;
+    const int sg = t / p.hs;
+    g = sg % p.G;
+    s = sg / p.G;
+  } else {
+    k = blockIdx.x;
+    g = blockIdx.y / p.hs;
+    j = blockIdx.y % p.hs;
+    s = blockIdx.z;
+  }
+  if (j != 0 || p.mapped) return;
+  const int len = *reinterpret_cast<const volatile int32_t *>(p.seqlens + s);
+  if (len < p.nq || len > p.capacity) return;
+  int t_begin, t_end;
+  if (MODE == Mode::kItems) {
+    t_begin = k * p.split_tokens;
+    t_end = min(len, t_begin + p.split_tokens);
+  } else {
+    const int tiles = (len + T - 1) / T;
+    const long long c = gridDim.x;
+    t_begin = static_cast<int>((k * static_cast<long long>(tiles)) / c) * T;
+    t_end = min(len, static_cast<int>(((k + 1) * static_cast<long long>(tiles)) / c) * T);
+  }
+  t_end = min(t_end, t_begin + p.prefetch_tiles * T);
+  constexpr int kHalves = D / 64;  // 64-element (128-byte) columns of a row
+  if (!PAGED) {
+    // box i: tile i / (2 kHalves), column (i / 2) % kHalves, K or V
+    const int n = (t_end - t_begin + T - 1) / T * 2 * kHalves;
+    for (int i = lane; i < n; i += 32) {
+      const int t0 = t_begin + (i / (2 * kHalves)) * T, h = (i >> 1) % kHalves;
+      tma_prefetch_l2_4d((i & 1) ? tm_v : tm_k, h * 64, t0, g, s);
+    }
+  } else {
+    // one lane per box of min(P, T) rows: a page, or a T-row window of a large page
+    const int P = p.page_size;
+    const int br = min(P, T);
+    const int32_t *pt_row = p.page_table + static_cast<size_t>(s) * p.max_pages;
+    for (int tb = t_begin + lane * br; tb < t_end; tb += 32 * br) {
+      const int id = *reinterpret_cast<const volatile int32_t *>(pt_row + tb / P);
+      if (id < 0 || id >= p.num_pages) continue;
+#pragma unroll
+      for (int h = 0; h < kHalves; ++h) {
+        tma_prefetch_l2_4d(tm_k, h * 64, tb % P, g, id);
+        tma_prefetch_l2_4d(tm_v, h * 64, tb % P, g, id);
+      }
+    }
+  }
 }
 
 // Tiles of each (sequence, group) unit of sequence s; 0 for an invalid length.
@@ -899,9 +969,12 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
     *item_bad = 0;
     fence_mbarrier_init();
   }
-  if (warp == nc && lane == 0) {
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
+  if (warp == nc) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    prefetch_piece_l2<D, T, MODE, PAGED>(&tm_k, &tm_v, p, lane);
   }
   __syncthreads();
 
@@ -1566,6 +1639,10 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p)
   const int s = row / (p.nq * p.H);
   const int len = __ldg(p.seqlens + s);
   float4 *dst = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D) + threadIdx.x % (D / 4);
+  // the next kernel on the stream (a dependent launch: the next step's decode)
+  // may set itself up and prefetch while this one runs; it waits for this
+  // grid to complete before touching memory
+  if (threadIdx.x == 0) pdl_launch_dependents();
   pdl_wait_primary();  // the partial states below come from the preceding kernel
   float *lse_dst = p.lse ? p.lse + row : nullptr;
   if (len < p.nq || len > p.max_len) {
@@ -1622,6 +1699,7 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
   const size_t row = row_ok ? row_at(h) : 0;
   float4 *dst = reinterpret_cast<float4 *>(p.out + row * D);
   const int len = __ldg(p.seqlens + s);
+  if (threadIdx.x == 0) pdl_launch_dependents();  // as in gqa_combine_kernel
   pdl_wait_primary();  // the header, unit records and partial states come from the decode kernel
   const int N = p.ws_header[0];
   const int capacity = p.ws_header[1];

@@ -782,9 +782,12 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     tc_alloc(smem_addr(const_cast<uint32_t *>(tmem_slot)), TT::kTmemCols);
     tc_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) {
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    prefetch_piece_l2<D, T, Mode::kItems, PAGED>(&tm_k, &tm_v, p, lane);
   }
   tc_fence_before();
   __syncthreads();

@@ -87,6 +87,16 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Bring one box of a 4-D tensor map into L2 (no shared memory, no completion
+// to wait for).  Coordinates outside the tensor are skipped, as a load would
+// fill them.
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
 // Streaming data is read once: mark it evict-first in L2.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t policy;
