@@ -759,8 +759,10 @@ int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t
   c.rq = a.sh.rq;
   const int rows = a.sh.b * a.sh.nq * a.sh.H;
   cudaLaunchConfig_t cfg = {};
+  // many splits: 512 threads, so that every split's row loads in one round
+  const bool wide = a.num_splits > gqa::kSerialMergeMax;
   cfg.gridDim = dim3(rows, 1, 1);
-  cfg.blockDim = dim3(128, 1, 1);
+  cfg.blockDim = dim3(wide ? 512 : 128, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -768,8 +770,13 @@ int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = a.sh.D == 128 ? cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<128>, c)
-                                : cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<64>, c);
+  cudaError_t e;
+  if (wide)
+    e = a.sh.D == 128 ? cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<128, 512>, c)
+                      : cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<64, 512>, c);
+  else
+    e = a.sh.D == 128 ? cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<128, 128>, c)
+                      : cudaLaunchKernelEx(&cfg, gqa::gqa_combine_kernel<64, 128>, c);
   return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 

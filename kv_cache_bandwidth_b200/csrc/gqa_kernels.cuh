@@ -491,25 +491,26 @@ __device__ __forceinline__ bool walker_next(Walker &wk, const DecodeParams &p, P
 // kernel's own merge).  `slot(k)` is the index of contribution k in the m/l
 // arrays (< 0: no contribution).  Any l < 0 (an invalid page) makes the row
 // zero.  The partial states are read through L2 (they may come from other
-// blocks of the same grid).  128 threads (tid 0..127) take part; `sync` is
-// their barrier and `sc` their shared scratch.
-template <int D>
+// blocks of the same grid).  NTH threads (tid 0 .. NTH-1) take part; `sync`
+// is their barrier and `sc` their shared scratch.
+template <int D, int NTH = 128>
 struct MergeScratch {
   static constexpr int kTPR = D / 4;        // threads per row (one float4 each)
-  static constexpr int kNG = 128 / kTPR;    // row groups
+  static constexpr int kNG = NTH / kTPR;    // row groups
+  static constexpr int kNW = NTH / 32;      // warps
   static constexpr int kChunk = 512;        // contributions per round
   float4 acc[kNG][kTPR];
   long long ps[kChunk];
   float w[kChunk], l[kChunk];
-  float wmax[4], L[kNG];
-  int wbad[4];
+  float wmax[kNW], L[kNG];
+  int wbad[kNW];
 };
 
-template <int D, typename SlotFn, typename SyncFn>
+template <int D, int NTH, typename SlotFn, typename SyncFn>
 __device__ __forceinline__ void merge_row(const float *part_o, const float *part_m, const float *part_l,
                                           int n_contrib, SlotFn slot, float4 *dst, float *lse_dst, int tid,
-                                          MergeScratch<D> &sc, SyncFn sync) {
-  using SC = MergeScratch<D>;
+                                          MergeScratch<D, NTH> &sc, SyncFn sync) {
+  using SC = MergeScratch<D, NTH>;
   constexpr int kTPR = SC::kTPR;
   constexpr int kNG = SC::kNG;
   constexpr int kChunk = SC::kChunk;
@@ -525,7 +526,7 @@ __device__ __forceinline__ void merge_row(const float *part_o, const float *part
     const int cnt = min(kChunk, n_contrib - base);
     float mx = kNegInf;
     int bd = 0;
-    for (int i = tid; i < cnt; i += 128) {
+    for (int i = tid; i < cnt; i += NTH) {
       const long long ps = slot(base + i);
       sc.ps[i] = ps;
       float m = kNegInf, l = 0.f;
@@ -546,8 +547,12 @@ __device__ __forceinline__ void merge_row(const float *part_o, const float *part
       sc.wbad[warp] = bd;
     }
     sync();
-    mx = fmaxf(fmaxf(sc.wmax[0], sc.wmax[1]), fmaxf(sc.wmax[2], sc.wmax[3]));
-    bad = sc.wbad[0] | sc.wbad[1] | sc.wbad[2] | sc.wbad[3];
+    bad = 0;
+#pragma unroll
+    for (int w = 0; w < SC::kNW; ++w) {
+      mx = fmaxf(mx, sc.wmax[w]);
+      bad |= sc.wbad[w];
+    }
     if (!bad && mx != kNegInf) {
       const float Mn = fmaxf(M, mx);
       const float rescale = (M == kNegInf) ? 0.f : ex2(M - Mn);
@@ -557,7 +562,7 @@ __device__ __forceinline__ void merge_row(const float *part_o, const float *part
       acc.z *= rescale;
       acc.w *= rescale;
       M = Mn;
-      for (int i = tid; i < cnt; i += 128) sc.w[i] = (sc.ps[i] >= 0) ? ex2(sc.w[i] - Mn) : 0.f;
+      for (int i = tid; i < cnt; i += NTH) sc.w[i] = (sc.ps[i] >= 0) ? ex2(sc.w[i] - Mn) : 0.f;
       sync();
 #pragma unroll 8
       for (int i = grp; i < cnt; i += kNG) {
@@ -728,6 +733,37 @@ __device__ __forceinline__ void merge_serial(const float *part_o, const float *p
                                              float *lse_dst) {
   merge_serial_at<D, NV>(part_o, part_m, part_l, [base](int k) -> long long { return base + k; }, ns, c4_0, c4_step,
                          dst_row, lse_dst);
+}
+
+// Items mode with arrival words, for kernels whose rows' partial states are
+// written by NTH threads: count this split's arrival at its unit and, in the
+// block whose split completes the unit, merge the unit's splits into the
+// output rows (two float4 columns of one row per thread, half a row apart).
+// Called by all NTH threads (named barrier 1) after the partial states are
+// written.
+template <int D, int NTH>
+__device__ __forceinline__ void merge_unit_by_last(const DecodeParams &p, const Piece &pc, int tid,
+                                                   volatile int *merge_here) {
+  named_barrier(1, NTH);
+  const int ns = (pc.len + p.split_tokens - 1) / p.split_tokens;
+  if (tid == 0) {
+    __threadfence();
+    const size_t u = (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j;
+    *merge_here = unit_arrive(p.unit_ctr + u, p.epoch, ns, p.status) ? 1 : 0;
+    __threadfence();
+  }
+  named_barrier(1, NTH);
+  if (*merge_here) {
+    constexpr int kHalfRow = D / 8;
+    for (int rb = 0; rb < pc.nh; rb += NTH / kHalfRow) {
+      const int h = rb + tid / kHalfRow, c4 = tid % kHalfRow;
+      if (h < pc.nh) {
+        const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
+        merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns, c4,
+                           kHalfRow, reinterpret_cast<float4 *>(p.out + mrow * D), p.lse ? p.lse + mrow : nullptr);
+      }
+    }
+  }
 }
 
 // The q.k and p.v contractions on CUDA cores (fp32 FMA) for group ratios
@@ -1633,8 +1669,8 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
 
 // Fixed splits: one block per (sequence, head) row merges the splits
 // k < ceil(len / split_tokens) of that row.
-template <int D>
-__global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p) {
+template <int D, int NTH>
+__global__ void __launch_bounds__(NTH) gqa_combine_kernel(const CombineParams p) {
   const int row = blockIdx.x;       // [b, nq, H] flattened
   const int s = row / (p.nq * p.H);
   const int len = __ldg(p.seqlens + s);
@@ -1661,8 +1697,8 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const CombineParams p)
                          reinterpret_cast<float4 *>(p.out + static_cast<size_t>(row) * D), lse_dst);
     return;
   }
-  __shared__ MergeScratch<D> sc;
-  merge_row<D>(p.part_o, p.part_m, p.part_l, ns, [&](int k) -> long long { return base + k; }, dst, lse_dst,
+  __shared__ MergeScratch<D, NTH> sc;
+  merge_row<D, NTH>(p.part_o, p.part_m, p.part_l, ns, [&](int k) -> long long { return base + k; }, dst, lse_dst,
                threadIdx.x, sc, [] { __syncthreads(); });
 }
 
@@ -1727,10 +1763,10 @@ __global__ void __launch_bounds__(128) gqa_combine_balanced_kernel(const Combine
                             nc, c4, 0, dst, lse_dst);
     return;
   }
-  __shared__ MergeScratch<D> sc;
+  __shared__ MergeScratch<D, 128> sc;
   for (int hh = h0; hh < h0 + kRPB && hh < slice_rows; ++hh) {  // (uniform in the block)
     const size_t row2 = row_at(hh);
-    merge_row<D>(p.part_o, p.part_m, p.part_l, nc,
+    merge_row<D, 128>(p.part_o, p.part_m, p.part_l, nc,
                  [&](int k) -> long long {
                    const long long c = c_lo + k;
                    if (k > 0 && (c * W / N) == ((c + 1) * W / N)) return -1;  // empty range

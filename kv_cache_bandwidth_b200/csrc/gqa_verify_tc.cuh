@@ -245,32 +245,10 @@ __device__ __forceinline__ void tc_produce_drain(const TcBars &bars, int tile, i
 }
 
 // The block whose split completes the unit merges the unit's splits (as in
-// the mma.sync kernel): the 256 softmax threads, two float4 columns of one row
-// each.  Called by all of them, after their partial states are written.
+// the mma.sync kernel): the 256 softmax threads.
 __device__ __forceinline__ void tc_merge_unit(const DecodeParams &p, const Piece &pc, int sm,
                                               volatile int *merge_here) {
-  constexpr int D = 128;
-  constexpr int kSM = 32 * TcTile::kSoftmaxWarps;
-  named_barrier(1, kSM);
-  const int ns = (pc.len + p.split_tokens - 1) / p.split_tokens;
-  if (sm == 0) {
-    __threadfence();
-    const size_t u = (static_cast<size_t>(pc.s) * p.G + pc.g) * p.hs + pc.j;
-    *merge_here = unit_arrive(p.unit_ctr + u, p.epoch, ns, p.status) ? 1 : 0;
-    __threadfence();
-  }
-  named_barrier(1, kSM);
-  if (*merge_here) {
-    constexpr int kHalfRow = D / 8;  // two float4 columns per thread, half a row apart
-    for (int rb = 0; rb < pc.nh; rb += kSM / kHalfRow) {
-      const int h = rb + sm / kHalfRow, c4 = sm % kHalfRow;
-      if (h < pc.nh) {
-        const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
-        merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns, c4,
-                           kHalfRow, reinterpret_cast<float4 *>(p.out + mrow * D), p.lse ? p.lse + mrow : nullptr);
-      }
-    }
-  }
+  merge_unit_by_last<128, 32 * TcTile::kSoftmaxWarps>(p, pc, sm, merge_here);
 }
 
 // Where the rows of a piece go.  final_row: normalised rows into out (and
@@ -447,6 +425,9 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
   const size_t ps = tc_part_index(p, pc, dest, row, rho);
   const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
   const float s0 = dest.final_row ? w0 * inv : w0, s1 = dest.final_row ? w1 * inv : w1;
+  // a final row without a valid result is zero (a select: O may hold anything
+  // after a skipped page or a timeout)
+  const bool zero_row = dest.final_row && inv == 0.f;
   {
     // this thread writes columns [64 half + 32 sub, + 32) of the row
     uint32_t oa[32], ob[32];
@@ -460,7 +441,8 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
       for (int j = 0; j < 8; ++j) {
         float v[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = __uint_as_float(oa[4 * j + e]) * s0 + __uint_as_float(ob[4 * j + e]) * s1;
+        for (int e = 0; e < 4; ++e)
+          v[e] = zero_row ? 0.f : __uint_as_float(oa[4 * j + e]) * s0 + __uint_as_float(ob[4 * j + e]) * s1;
         dst[j] = make_float4(v[0], v[1], v[2], v[3]);
       }
     }
@@ -624,6 +606,9 @@ __device__ __forceinline__ bool tc_softmax_wide(const DecodeParams &p, const Pie
   const size_t ps = tc_part_index(p, pc, dest, row, r);
   const float inv = (!bad && done && l_row > 0.f) ? 1.f / l_row : 0.f;
   const float s0 = dest.final_row ? w0 * inv : w0, s1 = dest.final_row ? w1 * inv : w1;
+  // a final row without a valid result is zero (a select: O may hold anything
+  // after a skipped page or a timeout)
+  const bool zero_row = dest.final_row && inv == 0.f;
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     uint32_t oa[32], ob[32];
@@ -637,7 +622,8 @@ __device__ __forceinline__ bool tc_softmax_wide(const DecodeParams &p, const Pie
       for (int j = 0; j < 8; ++j) {
         float v[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = __uint_as_float(oa[4 * j + e]) * s0 + __uint_as_float(ob[4 * j + e]) * s1;
+        for (int e = 0; e < 4; ++e)
+          v[e] = zero_row ? 0.f : __uint_as_float(oa[4 * j + e]) * s0 + __uint_as_float(ob[4 * j + e]) * s1;
         dst[j] = make_float4(v[0], v[1], v[2], v[3]);
       }
     }
