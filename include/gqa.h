@@ -341,9 +341,14 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
  *                          thread-block cluster (<= 8) sharing each unit's
  *                          tokens and merging through distributed shared
  *                          memory, one kernel and no workspace (the workspace
- *                          passed is not touched).
+ *                          passed is not touched); taken only when every
+ *                          cluster of the grid is resident at once on the
+ *                          device (clusters sit inside one GPC), else the
+ *                          fixed splits.
  * split_tokens_out / cluster_out may be NULL.  num_sms <= 0 queries the
- * current device.  A negative value is a GQA_ERR_* code.
+ * current device (its cluster occupancy included); num_sms > 0 plans for a
+ * device of that many SMs without asking it.  A negative value is a GQA_ERR_*
+ * code.
  */
 #define GQA_PLAN_EQUAL_WORK 0
 #define GQA_PLAN_FIXED_SPLITS 1

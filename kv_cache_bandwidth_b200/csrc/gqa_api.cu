@@ -258,6 +258,7 @@ struct Launch {
   int cluster;
   cudaStream_t stream;
   bool pdl = false;  // programmatic dependent launch (the kernel waits before its first global read)
+  bool query = false;  // cluster mode: only ask whether every cluster of the grid is resident at once
 };
 
 template <int D, int NT, int NHB, int STAGES, bool PAGED, Mode MODE, int FMA = 0>
@@ -314,6 +315,12 @@ int launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const DecodePa
     attr[0].val.clusterDim.x = l.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    if (l.query) {
+      // 1: one wave holds every cluster (a second wave would double the step)
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) return GQA_ERR_CUDA;
+      return static_cast<long long>(n) >= static_cast<long long>(l.grid.y) * l.grid.z ? 1 : 0;
+    }
     if (l.pdl) {
       attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
       attr[1].val.programmaticStreamSerializationAllowed = 1;
@@ -686,6 +693,17 @@ int auto_cluster(const Shape &sh, bool paged, bool lse, int sms) {
   return (4 * blocks >= 3 * slots && 10 * blocks <= 9 * slots) ? c : 0;
 }
 
+// Whether the cluster decomposition's clusters all fit the current device at
+// once (thread-block clusters must sit inside one GPC; on B200 eight blocks
+// of one SM each fit 15 times, of half an SM each 33 times).
+bool cluster_fits(const Shape &sh, int c) {
+  CUtensorMap tk{}, tv{};
+  DecodeParams p{};
+  Launch l{dim3(c, sh.G * sh.hs, sh.b), c, nullptr, true};
+  l.query = true;
+  return launch_decode<Mode::kCluster>(sh, tk, tv, p, l) == 1;
+}
+
 // split_tokens == 0 in the split API: checks shared by its entry points.
 int prepare_auto(const gqa_dims *dims, bool paged, int32_t max_seqlen, const void *workspace,
                  size_t workspace_bytes, Shape *sh, int nq = 1, const int32_t *group_of_head = nullptr) {
@@ -818,7 +836,7 @@ int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, c
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
     const int c = auto_cluster(sh, dims_paged(dims), ex.lse != nullptr, std::min(dev.sms, 256));
-    if (c > 0) return run_cluster(sh, c, q, k_cache, v_cache, seqlens, page_table, out, scale, status, st);
+    if (c > 0 && cluster_fits(sh, c)) return run_cluster(sh, c, q, k_cache, v_cache, seqlens, page_table, out, scale, status, st);
     // (a group map runs on fixed splits only: the library picks them as for a contiguous cache)
     const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) {
@@ -937,7 +955,8 @@ int32_t gqa_plan_decomposition(const gqa_dims *dims, int32_t max_seqlen, int32_t
   int rc = check_dims(dims, dims_paged(dims), &sh);
   if (rc != GQA_OK) return rc;
   if (max_seqlen < 1) return GQA_ERR_DIMS;
-  if (num_sms <= 0) {
+  const bool on_device = num_sms <= 0;  // plan for the current device (its cluster occupancy included)
+  if (on_device) {
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
     num_sms = dev.sms;
@@ -946,7 +965,7 @@ int32_t gqa_plan_decomposition(const gqa_dims *dims, int32_t max_seqlen, int32_t
   if (split_tokens_out) *split_tokens_out = 0;
   if (cluster_out) *cluster_out = 1;
   const int c = auto_cluster(sh, dims_paged(dims), false, num_sms);
-  if (c > 0) {
+  if (c > 0 && (!on_device || cluster_fits(sh, c))) {
     if (cluster_out) *cluster_out = c;
     return GQA_PLAN_CLUSTERS;
   }
