@@ -54,14 +54,15 @@ namespace gqa {
 // QROWS = 64 (at most 64 rows, SPREAD): M = 64, whose accumulator rows sit in
 // the first 16 lanes of each 32-lane quarter (row m in lane m % 16 + 32 (m /
 // 16)), exactly where the spread softmax reads them; Q then takes half the
-// shared memory.  The P.V product always has M = 128 (P from tensor memory,
-// lane = row): the lanes no row uses hold leftovers whose products land in O
-// rows that are never read.
+// shared memory.  The P.V product takes P from tensor memory with the same
+// M: with 64 rows its A operand and accumulator use that same lane layout
+// (P written over the scores, O rows where the softmax threads read them),
+// half the work of a 128-row product; with 128 rows lane = row.
 template <int STAGES, int QBUFS, int QROWS>
 struct TcLayout {
   static constexpr int kD = 128;
   static constexpr int kT = 64;                        // tokens per tile
-  static constexpr int kM = 128;                       // rows of the P.V product (padded)
+  static constexpr int kM = 128;                       // rows at most (M of the 128-row products)
   static constexpr int kQRows = QROWS;                 // rows of the Q K^T product (padded)
   static constexpr int kStages = STAGES;
   static constexpr int kQBufs = QBUFS;
@@ -685,7 +686,7 @@ __device__ __forceinline__ bool tc_issue_pv(uint32_t sbase, uint32_t tmem, const
   constexpr int T = TT::kT;
   constexpr int ST = TT::kStages;
   constexpr int SP = TT::kSP;
-  constexpr uint32_t kIdescPV = tc_idesc_bf16(128, 128, true);
+  constexpr uint32_t kIdescPV = tc_idesc_bf16(TT::kQRows, 128, true);
   for (int u = 0; u < n_tiles; ++u) {
     const int gt = gt0 + u;
     const int st = gt % ST;
