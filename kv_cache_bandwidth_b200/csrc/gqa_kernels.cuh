@@ -754,13 +754,29 @@ __device__ __forceinline__ void merge_unit_by_last(const DecodeParams &p, const 
   }
   named_barrier(1, NTH);
   if (*merge_here) {
-    constexpr int kHalfRow = D / 8;
-    for (int rb = 0; rb < pc.nh; rb += NTH / kHalfRow) {
-      const int h = rb + tid / kHalfRow, c4 = tid % kHalfRow;
-      if (h < pc.nh) {
-        const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
-        merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns, c4,
-                           kHalfRow, reinterpret_cast<float4 *>(p.out + mrow * D), p.lse ? p.lse + mrow : nullptr);
+    constexpr int kHalfRow = D / 8;      // two float4 columns per thread, half a row apart
+    constexpr int kQuarterRow = D / 16;  // four float4 columns per thread, a quarter row apart
+    if (pc.nh > NTH / kHalfRow) {
+      // more rows than one pass of half rows: quarter rows, every load of
+      // the merge in flight at once
+      for (int rb = 0; rb < pc.nh; rb += NTH / kQuarterRow) {
+        const int h = rb + tid / kQuarterRow, c4 = tid % kQuarterRow;
+        if (h < pc.nh) {
+          const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
+          merge_serial<D, 4>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns, c4,
+                             kQuarterRow, reinterpret_cast<float4 *>(p.out + mrow * D),
+                             p.lse ? p.lse + mrow : nullptr);
+        }
+      }
+    } else {
+      for (int rb = 0; rb < pc.nh; rb += NTH / kHalfRow) {
+        const int h = rb + tid / kHalfRow, c4 = tid % kHalfRow;
+        if (h < pc.nh) {
+          const size_t mrow = row_of(p, pc.s, pc.g, pc.h0 + h);
+          merge_serial<D, 2>(p.part_o, p.part_m, p.part_l, static_cast<long long>(mrow) * p.num_splits, ns, c4,
+                             kHalfRow, reinterpret_cast<float4 *>(p.out + mrow * D),
+                             p.lse ? p.lse + mrow : nullptr);
+        }
       }
     }
   }
