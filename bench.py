@@ -388,7 +388,7 @@ class Case:
             n = gqa.gqa_decode_verify_workspace_size(self.dims, nq, self.max_seqlen, split)
             self.ws = torch.empty(max(256, n), dtype=torch.uint8, device="cuda")
         self.cluster = 0
-        self.tc = nq * w.r > gqa.TC_AUTO_ROWS and w.d == 128
+        self.tc = gqa.TC_AUTO_ROWS < nq * w.r <= (128 if w.d == 128 else 64)
         if split > 0:
             self.eff_split = split
         elif nq == 1 and self.entry == "split":

@@ -96,9 +96,10 @@ extern "C" {
 #define GQA_FLAG_CONTRACT_MMA 1u   /* tensor cores (mma.sync m16n8k16 bf16) */
 #define GQA_FLAG_CONTRACT_FMA 2u   /* fp32 FMA on CUDA cores; r = H/G <= 2 only (else GQA_ERR_HEADS) */
 #define GQA_FLAG_CONTRACT_TCGEN05 4u /* 5th-gen tensor cores (tcgen05, accumulators in tensor memory): one block
-                                        takes all rows of a group (r times the query tokens, <= 128), d = 128
-                                        only; split entry points (fixed splits) only.  flags == 0 picks it by
-                                        itself for more than GQA_TC_AUTO_ROWS rows per group at d = 128 */
+                                        takes all rows of a group (r times the query tokens): <= 128 at
+                                        d = 128, <= 64 at d = 64 (else GQA_ERR_HEADS); split entry points
+                                        (fixed splits) only.  flags == 0 picks it by itself for more than
+                                        GQA_TC_AUTO_ROWS rows per group */
 /* Above this many rows per group the mma.sync kernel would need a second 16-row slice. */
 #define GQA_TC_AUTO_ROWS 16
 
@@ -256,9 +257,9 @@ int gqa_decode_split_lse(const void *q, const void *k_cache, const void *v_cache
  * the end-aligned mask of a causal decoder.  For each KV group, the n_query * r
  * (token, head) pairs form the group's rows and share each K/V tile read from
  * HBM: with up to 16 rows per group (the mma.sync kernel), or up to 128 at
- * d = 128 (the tcgen05 kernel, taken by itself above GQA_TC_AUTO_ROWS rows),
- * the cache is read once per step for all drafts; with more rows, the
- * mma.sync kernel reads it once per 16-row slice.
+ * d = 128 and 64 at d = 64 (the tcgen05 kernel, taken by itself above
+ * GQA_TC_AUTO_ROWS rows), the cache is read once per step for all drafts;
+ * with more rows, the mma.sync kernel reads it once per 16-row slice.
  *
  * q: bf16 [b, n_query, H, d]; out: fp32 [b, n_query, H, d]; lse: fp32
  * [b, n_query, H] or NULL (the natural-log normaliser of each row, as in

@@ -98,7 +98,7 @@ int encode_pool(CUtensorMap *map, const void *base, int D, int rows_per_page, in
 struct Shape {
   int b, H, G, r, D, P, num_pages, max_pages;
   bool mapped;  // group of each head from a table (r = the largest group)
-  bool tc;      // the tcgen05 kernel: all rows of a group in one block (d = 128, <= 128 rows)
+  bool tc;      // the tcgen05 kernel: all rows of a group in one block (<= 128 rows at d = 128, 64 at d = 64)
   bool paged;
   long long capacity;
   int nt, nhb;  // kernel variant: n8 row tiles per consumer warp, row blocks of 8
@@ -178,12 +178,13 @@ int check_dims(const gqa_dims *dims, bool paged, Shape *sh, int nq = 1, const in
   s.nt = 1;
   s.nhb = (s.rc + 7) / 8;
   s.fma = (d.flags & GQA_FLAG_CONTRACT_FMA) != 0;
+  // rows one tcgen05 block takes: 128 at d = 128, 64 at d = 64 (the spread layout)
+  const int tc_rows = s.D == 128 ? gqa::TcTile::kM : gqa::TcTileSpread64::kQRows;
   s.tc = (d.flags & GQA_FLAG_CONTRACT_TCGEN05) != 0 ||
-         (auto_tc && d.flags == 0 && s.D == 128 && s.rq > kTcAutoRows && s.rq <= gqa::TcTile::kM);
+         (auto_tc && d.flags == 0 && s.rq > kTcAutoRows && s.rq <= tc_rows);
   if (s.tc) {
-    // one block takes all rows of a group: up to 128 rows, d = 128
-    if (s.D != 128) return GQA_ERR_HEAD_DIM;
-    if (s.rq > gqa::TcTile::kM) return GQA_ERR_HEADS;
+    // one block takes all rows of a group
+    if (s.rq > tc_rows) return GQA_ERR_HEADS;
     s.rc = s.rq;
     s.hs = 1;
   }
@@ -372,14 +373,19 @@ int launch_decode(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv,
 
 int tile_tokens(const Shape &sh) { return sh.D == 64 ? 128 : 64; }
 
-// The tcgen05 kernel (items mode; d = 128, 64-token tiles like the mma.sync kernel).
+// The tcgen05 kernel (items mode; d = 128 with 64-token tiles, d = 64 with
+// 128-token tiles, like the mma.sync kernel).
 int launch_verify_tc(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p,
                      const Launch &l) {
   // at most 64 rows: spread over the four lane quarters of tensor memory
+  // (always at d = 64)
   const bool spread = sh.rc <= 64;
-  auto kernel = sh.paged ? (spread ? gqa::gqa_verify_tc_kernel<true, true> : gqa::gqa_verify_tc_kernel<true, false>)
-                         : (spread ? gqa::gqa_verify_tc_kernel<false, true> : gqa::gqa_verify_tc_kernel<false, false>);
-  const int smem = spread ? gqa::TcTileSpread::kSmemBytes : gqa::TcTile::kSmemBytes;
+  auto kernel = sh.D == 64 ? (sh.paged ? gqa::gqa_verify_tc_kernel<true, true, 64>
+                                       : gqa::gqa_verify_tc_kernel<false, true, 64>)
+                : sh.paged ? (spread ? gqa::gqa_verify_tc_kernel<true, true> : gqa::gqa_verify_tc_kernel<true, false>)
+                           : (spread ? gqa::gqa_verify_tc_kernel<false, true> : gqa::gqa_verify_tc_kernel<false, false>);
+  const int smem = sh.D == 64 ? gqa::TcTileSpread64::kSmemBytes
+                              : spread ? gqa::TcTileSpread::kSmemBytes : gqa::TcTile::kSmemBytes;
   static std::atomic<unsigned long long> attr_set{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
@@ -391,6 +397,10 @@ int launch_verify_tc(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &
         return GQA_ERR_CUDA;
     for (auto k : {gqa::gqa_verify_tc_kernel<true, false>, gqa::gqa_verify_tc_kernel<false, false>})
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gqa::TcTile::kSmemBytes) !=
+          cudaSuccess)
+        return GQA_ERR_CUDA;
+    for (auto k : {gqa::gqa_verify_tc_kernel<true, true, 64>, gqa::gqa_verify_tc_kernel<false, true, 64>})
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gqa::TcTileSpread64::kSmemBytes) !=
           cudaSuccess)
         return GQA_ERR_CUDA;
     attr_set.fetch_or(bit, std::memory_order_acq_rel);

@@ -1,6 +1,8 @@
 // gqa_verify_tc.cuh -- decode of many rows per KV group on the 5th-generation
 // tensor cores (tcgen05): the rows of a verification step (n query tokens x r
-// heads) or of a large group ratio, up to 128 per block, against d = 128.
+// heads) or of a large group ratio, up to 128 per block at d = 128 (64-token
+// tiles), up to 64 at d = 64 (128-token tiles: the same 16 KB of K per tile,
+// S and P 128 columns wide).
 //
 // With more than 16 rows per group the mma.sync kernel has to cut the rows
 // into 16-row slices, each with its own pass over the group's keys and values
@@ -58,20 +60,22 @@ namespace gqa {
 // M: with 64 rows its A operand and accumulator use that same lane layout
 // (P written over the scores, O rows where the softmax threads read them),
 // half the work of a 128-row product; with 128 rows lane = row.
-template <int STAGES, int QBUFS, int QROWS>
+template <int STAGES, int QBUFS, int QROWS, int D = 128>
 struct TcLayout {
-  static constexpr int kD = 128;
-  static constexpr int kT = 64;                        // tokens per tile
+  static_assert(D == 64 || D == 128, "d = 64 or 128");
+  static constexpr int kD = D;
+  static constexpr int kT = D == 64 ? 128 : 64;        // tokens per tile (16 KB of K either way)
+  static constexpr int kHalves = D / 64;               // 64-column (128-byte) halves of a row
   static constexpr int kM = 128;                       // rows at most (M of the 128-row products)
   static constexpr int kQRows = QROWS;                 // rows of the Q K^T product (padded)
   static constexpr int kStages = STAGES;
   static constexpr int kQBufs = QBUFS;
   static constexpr int kHalf = kT * 128;               // one 64-column half of a K or V tile
-  static constexpr int kTileBytes = 2 * kHalf;         // 16 KB
+  static constexpr int kTileBytes = kHalves * kHalf;   // 16 KB
   static constexpr int kStageBytes = 2 * kTileBytes;   // K + V
-  static constexpr int kQOff = kStages * kStageBytes;  // Q: two halves of QROWS rows x 128 B per buffer
+  static constexpr int kQOff = kStages * kStageBytes;  // Q: kHalves halves of QROWS rows x 128 B per buffer
   static constexpr int kQHalf = kQRows * 128;
-  static constexpr int kQBytes = 2 * kQHalf;
+  static constexpr int kQBytes = kHalves * kQHalf;
   static constexpr int kBarOff = kQOff + kQBufs * kQBytes;
   static constexpr int kSP = 3;                        // S/P buffers in tensor memory
   // full[kStages], empty[kStages], s_full[kSP], p_full[kSP], pv_done[kSP],
@@ -84,17 +88,21 @@ struct TcLayout {
   static constexpr int kSmemBytes = 1024 + kMiscOff + 4 * (kStages + 4);
   static constexpr int kSoftmaxWarps = 8;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
-  static constexpr uint32_t kOCol = 256;               // O of the first halves: 256 .. 383, second: 384 .. 511
-  static constexpr uint32_t kTmemCols = 512;           // S, then P over it (kSP x 64 columns) + 2 O
+  // S, then P over it (kSP x kT columns), then the two O of kD columns
+  static constexpr uint32_t kOCol = D == 128 ? 256 : kSP * kT;
+  static constexpr uint32_t kTmemCols = 512;
   static_assert(kSP * kT <= static_cast<int>(kOCol) && kOCol + 2 * kD <= kTmemCols, "tensor-memory columns");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 // One piece per block (up to 128 rows), and its SPREAD form (up to 64 rows,
 // whose smaller Q leaves room for a sixth ring stage).
+// d = 64 runs the SPREAD form only (128-token tiles).
 using TcTile = TcLayout<5, 1, 128>;
 using TcTileSpread = TcLayout<6, 1, 64>;
-template <bool SPREAD>
-using TcItemTile = typename std::conditional<SPREAD, TcTileSpread, TcTile>::type;
+using TcTileSpread64 = TcLayout<6, 1, 64, 64>;
+template <bool SPREAD, int D = 128>
+using TcItemTile = typename std::conditional<D == 64, TcTileSpread64,
+                                             typename std::conditional<SPREAD, TcTileSpread, TcTile>::type>::type;
 
 struct TcBars {
   uint32_t full0, empty0, s_full0, p_full0, pv_done0, drain0, q_full0, q_empty0, o_free;
@@ -151,7 +159,7 @@ __device__ __forceinline__ int tc_slot_row(int r, int nh) {
   return r < nh ? r : -1;
 }
 
-// Byte offset of 16-byte chunk c (of 16) of Q slot r: two 64-column halves in
+// Byte offset of 16-byte chunk c (of d / 8) of Q slot r: 64-column halves in
 // the 128-byte swizzle TMA would write.
 template <class TT>
 __device__ __forceinline__ int tc_q_offset(int r, int c) {
@@ -172,7 +180,7 @@ __device__ __forceinline__ bool tc_produce_piece(const CUtensorMap *tm_k, const 
   const int P = p.page_size;
   const int ppt = PAGED ? max(1, T / P) : 1;  // pages per tile
   const int br = PAGED ? min(P, T) : T;        // rows per TMA box
-  const uint32_t box_bytes = static_cast<uint32_t>(2 * br * 128);
+  const uint32_t box_bytes = static_cast<uint32_t>(TT::kHalves * br * 128);
   const int32_t *pt_row = PAGED ? p.page_table + static_cast<size_t>(pc.s) * p.max_pages : nullptr;
   const int lp_end = PAGED ? (pc.t_end + P - 1) / P : 0;
   int cur_w = -1, nxt_w = -1, win = -1, nxt = -1;
@@ -220,7 +228,7 @@ __device__ __forceinline__ bool tc_produce_piece(const CUtensorMap *tm_k, const 
         const int row = (P >= T) ? (t0 % P) : 0;
         const uint32_t off = static_cast<uint32_t>(lane * br * 128);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < TT::kHalves; ++h) {
           tma_load_4d(dst_k + h * TT::kHalf + off, tm_k, full, h * 64, row, pc.g, id, policy);
           tma_load_4d(dst_v + h * TT::kHalf + off, tm_v, full, h * 64, row, pc.g, id, policy);
         }
@@ -228,7 +236,7 @@ __device__ __forceinline__ bool tc_produce_piece(const CUtensorMap *tm_k, const 
     } else if (lane == 0) {
       mbar_arrive_expect_tx(full, 2u * box_bytes);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < TT::kHalves; ++h) {
         tma_load_4d(dst_k + h * TT::kHalf, tm_k, full, h * 64, t0, pc.g, pc.s, policy);
         tma_load_4d(dst_v + h * TT::kHalf, tm_v, full, h * 64, t0, pc.g, pc.s, policy);
       }
@@ -247,9 +255,10 @@ __device__ __forceinline__ void tc_produce_drain(const TcBars &bars, int tile, i
 
 // The block whose split completes the unit merges the unit's splits (as in
 // the mma.sync kernel): the 256 softmax threads.
+template <int D>
 __device__ __forceinline__ void tc_merge_unit(const DecodeParams &p, const Piece &pc, int sm,
                                               volatile int *merge_here) {
-  merge_unit_by_last<128, 32 * TcTile::kSoftmaxWarps>(p, pc, sm, merge_here);
+  merge_unit_by_last<D, 32 * TcTile::kSoftmaxWarps>(p, pc, sm, merge_here);
 }
 
 // Where the rows of a piece go.  final_row: normalised rows into out (and
@@ -279,13 +288,13 @@ __device__ __forceinline__ bool tc_piece_done(volatile int *stop, volatile int *
 // Softmax warps with at most 64 rows (SPREAD), for one piece of n_tiles tiles
 // starting at global tile gt0 of the block's pipeline: quarter qd = warp % 4 of
 // the tensor-memory lanes holds rows qd * rpq .. in its first rpq <= 16 lanes
-// (rpq = ceil(rows / 4)).  Warp w takes tokens [32 h, 32 h + 32) of every
-// tile, h = w / 4, and within it thread t the 16 tokens [32 h + 16 (t / 16),
-// + 16) of lane t % 16 (the 16x32bx2 shape).  The two threads of a row in one
+// (rpq = ceil(rows / 4)).  Warp w takes tokens [T/2 h, T/2 h + T/2) of every
+// tile (T = 64, or 128 at d = 64), h = w / 4, and within it thread t the T/4
+// tokens [T/2 h + T/4 (t / 16), + T/4) of lane t % 16 (the 16x32bx2 shape).  The two threads of a row in one
 // warp share its running base (their maximum meets through one shuffle) and
 // the row's O_h in tensor memory; the two warps of a quarter keep separate
 // states and O_h, merged once at the end.  P's high part goes over the
-// thread's first 8 score columns, its residual over the next 8.  Returns
+// thread's first T/8 score columns, its residual over the next T/8.  Returns
 // false once the block stops (a timeout).
 template <class TT, bool PAGED>
 __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const Piece &pc, uint8_t *smem,
@@ -298,11 +307,14 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
   constexpr int ST = TT::kStages;
   constexpr int SP = TT::kSP;
   constexpr int kSM = 32 * TT::kSoftmaxWarps;
+  constexpr int HT = T / 2;                // tokens of a warp half
+  constexpr int TPT = T / 4;               // tokens (score columns) of a thread: 16, or 32 at d = 64
+  constexpr int CW = D / 4;                // output columns of a thread
   const float kNegInf = -__int_as_float(0x7f800000);
   const int sm = threadIdx.x;
   const int qd = warp % 4;                 // lane quarter
-  const int half = warp / 4;               // tokens [32 half, 32 half + 32) of every tile
-  const int sub = lane >> 4;               // ... of which [16 sub, 16 sub + 16)
+  const int half = warp / 4;               // tokens [HT half, HT half + HT) of every tile
+  const int sub = lane >> 4;               // ... of which [TPT sub, TPT sub + TPT)
   const int li = lane & 15;                // lane within the quarter
   const int rpq = (pc.nh + 3) / 4;         // rows per quarter
   const int rho = qd * rpq + li;           // row of the slice
@@ -327,8 +339,8 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
     ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full0 + 8 * b, (gt / SP) & 1));
     if (!ok) break;
     tc_fence_after();
-    uint32_t sv[16];
-    tc_ld16x2_x16<16>(lane_tmem + b * 64 + half * 32, sv);
+    uint32_t sv[TPT];
+    tc_ld16x2_cols<TPT, TPT>(lane_tmem + b * T + half * HT, sv);
     tc_wait_ld();
     if (PAGED) bad |= tile_bad[st];
     // V rows past the piece's end may hold anything (even NaN): zero them so
@@ -336,29 +348,32 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
     const int valid_rows = min(T, pc.t_end - t0);
     if (valid_rows < T) {
       uint8_t *vt = smem + st * TT::kStageBytes + TT::kTileBytes;
-      for (int idx = sm; idx < (T - valid_rows) * 16; idx += kSM) {
-        const int row = valid_rows + idx / 16, c = idx % 16;
+      for (int idx = sm; idx < (T - valid_rows) * (D / 8); idx += kSM) {
+        const int row = valid_rows + idx / (D / 8), c = idx % (D / 8);
         *reinterpret_cast<uint4 *>(vt + (c >> 3) * TT::kHalf + row * 128 + ((c & 7) << 4)) =
             make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    float x[16];
-    const int tb = t0 + half * 32 + sub * 16;  // this thread's first token of the tile
-    if (tb + 16 <= lim) {
+    float x[TPT];
+    const int tb = t0 + half * HT + sub * TPT;  // this thread's first token of the tile
+    if (tb + TPT <= lim) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = __uint_as_float(sv[j]) * sl;
+      for (int j = 0; j < TPT; ++j) x[j] = __uint_as_float(sv[j]) * sl;
     } else {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
+      for (int j = 0; j < TPT; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
     }
     float mx;
     {
-      float m4[4];
+      float m4[TPT / 4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) m4[k] = fmaxf(fmaxf(x[4 * k], x[4 * k + 1]), fmaxf(x[4 * k + 2], x[4 * k + 3]));
-      mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      for (int k = 0; k < TPT / 4; ++k)
+        m4[k] = fmaxf(fmaxf(x[4 * k], x[4 * k + 1]), fmaxf(x[4 * k + 2], x[4 * k + 3]));
+      mx = m4[0];
+#pragma unroll
+      for (int k = 1; k < TPT / 4; ++k) mx = fmaxf(mx, m4[k]);
     }
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the row's other 16 tokens of this half
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the row's other TPT tokens of this half
     if (warp_active) {
       // lazy rescale: only when a score passes the base by more than 2^8 (the
       // same decision in both threads of the row)
@@ -369,18 +384,18 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
         l_run *= alpha;
         if (t > 0) {
           // O_h holds the piece's tiles 0 .. t-1: rescale it once their MMAs
-          // are done; thread sub takes columns [64 sub, 64 sub + 64) of the row
+          // are done; thread sub takes columns [D/2 sub, D/2 sub + D/2) of the row
           ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done0 + 8 * ((gt - 1) % SP), ((gt - 1) / SP) & 1));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < D / 64; ++c) {
             uint32_t ov[32];
-            tc_ld16x2_x32<64>(lane_tmem + TT::kOCol + half * D + c * 32, ov);
+            tc_ld16x2_x32<D / 2>(lane_tmem + TT::kOCol + half * D + c * 32, ov);
             tc_wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-            tc_st16x2_x32<64>(lane_tmem + TT::kOCol + half * D + c * 32, ov);
+            tc_st16x2_x32<D / 2>(lane_tmem + TT::kOCol + half * D + c * 32, ov);
           }
           tc_wait_st();
           tc_fence_before();
@@ -388,15 +403,15 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
         m_run = mn;
       }
       const float base = (m_run == kNegInf) ? 0.f : m_run;
-      uint32_t hi[8], lo[8];
+      uint32_t hi[TPT / 2], lo[TPT / 2];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < TPT / 2; ++e) {
         const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
         l_run += p0 + p1;
         split_bf16x2_rz(p0, p1, hi[e], lo[e]);
       }
-      tc_st16x2_x8<16>(lane_tmem + b * 64 + half * 32, hi);
-      tc_st16x2_x8<16>(lane_tmem + b * 64 + half * 32 + 8, lo);
+      tc_st16x2_cols<TPT / 2, TPT>(lane_tmem + b * T + half * HT, hi);
+      tc_st16x2_cols<TPT / 2, TPT>(lane_tmem + b * T + half * HT + TPT / 2, lo);
       tc_wait_st();
     }
     tc_fence_before();
@@ -430,16 +445,16 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
   // after a skipped page or a timeout)
   const bool zero_row = dest.final_row && inv == 0.f;
   {
-    // this thread writes columns [64 half + 32 sub, + 32) of the row
-    uint32_t oa[32], ob[32];
-    tc_ld16x2_x32<32>(lane_tmem + TT::kOCol + half * 64, oa);
-    tc_ld16x2_x32<32>(lane_tmem + TT::kOCol + D + half * 64, ob);
+    // this thread writes columns [D/2 half + CW sub, + CW) of the row
+    uint32_t oa[CW], ob[CW];
+    tc_ld16x2_cols<CW, CW>(lane_tmem + TT::kOCol + half * (D / 2), oa);
+    tc_ld16x2_cols<CW, CW>(lane_tmem + TT::kOCol + D + half * (D / 2), ob);
     tc_wait_ld();
     if (valid) {
-      const int col = half * 64 + sub * 32;
+      const int col = half * (D / 2) + sub * CW;
       float4 *dst = reinterpret_cast<float4 *>((dest.final_row ? p.out + row * D : p.part_o + ps * D) + col);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < CW / 4; ++j) {
         float v[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -458,7 +473,7 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
     }
   }
   tc_fence_before();
-  if (dest.slot < 0 && p.unit_ctr != nullptr && !dest.final_row) tc_merge_unit(p, pc, sm, merge_here);
+  if (dest.slot < 0 && p.unit_ctr != nullptr && !dest.final_row) tc_merge_unit<D>(p, pc, sm, merge_here);
   return tc_piece_done(stop, abort_flag, sm, kSM) && ok;
 }
 
@@ -472,6 +487,7 @@ __device__ __forceinline__ bool tc_softmax_wide(const DecodeParams &p, const Pie
                                                 volatile int *abort_flag, volatile int *merge_here,
                                                   volatile int *stop, int gt0,
                                                 int n_tiles, const TcDest &dest, int warp, int lane) {
+  static_assert(TT::kD == 128, "the 128-row layout runs at d = 128");
   constexpr int D = TT::kD;
   constexpr int T = TT::kT;
   constexpr int ST = TT::kStages;
@@ -639,7 +655,7 @@ __device__ __forceinline__ bool tc_softmax_wide(const DecodeParams &p, const Pie
     }
   }
   tc_fence_before();
-  if (dest.slot < 0 && p.unit_ctr != nullptr && !dest.final_row) tc_merge_unit(p, pc, sm, merge_here);
+  if (dest.slot < 0 && p.unit_ctr != nullptr && !dest.final_row) tc_merge_unit<128>(p, pc, sm, merge_here);
   return tc_piece_done(stop, abort_flag, sm, kSM) && ok;
 }
 
@@ -651,7 +667,8 @@ __device__ __forceinline__ bool tc_issue_qk(uint32_t sbase, uint32_t qbuf, uint3
   constexpr int D = TT::kD;
   constexpr int ST = TT::kStages;
   constexpr int SP = TT::kSP;
-  constexpr uint32_t kIdescQK = tc_idesc_bf16(TT::kQRows, 64, false);
+  constexpr int T = TT::kT;
+  constexpr uint32_t kIdescQK = tc_idesc_bf16(TT::kQRows, T, false);
   // Q's descriptors are the same for every tile; a K-step adds to the
   // start-address field (addresses stay below 256 KB: no carry)
   uint64_t qd[D / 16];
@@ -666,7 +683,7 @@ __device__ __forceinline__ bool tc_issue_qk(uint32_t sbase, uint32_t qbuf, uint3
     if (!ok) return false;
     tc_fence_after();
     const uint64_t kd = tc_smem_desc(sbase + st * TT::kStageBytes, 16, 1024);
-    const uint32_t d = tmem + (gt % SP) * 64;
+    const uint32_t d = tmem + (gt % SP) * T;
     tc_mma(d, qd[0], kd, kIdescQK, 0u);
 #pragma unroll
     for (int ks = 1; ks < D / 16; ++ks)
@@ -686,25 +703,31 @@ __device__ __forceinline__ bool tc_issue_pv(uint32_t sbase, uint32_t tmem, const
   constexpr int T = TT::kT;
   constexpr int ST = TT::kStages;
   constexpr int SP = TT::kSP;
-  constexpr uint32_t kIdescPV = tc_idesc_bf16(TT::kQRows, 128, true);
+  constexpr uint32_t kIdescPV = tc_idesc_bf16(TT::kQRows, D, true);
+  // each thread wrote the P of TPT tokens over its TPT score columns: the high
+  // part over the first TPT/2, the residual over the next TPT/2 (SPREAD: four
+  // threads per row, TPT = T/4; otherwise two, TPT = T/2)
+  constexpr int TPT = SPREAD ? T / 4 : T / 2;
   for (int u = 0; u < n_tiles; ++u) {
     const int gt = gt0 + u;
     const int st = gt % ST;
     if (!mbar_wait(bars.p_full0 + 8 * (gt % SP), (gt / SP) & 1)) return false;
     tc_fence_after();
     const uint64_t vd = tc_smem_desc(sbase + st * TT::kStageBytes + TT::kTileBytes, TT::kHalf, 1024);
-    const uint32_t pb = tmem + (gt % SP) * 64;
+    const uint32_t pb = tmem + (gt % SP) * T;
 #pragma unroll
     for (int ks = 0; ks < T / 16; ++ks) {
-      // tokens 16 ks ..: high part at column 32 (ks / 2) + 8 (ks % 2) of the
-      // buffer, the residual 16 columns further (SPREAD: the thread of those
-      // tokens wrote its high part at column 16 ks, its residual 8 further);
-      // into the O of the half of the row that owns them
+      // tokens 16 ks .. 16 ks + 15: those of thread group g = 16 ks / TPT, its
+      // (16 ks % TPT) / 16-th 16 tokens; into the O of the half of the row
+      // (tokens [T/2 h, T/2 h + T/2)) that owns them
       const uint64_t vdk = vd + ((ks * 16 * 128) >> 4);
-      const uint32_t pa = SPREAD ? pb + 16 * ks : pb + 32 * (ks >> 1) + 8 * (ks & 1);
-      const uint32_t od = tmem + TT::kOCol + D * (ks >> 1);
-      tc_mma_ts(od, pa, vdk, kIdescPV, (u > 0 || (ks & 1)) ? 1u : 0u);
-      tc_mma_ts(od, pa + (SPREAD ? 8 : 16), vdk, kIdescPV, 1u);
+      const int g = (16 * ks) / TPT, k2 = ((16 * ks) % TPT) / 16;
+      const uint32_t pa = pb + g * TPT + 8 * k2;
+      const int h = (16 * ks) / (T / 2);
+      const uint32_t od = tmem + TT::kOCol + D * h;
+      const bool first = (16 * ks) % (T / 2) == 0;  // the half's first tokens of the tile
+      tc_mma_ts(od, pa, vdk, kIdescPV, (u > 0 || !first) ? 1u : 0u);
+      tc_mma_ts(od, pa + TPT / 2, vdk, kIdescPV, 1u);
     }
     // K was read by the scores of this tile, done before its P existed; V and
     // P by these products
@@ -732,11 +755,12 @@ __device__ __forceinline__ void tc_abort(const DecodeParams &p, volatile int *ab
 // each row (two warps, 16 tokens each of their 32), through the 16-lane
 // tensor-memory shapes.  Otherwise (up to 128 rows) row i is lane i and two
 // threads take each row.
-template <bool PAGED, bool SPREAD>
+template <bool PAGED, bool SPREAD, int DH = 128>
 __global__ void __launch_bounds__(TcTile::kThreads, 1)
     gqa_verify_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const DecodeParams p) {
-  using TT = TcItemTile<SPREAD>;
+  static_assert(DH == 128 || SPREAD, "d = 64 runs the spread layout (at most 64 rows)");
+  using TT = TcItemTile<SPREAD, DH>;
   constexpr int D = TT::kD;
   constexpr int T = TT::kT;
   const float kNegInf = -__int_as_float(0x7f800000);
@@ -812,7 +836,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     const uint4 *src = rho >= 0 ? reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + rho) * D)
                                 : nullptr;
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 0; c < D / 8; ++c) {
       const uint4 v = rho >= 0 ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4 *>(smem + TT::kQOff + tc_q_offset<TT>(r, c)) = v;
     }
@@ -842,7 +866,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   } else {
     // ============================================================ softmax rows
     const TcDest dest{((pc.len + p.split_tokens - 1) / p.split_tokens == 1) && p.out != nullptr, -1};
-    if (SPREAD)
+    if constexpr (SPREAD)
       (void)tc_softmax_spread<TT, PAGED>(p, pc, smem, tmem, bars, tile_bad, abort_flag, merge_here, stop, 0,
                                          n_tiles, dest, warp, lane);
     else

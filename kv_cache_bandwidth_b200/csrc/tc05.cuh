@@ -176,6 +176,17 @@ __device__ __forceinline__ void tc_st16x2_x8(uint32_t taddr, const uint32_t (&r)
 }
 
 template <int OFF>
+__device__ __forceinline__ void tc_st16x2_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, "
+      "{%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17};"
+      :
+      : "r"(taddr), "n"(OFF), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+template <int OFF>
 __device__ __forceinline__ void tc_st16x2_x32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
@@ -187,6 +198,20 @@ __device__ __forceinline__ void tc_st16x2_x32(uint32_t taddr, const uint32_t (&r
         "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
         "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+// 16x32bx2 loads and stores of N = 8, 16 or 32 columns per thread, the upper
+// 16 threads OFF columns further (see tc_ld16x2_x16).
+template <int N, int OFF>
+__device__ __forceinline__ void tc_ld16x2_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 32) tc_ld16x2_x32<OFF>(taddr, r);
+  else tc_ld16x2_x16<OFF>(taddr, r);
+}
+template <int N, int OFF>
+__device__ __forceinline__ void tc_st16x2_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 32) tc_st16x2_x32<OFF>(taddr, r);
+  else if constexpr (N == 16) tc_st16x2_x16<OFF>(taddr, r);
+  else tc_st16x2_x8<OFF>(taddr, r);
 }
 
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

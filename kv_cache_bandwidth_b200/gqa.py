@@ -317,7 +317,7 @@ def gqa_decode_verify(q, k_cache, v_cache, seqlens, page_table=None, *, split_to
     sees the cache up to seqlens[s] - (n_query - 1 - t).  Returns out
     [b, n_query, H, d] (and lse [b, n_query, H] when want_lse or lse is given).
     With flags == 0, more than TC_AUTO_ROWS rows per KV group (n_query * H/G,
-    at most 128, d = 128) run on the tcgen05 kernel."""
+    at most 128 at d = 128, 64 at d = 64) run on the tcgen05 kernel."""
     b, nq, H, d = q.shape
     if out is None:
         out = torch.empty((b, nq, H, d), dtype=torch.float32, device=q.device)

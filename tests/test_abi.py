@@ -249,12 +249,15 @@ def test_kv_append_argument_checks(lib):
 
 def test_tcgen05_flag_checks(lib):
     """The tcgen05 contraction is rejected on the host where it does not
-    apply: d = 64, more than 128 rows per group, the cluster entry point, or
-    together with another contraction flag."""
+    apply: more than 64 rows per group at d = 64 or 128 at d = 128, the
+    cluster entry point, or together with another contraction flag."""
     tc = gqa.FLAG_CONTRACT_TCGEN05
-    d64 = _dims(head_dim=64, flags=tc)
-    assert lib.gqa_decode_split(FAKE, FAKE, FAKE, FAKE, None, FAKE, ctypes.byref(d64), 0.125, None, 128, 256,
-                                FAKE, 1 << 20, None) == -4
+    d64 = _dims(head_dim=64, num_heads=16, num_kv_heads=2, flags=tc)     # r = 8
+    # 9 query tokens x 8 heads = 72 rows per group > 64 at d = 64
+    assert lib.gqa_decode_verify(FAKE, FAKE, FAKE, FAKE, None, FAKE, None, ctypes.byref(d64), 9, 0.125, None,
+                                 128, 256, FAKE, 1 << 24, None) == -3
+    # 8 x 8 = 64 rows fit at d = 64
+    assert lib.gqa_decode_verify_workspace_size(ctypes.byref(d64), 8, 256, 128) > 0
     d128 = _dims(head_dim=128, num_heads=16, num_kv_heads=2, flags=tc)   # r = 8
     # 17 query tokens x 8 heads = 136 rows per group > 128
     assert lib.gqa_decode_verify(FAKE, FAKE, FAKE, FAKE, None, FAKE, None, ctypes.byref(d128), 17, 0.125, None,

@@ -30,17 +30,20 @@ def oracle_verify(inp, q):
 
 
 ROWS = [(1, 8), (2, 8), (4, 8), (8, 8), (3, 5), (2, 32), (1, 64), (16, 8), (2, 64)]
+# d = 64: the spread layout only (at most 64 rows), 128-token tiles
+ROWS64 = [(1, 8), (2, 8), (8, 8), (3, 5), (1, 32), (1, 64)]
+CASES = [(128,) + c for c in ROWS] + [(64,) + c for c in ROWS64]
 
 
-@pytest.mark.parametrize("nq,r", ROWS, ids=["n%d_r%d" % c for c in ROWS])
+@pytest.mark.parametrize("d,nq,r", CASES, ids=["d%d_n%d_r%d" % c for c in CASES])
 @pytest.mark.parametrize("layout", ["contig", "P16", "P64"])
 @pytest.mark.parametrize("split", [0, 128, 512])
-def test_tc_verify_against_oracle(nq, r, layout, split):
+def test_tc_verify_against_oracle(d, nq, r, layout, split):
     P = {"contig": None, "P16": 16, "P64": 64}[layout]
     G = 2 if r * nq <= 64 else 1
-    lens = [nq, 63, 64, 65, 700, 1500]
-    w = Workload(name="tc", b=len(lens), H=r * G, G=G, d=128, m=1536, page_size=P, len_lo=1 if P else None,
-                 len_hi=1536 if P else None, seed=nq * 13 + r)
+    lens = [nq, 63, 64, 65, 127, 128, 129, 700, 1500]
+    w = Workload(name="tc", b=len(lens), H=r * G, G=G, d=d, m=1536, page_size=P, len_lo=1 if P else None,
+                 len_hi=1536 if P else None, seed=nq * 13 + r + d)
     inp, q = drafts(w, nq, lens, seed=r)
     ref, ref_lse, st_ref = oracle_verify(inp, q)
     assert st_ref == 0
@@ -49,18 +52,19 @@ def test_tc_verify_against_oracle(nq, r, layout, split):
                                      want_lse=True, status=st, flags=TC)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    assert_parity(out, ref, "tc n=%d r=%d %s split=%d" % (nq, r, layout, split))
-    assert_lse(lse, ref_lse, "tc n=%d r=%d" % (nq, r))
+    assert_parity(out, ref, "tc d=%d n=%d r=%d %s split=%d" % (d, nq, r, layout, split))
+    assert_lse(lse, ref_lse, "tc d=%d n=%d r=%d" % (d, nq, r))
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("split", [128, 1024])
-def test_tc_poison_and_invalid_rows(split):
+def test_tc_poison_and_invalid_rows(split, d):
     """NaN past every length and in spare pages, an invalid length and a page
     id outside the pool: the tcgen05 kernel zeroes the tail of its V tiles
     and flags the bad rows like the mma.sync kernel."""
     nq, r, G, P = 4, 8, 2, 16
     lens = [300, 17, 1000, 64]
-    w = Workload(name="tcp", b=4, H=r * G, G=G, d=128, m=1024, page_size=P, len_lo=1, len_hi=1024, seed=5)
+    w = Workload(name="tcp", b=4, H=r * G, G=G, d=d, m=1024, page_size=P, len_lo=1, len_hi=1024, seed=5)
     inp, q = drafts(w, nq, lens, seed=3, poison=True)
     ref, _, _ = oracle_verify(inp, q)
     out = gqa.gqa_decode_verify(q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table, split_tokens=split,
@@ -110,9 +114,10 @@ def test_tc_group_map():
 def test_tc_rejections():
     w = Workload(name="tcx", b=1, H=8, G=1, d=64, m=128, seed=2)
     inp = make_inputs(w, device="cuda", lens=[128])
-    with pytest.raises(gqa.GqaError) as e:        # d = 64
-        gqa.gqa_decode_split(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, None, split_tokens=128, flags=TC)
-    assert e.value.code == -4
+    q = torch.randn(1, 9, 8, 64).to(torch.bfloat16).cuda()     # 72 rows at d = 64
+    with pytest.raises(gqa.GqaError) as e:
+        gqa.gqa_decode_verify(q, inp.k_cache, inp.v_cache, inp.seqlens, None, split_tokens=128, flags=TC)
+    assert e.value.code == -3
     w = Workload(name="tcy", b=1, H=8, G=1, d=128, m=128, seed=2)
     inp = make_inputs(w, device="cuda", lens=[128])
     q = torch.randn(1, 17, 8, 128).to(torch.bfloat16).cuda()   # 136 rows
