@@ -327,7 +327,10 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
   const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(qd * 32) << 16);
   float *mbase = reinterpret_cast<float *>(smem + TT::kXOff);  // [half][slot]
   float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);   // [half][slot]
-  const float sl = p.scale_log2;
+  // |scale| log2(e): a negative scale's sign is folded into Q when it is
+  // loaded, so that the maximum of the raw scores is the maximum of the
+  // scaled ones and the exponent is one fma of the raw score
+  const float sl = fabsf(p.scale_log2);
   float m_run = kNegInf, l_run = 0.f;  // this half's base (shared by the pair) and this thread's sum
   int bad = 0;
   bool ok = true;
@@ -354,14 +357,16 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
             make_uint4(0u, 0u, 0u, 0u);
       }
     }
+    // raw scores (-inf past the row's limit)
     float x[TPT];
     const int tb = t0 + half * HT + sub * TPT;  // this thread's first token of the tile
-    if (tb + TPT <= lim) {
+    const bool edge = tb + TPT > lim;
+    if (!edge) {
 #pragma unroll
-      for (int j = 0; j < TPT; ++j) x[j] = __uint_as_float(sv[j]) * sl;
+      for (int j = 0; j < TPT; ++j) x[j] = __uint_as_float(sv[j]);
     } else {
 #pragma unroll
-      for (int j = 0; j < TPT; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) * sl : kNegInf;
+      for (int j = 0; j < TPT; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) : kNegInf;
     }
     float mx;
     {
@@ -373,6 +378,7 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
 #pragma unroll
       for (int k = 1; k < TPT / 4; ++k) mx = fmaxf(mx, m4[k]);
     }
+    mx = (mx == kNegInf) ? kNegInf : mx * sl;              // the scaled maximum
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the row's other TPT tokens of this half
     if (warp_active) {
       // lazy rescale: only when a score passes the base by more than 2^8 (the
@@ -402,11 +408,19 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
         }
         m_run = mn;
       }
-      const float base = (m_run == kNegInf) ? 0.f : m_run;
+      const float nb = (m_run == kNegInf) ? 0.f : -m_run;
+      if (edge) {
+        // the exponent of a masked score is -inf whatever the scale
+#pragma unroll
+        for (int j = 0; j < TPT; ++j) x[j] = (x[j] == kNegInf) ? kNegInf : fmaf(x[j], sl, nb);
+      } else {
+#pragma unroll
+        for (int j = 0; j < TPT; ++j) x[j] = fmaf(x[j], sl, nb);
+      }
       uint32_t hi[TPT / 2], lo[TPT / 2];
 #pragma unroll
       for (int e = 0; e < TPT / 2; ++e) {
-        const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
+        const float p0 = ex2(x[2 * e]), p1 = ex2(x[2 * e + 1]);
         l_run += p0 + p1;
         split_bf16x2_rz(p0, p1, hi[e], lo[e]);
       }
@@ -507,7 +521,7 @@ __device__ __forceinline__ bool tc_softmax_wide(const DecodeParams &p, const Pie
   const uint32_t lane_tmem = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
   float *mbase = reinterpret_cast<float *>(smem + TT::kXOff);  // [half][row]
   float *lsum = reinterpret_cast<float *>(smem + TT::kLOff);   // [half][row]
-  const float sl = p.scale_log2;
+  const float sl = fabsf(p.scale_log2);  // (a negative scale's sign is in Q)
   float m_run = kNegInf, l_run = 0.f;  // this half's base and sum
   int bad = 0;
   bool ok = true;
@@ -835,9 +849,16 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
     const int rho = tc_slot_row<SPREAD>(r, pc.nh);
     const uint4 *src = rho >= 0 ? reinterpret_cast<const uint4 *>(p.q + row_of(p, pc.s, pc.g, pc.h0 + rho) * D)
                                 : nullptr;
+    // (a negative scale: the sign goes into q, exactly, so that the softmax
+    // threads scale by |scale|)
+    const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
-      const uint4 v = rho >= 0 ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+      uint4 v = rho >= 0 ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+      v.x ^= flip;
+      v.y ^= flip;
+      v.z ^= flip;
+      v.w ^= flip;
       *reinterpret_cast<uint4 *>(smem + TT::kQOff + tc_q_offset<TT>(r, c)) = v;
     }
     fence_proxy_async_smem();

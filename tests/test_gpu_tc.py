@@ -127,3 +127,25 @@ def test_tc_rejections():
     with pytest.raises(gqa.GqaError) as e:        # the cluster entry point has no tcgen05 variant
         gqa.gqa_decode(inp.q, inp.k_cache, inp.v_cache, inp.seqlens, None, flags=TC)
     assert e.value.code == -6
+
+
+@pytest.mark.parametrize("scale", [-0.08, 0.0, 0.3])
+@pytest.mark.parametrize("d", [128, 64])
+def test_tc_scale_sign_and_zero(scale, d):
+    """Any finite scale: the tcgen05 kernel takes the maximum of the raw
+    scores and folds a negative scale's sign into q (exactly), so a negative,
+    a zero (uniform weights over the visible positions) and a large scale
+    all agree with the oracle, masked drafts included."""
+    nq, r, G = 4, 8, 2
+    lens = [nq, 100, 700, 1024]
+    w = Workload(name="tcs", b=len(lens), H=r * G, G=G, d=d, m=1024, seed=77)
+    inp, q = drafts(w, nq, lens, seed=5)
+    ref, _, st_ref = oracle.gqa_decode_verify(q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu(), inp.seqlens.cpu(),
+                                              num_kv_heads=G, scale=scale)
+    assert st_ref == 0
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gqa.gqa_decode_verify(q, inp.k_cache, inp.v_cache, inp.seqlens, None, split_tokens=512, scale=scale,
+                                status=st, flags=TC)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_parity(out, ref, "tc d=%d scale=%g" % (d, scale))

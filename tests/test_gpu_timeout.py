@@ -68,6 +68,8 @@ CASES = [
      Workload(name="t4", b=2, H=16, G=2, d=128, m=1024, seed=34), 4, 256, TC, (1, 1)),
     ("tcgen05 kernel, split 0 (fixed splits of the library's choice)",
      Workload(name="t6", b=4, H=16, G=2, d=128, m=4096, seed=36), 4, 0, TC, (0, 1)),
+    ("tcgen05 kernel, d = 64 (128-token tiles)",
+     Workload(name="t7", b=2, H=16, G=2, d=64, m=2048, seed=37), 8, 512, TC, (1, 2)),
 ]
 
 
