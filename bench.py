@@ -70,6 +70,7 @@ def peaks():
 # these hash the same.
 KERNEL_SOURCES = {
     "gqa_decode_kernel": ("gqa_api.cu", "gqa_kernels.cuh", "ptx.cuh"),
+    "gqa_combine_kernel": ("gqa_api.cu", "gqa_kernels.cuh", "ptx.cuh"),
     "gqa_verify_tc_kernel": ("gqa_api.cu", "gqa_kernels.cuh", "gqa_verify_tc.cuh", "ptx.cuh", "tc05.cuh"),
 }
 
