@@ -14,12 +14,16 @@
 //   S[rows, 64 tokens]  = Q[rows, 128] . K_tile[64, 128]^T        (M = 128, N = 64)
 //   O[rows, 128]       += P[rows, 64] . V_tile[64, 128]            (M = 128, N = 128)
 //
-// Rows are padded to M = 128; P enters as a bf16 high part and a bf16
-// residual (two MMAs), as in the mma.sync kernel, here both truncated (byte
-// permutes, no conversions: P to within 2^-14 relative).  P is written to
-// tensor memory over its own scores (each thread over the columns it has read)
-// and the P.V product takes its A operand from there, which leaves shared
-// memory to a 5-stage K/V ring.  Warp roles:
+// With up to 128 rows (the layout described here) the rows are padded to
+// M = 128; with up to 64 (the spread layout, see tc_softmax_spread; the only
+// one at d = 64) both products have M = 64 and the rows sit in the first 16
+// lanes of each tensor-memory lane quarter, four threads per row.  P enters
+// as a bf16 high part and a bf16 residual (two MMAs), as in the mma.sync
+// kernel, here both truncated (byte permutes, no conversions: P to within
+// 2^-14 relative).  P is written to tensor memory over its own scores (each
+// thread over the columns it has read) and the P.V product takes its A
+// operand from there, which leaves shared memory to a 5-stage K/V ring (6 in
+// the spread layout, whose Q is half as large).  Warp roles:
 //   * warps 0-7: two threads per row (warps w and w+4 share the tensor-memory
 //     lanes of rows 32(w%4) ..), each taking 32 of a tile's 64 tokens with a
 //     softmax state of its own: its running base and sum, and its own O in
