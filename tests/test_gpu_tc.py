@@ -149,3 +149,26 @@ def test_tc_scale_sign_and_zero(scale, d):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert_parity(out, ref, "tc d=%d scale=%g" % (d, scale))
+
+
+@pytest.mark.parametrize("P", [8, 256])
+@pytest.mark.parametrize("d", [128, 64])
+def test_tc_small_and_large_pages(d, P):
+    """Pages of 8 tokens (8 or 16 boxes per tile) and of 256 (a tile inside a
+    page, at its row offset) on the tcgen05 kernel, lengths around page and
+    tile edges, fixed splits and the library's choice."""
+    nq, r, G = 4, 8, 2
+    lens = [nq, 8, 9, 255, 256, 257, 900]
+    w = Workload(name="tcP", b=len(lens), H=r * G, G=G, d=d, m=1024, page_size=P, len_lo=1, len_hi=1024,
+                 seed=d + P)
+    inp, q = drafts(w, nq, lens, seed=11)
+    ref, ref_lse, st_ref = oracle_verify(inp, q)
+    assert st_ref == 0
+    for split in (0, 256):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out, lse = gqa.gqa_decode_verify(q, inp.k_cache, inp.v_cache, inp.seqlens, inp.page_table,
+                                         split_tokens=split, want_lse=True, status=st, flags=TC)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert_parity(out, ref, "tc d=%d P=%d split=%d" % (d, P, split))
+        assert_lse(lse, ref_lse, "tc d=%d P=%d" % (d, P))
