@@ -524,9 +524,11 @@ int run_items(const Shape &sh, const void *q, const void *k, const void *v, cons
   if (items > (1ll << 31) - 1) return GQA_ERR_DIMS;
   // Programmatic dependent launch pays off when the grid follows a short or
   // partly idle kernel (a combine, a previous step's merge); with one item per
-  // unit the grid follows a full decode grid, where measured it cost ~3 %
-  // (its early blocks only wait, and the grid no longer starts as one wave).
-  Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream, num_splits > 1 || ex.force_pdl};
+  // unit the mma.sync grid follows a full decode grid, where measured it cost
+  // ~1-3 % (its early blocks only wait, and the grid no longer starts as one
+  // wave); the tcgen05 grid of one item per unit gains ~1 % from it (its
+  // blocks set up tensor memory and prefetch while the previous grid ends).
+  Launch l{dim3(static_cast<unsigned>(items), 1, 1), 1, stream, num_splits > 1 || ex.force_pdl || sh.tc};
   if (l.pdl) p.prefetch_tiles = prefetch_tiles(sh, items, split_tokens);
   if (sh.tc) return launch_verify_tc(sh, tk, tv, p, l);
   return launch_decode<Mode::kItems>(sh, tk, tv, p, l);

@@ -293,8 +293,9 @@ __device__ __forceinline__ Piece make_item(const DecodeParams &p) {
 // dependent launch lets the block start while that kernel still runs): bring
 // the first p.prefetch_tiles tiles of the block's piece into L2, so that the
 // HBM reads of this step overlap the tail of the previous one (its last
-// blocks' merges).  The length and page ids read here may still be written by
-// that kernel, so they are only a hint: they pick the addresses to prefetch
+// blocks' merges).  The length and page ids read here (relaxed loads) may
+// still be written by that kernel, so they are only a hint: they pick the
+// addresses to prefetch
 // (page ids outside the pool are skipped, coordinates outside the cache are
 // skipped by the tensor map) and nothing else; the piece itself is computed
 // from the values read after the wait.  One slice per unit prefetches (the
@@ -319,7 +320,7 @@ __device__ __forceinline__ void prefetch_piece_l2(const CUtensorMap *tm_k, const
     s = blockIdx.z;
   }
   if (j != 0 || p.mapped) return;
-  const int len = *reinterpret_cast<const volatile int32_t *>(p.seqlens + s);
+  const int len = ld_relaxed_gpu(p.seqlens + s);
   if (len < p.nq || len > p.capacity) return;
   int t_begin, t_end;
   if (MODE == Mode::kItems) {
@@ -346,7 +347,7 @@ __device__ __forceinline__ void prefetch_piece_l2(const CUtensorMap *tm_k, const
     const int br = min(P, T);
     const int32_t *pt_row = p.page_table + static_cast<size_t>(s) * p.max_pages;
     for (int tb = t_begin + lane * br; tb < t_end; tb += 32 * br) {
-      const int id = *reinterpret_cast<const volatile int32_t *>(pt_row + tb / P);
+      const int id = ld_relaxed_gpu(pt_row + tb / P);
       if (id < 0 || id >= p.num_pages) continue;
 #pragma unroll
       for (int h = 0; h < kHalves; ++h) {

@@ -97,6 +97,14 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c
                : "memory");
 }
 
+// A relaxed load at GPU scope: a value another kernel may be writing at the
+// same time (no data race; the caller treats it as a hint).
+__device__ __forceinline__ int32_t ld_relaxed_gpu(const int32_t *p) {
+  int32_t v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Streaming data is read once: mark it evict-first in L2.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t policy;
