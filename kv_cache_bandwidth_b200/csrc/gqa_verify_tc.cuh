@@ -54,6 +54,74 @@
 
 namespace gqa {
 
+// Packed fp32 arithmetic (sm_100) for the softmax threads: two fp32 values in
+// one 64-bit register pair, operated on by one instruction; each lane is
+// rounded exactly as the scalar instruction rounds it.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f32x2_get(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// max(a, b, c) in one instruction (a NaN operand is ignored, as by fmaxf)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Maximum of N values (N even, >= 4): two independent chains of three-input
+// maxima over the halves, joined at the end.
+template <int N>
+__device__ __forceinline__ float max_of(const float *x) {
+  static_assert(N >= 4 && N % 2 == 0, "two chains of at least two values");
+  constexpr int H = N / 2;
+  float a = fmaxf(x[0], x[1]), b = fmaxf(x[H], x[H + 1]);
+#pragma unroll
+  for (int k = 2; k + 1 < H; k += 2) {
+    a = fmax3(a, x[k], x[k + 1]);
+    b = fmax3(b, x[H + k], x[H + k + 1]);
+  }
+  if (H % 2) {
+    a = fmaxf(a, x[H - 1]);
+    b = fmaxf(b, x[N - 1]);
+  }
+  return fmaxf(a, b);
+}
+
+// split_bf16x2_rz with the two residuals taken by one packed subtraction
+// (the same bits: each residual is exact in fp32).
+__device__ __forceinline__ void split_bf16x2_rz_x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+  hi = __byte_perm(ua, ub, 0x7632);
+  float ra, rb;
+  f32x2_get(sub_f32x2(f32x2(a, b), f32x2(__uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u))),
+            ra, rb);
+  lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
+}
+
 // Shared-memory layout of the tcgen05 kernels: a STAGES-deep ring of K/V tiles
 // of 64 tokens (32 KB per stage) and QBUFS buffers of Q (QROWS rows x d = 128).
 // QROWS = 128: the Q K^T product has M = 128, row i in tensor-memory lane i.
@@ -372,16 +440,7 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
 #pragma unroll
       for (int j = 0; j < TPT; ++j) x[j] = (tb + j < lim) ? __uint_as_float(sv[j]) : kNegInf;
     }
-    float mx;
-    {
-      float m4[TPT / 4];
-#pragma unroll
-      for (int k = 0; k < TPT / 4; ++k)
-        m4[k] = fmaxf(fmaxf(x[4 * k], x[4 * k + 1]), fmaxf(x[4 * k + 2], x[4 * k + 3]));
-      mx = m4[0];
-#pragma unroll
-      for (int k = 1; k < TPT / 4; ++k) mx = fmaxf(mx, m4[k]);
-    }
+    float mx = max_of<TPT>(x);
     mx = (mx == kNegInf) ? kNegInf : mx * sl;              // the scaled maximum
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the row's other TPT tokens of this half
     if (warp_active) {
@@ -418,15 +477,24 @@ __device__ __forceinline__ bool tc_softmax_spread(const DecodeParams &p, const P
 #pragma unroll
         for (int j = 0; j < TPT; ++j) x[j] = (x[j] == kNegInf) ? kNegInf : fmaf(x[j], sl, nb);
       } else {
+        // score * |scale| log2(e) - base, two scores per instruction
+        const uint64_t sl2 = f32x2(sl, sl), nb2 = f32x2(nb, nb);
 #pragma unroll
-        for (int j = 0; j < TPT; ++j) x[j] = fmaf(x[j], sl, nb);
+        for (int e = 0; e < TPT / 2; ++e)
+          f32x2_get(fma_f32x2(f32x2(x[2 * e], x[2 * e + 1]), sl2, nb2), x[2 * e], x[2 * e + 1]);
       }
       uint32_t hi[TPT / 2], lo[TPT / 2];
+      uint64_t ls2 = f32x2(0.f, 0.f);  // the tile's sum, even and odd columns apart
 #pragma unroll
       for (int e = 0; e < TPT / 2; ++e) {
         const float p0 = ex2(x[2 * e]), p1 = ex2(x[2 * e + 1]);
-        l_run += p0 + p1;
-        split_bf16x2_rz(p0, p1, hi[e], lo[e]);
+        ls2 = add_f32x2(ls2, f32x2(p0, p1));
+        split_bf16x2_rz_x2(p0, p1, hi[e], lo[e]);
+      }
+      {
+        float la, lb;
+        f32x2_get(ls2, la, lb);
+        l_run += la + lb;
       }
       tc_st16x2_cols<TPT / 2, TPT>(lane_tmem + b * T + half * HT, hi);
       tc_st16x2_cols<TPT / 2, TPT>(lane_tmem + b * T + half * HT + TPT / 2, lo);
@@ -601,11 +669,17 @@ __device__ __forceinline__ bool tc_softmax_wide(const DecodeParams &p, const Pie
       // longer needed, and the MMAs of tile t-SP that read it are done, since
       // the scores of tile t came after them)
       uint32_t hi[16], lo[16];
+      uint64_t ls2 = f32x2(0.f, 0.f);  // the tile's sum, even and odd columns apart
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const float p0 = ex2(x[2 * e] - base), p1 = ex2(x[2 * e + 1] - base);
-        l_run += p0 + p1;
-        split_bf16x2_rz(p0, p1, hi[e], lo[e]);
+        ls2 = add_f32x2(ls2, f32x2(p0, p1));
+        split_bf16x2_rz_x2(p0, p1, hi[e], lo[e]);
+      }
+      {
+        float la, lb;
+        f32x2_get(ls2, la, lb);
+        l_run += la + lb;
       }
       tc_st16(lane_tmem + b * 64 + half * 32, hi);
       tc_st16(lane_tmem + b * 64 + half * 32 + 16, lo);
