@@ -159,9 +159,10 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
  *               Contiguous dims (max_pages_per_seq == 0) get fixed splits:
  *               one per unit when the units fill at least three quarters of
  *               the GPU's resident blocks (no combine); with too few units
- *               for that, gqa_decode_split (one query token, no lse) runs
+ *               for that, gqa_decode_split (and its lse, verification and
+ *               group-map forms, on the mma.sync contraction) runs
  *               thread-block clusters when they fill the GPU (see
- *               gqa_plan_decomposition); otherwise as many splits
+ *               gqa_plan_decomposition_ex); otherwise as many splits
  *               per unit as still fit one wave of resident blocks.
  * max_seqlen:   an upper bound of every seqlens[s] (sizes the grid and the
  *               workspace); a length above it is treated as invalid
@@ -290,8 +291,9 @@ int gqa_decode_verify(const void *q, const void *k_cache, const void *v_cache,
  * group_of_head: HOST memory, num_heads int32 entries in [0, num_kv_heads)
  * (else GQA_ERR_HEADS); num_heads <= 256, num_kv_heads <= 256.  The map is
  * read during the call only.  lse: fp32 [b, H] or NULL, as in
- * gqa_decode_split_lse.  Runs on fixed splits (split_tokens = 0: the library
- * picks them, for paged caches too); the workspace comes from
+ * gqa_decode_split_lse.  split_tokens = 0: the library picks the
+ * decomposition as for gqa_decode_split (gqa_plan_decomposition_ex with the
+ * same map tells which); the workspace comes from
  * gqa_decode_split_mapped_workspace_size with the same arguments.  The
  * CUDA-core contraction flag is not available with a map.  A map
  * g(i) = i / (H/G) gives exactly gqa_decode_split's result.
@@ -330,9 +332,9 @@ int gqa_merge_lse(const float *o_parts, const float *lse_parts, int32_t n_parts,
 int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms);
 
 /*
- * The decomposition gqa_decode_split runs with split_tokens == 0 for one
- * query token per sequence (gqa_decode_split_lse, gqa_decode_verify and
- * gqa_decode_split_mapped never take the cluster one):
+ * The decomposition gqa_decode_split (and gqa_decode_split_lse) runs with
+ * split_tokens == 0, one query token per sequence and no group table
+ * (gqa_plan_decomposition_ex: with them):
  *   GQA_PLAN_EQUAL_WORK    equal-work ranges + combine kernel (paged dims);
  *   GQA_PLAN_FIXED_SPLITS  fixed splits of *split_tokens_out tokens, merged in
  *                          the decode kernel (<= 8 splits) or by the combine;
@@ -356,6 +358,19 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
 #define GQA_PLAN_CLUSTERS 2
 int32_t gqa_plan_decomposition(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms,
                                int32_t *split_tokens_out, int32_t *cluster_out);
+
+/*
+ * gqa_plan_decomposition for a call with num_query_tokens query tokens per
+ * sequence (gqa_decode_verify; >= 1, else GQA_ERR_DIMS) and, with one query
+ * token, an optional HOST group table (gqa_decode_split_mapped, NULL for the
+ * uniform grouping; checked as there).  Clusters are planned for the mma.sync
+ * contraction only: with more than GQA_TC_AUTO_ROWS rows per group (or the
+ * tcgen05 or CUDA-core flag in dims->flags) the plan is fixed splits or
+ * equal-work ranges.  The same results and errors otherwise.
+ */
+int32_t gqa_plan_decomposition_ex(const gqa_dims *dims, int32_t max_seqlen, int32_t num_query_tokens,
+                                  const int32_t *group_of_head, int32_t num_sms, int32_t *split_tokens_out,
+                                  int32_t *cluster_out);
 
 /*
  * gqa_decode_split_static -- gqa_decode_split without a caller-provided

@@ -688,16 +688,17 @@ AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
   return {false, round_split((max_seqlen + splits - 1) / splits)};
 }
 
-// split_tokens == 0 in gqa_decode_split: a contiguous cache whose (sequence,
-// group) units are too few to fill the GPU one block each runs the cluster
-// decomposition of gqa_decode instead of fixed splits when that fills at least
-// three quarters of the resident blocks with portable clusters (<= 8 blocks):
-// one kernel, the splits of a unit merged through distributed shared memory,
-// no workspace.  Only for one query token without lse output or group table
-// (the cluster kernel writes final rows only), and not for the tcgen05 kernel.
+// split_tokens == 0 in gqa_decode_split (and its verification, lse and group
+// map forms): a contiguous cache whose (sequence, group) units are too few to
+// fill the GPU one block each runs the cluster decomposition of gqa_decode
+// instead of fixed splits when that fills at least three quarters of the
+// resident blocks with portable clusters (<= 8 blocks): one kernel, the splits
+// of a unit merged through distributed shared memory, no workspace.  The
+// cluster kernel writes final rows (and their lse) only, so the partial-state
+// entry points keep fixed splits; the tcgen05 and CUDA-core paths do too.
 // Returns the blocks per cluster, or 0 for the fixed-split / equal-work plan.
-int auto_cluster(const Shape &sh, bool paged, bool lse, int sms) {
-  if (paged || lse || sh.mapped || sh.tc || sh.fma || sh.nq != 1) return 0;
+int auto_cluster(const Shape &sh, bool paged, int sms) {
+  if (paged || sh.tc || sh.fma) return 0;
   const int c = cluster_plan(sh, sms);
   if (c < 2 || c > 8) return 0;
   const long long blocks = units_of(sh) * c;
@@ -813,12 +814,19 @@ int run_combine(const SplitArgs &a, const int32_t *seqlens, float *out, uint32_t
 // The cluster decomposition (gqa_decode, and gqa_decode_split's choice for
 // contiguous caches with few units): grid (c, G x slices, b), clusters of c.
 int run_cluster(const Shape &sh, int c, const void *q, const void *k, const void *v, const int32_t *seqlens,
-                const int32_t *pt, float *out, float scale, uint32_t *status, cudaStream_t st) {
+                const int32_t *pt, float *out, float scale, uint32_t *status, cudaStream_t st,
+                const RowExtras &ex = RowExtras()) {
   CUtensorMap tk, tv;
   int rc = encode_maps(sh, k, v, &tk, &tv);
   if (rc != GQA_OK) return rc;
   DecodeParams p = base_params(sh, q, seqlens, pt, status, scale);
   p.out = out;
+  p.lse = ex.lse;
+  p.empty_ok = ex.empty_ok ? 1 : 0;
+  if (ex.group_of_head) {
+    p.mapped = 1;
+    fill_group_map(ex.group_of_head, sh.H, sh.G, sh.rc, &p.map);
+  }
   // launched as a programmatic dependent: the blocks set themselves up while
   // the previous kernel on the stream finishes
   Launch l{dim3(c, sh.G * sh.hs, sh.b), c, st, true};
@@ -847,9 +855,9 @@ int decode_split_impl(const void *q, const void *k_cache, const void *v_cache, c
       return rc;
     DeviceInfo dev;
     if ((rc = current_device_info(&dev)) != GQA_OK) return rc;
-    const int c = auto_cluster(sh, dims_paged(dims), ex.lse != nullptr, std::min(dev.sms, 256));
-    if (c > 0 && cluster_fits(sh, c)) return run_cluster(sh, c, q, k_cache, v_cache, seqlens, page_table, out, scale, status, st);
-    // (a group map runs on fixed splits only: the library picks them as for a contiguous cache)
+    const int c = auto_cluster(sh, dims_paged(dims), std::min(dev.sms, 256));
+    if (c > 0 && cluster_fits(sh, c))
+      return run_cluster(sh, c, q, k_cache, v_cache, seqlens, page_table, out, scale, status, st, ex);
     const AutoChoice ch = choose_auto(sh, balanced_ok(dims, sh), max_seqlen, std::min(dev.sms, 256));
     if (ch.balanced) {
       rc = run_balanced_decode(sh, dev.sms, q, k_cache, v_cache, seqlens, page_table, out, scale, status,
@@ -962,9 +970,16 @@ int32_t gqa_plan_split_tokens(const gqa_dims *dims, int32_t max_seqlen, int32_t 
 
 int32_t gqa_plan_decomposition(const gqa_dims *dims, int32_t max_seqlen, int32_t num_sms,
                                int32_t *split_tokens_out, int32_t *cluster_out) {
+  return gqa_plan_decomposition_ex(dims, max_seqlen, 1, nullptr, num_sms, split_tokens_out, cluster_out);
+}
+
+int32_t gqa_plan_decomposition_ex(const gqa_dims *dims, int32_t max_seqlen, int32_t num_query_tokens,
+                                  const int32_t *group_of_head, int32_t num_sms, int32_t *split_tokens_out,
+                                  int32_t *cluster_out) {
   Shape sh;
   if (!dims) return GQA_ERR_NULL_POINTER;
-  int rc = check_dims(dims, dims_paged(dims), &sh);
+  if (num_query_tokens < 1) return GQA_ERR_DIMS;
+  int rc = check_dims(dims, dims_paged(dims), &sh, num_query_tokens, group_of_head);
   if (rc != GQA_OK) return rc;
   if (max_seqlen < 1) return GQA_ERR_DIMS;
   const bool on_device = num_sms <= 0;  // plan for the current device (its cluster occupancy included)
@@ -976,7 +991,7 @@ int32_t gqa_plan_decomposition(const gqa_dims *dims, int32_t max_seqlen, int32_t
   num_sms = std::min(num_sms, 256);
   if (split_tokens_out) *split_tokens_out = 0;
   if (cluster_out) *cluster_out = 1;
-  const int c = auto_cluster(sh, dims_paged(dims), false, num_sms);
+  const int c = auto_cluster(sh, dims_paged(dims), num_sms);
   if (c > 0 && (!on_device || cluster_fits(sh, c))) {
     if (cluster_out) *cluster_out = c;
     return GQA_PLAN_CLUSTERS;

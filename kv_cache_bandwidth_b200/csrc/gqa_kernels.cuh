@@ -1062,6 +1062,10 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
     }
   }
   if (MODE != Mode::kItems && threadIdx.x == 0) pdl_launch_dependents();
+  // cluster mode, a slice past the rows of a small group (group map): every
+  // block of the cluster has the same (group, slice), so all of them leave
+  // here, before the cluster's barriers
+  if (MODE == Mode::kCluster && pc.nh <= 0) return;
   // a unit with several splits: claim its arrival word for this call
   if (MODE == Mode::kItems && threadIdx.x == 0 && p.unit_ctr != nullptr &&
       (pc.len + p.split_tokens - 1) / p.split_tokens > 1)
@@ -1679,8 +1683,12 @@ __global__ void __launch_bounds__(Tile<D, NT, NHB, CH, STAGES, MODE == Mode::kBa
       if (L > 0.f) res = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
       const size_t row = row_of(p, pc.s, pc.g, pc.h0 + r_lo + hr);
       reinterpret_cast<float4 *>(p.out + row * D)[c4] = res;
+      if (c4 == 0 && p.lse) p.lse[row] = bad ? kNegInf : lse_from_state(M, L);
     }
-    if (rank == 0 && threadIdx.x == 0 && !pc.len_ok && p.status) atomicOr(p.status, kStatusBadSeqlen);
+    // (a length of 0 where empty sequences are allowed: zero rows, lse -inf,
+    // no status bit)
+    if (rank == 0 && threadIdx.x == 0 && !pc.len_ok && p.status && !(p.empty_ok && pc.len == 0))
+      atomicOr(p.status, kStatusBadSeqlen);
   }
 }
 

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "GqaError", "Dims", "load", "lib_path", "gqa_decode", "gqa_decode_split",
     "gqa_split_partials", "gqa_split_combine", "gqa_decode_split_workspace_size",
-    "gqa_plan_split_tokens", "gqa_plan_decomposition", "PLAN_EQUAL_WORK", "PLAN_FIXED_SPLITS", "PLAN_CLUSTERS",
+    "gqa_plan_split_tokens", "gqa_plan_decomposition", "gqa_plan_decomposition_ex", "PLAN_EQUAL_WORK", "PLAN_FIXED_SPLITS", "PLAN_CLUSTERS",
     "gqa_status_string", "gqa_abi_version", "dims_for",
     "STATUS_BAD_SEQLEN", "STATUS_BAD_PAGE", "STATUS_TIMEOUT", "FLAG_CONTRACT_MMA",
     "FLAG_CONTRACT_FMA", "FLAG_CONTRACT_TCGEN05", "ERRORS", "gqa_decode_split_static", "STATIC_WORKSPACE_BYTES",
@@ -99,6 +99,10 @@ def load():
     lib.gqa_plan_decomposition.restype = ctypes.c_int32
     lib.gqa_plan_decomposition.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32,
                                            ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
+    lib.gqa_plan_decomposition_ex.restype = ctypes.c_int32
+    lib.gqa_plan_decomposition_ex.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32, _vp,
+                                              ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
+                                              ctypes.POINTER(ctypes.c_int32)]
     lib.gqa_decode_split_static.restype = ctypes.c_int
     lib.gqa_decode_split_static.argtypes = _DECODE_ARGS + [ctypes.c_int32, ctypes.c_int32, _vp]
     lib.gqa_decode_split_lse.restype = ctypes.c_int
@@ -220,6 +224,20 @@ def gqa_plan_decomposition(dims: Dims, max_seqlen: int, num_sms: int = 0):
                                            ctypes.byref(split), ctypes.byref(cluster)))
     if rc < 0:
         raise GqaError(rc, "gqa_plan_decomposition")
+    return rc, int(split.value), int(cluster.value)
+
+
+def gqa_plan_decomposition_ex(dims: Dims, max_seqlen: int, num_query_tokens: int = 1, group_of_head=None,
+                              num_sms: int = 0):
+    """gqa_plan_decomposition for num_query_tokens query tokens per sequence
+    (gqa_decode_verify) and an optional host group table (gqa_decode_split_mapped)."""
+    split, cluster = ctypes.c_int32(0), ctypes.c_int32(0)
+    gmap = None if group_of_head is None else _host_map(group_of_head)
+    rc = int(load().gqa_plan_decomposition_ex(ctypes.byref(dims), int(max_seqlen), int(num_query_tokens),
+                                              gmap, int(num_sms),
+                                              ctypes.byref(split), ctypes.byref(cluster)))
+    if rc < 0:
+        raise GqaError(rc, "gqa_plan_decomposition_ex")
     return rc, int(split.value), int(cluster.value)
 
 

@@ -30,7 +30,8 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("gqa_decode", "gqa_decode_split", "gqa_decode_split_workspace_size", "gqa_split_partials",
-              "gqa_split_combine", "gqa_plan_split_tokens", "gqa_plan_decomposition", "gqa_status_string",
+              "gqa_split_combine", "gqa_plan_split_tokens", "gqa_plan_decomposition", "gqa_plan_decomposition_ex",
+              "gqa_status_string",
               "gqa_abi_version",
               "gqa_decode_split_lse", "gqa_merge_lse", "gqa_decode_split_static", "gqa_kv_append",
               "gqa_page_pool_create", "gqa_page_pool_alloc", "gqa_page_pool_free", "gqa_page_pool_available",
@@ -325,3 +326,39 @@ def test_plan_decomposition(lib):
     assert gqa.gqa_plan_split_tokens(_dims(num_kv_heads=2, **sweep), 8192, 148) == 1024
     assert lib.gqa_plan_decomposition(None, 10, 148, None, None) == -1
     assert lib.gqa_plan_decomposition(ctypes.byref(_dims(num_heads=9)), 10, 148, None, None) == -3
+
+
+def test_plan_decomposition_ex(lib):
+    """The plan of a verification call (several query tokens) or of a group
+    table: clusters on the mma.sync contraction (up to 16 rows per group),
+    fixed splits once the rows go to the tcgen05 kernel; the one-token,
+    no-table plan is gqa_plan_decomposition's."""
+    sweep = dict(batch=16, num_heads=32, head_dim=128, page_size=8192)
+
+    def plan(nq=1, gmap=None, **kw):
+        return gqa.gqa_plan_decomposition_ex(_dims(**kw), kw["page_size"], nq, gmap, 148)
+    for G in (1, 2, 4, 8, 32):
+        assert plan(num_kv_heads=G, **sweep) == gqa.gqa_plan_decomposition(_dims(num_kv_heads=G, **sweep), 8192, 148)
+    # r = 4: 2 and 4 query tokens keep 8 and 16 rows per group on mma.sync, 128 units in clusters of 2
+    assert plan(2, num_kv_heads=8, **sweep) == (gqa.PLAN_CLUSTERS, 0, 2)
+    assert plan(4, num_kv_heads=8, **sweep) == (gqa.PLAN_CLUSTERS, 0, 2)
+    # 8 query tokens: 32 rows, the tcgen05 kernel, one split per unit (128 units, one block per SM)
+    assert plan(8, num_kv_heads=8, **sweep) == (gqa.PLAN_FIXED_SPLITS, 8192, 1)
+    # r = 16, 2 tokens: 32 rows on tcgen05, 32 units: four splits each
+    assert plan(2, num_kv_heads=2, **sweep) == (gqa.PLAN_FIXED_SPLITS, 2048, 1)
+    # a table over 4 groups, the largest of 12 heads (one slice), one group empty: 64 units, clusters of 4
+    gmap = [0] * 12 + [1] * 10 + [2] * 10
+    assert plan(1, gmap, num_kv_heads=4, **sweep) == (gqa.PLAN_CLUSTERS, 0, 4)
+    # a group of 20 heads: the tcgen05 kernel by itself (64 units, two splits each); on mma.sync two
+    # 16-row slices per group, 128 units, clusters of 2
+    gmap = [0] * 20 + [1] * 6 + [2] * 6
+    assert plan(1, gmap, num_kv_heads=4, **sweep) == (gqa.PLAN_FIXED_SPLITS, 4096, 1)
+    assert plan(1, gmap, num_kv_heads=4, flags=gqa.FLAG_CONTRACT_MMA, **sweep) == (gqa.PLAN_CLUSTERS, 0, 2)
+    # errors: no query token; a table with several query tokens; a group outside [0, G)
+    d = _dims(num_kv_heads=4, **sweep)
+    assert lib.gqa_plan_decomposition_ex(ctypes.byref(d), 8192, 0, None, 148, None, None) == -6
+    tab = (ctypes.c_int32 * 32)(*([0] * 32))
+    assert lib.gqa_plan_decomposition_ex(ctypes.byref(d), 8192, 2, tab, 148, None, None) == -3
+    tab[5] = 4
+    assert lib.gqa_plan_decomposition_ex(ctypes.byref(d), 8192, 1, tab, 148, None, None) == -3
+    assert lib.gqa_plan_decomposition_ex(None, 8192, 1, None, 148, None, None) == -1

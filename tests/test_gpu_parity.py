@@ -501,7 +501,7 @@ def test_split_entry_runs_clusters_for_few_units():
     with split_tokens = 0 runs thread-block clusters (merged through
     distributed shared memory) and agrees with the oracle, lengths from 1 to
     the capacity mixed; an invalid length sets its status bit and zeroes its
-    rows; the lse entry point keeps to fixed splits and agrees too."""
+    rows; the lse entry point runs the same clusters and agrees too."""
     w = Workload(name="few units", b=16, H=8, G=2, d=64, m=2048, seed=41)
     lens = [2048, 1, 5, 129, 2047, 300, 1024, 77, 2048, 640, 1500, 64, 65, 999, 2000, 3]
     inp = make_inputs(w, device="cuda", lens=lens)
