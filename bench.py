@@ -392,8 +392,8 @@ class Case:
         self.tc = gqa.TC_AUTO_ROWS < nq * w.r <= (128 if w.d == 128 else 64)
         if split > 0:
             self.eff_split = split
-        elif nq == 1 and self.entry == "split":
-            kind, self.eff_split, c = gqa.gqa_plan_decomposition(self.dims, self.max_seqlen)
+        elif self.entry == "split":
+            kind, self.eff_split, c = gqa.gqa_plan_decomposition_ex(self.dims, self.max_seqlen, nq)
             self.cluster = c if kind == gqa.PLAN_CLUSTERS else 0
         else:
             self.eff_split = gqa.gqa_plan_split_tokens(self.dims, self.max_seqlen)
