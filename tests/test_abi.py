@@ -357,6 +357,7 @@ def test_plan_decomposition_ex(lib):
     # errors: no query token; a table with several query tokens; a group outside [0, G)
     d = _dims(num_kv_heads=4, **sweep)
     assert lib.gqa_plan_decomposition_ex(ctypes.byref(d), 8192, 0, None, 148, None, None) == -6
+    assert lib.gqa_plan_decomposition_ex(ctypes.byref(d), 8192, 65, None, 148, None, None) == -6  # as the verify call
     tab = (ctypes.c_int32 * 32)(*([0] * 32))
     assert lib.gqa_plan_decomposition_ex(ctypes.byref(d), 8192, 2, tab, 148, None, None) == -3
     tab[5] = 4
