@@ -353,7 +353,16 @@ int launch_decode_d(const Shape &sh, const CUtensorMap &tk, const CUtensorMap &t
   if (sh.fma)
     return sh.r == 1 ? launch_decode_t<D, 1, 1, 3, PAGED, MODE, 1>(tk, tv, p, l)
                      : launch_decode_t<D, 1, 1, 3, PAGED, MODE, 2>(tk, tv, p, l);
-  if (sh.nhb == 2) return launch_decode_t<D, 1, 2, 3, PAGED, MODE>(tk, tv, p, l);
+  if (sh.nhb == 2) {
+    // 16 rows: two 288-thread blocks per SM get 96 registers a thread, too few
+    // for the equal-work walker at d = 128 (it spilled 180-208 bytes), so
+    // there equal-work ranges run one block per SM with a six-stage ring
+    // (measured 7-8 % faster on paged 16-row batches).  At d = 64 the
+    // two-block form, which spills only 12-20 bytes, stays: it measured 12 %
+    // faster there.
+    if constexpr (MODE == Mode::kBalanced && D == 128) return launch_decode_t<D, 1, 2, 6, PAGED, MODE>(tk, tv, p, l);
+    else return launch_decode_t<D, 1, 2, 3, PAGED, MODE>(tk, tv, p, l);
+  }
   switch (pick_pipe(sh)) {
     case Pipe::kTrio: return launch_decode_t<D, 1, 1, 2, PAGED, MODE>(tk, tv, p, l);
     case Pipe::kSolo: return launch_decode_t<D, 1, 1, 6, PAGED, MODE>(tk, tv, p, l);
