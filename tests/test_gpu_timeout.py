@@ -70,6 +70,13 @@ CASES = [
      Workload(name="t6", b=4, H=16, G=2, d=128, m=4096, seed=36), 4, 0, TC, (0, 1)),
     ("tcgen05 kernel, d = 64 (128-token tiles)",
      Workload(name="t7", b=2, H=16, G=2, d=64, m=2048, seed=37), 8, 512, TC, (1, 2)),
+    # every cluster's rank 0 leaves out its second tile; the block still reaches
+    # the cluster's barriers, so its cluster ends and reports
+    ("thread-block clusters, merged in distributed shared memory",
+     Workload(name="t8", b=16, H=8, G=2, d=64, m=2048, seed=38), 1, 0, 0, (0, 1)),
+    ("equal-work ranges, paged, 16 rows (one block per SM)",
+     Workload(name="t9", b=8, H=32, G=2, d=128, m=8192, page_size=16, len_lo=4000, len_hi=8192, seed=39),
+     1, 0, 0, (0, 3)),
 ]
 
 
