@@ -163,7 +163,8 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
  *               group-map forms, on the mma.sync contraction) runs
  *               thread-block clusters when they fill the GPU (see
  *               gqa_plan_decomposition_ex); otherwise as many splits
- *               per unit as still fit one wave of resident blocks.
+ *               per unit as still fit one wave of resident blocks.  With
+ *               max_seqlen <= 256 no unit is split (one split of 256).
  * max_seqlen:   an upper bound of every seqlens[s] (sizes the grid and the
  *               workspace); a length above it is treated as invalid
  *               (GQA_STATUS_BAD_SEQLEN, row zeroed).

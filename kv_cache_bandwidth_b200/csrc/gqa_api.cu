@@ -684,11 +684,18 @@ int blocks_per_sm(const Shape &sh) {
   }
 }
 
+constexpr int kNoSplitTokens = 256;
+
 AutoChoice choose_auto(const Shape &sh, bool paged, int max_seqlen, int sms) {
   if (paged) {
     if (sh.b <= kMaxBalancedBatch) return {true, 0};
     return {false, kFallbackSplit};
   }
+  // A unit of at most kNoSplitTokens is not split: merging two halves costs
+  // more than the streaming they save (device-timed, graph replays: 256
+  // tokens at d = 128 in one split 6.3-6.7 us against 7.8-8.3 in two, at
+  // d = 64 4.8 against 6.7; from 512 tokens on, splits win).
+  if (max_seqlen <= kNoSplitTokens) return {false, round_split(max_seqlen)};
   // One block per unit when the units fill three quarters of the resident
   // slots; otherwise as many splits as still fit one wave.
   const long long units = units_of(sh);

@@ -322,6 +322,12 @@ def test_plan_decomposition(lib):
     d3 = _dims(batch=64, num_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=70000,
                max_pages_per_seq=2048)
     assert gqa.gqa_plan_decomposition(d3, 32768, 148) == (gqa.PLAN_EQUAL_WORK, 0, 1)
+    # a unit of at most 256 tokens is not split (the merge would cost more than it saves); 512 is
+    assert plan(batch=2, num_heads=8, num_kv_heads=2, head_dim=64, page_size=256) == (gqa.PLAN_FIXED_SPLITS, 256, 1)
+    assert plan(batch=1, num_heads=64, num_kv_heads=8, head_dim=128, page_size=200) == (
+        gqa.PLAN_FIXED_SPLITS, 256, 1)
+    assert plan(batch=1, num_heads=64, num_kv_heads=8, head_dim=128, page_size=512) == (
+        gqa.PLAN_FIXED_SPLITS, 128, 1)
     # the two-kernel plan is unchanged by the cluster choice
     assert gqa.gqa_plan_split_tokens(_dims(num_kv_heads=2, **sweep), 8192, 148) == 1024
     assert lib.gqa_plan_decomposition(None, 10, 148, None, None) == -1
