@@ -88,11 +88,12 @@ def test_fma_contraction_needs_one_token():
     assert e.value.code == -3
 
 
-@pytest.mark.parametrize("nq", [2, 4])
+@pytest.mark.parametrize("nq", [2, 4, 8, 16])
 def test_verify_llama_layer_sampled(nq):
     """The Llama-2-70B layer (b32 H64 G8 d128 m4096) with nq drafts per
-    sequence, in the decomposition the library picks; sampled rows against the
-    oracle."""
+    sequence, in the decomposition the library picks (with 8 and 16 drafts,
+    64 and 128 rows per group: the tcgen05 kernel, as the bench times it);
+    sampled rows against the oracle."""
     w = Workload(name="llama", b=32, H=64, G=8, d=128, m=4096, seed=1235)
     inp, q = drafts(w, nq, [4096] * 32, seed=nq)
     out, lse = run_verify(inp, q, 0)
