@@ -552,6 +552,26 @@ def measure_point(args, name, nq, world, rank, hbm):
     return d
 
 
+def sweep_fit(per_config):
+    """Does the step time of the group-ratio sweep follow its KV bytes?  A
+    least-squares line t = fixed + bytes / bandwidth through the sweep points
+    whose cache exceeds twice the L2 (their time is set by streaming the
+    cache), and every sweep point's time over that line's value (1.0: on the
+    line; above 1: a per-step cost beyond the line's fixed part)."""
+    pts = {k: v for k, v in per_config.items() if k.startswith("sweep_g")}
+    big = [(v["kv_bytes"], v["us_per_step"]) for v in pts.values() if v["kv_bytes"] > 2 * L2_BYTES]
+    if len(big) < 2:
+        return None
+    n = len(big)
+    mx = sum(x for x, _ in big) / n
+    my = sum(y for _, y in big) / n
+    sxx = sum((x - mx) ** 2 for x, _ in big)
+    slope = sum((x - mx) * (y - my) for x, y in big) / sxx  # us per byte
+    fixed = my - slope * mx
+    return {"fixed_us": fixed, "marginal_gbs": 1e-3 / slope, "fit_points": n,
+            "time_over_fit": {k: v["us_per_step"] / (fixed + slope * v["kv_bytes"]) for k, v in pts.items()}}
+
+
 def main_gpu(args):
     world, rank, local = dist_setup()
     hbm, hbm_kind = peaks()
@@ -641,6 +661,7 @@ def main_gpu(args):
             "entry": "gqa_decode_verify" if nq > 1 else "gqa_decode_split" if args.entry == "split" else "gqa_decode",
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk, "per_config": per_config,
+            "sweep_fit": sweep_fit(per_config),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

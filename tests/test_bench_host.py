@@ -74,3 +74,21 @@ def test_l2_plan_keeps_steps_out_of_l2():
     assert bench.l2_plan(256 * 1024) == ("flush", 1)
     assert bench.l2_plan(0) == ("flush", 1)
     assert "flushed" in bench.l2_desc(1000) and "copies" in bench.l2_desc(L2)
+
+
+def test_sweep_fit_recovers_a_line():
+    """Points on t = 5 us + bytes / 7 TB/s give back the line; a small point
+    that takes longer than the line reports its ratio."""
+    per = {}
+    for g, kv in ((1, 67108864), (4, 268435456), (8, 536870912), (32, 2147483648)):
+        per["sweep_g%d" % g] = {"kv_bytes": kv, "us_per_step": 5.0 + kv / 7e6}
+    per["sweep_g1"]["us_per_step"] *= 1.5
+    per["llama70b"] = {"kv_bytes": 536870912, "us_per_step": 1e9}  # not a sweep point
+    fit = bench.sweep_fit(per)
+    assert fit["fit_points"] == 3
+    assert abs(fit["fixed_us"] - 5.0) < 1e-6
+    assert abs(fit["marginal_gbs"] - 7000.0) < 1e-6
+    assert abs(fit["time_over_fit"]["sweep_g1"] - 1.5) < 1e-9
+    assert abs(fit["time_over_fit"]["sweep_g8"] - 1.0) < 1e-9
+    assert "llama70b" not in fit["time_over_fit"]
+    assert bench.sweep_fit({"sweep_g1": per["sweep_g1"]}) is None
