@@ -122,6 +122,35 @@ __device__ __forceinline__ void split_bf16x2_rz_x2(float a, float b, uint32_t &h
   lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
 }
 
+// The waits of the single-thread roles (the TMA producer and the two MMA
+// issuers), which spend most of each tile waiting: mbarrier.try_wait with a
+// suspend-time hint, so that the waiting warp sleeps until the phase completes
+// (or the hint runs out) instead of polling, and leaves the issue slots of its
+// SM sub-partition to the two softmax warps there.  Bounded as mbar_wait is:
+// false once the wait has run past kWaitLimitCycles.
+constexpr uint32_t kRoleSuspendNs = 100000;
+
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(kRoleSuspendNs)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_role(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait_suspend(bar, parity)) return true;
+  const long long start = clock64();
+  while (!mbar_try_wait_suspend(bar, parity)) {
+    if (clock64() - start > kWaitLimitCycles) return false;
+  }
+  return true;
+}
+
 // Shared-memory layout of the tcgen05 kernels: a STAGES-deep ring of K/V tiles
 // of 64 tokens (32 KB per stage) and QBUFS buffers of Q (QROWS rows x d = 128).
 // QROWS = 128: the Q K^T product has M = 128, row i in tensor-memory lane i.
@@ -260,7 +289,7 @@ __device__ __forceinline__ bool tc_produce_piece(const CUtensorMap *tm_k, const 
     const int stage = tile % ST;
     const uint32_t full = bars.full0 + 8 * stage;
     if (tile >= ST) {
-      bool ok = mbar_wait(bars.empty0 + 8 * stage, ((tile / ST) - 1) & 1);
+      bool ok = mbar_wait_role(bars.empty0 + 8 * stage, ((tile / ST) - 1) & 1);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok || *abort_flag) {
         if (lane == 0) {
@@ -770,8 +799,8 @@ __device__ __forceinline__ bool tc_issue_qk(uint32_t sbase, uint32_t qbuf, uint3
   for (int t = 0; t < n_tiles; ++t) {
     const int gt = gt0 + t;
     const int st = gt % ST;
-    bool ok = mbar_wait(bars.full0 + 8 * st, (gt / ST) & 1);
-    if (ok && gt >= SP) ok = mbar_wait(bars.pv_done0 + 8 * (gt % SP), ((gt / SP) - 1) & 1);
+    bool ok = mbar_wait_role(bars.full0 + 8 * st, (gt / ST) & 1);
+    if (ok && gt >= SP) ok = mbar_wait_role(bars.pv_done0 + 8 * (gt % SP), ((gt / SP) - 1) & 1);
     if (!ok) return false;
     tc_fence_after();
     const uint64_t kd = tc_smem_desc(sbase + st * TT::kStageBytes, 16, 1024);
@@ -803,7 +832,7 @@ __device__ __forceinline__ bool tc_issue_pv(uint32_t sbase, uint32_t tmem, const
   for (int u = 0; u < n_tiles; ++u) {
     const int gt = gt0 + u;
     const int st = gt % ST;
-    if (!mbar_wait(bars.p_full0 + 8 * (gt % SP), (gt / SP) & 1)) return false;
+    if (!mbar_wait_role(bars.p_full0 + 8 * (gt % SP), (gt / SP) & 1)) return false;
     tc_fence_after();
     const uint64_t vd = tc_smem_desc(sbase + st * TT::kStageBytes + TT::kTileBytes, TT::kHalf, 1024);
     const uint32_t pb = tmem + (gt % SP) * T;
@@ -952,7 +981,7 @@ __global__ void __launch_bounds__(TcTile::kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ============================================================ Q K^T issuer
     if (lane == 0) {
-      const bool ok = mbar_wait(bars.q_full0, 0) && tc_issue_qk<TT>(sbase, sbase + TT::kQOff, tmem, bars, 0, n_tiles);
+      const bool ok = mbar_wait_role(bars.q_full0, 0) && tc_issue_qk<TT>(sbase, sbase + TT::kQOff, tmem, bars, 0, n_tiles);
       if (!ok) tc_abort(p, abort_flag);
       tc_issuer_drain(bars.drain0, p);
     }
